@@ -1,0 +1,471 @@
+// ds4moe_capi.cu -- the C ABI (include/ds4moe.h): handle, buffer layout,
+// argument checks, loading, and the launch of the decode and prefill plans.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/ds4moe.h"
+#include "ds4moe_internal.cuh"
+
+namespace ds4 {
+__global__ void k_pack_q2k(const float* w, int64_t n_blocks, uint8_t* out);
+__global__ void k_pack_iq2(const float* w, int64_t n_blocks, const uint8_t* grid, uint8_t* out);
+__global__ void k_repack_iq2(const uint8_t* src, int R, int C, uint8_t* qs, uint16_t* dd);
+__global__ void k_repack_q2(const uint8_t* src, int R, int C, uint8_t* q, uint32_t* sc, uint32_t* dd);
+__global__ void k_repack_bf16(const uint4* src, int R, int C, uint4* dst);
+__global__ void k_dequant_iq2(const uint8_t* qs, const uint16_t* dd, const uint8_t* grid, int R, int C, float* out_f,
+                              __nv_bfloat16* out_b);
+__global__ void k_dequant_q2(const uint8_t* q, const uint32_t* sc, const uint32_t* dd, int R, int C, float* out_f,
+                             __nv_bfloat16* out_b);
+__global__ void k_dequant_bf16_tiles(const __nv_bfloat16* t, int R, int C, float* out_f, __nv_bfloat16* out_b);
+cudaError_t launch_decode(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n, float* out,
+                          int n_sm, cudaStream_t st, cudaEvent_t const* ev);
+int decode_launches();
+const char* decode_kernel_name(int i);
+cudaError_t launch_route(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n,
+                         cudaStream_t st);
+}  // namespace ds4
+
+using namespace ds4;
+
+namespace {
+
+thread_local std::string g_err;
+
+ds4moe_status fail(ds4moe_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+ds4moe_status fail(ds4moe_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return s;
+}
+
+ds4moe_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(DS4MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+struct WsLayout {
+    size_t hdr, logits, ids, wts, h_rt, hsum_rt, h_sh, y_rt, y_sh, x_stage, out_stage, total;
+};
+
+}  // namespace
+
+struct ds4moe {
+    ds4moe_shape shape;
+    Dims D;
+    int decode_max;
+    int n_sm;
+    // weight buffer layout
+    size_t off_grid, off_Wr, off_br, off_gate_qs, off_gate_d, off_up_qs, off_up_d, off_down_q, off_down_sc,
+        off_down_dd, off_sh_gate, off_sh_up, off_sh_down, weight_bytes;
+    size_t iq2_qs_stride, iq2_d_stride, q2_q_stride, q2_sc_stride, q2_dd_stride;
+    uint8_t* weights = nullptr;
+    uint8_t* ws = nullptr;
+    size_t ws_bytes = 0;
+    WsLayout L{};
+    std::vector<uint8_t> loaded;
+    bool grid_set = false, router_set = false, shared_set = false;
+
+    WsLayout layout(int cap) const {
+        WsLayout w{};
+        const size_t H = D.H, I = D.I, E = D.E, k = D.k;
+        const size_t nd = (size_t)(cap < decode_max ? cap : decode_max);
+        size_t o = 0;
+        w.hdr = o; o += 256;
+        w.logits = o; o += align256(nd * E * 4);
+        w.ids = o; o += align256(nd * k * 4);
+        w.wts = o; o += align256(nd * k * 4);
+        w.h_rt = o; o += align256(nd * k * I * 4);
+        w.hsum_rt = o; o += align256(nd * k * (I / 16) * 4);
+        w.h_sh = o; o += align256(nd * I * 4);
+        w.y_rt = o; o += align256(nd * k * H * 4);
+        w.y_sh = o; o += align256(nd * H * 4);
+        w.x_stage = o; o += align256((size_t)cap * H * (D.act_bf16 ? 2 : 4));
+        w.out_stage = o; o += align256((size_t)cap * H * 4);
+        w.total = o;
+        return w;
+    }
+
+    Weights weights_view() const {
+        Weights W{};
+        const uint8_t* b = weights;
+        W.grid_u8 = b + off_grid;
+        W.W_r = reinterpret_cast<const float*>(b + off_Wr);
+        W.b_r = shape.has_bias ? reinterpret_cast<const float*>(b + off_br) : nullptr;
+        W.gate_qs = b + off_gate_qs;
+        W.gate_d = reinterpret_cast<const uint16_t*>(b + off_gate_d);
+        W.up_qs = b + off_up_qs;
+        W.up_d = reinterpret_cast<const uint16_t*>(b + off_up_d);
+        W.down_q = b + off_down_q;
+        W.down_sc = reinterpret_cast<const uint32_t*>(b + off_down_sc);
+        W.down_dd = reinterpret_cast<const uint32_t*>(b + off_down_dd);
+        W.sh_gate = reinterpret_cast<const __nv_bfloat16*>(b + off_sh_gate);
+        W.sh_up = reinterpret_cast<const __nv_bfloat16*>(b + off_sh_up);
+        W.sh_down = reinterpret_cast<const __nv_bfloat16*>(b + off_sh_down);
+        W.iq2_qs_stride = iq2_qs_stride;
+        W.iq2_d_stride = iq2_d_stride;
+        W.q2_q_stride = q2_q_stride;
+        W.q2_sc_stride = q2_sc_stride;
+        W.q2_dd_stride = q2_dd_stride;
+        return W;
+    }
+
+    DecodeWs decode_ws() const {
+        DecodeWs w{};
+        uint32_t* hdr = reinterpret_cast<uint32_t*>(ws + L.hdr);
+        w.err = hdr + 0;
+        w.ticket = hdr + 1;
+        w.queue1 = hdr + 2;
+        w.queue2 = hdr + 3;
+        w.logits = reinterpret_cast<float*>(ws + L.logits);
+        w.ids = reinterpret_cast<int32_t*>(ws + L.ids);
+        w.wts = reinterpret_cast<float*>(ws + L.wts);
+        w.h_rt = reinterpret_cast<float*>(ws + L.h_rt);
+        w.hsum_rt = reinterpret_cast<float*>(ws + L.hsum_rt);
+        w.h_sh = reinterpret_cast<float*>(ws + L.h_sh);
+        w.y_rt = reinterpret_cast<float*>(ws + L.y_rt);
+        w.y_sh = reinterpret_cast<float*>(ws + L.y_sh);
+        return w;
+    }
+
+    bool ready(std::string* why) const {
+        if (!weights || !ws) { *why = "buffers not bound"; return false; }
+        if (!grid_set) { *why = "grid not set"; return false; }
+        if (!router_set) { *why = "router not set"; return false; }
+        if (shape.has_shared && !shared_set) { *why = "shared expert not set"; return false; }
+        for (size_t e = 0; e < loaded.size(); ++e)
+            if (!loaded[e]) { *why = "expert " + std::to_string(e) + " not loaded"; return false; }
+        return true;
+    }
+};
+
+extern "C" {
+
+const char* ds4moe_last_error(void) { return g_err.c_str(); }
+
+ds4moe_status ds4moe_create(const ds4moe_shape* s, ds4moe_t** out) {
+    if (!s || !out) return fail(DS4MOE_ERR_ARG, "create: NULL argument");
+    *out = nullptr;
+    if (s->hidden < 256 || s->hidden % 256) return fail(DS4MOE_ERR_SHAPE, "hidden %d: need a multiple of 256", s->hidden);
+    if (!(s->inter == 128 || (s->inter >= 256 && s->inter % 256 == 0)))
+        return fail(DS4MOE_ERR_SHAPE, "inter %d: need 128 or a multiple of 256", s->inter);
+    if (s->n_experts < 1 || s->n_experts > 1024) return fail(DS4MOE_ERR_SHAPE, "n_experts %d: need 1..1024", s->n_experts);
+    if (s->top_k < 1 || s->top_k > 16 || s->top_k > s->n_experts)
+        return fail(DS4MOE_ERR_SHAPE, "top_k %d: need 1..min(16, n_experts)", s->top_k);
+    if (s->max_tokens < 1) return fail(DS4MOE_ERR_SHAPE, "max_tokens %d: need >= 1", s->max_tokens);
+    if (s->act_dtype != DS4MOE_ACT_F32 && s->act_dtype != DS4MOE_ACT_BF16)
+        return fail(DS4MOE_ERR_SHAPE, "act_dtype %d unknown", s->act_dtype);
+    if (s->decode_max < 0 || s->decode_max > 8) return fail(DS4MOE_ERR_SHAPE, "decode_max %d: need 0..8", s->decode_max);
+    int dev = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
+    int n_sm = 0;
+    ce = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    if (ce != cudaSuccess) return cuda_fail(ce, "cudaDeviceGetAttribute");
+
+    ds4moe* h = new ds4moe();
+    h->shape = *s;
+    h->D.H = s->hidden;
+    h->D.I = s->inter;
+    h->D.E = s->n_experts;
+    h->D.k = s->top_k;
+    h->D.has_shared = s->has_shared ? 1 : 0;
+    h->D.act_bf16 = s->act_dtype == DS4MOE_ACT_BF16;
+    h->decode_max = s->decode_max ? s->decode_max : 8;
+    h->n_sm = n_sm;
+    const size_t H = s->hidden, I = s->inter, E = s->n_experts;
+    const size_t nsb_down = I >= 256 ? I / 256 : 1;
+    h->iq2_qs_stride = I * H / 4;
+    h->iq2_d_stride = I * H / 256;
+    h->q2_q_stride = H * I / 4;
+    h->q2_sc_stride = H * I / 64;
+    h->q2_dd_stride = H * nsb_down;
+    size_t o = 0;
+    h->off_grid = o; o += align256(256 * 8);
+    h->off_Wr = o; o += align256(E * H * 4);
+    h->off_br = o; o += align256(E * 4);
+    h->off_gate_qs = o; o += align256(E * h->iq2_qs_stride);
+    h->off_gate_d = o; o += align256(E * h->iq2_d_stride * 2);
+    h->off_up_qs = o; o += align256(E * h->iq2_qs_stride);
+    h->off_up_d = o; o += align256(E * h->iq2_d_stride * 2);
+    h->off_down_q = o; o += align256(E * h->q2_q_stride);
+    h->off_down_sc = o; o += align256(E * h->q2_sc_stride * 4);
+    h->off_down_dd = o; o += align256(E * h->q2_dd_stride * 4);
+    h->off_sh_gate = o; o += align256(s->has_shared ? I * H * 2 : 0);
+    h->off_sh_up = o; o += align256(s->has_shared ? I * H * 2 : 0);
+    h->off_sh_down = o; o += align256(s->has_shared ? H * I * 2 : 0);
+    h->weight_bytes = o;
+    h->loaded.assign(E, 0);
+    *out = h;
+    g_err.clear();
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_destroy(ds4moe_t* h) {
+    if (!h) return fail(DS4MOE_ERR_ARG, "destroy: NULL handle");
+    delete h;
+    return DS4MOE_OK;
+}
+
+size_t ds4moe_weight_bytes(const ds4moe_t* h) { return h ? h->weight_bytes : 0; }
+
+size_t ds4moe_workspace_bytes(const ds4moe_t* h, int32_t n_tokens) {
+    if (!h || n_tokens < 1) return 0;
+    return h->layout(n_tokens).total;
+}
+
+ds4moe_status ds4moe_bind(ds4moe_t* h, void* d_weights, size_t weight_bytes, void* d_workspace, size_t ws_bytes,
+                          void* stream) {
+    if (!h || !d_weights || !d_workspace) return fail(DS4MOE_ERR_ARG, "bind: NULL argument");
+    if (((uintptr_t)d_weights & 255) || ((uintptr_t)d_workspace & 255))
+        return fail(DS4MOE_ERR_ALIGN, "bind: buffers must be 256-byte aligned");
+    if (weight_bytes < h->weight_bytes)
+        return fail(DS4MOE_ERR_ARG, "bind: weight buffer %zu bytes < %zu", weight_bytes, h->weight_bytes);
+    WsLayout L = h->layout(h->shape.max_tokens);
+    if (ws_bytes < L.total) return fail(DS4MOE_ERR_ARG, "bind: workspace %zu bytes < %zu", ws_bytes, L.total);
+    cudaError_t ce = cudaMemsetAsync(static_cast<uint8_t*>(d_workspace) + L.hdr, 0, 256, (cudaStream_t)stream);
+    if (ce != cudaSuccess) return cuda_fail(ce, "bind: cudaMemsetAsync");
+    h->weights = static_cast<uint8_t*>(d_weights);
+    h->ws = static_cast<uint8_t*>(d_workspace);
+    h->ws_bytes = ws_bytes;
+    h->L = L;
+    std::fill(h->loaded.begin(), h->loaded.end(), 0);
+    h->grid_set = h->router_set = h->shared_set = false;
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_pack_q2k(const float* d_w, int64_t n, void* d_blocks, void* stream) {
+    if (!d_w || !d_blocks) return fail(DS4MOE_ERR_ARG, "pack_q2k: NULL argument");
+    if (n <= 0 || n % kQK) return fail(DS4MOE_ERR_ARG, "pack_q2k: n_weights %lld not a positive multiple of 256", (long long)n);
+    if (!aligned16(d_w)) return fail(DS4MOE_ERR_ALIGN, "pack_q2k: weights not 16-byte aligned");
+    const int64_t nb = n / kQK;
+    k_pack_q2k<<<(unsigned)((nb + 127) / 128), 128, 0, (cudaStream_t)stream>>>(d_w, nb, (uint8_t*)d_blocks);
+    cudaError_t ce = cudaGetLastError();
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "pack_q2k launch");
+}
+
+ds4moe_status ds4moe_pack_iq2xxs(const float* d_w, int64_t n, const uint8_t* d_grid, void* d_blocks, void* stream) {
+    if (!d_w || !d_blocks || !d_grid) return fail(DS4MOE_ERR_ARG, "pack_iq2xxs: NULL argument");
+    if (n <= 0 || n % kQK) return fail(DS4MOE_ERR_ARG, "pack_iq2xxs: n_weights %lld not a positive multiple of 256", (long long)n);
+    if (!aligned16(d_w)) return fail(DS4MOE_ERR_ALIGN, "pack_iq2xxs: weights not 16-byte aligned");
+    const int64_t nb = n / kQK;
+    k_pack_iq2<<<(unsigned)((nb + 3) / 4), 128, 0, (cudaStream_t)stream>>>(d_w, nb, d_grid, (uint8_t*)d_blocks);
+    cudaError_t ce = cudaGetLastError();
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "pack_iq2xxs launch");
+}
+
+ds4moe_status ds4moe_set_grid(ds4moe_t* h, const uint8_t* d_grid, void* stream) {
+    if (!h || !d_grid) return fail(DS4MOE_ERR_ARG, "set_grid: NULL argument");
+    if (!h->weights) return fail(DS4MOE_ERR_NOT_READY, "set_grid: buffers not bound");
+    cudaError_t ce = cudaMemcpyAsync(h->weights + h->off_grid, d_grid, 256 * 8, cudaMemcpyDeviceToDevice,
+                                     (cudaStream_t)stream);
+    if (ce != cudaSuccess) return cuda_fail(ce, "set_grid copy");
+    h->grid_set = true;
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_set_router(ds4moe_t* h, const float* d_W, const float* d_bias, void* stream) {
+    if (!h || !d_W) return fail(DS4MOE_ERR_ARG, "set_router: NULL argument");
+    if (!h->weights) return fail(DS4MOE_ERR_NOT_READY, "set_router: buffers not bound");
+    if (h->shape.has_bias && !d_bias) return fail(DS4MOE_ERR_ARG, "set_router: has_bias set but bias is NULL");
+    if (!h->shape.has_bias && d_bias) return fail(DS4MOE_ERR_ARG, "set_router: bias given but has_bias is 0");
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t E = h->D.E, H = h->D.H;
+    cudaError_t ce = cudaMemcpyAsync(h->weights + h->off_Wr, d_W, E * H * 4, cudaMemcpyDeviceToDevice, st);
+    if (ce == cudaSuccess && d_bias)
+        ce = cudaMemcpyAsync(h->weights + h->off_br, d_bias, E * 4, cudaMemcpyDeviceToDevice, st);
+    if (ce != cudaSuccess) return cuda_fail(ce, "set_router copy");
+    h->router_set = true;
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_set_expert(ds4moe_t* h, int32_t e, const void* d_gate, const void* d_up, const void* d_down,
+                                void* stream) {
+    if (!h || !d_gate || !d_up || !d_down) return fail(DS4MOE_ERR_ARG, "set_expert: NULL argument");
+    if (!h->weights) return fail(DS4MOE_ERR_NOT_READY, "set_expert: buffers not bound");
+    if (e < 0 || e >= h->D.E) return fail(DS4MOE_ERR_ARG, "set_expert: expert %d out of range", e);
+    cudaStream_t st = (cudaStream_t)stream;
+    const int H = h->D.H, I = h->D.I;
+    const int64_t nb = (int64_t)I * H / kQK;
+    const unsigned g1 = (unsigned)((nb * 8 + 255) / 256);
+    k_repack_iq2<<<g1, 256, 0, st>>>((const uint8_t*)d_gate, I, H, h->weights + h->off_gate_qs + e * h->iq2_qs_stride,
+                                     reinterpret_cast<uint16_t*>(h->weights + h->off_gate_d) + e * h->iq2_d_stride);
+    k_repack_iq2<<<g1, 256, 0, st>>>((const uint8_t*)d_up, I, H, h->weights + h->off_up_qs + e * h->iq2_qs_stride,
+                                     reinterpret_cast<uint16_t*>(h->weights + h->off_up_d) + e * h->iq2_d_stride);
+    const int64_t npieces = (int64_t)H * (I / 64);
+    k_repack_q2<<<(unsigned)((npieces + 255) / 256), 256, 0, st>>>(
+        (const uint8_t*)d_down, H, I, h->weights + h->off_down_q + e * h->q2_q_stride,
+        reinterpret_cast<uint32_t*>(h->weights + h->off_down_sc) + e * h->q2_sc_stride,
+        reinterpret_cast<uint32_t*>(h->weights + h->off_down_dd) + e * h->q2_dd_stride);
+    cudaError_t ce = cudaGetLastError();
+    if (ce != cudaSuccess) return cuda_fail(ce, "set_expert launch");
+    h->loaded[e] = 1;
+    return DS4MOE_OK;
+}
+
+ds4moe_status ds4moe_set_shared(ds4moe_t* h, const void* d_gate, const void* d_up, const void* d_down, void* stream) {
+    if (!h || !d_gate || !d_up || !d_down) return fail(DS4MOE_ERR_ARG, "set_shared: NULL argument");
+    if (!h->weights) return fail(DS4MOE_ERR_NOT_READY, "set_shared: buffers not bound");
+    if (!h->shape.has_shared) return fail(DS4MOE_ERR_ARG, "set_shared: layer created without a shared expert");
+    if (!aligned16(d_gate) || !aligned16(d_up) || !aligned16(d_down))
+        return fail(DS4MOE_ERR_ALIGN, "set_shared: matrices must be 16-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    const int H = h->D.H, I = h->D.I;
+    const int64_t n8 = (int64_t)I * H / 8;
+    const unsigned g = (unsigned)((n8 + 255) / 256);
+    k_repack_bf16<<<g, 256, 0, st>>>((const uint4*)d_gate, I, H, (uint4*)(h->weights + h->off_sh_gate));
+    k_repack_bf16<<<g, 256, 0, st>>>((const uint4*)d_up, I, H, (uint4*)(h->weights + h->off_sh_up));
+    k_repack_bf16<<<g, 256, 0, st>>>((const uint4*)d_down, H, I, (uint4*)(h->weights + h->off_sh_down));
+    cudaError_t ce = cudaGetLastError();
+    if (ce != cudaSuccess) return cuda_fail(ce, "set_shared launch");
+    h->shared_set = true;
+    return DS4MOE_OK;
+}
+
+static ds4moe_status check_forward(ds4moe_t* h, const void* x, int32_t n, const void* out, const char* who) {
+    if (!h) return fail(DS4MOE_ERR_ARG, "%s: NULL handle", who);
+    if (n < 0 || n > h->shape.max_tokens)
+        return fail(DS4MOE_ERR_ARG, "%s: n_tokens %d outside 0..%d", who, n, h->shape.max_tokens);
+    if (n > 0 && (!x || !out)) return fail(DS4MOE_ERR_ARG, "%s: NULL buffer", who);
+    std::string why;
+    if (!h->ready(&why)) return fail(DS4MOE_ERR_NOT_READY, "%s: %s", who, why.c_str());
+    return DS4MOE_OK;
+}
+
+static ds4moe_status forward_impl(ds4moe_t* h, const void* d_x, int32_t n, float* d_out, void* const* events,
+                                  void* stream, const char* who) {
+    ds4moe_status s = check_forward(h, d_x, n, d_out, who);
+    if (s != DS4MOE_OK) return s;
+    if (n == 0) return DS4MOE_OK;
+    if (!aligned16(d_x) || !aligned16(d_out)) return fail(DS4MOE_ERR_ALIGN, "%s: x and out must be 16-byte aligned", who);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaEvent_t const* ev = reinterpret_cast<cudaEvent_t const*>(events);
+    cudaError_t ce;
+    if (n <= h->decode_max) {
+        ce = launch_decode(h->weights_view(), h->D, h->decode_ws(), d_x, n, d_out, h->n_sm, st, ev);
+    } else {
+        return fail(DS4MOE_ERR_SHAPE, "%s: n_tokens %d > decode_max %d needs the prefill plan", who, n, h->decode_max);
+    }
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "forward launch");
+}
+
+ds4moe_status ds4moe_forward(ds4moe_t* h, const void* d_x, int32_t n, float* d_out, void* stream) {
+    return forward_impl(h, d_x, n, d_out, nullptr, stream, "forward");
+}
+
+ds4moe_status ds4moe_forward_profiled(ds4moe_t* h, const void* d_x, int32_t n, float* d_out, void* const* events,
+                                      void* stream) {
+    if (!events) return fail(DS4MOE_ERR_ARG, "forward_profiled: NULL events");
+    return forward_impl(h, d_x, n, d_out, events, stream, "forward_profiled");
+}
+
+int32_t ds4moe_plan_launches(const ds4moe_t* h, int32_t n) {
+    if (!h || n < 1 || n > h->shape.max_tokens) return 0;
+    if (n <= h->decode_max) return decode_launches();
+    return 0;
+}
+
+const char* ds4moe_plan_kernel(const ds4moe_t* h, int32_t n, int32_t i) {
+    if (i < 0 || i >= ds4moe_plan_launches(h, n)) return nullptr;
+    if (n <= h->decode_max) return decode_kernel_name(i);
+    return nullptr;
+}
+
+ds4moe_status ds4moe_forward_host(ds4moe_t* h, const void* x_host, int32_t n, float* out_host, void* stream) {
+    ds4moe_status s = check_forward(h, x_host, n, out_host, "forward_host");
+    if (s != DS4MOE_OK) return s;
+    if (n == 0) return DS4MOE_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t xb = (size_t)n * h->D.H * (h->D.act_bf16 ? 2 : 4), ob = (size_t)n * h->D.H * 4;
+    void* dx = h->ws + h->L.x_stage;
+    float* dout = reinterpret_cast<float*>(h->ws + h->L.out_stage);
+    cudaError_t ce = cudaMemcpyAsync(dx, x_host, xb, cudaMemcpyHostToDevice, st);
+    if (ce != cudaSuccess) return cuda_fail(ce, "forward_host: copy in");
+    s = ds4moe_forward(h, dx, n, dout, stream);
+    if (s != DS4MOE_OK) return s;
+    ce = cudaMemcpyAsync(out_host, dout, ob, cudaMemcpyDeviceToHost, st);
+    if (ce != cudaSuccess) return cuda_fail(ce, "forward_host: copy out");
+    ce = cudaStreamSynchronize(st);
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "forward_host: synchronize");
+}
+
+ds4moe_status ds4moe_route(ds4moe_t* h, const void* d_x, int32_t n, int32_t* d_ids, float* d_w, void* stream) {
+    ds4moe_status s = check_forward(h, d_x, n, d_ids, "route");
+    if (s != DS4MOE_OK) return s;
+    if (n == 0) return DS4MOE_OK;
+    if (!d_w) return fail(DS4MOE_ERR_ARG, "route: NULL weights");
+    if (!aligned16(d_x)) return fail(DS4MOE_ERR_ALIGN, "route: x must be 16-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    if (n > h->decode_max) return fail(DS4MOE_ERR_SHAPE, "route: n_tokens %d > decode_max", n);
+    DecodeWs ws = h->decode_ws();
+    cudaError_t ce = launch_route(h->weights_view(), h->D, ws, d_x, n, st);
+    if (ce == cudaSuccess)
+        ce = cudaMemcpyAsync(d_ids, ws.ids, (size_t)n * h->D.k * 4, cudaMemcpyDeviceToDevice, st);
+    if (ce == cudaSuccess)
+        ce = cudaMemcpyAsync(d_w, ws.wts, (size_t)n * h->D.k * 4, cudaMemcpyDeviceToDevice, st);
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "route");
+}
+
+ds4moe_status ds4moe_dequant(ds4moe_t* h, int32_t e, int32_t which, int32_t as_bf16, void* d_out, void* stream) {
+    if (!h || !d_out) return fail(DS4MOE_ERR_ARG, "dequant: NULL argument");
+    if (!h->weights) return fail(DS4MOE_ERR_NOT_READY, "dequant: buffers not bound");
+    cudaStream_t st = (cudaStream_t)stream;
+    const int H = h->D.H, I = h->D.I;
+    float* of = as_bf16 ? nullptr : (float*)d_out;
+    __nv_bfloat16* ob = as_bf16 ? (__nv_bfloat16*)d_out : nullptr;
+    const unsigned g = (unsigned)(((int64_t)H * I + 255) / 256);
+    if (e == -1) {   // the shared expert (bf16 as stored)
+        if (!h->shape.has_shared || !h->shared_set) return fail(DS4MOE_ERR_NOT_READY, "dequant: no shared expert");
+        const uint8_t* b = h->weights;
+        const __nv_bfloat16* t = reinterpret_cast<const __nv_bfloat16*>(
+            b + (which == 0 ? h->off_sh_gate : which == 1 ? h->off_sh_up : h->off_sh_down));
+        if (which < 0 || which > 2) return fail(DS4MOE_ERR_ARG, "dequant: which %d", which);
+        k_dequant_bf16_tiles<<<g, 256, 0, st>>>(t, which == 2 ? H : I, which == 2 ? I : H, of, ob);
+    } else {
+        if (e < 0 || e >= h->D.E) return fail(DS4MOE_ERR_ARG, "dequant: expert %d out of range", e);
+        if (!h->loaded[e]) return fail(DS4MOE_ERR_NOT_READY, "dequant: expert %d not loaded", e);
+        if (which == 0 || which == 1) {
+            if (!h->grid_set) return fail(DS4MOE_ERR_NOT_READY, "dequant: grid not set");
+            const size_t oq = which == 0 ? h->off_gate_qs : h->off_up_qs;
+            const size_t od = which == 0 ? h->off_gate_d : h->off_up_d;
+            k_dequant_iq2<<<g, 256, 0, st>>>(h->weights + oq + e * h->iq2_qs_stride,
+                                             reinterpret_cast<const uint16_t*>(h->weights + od) + e * h->iq2_d_stride,
+                                             h->weights + h->off_grid, I, H, of, ob);
+        } else if (which == 2) {
+            k_dequant_q2<<<g, 256, 0, st>>>(h->weights + h->off_down_q + e * h->q2_q_stride,
+                                            reinterpret_cast<const uint32_t*>(h->weights + h->off_down_sc) + e * h->q2_sc_stride,
+                                            reinterpret_cast<const uint32_t*>(h->weights + h->off_down_dd) + e * h->q2_dd_stride,
+                                            H, I, of, ob);
+        } else {
+            return fail(DS4MOE_ERR_ARG, "dequant: which %d", which);
+        }
+    }
+    cudaError_t ce = cudaGetLastError();
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "dequant launch");
+}
+
+ds4moe_status ds4moe_get_device_error(ds4moe_t* h, void* stream, int32_t* code) {
+    if (!h || !code) return fail(DS4MOE_ERR_ARG, "get_device_error: NULL argument");
+    if (!h->ws) return fail(DS4MOE_ERR_NOT_READY, "get_device_error: buffers not bound");
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t v = 0;
+    cudaError_t ce = cudaStreamSynchronize(st);
+    if (ce == cudaSuccess) ce = cudaMemcpy(&v, h->ws + h->L.hdr, 4, cudaMemcpyDeviceToHost);
+    if (ce == cudaSuccess && v) ce = cudaMemset(h->ws + h->L.hdr, 0, 4);
+    if (ce != cudaSuccess) return cuda_fail(ce, "get_device_error");
+    *code = (int32_t)v;
+    if (v & kErrTimeout) return fail(DS4MOE_ERR_TIMEOUT, "a bounded device wait timed out (code %u)", v);
+    if (v) return fail(DS4MOE_ERR_DEVICE, "device-side check failed (code %u)", v);
+    return DS4MOE_OK;
+}
+
+}  // extern "C"

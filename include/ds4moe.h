@@ -1,0 +1,200 @@
+/*
+ * ds4moe.h -- C ABI of the ds4 routed-MoE expert FFN on B200 (sm_100a).
+ *
+ * The operation (the pages describe the ds4 engine for DeepSeek V4 Flash):
+ *   "antirez가 만든 DeepSeek V4 Flash 전용 로컬 추론 엔진 ds4" (jeff.news),
+ *   2-bit quantization bullets: only the routed MoE experts are quantized --
+ *   up/gate in IQ2_XXS, down in Q2_K -- while the shared experts, the
+ *   projections and the routing stay at full precision.
+ *   "antirez/ds4 -- Metal용 DeepSeek V4 Flash 로컬 추론 엔진 완벽 가이드"
+ *   (sigco.tistory.com), "왜 독자 엔진이 필요할까": each input runs through only
+ *   some of the experts.
+ * For every token x (length H): router logits l = W_r x (+ b), the top-k
+ * experts by (logit desc, index asc), weights w = softmax over those k logits;
+ * for each selected expert e: h = silu(W_gate,e x) * (W_up,e x),
+ * y_e = W_down,e h; out = y_shared + sum_j w_j y_{e_j}, with the shared expert
+ * an unquantized bf16 SwiGLU FFN of the same intermediate size I.
+ *
+ * Conventions (every function):
+ *   - returns ds4moe_status: 0 on success, a negative code otherwise; on an
+ *     error nothing is launched and ds4moe_last_error() holds a message.
+ *   - pointers named d_* (and every tensor argument unless a function says
+ *     "host") are CUDA device pointers owned by the caller; the library never
+ *     allocates device memory and never frees the caller's buffers.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All device work is asynchronous on it unless stated.
+ *   - matrices are row-major with rows = output features:
+ *     W_gate, W_up: [I][H]; W_down: [H][I]; W_r: [E][H].
+ *
+ * Block formats (little endian; 256 weights per block, blocked over the
+ * row-major flat index of the matrix):
+ *   Q2_K-style, 84 bytes: [0,16) scale byte j = sc_j | m_j<<4 for sub-block
+ *     j (weights 16j..16j+15); [16,80) 2-bit code q_i at byte 16+i/4, bits
+ *     2(i%4); [80,82) d, [82,84) dmin as binary16.
+ *     weight_i = (d*sc_j)*q_i - dmin*m_j   (one rounding to binary32)
+ *   IQ2_XXS-style, 66 bytes: [0,2) d (binary16); eight 8-byte groups g at
+ *     2+8g: bytes 0..3 = grid rows a_c of chunks c (8 weights each), bytes
+ *     4..7 = uint32 S with sign field sigma_c in bits 7c..7c+6 and the group
+ *     scale s_g in bits 28..31.  Element i<7 of chunk c is negative when bit i
+ *     of sigma_c is set, element 7 when sigma_c has odd popcount.
+ *     weight = d*(2 s_g+1)/8 * G[a_c][i] * (+-1)   (exact in binary32)
+ *     G is a 256 x 8 table of uint8 magnitudes supplied by the caller.
+ */
+#ifndef DS4MOE_H
+#define DS4MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DS4MOE_OK = 0,
+    DS4MOE_ERR_ARG = -1,        /* NULL pointer, out-of-range count or index */
+    DS4MOE_ERR_ALIGN = -2,      /* a pointer is not 16-byte aligned */
+    DS4MOE_ERR_SHAPE = -3,      /* unsupported layer shape */
+    DS4MOE_ERR_NOT_READY = -4,  /* buffers not bound, or weights not all loaded */
+    DS4MOE_ERR_CUDA = -5,       /* a CUDA runtime call failed */
+    DS4MOE_ERR_TIMEOUT = -6,    /* a bounded device-side wait gave up */
+    DS4MOE_ERR_DEVICE = -7      /* a device-side check failed (see ds4moe_get_device_error) */
+} ds4moe_status;
+
+enum { DS4MOE_ACT_F32 = 0, DS4MOE_ACT_BF16 = 1 };
+
+typedef struct {
+    int32_t hidden;        /* H: multiple of 256 */
+    int32_t inter;         /* I: multiple of 256, or 128 */
+    int32_t n_experts;     /* E: 1 .. 1024 */
+    int32_t top_k;         /* k: 1 .. min(E, 16) */
+    int32_t max_tokens;    /* largest n_tokens any forward call will pass (>= 1) */
+    int32_t act_dtype;     /* DS4MOE_ACT_F32 or DS4MOE_ACT_BF16: element type of x */
+    int32_t has_shared;    /* 1: add the bf16 shared expert; 0: routed experts only */
+    int32_t has_bias;      /* 1: the router adds a bias b[E] */
+    int32_t decode_max;    /* n_tokens <= decode_max uses the fp32 GEMV plan
+                              (0 selects the default, 8); larger n uses the
+                              bf16 tensor-core plan */
+} ds4moe_shape;
+
+typedef struct ds4moe ds4moe_t;   /* opaque handle; host memory owned by the library */
+
+/* Validate the shape and create a handle.  *out receives the handle. */
+ds4moe_status ds4moe_create(const ds4moe_shape* shape, ds4moe_t** out);
+
+/* Free the handle (host memory only; bound device buffers stay the caller's). */
+ds4moe_status ds4moe_destroy(ds4moe_t* h);
+
+/* Bytes of device memory the caller must provide for the layer weights
+ * (router, grid, all experts in the device layout, shared expert). */
+size_t ds4moe_weight_bytes(const ds4moe_t* h);
+
+/* Bytes of device scratch a forward of up to n_tokens tokens needs
+ * (n_tokens <= max_tokens; pass max_tokens to size one buffer for all). */
+size_t ds4moe_workspace_bytes(const ds4moe_t* h, int32_t n_tokens);
+
+/* Bind caller-owned device buffers: d_weights (>= ds4moe_weight_bytes) and
+ * d_workspace (>= ds4moe_workspace_bytes(h, max_tokens)), both 256-byte
+ * aligned.  Clears the workspace's counters and error word on `stream`.
+ * Rebinding marks every expert as not loaded. */
+ds4moe_status ds4moe_bind(ds4moe_t* h, void* d_weights, size_t weight_bytes, void* d_workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* ---- packers (quantizers), on the device -------------------------------- */
+
+/* Quantize n_weights binary32 values d_w (n_weights a multiple of 256, read as
+ * consecutive 256-weight blocks of the flat row-major matrix) into Q2_K-style
+ * blocks at d_blocks (n_weights/256 * 84 bytes).  Decisions in fp64:
+ * per sub-block lo = min(0, min w), hi = max(0, max w), scale = (hi-lo)/3,
+ * min = -lo; d = half(max scale/15), dmin = half(max min/15);
+ * sc = clamp(rne(scale/d), 0, 15), m = clamp(rne(min/dmin), 0, 15);
+ * q = clamp(rne((w + dmin m)/(d sc)), 0, 3); zero divisors give zero fields. */
+ds4moe_status ds4moe_pack_q2k(const float* d_w, int64_t n_weights, void* d_blocks, void* stream);
+
+/* Quantize into IQ2_XXS-style blocks (n_weights/256 * 66 bytes) with grid
+ * d_grid [256*8] uint8.  Decisions in fp64: d = half(max|w| / (43*31/8))
+ * (zero block if d == 0); s_g = clamp(rne(4 max|w_g|/(43 d) - 0.5), 0, 15);
+ * per 8-weight chunk the negative flags, with the smallest-|w| element
+ * (lowest index on ties) flipped if their count is odd; the grid row
+ * minimizing sum (d(2s_g+1)/8 G[a][i] - t_i)^2 over t_i = +-|w_i| (ties to
+ * the lowest row). */
+ds4moe_status ds4moe_pack_iq2xxs(const float* d_w, int64_t n_weights, const uint8_t* d_grid, void* d_blocks,
+                                 void* stream);
+
+/* ---- loading (device pointers in; repacked into the bound weight buffer) - */
+
+/* Grid magnitudes [256][8] uint8. */
+ds4moe_status ds4moe_set_grid(ds4moe_t* h, const uint8_t* d_grid, void* stream);
+
+/* Router rows [E][H] binary32 and, when has_bias, bias [E] (else NULL). */
+ds4moe_status ds4moe_set_router(ds4moe_t* h, const float* d_W, const float* d_bias, void* stream);
+
+/* Expert e's three matrices as canonical blocks: gate, up IQ2_XXS-style
+ * ([I][H] -> I*H/256 blocks), down Q2_K-style ([H][I] -> H*I/256 blocks). */
+ds4moe_status ds4moe_set_expert(ds4moe_t* h, int32_t e, const void* d_gate, const void* d_up,
+                                const void* d_down, void* stream);
+
+/* Shared expert as bfloat16: gate, up [I][H]; down [H][I].  Required when
+ * has_shared = 1. */
+ds4moe_status ds4moe_set_shared(ds4moe_t* h, const void* d_gate, const void* d_up, const void* d_down,
+                                void* stream);
+
+/* ---- the hot path -------------------------------------------------------- */
+
+/* out[n_tokens][H] (binary32) = the layer applied to x[n_tokens][H] (element
+ * type act_dtype).  x and out are 16-byte aligned device buffers.  Plan:
+ * n_tokens <= decode_max -> fp32 GEMV path (router + top-k, fused gate/up +
+ * SwiGLU, down + gate-weighted combine); otherwise the bf16 tensor-core path
+ * (router, permutation by expert, grouped tcgen05 GEMMs, combine).
+ * n_tokens == 0 is a no-op.  Launches only; safe to capture in a CUDA graph. */
+ds4moe_status ds4moe_forward(ds4moe_t* h, const void* d_x, int32_t n_tokens, float* d_out, void* stream);
+
+/* The same computation with HOST buffers: copies x_host to the device (into
+ * the workspace), runs ds4moe_forward, copies the result to out_host and
+ * synchronizes `stream`.  Pinned host memory gives the fastest copies. */
+ds4moe_status ds4moe_forward_host(ds4moe_t* h, const void* x_host, int32_t n_tokens, float* out_host,
+                                  void* stream);
+
+/* ---- measurement ---------------------------------------------------------- */
+
+/* Number of kernel launches one ds4moe_forward of n_tokens makes (0 if n_tokens
+ * is outside 1..max_tokens). */
+int32_t ds4moe_plan_launches(const ds4moe_t* h, int32_t n_tokens);
+
+/* Name of launch i (0-based) of that plan, a static string; NULL if out of range. */
+const char* ds4moe_plan_kernel(const ds4moe_t* h, int32_t n_tokens, int32_t i);
+
+/* ds4moe_forward that also records events[2i] on `stream` right before launch
+ * i and events[2i+1] right after it, for i < ds4moe_plan_launches(h, n):
+ * cudaEvent_t handles created by the caller (with timing enabled).  The
+ * elapsed time between the two events of a launch is that kernel's duration
+ * on the stream.  Same results as ds4moe_forward. */
+ds4moe_status ds4moe_forward_profiled(ds4moe_t* h, const void* d_x, int32_t n_tokens, float* d_out,
+                                      void* const* events, void* stream);
+
+/* ---- inspection hooks (same device code as the hot path) ----------------- */
+
+/* Routing only: ids[n][k] (int32, rank order) and weights[n][k] (binary32). */
+ds4moe_status ds4moe_route(ds4moe_t* h, const void* d_x, int32_t n_tokens, int32_t* d_ids, float* d_weights,
+                           void* stream);
+
+/* Dequantize expert e's matrix `which` (0 gate, 1 up, 2 down) from the
+ * loaded device layout into d_out, row-major, as binary32 (as_bf16 = 0) or
+ * bfloat16 rounded to nearest even (as_bf16 = 1): exactly the values the
+ * kernels multiply. */
+ds4moe_status ds4moe_dequant(ds4moe_t* h, int32_t e, int32_t which, int32_t as_bf16, void* d_out,
+                             void* stream);
+
+/* Synchronize `stream`, then read and clear the workspace's device error word
+ * into *code (0 = none; bit 0 = an index check failed, bit 1 = a bounded
+ * wait timed out).  Returns DS4MOE_ERR_DEVICE / DS4MOE_ERR_TIMEOUT when set. */
+ds4moe_status ds4moe_get_device_error(ds4moe_t* h, void* stream, int32_t* code);
+
+/* Message of the last error on the calling thread ("" if none). */
+const char* ds4moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DS4MOE_H */

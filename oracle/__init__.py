@@ -58,6 +58,7 @@ def lib():
         L.orc_double_to_half.restype = ctypes.c_uint16
         L.orc_bf16_round.argtypes = [ctypes.c_float]
         L.orc_bf16_round.restype = ctypes.c_float
+        L.orc_bf16_round_array.argtypes = [vp, i64, vp]
         L.orc_dequant_q2k.argtypes = [vp, i64, vp]
         L.orc_dequant_iq2xxs.argtypes = [vp, i64, vp, vp]
         L.orc_pack_q2k.argtypes = [vp, i64, vp]
@@ -94,8 +95,9 @@ def double_to_half(v: float) -> int:
 def bf16_round(v) -> np.ndarray:
     """Elementwise bfloat16 round-half-to-even of binary32 values (returned as float32)."""
     a = np.ascontiguousarray(v, dtype=np.float32).ravel()
-    f = lib().orc_bf16_round
-    return np.array([f(float(x)) for x in a], dtype=np.float32).reshape(np.shape(v))
+    out = np.empty_like(a)
+    lib().orc_bf16_round_array(_p(a), a.size, _p(out))
+    return out.reshape(np.shape(v))
 
 
 # ---------------------------------------------------------------- formats
@@ -210,3 +212,31 @@ def moe_forward(layer: dict, x: np.ndarray, mode: int = 0):
     if rc != 0:
         raise ValueError("orc_moe_forward: bad argument or missing expert blocks")
     return out, ids, w
+
+
+def layer_from_torch(layer: dict, experts=None) -> dict:
+    """numpy view of a synthetic layer (torch tensors, any device) for moe_forward.
+
+    `experts` limits which experts' blocks are copied to the host (the others
+    stay None); the shared expert's bfloat16 tensors become uint16 bit patterns.
+    """
+    import torch
+
+    E = int(layer["E"])
+    keep = range(E) if experts is None else sorted(set(int(e) for e in experts))
+    gate, up, down = [None] * E, [None] * E, [None] * E
+    for e in keep:
+        gate[e] = layer["gate"][e].cpu().numpy()
+        up[e] = layer["up"][e].cpu().numpy()
+        down[e] = layer["down"][e].cpu().numpy()
+    b = layer.get("b_r")
+
+    def bits(t):
+        return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    out = dict(H=layer["H"], I=layer["I"], E=E, k=layer["k"], W_r=layer["W_r"].cpu().numpy(),
+               b_r=None if b is None else b.cpu().numpy(), grid=layer["grid"].cpu().numpy(),
+               gate=gate, up=up, down=down, sh_gate=None, sh_up=None, sh_down=None)
+    if layer.get("sh_gate") is not None:
+        out.update(sh_gate=bits(layer["sh_gate"]), sh_up=bits(layer["sh_up"]), sh_down=bits(layer["sh_down"]))
+    return out

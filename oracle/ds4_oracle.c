@@ -101,6 +101,11 @@ float orc_bf16_round(float v) {
     return signbit(v) ? -out : out;
 }
 
+/* orc_bf16_round over an array. */
+void orc_bf16_round_array(const float* v, int64_t n, float* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_bf16_round(v[i]);
+}
+
 static uint16_t rd16(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
 static uint32_t rd32(const uint8_t* p) {
     return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);

@@ -1,0 +1,51 @@
+"""The C-ABI library loads and exports every entry point include/ds4moe.h declares (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "ds4moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ds4moe_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def libpath():
+    from bit_quantized_moe_softmax_b200 import build
+
+    return build.build()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("ds4moe_create", "ds4moe_pack_q2k", "ds4moe_pack_iq2xxs", "ds4moe_forward"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(libpath):
+    lib = ctypes.CDLL(libpath)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", libpath], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (ds4moe_\w+)", out))
+    assert set(_declared()) <= exported
+
+
+def test_binding_names_match_header(libpath):
+    import bit_quantized_moe_softmax_b200 as m
+
+    assert set(m.EXPORTS) == set(_declared())
+    for name in _declared():
+        assert callable(getattr(m, name)), name
+
+
+def test_last_error_without_gpu(libpath):
+    import bit_quantized_moe_softmax_b200 as m
+
+    assert isinstance(m.ds4moe_last_error(), str)
