@@ -31,7 +31,7 @@ EXPORTS = ("ds4moe_create", "ds4moe_destroy", "ds4moe_weight_bytes", "ds4moe_wor
            "ds4moe_pack_q2k", "ds4moe_pack_iq2xxs", "ds4moe_set_grid", "ds4moe_set_router", "ds4moe_set_expert",
            "ds4moe_set_shared", "ds4moe_forward", "ds4moe_forward_host", "ds4moe_route", "ds4moe_dequant",
            "ds4moe_get_device_error", "ds4moe_last_error", "ds4moe_plan_launches", "ds4moe_plan_kernel",
-           "ds4moe_forward_profiled")
+           "ds4moe_forward_profiled", "ds4moe_route_noalloc")
 
 
 class ds4moe_shape(ctypes.Structure):
@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
             "ds4moe_plan_launches": ([vp, i32], i32),
             "ds4moe_plan_kernel": ([vp, i32, i32], ctypes.c_char_p),
             "ds4moe_forward_profiled": ([vp, vp, i32, vp, ctypes.POINTER(vp), vp], i32),
+            "ds4moe_route_noalloc": ([vp, vp, i32, vp, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -181,6 +182,18 @@ def ds4moe_forward_host(h: int, x_host: torch.Tensor, out_host: torch.Tensor, st
 
 def ds4moe_route(h: int, x: torch.Tensor, ids: torch.Tensor, w: torch.Tensor, stream=None):
     _ok(lib().ds4moe_route(h, _ptr(x), x.shape[0], _ptr(ids), _ptr(w), _stream(stream)), "ds4moe_route")
+
+
+def ds4moe_route_noalloc(h: int, x: torch.Tensor, ids: torch.Tensor, w: torch.Tensor, stream=None):
+    """Routing with the library's static device scratch instead of the bound workspace.
+
+    For callers that cannot allocate device memory (for example while a CUDA
+    graph is being captured, or inside a host that owns all device buffers);
+    see include/ds4moe.h for the limit (n_tokens * n_experts <= 8192) and the
+    rule that overlapping calls race on the shared scratch.
+    """
+    _ok(lib().ds4moe_route_noalloc(h, _ptr(x), x.shape[0], _ptr(ids), _ptr(w), _stream(stream)),
+        "ds4moe_route_noalloc")
 
 
 def ds4moe_dequant(h: int, e: int, which: int, as_bf16: int, out: torch.Tensor, stream=None):

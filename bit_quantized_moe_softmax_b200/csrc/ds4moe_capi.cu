@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -30,6 +31,14 @@ cudaError_t launch_route(const Weights& W, const Dims& D, const DecodeWs& ws, co
 }  // namespace ds4
 
 using namespace ds4;
+
+// Scratch of ds4moe_route_noalloc: a 64-word header (the router's ticket and
+// task counters; cleared before every call) followed by the logits of up to
+// kNoAllocLogits (token, expert) pairs.  One copy per device, for the life of
+// the process; its device address is looked up once per device.
+constexpr int kNoAllocHeader = 64;
+constexpr int kNoAllocLogits = 8192;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocHeader + kNoAllocLogits];
 
 namespace {
 
@@ -451,6 +460,51 @@ ds4moe_status ds4moe_dequant(ds4moe_t* h, int32_t e, int32_t which, int32_t as_b
     }
     cudaError_t ce = cudaGetLastError();
     return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "dequant launch");
+}
+
+ds4moe_status ds4moe_route_noalloc(ds4moe_t* h, const void* d_x, int32_t n, int32_t* d_ids, float* d_w,
+                                   void* stream) {
+    static std::mutex mu;
+    static float* scratch_of_device[64] = {};
+    ds4moe_status s = check_forward(h, d_x, n, d_ids, "route_noalloc");
+    if (s != DS4MOE_OK) return s;
+    if (n == 0) return DS4MOE_OK;
+    if (!d_w) return fail(DS4MOE_ERR_ARG, "route_noalloc: NULL weights");
+    if (!aligned16(d_x)) return fail(DS4MOE_ERR_ALIGN, "route_noalloc: x must be 16-byte aligned");
+    if (n > h->decode_max) return fail(DS4MOE_ERR_ARG, "route_noalloc: n_tokens %d > decode_max %d", n, h->decode_max);
+    if ((int64_t)n * h->D.E > kNoAllocLogits)
+        return fail(DS4MOE_ERR_ARG, "route_noalloc: n_tokens * n_experts = %lld exceeds the static scratch limit %d",
+                    (long long)n * h->D.E, kNoAllocLogits);
+    int dev = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce != cudaSuccess) return cuda_fail(ce, "route_noalloc: cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(DS4MOE_ERR_ARG, "route_noalloc: device %d beyond 64", dev);
+    float* base = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!scratch_of_device[dev]) {
+            void* p = nullptr;
+            ce = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+            if (ce != cudaSuccess) return cuda_fail(ce, "route_noalloc: cudaGetSymbolAddress");
+            scratch_of_device[dev] = static_cast<float*>(p);
+        }
+        base = scratch_of_device[dev];
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    // the counters must start at zero; the previous call's contents are stale
+    ce = cudaMemsetAsync(base, 0, kNoAllocHeader * sizeof(float), st);
+    if (ce != cudaSuccess) return cuda_fail(ce, "route_noalloc: clear header");
+    uint32_t* hdr = reinterpret_cast<uint32_t*>(base);
+    DecodeWs ws{};
+    ws.err = hdr + 0;
+    ws.ticket = hdr + 1;
+    ws.queue1 = hdr + 2;
+    ws.queue2 = hdr + 3;
+    ws.logits = base + kNoAllocHeader;
+    ws.ids = d_ids;
+    ws.wts = d_w;
+    ce = launch_route(h->weights_view(), h->D, ws, d_x, n, st);
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "route_noalloc launch");
 }
 
 ds4moe_status ds4moe_get_device_error(ds4moe_t* h, void* stream, int32_t* code) {

@@ -185,6 +185,27 @@ ds4moe_status ds4moe_route(ds4moe_t* h, const void* d_x, int32_t n_tokens, int32
 ds4moe_status ds4moe_dequant(ds4moe_t* h, int32_t e, int32_t which, int32_t as_bf16, void* d_out,
                              void* stream);
 
+/* ---- routing without device allocation ------------------------------------ */
+
+/* ds4moe_route for callers that cannot allocate device memory: code that runs
+ * while a CUDA graph is being captured (allocation is not allowed there and a
+ * synchronizing allocator would break the capture), and hosts that own every
+ * device buffer and hand this library only its inputs and outputs.  The
+ * pages have no counterpart; this is an interface convenience.
+ * The router's scratch (logits of up to 8192 token-expert pairs, i.e.
+ * n_tokens * n_experts <= 8192, and a 256-byte counter header) lives in one
+ * static device array inside the library, which every GPU that loads the
+ * library holds until the process exits; the bound workspace is not used.
+ * The caller passes x and the outputs ids[n][k] (int32) and weights[n][k]
+ * (binary32), with the same results as ds4moe_route.  Larger n_tokens *
+ * n_experts, or n_tokens > decode_max, is rejected with DS4MOE_ERR_ARG.
+ * The first call on a device looks up the array's device address (make that
+ * first call before any stream capture).  Every call shares the one array:
+ * calls that overlap on the GPU (other streams, other threads) race, so
+ * serialize them. */
+ds4moe_status ds4moe_route_noalloc(ds4moe_t* h, const void* d_x, int32_t n_tokens, int32_t* d_ids,
+                                   float* d_weights, void* stream);
+
 /* Synchronize `stream`, then read and clear the workspace's device error word
  * into *code (0 = none; bit 0 = an index check failed, bit 1 = a bounded
  * wait timed out).  Returns DS4MOE_ERR_DEVICE / DS4MOE_ERR_TIMEOUT when set. */
