@@ -184,16 +184,21 @@ def run_ours(args, wl, rank, local, world):
     # graphs of S consecutive steps (cycling instances and token vectors)
     S = max(1, min(args.steps, 64 if R * P >= 64 else R))
 
+    def new_events(count):
+        # torch creates the CUDA event on first record: record each once before capture
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nl)] for _ in range(count)]
+        for ev in evs:
+            for e in ev:
+                e.record(stream)
+        stream.synchronize()
+        return evs
+
     def capture(count, first, profiled):
         g = torch.cuda.CUDAGraph()
-        evs = []
+        evs = new_events(count) if profiled else []
         with torch.cuda.graph(g, stream=stream):
             for j in range(count):
-                ev = None
-                if profiled:
-                    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * nl)]
-                    evs.append(ev)
-                step(first + j, ev)
+                step(first + j, evs[j] if profiled else None)
         return g, evs
 
     def graphs_for(K, profiled):

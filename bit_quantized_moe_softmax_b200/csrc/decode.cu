@@ -1,68 +1,100 @@
-// decode.cu -- the fp32 GEMV plan for 1..decode_max tokens.
+// decode.cu -- the fp32 GEMV plan for 1..decode_max tokens (three launches).
 //
-//   k_router_decode   logits in the canonical binary32 order, then (last CTA)
-//                     top-k by (logit desc, index asc) and the softmax over
-//                     the selected logits
-//   k_gateup_decode   for every selected expert (each read once, applied to
-//                     all tokens that chose it) and the shared expert:
-//                     g = W_gate x, u = W_up x, h = silu(g) * u
-//   k_down_decode     y = W_down h per selected expert slot and for the shared
-//                     expert
-//   k_combine_decode  out = y_shared + sum_j w_j y_j, j in rank order
+//   k_router_decode  warp per expert row, logits in the canonical binary32
+//                    order; the last CTA picks the top-k by (logit desc,
+//                    index asc) and the softmax over the selected logits.
+//   k_gateup_decode  h = silu(W_gate x) * (W_up x) for every selected expert
+//                    (read once, applied to all tokens that chose it) and for
+//                    the shared expert.
+//   k_down_decode    y = W_down h per selected expert and for the shared
+//                    expert; the last task to finish a 32-row block of the
+//                    output sums out = y_shared + sum_j w_j y_j in rank order.
 //
-// The weights are streamed once from HBM with 128-bit loads that skip L1;
-// the IQ2 grid is expanded to binary32 in shared memory in 8 interleaved
+// The two GEMV kernels are persistent (one CTA per SM): a producer warp pulls
+// row tasks from an atomic queue and streams their weights into a ring of
+// shared-memory stages with bulk copies (cp.async.bulk + mbarrier), eight
+// consumer warps dequantize and multiply out of shared memory.  Each is
+// launched with programmatic dependent launch: the gate/up grid starts its
+// shared-expert tasks while the router still runs, and the down grid streams
+// its weights while gate/up finishes; both wait (griddepcontrol.wait) only
+// where they read the previous grid's results.
+//
+// The IQ2 grid is expanded to binary32 in shared memory, in 8 interleaved
 // copies so that the per-lane random row lookups of a quarter warp never
-// share a bank.  Work is split into row tasks handed out by an atomic queue,
-// larger tasks first.
+// share a bank.
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "ds4moe_internal.cuh"
 
 namespace ds4 {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
-constexpr int kMaxSlots = 128;          // decode_max (<= 8) * top_k (<= 16)
-constexpr int kTabFloats = 256 * 2 * 8 * 4;
+// Consumer warps per CTA of the GEMV kernels (plus one producer warp).
+template <int NT>
+struct Warps {
+    static constexpr int CW = NT <= 2 ? 16 : 8;
+    static constexpr int kThreads = (CW + 1) * 32;
+};
+constexpr int kMaxSlots = 128;                 // decode_max (<= 8) * top_k (<= 16)
+constexpr int kStageBytes = 34816;             // 32 KB of weights + 2 KB of scales
+constexpr int kRWarps = 4;                     // router warps per CTA
 
 // ---------------------------------------------------------------- router
 __device__ __forceinline__ float4 load_x4(const void* x, int act_bf16, int64_t idx) {
     if (act_bf16) {
-        uint2 v = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(x) + idx);
+        uint2 v = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(x) + idx));
         return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
                            __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
     }
-    return *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + idx);
+    return __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + idx));
 }
 
 __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
     return v > bv || (v == bv && i < bi);
 }
 
-// Top-k and softmax of one token's logits by one warp.
-__device__ void topk_softmax_warp(const float* logits, int E, int k, int32_t* ids, float* wts) {
-    int lane = threadIdx.x & 31;
+// Order-preserving map binary32 -> uint32 (larger logit, larger key).
+__device__ __forceinline__ uint32_t order_key(float v) {
+    const uint32_t u = __float_as_uint(v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Top-k and softmax of one token's logits by one warp.  Each lane keeps the
+// best of its own candidates (experts lane, lane + 32, ...); a round picks the
+// warp maximum with two warp reductions (largest key, then the lowest expert
+// index among equal keys) and the winning lane advances to its next best.
+// `buf` is E floats of shared memory.
+__device__ void topk_softmax_warp(const float* logits_g, float* buf, int E, int k, int32_t* ids, float* wts) {
+    const int lane = threadIdx.x & 31;
+    for (int e = lane; e < E; e += 32) buf[e] = __ldcg(logits_g + e);
+    __syncwarp();
     uint32_t taken = 0;   // bit m: candidate lane + 32 m already chosen (E <= 1024)
+    auto local_best = [&](uint32_t& key, int& idx) {
+        key = 0;
+        idx = 0x7fffffff;
+        for (int m = 0; lane + 32 * m < E; ++m) {
+            if (taken & (1u << m)) continue;
+            const uint32_t kk = order_key(buf[lane + 32 * m]);
+            if (kk > key) { key = kk; idx = lane + 32 * m; }   // ascending index: strict > keeps the lowest
+        }
+    };
+    uint32_t key;
+    int idx;
+    local_best(key, idx);
     float my_l = 0.f;
     int my_id = 0;
     for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-        for (int m = 0; lane + 32 * m < E; ++m) {
-            if (taken & (1u << m)) continue;
-            int e = lane + 32 * m;
-            float v = __ldcg(logits + e);
-            if (better(v, e, bv, bi)) { bv = v; bi = e; }
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+        const int win = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)idx : 0xffffffffu);
+        if (lane == j) { my_l = buf[win]; my_id = win; }
+        if ((win & 31) == lane) {
+            taken |= 1u << (win >> 5);
+            local_best(key, idx);
         }
-        for (int off = 16; off >= 1; off >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-        }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (lane == j) { my_l = bv; my_id = bi; }
     }
-    float lmax = __shfl_sync(0xffffffffu, my_l, 0);
-    float ex = lane < k ? __expf(my_l - lmax) : 0.f;
+    const float lmax = __shfl_sync(0xffffffffu, my_l, 0);
+    const float ex = lane < k ? __expf(my_l - lmax) : 0.f;
     float den = ex;
     for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
     if (lane < k) {
@@ -72,26 +104,45 @@ __device__ void topk_softmax_warp(const float* logits, int E, int k, int32_t* id
 }
 
 template <int NT>
-__global__ void __launch_bounds__(kThreads) k_router_decode(Weights W, Dims D, DecodeWs ws, const void* x, int n) {
+__global__ void __launch_bounds__(kRWarps * 32) k_router_decode(Weights W, Dims D, DecodeWs ws, const void* x, int n) {
+    griddep_launch();   // the gate/up grid may start its shared-expert work now
+    extern __shared__ __align__(16) float xs_r[];   // [n][H]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = blockIdx.x * kWarps + warp;
+    const int e = blockIdx.x * kRWarps + warp;
     const int H = D.H, E = D.E;
+    constexpr int B = 16;
+    const float* wr = W.W_r + (int64_t)(e < E ? e : 0) * H + 4 * lane;
+    uint4 w4[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b)   // first batch in flight while x is staged
+        if (b < H / 128) w4[b] = ld_stream_v4(wr + 128 * b);
+    for (int i = threadIdx.x * 4; i < n * H; i += kRWarps * 32 * 4)
+        *reinterpret_cast<float4*>(xs_r + i) = load_x4(x, D.act_bf16, i);
+    __syncthreads();
     if (e < E) {
         float acc[NT];
 #pragma unroll
         for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-        const float* wr = W.W_r + (int64_t)e * H + 4 * lane;
-#pragma unroll 4
-        for (int i = 0; i < H / 128; ++i) {
-            float4 w4 = __ldg(reinterpret_cast<const float4*>(wr + 128 * i));
+        for (int i0 = 0; i0 < H / 128; i0 += B) {
+            if (i0 > 0) {
 #pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                if (t < n) {
-                    float4 x4 = load_x4(x, D.act_bf16, (int64_t)t * H + 128 * i + 4 * lane);
-                    acc[t] = fmaf(x4.x, w4.x, acc[t]);
-                    acc[t] = fmaf(x4.y, w4.y, acc[t]);
-                    acc[t] = fmaf(x4.z, w4.z, acc[t]);
-                    acc[t] = fmaf(x4.w, w4.w, acc[t]);
+                for (int b = 0; b < B; ++b)
+                    if (i0 + b < H / 128) w4[b] = ld_stream_v4(wr + 128 * (i0 + b));
+            }
+#pragma unroll
+            for (int b = 0; b < B; ++b) {
+                if (i0 + b >= H / 128) break;
+                const float4 wv = make_float4(__uint_as_float(w4[b].x), __uint_as_float(w4[b].y),
+                                              __uint_as_float(w4[b].z), __uint_as_float(w4[b].w));
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    if (t < n) {
+                        const float4 x4 = *reinterpret_cast<const float4*>(xs_r + t * H + 128 * (i0 + b) + 4 * lane);
+                        acc[t] = fmaf(x4.x, wv.x, acc[t]);
+                        acc[t] = fmaf(x4.y, wv.y, acc[t]);
+                        acc[t] = fmaf(x4.z, wv.z, acc[t]);
+                        acc[t] = fmaf(x4.w, wv.w, acc[t]);
+                    }
                 }
             }
         }
@@ -101,32 +152,31 @@ __global__ void __launch_bounds__(kThreads) k_router_decode(Weights W, Dims D, D
             for (int m = 16; m >= 1; m >>= 1) acc[t] = acc[t] + __shfl_xor_sync(0xffffffffu, acc[t], m);
         }
         if (lane == 0) {
-            float b = W.b_r ? W.b_r[e] : 0.f;
+            const float b = W.b_r ? W.b_r[e] : 0.f;
 #pragma unroll
             for (int t = 0; t < NT; ++t)
                 if (t < n) ws.logits[(int64_t)t * E + e] = W.b_r ? acc[t] + b : acc[t];
         }
     }
     __shared__ bool s_last;
+    __shared__ float s_logits[kRWarps][1024];
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        unsigned prev = atomicAdd(ws.ticket, 1u);
+        const unsigned prev = atomicAdd(ws.ticket, 1u);
         s_last = (prev == gridDim.x - 1);
     }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    if (threadIdx.x == 0) {
-        *ws.ticket = 0;
-        *ws.queue1 = 0;
-    }
-    if (warp < n) topk_softmax_warp(ws.logits + (int64_t)warp * E, E, D.k, ws.ids + warp * D.k, ws.wts + warp * D.k);
+    if (threadIdx.x == 0) *ws.ticket = 0;
+    for (int t = warp; t < n; t += kRWarps)
+        topk_softmax_warp(ws.logits + (int64_t)t * E, s_logits[warp], E, D.k, ws.ids + t * D.k, ws.wts + t * D.k);
 }
 
 // ---------------------------------------------------------------- routing table
 // Unique selected experts in ascending order, and for each the slots
-// (t * k + j) that chose it, in increasing slot order.
+// (t * k + j) that chose it, in increasing slot order.  Built by one warp.
 struct Routing {
     int nu;
     int uniq[kMaxSlots];
@@ -134,81 +184,173 @@ struct Routing {
     int slot[kMaxSlots];
     int ids[kMaxSlots];
     int first[kMaxSlots];
+    int rank[kMaxSlots];
+    int pos[kMaxSlots];
 };
 
-__device__ void build_routing(Routing& R, const int32_t* ids, int nk) {
-    int tid = threadIdx.x;
-    if (tid < nk) R.ids[tid] = __ldcg(ids + tid);
-    __syncthreads();
-    int e = 0, pos = 0, first = 0;
-    if (tid < nk) {
-        e = R.ids[tid];
-        first = 1;
-        for (int s = 0; s < tid; ++s)
-            if (R.ids[s] == e) { first = 0; ++pos; }
-        R.first[tid] = first;
+__device__ void build_routing_warp(Routing& R, const int32_t* ids, int nk) {
+    const int lane = threadIdx.x & 31;
+    for (int s = lane; s < nk; s += 32) R.ids[s] = __ldcg(ids + s);
+    __syncwarp();
+    for (int s = lane; s < nk; s += 32) {
+        const int e = R.ids[s];
+        int first = 1, pos = 0;
+        for (int q = 0; q < s; ++q)
+            if (R.ids[q] == e) { first = 0; ++pos; }
+        R.first[s] = first;
+        R.pos[s] = pos;
     }
-    __syncthreads();
-    int rank = 0;
-    if (tid < nk) {
-        for (int s = 0; s < nk; ++s)
-            if (R.first[s] && R.ids[s] < e) ++rank;
+    __syncwarp();
+    for (int s = lane; s < nk; s += 32) {
+        const int e = R.ids[s];
+        int rank = 0, cnt = 0;
+        for (int q = 0; q < nk; ++q) {
+            rank += (R.first[q] && R.ids[q] < e);
+            cnt += R.ids[q] == e;
+        }
+        R.rank[s] = rank;
+        if (R.first[s]) {
+            R.uniq[rank] = e;
+            R.ustart[rank + 1] = cnt;
+        }
     }
-    if (tid < nk && first) {
-        int cnt = 0;
-        for (int s = 0; s < nk; ++s) cnt += R.ids[s] == e;
-        R.uniq[rank] = e;
-        R.ustart[rank + 1] = cnt;   // counts; prefix below
-    }
-    __syncthreads();
-    if (tid == 0) {
+    __syncwarp();
+    if (lane == 0) {
         int nu = 0;
         for (int s = 0; s < nk; ++s) nu += R.first[s];
         R.nu = nu;
         R.ustart[0] = 0;
         for (int u = 0; u < nu; ++u) R.ustart[u + 1] += R.ustart[u];
     }
-    __syncthreads();
-    if (tid < nk) R.slot[R.ustart[rank] + pos] = tid;
-    __syncthreads();
+    __syncwarp();
+    for (int s = lane; s < nk; s += 32) R.slot[R.ustart[R.rank[s]] + R.pos[s]] = s;
+    __syncwarp();
 }
 
-// ---------------------------------------------------------------- gate/up
-// IQ2 group of 32 weights (4 chunks of 8) against NT token vectors.
-template <int NT>
-__device__ __forceinline__ void iq2_group(uint32_t idx, uint32_t S, float d, const float* __restrict__ tabp,
-                                          const float* __restrict__ xcol, int H, const int* tok, int ns,
-                                          float* acc) {
-    float2 gs[NT];
+// ---------------------------------------------------------------- pipeline state
+struct ChunkInfo {
+    int task;      // -1: no more work
+    int chunk;     // chunk index within the task
+    int nchunk;    // chunks of the task
+    int lo, cnt;   // first k step of the chunk and how many
+};
+
+struct Pipe {
+    uint64_t full[4];
+    uint64_t empty[4];
+    uint64_t cons;        // barrier of the consumer warps (task epilogues)
+    ChunkInfo info[4];
+    int abort;            // set after a timed-out wait: every loop leaves
+};
+
+__device__ void pipe_init(Pipe& P, int NS, int CW) {
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&P.full[s], 1);
+            mbar_init(&P.empty[s], CW);
+        }
+        mbar_init(&P.cons, CW);
+        P.abort = 0;
+        fence_barrier_init();
+    }
+}
+
+__device__ __forceinline__ bool aborted(const Pipe& P) { return *(volatile const int*)&P.abort != 0; }
+__device__ __forceinline__ void set_abort(Pipe& P) { *(volatile int*)&P.abort = 1; }
+
+// Bounded barrier of the consumer warps (instead of bar.sync, which
+// cannot time out).  Returns false after a timeout.
+__device__ __forceinline__ bool cons_sync(Pipe& P, uint32_t& phase, uint32_t* err) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&P.cons);
+    const bool ok = mbar_wait(&P.cons, phase, err);
+    phase ^= 1u;
+    if (!ok) set_abort(P);
+    return ok;
+}
+
+// Producer: wait until the last NS issued copies have landed (bounded), then
+// publish the stop marker.  Leaves no bulk copy in flight.
+__device__ void producer_finish(Pipe& P, uint32_t it, int NS, uint32_t* err) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t j0 = it > (uint32_t)NS ? it - NS : 0;
+    for (uint32_t j = j0; j < it; ++j) mbar_wait(&P.full[j % NS], (j / NS) & 1, err);
+    const int s = it % NS;
+    if (!aborted(P)) {
+        if (!mbar_wait(&P.empty[s], ((it / NS) & 1) ^ 1, err)) set_abort(P);
+    }
+    if (lane == 0) {
+        P.info[s].task = -1;
+        mbar_arrive(&P.full[s]);
+    }
+    __syncwarp();
+}
+
+// ---------------------------------------------------------------- IQ2 groups
+// The eight signed grid magnitudes of one IQ2 chunk (grid row a, 7 sign bits
+// + parity taken from S), as binary32.  tabp: this lane's grid replica.
+template <int TR>
+__device__ __forceinline__ void iq2_chunk(uint32_t idx, uint32_t S, int c, const float* __restrict__ tabp,
+                                          float* w) {
+    const uint32_t a = (idx >> (8 * c)) & 255u;
+    uint32_t sg = (S >> (7 * c)) & 127u;
+    sg |= ((uint32_t)__popc(sg) & 1u) << 7;
+    const float* trow = tabp + a * (8 * TR);
+    const float4 g0 = *reinterpret_cast<const float4*>(trow);
+    const float4 g1 = *reinterpret_cast<const float4*>(trow + 4 * TR);
+    w[0] = g0.x; w[1] = g0.y; w[2] = g0.z; w[3] = g0.w;
+    w[4] = g1.x; w[5] = g1.y; w[6] = g1.z; w[7] = g1.w;
 #pragma unroll
-    for (int t = 0; t < NT; ++t) gs[t] = make_float2(0.f, 0.f);
+    for (int i = 0; i < 8; ++i) w[i] = __uint_as_float(__float_as_uint(w[i]) ^ ((sg << (31 - i)) & 0x80000000u));
+}
+
+// d * (2s + 1) / 8 for the group scale s in bits 28..31 of S (no int->float
+// conversion unit: 2s+1 < 2^23 is placed under exponent 2^23 and the bias
+// subtracted exactly).
+__device__ __forceinline__ float iq2_scale(uint32_t S, float d) {
+    const float odd = __uint_as_float(0x4b000001u | ((S >> 27) & 0x1eu)) - 8388608.0f;
+    return d * odd * 0.125f;
+}
+
+// A gate group and the up group at the same columns (32 weights each) against
+// NT token vectors; the token values are read once for both.
+template <int NT, int TR>
+__device__ __forceinline__ void iq2_group_pair(uint4 pg, uint4 pu, int half, float dg, float du,
+                                               const float* __restrict__ tabp, const float* __restrict__ xcol,
+                                               int H, const int* tok, int ns, float* ag, float* au) {
+    const uint32_t gi = half ? pg.z : pg.x, gS = half ? pg.w : pg.y;
+    const uint32_t ui = half ? pu.z : pu.x, uS = half ? pu.w : pu.y;
+    float2 gs[NT], us[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) gs[t] = us[t] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        uint32_t a = (idx >> (8 * c)) & 255u;
-        uint32_t sg = (S >> (7 * c)) & 127u;
-        sg |= ((uint32_t)__popc(sg) & 1u) << 7;
-        const float* trow = tabp + a * 64;
-        float4 g0 = *reinterpret_cast<const float4*>(trow);
-        float4 g1 = *reinterpret_cast<const float4*>(trow + 32);
-        float w[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) w[i] = __uint_as_float(__float_as_uint(w[i]) ^ ((sg << (31 - i)) & 0x80000000u));
+        float wg[8], wu[8];
+        iq2_chunk<TR>(gi, gS, c, tabp, wg);
+        iq2_chunk<TR>(ui, uS, c, tabp, wu);
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
             if (t < ns) {
                 const float* xr = xcol + tok[t] * H + 8 * c;
-                float4 x0 = *reinterpret_cast<const float4*>(xr);
-                float4 x1 = *reinterpret_cast<const float4*>(xr + 4);
-                gs[t] = ffma2(make_float2(w[0], w[1]), make_float2(x0.x, x0.y), gs[t]);
-                gs[t] = ffma2(make_float2(w[2], w[3]), make_float2(x0.z, x0.w), gs[t]);
-                gs[t] = ffma2(make_float2(w[4], w[5]), make_float2(x1.x, x1.y), gs[t]);
-                gs[t] = ffma2(make_float2(w[6], w[7]), make_float2(x1.z, x1.w), gs[t]);
+                const float4 x0 = *reinterpret_cast<const float4*>(xr);
+                const float4 x1 = *reinterpret_cast<const float4*>(xr + 4);
+                gs[t] = ffma2(make_float2(wg[0], wg[1]), make_float2(x0.x, x0.y), gs[t]);
+                us[t] = ffma2(make_float2(wu[0], wu[1]), make_float2(x0.x, x0.y), us[t]);
+                gs[t] = ffma2(make_float2(wg[2], wg[3]), make_float2(x0.z, x0.w), gs[t]);
+                us[t] = ffma2(make_float2(wu[2], wu[3]), make_float2(x0.z, x0.w), us[t]);
+                gs[t] = ffma2(make_float2(wg[4], wg[5]), make_float2(x1.x, x1.y), gs[t]);
+                us[t] = ffma2(make_float2(wu[4], wu[5]), make_float2(x1.x, x1.y), us[t]);
+                gs[t] = ffma2(make_float2(wg[6], wg[7]), make_float2(x1.z, x1.w), gs[t]);
+                us[t] = ffma2(make_float2(wu[6], wu[7]), make_float2(x1.z, x1.w), us[t]);
             }
         }
     }
-    float db = d * (float)(2 * (S >> 28) + 1) * 0.125f;
+    const float sgate = iq2_scale(gS, dg), sup = iq2_scale(uS, du);
 #pragma unroll
-    for (int t = 0; t < NT; ++t) acc[t] = fmaf(db, gs[t].x + gs[t].y, acc[t]);
+    for (int t = 0; t < NT; ++t) {
+        ag[t] = fmaf(sgate, gs[t].x + gs[t].y, ag[t]);
+        au[t] = fmaf(sup, us[t].x + us[t].y, au[t]);
+    }
 }
 
 // bf16x2 word -> two binary32 values, multiply-accumulated against x pairs.
@@ -216,169 +358,243 @@ __device__ __forceinline__ float2 bf16x2_fma(uint32_t wbits, float2 x, float2 ac
     return ffma2(make_float2(__uint_as_float(wbits << 16), __uint_as_float(wbits & 0xffff0000u)), x, acc);
 }
 
+__device__ __forceinline__ void bf16x8_dot(uint4 w, const float* xr, float2& acc) {
+    const float4 x0 = *reinterpret_cast<const float4*>(xr);
+    const float4 x1 = *reinterpret_cast<const float4*>(xr + 4);
+    acc = bf16x2_fma(w.x, make_float2(x0.x, x0.y), acc);
+    acc = bf16x2_fma(w.y, make_float2(x0.z, x0.w), acc);
+    acc = bf16x2_fma(w.z, make_float2(x1.x, x1.y), acc);
+    acc = bf16x2_fma(w.w, make_float2(x1.z, x1.w), acc);
+}
+
+// ---------------------------------------------------------------- gate/up
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1)
+struct GateUpCfg {
+    static constexpr int TR = NT <= 2 ? 8 : 1;            // grid replicas
+    static constexpr int NS = NT <= 4 ? 3 : 2;            // stages
+    static constexpr int kTabFloats = 256 * 8 * TR;
+    static constexpr int CW = Warps<NT>::CW;
+    static constexpr int kRedFloats = CW * 2 * NT * 32;
+};
+
+template <int NT>
+__global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
     k_gateup_decode(Weights W, Dims D, DecodeWs ws, const void* x, int n) {
-    extern __shared__ __align__(16) float smem[];
-    float* tab = smem;                      // kTabFloats
-    float* xs = tab + kTabFloats;           // [n][H]
-    float* red = xs + n * D.H;              // [kWarps][2][NT][32]
+    using C = GateUpCfg<NT>;
+    constexpr int NS = C::NS, TR = C::TR, CW = C::CW, kGThreads = Warps<NT>::kThreads;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char* stages = smem_raw;                                   // NS x kStageBytes
+    float* tab = reinterpret_cast<float*>(smem_raw + NS * kStageBytes);  // kTabFloats
+    float* red = tab + C::kTabFloats;                                   // kRedFloats
+    float* xs = red + C::kRedFloats;                                    // [n][H]
+    __shared__ Pipe P;
     __shared__ Routing R;
-    __shared__ int s_task;
+    __shared__ int s_last;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = D.H, I = D.I, k = D.k;
-    if (blockIdx.x == 0 && tid == 0) *ws.queue2 = 0;
-
-    for (int i = tid; i < kTabFloats; i += kThreads) {
-        int a = i >> 6, hf = (i >> 5) & 1, j = i & 3;
-        tab[i] = (float)W.grid_u8[a * 8 + hf * 4 + j];
-    }
-    for (int i = tid * 4; i < n * H; i += kThreads * 4) *reinterpret_cast<float4*>(xs + i) = load_x4(x, D.act_bf16, i);
-    build_routing(R, ws.ids, n * k);   // syncs
-
+    const int nkt = H / 64, nsb = H / 256;
     const int n_sh = D.has_shared ? I / 8 : 0;
     const int rb_per_e = I / 32;
-    const int total = n_sh + R.nu * rb_per_e;
-    const float* tabp = tab + (lane & 7) * 4;
-    const int nkt = H / 64, nsb = H / 256;
+    const int ck_rt = nkt < 32 ? nkt : 32;            // k steps (64 columns) per routed chunk
+    const int nch_rt = nkt / ck_rt;
+    const int ck_sh = H / 8 < 128 ? H / 8 : 128;      // 8-column tiles per shared chunk
+    const int nch_sh = (H / 8) / ck_sh;
 
-    for (;;) {
-        if (tid == 0) s_task = atomicAdd(ws.queue1, 1u);
-        __syncthreads();
-        const int task = s_task;
-        if (task >= total) break;
-        if (task < n_sh) {
-            // shared expert rows 8*task .. +7; lane = (row, k-quarter)
-            const int rr = lane & 7, kq = lane >> 3;
-            const int64_t tile0 = (int64_t)task * (H / 8);
-            float2 ag[NT], au[NT];
+    pipe_init(P, NS, CW);
+    // grid: one 32-bit load per 4 magnitudes, expanded to TR interleaved copies
+    for (int q = tid; q < 512; q += kGThreads) {
+        const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(W.grid_u8) + q);
+        const int a = q >> 1, hf = q & 1;
+        const float4 f = make_float4((float)(v & 0xffu), (float)((v >> 8) & 0xffu), (float)((v >> 16) & 0xffu),
+                                     (float)(v >> 24));
 #pragma unroll
-            for (int t = 0; t < NT; ++t) ag[t] = au[t] = make_float2(0.f, 0.f);
-            constexpr int KB = 8;
-            for (int kc0 = warp * 4 + kq; kc0 < H / 8; kc0 += 32 * KB) {
-                uint4 wg[KB], wu[KB];
-#pragma unroll
-                for (int b = 0; b < KB; ++b) {
-                    const int kc = kc0 + 32 * b;
-                    if (kc < H / 8) {
-                        wg[b] = ld_stream_v4(W.sh_gate + ((tile0 + kc) * 8 + rr) * 8);
-                        wu[b] = ld_stream_v4(W.sh_up + ((tile0 + kc) * 8 + rr) * 8);
+        for (int p = 0; p < TR; ++p) *reinterpret_cast<float4*>(tab + a * (8 * TR) + hf * (4 * TR) + p * 4) = f;
+    }
+    for (int i = tid * 4; i < n * H; i += kGThreads * 4) *reinterpret_cast<float4*>(xs + i) = load_x4(x, D.act_bf16, i);
+    __syncthreads();
+
+    if (warp == CW) {
+        // ------------------------------------------------ producer warp
+        const uint64_t pol = policy_evict_first();
+        uint32_t it = 0;
+        bool routed = false;
+        int total = 0x7fffffff;
+        int next = 0;
+        if (lane == 0) next = (int)atomicAdd(ws.queue1, 1u);
+        for (;;) {
+            if (aborted(P)) break;
+            int task = __shfl_sync(0xffffffffu, next, 0);
+            if (lane == 0) next = (int)atomicAdd(ws.queue1, 1u);   // in flight while this task streams
+            if (task >= n_sh && !routed) {
+                griddep_wait();                   // router results visible
+                build_routing_warp(R, ws.ids, n * k);
+                routed = true;
+                total = n_sh + R.nu * rb_per_e;
+                griddep_launch();                 // the down grid may start streaming
+            }
+            if (task >= total) break;
+            const bool sh = task < n_sh;
+            const int nch = sh ? nch_sh : nch_rt;
+            for (int c = 0; c < nch; ++c) {
+                const int s = it % NS;
+                const uint32_t ph = (it / NS) & 1;
+                if (!mbar_wait(&P.empty[s], ph ^ 1, ws.err)) { set_abort(P); break; }
+                if (lane == 0) {
+                    unsigned char* st = stages + s * kStageBytes;
+                    if (sh) {
+                        const int kc0 = c * ck_sh;
+                        const size_t off = ((size_t)task * (H / 8) + kc0) * 64;   // elements
+                        const uint32_t bytes = ck_sh * 128;
+                        P.info[s] = ChunkInfo{task, c, nch, kc0, ck_sh};
+                        mbar_arrive_expect_tx(&P.full[s], 2 * bytes);
+                        bulk_load(st, W.sh_gate + off, bytes, &P.full[s], pol);
+                        bulk_load(st + bytes, W.sh_up + off, bytes, &P.full[s], pol);
+                    } else {
+                        const int tt = task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
+                        const int e = R.uniq[u];
+                        const int kt0 = c * ck_rt;
+                        const uint32_t pb = ck_rt * 512, db = ck_rt * 16;
+                        const size_t qoff = (size_t)e * W.iq2_qs_stride + ((size_t)rb * nkt + kt0) * 512;
+                        const size_t doff = (size_t)e * W.iq2_d_stride + ((size_t)rb * nsb + kt0 / 4) * 32;
+                        P.info[s] = ChunkInfo{task, c, nch, kt0, ck_rt};
+                        mbar_arrive_expect_tx(&P.full[s], 2 * pb + 2 * db);
+                        bulk_load(st, W.gate_qs + qoff, pb, &P.full[s], pol);
+                        bulk_load(st + pb, W.up_qs + qoff, pb, &P.full[s], pol);
+                        bulk_load(st + 2 * pb, W.gate_d + doff, db, &P.full[s], pol);
+                        bulk_load(st + 2 * pb + db, W.up_d + doff, db, &P.full[s], pol);
                     }
                 }
+                __syncwarp();
+                ++it;
+            }
+        }
+        producer_finish(P, it, NS, ws.err);
+    } else {
+        // ------------------------------------------------ consumer warps
+        const float* tabp = tab + (lane & (TR - 1)) * 4;
+        uint32_t it = 0, cph = 0;
+        float2 sg2[NT], su2[NT];     // shared-task partials (this lane's row, k quarter)
+        float ag[NT], au[NT];        // routed-task partials (this lane's row)
+        int tok[NT];
+        for (;;) {
+            const int s = it % NS;
+            if (!mbar_wait(&P.full[s], (it / NS) & 1, ws.err)) { set_abort(P); break; }
+            const ChunkInfo inf = P.info[s];
+            if (inf.task < 0 || aborted(P)) break;
+            const unsigned char* st = stages + s * kStageBytes;
+            const bool sh = inf.task < n_sh;
+            if (sh) {
+                const int rr = lane & 7, kq = lane >> 3;
+                if (inf.chunk == 0) {
 #pragma unroll
-                for (int b = 0; b < KB; ++b) {
-                    const int kc = kc0 + 32 * b;
-                    if (kc >= H / 8) break;
+                    for (int t = 0; t < NT; ++t) sg2[t] = su2[t] = make_float2(0.f, 0.f);
+                }
+                const uint4* gt = reinterpret_cast<const uint4*>(st);
+                const uint4* ut = reinterpret_cast<const uint4*>(st + inf.cnt * 128);
+                for (int kc = warp * 4 + kq; kc < inf.cnt; kc += 4 * CW) {
+                    const uint4 wg = gt[kc * 8 + rr], wu = ut[kc * 8 + rr];
+                    const int col = 8 * (inf.lo + kc);
 #pragma unroll
                     for (int t = 0; t < NT; ++t) {
                         if (t < n) {
-                            const float* xr = xs + t * H + 8 * kc;
-                            float4 x0 = *reinterpret_cast<const float4*>(xr);
-                            float4 x1 = *reinterpret_cast<const float4*>(xr + 4);
-                            ag[t] = bf16x2_fma(wg[b].x, make_float2(x0.x, x0.y), ag[t]);
-                            ag[t] = bf16x2_fma(wg[b].y, make_float2(x0.z, x0.w), ag[t]);
-                            ag[t] = bf16x2_fma(wg[b].z, make_float2(x1.x, x1.y), ag[t]);
-                            ag[t] = bf16x2_fma(wg[b].w, make_float2(x1.z, x1.w), ag[t]);
-                            au[t] = bf16x2_fma(wu[b].x, make_float2(x0.x, x0.y), au[t]);
-                            au[t] = bf16x2_fma(wu[b].y, make_float2(x0.z, x0.w), au[t]);
-                            au[t] = bf16x2_fma(wu[b].z, make_float2(x1.x, x1.y), au[t]);
-                            au[t] = bf16x2_fma(wu[b].w, make_float2(x1.z, x1.w), au[t]);
+                            bf16x8_dot(wg, xs + t * H + col, sg2[t]);
+                            bf16x8_dot(wu, xs + t * H + col, su2[t]);
                         }
                     }
                 }
-            }
+            } else {
+                const int tt = inf.task - n_sh, u = tt / rb_per_e;
+                const int s0 = R.ustart[u], ns = R.ustart[u + 1] - s0;
+                if (inf.chunk == 0) {
 #pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                float g = ag[t].x + ag[t].y, u = au[t].x + au[t].y;
-                g += __shfl_xor_sync(0xffffffffu, g, 8);
-                g += __shfl_xor_sync(0xffffffffu, g, 16);
-                u += __shfl_xor_sync(0xffffffffu, u, 8);
-                u += __shfl_xor_sync(0xffffffffu, u, 16);
-                if (kq == 0 && t < n) {
-                    red[((warp * 2 + 0) * NT + t) * 32 + rr] = g;
-                    red[((warp * 2 + 1) * NT + t) * 32 + rr] = u;
-                }
-            }
-            __syncthreads();
-            if (tid < 8 * n) {
-                const int r = tid & 7, t = tid >> 3;
-                float g = 0.f, u = 0.f;
-                for (int w = 0; w < kWarps; ++w) {
-                    g += red[((w * 2 + 0) * NT + t) * 32 + r];
-                    u += red[((w * 2 + 1) * NT + t) * 32 + r];
-                }
-                ws.h_sh[(int64_t)t * I + 8 * task + r] = silu(g) * u;
-            }
-        } else {
-            // routed expert uniq[u], rows 32*rb + lane
-            const int tt = task - n_sh;
-            const int u = tt / rb_per_e, rb = tt % rb_per_e;
-            const int e = R.uniq[u];
-            const int s0 = R.ustart[u], ns = R.ustart[u + 1] - s0;
-            int tok[NT];
-#pragma unroll
-            for (int t = 0; t < NT; ++t) tok[t] = t < ns ? R.slot[s0 + t] / k : 0;
-            float ag[NT], au[NT];
-#pragma unroll
-            for (int t = 0; t < NT; ++t) ag[t] = au[t] = 0.f;
-            const uint8_t* gq = W.gate_qs + (int64_t)e * W.iq2_qs_stride + ((int64_t)rb * nkt * 32 + lane) * 16;
-            const uint8_t* uq = W.up_qs + (int64_t)e * W.iq2_qs_stride + ((int64_t)rb * nkt * 32 + lane) * 16;
-            const uint16_t* gd = W.gate_d + (int64_t)e * W.iq2_d_stride + (int64_t)rb * nsb * 32 + lane;
-            const uint16_t* ud = W.up_d + (int64_t)e * W.iq2_d_stride + (int64_t)rb * nsb * 32 + lane;
-            constexpr int KB = 8;
-            for (int kt0 = warp * KB; kt0 < nkt; kt0 += kWarps * KB) {
-                uint4 pg[KB], pu[KB];
-                float dg[KB / 4], du[KB / 4];
-#pragma unroll
-                for (int b = 0; b < KB; ++b) {
-                    if (kt0 + b < nkt) {
-                        pg[b] = ld_stream_v4(gq + (int64_t)(kt0 + b) * 512);
-                        pu[b] = ld_stream_v4(uq + (int64_t)(kt0 + b) * 512);
+                    for (int t = 0; t < NT; ++t) {
+                        ag[t] = au[t] = 0.f;
+                        tok[t] = t < ns ? R.slot[s0 + t] / k : 0;
                     }
                 }
+                const uint4* gp = reinterpret_cast<const uint4*>(st);
+                const uint4* up = reinterpret_cast<const uint4*>(st + inf.cnt * 512);
+                const uint16_t* gd = reinterpret_cast<const uint16_t*>(st + 2 * inf.cnt * 512);
+                const uint16_t* ud = gd + inf.cnt * 8;
+                for (int kt = warp; kt < inf.cnt; kt += CW) {
+                    const uint4 pg = gp[kt * 32 + lane], pu = up[kt * 32 + lane];
+                    const float dg = half_bits(gd[(kt >> 2) * 32 + lane]);
+                    const float du = half_bits(ud[(kt >> 2) * 32 + lane]);
+                    const float* xcol = xs + 64 * (inf.lo + kt);
+                    iq2_group_pair<NT, TR>(pg, pu, 0, dg, du, tabp, xcol, H, tok, ns, ag, au);
+                    iq2_group_pair<NT, TR>(pg, pu, 1, dg, du, tabp, xcol + 32, H, tok, ns, ag, au);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&P.empty[s]);
+            if (inf.chunk == inf.nchunk - 1) {
+                // task epilogue: reduce the eight warps' partials, SwiGLU, store h
+                if (sh) {
+                    const int rr = lane & 7, kq = lane >> 3;
 #pragma unroll
-                for (int b = 0; b < KB / 4; ++b) {
-                    if (kt0 + 4 * b < nkt) {
-                        dg[b] = half_bits(ld_stream_u16(gd + ((kt0 >> 2) + b) * 32));
-                        du[b] = half_bits(ld_stream_u16(ud + ((kt0 >> 2) + b) * 32));
+                    for (int t = 0; t < NT; ++t) {
+                        float g = sg2[t].x + sg2[t].y, uu = su2[t].x + su2[t].y;
+                        g += __shfl_xor_sync(0xffffffffu, g, 8);
+                        g += __shfl_xor_sync(0xffffffffu, g, 16);
+                        uu += __shfl_xor_sync(0xffffffffu, uu, 8);
+                        uu += __shfl_xor_sync(0xffffffffu, uu, 16);
+                        if (kq == 0 && t < n) {
+                            red[((warp * 2 + 0) * NT + t) * 32 + rr] = g;
+                            red[((warp * 2 + 1) * NT + t) * 32 + rr] = uu;
+                        }
+                    }
+                    if (!cons_sync(P, cph, ws.err)) break;
+                    if (tid < 8 * n) {
+                        const int r = tid & 7, t = tid >> 3;
+                        float g = 0.f, uu = 0.f;
+                        for (int w = 0; w < CW; ++w) {
+                            g += red[((w * 2 + 0) * NT + t) * 32 + r];
+                            uu += red[((w * 2 + 1) * NT + t) * 32 + r];
+                        }
+                        ws.h_sh[(int64_t)t * I + 8 * inf.task + r] = silu(g) * uu;
+                    }
+                } else {
+                    const int tt = inf.task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
+                    const int s0 = R.ustart[u], ns = R.ustart[u + 1] - s0;
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        if (t < ns) {
+                            red[((warp * 2 + 0) * NT + t) * 32 + lane] = ag[t];
+                            red[((warp * 2 + 1) * NT + t) * 32 + lane] = au[t];
+                        }
+                    }
+                    if (!cons_sync(P, cph, ws.err)) break;
+                    if (warp < ns) {
+                        const int t = warp;
+                        float g = 0.f, uu = 0.f;
+                        for (int w = 0; w < CW; ++w) {
+                            g += red[((w * 2 + 0) * NT + t) * 32 + lane];
+                            uu += red[((w * 2 + 1) * NT + t) * 32 + lane];
+                        }
+                        const float h = silu(g) * uu;
+                        const int slot = R.slot[s0 + t];
+                        ws.h_rt[(int64_t)slot * I + 32 * rb + lane] = h;
+                        float hs = h;
+#pragma unroll
+                        for (int m = 1; m <= 8; m <<= 1) hs += __shfl_xor_sync(0xffffffffu, hs, m);
+                        if ((lane & 15) == 0) ws.hsum_rt[(int64_t)slot * (I / 16) + 2 * rb + (lane >> 4)] = hs;
                     }
                 }
-#pragma unroll
-                for (int b = 0; b < KB; ++b) {
-                    const int kt = kt0 + b;
-                    if (kt >= nkt) break;
-                    const float* xcol = xs + 64 * kt;
-                    iq2_group<NT>(pg[b].x, pg[b].y, dg[b >> 2], tabp, xcol, H, tok, ns, ag);
-                    iq2_group<NT>(pg[b].z, pg[b].w, dg[b >> 2], tabp, xcol + 32, H, tok, ns, ag);
-                    iq2_group<NT>(pu[b].x, pu[b].y, du[b >> 2], tabp, xcol, H, tok, ns, au);
-                    iq2_group<NT>(pu[b].z, pu[b].w, du[b >> 2], tabp, xcol + 32, H, tok, ns, au);
-                }
+                if (!cons_sync(P, cph, ws.err)) break;
             }
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                if (t < ns) {
-                    red[((warp * 2 + 0) * NT + t) * 32 + lane] = ag[t];
-                    red[((warp * 2 + 1) * NT + t) * 32 + lane] = au[t];
-                }
-            }
-            __syncthreads();
-            if (warp < ns) {
-                const int t = warp;
-                float g = 0.f, uu = 0.f;
-                for (int w = 0; w < kWarps; ++w) {
-                    g += red[((w * 2 + 0) * NT + t) * 32 + lane];
-                    uu += red[((w * 2 + 1) * NT + t) * 32 + lane];
-                }
-                float h = silu(g) * uu;
-                const int slot = R.slot[s0 + t];
-                ws.h_rt[(int64_t)slot * I + 32 * rb + lane] = h;
-                float hs = h;
-#pragma unroll
-                for (int m = 1; m <= 8; m <<= 1) hs += __shfl_xor_sync(0xffffffffu, hs, m);
-                if ((lane & 15) == 0) ws.hsum_rt[(int64_t)slot * (I / 16) + 2 * rb + (lane >> 4)] = hs;
-            }
+            ++it;
         }
-        __syncthreads();
+    }
+    griddep_launch();
+    // last CTA to leave resets the task queue for the next forward
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        s_last = atomicAdd(ws.done1, 1u) == gridDim.x - 1;
+        if (s_last) {
+            *ws.queue1 = 0;
+            *ws.done1 = 0;
+        }
     }
 }
 
@@ -386,11 +602,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // sum_i (1 + q_i/4) h_i over the 16 codes of one 32-bit word, against NT slots.
 template <int NT>
 __device__ __forceinline__ void q2_word(uint32_t word, const float* const* hp, int ns, float* A) {
-    uint32_t t0 = ((word << 5) & 0x60606060u) | 0x80808080u;
-    uint32_t t1 = ((word << 3) & 0x60606060u) | 0x80808080u;
-    uint32_t t2 = ((word << 1) & 0x60606060u) | 0x80808080u;
-    uint32_t t3 = ((word >> 1) & 0x60606060u) | 0x80808080u;
-    // byte j of t_k holds code 4j + k at bits 5..6 (over a set bit 7)
+    const uint32_t t0 = ((word << 5) & 0x60606060u) | 0x80808080u;
+    const uint32_t t1 = ((word << 3) & 0x60606060u) | 0x80808080u;
+    const uint32_t t2 = ((word << 1) & 0x60606060u) | 0x80808080u;
+    const uint32_t t3 = ((word >> 1) & 0x60606060u) | 0x80808080u;
+    // byte j of t_k holds code 4j + k at bits 5..6 (over a set bit 7); a byte
+    // permute puts it under exponent 0x3f8: the binary32 value 1 + code/4
     float f[16];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -406,7 +623,7 @@ __device__ __forceinline__ void q2_word(uint32_t word, const float* const* hp, i
             float2 a = make_float2(0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < 16; i += 4) {
-                float4 hv = *reinterpret_cast<const float4*>(hp[t] + i);
+                const float4 hv = *reinterpret_cast<const float4*>(hp[t] + i);
                 a = ffma2(make_float2(f[i], f[i + 1]), make_float2(hv.x, hv.y), a);
                 a = ffma2(make_float2(f[i + 2], f[i + 3]), make_float2(hv.z, hv.w), a);
             }
@@ -416,235 +633,379 @@ __device__ __forceinline__ void q2_word(uint32_t word, const float* const* hp, i
 }
 
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1)
-    k_down_decode(Weights W, Dims D, DecodeWs ws, int n) {
-    extern __shared__ __align__(16) float smem[];
-    float* hsh = smem;                      // [n][I] shared-expert h
-    float* red = hsh + n * D.I;             // [kWarps][NT][32]
+struct DownCfg {
+    static constexpr int NS = 4;
+    static constexpr int CW = Warps<NT>::CW;
+    static constexpr int kRedFloats = CW * NT * 32;
+};
+
+// k steps (64 columns) per routed down chunk for an expert chosen by ns
+// slots: codes, scales, (d, dmin) and the slots' h (and per-16 sums of h)
+// for those columns must fit one stage.
+__device__ __forceinline__ int down_chunk_ksteps(int nkt, int nsb, int ns) {
+    int ck = nkt < 32 ? nkt : 32;
+    for (; ck > 1; ck >>= 1) {
+        const int nsbc = nsb > 1 ? (ck + 3) / 4 : 1;
+        if (ck * 640 + nsbc * 128 + ns * ck * 272 <= kStageBytes) break;
+    }
+    return ck;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
+    k_down_decode(Weights W, Dims D, DecodeWs ws, float* out, int n) {
+    using C = DownCfg<NT>;
+    constexpr int NS = C::NS, CW = C::CW;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char* stages = smem_raw;
+    float* red = reinterpret_cast<float*>(smem_raw + NS * kStageBytes);   // kRedFloats
+    float* hsh = red + C::kRedFloats;                                     // [n][I]
+    __shared__ Pipe P;
     __shared__ Routing R;
-    __shared__ int s_task;
+    __shared__ int s_last;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = D.H, I = D.I, k = D.k;
-
-    if (D.has_shared)
-        for (int i = tid * 4; i < n * I; i += kThreads * 4)
-            *reinterpret_cast<float4*>(hsh + i) = __ldcg(reinterpret_cast<const float4*>(ws.h_sh + i));
-    build_routing(R, ws.ids, n * k);
-
+    const int nkt = I / 64, nsb = I >= 256 ? I / 256 : 1;
     const int n_sh = D.has_shared ? H / 8 : 0;
     const int rb_per_e = H / 32;
-    const int total = n_sh + R.nu * rb_per_e;
-    const int nkt = I / 64, nsb = I >= 256 ? I / 256 : 1;
+    const int ck_sh = I / 8 < 256 ? I / 8 : 256;
+    const int nch_sh = (I / 8) / ck_sh;
 
-    for (;;) {
-        if (tid == 0) s_task = atomicAdd(ws.queue2, 1u);
-        __syncthreads();
-        const int task = s_task;
-        if (task >= total) break;
-        if (task < n_sh) {
-            const int rr = lane & 7, kq = lane >> 3;
-            const int64_t tile0 = (int64_t)task * (I / 8);
-            float2 ay[NT];
-#pragma unroll
-            for (int t = 0; t < NT; ++t) ay[t] = make_float2(0.f, 0.f);
-            constexpr int KB = 8;
-            for (int kc0 = warp * 4 + kq; kc0 < I / 8; kc0 += 32 * KB) {
-                uint4 wd[KB];
-#pragma unroll
-                for (int b = 0; b < KB; ++b)
-                    if (kc0 + 32 * b < I / 8) wd[b] = ld_stream_v4(W.sh_down + ((tile0 + kc0 + 32 * b) * 8 + rr) * 8);
-#pragma unroll
-                for (int b = 0; b < KB; ++b) {
-                    const int kc = kc0 + 32 * b;
-                    if (kc >= I / 8) break;
-#pragma unroll
-                    for (int t = 0; t < NT; ++t) {
-                        if (t < n) {
-                            const float* hr = hsh + t * I + 8 * kc;
-                            float4 h0 = *reinterpret_cast<const float4*>(hr);
-                            float4 h1 = *reinterpret_cast<const float4*>(hr + 4);
-                            ay[t] = bf16x2_fma(wd[b].x, make_float2(h0.x, h0.y), ay[t]);
-                            ay[t] = bf16x2_fma(wd[b].y, make_float2(h0.z, h0.w), ay[t]);
-                            ay[t] = bf16x2_fma(wd[b].z, make_float2(h1.x, h1.y), ay[t]);
-                            ay[t] = bf16x2_fma(wd[b].w, make_float2(h1.z, h1.w), ay[t]);
+    pipe_init(P, NS, CW);
+    if (warp == CW) build_routing_warp(R, ws.ids, n * k);   // ids final: the router grid is complete
+    __syncthreads();
+    const int total = n_sh + R.nu * rb_per_e;
+
+    if (warp == CW) {
+        // ------------------------------------------------ producer warp
+        griddep_wait();   // h of the gate/up grid is copied along with the weights
+        const uint64_t pol = policy_evict_first();
+        uint32_t it = 0;
+        int next = 0;
+        if (lane == 0) next = (int)atomicAdd(ws.queue2, 1u);
+        for (;;) {
+            if (aborted(P)) break;
+            const int task = __shfl_sync(0xffffffffu, next, 0);
+            if (lane == 0) next = (int)atomicAdd(ws.queue2, 1u);   // in flight while this task streams
+            if (task >= total) break;
+            const bool sh = task < n_sh;
+            int u = 0, rb = 0, ns = 0, ck = 0;
+            if (!sh) {
+                u = (task - n_sh) / rb_per_e;
+                rb = (task - n_sh) % rb_per_e;
+                ns = R.ustart[u + 1] - R.ustart[u];
+                ck = down_chunk_ksteps(nkt, nsb, ns);
+            }
+            const int nch = sh ? nch_sh : nkt / ck;
+            for (int c = 0; c < nch; ++c) {
+                const int s = it % NS;
+                const uint32_t ph = (it / NS) & 1;
+                if (!mbar_wait(&P.empty[s], ph ^ 1, ws.err)) { set_abort(P); break; }
+                if (lane == 0) {
+                    unsigned char* st = stages + s * kStageBytes;
+                    if (sh) {
+                        const int kc0 = c * ck_sh;
+                        const uint32_t bytes = ck_sh * 128;
+                        P.info[s] = ChunkInfo{task, c, nch, kc0, ck_sh};
+                        mbar_arrive_expect_tx(&P.full[s], bytes);
+                        bulk_load(st, W.sh_down + ((size_t)task * (I / 8) + kc0) * 64, bytes, &P.full[s], pol);
+                    } else {
+                        const int e = R.uniq[u], s0 = R.ustart[u];
+                        const int kt0 = c * ck;
+                        const int sb0 = nsb > 1 ? kt0 / 4 : 0, nsbc = nsb > 1 ? (ck + 3) / 4 : 1;
+                        const uint32_t qb = ck * 512, sb = ck * 128, dbb = nsbc * 128;
+                        const uint32_t hb = ck * 256, hsb = ck * 16;
+                        P.info[s] = ChunkInfo{task, c, nch, kt0, ck};
+                        mbar_arrive_expect_tx(&P.full[s], qb + sb + dbb + ns * (hb + hsb));
+                        bulk_load(st, W.down_q + (size_t)e * W.q2_q_stride + ((size_t)rb * nkt + kt0) * 512, qb,
+                                  &P.full[s], pol);
+                        bulk_load(st + qb, W.down_sc + (size_t)e * W.q2_sc_stride + ((size_t)rb * nkt + kt0) * 32,
+                                  sb, &P.full[s], pol);
+                        bulk_load(st + qb + sb,
+                                  W.down_dd + (size_t)e * W.q2_dd_stride + ((size_t)rb * nsb + sb0) * 32, dbb,
+                                  &P.full[s], pol);
+                        unsigned char* hdst = st + qb + sb + dbb;
+                        for (int t = 0; t < ns; ++t) {
+                            const int slot = R.slot[s0 + t];
+                            bulk_load_plain(hdst + t * hb, ws.h_rt + (size_t)slot * I + 64 * kt0, hb, &P.full[s]);
+                            bulk_load_plain(hdst + ns * hb + t * hsb, ws.hsum_rt + (size_t)slot * (I / 16) + 4 * kt0,
+                                            hsb, &P.full[s]);
                         }
                     }
                 }
+                __syncwarp();
+                ++it;
             }
+        }
+        producer_finish(P, it, NS, ws.err);
+    } else {
+        // ------------------------------------------------ consumer warps
+        griddep_wait();   // h from the gate/up grid
+        if (D.has_shared)
+            for (int i = tid * 4; i < n * I; i += CW * 32 * 4)
+                *reinterpret_cast<float4*>(hsh + i) = __ldcg(reinterpret_cast<const float4*>(ws.h_sh + i));
+        uint32_t it = 0, cph = 0;
+        const bool staged = cons_sync(P, cph, ws.err);
+        float2 ay2[NT];
+        float acc[NT];
+        for (; staged;) {
+            const int s = it % NS;
+            if (!mbar_wait(&P.full[s], (it / NS) & 1, ws.err)) { set_abort(P); break; }
+            const ChunkInfo inf = P.info[s];
+            if (inf.task < 0 || aborted(P)) break;
+            const unsigned char* st = stages + s * kStageBytes;
+            const bool sh = inf.task < n_sh;
+            int rb, ns = 0, s0 = 0;
+            if (sh) {
+                const int rr = lane & 7, kq = lane >> 3;
+                if (inf.chunk == 0) {
 #pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                float y = ay[t].x + ay[t].y;
-                y += __shfl_xor_sync(0xffffffffu, y, 8);
-                y += __shfl_xor_sync(0xffffffffu, y, 16);
-                if (kq == 0 && t < n) red[(warp * NT + t) * 32 + rr] = y;
-            }
-            __syncthreads();
-            if (tid < 8 * n) {
-                const int r = tid & 7, t = tid >> 3;
-                float y = 0.f;
-                for (int w = 0; w < kWarps; ++w) y += red[(w * NT + t) * 32 + r];
-                ws.y_sh[(int64_t)t * H + 8 * task + r] = y;
-            }
-        } else {
-            const int tt = task - n_sh;
-            const int u = tt / rb_per_e, rb = tt % rb_per_e;
-            const int e = R.uniq[u];
-            const int s0 = R.ustart[u], ns = R.ustart[u + 1] - s0;
-            int slot[NT];
-#pragma unroll
-            for (int t = 0; t < NT; ++t) slot[t] = t < ns ? R.slot[s0 + t] : 0;
-            float acc[NT];
-#pragma unroll
-            for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-            const uint8_t* qb = W.down_q + (int64_t)e * W.q2_q_stride + ((int64_t)rb * nkt * 32 + lane) * 16;
-            const uint32_t* scb = W.down_sc + (int64_t)e * W.q2_sc_stride + (int64_t)rb * nkt * 32 + lane;
-            const uint32_t* ddb = W.down_dd + (int64_t)e * W.q2_dd_stride + (int64_t)rb * nsb * 32 + lane;
-            constexpr int KB = 4;
-            for (int kt0 = warp * KB; kt0 < nkt; kt0 += kWarps * KB) {
-                uint4 qv[KB];
-                uint32_t scv[KB], ddv[KB];
-#pragma unroll
-                for (int b = 0; b < KB; ++b) {
-                    const int kt = kt0 + b;
-                    if (kt < nkt) {
-                        qv[b] = ld_stream_v4(qb + (int64_t)kt * 512);
-                        scv[b] = ld_stream_u32(scb + kt * 32);
-                        ddv[b] = ld_stream_u32(ddb + (nsb > 1 ? (kt >> 2) : 0) * 32);
-                    }
+                    for (int t = 0; t < NT; ++t) ay2[t] = make_float2(0.f, 0.f);
                 }
+                const uint4* dt = reinterpret_cast<const uint4*>(st);
+                for (int kc = warp * 4 + kq; kc < inf.cnt; kc += 4 * CW) {
+                    const uint4 wd = dt[kc * 8 + rr];
+                    const int col = 8 * (inf.lo + kc);
 #pragma unroll
-                for (int b = 0; b < KB; ++b) {
-                    const int kt = kt0 + b;
-                    if (kt >= nkt) break;
-                    const float d = half_bits(ddv[b] & 0xffffu), dmin = half_bits(ddv[b] >> 16);
-                    const uint32_t words[4] = {qv[b].x, qv[b].y, qv[b].z, qv[b].w};
+                    for (int t = 0; t < NT; ++t)
+                        if (t < n) bf16x8_dot(wd, hsh + t * I + col, ay2[t]);
+                }
+            } else {
+                const int tt = inf.task - n_sh, u = tt / rb_per_e;
+                rb = tt % rb_per_e;
+                s0 = R.ustart[u];
+                ns = R.ustart[u + 1] - s0;
+                if (inf.chunk == 0) {
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+                }
+                const int nsbc = nsb > 1 ? (inf.cnt + 3) / 4 : 1;
+                const uint4* qv = reinterpret_cast<const uint4*>(st);
+                const uint32_t* scv = reinterpret_cast<const uint32_t*>(st + inf.cnt * 512);
+                const uint32_t* ddv = reinterpret_cast<const uint32_t*>(st + inf.cnt * 640);
+                const float* hst = reinterpret_cast<const float*>(st + inf.cnt * 640 + nsbc * 128);
+                const float* hsst = hst + ns * inf.cnt * 64;
+                for (int kt = warp; kt < inf.cnt; kt += CW) {
+                    const uint4 q = qv[kt * 32 + lane];
+                    const uint32_t scw = scv[kt * 32 + lane];
+                    const uint32_t dd = ddv[(nsb > 1 ? (kt >> 2) : 0) * 32 + lane];
+                    const float d = half_bits(dd & 0xffffu), dmin = half_bits(dd >> 16);
+                    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
                         const float* hp[NT];
                         float S[NT];
 #pragma unroll
                         for (int t = 0; t < NT; ++t) {
-                            hp[t] = ws.h_rt + (int64_t)slot[t] * I + 64 * kt + 16 * jj;
-                            S[t] = t < ns ? __ldg(ws.hsum_rt + (int64_t)slot[t] * (I / 16) + 4 * kt + jj) : 0.f;
+                            hp[t] = hst + (t * inf.cnt + kt) * 64 + 16 * jj;
+                            S[t] = t < ns ? hsst[(t * inf.cnt + kt) * 4 + jj] : 0.f;
                         }
                         float A[NT];
                         q2_word<NT>(words[jj], hp, ns, A);
-                        const uint32_t sb = (scv[b] >> (8 * jj)) & 0xffu;
-                        const float a4 = 4.0f * d * (float)(sb & 15u);
-                        const float bb = a4 + dmin * (float)(sb >> 4);
+                        const uint32_t sb = (scw >> (8 * jj)) & 0xffu;
+                        const float scf = __uint_as_float(0x4b000000u | (sb & 15u)) - 8388608.0f;
+                        const float mf = __uint_as_float(0x4b000000u | (sb >> 4)) - 8388608.0f;
+                        const float a4 = 4.0f * d * scf;
+                        const float bb = fmaf(dmin, mf, a4);
 #pragma unroll
                         for (int t = 0; t < NT; ++t)
                             if (t < ns) acc[t] = fmaf(a4, A[t], fmaf(-bb, S[t], acc[t]));
                     }
                 }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&P.empty[s]);
+            if (inf.chunk == inf.nchunk - 1) {
+                // task epilogue: reduce, store y, count the task in its 32-row block
+                if (sh) {
+                    const int rr = lane & 7, kq = lane >> 3;
 #pragma unroll
-            for (int t = 0; t < NT; ++t)
-                if (t < ns) red[(warp * NT + t) * 32 + lane] = acc[t];
-            __syncthreads();
-            if (warp < ns) {
-                const int t = warp;
-                float y = 0.f;
-                for (int w = 0; w < kWarps; ++w) y += red[(w * NT + t) * 32 + lane];
-                ws.y_rt[(int64_t)R.slot[s0 + t] * H + 32 * rb + lane] = y;
+                    for (int t = 0; t < NT; ++t) {
+                        float y = ay2[t].x + ay2[t].y;
+                        y += __shfl_xor_sync(0xffffffffu, y, 8);
+                        y += __shfl_xor_sync(0xffffffffu, y, 16);
+                        if (kq == 0 && t < n) red[(warp * NT + t) * 32 + rr] = y;
+                    }
+                    if (!cons_sync(P, cph, ws.err)) break;
+                    if (tid < 8 * n) {
+                        const int r = tid & 7, t = tid >> 3;
+                        float y = 0.f;
+                        for (int w = 0; w < CW; ++w) y += red[(w * NT + t) * 32 + r];
+                        ws.y_sh[(int64_t)t * H + 8 * inf.task + r] = y;
+                    }
+                } else {
+#pragma unroll
+                    for (int t = 0; t < NT; ++t)
+                        if (t < ns) red[(warp * NT + t) * 32 + lane] = acc[t];
+                    if (!cons_sync(P, cph, ws.err)) break;
+                    if (warp < ns) {
+                        float y = 0.f;
+                        for (int w = 0; w < CW; ++w) y += red[(w * NT + warp) * 32 + lane];
+                        ws.y_rt[(int64_t)R.slot[s0 + warp] * H + 32 * rb + lane] = y;
+                    }
+                }
+                if (!cons_sync(P, cph, ws.err)) break;
             }
+            ++it;
         }
-        __syncthreads();
+    }
+    griddep_launch();
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        s_last = atomicAdd(ws.done2, 1u) == gridDim.x - 1;
+        if (s_last) {
+            *ws.queue2 = 0;
+            *ws.done2 = 0;
+        }
     }
 }
 
 // ---------------------------------------------------------------- combine
-__global__ void k_combine_decode(Dims D, DecodeWs ws, float* out, int n) {
-    const int64_t i4 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+// out[t][r] = y_shared[t][r] + sum_j w[t][j] y[t*k + j][r], j in rank order.
+__global__ void __launch_bounds__(256) k_combine_decode(Dims D, DecodeWs ws, float* out, int n) {
+    griddep_wait();   // y of the down grid
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int H = D.H, k = D.k;
-    if (i4 >= (int64_t)n * H) return;
-    const int t = (int)(i4 / H), r = (int)(i4 % H);
-    float4 acc = D.has_shared ? __ldcg(reinterpret_cast<const float4*>(ws.y_sh + (int64_t)t * H + r))
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-        const float w = __ldcg(ws.wts + t * k + j);
-        const float4 y = __ldcg(reinterpret_cast<const float4*>(ws.y_rt + (int64_t)(t * k + j) * H + r));
-        acc.x = fmaf(w, y.x, acc.x);
-        acc.y = fmaf(w, y.y, acc.y);
-        acc.z = fmaf(w, y.z, acc.z);
-        acc.w = fmaf(w, y.w, acc.w);
+    if (i >= (int64_t)n * H) return;
+    const int t = (int)(i / H), r = (int)(i % H);
+    float w[16], y[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {   // all loads first: k <= 16
+        if (j < k) {
+            w[j] = __ldcg(ws.wts + t * k + j);
+            y[j] = __ldcg(ws.y_rt + (int64_t)(t * k + j) * H + r);
+        }
     }
-    *reinterpret_cast<float4*>(out + i4) = acc;
+    float acc = D.has_shared ? __ldcg(ws.y_sh + (int64_t)t * H + r) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        if (j < k) acc = fmaf(w[j], y[j], acc);
+    out[i] = acc;
 }
 
 // ---------------------------------------------------------------- launchers
-size_t gateup_smem_bytes(const Dims& D, int n, int NT) {
-    return sizeof(float) * ((size_t)kTabFloats + (size_t)n * D.H + (size_t)kWarps * 2 * NT * 32);
-}
-size_t down_smem_bytes(const Dims& D, int n, int NT) {
-    return sizeof(float) * ((size_t)n * D.I + (size_t)kWarps * NT * 32);
+template <int NT>
+size_t gateup_smem_bytes(const Dims& D, int n) {
+    using C = GateUpCfg<NT>;
+    return (size_t)C::NS * kStageBytes + sizeof(float) * ((size_t)C::kTabFloats + C::kRedFloats + (size_t)n * D.H);
 }
 
-// Events (optional): ev[2i] / ev[2i+1] recorded around launch i.
+template <int NT>
+size_t down_smem_bytes(const Dims& D, int n) {
+    using C = DownCfg<NT>;
+    return (size_t)C::NS * kStageBytes + sizeof(float) * ((size_t)C::kRedFloats + (size_t)n * D.I);
+}
+
+size_t router_smem_bytes(const Dims& D, int n) { return sizeof(float) * (size_t)n * D.H; }
+
+// Events (optional): ev[2i] / ev[2i+1] recorded around launch i.  Under
+// stream capture they become external event-record nodes, so that replays
+// of the graph time each kernel.
 struct Marks {
     cudaEvent_t const* ev;
     cudaStream_t st;
     int i = 0;
-    void before() { if (ev) cudaEventRecord(ev[2 * i], st); }
-    void after() { if (ev) cudaEventRecord(ev[2 * i + 1], st); ++i; }
+    unsigned flags = 0;
+    Marks(cudaEvent_t const* e, cudaStream_t s) : ev(e), st(s) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (ev && cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+            flags = cudaEventRecordExternal;
+    }
+    void before() { if (ev) cudaEventRecordWithFlags(ev[2 * i], st, flags); }
+    void after() {
+        if (ev) cudaEventRecordWithFlags(ev[2 * i + 1], st, flags);
+        ++i;
+    }
 };
 
 const char* const kDecodeKernels[4] = {"k_router_decode", "k_gateup_decode", "k_down_decode", "k_combine_decode"};
 
-// Per (kernel instance, device): dynamic shared memory opt-in and resident
-// CTAs per SM, set once outside any stream capture.
-struct KernelCfg {
-    size_t smem = 0;
-    int per_sm = 0;
-};
 
+// Dynamic shared memory opt-in: raised once per (kernel, device) to the
+// device's per-block maximum, outside any stream capture (the first forward
+// of a shape does it).
 template <typename K>
-cudaError_t configure(K kernel, size_t smem, KernelCfg* cfg) {
-    if (cfg->smem >= smem && cfg->per_sm > 0) return cudaSuccess;
-    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+cudaError_t configure(K kernel) {
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, bool> done;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem);
+    std::lock_guard<std::mutex> lock(mu);
+    auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+    if (done.count(key)) return cudaSuccess;
+    int optin = 0;
+    err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (err != cudaSuccess) return err;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    cfg->smem = smem;
-    cfg->per_sm = per_sm;
+    cudaFuncAttributes fa;
+    err = cudaFuncGetAttributes(&fa, kernel);
+    if (err != cudaSuccess) return err;
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
+    if (err != cudaSuccess) return err;
+    done[key] = true;
     return cudaSuccess;
 }
 
-constexpr int kMaxDevices = 64;
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 template <int NT>
 cudaError_t launch_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n, float* out,
                             int n_sm, cudaStream_t st, cudaEvent_t const* ev) {
-    static KernelCfg cfg1[kMaxDevices], cfg2[kMaxDevices];
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
+    cudaError_t err;
+    const size_t s1 = gateup_smem_bytes<NT>(D, n), s2 = down_smem_bytes<NT>(D, n);
+    if ((err = configure(k_gateup_decode<NT>)) != cudaSuccess) return err;
+    if ((err = configure(k_down_decode<NT>)) != cudaSuccess) return err;
+    if ((err = configure(k_router_decode<NT>)) != cudaSuccess) return err;
+    Marks mk(ev, st);
+    const bool pdl = ev == nullptr;   // profiled runs keep the kernels apart
+    const int rgrid = (D.E + kRWarps - 1) / kRWarps;
+    mk.before();
+    k_router_decode<NT><<<rgrid, kRWarps * 32, router_smem_bytes(D, n), st>>>(W, D, ws, x, n);
+    mk.after();
+    mk.before();
+    err = launch_pdl(k_gateup_decode<NT>, dim3(n_sm), dim3(Warps<NT>::kThreads), s1, st, pdl, W, D, ws, x, n);
+    mk.after();
     if (err != cudaSuccess) return err;
-    if (dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    Marks mk{ev, st};
-    const int rgrid = (D.E + kWarps - 1) / kWarps;
-    const size_t s1 = gateup_smem_bytes(D, n, NT), s2 = down_smem_bytes(D, n, NT);
-    if ((err = configure(k_gateup_decode<NT>, s1, &cfg1[dev])) != cudaSuccess) return err;
-    if ((err = configure(k_down_decode<NT>, s2, &cfg2[dev])) != cudaSuccess) return err;
     mk.before();
-    k_router_decode<NT><<<rgrid, kThreads, 0, st>>>(W, D, ws, x, n);
+    err = launch_pdl(k_down_decode<NT>, dim3(n_sm), dim3(Warps<NT>::kThreads), s2, st, pdl, W, D, ws, out, n);
     mk.after();
+    if (err != cudaSuccess) return err;
+    const int64_t nel = (int64_t)n * D.H;
     mk.before();
-    k_gateup_decode<NT><<<n_sm * cfg1[dev].per_sm, kThreads, s1, st>>>(W, D, ws, x, n);
+    err = launch_pdl(k_combine_decode, dim3((unsigned)((nel + 255) / 256)), dim3(256), 0, st, pdl, D, ws, out, n);
     mk.after();
-    mk.before();
-    k_down_decode<NT><<<n_sm * cfg2[dev].per_sm, kThreads, s2, st>>>(W, D, ws, n);
-    mk.after();
-    const int64_t n4 = (int64_t)n * D.H / 4;
-    mk.before();
-    k_combine_decode<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(D, ws, out, n);
-    mk.after();
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 
 int decode_launches() { return 4; }
 const char* decode_kernel_name(int i) { return (i >= 0 && i < 4) ? kDecodeKernels[i] : nullptr; }
+
+// Dynamic shared memory of the larger decode kernel for n tokens, plus its
+// static shared memory (pipeline barriers, routing table).
+size_t decode_smem_bytes(const Dims& D, int n) {
+    size_t a, b;
+    if (n <= 1) { a = gateup_smem_bytes<1>(D, n); b = down_smem_bytes<1>(D, n); }
+    else if (n <= 2) { a = gateup_smem_bytes<2>(D, n); b = down_smem_bytes<2>(D, n); }
+    else if (n <= 4) { a = gateup_smem_bytes<4>(D, n); b = down_smem_bytes<4>(D, n); }
+    else { a = gateup_smem_bytes<8>(D, n); b = down_smem_bytes<8>(D, n); }
+    return (a > b ? a : b) + sizeof(Pipe) + sizeof(Routing) + 64;
+}
 
 cudaError_t launch_decode(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n, float* out,
                           int n_sm, cudaStream_t st, cudaEvent_t const* ev) {
@@ -654,14 +1015,22 @@ cudaError_t launch_decode(const Weights& W, const Dims& D, const DecodeWs& ws, c
     return launch_decode_t<8>(W, D, ws, x, n, out, n_sm, st, ev);
 }
 
+template <int NT>
+cudaError_t launch_route_t(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n,
+                           cudaStream_t st) {
+    cudaError_t err;
+    const size_t s0 = router_smem_bytes(D, n);
+    if ((err = configure(k_router_decode<NT>)) != cudaSuccess) return err;
+    k_router_decode<NT><<<(D.E + kRWarps - 1) / kRWarps, kRWarps * 32, s0, st>>>(W, D, ws, x, n);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_route(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n,
                          cudaStream_t st) {
-    const int rgrid = (D.E + kWarps - 1) / kWarps;
-    if (n <= 1) k_router_decode<1><<<rgrid, kThreads, 0, st>>>(W, D, ws, x, n);
-    else if (n <= 2) k_router_decode<2><<<rgrid, kThreads, 0, st>>>(W, D, ws, x, n);
-    else if (n <= 4) k_router_decode<4><<<rgrid, kThreads, 0, st>>>(W, D, ws, x, n);
-    else k_router_decode<8><<<rgrid, kThreads, 0, st>>>(W, D, ws, x, n);
-    return cudaGetLastError();
+    if (n <= 1) return launch_route_t<1>(W, D, ws, x, n, st);
+    if (n <= 2) return launch_route_t<2>(W, D, ws, x, n, st);
+    if (n <= 4) return launch_route_t<4>(W, D, ws, x, n, st);
+    return launch_route_t<8>(W, D, ws, x, n, st);
 }
 
 }  // namespace ds4

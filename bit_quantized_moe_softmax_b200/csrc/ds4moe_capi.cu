@@ -26,6 +26,7 @@ cudaError_t launch_decode(const Weights& W, const Dims& D, const DecodeWs& ws, c
                           int n_sm, cudaStream_t st, cudaEvent_t const* ev);
 int decode_launches();
 const char* decode_kernel_name(int i);
+size_t decode_smem_bytes(const Dims& D, int n);
 cudaError_t launch_route(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n,
                          cudaStream_t st);
 }  // namespace ds4
@@ -63,7 +64,7 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
 struct WsLayout {
-    size_t hdr, logits, ids, wts, h_rt, hsum_rt, h_sh, y_rt, y_sh, x_stage, out_stage, total;
+    size_t hdr, rbtick, logits, ids, wts, h_rt, hsum_rt, h_sh, y_rt, y_sh, x_stage, out_stage, total;
 };
 
 }  // namespace
@@ -90,6 +91,7 @@ struct ds4moe {
         const size_t nd = (size_t)(cap < decode_max ? cap : decode_max);
         size_t o = 0;
         w.hdr = o; o += 256;
+        w.rbtick = o; o += align256(H / 32 * 4);
         w.logits = o; o += align256(nd * E * 4);
         w.ids = o; o += align256(nd * k * 4);
         w.wts = o; o += align256(nd * k * 4);
@@ -135,6 +137,9 @@ struct ds4moe {
         w.ticket = hdr + 1;
         w.queue1 = hdr + 2;
         w.queue2 = hdr + 3;
+        w.done1 = hdr + 4;
+        w.done2 = hdr + 5;
+        w.rbtick = reinterpret_cast<uint32_t*>(ws + L.rbtick);
         w.logits = reinterpret_cast<float*>(ws + L.logits);
         w.ids = reinterpret_cast<int32_t*>(ws + L.ids);
         w.wts = reinterpret_cast<float*>(ws + L.wts);
@@ -191,6 +196,17 @@ ds4moe_status ds4moe_create(const ds4moe_shape* s, ds4moe_t** out) {
     h->D.act_bf16 = s->act_dtype == DS4MOE_ACT_BF16;
     h->decode_max = s->decode_max ? s->decode_max : 8;
     h->n_sm = n_sm;
+    {
+        int smem_optin = 0;
+        ce = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (ce != cudaSuccess) { delete h; return cuda_fail(ce, "cudaDeviceGetAttribute"); }
+        const size_t need = decode_smem_bytes(h->D, h->decode_max);
+        if (need > (size_t)smem_optin) {
+            delete h;
+            return fail(DS4MOE_ERR_SHAPE, "decode plan needs %zu bytes of shared memory per CTA (device: %d); "
+                        "lower decode_max or hidden", need, smem_optin);
+        }
+    }
     const size_t H = s->hidden, I = s->inter, E = s->n_experts;
     const size_t nsb_down = I >= 256 ? I / 256 : 1;
     h->iq2_qs_stride = I * H / 4;
@@ -241,7 +257,8 @@ ds4moe_status ds4moe_bind(ds4moe_t* h, void* d_weights, size_t weight_bytes, voi
         return fail(DS4MOE_ERR_ARG, "bind: weight buffer %zu bytes < %zu", weight_bytes, h->weight_bytes);
     WsLayout L = h->layout(h->shape.max_tokens);
     if (ws_bytes < L.total) return fail(DS4MOE_ERR_ARG, "bind: workspace %zu bytes < %zu", ws_bytes, L.total);
-    cudaError_t ce = cudaMemsetAsync(static_cast<uint8_t*>(d_workspace) + L.hdr, 0, 256, (cudaStream_t)stream);
+    cudaError_t ce = cudaMemsetAsync(static_cast<uint8_t*>(d_workspace) + L.hdr, 0, L.logits - L.hdr,
+                                     (cudaStream_t)stream);
     if (ce != cudaSuccess) return cuda_fail(ce, "bind: cudaMemsetAsync");
     h->weights = static_cast<uint8_t*>(d_weights);
     h->ws = static_cast<uint8_t*>(d_workspace);
