@@ -44,7 +44,20 @@ WORKLOADS = {
                     desc="MTP-verify style decode: 8 tokens, one MoE layer of the decode shape"),
     "decode2": dict(n=2, H=4096, I=2048, E=256, k=8,
                     desc="MTP-verify style decode: 2 tokens, one MoE layer of the decode shape"),
+    "prefill512": dict(n=512, H=4096, I=2048, E=256, k=8, zipf=1.1, bf16=True,
+                       desc="short-prompt prefill: 512 bf16 tokens, one MoE layer of the decode shape, "
+                            "Zipf(1.1) expert popularity"),
+    "prefill11709": dict(n=11709, H=4096, I=2048, E=256, k=8, zipf=1.1, bf16=True,
+                         desc="long-prompt prefill: 11,709 bf16 tokens, one MoE layer (hidden 4096, expert "
+                              "intermediate 2048, 256 experts top-8 + shared), Zipf(1.1) expert popularity"),
 }
+
+
+def algorithmic_flops(w: dict) -> dict:
+    """Tensor-core FLOPs of each prefill GEMM launch (2 per multiply-add)."""
+    H, I, k, n = w["H"], w["I"], w["k"], w["n"]
+    return {"k_moe_gemm<gate_up>": 2 * n * k * H * 2 * I, "k_moe_gemm<down>": 2 * n * k * I * H,
+            "k_moe_gemm<shared_gate_up>": 2 * n * H * 2 * I, "k_moe_gemm<shared_down>": 2 * n * I * H}
 
 
 def load_peaks():
@@ -152,18 +165,21 @@ def run_ours(args, wl, rank, local, world):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     n, H, I, E, k = wl["n"], wl["H"], wl["I"], wl["E"], wl["k"]
-    R = args.instances
+    prefill = n > 8
+    R = 1 if prefill else args.instances
     shape = synth.Shape(H=H, I=I, E=E, k=k)
-    layers, raws = [], []
+    bias = synth.zipf_bias(E, wl["zipf"], seed=5).to(dev) if wl.get("zipf") else None
+    act = m.DS4MOE_ACT_BF16 if wl.get("bf16") else m.DS4MOE_ACT_F32
+    layers = []
     for r in range(R):
-        L = synth.packed_layer(shape, seed=1000 * rank + r, device=dev)
-        lay = m.MoELayer(H, I, E, k, max_tokens=max(n, 8), device=dev)
+        L = synth.packed_layer(shape, seed=1000 * rank + r, bias=bias, device=dev)
+        lay = m.MoELayer(H, I, E, k, max_tokens=max(n, 8), act_dtype=act, has_bias=bias is not None, device=dev)
         lay.load(L)
         layers.append(lay)
-        raws.append(L if r == 0 else None)
         del L
-    P = 64
-    xs = synth.tokens(P * n, H, seed=77 + rank, device=dev).view(P, n, H).contiguous()
+    P = 2 if prefill else 64
+    xs = synth.tokens(P * n, H, seed=77 + rank, device=dev,
+                      dtype=torch.bfloat16 if act == m.DS4MOE_ACT_BF16 else torch.float32).view(P, n, H).contiguous()
     outs = torch.empty(P, n, H, dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
     nl = m.ds4moe_plan_launches(layers[0].h, n)
@@ -182,7 +198,7 @@ def run_ours(args, wl, rank, local, world):
     stream.synchronize()
 
     # graphs of S consecutive steps (cycling instances and token vectors)
-    S = max(1, min(args.steps, 64 if R * P >= 64 else R))
+    S = max(1, min(args.steps, 2 if prefill else 64))
 
     def new_events(count):
         # torch creates the CUDA event on first record: record each once before capture
@@ -262,6 +278,7 @@ def run_ours(args, wl, rank, local, world):
 
     # e2e: host buffers through the public API, copies inside the timed region
     K2 = max(1, min(args.steps, 2000))
+    K2 = min(K2, 20) if prefill else K2
     xh = xs[: min(P, K2)].cpu().pin_memory()
     oh = torch.empty(xh.shape, dtype=torch.float32).pin_memory()
     for i in range(min(10, K2)):
@@ -272,7 +289,7 @@ def run_ours(args, wl, rank, local, world):
         m.ds4moe_forward_host(layers[i % R].h, xh[i % xh.shape[0]], oh[i % xh.shape[0]], stream)
     t1 = time.perf_counter()
     e2e_s = D.max_over_ranks(t1 - t0, dev)
-    e2e = {"value": n * K2 * world / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": n * H * 4,
+    e2e = {"value": n * K2 * world / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": n * H * xh.element_size(),
            "d2h_bytes_per_step": n * H * 4, "steps": K2}
 
     # roofline of the dominant kernel
@@ -281,20 +298,31 @@ def run_ours(args, wl, rank, local, world):
     dom = max(mean, key=lambda nm: mean[nm])
     U = min(n * k, E) if n == 1 else None
     ab = algorithmic_bytes(wl, U if U is not None else n * k)
-    achieved = ab[dom] / (mean[dom] * 1e-3) / 1e9
-    peak = peaks["hbm_gbs"]
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic_from_profile(dom, args.workload),
-                "algorithmic_bytes_per_launch": ab[dom], "mean_launch_us": round(mean[dom] * 1e3, 2),
-                "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs, burst copy)"}
+    if prefill:
+        fl = algorithmic_flops(wl)
+        achieved = fl[dom] / (mean[dom] * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
+                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic_from_profile(dom, args.workload),
+                    "algorithmic_flops_per_launch": fl[dom], "mean_launch_us": round(mean[dom] * 1e3, 2),
+                    "peak_source": peak_kind + " (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)"}
+    else:
+        achieved = ab[dom] / (mean[dom] * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                    "frac": round(achieved / peak, 4), "traffic": traffic_from_profile(dom, args.workload),
+                    "algorithmic_bytes_per_launch": ab[dom], "mean_launch_us": round(mean[dom] * 1e3, 2),
+                    "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs, burst copy)"}
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "bf16" if prefill else "f32", "data": "synthetic",
         "config": {"workload": wl["desc"], "n_tokens_per_step": n, "hidden": H, "expert_inter": I,
                    "experts": E, "top_k": k, "layer_instances": R, "token_vectors": P,
-                   "l2": "weights rotate over %d layer instances (%.1f GB) and %d token vectors: inputs larger "
-                         "than L2" % (R, R * layers[0].weights.numel() / 1e9, P),
+                   "l2": ("weights rotate over %d layer instances (%.1f GB) and %d token vectors: inputs larger "
+                          "than L2" % (R, R * layers[0].weights.numel() / 1e9, P)) if not prefill else
+                         "one layer (%.1f GB of weights) and %d token batches per step: inputs larger than L2"
+                         % (layers[0].weights.numel() / 1e9, n),
                    "parallelism": "dp%d replicas (no collective on the data path)" % world},
         "expert_weight_gbs": round(ab["routed"] / (ms_per_step * 1e-3) / 1e9, 1) if U else None,
         "layer_hbm_gbs": round(ab["layer"] / (ms_per_step * 1e-3) / 1e9, 1) if U else None,
@@ -313,16 +341,18 @@ def oracle_sample(wl, n_tokens, seed=0, budget_s=20.0, device="cuda"):
     from bit_quantized_moe_softmax_b200 import synth
 
     H, I, E, k = wl["H"], wl["I"], wl["E"], wl["k"]
-    L = synth.packed_layer(synth.Shape(H=H, I=I, E=E, k=k), seed=seed, device=device)
-    x = synth.tokens(n_tokens, H, seed=seed + 5)
-    lg = oracle.router_logits(x.numpy(), L["W_r"].cpu().numpy())
+    bias = synth.zipf_bias(E, wl["zipf"], seed=5) if wl.get("zipf") else None
+    L = synth.packed_layer(synth.Shape(H=H, I=I, E=E, k=k), seed=seed, bias=bias, device=device)
+    x = synth.tokens(n_tokens, H, seed=seed + 5, dtype=torch.bfloat16 if wl.get("bf16") else torch.float32).float()
+    mode = 1 if wl.get("bf16") else 0
+    lg = oracle.router_logits(x.numpy(), L["W_r"].cpu().numpy(), None if bias is None else bias.numpy())
     rid, _ = oracle.topk_softmax(lg, k)
     lay = oracle.layer_from_torch(L, experts=rid.ravel())
     del L
     t0 = time.perf_counter()
     done = 0
     for t in range(n_tokens):
-        oracle.moe_forward(lay, x[t:t + 1].numpy())
+        oracle.moe_forward(lay, x[t:t + 1].numpy(), mode=mode)
         done += 1
         if time.perf_counter() - t0 > budget_s:
             break

@@ -29,6 +29,13 @@ const char* decode_kernel_name(int i);
 size_t decode_smem_bytes(const Dims& D, int n);
 cudaError_t launch_route(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n,
                          cudaStream_t st);
+cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws, const void* x, int n, float* out,
+                           int n_sm, cudaStream_t st, cudaEvent_t const* ev);
+cudaError_t launch_route_prefill(const Weights& W, const Dims& D, const PrefillWs& ws, const void* x, int n,
+                                 cudaStream_t st);
+int prefill_launches(const Dims& D);
+const char* prefill_kernel_name(const Dims& D, int i);
+size_t gemm_smem_bytes();
 }  // namespace ds4
 
 using namespace ds4;
@@ -64,7 +71,11 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
 struct WsLayout {
-    size_t hdr, rbtick, logits, ids, wts, h_rt, hsum_rt, h_sh, y_rt, y_sh, x_stage, out_stage, total;
+    size_t hdr, rbtick, logits, ids, wts, h_rt, hsum_rt, h_sh, y_rt, y_sh, x_stage, out_stage;
+    // prefill plan (capacity > decode_max only)
+    size_t p_logits, p_ids, p_wts, p_blk_cnt, p_blk_off, p_counts, p_offs, p_mtp, p_pos, p_slot, p_xb, p_Xp, p_Hb,
+        p_Hs, p_Y, p_Ys;
+    size_t total;
 };
 
 }  // namespace
@@ -102,6 +113,25 @@ struct ds4moe {
         w.y_sh = o; o += align256(nd * H * 4);
         w.x_stage = o; o += align256((size_t)cap * H * (D.act_bf16 ? 2 : 4));
         w.out_stage = o; o += align256((size_t)cap * H * 4);
+        if (cap > decode_max) {
+            const size_t N = cap, NK = N * k, nblk = (NK + 1023) / 1024;
+            w.p_logits = o; o += align256(N * E * 4);
+            w.p_ids = o; o += align256(NK * 4);
+            w.p_wts = o; o += align256(NK * 4);
+            w.p_blk_cnt = o; o += align256(nblk * E * 4);
+            w.p_blk_off = o; o += align256(nblk * E * 4);
+            w.p_counts = o; o += align256(E * 4);
+            w.p_offs = o; o += align256((E + 1) * 4);
+            w.p_mtp = o; o += align256((E + 1) * 4);
+            w.p_pos = o; o += align256(NK * 4);
+            w.p_slot = o; o += align256(NK * 4);
+            w.p_xb = o; o += align256(N * H * 2);
+            w.p_Xp = o; o += align256(NK * H * 2);
+            w.p_Hb = o; o += align256(NK * I * 2);
+            w.p_Hs = o; o += align256(N * I * 2);
+            w.p_Y = o; o += align256(NK * H * 4);
+            w.p_Ys = o; o += align256(N * H * 4);
+        }
         w.total = o;
         return w;
     }
@@ -148,6 +178,28 @@ struct ds4moe {
         w.h_sh = reinterpret_cast<float*>(ws + L.h_sh);
         w.y_rt = reinterpret_cast<float*>(ws + L.y_rt);
         w.y_sh = reinterpret_cast<float*>(ws + L.y_sh);
+        return w;
+    }
+
+    PrefillWs prefill_ws() const {
+        PrefillWs w{};
+        w.logits = reinterpret_cast<float*>(ws + L.p_logits);
+        w.ids = reinterpret_cast<int32_t*>(ws + L.p_ids);
+        w.wts = reinterpret_cast<float*>(ws + L.p_wts);
+        w.blk_cnt = reinterpret_cast<int32_t*>(ws + L.p_blk_cnt);
+        w.blk_off = reinterpret_cast<int32_t*>(ws + L.p_blk_off);
+        w.counts = reinterpret_cast<int32_t*>(ws + L.p_counts);
+        w.offs = reinterpret_cast<int32_t*>(ws + L.p_offs);
+        w.mt_prefix = reinterpret_cast<int32_t*>(ws + L.p_mtp);
+        w.pos_of_slot = reinterpret_cast<int32_t*>(ws + L.p_pos);
+        w.slot_of_pos = reinterpret_cast<int32_t*>(ws + L.p_slot);
+        w.xb = reinterpret_cast<__nv_bfloat16*>(ws + L.p_xb);
+        w.Xp = reinterpret_cast<__nv_bfloat16*>(ws + L.p_Xp);
+        w.Hb = reinterpret_cast<__nv_bfloat16*>(ws + L.p_Hb);
+        w.Hs = reinterpret_cast<__nv_bfloat16*>(ws + L.p_Hs);
+        w.Y = reinterpret_cast<float*>(ws + L.p_Y);
+        w.Ys = reinterpret_cast<float*>(ws + L.p_Ys);
+        w.err = reinterpret_cast<uint32_t*>(ws + L.hdr);
         return w;
     }
 
@@ -200,7 +252,8 @@ ds4moe_status ds4moe_create(const ds4moe_shape* s, ds4moe_t** out) {
         int smem_optin = 0;
         ce = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         if (ce != cudaSuccess) { delete h; return cuda_fail(ce, "cudaDeviceGetAttribute"); }
-        const size_t need = decode_smem_bytes(h->D, h->decode_max);
+        size_t need = decode_smem_bytes(h->D, h->decode_max);
+        if (s->max_tokens > h->decode_max && gemm_smem_bytes() + 8192 > need) need = gemm_smem_bytes() + 8192;
         if (need > (size_t)smem_optin) {
             delete h;
             return fail(DS4MOE_ERR_SHAPE, "decode plan needs %zu bytes of shared memory per CTA (device: %d); "
@@ -376,11 +429,10 @@ static ds4moe_status forward_impl(ds4moe_t* h, const void* d_x, int32_t n, float
     cudaStream_t st = (cudaStream_t)stream;
     cudaEvent_t const* ev = reinterpret_cast<cudaEvent_t const*>(events);
     cudaError_t ce;
-    if (n <= h->decode_max) {
+    if (n <= h->decode_max)
         ce = launch_decode(h->weights_view(), h->D, h->decode_ws(), d_x, n, d_out, h->n_sm, st, ev);
-    } else {
-        return fail(DS4MOE_ERR_SHAPE, "%s: n_tokens %d > decode_max %d needs the prefill plan", who, n, h->decode_max);
-    }
+    else
+        ce = launch_prefill(h->weights_view(), h->D, h->prefill_ws(), d_x, n, d_out, h->n_sm, st, ev);
     return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "forward launch");
 }
 
@@ -397,13 +449,13 @@ ds4moe_status ds4moe_forward_profiled(ds4moe_t* h, const void* d_x, int32_t n, f
 int32_t ds4moe_plan_launches(const ds4moe_t* h, int32_t n) {
     if (!h || n < 1 || n > h->shape.max_tokens) return 0;
     if (n <= h->decode_max) return decode_launches();
-    return 0;
+    return prefill_launches(h->D);
 }
 
 const char* ds4moe_plan_kernel(const ds4moe_t* h, int32_t n, int32_t i) {
     if (i < 0 || i >= ds4moe_plan_launches(h, n)) return nullptr;
     if (n <= h->decode_max) return decode_kernel_name(i);
-    return nullptr;
+    return prefill_kernel_name(h->D, i);
 }
 
 ds4moe_status ds4moe_forward_host(ds4moe_t* h, const void* x_host, int32_t n, float* out_host, void* stream) {
@@ -431,13 +483,24 @@ ds4moe_status ds4moe_route(ds4moe_t* h, const void* d_x, int32_t n, int32_t* d_i
     if (!d_w) return fail(DS4MOE_ERR_ARG, "route: NULL weights");
     if (!aligned16(d_x)) return fail(DS4MOE_ERR_ALIGN, "route: x must be 16-byte aligned");
     cudaStream_t st = (cudaStream_t)stream;
-    if (n > h->decode_max) return fail(DS4MOE_ERR_SHAPE, "route: n_tokens %d > decode_max", n);
-    DecodeWs ws = h->decode_ws();
-    cudaError_t ce = launch_route(h->weights_view(), h->D, ws, d_x, n, st);
+    const int32_t* ids_src;
+    const float* w_src;
+    cudaError_t ce;
+    if (n <= h->decode_max) {
+        DecodeWs ws = h->decode_ws();
+        ce = launch_route(h->weights_view(), h->D, ws, d_x, n, st);
+        ids_src = ws.ids;
+        w_src = ws.wts;
+    } else {
+        PrefillWs ws = h->prefill_ws();
+        ce = launch_route_prefill(h->weights_view(), h->D, ws, d_x, n, st);
+        ids_src = ws.ids;
+        w_src = ws.wts;
+    }
     if (ce == cudaSuccess)
-        ce = cudaMemcpyAsync(d_ids, ws.ids, (size_t)n * h->D.k * 4, cudaMemcpyDeviceToDevice, st);
+        ce = cudaMemcpyAsync(d_ids, ids_src, (size_t)n * h->D.k * 4, cudaMemcpyDeviceToDevice, st);
     if (ce == cudaSuccess)
-        ce = cudaMemcpyAsync(d_w, ws.wts, (size_t)n * h->D.k * 4, cudaMemcpyDeviceToDevice, st);
+        ce = cudaMemcpyAsync(d_w, w_src, (size_t)n * h->D.k * 4, cudaMemcpyDeviceToDevice, st);
     return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "route");
 }
 

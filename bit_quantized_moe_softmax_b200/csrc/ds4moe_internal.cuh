@@ -75,6 +75,27 @@ struct DecodeWs {
     float* y_sh;            // [n][H]
 };
 
+// Workspace pointers (prefill plan).
+struct PrefillWs {
+    float* logits;          // [n][E]
+    int32_t* ids;           // [n][k]
+    float* wts;             // [n][k]
+    int32_t* blk_cnt;       // [blocks of 1024 slots][E]
+    int32_t* blk_off;       // [blocks][E]
+    int32_t* counts;        // [E] slots per expert
+    int32_t* offs;          // [E + 1] first position of each expert
+    int32_t* mt_prefix;     // [E + 1] 128-row tiles before each expert
+    int32_t* pos_of_slot;   // [n k]
+    int32_t* slot_of_pos;   // [n k]
+    __nv_bfloat16* xb;      // [n][H] x in bf16 (binary32 activations only)
+    __nv_bfloat16* Xp;      // [n k][H] permuted activations
+    __nv_bfloat16* Hb;      // [n k][I] routed h
+    __nv_bfloat16* Hs;      // [n][I] shared h
+    float* Y;               // [n k][H] routed outputs (unweighted)
+    float* Ys;              // [n][H] shared output
+    uint32_t* err;
+};
+
 // ---------------------------------------------------------------- helpers
 __device__ __forceinline__ float half_bits(uint32_t b) { return __half2float(__ushort_as_half((unsigned short)b)); }
 

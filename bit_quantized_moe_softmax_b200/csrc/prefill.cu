@@ -1,0 +1,744 @@
+// prefill.cu -- the bf16 tensor-core plan for more than decode_max tokens.
+//
+//   k_router_prefill   logits in the canonical binary32 order (each lane of a
+//                      warp owns one of the 32 partial chains of a tile of
+//                      8 tokens x 8 experts; butterfly at the end)
+//   k_topk_prefill     warp per token: top-k and softmax over the selection
+//   k_hist / k_scan / k_scatter   stable counting sort of the (token, slot)
+//                      pairs by expert: slot s = t*k + j goes to position
+//                      offs[e] + (number of earlier slots with the same expert)
+//   k_gather           Xp[pos] = bf16(x[slot(pos) / k])
+//   k_moe_gemm<mode>   persistent grouped GEMM on tcgen05: per (expert,
+//                      128-row tile, n tile) D[128 x 256] = A[128 x K] B[256 x K]^T
+//                      with A = permuted activations (TMA, 128-byte swizzle)
+//                      and B = the expert's weights dequantized to bf16 in
+//                      shared memory by eight warps, accumulators in TMEM
+//                      (two 256-column buffers), epilogue by four warps:
+//                      gate/up -> silu(g) * u as bf16, down -> binary32
+//   k_combine_prefill  out = y_shared + sum_j w_j y_{pos(t, j)}, rank order
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "ds4moe_internal.cuh"
+#include "tcgen05.cuh"
+#include "topk.cuh"
+
+namespace ds4 {
+
+// ---------------------------------------------------------------- router
+// CTA: 16 warps as 4 token groups x 4 expert groups, warp tile 8 x 8 -> CTA
+// tile 32 tokens x 32 experts.  For every 128-column step the CTA stages the
+// 32 x 128 slices of x and W_r in shared memory; lane L multiplies columns
+// 4L .. 4L+3 of the slice into its chain (fma in column order).
+constexpr int kRP_T = 32, kRP_E = 32;
+
+__global__ void __launch_bounds__(512) k_router_prefill(Weights W, Dims D, const void* x, int n, float* logits) {
+    __shared__ __align__(16) float xs[kRP_T][128];
+    __shared__ __align__(16) float wsm[kRP_E][128];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t0 = blockIdx.x * kRP_T, e0 = blockIdx.y * kRP_E;
+    const int wt = (warp & 3) * 8, we = (warp >> 2) * 8;   // warp's 8 tokens / 8 experts in the CTA tile
+    const int H = D.H, E = D.E;
+    float2 acc[8][4];   // [token][expert pair]
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = make_float2(0.f, 0.f);
+    for (int i = 0; i < H / 128; ++i) {
+        // stage: 32 rows x 128 floats each = 1024 float4 per matrix, 2 per thread
+        for (int q = tid; q < kRP_T * 32; q += 512) {
+            const int row = q >> 5, c4 = q & 31;
+            const int t = t0 + row, e = e0 + row;
+            float4 xv = make_float4(0.f, 0.f, 0.f, 0.f), wv = xv;
+            if (t < n) {
+                const int64_t idx = (int64_t)t * H + 128 * i + 4 * c4;
+                if (D.act_bf16) {
+                    const uint2 v = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(x) + idx));
+                    xv = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                                     __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+                } else {
+                    xv = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + idx));
+                }
+            }
+            if (e < E) wv = __ldg(reinterpret_cast<const float4*>(W.W_r + (int64_t)e * H + 128 * i + 4 * c4));
+            *reinterpret_cast<float4*>(&xs[row][4 * c4]) = xv;
+            *reinterpret_cast<float4*>(&wsm[row][4 * c4]) = wv;
+        }
+        __syncthreads();
+        float4 xv[8], wv[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) xv[a] = *reinterpret_cast<const float4*>(&xs[wt + a][4 * lane]);
+#pragma unroll
+        for (int b = 0; b < 8; ++b) wv[b] = *reinterpret_cast<const float4*>(&wsm[we + b][4 * lane]);
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                acc[a][b] = ffma2(make_float2(xv[a].x, xv[a].x), make_float2(wv[2 * b].x, wv[2 * b + 1].x), acc[a][b]);
+                acc[a][b] = ffma2(make_float2(xv[a].y, xv[a].y), make_float2(wv[2 * b].y, wv[2 * b + 1].y), acc[a][b]);
+                acc[a][b] = ffma2(make_float2(xv[a].z, xv[a].z), make_float2(wv[2 * b].z, wv[2 * b + 1].z), acc[a][b]);
+                acc[a][b] = ffma2(make_float2(xv[a].w, xv[a].w), make_float2(wv[2 * b].w, wv[2 * b + 1].w), acc[a][b]);
+            }
+        }
+        __syncthreads();
+    }
+    // butterfly over the 32 chains, then one lane writes each logit
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            float lo = acc[a][b].x, hi = acc[a][b].y;
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) {
+                lo = lo + __shfl_xor_sync(0xffffffffu, lo, m);
+                hi = hi + __shfl_xor_sync(0xffffffffu, hi, m);
+            }
+            const int t = t0 + wt + a;
+            const int e = e0 + we + 2 * b;
+            if (lane == ((a * 4 + b) & 31) && t < n) {
+                if (e < E) logits[(int64_t)t * E + e] = W.b_r ? lo + W.b_r[e] : lo;
+                if (e + 1 < E) logits[(int64_t)t * E + e + 1] = W.b_r ? hi + W.b_r[e + 1] : hi;
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) k_topk_prefill(Dims D, const float* logits, int n, int32_t* ids, float* wts) {
+    __shared__ float buf[8][1024];
+    const int warp = threadIdx.x >> 5;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= n) return;
+    topk_softmax_warp(logits + (int64_t)t * D.E, buf[warp], D.E, D.k, ids + (int64_t)t * D.k, wts + (int64_t)t * D.k);
+}
+
+// ---------------------------------------------------------------- permutation
+constexpr int kSortBlock = 1024;   // slots per block of the counting sort
+
+__global__ void __launch_bounds__(kSortBlock) k_hist(const int32_t* ids, int nslots, int E, int32_t* blk_cnt) {
+    extern __shared__ int cnt[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+    const int s = blockIdx.x * kSortBlock + threadIdx.x;
+    if (s < nslots) atomicAdd(&cnt[ids[s]], 1);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) blk_cnt[(int64_t)blockIdx.x * E + e] = cnt[e];
+}
+
+// One CTA: counts, exclusive offsets, per-block offsets, and the m-tile prefix.
+__global__ void __launch_bounds__(1024) k_scan(const int32_t* blk_cnt, int nblk, int E, int32_t* counts,
+                                               int32_t* offs, int32_t* blk_off, int32_t* mt_prefix) {
+    __shared__ int tot[1024], mt[1024];
+    const int e = threadIdx.x;
+    int c = 0;
+    if (e < E)
+        for (int b = 0; b < nblk; ++b) c += blk_cnt[(int64_t)b * E + e];
+    tot[e] = e < E ? c : 0;
+    mt[e] = e < E ? (c + 127) / 128 : 0;
+    __syncthreads();
+    if (e == 0) {
+        int o = 0, m = 0;
+        for (int q = 0; q < E; ++q) {
+            const int cq = tot[q], mq = mt[q];
+            offs[q] = o;
+            mt_prefix[q] = m;
+            o += cq;
+            m += mq;
+        }
+        offs[E] = o;
+        mt_prefix[E] = m;
+    }
+    __syncthreads();
+    if (e < E) {
+        counts[e] = c;
+        int o = offs[e];
+        for (int b = 0; b < nblk; ++b) {
+            blk_off[(int64_t)b * E + e] = o;
+            o += blk_cnt[(int64_t)b * E + e];
+        }
+    }
+}
+
+// Stable positions inside a block: rank among same-expert slots of the same
+// warp (match_any), plus the counts of the block's earlier warps.
+__global__ void __launch_bounds__(kSortBlock) k_scatter(const int32_t* ids, int nslots, int E, const int32_t* blk_off,
+                                                        int32_t* pos_of_slot, int32_t* slot_of_pos) {
+    extern __shared__ int wcnt[];   // [32 warps][E]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
+    __syncthreads();
+    const int s = blockIdx.x * kSortBlock + tid;
+    const int e = s < nslots ? ids[s] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && rank == 0) wcnt[warp * E + e] = __popc(peers);
+    __syncthreads();
+    if (e >= 0) {
+        int before = 0;
+        for (int w = 0; w < warp; ++w) before += wcnt[w * E + e];
+        const int pos = blk_off[(int64_t)blockIdx.x * E + e] + before + rank;
+        pos_of_slot[s] = pos;
+        slot_of_pos[pos] = s;
+    }
+}
+
+// Xp[pos][:] = bf16(x[slot / k][:]), 8 elements per thread.
+__global__ void k_gather(const void* x, int act_bf16, const int32_t* slot_of_pos, int nslots, int k, int H,
+                         __nv_bfloat16* Xp) {
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int per = H / 8;
+    if (g >= (int64_t)nslots * per) return;
+    const int pos = (int)(g / per), c8 = (int)(g % per);
+    const int t = slot_of_pos[pos] / k;
+    uint4 v;
+    if (act_bf16) {
+        v = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(x) + (int64_t)t * H) + c8);
+    } else {
+        const float4* xr = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + (int64_t)t * H) + 2 * c8;
+        const float4 a = __ldg(xr), b = __ldg(xr + 1);
+        v = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+    }
+    reinterpret_cast<uint4*>(Xp + (int64_t)pos * H)[c8] = v;
+}
+
+// x (binary32) -> bf16, for the shared expert's A operand.
+__global__ void k_to_bf16(const float* x, int64_t n8, __nv_bfloat16* xb) {
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= n8) return;
+    const float4 a = __ldg(reinterpret_cast<const float4*>(x) + 2 * g), b = __ldg(reinterpret_cast<const float4*>(x) + 2 * g + 1);
+    reinterpret_cast<uint4*>(xb)[g] =
+        make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+}
+
+// ---------------------------------------------------------------- grouped GEMM
+enum GemmMode : int { kModeGateUp = 0, kModeDown = 1, kModeShGateUp = 2, kModeShDown = 3 };
+
+constexpr int kGBM = 128, kGBN = 256, kGBK = 64;
+constexpr int kGStages = 3;
+constexpr int kGAStage = kGBM * kGBK * 2;     // 16 KB
+constexpr int kGBStage = kGBN * kGBK * 2;     // 32 KB
+constexpr int kGWarps = 14;                   // TMA, MMA, 8 dequant, 4 epilogue
+constexpr int kGThreads = kGWarps * 32;
+constexpr int kGTabFloats = 256 * 8 * 8;      // binary32 grid, 8 interleaved copies
+constexpr uint32_t kGTmemCols = 512;          // two 256-column accumulators
+
+struct GemmArgs {
+    Weights W;
+    Dims D;
+    const int32_t* counts;      // [E] rows per expert (routed modes)
+    const int32_t* offs;        // [E + 1]
+    const int32_t* mt_prefix;   // [E + 1] 128-row tiles per expert, prefix
+    int n_rows;                 // shared modes: tokens
+    __nv_bfloat16* out_h;       // gate/up modes: [rows][I] bf16
+    float* out_y;               // down modes: [rows][H] binary32
+    uint32_t* err;
+};
+
+struct GemmSmem {
+    uint64_t fullA[kGStages], fullB[kGStages], empty[kGStages];
+    uint64_t accF[2], accE[2], done;
+    uint32_t tmem_base;
+    int abort;
+    int mtp[1025];
+};
+
+__device__ __forceinline__ bool g_aborted(const GemmSmem& S) { return *(volatile const int*)&S.abort != 0; }
+__device__ __forceinline__ void g_set_abort(GemmSmem& S) { *(volatile int*)&S.abort = 1; }
+
+struct TileInfo {
+    int e;        // expert (-1: shared)
+    int row0;     // first row of the tile in A / the outputs
+    int mvalid;   // rows of the tile that belong to the expert
+    int nb;       // n tile
+};
+
+template <int MODE>
+__device__ __forceinline__ TileInfo tile_info(const GemmSmem& S, const GemmArgs& a, int tile, int NB) {
+    TileInfo ti;
+    const int mtg = tile / NB;
+    ti.nb = tile % NB;
+    if (MODE == kModeGateUp || MODE == kModeDown) {
+        int lo = 0, hi = a.D.E;   // largest e with mtp[e] <= mtg
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (S.mtp[mid] <= mtg) lo = mid;
+            else hi = mid - 1;
+        }
+        const int mt = mtg - S.mtp[lo];
+        ti.e = lo;
+        ti.row0 = __ldg(a.offs + lo) + kGBM * mt;
+        const int rem = __ldg(a.counts + lo) - kGBM * mt;
+        ti.mvalid = rem < kGBM ? rem : kGBM;
+    } else {
+        ti.e = -1;
+        ti.row0 = kGBM * mtg;
+        const int rem = a.n_rows - ti.row0;
+        ti.mvalid = rem < kGBM ? rem : kGBM;
+    }
+    return ti;
+}
+
+// B-tile unit (row r, 16-byte unit u) inside a 128-byte-swizzled K-major tile.
+__device__ __forceinline__ uint32_t b_unit_off(int r, int u) {
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((u ^ (r & 7)) << 4));
+}
+
+// One IQ2 chunk (8 weights) -> 8 bf16 (16 bytes): d(2s+1)/8 * G[a][i] * (+-1), rounded.
+__device__ __forceinline__ uint4 iq2_chunk_bf16(uint32_t idx, uint32_t S, int c, float db, const float* tabp) {
+    const uint32_t a = (idx >> (8 * c)) & 255u;
+    uint32_t sg = (S >> (7 * c)) & 127u;
+    sg |= ((uint32_t)__popc(sg) & 1u) << 7;
+    const float* trow = tabp + a * 64;
+    const float4 g0 = *reinterpret_cast<const float4*>(trow);
+    const float4 g1 = *reinterpret_cast<const float4*>(trow + 32);
+    float w[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = __uint_as_float(__float_as_uint(db * w[i]) ^ ((sg << (31 - i)) & 0x80000000u));
+    return make_uint4(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]), pack_bf16x2(w[4], w[5]), pack_bf16x2(w[6], w[7]));
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kGThreads, 1)
+    k_moe_gemm(const __grid_constant__ CUtensorMap tmapA, GemmArgs a) {
+    extern __shared__ __align__(1024) unsigned char g_smem_raw[];
+    // 1024-byte aligned stages (the swizzle pattern repeats every 1024 bytes)
+    unsigned char* base = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(g_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    unsigned char* stA = base;                                   // kGStages x 16 KB
+    unsigned char* stB = base + kGStages * kGAStage;              // kGStages x 32 KB
+    float* tab = reinterpret_cast<float*>(stB + kGStages * kGBStage);
+    __shared__ GemmSmem S;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = a.D.H, I = a.D.I;
+    const int K = (MODE == kModeGateUp || MODE == kModeShGateUp) ? H : I;
+    const int KS = K / kGBK;
+    const int NB = (MODE == kModeGateUp || MODE == kModeShGateUp) ? I / 128 : H / kGBN;
+    const bool routed = MODE == kModeGateUp || MODE == kModeDown;
+
+    if (tid == 0) {
+        for (int s = 0; s < kGStages; ++s) {
+            mbar_init(&S.fullA[s], 1);
+            mbar_init(&S.fullB[s], 8);
+            mbar_init(&S.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&S.accF[b], 1);
+            mbar_init(&S.accE[b], 4);
+        }
+        mbar_init(&S.done, 1);
+        S.abort = 0;
+        fence_barrier_init();
+    }
+    if (routed)
+        for (int e = tid; e <= a.D.E; e += kGThreads) S.mtp[e] = __ldg(a.mt_prefix + e);
+    if (MODE == kModeGateUp) {
+        for (int q = tid; q < 512; q += kGThreads) {
+            const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(a.W.grid_u8) + q);
+            const int g = q >> 1, hf = q & 1;
+            const float4 f = make_float4((float)(v & 0xffu), (float)((v >> 8) & 0xffu), (float)((v >> 16) & 0xffu),
+                                         (float)(v >> 24));
+#pragma unroll
+            for (int p = 0; p < 8; ++p) *reinterpret_cast<float4*>(tab + g * 64 + hf * 32 + p * 4) = f;
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(&S.tmem_base, kGTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    const int total_mt = routed ? S.mtp[a.D.E] : (a.n_rows + kGBM - 1) / kGBM;
+    const int ntiles = total_mt * NB;
+
+    if (warp == 0) {
+        // ------------------------------------------------ A tiles (TMA)
+        uint32_t it = 0;
+        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(S); tile += gridDim.x) {
+            const TileInfo ti = tile_info<MODE>(S, a, tile, NB);
+            for (int ks = 0; ks < KS; ++ks, ++it) {
+                const int s = it % kGStages;
+                if (!mbar_wait(&S.empty[s], ((it / kGStages) & 1) ^ 1, a.err)) { g_set_abort(S); break; }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&S.fullA[s], kGAStage);
+                    tma_load_2d(stA + s * kGAStage, &tmapA, ks * kGBK, ti.row0, &S.fullA[s]);
+                }
+                __syncwarp();
+            }
+        }
+        // drain: the last issued copies land before the CTA leaves
+        const uint32_t j0 = it > (uint32_t)kGStages ? it - kGStages : 0;
+        for (uint32_t j = j0; j < it; ++j) mbar_wait(&S.fullA[j % kGStages], (j / kGStages) & 1, a.err);
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issue
+        const uint32_t idesc = umma_idesc_bf16(kGBM, kGBN);
+        uint32_t it = 0, lt = 0;
+        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(S); tile += gridDim.x, ++lt) {
+            const uint32_t ab = lt & 1, aph = (lt >> 1) & 1;
+            if (!mbar_wait(&S.accE[ab], aph ^ 1, a.err)) { g_set_abort(S); break; }
+            tc_fence_after();
+            const uint32_t dtm = tmem + ab * kGBN;
+            for (int ks = 0; ks < KS; ++ks, ++it) {
+                const int s = it % kGStages;
+                const uint32_t ph = (it / kGStages) & 1;
+                if (!mbar_wait(&S.fullA[s], ph, a.err) || !mbar_wait(&S.fullB[s], ph, a.err)) {
+                    g_set_abort(S);
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint64_t da = umma_desc_sw128(smem_addr(stA + s * kGAStage));
+                    const uint64_t db = umma_desc_sw128(smem_addr(stB + s * kGBStage));
+#pragma unroll
+                    for (int kk = 0; kk < kGBK / 16; ++kk)
+                        umma_bf16(dtm, da + 2 * kk, db + 2 * kk, idesc, (ks | kk) != 0);
+                    umma_commit(&S.empty[s]);
+                }
+                __syncwarp();
+            }
+            if (g_aborted(S)) break;
+            if (lane == 0) umma_commit(&S.accF[ab]);
+            __syncwarp();
+        }
+        // every issued MMA has finished before TMEM is released
+        if (lane == 0) umma_commit(&S.done);
+        __syncwarp();
+        mbar_wait(&S.done, 0, a.err);
+    } else if (warp < 10) {
+        // ------------------------------------------------ B tiles (dequantize to bf16)
+        const int r = tid - 64;   // B-tile row 0..255
+        const float* tabp = tab + (lane & 7) * 4;
+        uint32_t it = 0;
+        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(S); tile += gridDim.x) {
+            const TileInfo ti = tile_info<MODE>(S, a, tile, NB);
+            // source row of this thread
+            const uint8_t* qs = nullptr;
+            const uint16_t* dq = nullptr;
+            const uint32_t* scp = nullptr;
+            const uint32_t* ddp = nullptr;
+            const __nv_bfloat16* bfrow = nullptr;
+            int row = 0;
+            if (MODE == kModeGateUp) {
+                row = 128 * ti.nb + (r & 127);
+                const size_t e = (size_t)ti.e;
+                qs = (r < 128 ? a.W.gate_qs : a.W.up_qs) + e * a.W.iq2_qs_stride + (size_t)(row >> 5) * (H / 64) * 512 +
+                     (row & 31) * 16;
+                dq = (r < 128 ? a.W.gate_d : a.W.up_d) + e * a.W.iq2_d_stride + (size_t)(row >> 5) * (H / 256) * 32 +
+                     (row & 31);
+            } else if (MODE == kModeDown) {
+                row = kGBN * ti.nb + r;
+                const size_t e = (size_t)ti.e;
+                const int nkt = I / 64, nsb = I >= 256 ? I / 256 : 1;
+                qs = a.W.down_q + e * a.W.q2_q_stride + ((size_t)(row >> 5) * nkt * 32 + (row & 31)) * 16;
+                scp = a.W.down_sc + e * a.W.q2_sc_stride + (size_t)(row >> 5) * nkt * 32 + (row & 31);
+                ddp = a.W.down_dd + e * a.W.q2_dd_stride + (size_t)(row >> 5) * nsb * 32 + (row & 31);
+            } else if (MODE == kModeShGateUp) {
+                row = 128 * ti.nb + (r & 127);
+                bfrow = (r < 128 ? a.W.sh_gate : a.W.sh_up) + (size_t)(row >> 3) * (H / 8) * 64 + (row & 7) * 8;
+            } else {
+                row = kGBN * ti.nb + r;
+                bfrow = a.W.sh_down + (size_t)(row >> 3) * (I / 8) * 64 + (row & 7) * 8;
+            }
+            for (int ks = 0; ks < KS; ++ks, ++it) {
+                // fetch this row's piece of the k step before waiting for the stage
+                uint4 q = make_uint4(0, 0, 0, 0);
+                uint32_t aux0 = 0, aux1 = 0;
+                uint4 bf[8];
+                if (MODE == kModeGateUp) {
+                    q = ld_stream_v4(qs + (size_t)ks * 512);
+                    aux0 = ld_stream_u16(dq + (ks >> 2) * 32);
+                } else if (MODE == kModeDown) {
+                    q = ld_stream_v4(qs + (size_t)ks * 512);
+                    aux0 = ld_stream_u32(scp + ks * 32);
+                    aux1 = ld_stream_u32(ddp + (I >= 256 ? (ks >> 2) : 0) * 32);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) bf[u] = ld_stream_v4(bfrow + (size_t)(8 * ks + u) * 64);
+                }
+                const int s = it % kGStages;
+                if (!mbar_wait(&S.empty[s], ((it / kGStages) & 1) ^ 1, a.err)) { g_set_abort(S); break; }
+                unsigned char* bt = stB + s * kGBStage;
+                if (MODE == kModeGateUp) {
+                    const float d = half_bits(aux0);
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const uint32_t idx = hf ? q.z : q.x, Sw = hf ? q.w : q.y;
+                        const float db = d * (__uint_as_float(0x4b000001u | ((Sw >> 27) & 0x1eu)) - 8388608.0f) * 0.125f;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            *reinterpret_cast<uint4*>(bt + b_unit_off(r, 4 * hf + c)) = iq2_chunk_bf16(idx, Sw, c, db, tabp);
+                    }
+                } else if (MODE == kModeDown) {
+                    const float d = half_bits(aux1 & 0xffffu), dmin = half_bits(aux1 >> 16);
+                    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const uint32_t sb = (aux0 >> (8 * (u >> 1))) & 0xffu;
+                        const float sc = d * (float)(sb & 15u), mn = dmin * (float)(sb >> 4);
+                        const uint32_t codes = words[u >> 1] >> (16 * (u & 1));
+                        float w[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) w[i] = fmaf(sc, (float)((codes >> (2 * i)) & 3u), -mn);
+                        *reinterpret_cast<uint4*>(bt + b_unit_off(r, u)) =
+                            make_uint4(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]), pack_bf16x2(w[4], w[5]),
+                                       pack_bf16x2(w[6], w[7]));
+                    }
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(bt + b_unit_off(r, u)) = bf[u];
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.fullB[s]);
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (TMEM -> registers -> global)
+        const int qd = warp & 3;          // TMEM lanes 32 qd .. 32 qd + 31
+        const int m = 32 * qd + lane;     // tile row of this thread
+        uint32_t lt = 0;
+        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(S); tile += gridDim.x, ++lt) {
+            const TileInfo ti = tile_info<MODE>(S, a, tile, NB);
+            const uint32_t ab = lt & 1, aph = (lt >> 1) & 1;
+            if (!mbar_wait(&S.accF[ab], aph, a.err)) { g_set_abort(S); break; }
+            tc_fence_after();
+            const uint32_t taddr = tmem + ((uint32_t)(32 * qd) << 16) + ab * kGBN;
+            const bool live = m < ti.mvalid;
+            if (MODE == kModeGateUp || MODE == kModeShGateUp) {
+                __nv_bfloat16* dst = a.out_h + (size_t)(ti.row0 + m) * I + 128 * ti.nb;
+#pragma unroll 1
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    uint32_t g[32], u[32];
+                    tmem_ld_32x32(taddr + c0, g);
+                    tmem_ld_32x32(taddr + 128 + c0, u);
+                    tmem_wait_ld();
+                    uint32_t hp[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float h0 = silu(__uint_as_float(g[2 * j])) * __uint_as_float(u[2 * j]);
+                        const float h1 = silu(__uint_as_float(g[2 * j + 1])) * __uint_as_float(u[2 * j + 1]);
+                        hp[j] = pack_bf16x2(h0, h1);
+                    }
+                    if (live) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) d4[j] = make_uint4(hp[4 * j], hp[4 * j + 1], hp[4 * j + 2], hp[4 * j + 3]);
+                    }
+                }
+            } else {
+                float* dst = a.out_y + (size_t)(ti.row0 + m) * H + kGBN * ti.nb;
+#pragma unroll 1
+                for (int c0 = 0; c0 < kGBN; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld_32x32(taddr + c0, v);
+                    tmem_wait_ld();
+                    if (live) {
+                        float4* d4 = reinterpret_cast<float4*>(dst + c0);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            d4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.accE[ab]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kGTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- combine
+__global__ void k_combine_prefill(Dims D, const float* ys, const float* y, const float* wts, const int32_t* pos_of_slot,
+                                  int n, float* out) {
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // float4 index
+    const int H = D.H, k = D.k;
+    if (g >= (int64_t)n * H / 4) return;
+    const int t = (int)(g / (H / 4)), r4 = (int)(g % (H / 4));
+    float4 acc = D.has_shared ? __ldg(reinterpret_cast<const float4*>(ys + (int64_t)t * H) + r4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+        const float w = __ldg(wts + (int64_t)t * k + j);
+        const int pos = __ldg(pos_of_slot + (int64_t)t * k + j);
+        const float4 v = __ldg(reinterpret_cast<const float4*>(y + (int64_t)pos * H) + r4);
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
+    }
+    reinterpret_cast<float4*>(out + (int64_t)t * H)[r4] = acc;
+}
+
+// ---------------------------------------------------------------- host side
+size_t gemm_smem_bytes() { return 1024 + (size_t)kGStages * (kGAStage + kGBStage) + kGTabFloats * 4; }
+
+static cudaError_t encode_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p) return cudaErrorNotSupported;
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {kGBK, kGBM};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int MODE>
+static cudaError_t launch_gemm(const CUtensorMap& map, const GemmArgs& args, int n_sm, cudaStream_t st) {
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const size_t smem = gemm_smem_bytes();
+    if (dev < 64 && !configured[dev]) {
+        e = cudaFuncSetAttribute(k_moe_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured[dev] = true;
+    }
+    k_moe_gemm<MODE><<<n_sm, kGThreads, smem, st>>>(map, args);
+    return cudaGetLastError();
+}
+
+const char* const kPrefillKernels[] = {"k_router_prefill", "k_topk_prefill", "k_hist", "k_scan", "k_scatter",
+                                       "k_gather", "k_moe_gemm<gate_up>", "k_moe_gemm<down>",
+                                       "k_moe_gemm<shared_gate_up>", "k_moe_gemm<shared_down>", "k_combine_prefill",
+                                       "k_to_bf16"};
+
+int prefill_launches(const Dims& D) { return D.has_shared ? (D.act_bf16 ? 11 : 12) : 9; }
+const char* prefill_kernel_name(const Dims& D, int i) {
+    static const int with_shared_f32[] = {11, 0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10};
+    static const int with_shared_bf16[] = {0, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10};
+    static const int routed_only[] = {0, 1, 2, 3, 4, 5, 6, 7, 10};
+    const int n = prefill_launches(D);
+    if (i < 0 || i >= n) return nullptr;
+    const int* order = D.has_shared ? (D.act_bf16 ? with_shared_bf16 : with_shared_f32) : routed_only;
+    return kPrefillKernels[order[i]];
+}
+
+struct Marks2 {
+    cudaEvent_t const* ev;
+    cudaStream_t st;
+    int i = 0;
+    unsigned flags = 0;
+    Marks2(cudaEvent_t const* e, cudaStream_t s) : ev(e), st(s) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (ev && cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+            flags = cudaEventRecordExternal;
+    }
+    void before() { if (ev) cudaEventRecordWithFlags(ev[2 * i], st, flags); }
+    void after() {
+        if (ev) cudaEventRecordWithFlags(ev[2 * i + 1], st, flags);
+        ++i;
+    }
+};
+
+cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws, const void* x, int n, float* out,
+                           int n_sm, cudaStream_t st, cudaEvent_t const* ev) {
+    cudaError_t e;
+    Marks2 mk(ev, st);
+    const int H = D.H, E = D.E, k = D.k, nslots = n * k;
+    const int nblk = (nslots + kSortBlock - 1) / kSortBlock;
+    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    if (D.has_shared && !D.act_bf16) {
+        const int64_t n8 = (int64_t)n * H / 8;
+        mk.before();
+        k_to_bf16<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(reinterpret_cast<const float*>(x), n8, ws.xb);
+        mk.after();
+        xb = ws.xb;
+    }
+    mk.before();
+    k_router_prefill<<<dim3((n + kRP_T - 1) / kRP_T, (E + kRP_E - 1) / kRP_E), 512, 0, st>>>(W, D, x, n, ws.logits);
+    mk.after();
+    mk.before();
+    k_topk_prefill<<<(n + 7) / 8, 256, 0, st>>>(D, ws.logits, n, ws.ids, ws.wts);
+    mk.after();
+    mk.before();
+    k_hist<<<nblk, kSortBlock, E * sizeof(int), st>>>(ws.ids, nslots, E, ws.blk_cnt);
+    mk.after();
+    mk.before();
+    k_scan<<<1, 1024, 0, st>>>(ws.blk_cnt, nblk, E, ws.counts, ws.offs, ws.blk_off, ws.mt_prefix);
+    mk.after();
+    {
+        static bool big[64] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (32 * E * sizeof(int) > 48 * 1024 && dev < 64 && !big[dev]) {
+            e = cudaFuncSetAttribute(k_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * E * (int)sizeof(int));
+            if (e != cudaSuccess) return e;
+            big[dev] = true;
+        }
+    }
+    mk.before();
+    k_scatter<<<nblk, kSortBlock, 32 * E * sizeof(int), st>>>(ws.ids, nslots, E, ws.blk_off, ws.pos_of_slot,
+                                                               ws.slot_of_pos);
+    mk.after();
+    const int64_t ng = (int64_t)nslots * H / 8;
+    mk.before();
+    k_gather<<<(unsigned)((ng + 255) / 256), 256, 0, st>>>(x, D.act_bf16, ws.slot_of_pos, nslots, k, H, ws.Xp);
+    mk.after();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    GemmArgs ga{};
+    ga.W = W;
+    ga.D = D;
+    ga.counts = ws.counts;
+    ga.offs = ws.offs;
+    ga.mt_prefix = ws.mt_prefix;
+    ga.err = ws.err;
+    CUtensorMap mA;
+    // routed gate/up: A = Xp [n k][H] -> Hb [n k][I]
+    if ((e = encode_tmap(&mA, ws.Xp, nslots, H)) != cudaSuccess) return e;
+    ga.out_h = ws.Hb;
+    mk.before();
+    if ((e = launch_gemm<kModeGateUp>(mA, ga, n_sm, st)) != cudaSuccess) return e;
+    mk.after();
+    // routed down: A = Hb [n k][I] -> Y [n k][H]
+    if ((e = encode_tmap(&mA, ws.Hb, nslots, D.I)) != cudaSuccess) return e;
+    ga.out_y = ws.Y;
+    mk.before();
+    if ((e = launch_gemm<kModeDown>(mA, ga, n_sm, st)) != cudaSuccess) return e;
+    mk.after();
+    if (D.has_shared) {
+        ga.n_rows = n;
+        if ((e = encode_tmap(&mA, xb, n, H)) != cudaSuccess) return e;
+        ga.out_h = ws.Hs;
+        mk.before();
+        if ((e = launch_gemm<kModeShGateUp>(mA, ga, n_sm, st)) != cudaSuccess) return e;
+        mk.after();
+        if ((e = encode_tmap(&mA, ws.Hs, n, D.I)) != cudaSuccess) return e;
+        ga.out_y = ws.Ys;
+        mk.before();
+        if ((e = launch_gemm<kModeShDown>(mA, ga, n_sm, st)) != cudaSuccess) return e;
+        mk.after();
+    }
+    const int64_t n4 = (int64_t)n * H / 4;
+    mk.before();
+    k_combine_prefill<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(D, ws.Ys, ws.Y, ws.wts, ws.pos_of_slot, n, out);
+    mk.after();
+    return cudaGetLastError();
+}
+
+// Routing only (prefill sizes): logits and top-k.
+cudaError_t launch_route_prefill(const Weights& W, const Dims& D, const PrefillWs& ws, const void* x, int n,
+                                 cudaStream_t st) {
+    k_router_prefill<<<dim3((n + kRP_T - 1) / kRP_T, (D.E + kRP_E - 1) / kRP_E), 512, 0, st>>>(W, D, x, n, ws.logits);
+    k_topk_prefill<<<(n + 7) / 8, 256, 0, st>>>(D, ws.logits, n, ws.ids, ws.wts);
+    return cudaGetLastError();
+}
+
+}  // namespace ds4

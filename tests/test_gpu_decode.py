@@ -60,7 +60,8 @@ def test_pack_iq2_bytes_match_oracle(orc, nblocks):
     g = synth.gen(100 + nblocks)
     w = synth.normal((nblocks * 256,), 0.02, g)
     w[:256] *= 0
-    w[300] = -0.0
+    if nblocks > 1:
+        w[300] = -0.0
     grid = synth.grid_table(0)
     ref = orc.pack_iq2xxs(w.numpy(), grid.numpy())
     out = torch.empty(nblocks, 66, dtype=torch.uint8, device="cuda")

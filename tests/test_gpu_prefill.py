@@ -1,0 +1,103 @@
+"""GPU parity of the prefill (bf16 tensor-core) plan against the CPU oracle, through the C ABI.
+
+Bars: routed expert ids bit-exact (canonical binary32 logits); outputs within
+2e-3 of max|ref| against the oracle's bf16 reading (x, dequantized weights and
+h rounded to bfloat16 where the tensor-core path rounds them).
+"""
+import numpy as np
+import pytest
+import torch
+
+import bit_quantized_moe_softmax_b200 as m
+from bit_quantized_moe_softmax_b200 import synth
+from tests._util import oracle_layer, pack_with_oracle, rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_quantized_moe_softmax_b200 import build
+
+    build.build()
+
+
+def _tiny(orc, E=8, k=2, seed=0, bias=False, shared=True, router_std=0.02):
+    b = synth.zipf_bias(E, 1.1, seed) if bias else None
+    L = synth.float_layer(synth.Shape(H=256, I=128, E=E, k=k, shared=shared), seed, router_std=router_std, bias=b)
+    L.update(pack_with_oracle(orc, L))
+    return L
+
+
+def _gpu(L, max_tokens, act=m.DS4MOE_ACT_BF16):
+    lay = m.MoELayer(L["H"], L["I"], L["E"], L["k"], max_tokens, act_dtype=act,
+                     has_shared=L.get("sh_gate") is not None, has_bias=L.get("b_r") is not None)
+    lay.load(L)
+    return lay
+
+
+@pytest.mark.parametrize("n", [9, 24, 200])
+def test_prefill_tiny_matches_oracle(orc, n):
+    L = _tiny(orc)
+    lay = _gpu(L, max_tokens=256)
+    x = synth.tokens(n, 256, seed=40 + n, dtype=torch.bfloat16)
+    out = lay.forward(x.cuda()).cpu().numpy()
+    ids, _ = lay.route(x.cuda())
+    ref, rid, _ = orc.moe_forward(oracle_layer(L), x.float().numpy(), mode=1)
+    assert np.array_equal(ids.cpu().numpy(), rid)
+    assert rel_err(out, ref) < TOL
+
+
+@pytest.mark.parametrize("variant", ["f32_act", "no_shared", "bias", "many_rows_per_expert", "one_expert"])
+def test_prefill_tiny_variants(orc, variant):
+    kw = {}
+    n, act = 64, m.DS4MOE_ACT_BF16
+    if variant == "f32_act":
+        act = m.DS4MOE_ACT_F32
+    if variant == "no_shared":
+        kw["shared"] = False
+    if variant == "bias":
+        kw["bias"] = True
+    if variant == "many_rows_per_expert":   # ~300 slots per expert: 3 row tiles, ragged tail
+        kw.update(E=4, k=2)
+        n = 600
+    if variant == "one_expert":
+        kw.update(E=1, k=1)
+        n = 130
+    L = _tiny(orc, **kw)
+    lay = _gpu(L, max_tokens=1024, act=act)
+    x = synth.tokens(n, 256, seed=7, dtype=torch.float32 if act == m.DS4MOE_ACT_F32 else torch.bfloat16)
+    out = lay.forward(x.cuda()).cpu().numpy()
+    ref, _, _ = orc.moe_forward(oracle_layer(L), x.float().numpy(), mode=1)
+    assert rel_err(out, ref) < TOL
+
+
+def test_prefill_repeatable(orc):
+    L = _tiny(orc)
+    lay = _gpu(L, max_tokens=256)
+    x = synth.tokens(100, 256, seed=3, dtype=torch.bfloat16).cuda()
+    a = lay.forward(x).cpu()
+    b = lay.forward(x).cpu()
+    assert torch.equal(a, b)
+
+
+def test_prefill_full_shape_short_prompt(orc):
+    """512 tokens through a full-size layer with Zipf(1.1) expert popularity (sampled outputs)."""
+    bias = synth.zipf_bias(256, 1.1, seed=5)
+    L = synth.packed_layer(synth.FULL, 5, bias=bias, device="cuda")
+    n = 512
+    lay = _gpu(L, max_tokens=n)
+    x = synth.tokens(n, 4096, seed=9, dtype=torch.bfloat16)
+    out = lay.forward(x.cuda()).cpu().numpy()
+    ids, _ = lay.route(x.cuda())
+    lg = orc.router_logits(x.float().numpy(), L["W_r"].cpu().numpy(), bias.numpy())
+    rid, _ = orc.topk_softmax(lg, 8)
+    assert np.array_equal(ids.cpu().numpy(), rid)
+    sample = [0, 1, 255, 511]
+    need = rid[sample].ravel()
+    ref, _, _ = orc.moe_forward(oracle_layer(L, experts=need), x[sample].float().numpy(), mode=1)
+    assert rel_err(out[sample], ref) < TOL
