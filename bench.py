@@ -196,6 +196,10 @@ def run_ours(args, wl, rank, local, world):
         for i in range(max(2, R)):
             step(i)             # first calls set kernel attributes outside capture
     stream.synchronize()
+    for lay in layers:          # a device-side check or bounded wait that failed ends the run here
+        code = m.ds4moe_get_device_error(lay.h, stream)
+        if code:
+            raise SystemExit("device error code %d after the first forward calls" % code)
 
     # graphs of S consecutive steps (cycling instances and token vectors)
     S = max(1, min(args.steps, 2 if prefill else 64))

@@ -36,6 +36,7 @@ cudaError_t launch_route_prefill(const Weights& W, const Dims& D, const PrefillW
 int prefill_launches(const Dims& D);
 const char* prefill_kernel_name(const Dims& D, int i);
 size_t gemm_smem_bytes();
+size_t gemm_static_smem_bytes();
 }  // namespace ds4
 
 using namespace ds4;
@@ -253,10 +254,11 @@ ds4moe_status ds4moe_create(const ds4moe_shape* s, ds4moe_t** out) {
         ce = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         if (ce != cudaSuccess) { delete h; return cuda_fail(ce, "cudaDeviceGetAttribute"); }
         size_t need = decode_smem_bytes(h->D, h->decode_max);
-        if (s->max_tokens > h->decode_max && gemm_smem_bytes() + 8192 > need) need = gemm_smem_bytes() + 8192;
+        const size_t gemm_need = gemm_smem_bytes() + gemm_static_smem_bytes();
+        if (s->max_tokens > h->decode_max && gemm_need > need) need = gemm_need;
         if (need > (size_t)smem_optin) {
             delete h;
-            return fail(DS4MOE_ERR_SHAPE, "decode plan needs %zu bytes of shared memory per CTA (device: %d); "
+            return fail(DS4MOE_ERR_SHAPE, "the plan needs %zu bytes of shared memory per CTA (device: %d); "
                         "lower decode_max or hidden", need, smem_optin);
         }
     }

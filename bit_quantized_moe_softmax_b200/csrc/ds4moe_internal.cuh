@@ -30,7 +30,7 @@ constexpr int kQK = 256;
 constexpr int kQ2Bytes = 84;
 constexpr int kIQ2Bytes = 66;
 
-enum : uint32_t { kErrBounds = 1u, kErrTimeout = 2u };
+enum : uint32_t { kErrBounds = 1u, kErrTimeout = 2u, kErrGrid = 4u };
 
 // Pointers into the caller's weight buffer, in the layout above.
 struct Weights {
@@ -117,6 +117,24 @@ __device__ __forceinline__ uint32_t ld_stream_u16(const void* p) {
     unsigned short v;
     asm("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
     return v;
+}
+
+// Packed binary32 pair multiply (sm_100): d = a * b elementwise.
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    unsigned long long A, B, D;
+    A = *reinterpret_cast<unsigned long long*>(&a);
+    B = *reinterpret_cast<unsigned long long*>(&b);
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(A), "l"(B));
+    return *reinterpret_cast<float2*>(&D);
+}
+
+// Packed binary32 pair add (sm_100): d = a + b elementwise.
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    unsigned long long A, B, D;
+    A = *reinterpret_cast<unsigned long long*>(&a);
+    B = *reinterpret_cast<unsigned long long*>(&b);
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(A), "l"(B));
+    return *reinterpret_cast<float2*>(&D);
 }
 
 // Packed binary32 pair FMA (sm_100): d = a * b + c elementwise.

@@ -111,6 +111,22 @@ __global__ void __launch_bounds__(256) k_topk_prefill(Dims D, const float* logit
     topk_softmax_warp(logits + (int64_t)t * D.E, buf[warp], D.E, D.k, ids + (int64_t)t * D.k, wts + (int64_t)t * D.k);
 }
 
+// ---------------------------------------------------------------- grouped-GEMM tiling
+// A tile is 256 rows (two 128-row tensor-core halves that share one dequantized
+// B tile) by 256 columns, stepped 64 along K through three shared-memory stages.
+constexpr int kGBM = 256, kGHalf = 128;
+constexpr int kGBN = 256, kGBK = 64;
+constexpr int kGStages = 3;
+constexpr int kGAHalf = kGHalf * kGBK * 2;    // 16 KB
+constexpr int kGAStage = 2 * kGAHalf;         // 32 KB
+constexpr int kGBStage = kGBN * kGBK * 2;     // 32 KB
+constexpr int kGDqWarps = 8, kGEpiWarps = 8;
+constexpr int kGWarps = 2 + kGDqWarps + kGEpiWarps;
+constexpr int kGThreads = kGWarps * 32;
+constexpr int kGSelRep = 16;                  // selector-table copies: conflict-free 8-byte reads
+constexpr int kGSelBytes = 256 * kGSelRep * 8;
+constexpr uint32_t kGTmemCols = 512;          // two 128-lane x 256-column binary32 accumulators
+
 // ---------------------------------------------------------------- permutation
 constexpr int kSortBlock = 1024;   // slots per block of the counting sort
 
@@ -133,7 +149,7 @@ __global__ void __launch_bounds__(1024) k_scan(const int32_t* blk_cnt, int nblk,
     if (e < E)
         for (int b = 0; b < nblk; ++b) c += blk_cnt[(int64_t)b * E + e];
     tot[e] = e < E ? c : 0;
-    mt[e] = e < E ? (c + 127) / 128 : 0;
+    mt[e] = e < E ? (c + kGBM - 1) / kGBM : 0;
     __syncthreads();
     if (e == 0) {
         int o = 0, m = 0;
@@ -212,21 +228,12 @@ __global__ void k_to_bf16(const float* x, int64_t n8, __nv_bfloat16* xb) {
 // ---------------------------------------------------------------- grouped GEMM
 enum GemmMode : int { kModeGateUp = 0, kModeDown = 1, kModeShGateUp = 2, kModeShDown = 3 };
 
-constexpr int kGBM = 128, kGBN = 256, kGBK = 64;
-constexpr int kGStages = 3;
-constexpr int kGAStage = kGBM * kGBK * 2;     // 16 KB
-constexpr int kGBStage = kGBN * kGBK * 2;     // 32 KB
-constexpr int kGWarps = 14;                   // TMA, MMA, 8 dequant, 4 epilogue
-constexpr int kGThreads = kGWarps * 32;
-constexpr int kGTabFloats = 256 * 8 * 8;      // binary32 grid, 8 interleaved copies
-constexpr uint32_t kGTmemCols = 512;          // two 256-column accumulators
-
 struct GemmArgs {
     Weights W;
     Dims D;
     const int32_t* counts;      // [E] rows per expert (routed modes)
     const int32_t* offs;        // [E + 1]
-    const int32_t* mt_prefix;   // [E + 1] 128-row tiles per expert, prefix
+    const int32_t* mt_prefix;   // [E + 1] kGBM-row tiles per expert, prefix
     int n_rows;                 // shared modes: tokens
     __nv_bfloat16* out_h;       // gate/up modes: [rows][I] bf16
     float* out_y;               // down modes: [rows][H] binary32
@@ -235,10 +242,11 @@ struct GemmArgs {
 
 struct GemmSmem {
     uint64_t fullA[kGStages], fullB[kGStages], empty[kGStages];
-    uint64_t accF[2], accE[2], done;
+    uint64_t accF, accE, done;
     uint32_t tmem_base;
     int abort;
-    int mtp[1025];
+    int nval;          // distinct grid magnitudes (gate/up mode)
+    float gval[4];
 };
 
 __device__ __forceinline__ bool g_aborted(const GemmSmem& S) { return *(volatile const int*)&S.abort != 0; }
@@ -247,23 +255,23 @@ __device__ __forceinline__ void g_set_abort(GemmSmem& S) { *(volatile int*)&S.ab
 struct TileInfo {
     int e;        // expert (-1: shared)
     int row0;     // first row of the tile in A / the outputs
-    int mvalid;   // rows of the tile that belong to the expert
+    int mvalid;   // rows of the tile that belong to the expert (1 .. kGBM)
     int nb;       // n tile
 };
 
 template <int MODE>
-__device__ __forceinline__ TileInfo tile_info(const GemmSmem& S, const GemmArgs& a, int tile, int NB) {
+__device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, int tile, int NB) {
     TileInfo ti;
     const int mtg = tile / NB;
     ti.nb = tile % NB;
     if (MODE == kModeGateUp || MODE == kModeDown) {
-        int lo = 0, hi = a.D.E;   // largest e with mtp[e] <= mtg
+        int lo = 0, hi = a.D.E;   // largest e with mt_prefix[e] <= mtg
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (S.mtp[mid] <= mtg) lo = mid;
+            if (__ldg(a.mt_prefix + mid) <= mtg) lo = mid;
             else hi = mid - 1;
         }
-        const int mt = mtg - S.mtp[lo];
+        const int mt = mtg - __ldg(a.mt_prefix + lo);
         ti.e = lo;
         ti.row0 = __ldg(a.offs + lo) + kGBM * mt;
         const int rem = __ldg(a.counts + lo) - kGBM * mt;
@@ -282,63 +290,124 @@ __device__ __forceinline__ uint32_t b_unit_off(int r, int u) {
     return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((u ^ (r & 7)) << 4));
 }
 
-// One IQ2 chunk (8 weights) -> 8 bf16 (16 bytes): d(2s+1)/8 * G[a][i] * (+-1), rounded.
-__device__ __forceinline__ uint4 iq2_chunk_bf16(uint32_t idx, uint32_t S, int c, float db, const float* tabp) {
+// IQ2 chunk (8 weights) -> 8 bf16 (16 bytes): d(2s+1)/8 * G[a][i] * (+-1).
+// The grid holds at most four distinct magnitudes v_c, so each group of 32
+// weights first rounds its four candidates d(2s+1)/8 * v_c to bf16 (the
+// binary32 products are exact: at most 22 significant bits), held as bytes
+// 0..7 of (cand01, cand23).  Row a of the selector table gives, per pair of
+// weights, the byte-permute selector that picks the two rounded candidates;
+// rounding is symmetric, so the signs are applied to the picked pairs:
+// sg * C_j places sign bit 2j at bit 15 and bit 2j+1 at bit 31 (the two
+// shifted copies of the 8-bit sign byte do not overlap, so no carries).
+__device__ __forceinline__ uint4 iq2_chunk_bf16(uint32_t idx, uint32_t S, int c, uint32_t cand01, uint32_t cand23,
+                                               const unsigned char* selp) {
     const uint32_t a = (idx >> (8 * c)) & 255u;
     uint32_t sg = (S >> (7 * c)) & 127u;
     sg |= ((uint32_t)__popc(sg) & 1u) << 7;
-    const float* trow = tabp + a * 64;
-    const float4 g0 = *reinterpret_cast<const float4*>(trow);
-    const float4 g1 = *reinterpret_cast<const float4*>(trow + 32);
-    float w[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = __uint_as_float(__float_as_uint(db * w[i]) ^ ((sg << (31 - i)) & 0x80000000u));
-    return make_uint4(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]), pack_bf16x2(w[4], w[5]), pack_bf16x2(w[6], w[7]));
+    const uint2 sl = *reinterpret_cast<const uint2*>(selp + a * (kGSelRep * 8));
+    return make_uint4(__byte_perm(cand01, cand23, sl.x) ^ ((sg * 0x40008000u) & 0x80008000u),
+                      __byte_perm(cand01, cand23, sl.x >> 16) ^ ((sg * 0x10002000u) & 0x80008000u),
+                      __byte_perm(cand01, cand23, sl.y) ^ ((sg * 0x04000800u) & 0x80008000u),
+                      __byte_perm(cand01, cand23, sl.y >> 16) ^ ((sg * 0x01000200u) & 0x80008000u));
 }
 
+// Eight 2-bit codes (bits 2i of x, i = 0..7) -> 8 bf16 of (d sc) q - dmin m.
+// Code i becomes the binary32 2^(23-2i) + q with one AND-OR (biased exponent
+// 150 - 2i, the code left in place in the mantissa); subtracting 2^(23-2i) gives
+// q exactly, and one FMA gives the binary32 weight before the bf16 rounding.
+__device__ __forceinline__ uint4 q2_unit_bf16(uint32_t x, float2 sc2, float2 nmn2) {
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int i0 = 2 * j, i1 = 2 * j + 1;
+        const float f0 = __uint_as_float(((150u - 2u * i0) << 23) | (x & (3u << (2 * i0))));
+        const float f1 = __uint_as_float(((150u - 2u * i1) << 23) | (x & (3u << (2 * i1))));
+        const float2 q = fadd2(make_float2(f0, f1), make_float2(-__uint_as_float((150u - 2u * i0) << 23),
+                                                                -__uint_as_float((150u - 2u * i1) << 23)));
+        const float2 w = ffma2(sc2, q, nmn2);
+        o[j] = pack_bf16x2(w.x, w.y);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// One dequantizing thread's packed weights for one k step (64 weights of one B row).
+struct BFrag {
+    uint4 q;        // IQ2: two (grid indices, signs+scale) pairs; Q2: 64 codes
+    uint32_t a0;    // IQ2: d (binary16 bits); Q2: four scale bytes
+    uint32_t a1;    // Q2: d | dmin << 16
+};
+
+// Warp roles: 0 TMA, 1 MMA, 2..9 dequantize B, 10..17 epilogue.
 template <int MODE>
 __global__ void __launch_bounds__(kGThreads, 1)
-    k_moe_gemm(const __grid_constant__ CUtensorMap tmapA, GemmArgs a) {
+    k_moe_gemm(const __grid_constant__ CUtensorMap tmapA, const __grid_constant__ CUtensorMap tmapB0,
+               const __grid_constant__ CUtensorMap tmapB1, GemmArgs a) {
     extern __shared__ __align__(1024) unsigned char g_smem_raw[];
     // 1024-byte aligned stages (the swizzle pattern repeats every 1024 bytes)
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(g_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    unsigned char* stA = base;                                   // kGStages x 16 KB
+    unsigned char* stA = base;                                   // kGStages x 32 KB
     unsigned char* stB = base + kGStages * kGAStage;              // kGStages x 32 KB
-    float* tab = reinterpret_cast<float*>(stB + kGStages * kGBStage);
+    unsigned char* seltab = stB + kGStages * kGBStage;            // [256][kGSelRep] x 8-byte selectors
     __shared__ GemmSmem S;
 
+    constexpr bool kRouted = MODE == kModeGateUp || MODE == kModeDown;
+    constexpr bool kGateUp = MODE == kModeGateUp || MODE == kModeShGateUp;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = a.D.H, I = a.D.I;
-    const int K = (MODE == kModeGateUp || MODE == kModeShGateUp) ? H : I;
+    const int K = kGateUp ? H : I;
     const int KS = K / kGBK;
-    const int NB = (MODE == kModeGateUp || MODE == kModeShGateUp) ? I / 128 : H / kGBN;
-    const bool routed = MODE == kModeGateUp || MODE == kModeDown;
+    const int NB = kGateUp ? I / 128 : H / kGBN;
 
     if (tid == 0) {
         for (int s = 0; s < kGStages; ++s) {
             mbar_init(&S.fullA[s], 1);
-            mbar_init(&S.fullB[s], 8);
+            mbar_init(&S.fullB[s], kGDqWarps);
             mbar_init(&S.empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&S.accF[b], 1);
-            mbar_init(&S.accE[b], 4);
-        }
+        mbar_init(&S.accF, 1);
+        mbar_init(&S.accE, kGEpiWarps);
         mbar_init(&S.done, 1);
         S.abort = 0;
         fence_barrier_init();
     }
-    if (routed)
-        for (int e = tid; e <= a.D.E; e += kGThreads) S.mtp[e] = __ldg(a.mt_prefix + e);
     if (MODE == kModeGateUp) {
-        for (int q = tid; q < 512; q += kGThreads) {
-            const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(a.W.grid_u8) + q);
-            const int g = q >> 1, hf = q & 1;
-            const float4 f = make_float4((float)(v & 0xffu), (float)((v >> 8) & 0xffu), (float)((v >> 16) & 0xffu),
-                                         (float)(v >> 24));
+        // magnitude classes of the grid bytes (stage A is free until the pipeline starts)
+        int* present = reinterpret_cast<int*>(stA);
+        int* cls = present + 256;
+        for (int v = tid; v < 256; v += kGThreads) present[v] = 0;
+        __syncthreads();
+        for (int q = tid; q < 2048; q += kGThreads) present[a.W.grid_u8[q]] = 1;
+        __syncthreads();
+        if (tid == 0) {
+            int nv = 0;
+            for (int v = 0; v < 256; ++v) {
+                cls[v] = nv < 4 ? nv : 3;
+                if (present[v]) {
+                    if (nv < 4) S.gval[nv] = (float)v;
+                    ++nv;
+                }
+            }
+            for (int c = nv; c < 4; ++c) S.gval[c] = 0.f;
+            S.nval = nv;
+            if (nv > 4) {
+                set_err(a.err, kErrGrid);
+                S.abort = 1;
+            }
+        }
+        __syncthreads();
+        for (int row = tid; row < 256; row += kGThreads) {
+            uint32_t sel[4];
 #pragma unroll
-            for (int p = 0; p < 8; ++p) *reinterpret_cast<float4*>(tab + g * 64 + hf * 32 + p * 4) = f;
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t ca = (uint32_t)cls[a.W.grid_u8[row * 8 + 2 * j]];
+                const uint32_t cb = (uint32_t)cls[a.W.grid_u8[row * 8 + 2 * j + 1]];
+                sel[j] = 0x1010u + 0x22u * ca + 0x2200u * cb;   // bytes 2c, 2c+1 hold candidate c
+            }
+            const uint2 ent = make_uint2(sel[0] | (sel[1] << 16), sel[2] | (sel[3] << 16));
+#pragma unroll
+            for (int p = 0; p < kGSelRep; ++p)
+                *reinterpret_cast<uint2*>(seltab + row * (kGSelRep * 8) + p * 8) = ent;
         }
     }
     if (warp == 1) {
@@ -349,20 +418,30 @@ __global__ void __launch_bounds__(kGThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
-    const int total_mt = routed ? S.mtp[a.D.E] : (a.n_rows + kGBM - 1) / kGBM;
+    const int total_mt = kRouted ? __ldg(a.mt_prefix + a.D.E) : (a.n_rows + kGBM - 1) / kGBM;
     const int ntiles = total_mt * NB;
 
     if (warp == 0) {
-        // ------------------------------------------------ A tiles (TMA)
+        // ------------------------------------------------ A tiles (and shared-expert B tiles) by TMA
         uint32_t it = 0;
         for (int tile = blockIdx.x; tile < ntiles && !g_aborted(S); tile += gridDim.x) {
-            const TileInfo ti = tile_info<MODE>(S, a, tile, NB);
+            const TileInfo ti = tile_info<MODE>(a, tile, NB);
+            const bool two = ti.mvalid > kGHalf;
             for (int ks = 0; ks < KS; ++ks, ++it) {
                 const int s = it % kGStages;
                 if (!mbar_wait(&S.empty[s], ((it / kGStages) & 1) ^ 1, a.err)) { g_set_abort(S); break; }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&S.fullA[s], kGAStage);
+                    mbar_arrive_expect_tx(&S.fullA[s], (two ? 2 : 1) * kGAHalf + (kRouted ? 0 : kGBStage));
                     tma_load_2d(stA + s * kGAStage, &tmapA, ks * kGBK, ti.row0, &S.fullA[s]);
+                    if (two) tma_load_2d(stA + s * kGAStage + kGAHalf, &tmapA, ks * kGBK, ti.row0 + kGHalf, &S.fullA[s]);
+                    if (MODE == kModeShGateUp) {   // rows 0..127: gate rows, 128..255: up rows of n tile nb
+                        tma_load_3d(stB + s * kGBStage, &tmapB0, 0, 8 * ks, 16 * ti.nb, &S.fullA[s]);
+                        tma_load_3d(stB + s * kGBStage + kGBStage / 2, &tmapB1, 0, 8 * ks, 16 * ti.nb, &S.fullA[s]);
+                    } else if (MODE == kModeShDown) {
+                        tma_load_3d(stB + s * kGBStage, &tmapB0, 0, 8 * ks, 32 * ti.nb, &S.fullA[s]);
+                        tma_load_3d(stB + s * kGBStage + kGBStage / 2, &tmapB0, 0, 8 * ks, 32 * ti.nb + 16,
+                                    &S.fullA[s]);
+                    }
                 }
                 __syncwarp();
             }
@@ -371,180 +450,205 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const uint32_t j0 = it > (uint32_t)kGStages ? it - kGStages : 0;
         for (uint32_t j = j0; j < it; ++j) mbar_wait(&S.fullA[j % kGStages], (j / kGStages) & 1, a.err);
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issue
-        const uint32_t idesc = umma_idesc_bf16(kGBM, kGBN);
+        // ------------------------------------------------ MMA issue: two 128 x 256 x 16 MMAs per k16 share B
+        const uint32_t idesc = umma_idesc_bf16(kGHalf, kGBN);
         uint32_t it = 0, lt = 0;
         for (int tile = blockIdx.x; tile < ntiles && !g_aborted(S); tile += gridDim.x, ++lt) {
-            const uint32_t ab = lt & 1, aph = (lt >> 1) & 1;
-            if (!mbar_wait(&S.accE[ab], aph ^ 1, a.err)) { g_set_abort(S); break; }
+            const TileInfo ti = tile_info<MODE>(a, tile, NB);
+            const bool two = ti.mvalid > kGHalf;
+            if (!mbar_wait(&S.accE, (lt & 1) ^ 1, a.err)) { g_set_abort(S); break; }
             tc_fence_after();
-            const uint32_t dtm = tmem + ab * kGBN;
             for (int ks = 0; ks < KS; ++ks, ++it) {
                 const int s = it % kGStages;
                 const uint32_t ph = (it / kGStages) & 1;
-                if (!mbar_wait(&S.fullA[s], ph, a.err) || !mbar_wait(&S.fullB[s], ph, a.err)) {
+                if (!mbar_wait(&S.fullA[s], ph, a.err) || (kRouted && !mbar_wait(&S.fullB[s], ph, a.err))) {
                     g_set_abort(S);
                     break;
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint64_t da = umma_desc_sw128(smem_addr(stA + s * kGAStage));
-                    const uint64_t db = umma_desc_sw128(smem_addr(stB + s * kGBStage));
+                    const uint64_t da0 = umma_desc_sw128(smem_addr(stA + s * kGAStage));
+                    const uint64_t da1 = umma_desc_sw128(smem_addr(stA + s * kGAStage + kGAHalf));
+                    // dequantized tiles: 128-byte swizzle; shared-expert tiles: core-matrix blocks as stored
+                    const uint64_t db = kRouted ? umma_desc_sw128(smem_addr(stB + s * kGBStage))
+                                                : umma_desc_core(smem_addr(stB + s * kGBStage));
+                    // K advance per 16 elements: 32 bytes in a swizzled row, two 128-byte blocks unswizzled
+                    const uint32_t bstep = kRouted ? 2u : 16u;
 #pragma unroll
-                    for (int kk = 0; kk < kGBK / 16; ++kk)
-                        umma_bf16(dtm, da + 2 * kk, db + 2 * kk, idesc, (ks | kk) != 0);
+                    for (int kk = 0; kk < kGBK / 16; ++kk) {
+                        umma_bf16(tmem, da0 + 2 * kk, db + bstep * kk, idesc, (ks | kk) != 0);
+                        if (two) umma_bf16(tmem + kGBN, da1 + 2 * kk, db + bstep * kk, idesc, (ks | kk) != 0);
+                    }
                     umma_commit(&S.empty[s]);
                 }
                 __syncwarp();
             }
             if (g_aborted(S)) break;
-            if (lane == 0) umma_commit(&S.accF[ab]);
+            if (lane == 0) umma_commit(&S.accF);
             __syncwarp();
         }
         // every issued MMA has finished before TMEM is released
         if (lane == 0) umma_commit(&S.done);
         __syncwarp();
         mbar_wait(&S.done, 0, a.err);
-    } else if (warp < 10) {
+    } else if (warp < 2 + kGDqWarps) {
         // ------------------------------------------------ B tiles (dequantize to bf16)
-        const int r = tid - 64;   // B-tile row 0..255
-        const float* tabp = tab + (lane & 7) * 4;
-        uint32_t it = 0;
-        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(S); tile += gridDim.x) {
-            const TileInfo ti = tile_info<MODE>(S, a, tile, NB);
-            // source row of this thread
+        if (kRouted) {
+            const int r = tid - 64;   // B-tile row 0..255
+            const unsigned char* selp = seltab + (lane & 15) * 8;
+            float2 gv01 = make_float2(0.f, 0.f), gv23 = make_float2(0.f, 0.f);
+            if (MODE == kModeGateUp) {
+                gv01 = make_float2(S.gval[0], S.gval[1]);
+                gv23 = make_float2(S.gval[2], S.gval[3]);
+            }
+            const int my_tiles = (int)blockIdx.x < ntiles ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+            const int total = my_tiles * KS;
+            // load cursor: tile, k step and this row's packed-weight pointers
+            int ctile = blockIdx.x, cks = 0;
             const uint8_t* qs = nullptr;
             const uint16_t* dq = nullptr;
             const uint32_t* scp = nullptr;
             const uint32_t* ddp = nullptr;
-            const __nv_bfloat16* bfrow = nullptr;
-            int row = 0;
-            if (MODE == kModeGateUp) {
-                row = 128 * ti.nb + (r & 127);
+            auto set_src = [&](int tile) {
+                const TileInfo ti = tile_info<MODE>(a, tile, NB);
                 const size_t e = (size_t)ti.e;
-                qs = (r < 128 ? a.W.gate_qs : a.W.up_qs) + e * a.W.iq2_qs_stride + (size_t)(row >> 5) * (H / 64) * 512 +
-                     (row & 31) * 16;
-                dq = (r < 128 ? a.W.gate_d : a.W.up_d) + e * a.W.iq2_d_stride + (size_t)(row >> 5) * (H / 256) * 32 +
-                     (row & 31);
-            } else if (MODE == kModeDown) {
-                row = kGBN * ti.nb + r;
-                const size_t e = (size_t)ti.e;
-                const int nkt = I / 64, nsb = I >= 256 ? I / 256 : 1;
-                qs = a.W.down_q + e * a.W.q2_q_stride + ((size_t)(row >> 5) * nkt * 32 + (row & 31)) * 16;
-                scp = a.W.down_sc + e * a.W.q2_sc_stride + (size_t)(row >> 5) * nkt * 32 + (row & 31);
-                ddp = a.W.down_dd + e * a.W.q2_dd_stride + (size_t)(row >> 5) * nsb * 32 + (row & 31);
-            } else if (MODE == kModeShGateUp) {
-                row = 128 * ti.nb + (r & 127);
-                bfrow = (r < 128 ? a.W.sh_gate : a.W.sh_up) + (size_t)(row >> 3) * (H / 8) * 64 + (row & 7) * 8;
-            } else {
-                row = kGBN * ti.nb + r;
-                bfrow = a.W.sh_down + (size_t)(row >> 3) * (I / 8) * 64 + (row & 7) * 8;
-            }
-            for (int ks = 0; ks < KS; ++ks, ++it) {
-                // fetch this row's piece of the k step before waiting for the stage
-                uint4 q = make_uint4(0, 0, 0, 0);
-                uint32_t aux0 = 0, aux1 = 0;
-                uint4 bf[8];
                 if (MODE == kModeGateUp) {
-                    q = ld_stream_v4(qs + (size_t)ks * 512);
-                    aux0 = ld_stream_u16(dq + (ks >> 2) * 32);
-                } else if (MODE == kModeDown) {
-                    q = ld_stream_v4(qs + (size_t)ks * 512);
-                    aux0 = ld_stream_u32(scp + ks * 32);
-                    aux1 = ld_stream_u32(ddp + (I >= 256 ? (ks >> 2) : 0) * 32);
+                    const int row = 128 * ti.nb + (r & 127);
+                    qs = (r < 128 ? a.W.gate_qs : a.W.up_qs) + e * a.W.iq2_qs_stride +
+                         (size_t)(row >> 5) * (H / 64) * 512 + (row & 31) * 16;
+                    dq = (r < 128 ? a.W.gate_d : a.W.up_d) + e * a.W.iq2_d_stride + (size_t)(row >> 5) * (H / 256) * 32 +
+                         (row & 31);
                 } else {
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) bf[u] = ld_stream_v4(bfrow + (size_t)(8 * ks + u) * 64);
+                    const int row = kGBN * ti.nb + r;
+                    const int nkt = I / 64, nsb = I >= 256 ? I / 256 : 1;
+                    qs = a.W.down_q + e * a.W.q2_q_stride + ((size_t)(row >> 5) * nkt * 32 + (row & 31)) * 16;
+                    scp = a.W.down_sc + e * a.W.q2_sc_stride + (size_t)(row >> 5) * nkt * 32 + (row & 31);
+                    ddp = a.W.down_dd + e * a.W.q2_dd_stride + (size_t)(row >> 5) * nsb * 32 + (row & 31);
                 }
-                const int s = it % kGStages;
-                if (!mbar_wait(&S.empty[s], ((it / kGStages) & 1) ^ 1, a.err)) { g_set_abort(S); break; }
-                unsigned char* bt = stB + s * kGBStage;
+            };
+            auto fetch = [&](BFrag& f) {
+                f.q = ld_stream_v4(qs + (size_t)cks * 512);
                 if (MODE == kModeGateUp) {
-                    const float d = half_bits(aux0);
-#pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        const uint32_t idx = hf ? q.z : q.x, Sw = hf ? q.w : q.y;
-                        const float db = d * (__uint_as_float(0x4b000001u | ((Sw >> 27) & 0x1eu)) - 8388608.0f) * 0.125f;
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            *reinterpret_cast<uint4*>(bt + b_unit_off(r, 4 * hf + c)) = iq2_chunk_bf16(idx, Sw, c, db, tabp);
-                    }
-                } else if (MODE == kModeDown) {
-                    const float d = half_bits(aux1 & 0xffffu), dmin = half_bits(aux1 >> 16);
-                    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const uint32_t sb = (aux0 >> (8 * (u >> 1))) & 0xffu;
-                        const float sc = d * (float)(sb & 15u), mn = dmin * (float)(sb >> 4);
-                        const uint32_t codes = words[u >> 1] >> (16 * (u & 1));
-                        float w[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) w[i] = fmaf(sc, (float)((codes >> (2 * i)) & 3u), -mn);
-                        *reinterpret_cast<uint4*>(bt + b_unit_off(r, u)) =
-                            make_uint4(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]), pack_bf16x2(w[4], w[5]),
-                                       pack_bf16x2(w[6], w[7]));
-                    }
+                    f.a0 = ld_stream_u16(dq + (cks >> 2) * 32);
                 } else {
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(bt + b_unit_off(r, u)) = bf[u];
+                    f.a0 = ld_stream_u32(scp + cks * 32);
+                    f.a1 = ld_stream_u32(ddp + (I >= 256 ? (cks >> 2) : 0) * 32);
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&S.fullB[s]);
+                if (++cks == KS) {
+                    cks = 0;
+                    ctile += gridDim.x;
+                    if (ctile < ntiles) set_src(ctile);
+                }
+            };
+            constexpr int PD = 4;   // k steps of packed weights in flight
+            BFrag ring[PD];
+            if (total > 0) set_src(ctile);
+#pragma unroll
+            for (int p = 0; p < PD; ++p)
+                if (p < total) fetch(ring[p]);
+            uint32_t it = 0;
+            for (int j0 = 0; j0 < total && !g_aborted(S); j0 += PD) {
+#pragma unroll
+                for (int p = 0; p < PD; ++p) {
+                    if (j0 + p >= total) break;
+                    const BFrag cur = ring[p];
+                    if (j0 + p + PD < total) fetch(ring[p]);
+                    const int s = it % kGStages;
+                    if (!mbar_wait(&S.empty[s], ((it / kGStages) & 1) ^ 1, a.err)) {
+                        g_set_abort(S);
+                        break;
+                    }
+                    unsigned char* bt = stB + s * kGBStage;
+                    if (MODE == kModeGateUp) {
+                        const float d = half_bits(cur.a0);
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const uint32_t idx = hf ? cur.q.z : cur.q.x, Sw = hf ? cur.q.w : cur.q.y;
+                            const float db =
+                                d * (__uint_as_float(0x4b000001u | ((Sw >> 27) & 0x1eu)) - 8388608.0f) * 0.125f;
+                            const float2 db2 = make_float2(db, db);
+                            const float2 c01 = fmul2(db2, gv01), c23 = fmul2(db2, gv23);
+                            const uint32_t cand01 = pack_bf16x2(c01.x, c01.y), cand23 = pack_bf16x2(c23.x, c23.y);
+#pragma unroll
+                            for (int c = 0; c < 4; ++c)
+                                *reinterpret_cast<uint4*>(bt + b_unit_off(r, 4 * hf + c)) =
+                                    iq2_chunk_bf16(idx, Sw, c, cand01, cand23, selp);
+                        }
+                    } else {
+                        const float d = half_bits(cur.a1 & 0xffffu), dmin = half_bits(cur.a1 >> 16);
+                        // two sub-blocks per pass: a full unroll schedules all eight units at once and spills
+#pragma unroll 2
+                        for (int sbk = 0; sbk < 4; ++sbk) {
+                            const uint32_t w = (sbk & 2) ? ((sbk & 1) ? cur.q.w : cur.q.z) : ((sbk & 1) ? cur.q.y : cur.q.x);
+                            const uint32_t sb = (cur.a0 >> (8 * sbk)) & 0xffu;
+                            const float sc = d * (float)(sb & 15u), mn = dmin * (float)(sb >> 4);
+                            const float2 sc2 = make_float2(sc, sc), nmn2 = make_float2(-mn, -mn);
+                            *reinterpret_cast<uint4*>(bt + b_unit_off(r, 2 * sbk)) = q2_unit_bf16(w, sc2, nmn2);
+                            *reinterpret_cast<uint4*>(bt + b_unit_off(r, 2 * sbk + 1)) = q2_unit_bf16(w >> 16, sc2, nmn2);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S.fullB[s]);
+                    ++it;
+                }
             }
         }
     } else {
         // ------------------------------------------------ epilogue (TMEM -> registers -> global)
-        const int qd = warp & 3;          // TMEM lanes 32 qd .. 32 qd + 31
-        const int m = 32 * qd + lane;     // tile row of this thread
+        const int qd = warp & 3;                          // TMEM lanes 32 qd .. 32 qd + 31
+        const int half = (warp - 2 - kGDqWarps) >> 2;     // accumulator (row half) of this warp
+        const int m = kGHalf * half + 32 * qd + lane;     // tile row of this thread
         uint32_t lt = 0;
         for (int tile = blockIdx.x; tile < ntiles && !g_aborted(S); tile += gridDim.x, ++lt) {
-            const TileInfo ti = tile_info<MODE>(S, a, tile, NB);
-            const uint32_t ab = lt & 1, aph = (lt >> 1) & 1;
-            if (!mbar_wait(&S.accF[ab], aph, a.err)) { g_set_abort(S); break; }
+            const TileInfo ti = tile_info<MODE>(a, tile, NB);
+            if (!mbar_wait(&S.accF, lt & 1, a.err)) { g_set_abort(S); break; }
             tc_fence_after();
-            const uint32_t taddr = tmem + ((uint32_t)(32 * qd) << 16) + ab * kGBN;
+            const uint32_t taddr = tmem + ((uint32_t)(32 * qd) << 16) + half * kGBN;
             const bool live = m < ti.mvalid;
-            if (MODE == kModeGateUp || MODE == kModeShGateUp) {
-                __nv_bfloat16* dst = a.out_h + (size_t)(ti.row0 + m) * I + 128 * ti.nb;
+            if (ti.mvalid > kGHalf * half) {   // this half was computed
+                if (kGateUp) {
+                    __nv_bfloat16* dst = a.out_h + (size_t)(ti.row0 + m) * I + 128 * ti.nb;
 #pragma unroll 1
-                for (int c0 = 0; c0 < 128; c0 += 32) {
-                    uint32_t g[32], u[32];
-                    tmem_ld_32x32(taddr + c0, g);
-                    tmem_ld_32x32(taddr + 128 + c0, u);
-                    tmem_wait_ld();
-                    uint32_t hp[16];
+                    for (int c0 = 0; c0 < 128; c0 += 32) {
+                        uint32_t g[32], u[32];
+                        tmem_ld_32x32(taddr + c0, g);
+                        tmem_ld_32x32(taddr + 128 + c0, u);
+                        tmem_wait_ld();
+                        uint32_t hp[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float h0 = silu(__uint_as_float(g[2 * j])) * __uint_as_float(u[2 * j]);
-                        const float h1 = silu(__uint_as_float(g[2 * j + 1])) * __uint_as_float(u[2 * j + 1]);
-                        hp[j] = pack_bf16x2(h0, h1);
-                    }
-                    if (live) {
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+                        for (int j = 0; j < 16; ++j) {
+                            const float h0 = silu(__uint_as_float(g[2 * j])) * __uint_as_float(u[2 * j]);
+                            const float h1 = silu(__uint_as_float(g[2 * j + 1])) * __uint_as_float(u[2 * j + 1]);
+                            hp[j] = pack_bf16x2(h0, h1);
+                        }
+                        if (live) {
+                            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) d4[j] = make_uint4(hp[4 * j], hp[4 * j + 1], hp[4 * j + 2], hp[4 * j + 3]);
+                            for (int j = 0; j < 4; ++j)
+                                d4[j] = make_uint4(hp[4 * j], hp[4 * j + 1], hp[4 * j + 2], hp[4 * j + 3]);
+                        }
                     }
-                }
-            } else {
-                float* dst = a.out_y + (size_t)(ti.row0 + m) * H + kGBN * ti.nb;
+                } else {
+                    float* dst = a.out_y + (size_t)(ti.row0 + m) * H + kGBN * ti.nb;
 #pragma unroll 1
-                for (int c0 = 0; c0 < kGBN; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld_32x32(taddr + c0, v);
-                    tmem_wait_ld();
-                    if (live) {
-                        float4* d4 = reinterpret_cast<float4*>(dst + c0);
+                    for (int c0 = 0; c0 < kGBN; c0 += 32) {
+                        uint32_t v[32];
+                        tmem_ld_32x32(taddr + c0, v);
+                        tmem_wait_ld();
+                        if (live) {
+                            float4* d4 = reinterpret_cast<float4*>(dst + c0);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            d4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                            for (int j = 0; j < 8; ++j)
+                                d4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                    __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                        }
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&S.accE[ab]);
+            if (lane == 0) mbar_arrive(&S.accE);
         }
     }
     tc_fence_before();
@@ -577,20 +681,37 @@ __global__ void k_combine_prefill(Dims D, const float* ys, const float* y, const
 }
 
 // ---------------------------------------------------------------- host side
-size_t gemm_smem_bytes() { return 1024 + (size_t)kGStages * (kGAStage + kGBStage) + kGTabFloats * 4; }
+size_t gemm_smem_bytes() { return 1024 + (size_t)kGStages * (kGAStage + kGBStage) + kGSelBytes; }
+// Static shared memory of the GEMM kernels (the largest of the four modes).
+size_t gemm_static_smem_bytes() {
+    size_t m = 0;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeGateUp>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeDown>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeShGateUp>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeShDown>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    return m > sizeof(GemmSmem) ? m : sizeof(GemmSmem);
+}
 
-static cudaError_t encode_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+static PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
         cudaDriverEntryPointQueryResult q;
         void* p = nullptr;
         cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
-        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p) return cudaErrorNotSupported;
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p) return nullptr;
         fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
     }
+    return fn;
+}
+
+// Row-major bf16 [rows][cols] read as 128-row x 64-column boxes (one tensor-core half) with the 128-byte swizzle.
+static cudaError_t encode_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+    const PFN_cuTensorMapEncodeTiled_v12000 fn = tmap_encoder();
+    if (!fn) return cudaErrorNotSupported;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {kGBK, kGBM};
+    const cuuint32_t box[2] = {kGBK, kGHalf};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -598,8 +719,25 @@ static cudaError_t encode_tmap(CUtensorMap* map, const void* base, uint64_t rows
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// bf16 core-matrix tiles [rows/8][cols/8][8][8] (the shared expert's layout) as a
+// 3-D tensor (64-element core matrix, k chunk, 8-row group); one box is 128 rows
+// x 64 columns and lands in shared memory in the same order (no swizzle).
+static cudaError_t encode_tmap_core(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+    const PFN_cuTensorMapEncodeTiled_v12000 fn = tmap_encoder();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {64, cols / 8, rows / 8};
+    const cuuint64_t strides[2] = {128, (cols / 8) * 128};
+    const cuuint32_t box[3] = {64, kGBK / 8, kGHalf / 8};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int MODE>
-static cudaError_t launch_gemm(const CUtensorMap& map, const GemmArgs& args, int n_sm, cudaStream_t st) {
+static cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
+                               const GemmArgs& args, int n_sm, cudaStream_t st) {
     static bool configured[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -610,7 +748,7 @@ static cudaError_t launch_gemm(const CUtensorMap& map, const GemmArgs& args, int
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
-    k_moe_gemm<MODE><<<n_sm, kGThreads, smem, st>>>(map, args);
+    k_moe_gemm<MODE><<<n_sm, kGThreads, smem, st>>>(mapA, mapB0, mapB1, args);
     return cudaGetLastError();
 }
 
@@ -705,25 +843,29 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
     if ((e = encode_tmap(&mA, ws.Xp, nslots, H)) != cudaSuccess) return e;
     ga.out_h = ws.Hb;
     mk.before();
-    if ((e = launch_gemm<kModeGateUp>(mA, ga, n_sm, st)) != cudaSuccess) return e;
+    if ((e = launch_gemm<kModeGateUp>(mA, mA, mA, ga, n_sm, st)) != cudaSuccess) return e;
     mk.after();
     // routed down: A = Hb [n k][I] -> Y [n k][H]
     if ((e = encode_tmap(&mA, ws.Hb, nslots, D.I)) != cudaSuccess) return e;
     ga.out_y = ws.Y;
     mk.before();
-    if ((e = launch_gemm<kModeDown>(mA, ga, n_sm, st)) != cudaSuccess) return e;
+    if ((e = launch_gemm<kModeDown>(mA, mA, mA, ga, n_sm, st)) != cudaSuccess) return e;
     mk.after();
     if (D.has_shared) {
         ga.n_rows = n;
+        CUtensorMap mB0, mB1;
         if ((e = encode_tmap(&mA, xb, n, H)) != cudaSuccess) return e;
+        if ((e = encode_tmap_core(&mB0, W.sh_gate, D.I, H)) != cudaSuccess) return e;
+        if ((e = encode_tmap_core(&mB1, W.sh_up, D.I, H)) != cudaSuccess) return e;
         ga.out_h = ws.Hs;
         mk.before();
-        if ((e = launch_gemm<kModeShGateUp>(mA, ga, n_sm, st)) != cudaSuccess) return e;
+        if ((e = launch_gemm<kModeShGateUp>(mA, mB0, mB1, ga, n_sm, st)) != cudaSuccess) return e;
         mk.after();
         if ((e = encode_tmap(&mA, ws.Hs, n, D.I)) != cudaSuccess) return e;
+        if ((e = encode_tmap_core(&mB0, W.sh_down, H, D.I)) != cudaSuccess) return e;
         ga.out_y = ws.Ys;
         mk.before();
-        if ((e = launch_gemm<kModeShDown>(mA, ga, n_sm, st)) != cudaSuccess) return e;
+        if ((e = launch_gemm<kModeShDown>(mA, mB0, mB0, ga, n_sm, st)) != cudaSuccess) return e;
         mk.after();
     }
     const int64_t n4 = (int64_t)n * H / 4;

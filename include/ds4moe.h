@@ -123,7 +123,10 @@ ds4moe_status ds4moe_pack_iq2xxs(const float* d_w, int64_t n_weights, const uint
 
 /* ---- loading (device pointers in; repacked into the bound weight buffer) - */
 
-/* Grid magnitudes [256][8] uint8. */
+/* Grid magnitudes [256][8] uint8.  The prefill plan (n_tokens > decode_max)
+ * expects at most four distinct byte values in the grid (the format's grid
+ * uses three); with more, a prefill forward writes no output and records
+ * device error bit 2 (see ds4moe_get_device_error). */
 ds4moe_status ds4moe_set_grid(ds4moe_t* h, const uint8_t* d_grid, void* stream);
 
 /* Router rows [E][H] binary32 and, when has_bias, bias [E] (else NULL). */
@@ -208,7 +211,7 @@ ds4moe_status ds4moe_route_noalloc(ds4moe_t* h, const void* d_x, int32_t n_token
 
 /* Synchronize `stream`, then read and clear the workspace's device error word
  * into *code (0 = none; bit 0 = an index check failed, bit 1 = a bounded
- * wait timed out).  Returns DS4MOE_ERR_DEVICE / DS4MOE_ERR_TIMEOUT when set. */
+ * wait timed out, bit 2 = the grid has more than four distinct magnitudes).  Returns DS4MOE_ERR_DEVICE / DS4MOE_ERR_TIMEOUT when set. */
 ds4moe_status ds4moe_get_device_error(ds4moe_t* h, void* stream, int32_t* code);
 
 /* Message of the last error on the calling thread ("" if none). */
