@@ -17,6 +17,7 @@ __global__ void k_pack_iq2(const float* w, int64_t n_blocks, const uint8_t* grid
 __global__ void k_repack_iq2(const uint8_t* src, int R, int C, uint8_t* qs, uint16_t* dd);
 __global__ void k_repack_q2(const uint8_t* src, int R, int C, uint8_t* q, uint32_t* sc, uint32_t* dd);
 __global__ void k_repack_bf16(const uint4* src, int R, int C, uint4* dst);
+__global__ void k_interleave_router(const float* W, int E, int H, float* W2);
 __global__ void k_dequant_iq2(const uint8_t* qs, const uint16_t* dd, const uint8_t* grid, int R, int C, float* out_f,
                               __nv_bfloat16* out_b);
 __global__ void k_dequant_q2(const uint8_t* q, const uint32_t* sc, const uint32_t* dd, int R, int C, float* out_f,
@@ -87,7 +88,7 @@ struct ds4moe {
     int decode_max;
     int n_sm;
     // weight buffer layout
-    size_t off_grid, off_Wr, off_br, off_gate_qs, off_gate_d, off_up_qs, off_up_d, off_down_q, off_down_sc,
+    size_t off_grid, off_Wr, off_Wr2, off_br, off_gate_qs, off_gate_d, off_up_qs, off_up_d, off_down_q, off_down_sc,
         off_down_dd, off_sh_gate, off_sh_up, off_sh_down, weight_bytes;
     size_t iq2_qs_stride, iq2_d_stride, q2_q_stride, q2_sc_stride, q2_dd_stride;
     uint8_t* weights = nullptr;
@@ -142,6 +143,7 @@ struct ds4moe {
         const uint8_t* b = weights;
         W.grid_u8 = b + off_grid;
         W.W_r = reinterpret_cast<const float*>(b + off_Wr);
+        W.W_r2 = shape.max_tokens > decode_max ? reinterpret_cast<const float*>(b + off_Wr2) : nullptr;
         W.b_r = shape.has_bias ? reinterpret_cast<const float*>(b + off_br) : nullptr;
         W.gate_qs = b + off_gate_qs;
         W.gate_d = reinterpret_cast<const uint16_t*>(b + off_gate_d);
@@ -272,6 +274,7 @@ ds4moe_status ds4moe_create(const ds4moe_shape* s, ds4moe_t** out) {
     size_t o = 0;
     h->off_grid = o; o += align256(256 * 8);
     h->off_Wr = o; o += align256(E * H * 4);
+    h->off_Wr2 = o; o += align256(s->max_tokens > h->decode_max ? (E + 1) / 2 * 2 * H * 4 : 0);
     h->off_br = o; o += align256(E * 4);
     h->off_gate_qs = o; o += align256(E * h->iq2_qs_stride);
     h->off_gate_d = o; o += align256(E * h->iq2_d_stride * 2);
@@ -362,6 +365,13 @@ ds4moe_status ds4moe_set_router(ds4moe_t* h, const float* d_W, const float* d_bi
     cudaStream_t st = (cudaStream_t)stream;
     const size_t E = h->D.E, H = h->D.H;
     cudaError_t ce = cudaMemcpyAsync(h->weights + h->off_Wr, d_W, E * H * 4, cudaMemcpyDeviceToDevice, st);
+    if (ce == cudaSuccess && h->shape.max_tokens > h->decode_max) {
+        const int64_t m = (int64_t)(E + 1) / 2 * H;
+        k_interleave_router<<<(unsigned)((m + 255) / 256), 256, 0, st>>>(
+            reinterpret_cast<const float*>(h->weights + h->off_Wr), (int)E, (int)H,
+            reinterpret_cast<float*>(h->weights + h->off_Wr2));
+        ce = cudaGetLastError();
+    }
     if (ce == cudaSuccess && d_bias)
         ce = cudaMemcpyAsync(h->weights + h->off_br, d_bias, E * 4, cudaMemcpyDeviceToDevice, st);
     if (ce != cudaSuccess) return cuda_fail(ce, "set_router copy");

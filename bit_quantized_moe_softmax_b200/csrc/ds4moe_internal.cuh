@@ -36,6 +36,7 @@ enum : uint32_t { kErrBounds = 1u, kErrTimeout = 2u, kErrGrid = 4u };
 struct Weights {
     const uint8_t* grid_u8;     // [256][8]
     const float* W_r;           // [E][H]
+    const float* W_r2;          // [ceil(E/2)][H][2]: expert pairs interleaved per column (prefill plan), or nullptr
     const float* b_r;           // [E] or nullptr
     const uint8_t* gate_qs;     // IQ2 payload, expert stride iq2_qs_stride bytes
     const uint16_t* gate_d;     // IQ2 d, expert stride iq2_d_stride elements
@@ -107,6 +108,12 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     return v;
 }
 
+__device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
+    uint2 v;
+    asm("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
     uint32_t v;
     asm("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
@@ -117,6 +124,14 @@ __device__ __forceinline__ uint32_t ld_stream_u16(const void* p) {
     unsigned short v;
     asm("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
     return v;
+}
+
+// One 32-byte global store (sm_100 256-bit vector store).
+__device__ __forceinline__ void st_global_v8(void* p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4,
+                                             uint32_t a5, uint32_t a6, uint32_t a7) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a0), "r"(a1), "r"(a2), "r"(a3),
+                 "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+                 : "memory");
 }
 
 // Packed binary32 pair multiply (sm_100): d = a * b elementwise.
@@ -239,6 +254,8 @@ __device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-__device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
+// silu(z) = z / (1 + e^-z) with the fast exponential and reciprocal (relative
+// error a few ulp of binary32; e^-z = inf gives -0 or 0, the limit).
+__device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 }  // namespace ds4

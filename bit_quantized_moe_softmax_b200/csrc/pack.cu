@@ -177,6 +177,18 @@ __global__ void k_repack_bf16(const uint4* __restrict__ src, int R, int C, uint4
     dst[((int64_t)(r >> 3) * nc8 + c8) * 8 + (r & 7)] = src[gid];
 }
 
+// Router rows [E][H] -> expert pairs interleaved per column [ceil(E/2)][H][2]
+// (a missing partner of an odd last expert reads as zero).
+__global__ void k_interleave_router(const float* __restrict__ W, int E, int H, float* __restrict__ W2) {
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t npairs = (E + 1) / 2;
+    if (gid >= npairs * H) return;
+    const int p = (int)(gid / H), c = (int)(gid % H);
+    const int e0 = 2 * p, e1 = 2 * p + 1;
+    W2[2 * gid] = W[(int64_t)e0 * H + c];
+    W2[2 * gid + 1] = e1 < E ? W[(int64_t)e1 * H + c] : 0.f;
+}
+
 // Inverse views for the dequant hook: expert matrix -> row-major values.
 __global__ void k_dequant_iq2(const uint8_t* __restrict__ qs, const uint16_t* __restrict__ dd,
                               const uint8_t* __restrict__ grid, int R, int C, float* out_f, __nv_bfloat16* out_b) {

@@ -26,62 +26,104 @@
 namespace ds4 {
 
 // ---------------------------------------------------------------- router
-// CTA: 16 warps as 4 token groups x 4 expert groups, warp tile 8 x 8 -> CTA
-// tile 32 tokens x 32 experts.  For every 128-column step the CTA stages the
-// 32 x 128 slices of x and W_r in shared memory; lane L multiplies columns
-// 4L .. 4L+3 of the slice into its chain (fma in column order).
-constexpr int kRP_T = 32, kRP_E = 32;
+// CTA: 16 warps as 4 token groups x 4 expert groups, warp tile 8 tokens x 8
+// experts (4 expert pairs) -> CTA tile 32 tokens x 32 experts.  The 32 x 128
+// slices of x and of the pair-interleaved router rows (W_r2: for each column the
+// weights of experts 2p and 2p+1 side by side) for each 128-column step stream
+// into a kRP_S-stage shared-memory ring with 16-byte asynchronous copies (rows
+// past n or E are zero-filled).  Lane L multiplies columns 4L .. 4L+3 of the
+// slice into its chain, fma in column order; one packed FMA advances the
+// chains of an expert pair, whose weights arrive as adjacent words.
+constexpr int kRP_T = 32, kRP_E = 32, kRP_S = 4;
 
-__global__ void __launch_bounds__(512) k_router_prefill(Weights W, Dims D, const void* x, int n, float* logits) {
-    __shared__ __align__(16) float xs[kRP_T][128];
-    __shared__ __align__(16) float wsm[kRP_E][128];
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <bool BF16X>
+__global__ void __launch_bounds__(512, 1) k_router_prefill(Weights W, Dims D, const void* x, int n, float* logits) {
+    constexpr int XB = BF16X ? 2 : 4;                       // bytes per x element
+    constexpr int XSTAGE = kRP_T * 128 * XB, WSTAGE = kRP_E * 128 * 4;
+    extern __shared__ __align__(16) unsigned char rp_smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t0 = blockIdx.x * kRP_T, e0 = blockIdx.y * kRP_E;
-    const int wt = (warp & 3) * 8, we = (warp >> 2) * 8;   // warp's 8 tokens / 8 experts in the CTA tile
-    const int H = D.H, E = D.E;
+    const int wt = (warp & 3) * 8, wq = (warp >> 2) * 4;   // warp's 8 tokens / 4 expert pairs in the CTA tile
+    const int H = D.H, E = D.E, steps = H / 128;
+    const int npairs = (E + 1) / 2, p0 = e0 / 2;
+    const unsigned char* xb = reinterpret_cast<const unsigned char*>(x);
+    const unsigned char* w2 = reinterpret_cast<const unsigned char*>(W.W_r2);
+
+    auto issue = [&](int i) {
+        unsigned char* xs = rp_smem + (i % kRP_S) * (XSTAGE + WSTAGE);
+        unsigned char* ws = xs + XSTAGE;
+        // x: 32 rows x (128 * XB) bytes
+        for (int q = tid; q < kRP_T * 8 * XB; q += 512) {
+            const int row = q / (8 * XB), c = q % (8 * XB);
+            const int t = t0 + row;
+            const bool ok = t < n;
+            cp_async16(xs + row * 128 * XB + 16 * c, xb + ((int64_t)(ok ? t : 0) * H + 128 * i) * XB + 16 * c, ok);
+        }
+        // W_r2: 16 expert pairs x 1024 bytes
+        for (int q = tid; q < (kRP_E / 2) * 64; q += 512) {
+            const int pr = q >> 6, c = q & 63;
+            const int p = p0 + pr;
+            const bool ok = p < npairs;
+            // 16-byte chunk c holds columns 2c, 2c+1 of the pair; lane L reads chunks 2L and 2L+1,
+            // stored 512 bytes apart so that each read of the warp is one contiguous 512-byte run
+            cp_async16(ws + pr * 1024 + (c & 1) * 512 + (c >> 1) * 16,
+                       w2 + ((int64_t)(ok ? p : 0) * H + 128 * i) * 8 + 16 * c, ok);
+        }
+    };
+
     float2 acc[8][4];   // [token][expert pair]
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b) acc[a][b] = make_float2(0.f, 0.f);
-    for (int i = 0; i < H / 128; ++i) {
-        // stage: 32 rows x 128 floats each = 1024 float4 per matrix, 2 per thread
-        for (int q = tid; q < kRP_T * 32; q += 512) {
-            const int row = q >> 5, c4 = q & 31;
-            const int t = t0 + row, e = e0 + row;
-            float4 xv = make_float4(0.f, 0.f, 0.f, 0.f), wv = xv;
-            if (t < n) {
-                const int64_t idx = (int64_t)t * H + 128 * i + 4 * c4;
-                if (D.act_bf16) {
-                    const uint2 v = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(x) + idx));
-                    xv = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
-                                     __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
-                } else {
-                    xv = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + idx));
-                }
-            }
-            if (e < E) wv = __ldg(reinterpret_cast<const float4*>(W.W_r + (int64_t)e * H + 128 * i + 4 * c4));
-            *reinterpret_cast<float4*>(&xs[row][4 * c4]) = xv;
-            *reinterpret_cast<float4*>(&wsm[row][4 * c4]) = wv;
+#pragma unroll
+    for (int i = 0; i < kRP_S - 1; ++i) {
+        if (i < steps) issue(i);
+        cp_async_commit();
+    }
+    for (int i = 0; i < steps; ++i) {
+        cp_async_wait<kRP_S - 2>();
+        __syncthreads();   // step i has landed everywhere; step i-1's stage is free
+        if (i + kRP_S - 1 < steps) issue(i + kRP_S - 1);
+        cp_async_commit();
+        const unsigned char* xs = rp_smem + (i % kRP_S) * (XSTAGE + WSTAGE);
+        const float* ws = reinterpret_cast<const float*>(xs + XSTAGE);
+        float4 wp[4][2];   // [pair][columns (0,1) | (2,3)] as (w_e, w_e+1) pairs
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            wp[b][0] = *reinterpret_cast<const float4*>(ws + (wq + b) * 256 + 4 * lane);
+            wp[b][1] = *reinterpret_cast<const float4*>(ws + (wq + b) * 256 + 128 + 4 * lane);
         }
-        __syncthreads();
-        float4 xv[8], wv[8];
-#pragma unroll
-        for (int a = 0; a < 8; ++a) xv[a] = *reinterpret_cast<const float4*>(&xs[wt + a][4 * lane]);
-#pragma unroll
-        for (int b = 0; b < 8; ++b) wv[b] = *reinterpret_cast<const float4*>(&wsm[we + b][4 * lane]);
 #pragma unroll
         for (int a = 0; a < 8; ++a) {
+            float4 xv;
+            if (BF16X) {
+                const uint2 v = *reinterpret_cast<const uint2*>(xs + ((wt + a) * 128 + 4 * lane) * 2);
+                xv = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                                 __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+            } else {
+                xv = *reinterpret_cast<const float4*>(xs + ((wt + a) * 128 + 4 * lane) * 4);
+            }
+            const float2 x0 = make_float2(xv.x, xv.x), x1 = make_float2(xv.y, xv.y);
+            const float2 x2 = make_float2(xv.z, xv.z), x3 = make_float2(xv.w, xv.w);
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-                acc[a][b] = ffma2(make_float2(xv[a].x, xv[a].x), make_float2(wv[2 * b].x, wv[2 * b + 1].x), acc[a][b]);
-                acc[a][b] = ffma2(make_float2(xv[a].y, xv[a].y), make_float2(wv[2 * b].y, wv[2 * b + 1].y), acc[a][b]);
-                acc[a][b] = ffma2(make_float2(xv[a].z, xv[a].z), make_float2(wv[2 * b].z, wv[2 * b + 1].z), acc[a][b]);
-                acc[a][b] = ffma2(make_float2(xv[a].w, xv[a].w), make_float2(wv[2 * b].w, wv[2 * b + 1].w), acc[a][b]);
+                acc[a][b] = ffma2(x0, make_float2(wp[b][0].x, wp[b][0].y), acc[a][b]);
+                acc[a][b] = ffma2(x1, make_float2(wp[b][0].z, wp[b][0].w), acc[a][b]);
+                acc[a][b] = ffma2(x2, make_float2(wp[b][1].x, wp[b][1].y), acc[a][b]);
+                acc[a][b] = ffma2(x3, make_float2(wp[b][1].z, wp[b][1].w), acc[a][b]);
             }
         }
-        __syncthreads();
     }
+    cp_async_wait<0>();
     // butterfly over the 32 chains, then one lane writes each logit
 #pragma unroll
     for (int a = 0; a < 8; ++a) {
@@ -94,13 +136,43 @@ __global__ void __launch_bounds__(512) k_router_prefill(Weights W, Dims D, const
                 hi = hi + __shfl_xor_sync(0xffffffffu, hi, m);
             }
             const int t = t0 + wt + a;
-            const int e = e0 + we + 2 * b;
+            const int e = e0 + 2 * (wq + b);
             if (lane == ((a * 4 + b) & 31) && t < n) {
                 if (e < E) logits[(int64_t)t * E + e] = W.b_r ? lo + W.b_r[e] : lo;
                 if (e + 1 < E) logits[(int64_t)t * E + e + 1] = W.b_r ? hi + W.b_r[e + 1] : hi;
             }
         }
     }
+}
+
+// Launch of the router for n tokens (stage ring in dynamic shared memory).
+static cudaError_t launch_router_prefill(const Weights& W, const Dims& D, const void* x, int n, float* logits,
+                                         cudaStream_t st) {
+    const dim3 grid((n + kRP_T - 1) / kRP_T, (D.E + kRP_E - 1) / kRP_E);
+    if (D.act_bf16) {
+        const int smem = kRP_S * (kRP_T * 128 * 2 + kRP_E * 128 * 4);
+        static bool configured[64] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev < 64 && !configured[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(k_router_prefill<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return e;
+            configured[dev] = true;
+        }
+        k_router_prefill<true><<<grid, 512, smem, st>>>(W, D, x, n, logits);
+    } else {
+        const int smem = kRP_S * (kRP_T * 128 * 4 + kRP_E * 128 * 4);
+        static bool configured[64] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev < 64 && !configured[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(k_router_prefill<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return e;
+            configured[dev] = true;
+        }
+        k_router_prefill<false><<<grid, 512, smem, st>>>(W, D, x, n, logits);
+    }
+    return cudaGetLastError();
 }
 
 __global__ void __launch_bounds__(256) k_topk_prefill(Dims D, const float* logits, int n, int32_t* ids, float* wts) {
@@ -120,11 +192,11 @@ constexpr int kGStages = 3;
 constexpr int kGAHalf = kGHalf * kGBK * 2;    // 16 KB
 constexpr int kGAStage = 2 * kGAHalf;         // 32 KB
 constexpr int kGBStage = kGBN * kGBK * 2;     // 32 KB
-constexpr int kGDqWarps = 8, kGEpiWarps = 8;
+constexpr int kGDqWarps = 16, kGEpiWarps = 8;  // two dequantizing threads per B row
 constexpr int kGWarps = 2 + kGDqWarps + kGEpiWarps;
 constexpr int kGThreads = kGWarps * 32;
-constexpr int kGSelRep = 16;                  // selector-table copies: conflict-free 8-byte reads
-constexpr int kGSelBytes = 256 * kGSelRep * 8;
+constexpr int kGSelRep = 8;                   // selector-table copies: conflict-free 16-byte reads
+constexpr int kGSelBytes = 256 * kGSelRep * 16;
 constexpr uint32_t kGTmemCols = 512;          // two 128-lane x 256-column binary32 accumulators
 
 // ---------------------------------------------------------------- permutation
@@ -285,30 +357,28 @@ __device__ __forceinline__ TileInfo tile_info(const GemmArgs& a, int tile, int N
     return ti;
 }
 
-// B-tile unit (row r, 16-byte unit u) inside a 128-byte-swizzled K-major tile.
-__device__ __forceinline__ uint32_t b_unit_off(int r, int u) {
-    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((u ^ (r & 7)) << 4));
-}
+// B tiles are K-major core-matrix blocks (no swizzle): row r's 16-byte unit u
+// (k = 8u .. 8u+7 of the 64-column step) sits at (r / 8) * 1024 + u * 128 +
+// (r % 8) * 16, so eight consecutive rows fill one 128-byte line per unit.
+__device__ __forceinline__ uint32_t b_row_off(int r) { return (uint32_t)((r >> 3) * 1024 + (r & 7) * 16); }
 
 // IQ2 chunk (8 weights) -> 8 bf16 (16 bytes): d(2s+1)/8 * G[a][i] * (+-1).
 // The grid holds at most four distinct magnitudes v_c, so each group of 32
 // weights first rounds its four candidates d(2s+1)/8 * v_c to bf16 (the
 // binary32 products are exact: at most 22 significant bits), held as bytes
-// 0..7 of (cand01, cand23).  Row a of the selector table gives, per pair of
-// weights, the byte-permute selector that picks the two rounded candidates;
-// rounding is symmetric, so the signs are applied to the picked pairs:
-// sg * C_j places sign bit 2j at bit 15 and bit 2j+1 at bit 31 (the two
-// shifted copies of the 8-bit sign byte do not overlap, so no carries).
-__device__ __forceinline__ uint4 iq2_chunk_bf16(uint32_t idx, uint32_t S, int c, uint32_t cand01, uint32_t cand23,
-                                               const unsigned char* selp) {
-    const uint32_t a = (idx >> (8 * c)) & 255u;
+// 0..7 of (cand01, cand23).  Row a of the selector table (sl, four 32-bit
+// words loaded by the caller) gives, per pair of weights, the byte-permute
+// selector that picks the two rounded candidates.  Rounding is symmetric, so
+// the signs are applied to the picked pairs: sg * C_j places sign bit 2j at
+// bit 15 and bit 2j+1 at bit 31 (the two shifted copies of the 8-bit sign byte
+// do not overlap, so the multiply has no carries).
+__device__ __forceinline__ uint4 iq2_chunk_bf16(uint4 sl, uint32_t S, int c, uint32_t cand01, uint32_t cand23) {
     uint32_t sg = (S >> (7 * c)) & 127u;
     sg |= ((uint32_t)__popc(sg) & 1u) << 7;
-    const uint2 sl = *reinterpret_cast<const uint2*>(selp + a * (kGSelRep * 8));
     return make_uint4(__byte_perm(cand01, cand23, sl.x) ^ ((sg * 0x40008000u) & 0x80008000u),
-                      __byte_perm(cand01, cand23, sl.x >> 16) ^ ((sg * 0x10002000u) & 0x80008000u),
-                      __byte_perm(cand01, cand23, sl.y) ^ ((sg * 0x04000800u) & 0x80008000u),
-                      __byte_perm(cand01, cand23, sl.y >> 16) ^ ((sg * 0x01000200u) & 0x80008000u));
+                      __byte_perm(cand01, cand23, sl.y) ^ ((sg * 0x10002000u) & 0x80008000u),
+                      __byte_perm(cand01, cand23, sl.z) ^ ((sg * 0x04000800u) & 0x80008000u),
+                      __byte_perm(cand01, cand23, sl.w) ^ ((sg * 0x01000200u) & 0x80008000u));
 }
 
 // Eight 2-bit codes (bits 2i of x, i = 0..7) -> 8 bf16 of (d sc) q - dmin m.
@@ -330,10 +400,10 @@ __device__ __forceinline__ uint4 q2_unit_bf16(uint32_t x, float2 sc2, float2 nmn
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// One dequantizing thread's packed weights for one k step (64 weights of one B row).
+// One dequantizing thread's packed weights for one k step (32 weights of one B row).
 struct BFrag {
-    uint4 q;        // IQ2: two (grid indices, signs+scale) pairs; Q2: 64 codes
-    uint32_t a0;    // IQ2: d (binary16 bits); Q2: four scale bytes
+    uint2 q;        // IQ2: (grid indices, signs+scale) of the group; Q2: 32 codes (two sub-blocks)
+    uint32_t a0;    // IQ2: d (binary16 bits); Q2: the two sub-blocks' scale bytes in bits 0..15
     uint32_t a1;    // Q2: d | dmin << 16
 };
 
@@ -348,7 +418,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         (reinterpret_cast<uintptr_t>(g_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     unsigned char* stA = base;                                   // kGStages x 32 KB
     unsigned char* stB = base + kGStages * kGAStage;              // kGStages x 32 KB
-    unsigned char* seltab = stB + kGStages * kGBStage;            // [256][kGSelRep] x 8-byte selectors
+    unsigned char* seltab = stB + kGStages * kGBStage;            // [256][kGSelRep] x 4 selectors (16 bytes)
     __shared__ GemmSmem S;
 
     constexpr bool kRouted = MODE == kModeGateUp || MODE == kModeDown;
@@ -404,10 +474,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 const uint32_t cb = (uint32_t)cls[a.W.grid_u8[row * 8 + 2 * j + 1]];
                 sel[j] = 0x1010u + 0x22u * ca + 0x2200u * cb;   // bytes 2c, 2c+1 hold candidate c
             }
-            const uint2 ent = make_uint2(sel[0] | (sel[1] << 16), sel[2] | (sel[3] << 16));
+            const uint4 ent = make_uint4(sel[0], sel[1], sel[2], sel[3]);
 #pragma unroll
             for (int p = 0; p < kGSelRep; ++p)
-                *reinterpret_cast<uint2*>(seltab + row * (kGSelRep * 8) + p * 8) = ent;
+                *reinterpret_cast<uint4*>(seltab + row * (kGSelRep * 16) + p * 16) = ent;
         }
     }
     if (warp == 1) {
@@ -469,11 +539,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 if (lane == 0) {
                     const uint64_t da0 = umma_desc_sw128(smem_addr(stA + s * kGAStage));
                     const uint64_t da1 = umma_desc_sw128(smem_addr(stA + s * kGAStage + kGAHalf));
-                    // dequantized tiles: 128-byte swizzle; shared-expert tiles: core-matrix blocks as stored
-                    const uint64_t db = kRouted ? umma_desc_sw128(smem_addr(stB + s * kGBStage))
-                                                : umma_desc_core(smem_addr(stB + s * kGBStage));
-                    // K advance per 16 elements: 32 bytes in a swizzled row, two 128-byte blocks unswizzled
-                    const uint32_t bstep = kRouted ? 2u : 16u;
+                    // B (dequantized or copied) is in core-matrix blocks: K advance per 16 elements is
+                    // two 128-byte blocks; A is 128-byte swizzled: 32 bytes per 16 elements
+                    const uint64_t db = umma_desc_core(smem_addr(stB + s * kGBStage));
+                    constexpr uint32_t bstep = 16u;
 #pragma unroll
                     for (int kk = 0; kk < kGBK / 16; ++kk) {
                         umma_bf16(tmem, da0 + 2 * kk, db + bstep * kk, idesc, (ks | kk) != 0);
@@ -494,8 +563,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
     } else if (warp < 2 + kGDqWarps) {
         // ------------------------------------------------ B tiles (dequantize to bf16)
         if (kRouted) {
-            const int r = tid - 64;   // B-tile row 0..255
-            const unsigned char* selp = seltab + (lane & 15) * 8;
+            // thread -> (B-tile row r, 32-weight group hf of the 64-column k step): lanes 0..15 of a
+            // warp take group 0 of 16 rows, lanes 16..31 group 1, so that each 8-lane phase of a
+            // 16-byte shared store covers 8 rows of one unit (conflict-free)
+            const int dw = warp - 2;
+            const int hf = lane >> 4;
+            const int r = 16 * dw + (lane & 15);
+            const unsigned char* selp = seltab + (lane & 7) * 16;
             float2 gv01 = make_float2(0.f, 0.f), gv23 = make_float2(0.f, 0.f);
             if (MODE == kModeGateUp) {
                 gv01 = make_float2(S.gval[0], S.gval[1]);
@@ -503,7 +577,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             }
             const int my_tiles = (int)blockIdx.x < ntiles ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
             const int total = my_tiles * KS;
-            // load cursor: tile, k step and this row's packed-weight pointers
+            // load cursor: tile, k step and this thread's packed-weight pointers
             int ctile = blockIdx.x, cks = 0;
             const uint8_t* qs = nullptr;
             const uint16_t* dq = nullptr;
@@ -515,23 +589,23 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 if (MODE == kModeGateUp) {
                     const int row = 128 * ti.nb + (r & 127);
                     qs = (r < 128 ? a.W.gate_qs : a.W.up_qs) + e * a.W.iq2_qs_stride +
-                         (size_t)(row >> 5) * (H / 64) * 512 + (row & 31) * 16;
+                         (size_t)(row >> 5) * (H / 64) * 512 + (row & 31) * 16 + hf * 8;
                     dq = (r < 128 ? a.W.gate_d : a.W.up_d) + e * a.W.iq2_d_stride + (size_t)(row >> 5) * (H / 256) * 32 +
                          (row & 31);
                 } else {
                     const int row = kGBN * ti.nb + r;
                     const int nkt = I / 64, nsb = I >= 256 ? I / 256 : 1;
-                    qs = a.W.down_q + e * a.W.q2_q_stride + ((size_t)(row >> 5) * nkt * 32 + (row & 31)) * 16;
+                    qs = a.W.down_q + e * a.W.q2_q_stride + ((size_t)(row >> 5) * nkt * 32 + (row & 31)) * 16 + hf * 8;
                     scp = a.W.down_sc + e * a.W.q2_sc_stride + (size_t)(row >> 5) * nkt * 32 + (row & 31);
                     ddp = a.W.down_dd + e * a.W.q2_dd_stride + (size_t)(row >> 5) * nsb * 32 + (row & 31);
                 }
             };
             auto fetch = [&](BFrag& f) {
-                f.q = ld_stream_v4(qs + (size_t)cks * 512);
+                f.q = ld_stream_v2(qs + (size_t)cks * 512);
                 if (MODE == kModeGateUp) {
                     f.a0 = ld_stream_u16(dq + (cks >> 2) * 32);
                 } else {
-                    f.a0 = ld_stream_u32(scp + cks * 32);
+                    f.a0 = ld_stream_u32(scp + cks * 32) >> (16 * hf);
                     f.a1 = ld_stream_u32(ddp + (I >= 256 ? (cks >> 2) : 0) * 32);
                 }
                 if (++cks == KS) {
@@ -540,7 +614,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     if (ctile < ntiles) set_src(ctile);
                 }
             };
-            constexpr int PD = 4;   // k steps of packed weights in flight
+            constexpr int PD = 3;   // k steps of packed weights in flight
             BFrag ring[PD];
             if (total > 0) set_src(ctile);
 #pragma unroll
@@ -558,33 +632,33 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         g_set_abort(S);
                         break;
                     }
-                    unsigned char* bt = stB + s * kGBStage;
+                    unsigned char* bt = stB + s * kGBStage + b_row_off(r) + hf * 4 * 128;
                     if (MODE == kModeGateUp) {
-                        const float d = half_bits(cur.a0);
+                        // the group's four selector rows first: the loads then overlap instead of
+                        // waiting behind the tile stores (which the compiler cannot reorder)
+                        const uint32_t idx = cur.q.x, Sw = cur.q.y;
+                        uint4 sl[4];
 #pragma unroll
-                        for (int hf = 0; hf < 2; ++hf) {
-                            const uint32_t idx = hf ? cur.q.z : cur.q.x, Sw = hf ? cur.q.w : cur.q.y;
-                            const float db =
-                                d * (__uint_as_float(0x4b000001u | ((Sw >> 27) & 0x1eu)) - 8388608.0f) * 0.125f;
-                            const float2 db2 = make_float2(db, db);
-                            const float2 c01 = fmul2(db2, gv01), c23 = fmul2(db2, gv23);
-                            const uint32_t cand01 = pack_bf16x2(c01.x, c01.y), cand23 = pack_bf16x2(c23.x, c23.y);
+                        for (int c = 0; c < 4; ++c)
+                            sl[c] = *reinterpret_cast<const uint4*>(selp + __byte_perm(idx, 0u, 0x4440u | c) * (kGSelRep * 16));
+                        const float db = half_bits(cur.a0) *
+                                         (__uint_as_float(0x4b000001u | ((Sw >> 27) & 0x1eu)) - 8388608.0f) * 0.125f;
+                        const float2 db2 = make_float2(db, db);
+                        const float2 c01 = fmul2(db2, gv01), c23 = fmul2(db2, gv23);
+                        const uint32_t cand01 = pack_bf16x2(c01.x, c01.y), cand23 = pack_bf16x2(c23.x, c23.y);
 #pragma unroll
-                            for (int c = 0; c < 4; ++c)
-                                *reinterpret_cast<uint4*>(bt + b_unit_off(r, 4 * hf + c)) =
-                                    iq2_chunk_bf16(idx, Sw, c, cand01, cand23, selp);
-                        }
+                        for (int c = 0; c < 4; ++c)
+                            *reinterpret_cast<uint4*>(bt + c * 128) = iq2_chunk_bf16(sl[c], Sw, c, cand01, cand23);
                     } else {
                         const float d = half_bits(cur.a1 & 0xffffu), dmin = half_bits(cur.a1 >> 16);
-                        // two sub-blocks per pass: a full unroll schedules all eight units at once and spills
-#pragma unroll 2
-                        for (int sbk = 0; sbk < 4; ++sbk) {
-                            const uint32_t w = (sbk & 2) ? ((sbk & 1) ? cur.q.w : cur.q.z) : ((sbk & 1) ? cur.q.y : cur.q.x);
+#pragma unroll
+                        for (int sbk = 0; sbk < 2; ++sbk) {
+                            const uint32_t w = sbk ? cur.q.y : cur.q.x;
                             const uint32_t sb = (cur.a0 >> (8 * sbk)) & 0xffu;
                             const float sc = d * (float)(sb & 15u), mn = dmin * (float)(sb >> 4);
                             const float2 sc2 = make_float2(sc, sc), nmn2 = make_float2(-mn, -mn);
-                            *reinterpret_cast<uint4*>(bt + b_unit_off(r, 2 * sbk)) = q2_unit_bf16(w, sc2, nmn2);
-                            *reinterpret_cast<uint4*>(bt + b_unit_off(r, 2 * sbk + 1)) = q2_unit_bf16(w >> 16, sc2, nmn2);
+                            *reinterpret_cast<uint4*>(bt + (2 * sbk) * 128) = q2_unit_bf16(w, sc2, nmn2);
+                            *reinterpret_cast<uint4*>(bt + (2 * sbk + 1) * 128) = q2_unit_bf16(w >> 16, sc2, nmn2);
                         }
                     }
                     fence_proxy_async_smem();
@@ -607,41 +681,34 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const uint32_t taddr = tmem + ((uint32_t)(32 * qd) << 16) + half * kGBN;
             const bool live = m < ti.mvalid;
             if (ti.mvalid > kGHalf * half) {   // this half was computed
+                // 16-column TMEM reads; each thread stores 32-byte pieces of its own row
                 if (kGateUp) {
                     __nv_bfloat16* dst = a.out_h + (size_t)(ti.row0 + m) * I + 128 * ti.nb;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < 128; c0 += 32) {
-                        uint32_t g[32], u[32];
-                        tmem_ld_32x32(taddr + c0, g);
-                        tmem_ld_32x32(taddr + 128 + c0, u);
+                    for (int c0 = 0; c0 < 128; c0 += 16) {
+                        uint32_t g[16], u[16];
+                        tmem_ld_32x16(taddr + c0, g);
+                        tmem_ld_32x16(taddr + 128 + c0, u);
                         tmem_wait_ld();
-                        uint32_t hp[16];
+                        uint32_t hp[8];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
+                        for (int j = 0; j < 8; ++j) {
                             const float h0 = silu(__uint_as_float(g[2 * j])) * __uint_as_float(u[2 * j]);
                             const float h1 = silu(__uint_as_float(g[2 * j + 1])) * __uint_as_float(u[2 * j + 1]);
                             hp[j] = pack_bf16x2(h0, h1);
                         }
-                        if (live) {
-                            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
-#pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                d4[j] = make_uint4(hp[4 * j], hp[4 * j + 1], hp[4 * j + 2], hp[4 * j + 3]);
-                        }
+                        if (live) st_global_v8(dst + c0, hp[0], hp[1], hp[2], hp[3], hp[4], hp[5], hp[6], hp[7]);
                     }
                 } else {
                     float* dst = a.out_y + (size_t)(ti.row0 + m) * H + kGBN * ti.nb;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < kGBN; c0 += 32) {
-                        uint32_t v[32];
-                        tmem_ld_32x32(taddr + c0, v);
+                    for (int c0 = 0; c0 < kGBN; c0 += 16) {
+                        uint32_t v[16];
+                        tmem_ld_32x16(taddr + c0, v);
                         tmem_wait_ld();
                         if (live) {
-                            float4* d4 = reinterpret_cast<float4*>(dst + c0);
-#pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                d4[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                                    __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                            st_global_v8(dst + c0, v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+                            st_global_v8(dst + c0 + 8, v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
                         }
                     }
                 }
@@ -800,7 +867,7 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
         xb = ws.xb;
     }
     mk.before();
-    k_router_prefill<<<dim3((n + kRP_T - 1) / kRP_T, (E + kRP_E - 1) / kRP_E), 512, 0, st>>>(W, D, x, n, ws.logits);
+    if ((e = launch_router_prefill(W, D, x, n, ws.logits, st)) != cudaSuccess) return e;
     mk.after();
     mk.before();
     k_topk_prefill<<<(n + 7) / 8, 256, 0, st>>>(D, ws.logits, n, ws.ids, ws.wts);
@@ -878,7 +945,8 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
 // Routing only (prefill sizes): logits and top-k.
 cudaError_t launch_route_prefill(const Weights& W, const Dims& D, const PrefillWs& ws, const void* x, int n,
                                  cudaStream_t st) {
-    k_router_prefill<<<dim3((n + kRP_T - 1) / kRP_T, (D.E + kRP_E - 1) / kRP_E), 512, 0, st>>>(W, D, x, n, ws.logits);
+    cudaError_t e = launch_router_prefill(W, D, x, n, ws.logits, st);
+    if (e != cudaSuccess) return e;
     k_topk_prefill<<<(n + 7) / 8, 256, 0, st>>>(D, ws.logits, n, ws.ids, ws.wts);
     return cudaGetLastError();
 }
