@@ -192,11 +192,11 @@ constexpr int kGStages = 3;
 constexpr int kGAHalf = kGHalf * kGBK * 2;    // 16 KB
 constexpr int kGAStage = 2 * kGAHalf;         // 32 KB
 constexpr int kGBStage = kGBN * kGBK * 2;     // 32 KB
-constexpr int kGDqWarps = 16, kGEpiWarps = 8;  // two dequantizing threads per B row
+constexpr int kGDqWarps = 8, kGEpiWarps = 8;   // one dequantizing thread per B row
 constexpr int kGWarps = 2 + kGDqWarps + kGEpiWarps;
 constexpr int kGThreads = kGWarps * 32;
-constexpr int kGSelRep = 8;                   // selector-table copies: conflict-free 16-byte reads
-constexpr int kGSelBytes = 256 * kGSelRep * 16;
+constexpr int kGSelRep = 16;                  // selector-table copies: conflict-free 8-byte reads
+constexpr int kGSelBytes = 256 * kGSelRep * 8;
 constexpr uint32_t kGTmemCols = 512;          // two 128-lane x 256-column binary32 accumulators
 
 // ---------------------------------------------------------------- permutation
@@ -366,19 +366,20 @@ __device__ __forceinline__ uint32_t b_row_off(int r) { return (uint32_t)((r >> 3
 // The grid holds at most four distinct magnitudes v_c, so each group of 32
 // weights first rounds its four candidates d(2s+1)/8 * v_c to bf16 (the
 // binary32 products are exact: at most 22 significant bits), held as bytes
-// 0..7 of (cand01, cand23).  Row a of the selector table (sl, four 32-bit
-// words loaded by the caller) gives, per pair of weights, the byte-permute
+// 0..7 of (cand01, cand23).  Row a of the selector table (sl, four 16-bit
+// selectors loaded by the caller) gives, per pair of weights, the byte-permute
 // selector that picks the two rounded candidates.  Rounding is symmetric, so
 // the signs are applied to the picked pairs: sg * C_j places sign bit 2j at
 // bit 15 and bit 2j+1 at bit 31 (the two shifted copies of the 8-bit sign byte
 // do not overlap, so the multiply has no carries).
-__device__ __forceinline__ uint4 iq2_chunk_bf16(uint4 sl, uint32_t S, int c, uint32_t cand01, uint32_t cand23) {
-    uint32_t sg = (S >> (7 * c)) & 127u;
-    sg |= ((uint32_t)__popc(sg) & 1u) << 7;
+__device__ __forceinline__ uint4 iq2_chunk_bf16(uint2 sl, uint32_t S, int c, uint32_t cand01, uint32_t cand23) {
+    const uint32_t sg = (S >> (7 * c)) & 127u;
+    // sign of element 7 = parity of the seven stored bits, added at bit 31 of the last mask
+    const uint32_t m3 = sg * 0x01000200u + ((uint32_t)__popc(sg) << 31);
     return make_uint4(__byte_perm(cand01, cand23, sl.x) ^ ((sg * 0x40008000u) & 0x80008000u),
-                      __byte_perm(cand01, cand23, sl.y) ^ ((sg * 0x10002000u) & 0x80008000u),
-                      __byte_perm(cand01, cand23, sl.z) ^ ((sg * 0x04000800u) & 0x80008000u),
-                      __byte_perm(cand01, cand23, sl.w) ^ ((sg * 0x01000200u) & 0x80008000u));
+                      __byte_perm(cand01, cand23, sl.x >> 16) ^ ((sg * 0x10002000u) & 0x80008000u),
+                      __byte_perm(cand01, cand23, sl.y) ^ ((sg * 0x04000800u) & 0x80008000u),
+                      __byte_perm(cand01, cand23, sl.y >> 16) ^ (m3 & 0x80008000u));
 }
 
 // Eight 2-bit codes (bits 2i of x, i = 0..7) -> 8 bf16 of (d sc) q - dmin m.
@@ -400,10 +401,10 @@ __device__ __forceinline__ uint4 q2_unit_bf16(uint32_t x, float2 sc2, float2 nmn
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// One dequantizing thread's packed weights for one k step (32 weights of one B row).
+// One dequantizing thread's packed weights for one k step (64 weights of one B row).
 struct BFrag {
-    uint2 q;        // IQ2: (grid indices, signs+scale) of the group; Q2: 32 codes (two sub-blocks)
-    uint32_t a0;    // IQ2: d (binary16 bits); Q2: the two sub-blocks' scale bytes in bits 0..15
+    uint4 q;        // IQ2: two (grid indices, signs+scale) pairs; Q2: 64 codes
+    uint32_t a0;    // IQ2: d (binary16 bits); Q2: four scale bytes
     uint32_t a1;    // Q2: d | dmin << 16
 };
 
@@ -418,7 +419,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         (reinterpret_cast<uintptr_t>(g_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     unsigned char* stA = base;                                   // kGStages x 32 KB
     unsigned char* stB = base + kGStages * kGAStage;              // kGStages x 32 KB
-    unsigned char* seltab = stB + kGStages * kGBStage;            // [256][kGSelRep] x 4 selectors (16 bytes)
+    unsigned char* seltab = stB + kGStages * kGBStage;            // [256][kGSelRep] x 4 16-bit selectors
     __shared__ GemmSmem S;
 
     constexpr bool kRouted = MODE == kModeGateUp || MODE == kModeDown;
@@ -474,10 +475,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 const uint32_t cb = (uint32_t)cls[a.W.grid_u8[row * 8 + 2 * j + 1]];
                 sel[j] = 0x1010u + 0x22u * ca + 0x2200u * cb;   // bytes 2c, 2c+1 hold candidate c
             }
-            const uint4 ent = make_uint4(sel[0], sel[1], sel[2], sel[3]);
+            const uint2 ent = make_uint2(sel[0] | (sel[1] << 16), sel[2] | (sel[3] << 16));
 #pragma unroll
             for (int p = 0; p < kGSelRep; ++p)
-                *reinterpret_cast<uint4*>(seltab + row * (kGSelRep * 16) + p * 16) = ent;
+                *reinterpret_cast<uint2*>(seltab + row * (kGSelRep * 8) + p * 8) = ent;
         }
     }
     if (warp == 1) {
@@ -563,13 +564,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     } else if (warp < 2 + kGDqWarps) {
         // ------------------------------------------------ B tiles (dequantize to bf16)
         if (kRouted) {
-            // thread -> (B-tile row r, 32-weight group hf of the 64-column k step): lanes 0..15 of a
-            // warp take group 0 of 16 rows, lanes 16..31 group 1, so that each 8-lane phase of a
-            // 16-byte shared store covers 8 rows of one unit (conflict-free)
-            const int dw = warp - 2;
-            const int hf = lane >> 4;
-            const int r = 16 * dw + (lane & 15);
-            const unsigned char* selp = seltab + (lane & 7) * 16;
+            const int r = tid - 64;   // B-tile row 0..255
+            const unsigned char* selp = seltab + (lane & 15) * 8;
             float2 gv01 = make_float2(0.f, 0.f), gv23 = make_float2(0.f, 0.f);
             if (MODE == kModeGateUp) {
                 gv01 = make_float2(S.gval[0], S.gval[1]);
@@ -577,7 +573,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             }
             const int my_tiles = (int)blockIdx.x < ntiles ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
             const int total = my_tiles * KS;
-            // load cursor: tile, k step and this thread's packed-weight pointers
+            // load cursor: tile, k step and this row's packed-weight pointers
             int ctile = blockIdx.x, cks = 0;
             const uint8_t* qs = nullptr;
             const uint16_t* dq = nullptr;
@@ -589,23 +585,23 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 if (MODE == kModeGateUp) {
                     const int row = 128 * ti.nb + (r & 127);
                     qs = (r < 128 ? a.W.gate_qs : a.W.up_qs) + e * a.W.iq2_qs_stride +
-                         (size_t)(row >> 5) * (H / 64) * 512 + (row & 31) * 16 + hf * 8;
+                         (size_t)(row >> 5) * (H / 64) * 512 + (row & 31) * 16;
                     dq = (r < 128 ? a.W.gate_d : a.W.up_d) + e * a.W.iq2_d_stride + (size_t)(row >> 5) * (H / 256) * 32 +
                          (row & 31);
                 } else {
                     const int row = kGBN * ti.nb + r;
                     const int nkt = I / 64, nsb = I >= 256 ? I / 256 : 1;
-                    qs = a.W.down_q + e * a.W.q2_q_stride + ((size_t)(row >> 5) * nkt * 32 + (row & 31)) * 16 + hf * 8;
+                    qs = a.W.down_q + e * a.W.q2_q_stride + ((size_t)(row >> 5) * nkt * 32 + (row & 31)) * 16;
                     scp = a.W.down_sc + e * a.W.q2_sc_stride + (size_t)(row >> 5) * nkt * 32 + (row & 31);
                     ddp = a.W.down_dd + e * a.W.q2_dd_stride + (size_t)(row >> 5) * nsb * 32 + (row & 31);
                 }
             };
             auto fetch = [&](BFrag& f) {
-                f.q = ld_stream_v2(qs + (size_t)cks * 512);
+                f.q = ld_stream_v4(qs + (size_t)cks * 512);
                 if (MODE == kModeGateUp) {
                     f.a0 = ld_stream_u16(dq + (cks >> 2) * 32);
                 } else {
-                    f.a0 = ld_stream_u32(scp + cks * 32) >> (16 * hf);
+                    f.a0 = ld_stream_u32(scp + cks * 32);
                     f.a1 = ld_stream_u32(ddp + (I >= 256 ? (cks >> 2) : 0) * 32);
                 }
                 if (++cks == KS) {
@@ -614,7 +610,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     if (ctile < ntiles) set_src(ctile);
                 }
             };
-            constexpr int PD = 3;   // k steps of packed weights in flight
+            constexpr int PD = 4;   // k steps of packed weights in flight
             BFrag ring[PD];
             if (total > 0) set_src(ctile);
 #pragma unroll
@@ -632,28 +628,35 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         g_set_abort(S);
                         break;
                     }
-                    unsigned char* bt = stB + s * kGBStage + b_row_off(r) + hf * 4 * 128;
+                    unsigned char* bt = stB + s * kGBStage + b_row_off(r);
                     if (MODE == kModeGateUp) {
-                        // the group's four selector rows first: the loads then overlap instead of
-                        // waiting behind the tile stores (which the compiler cannot reorder)
-                        const uint32_t idx = cur.q.x, Sw = cur.q.y;
-                        uint4 sl[4];
+                        const float d = half_bits(cur.a0);
 #pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            sl[c] = *reinterpret_cast<const uint4*>(selp + __byte_perm(idx, 0u, 0x4440u | c) * (kGSelRep * 16));
-                        const float db = half_bits(cur.a0) *
-                                         (__uint_as_float(0x4b000001u | ((Sw >> 27) & 0x1eu)) - 8388608.0f) * 0.125f;
-                        const float2 db2 = make_float2(db, db);
-                        const float2 c01 = fmul2(db2, gv01), c23 = fmul2(db2, gv23);
-                        const uint32_t cand01 = pack_bf16x2(c01.x, c01.y), cand23 = pack_bf16x2(c23.x, c23.y);
+                        for (int hf = 0; hf < 2; ++hf) {
+                            // the group's four selector rows first: the loads then overlap instead of
+                            // waiting behind the tile stores (which the compiler cannot reorder)
+                            const uint32_t idx = hf ? cur.q.z : cur.q.x, Sw = hf ? cur.q.w : cur.q.y;
+                            uint2 sl[4];
 #pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            *reinterpret_cast<uint4*>(bt + c * 128) = iq2_chunk_bf16(sl[c], Sw, c, cand01, cand23);
+                            for (int c = 0; c < 4; ++c)
+                                sl[c] = *reinterpret_cast<const uint2*>(selp + __byte_perm(idx, 0u, 0x4440u | c) *
+                                                                                   (kGSelRep * 8));
+                            const float db =
+                                d * (__uint_as_float(0x4b000001u | ((Sw >> 27) & 0x1eu)) - 8388608.0f) * 0.125f;
+                            const float2 db2 = make_float2(db, db);
+                            const float2 c01 = fmul2(db2, gv01), c23 = fmul2(db2, gv23);
+                            const uint32_t cand01 = pack_bf16x2(c01.x, c01.y), cand23 = pack_bf16x2(c23.x, c23.y);
+#pragma unroll
+                            for (int c = 0; c < 4; ++c)
+                                *reinterpret_cast<uint4*>(bt + (4 * hf + c) * 128) =
+                                    iq2_chunk_bf16(sl[c], Sw, c, cand01, cand23);
+                        }
                     } else {
                         const float d = half_bits(cur.a1 & 0xffffu), dmin = half_bits(cur.a1 >> 16);
-#pragma unroll
-                        for (int sbk = 0; sbk < 2; ++sbk) {
-                            const uint32_t w = sbk ? cur.q.y : cur.q.x;
+                        // two sub-blocks per pass: a full unroll schedules all eight units at once and spills
+#pragma unroll 2
+                        for (int sbk = 0; sbk < 4; ++sbk) {
+                            const uint32_t w = (sbk & 2) ? ((sbk & 1) ? cur.q.w : cur.q.z) : ((sbk & 1) ? cur.q.y : cur.q.x);
                             const uint32_t sb = (cur.a0 >> (8 * sbk)) & 0xffu;
                             const float sc = d * (float)(sb & 15u), mn = dmin * (float)(sb >> 4);
                             const float2 sc2 = make_float2(sc, sc), nmn2 = make_float2(-mn, -mn);
