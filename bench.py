@@ -88,15 +88,19 @@ def algorithmic_bytes(w: dict, U: int) -> dict:
 
 def traffic_from_profile(kernel: str, workload: str):
     """dram bytes per launch recorded under profiles/, if the kernel source is unchanged since."""
-    p = os.path.join(ROOT, "profiles", "%s_%s.md" % (kernel, workload))
+    name = kernel.replace("<", "_").replace(">", "")
+    p = os.path.join(ROOT, "profiles", "%s_%s.md" % (name, workload))
     if not os.path.exists(p):
         return None
     txt = open(p).read()
     m1 = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
     m2 = re.search(r"source_sha256:\s*([0-9a-f]+)", txt)
+    m3 = re.search(r"source_file:\s*([A-Za-z0-9_.]+)", txt)
     if not (m1 and m2):
         return None
-    src = os.path.join(ROOT, "bit_quantized_moe_softmax_b200", "csrc", "decode.cu")
+    src = os.path.join(ROOT, "bit_quantized_moe_softmax_b200", "csrc", m3.group(1) if m3 else "decode.cu")
+    if not os.path.exists(src):
+        return None
     if hashlib.sha256(open(src, "rb").read()).hexdigest() != m2.group(1):
         return None
     return float(m1.group(1))
