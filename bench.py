@@ -28,6 +28,7 @@ import sys
 import tempfile
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -44,6 +45,9 @@ WORKLOADS = {
                     desc="MTP-verify style decode: 8 tokens, one MoE layer of the decode shape"),
     "decode2": dict(n=2, H=4096, I=2048, E=256, k=8,
                     desc="MTP-verify style decode: 2 tokens, one MoE layer of the decode shape"),
+    "mtp8": dict(n=2, H=4096, I=2048, E=256, k=8, layers=8, router_std=1.0 / 64, chain_scales=True,
+                 desc="MTP-verify style decode: 2 tokens through 8 chained MoE layers of the decode shape "
+                      "(x_{l+1} = x_l + MoE_l(x_l)), router logits N(0,1)"),
     "prefill512": dict(n=512, H=4096, I=2048, E=256, k=8, zipf=1.1, bf16=True,
                        desc="short-prompt prefill: 512 bf16 tokens, one MoE layer of the decode shape, "
                             "Zipf(1.1) expert popularity"),
@@ -170,13 +174,17 @@ def run_ours(args, wl, rank, local, world):
     torch.cuda.set_device(dev)
     n, H, I, E, k = wl["n"], wl["H"], wl["I"], wl["E"], wl["k"]
     prefill = n > 8
-    R = 1 if prefill else args.instances
+    C = wl.get("layers", 1)     # chained layers per step (x_{l+1} = x_l + MoE_l(x_l))
+    chain = C > 1
+    R = C if chain else (1 if prefill else args.instances)
     shape = synth.Shape(H=H, I=I, E=E, k=k)
     bias = synth.zipf_bias(E, wl["zipf"], seed=5).to(dev) if wl.get("zipf") else None
     act = m.DS4MOE_ACT_BF16 if wl.get("bf16") else m.DS4MOE_ACT_F32
     layers = []
     for r in range(R):
-        L = synth.packed_layer(shape, seed=1000 * rank + r, bias=bias, device=dev)
+        L = synth.packed_layer(shape, seed=1000 * rank + r, router_std=wl.get("router_std", 0.02), bias=bias,
+                               device=dev, d_range=synth.CHAIN_D_RANGE if wl.get("chain_scales") else (1e-3, 4e-3),
+                               shared_std=synth.CHAIN_SHARED_STD if wl.get("chain_scales") else 0.02)
         lay = m.MoELayer(H, I, E, k, max_tokens=max(n, 8), act_dtype=act, has_bias=bias is not None, device=dev)
         lay.load(L)
         layers.append(lay)
@@ -189,12 +197,46 @@ def run_ours(args, wl, rank, local, world):
     nl = m.ds4moe_plan_launches(layers[0].h, n)
     names = [m.ds4moe_plan_kernel(layers[0].h, n, i) for i in range(nl)]
 
+    cbufs = [torch.empty(n, H, dtype=torch.float32, device=dev) for _ in range(C)] if chain else []
+
     def step(i, events=None):
+        if chain:   # every layer of the chain, the residual added by each layer's combine kernel
+            cur = xs[i % P]
+            for l in range(C):
+                if events is None:
+                    m.ds4moe_forward_residual(layers[l].h, cur, cbufs[l], stream)
+                else:
+                    m.ds4moe_forward_residual_profiled(layers[l].h, cur, cbufs[l],
+                                                       events[2 * nl * l:2 * nl * (l + 1)], stream)
+                cur = cbufs[l]
+            return
         lay = layers[i % R]
         if events is None:
             m.ds4moe_forward(lay.h, xs[i % P], outs[i % P], stream)
         else:
             m.ds4moe_forward_profiled(lay.h, xs[i % P], outs[i % P], events, stream)
+
+    def distinct_experts():
+        """Mean number of distinct experts per layer forward over the steps the graphs replay."""
+        if prefill:
+            return None
+        tot, cnt = 0, 0
+        with torch.cuda.stream(stream):
+            for i in range(min(64, P * R)):
+                if chain:
+                    cur = xs[i % P]
+                    for l in range(C):
+                        ids, _ = layers[l].route(cur)
+                        tot += int(torch.unique(ids).numel())
+                        cnt += 1
+                        m.ds4moe_forward_residual(layers[l].h, cur, cbufs[l], stream)
+                        cur = cbufs[l]
+                else:
+                    ids, _ = layers[i % R].route(xs[i % P])
+                    tot += int(torch.unique(ids).numel())
+                    cnt += 1
+        stream.synchronize()
+        return tot / cnt
 
     with torch.cuda.stream(stream):
         for i in range(max(2, R)):
@@ -210,7 +252,7 @@ def run_ours(args, wl, rank, local, world):
 
     def new_events(count):
         # torch creates the CUDA event on first record: record each once before capture
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nl)] for _ in range(count)]
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nl * C)] for _ in range(count)]
         for ev in evs:
             for e in ev:
                 e.record(stream)
@@ -274,8 +316,9 @@ def run_ours(args, wl, rank, local, world):
     torch.cuda.synchronize(dev)
     for (g, evs), reps in prof:
         for ev in evs:
-            for i, nm in enumerate(names):
-                durs[nm].append(ev[2 * i].elapsed_time(ev[2 * i + 1]))
+            for l in range(C):
+                for i, nm in enumerate(names):
+                    durs[nm].append(ev[2 * nl * l + 2 * i].elapsed_time(ev[2 * nl * l + 2 * i + 1]))
     ms_prof = pstart.elapsed_time(pstop)
     clocks = sampler.stop()
 
@@ -289,12 +332,24 @@ def run_ours(args, wl, rank, local, world):
     K2 = min(K2, 20) if prefill else K2
     xh = xs[: min(P, K2)].cpu().pin_memory()
     oh = torch.empty(xh.shape, dtype=torch.float32).pin_memory()
+
+    def e2e_step(i):
+        if chain:   # pinned host x -> device, the chain, device -> pinned host, synchronize
+            xd = xs[0]
+            with torch.cuda.stream(stream):
+                xd.copy_(xh[i % xh.shape[0]], non_blocking=True)
+                step(0)
+                oh[i % xh.shape[0]].copy_(cbufs[-1], non_blocking=True)
+            stream.synchronize()
+        else:
+            m.ds4moe_forward_host(layers[i % R].h, xh[i % xh.shape[0]], oh[i % xh.shape[0]], stream)
+
     for i in range(min(10, K2)):
-        m.ds4moe_forward_host(layers[i % R].h, xh[i % xh.shape[0]], oh[i % xh.shape[0]], stream)
+        e2e_step(i)
     D.barrier()
     t0 = time.perf_counter()
     for i in range(K2):
-        m.ds4moe_forward_host(layers[i % R].h, xh[i % xh.shape[0]], oh[i % xh.shape[0]], stream)
+        e2e_step(i)
     t1 = time.perf_counter()
     e2e_s = D.max_over_ranks(t1 - t0, dev)
     e2e = {"value": n * K2 * world / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": n * H * xh.element_size(),
@@ -304,7 +359,7 @@ def run_ours(args, wl, rank, local, world):
     peaks, peak_kind = load_peaks()
     mean = {nm: (statistics.mean(v) if v else 0.0) for nm, v in durs.items()}
     dom = max(mean, key=lambda nm: mean[nm])
-    U = min(n * k, E) if n == 1 else None
+    U = distinct_experts()
     ab = algorithmic_bytes(wl, U if U is not None else n * k)
     if prefill:
         fl = algorithmic_flops(wl)
@@ -319,25 +374,28 @@ def run_ours(args, wl, rank, local, world):
         peak = peaks["hbm_gbs"]
         roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                     "frac": round(achieved / peak, 4), "traffic": traffic_from_profile(dom, args.workload),
-                    "algorithmic_bytes_per_launch": ab[dom], "mean_launch_us": round(mean[dom] * 1e3, 2),
+                    "algorithmic_bytes_per_launch": int(round(ab[dom])), "mean_launch_us": round(mean[dom] * 1e3, 2),
                     "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs, burst copy)"}
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if prefill else "f32", "data": "synthetic",
         "config": {"workload": wl["desc"], "n_tokens_per_step": n, "hidden": H, "expert_inter": I,
-                   "experts": E, "top_k": k, "layer_instances": R, "token_vectors": P,
-                   "l2": ("weights rotate over %d layer instances (%.1f GB) and %d token vectors: inputs larger "
+                   "experts": E, "top_k": k, "layer_instances": R, "chained_layers": C, "token_vectors": P,
+                   "mean_distinct_experts_per_layer": round(U, 2) if U else None,
+                   "l2": ("%d chained layers (%.1f GB of weights) and %d token vectors per step: inputs larger "
+                          "than L2" % (C, C * layers[0].weights.numel() / 1e9, P)) if chain else
+                         ("weights rotate over %d layer instances (%.1f GB) and %d token vectors: inputs larger "
                           "than L2" % (R, R * layers[0].weights.numel() / 1e9, P)) if not prefill else
                          "one layer (%.1f GB of weights) and %d token batches per step: inputs larger than L2"
                          % (layers[0].weights.numel() / 1e9, n),
                    "parallelism": "dp%d replicas (no collective on the data path)" % world},
-        "expert_weight_gbs": round(ab["routed"] / (ms_per_step * 1e-3) / 1e9, 1) if U else None,
-        "layer_hbm_gbs": round(ab["layer"] / (ms_per_step * 1e-3) / 1e9, 1) if U else None,
-        "layer_frac_of_hbm_peak": round(ab["layer"] / (ms_per_step * 1e-3) / 1e9 / peak, 4) if U else None,
+        "expert_weight_gbs": round(C * ab["routed"] / (ms_per_step * 1e-3) / 1e9, 1) if U else None,
+        "layer_hbm_gbs": round(C * ab["layer"] / (ms_per_step * 1e-3) / 1e9, 1) if U else None,
+        "layer_frac_of_hbm_peak": round(C * ab["layer"] / (ms_per_step * 1e-3) / 1e9 / peak, 4) if U else None,
         "kernel_us": {nm: round(mean[nm] * 1e3, 2) for nm in names},
         "ms_per_step_profiled": round(ms_prof / args.steps, 5),
-        "roofline": roofline, "e2e": e2e, "gpu_launches": nl * args.steps, "clocks": clocks,
+        "roofline": roofline, "e2e": e2e, "gpu_launches": nl * C * args.steps, "clocks": clocks,
     }
     return line
 
@@ -350,6 +408,8 @@ def oracle_sample(wl, n_tokens, seed=0, budget_s=20.0, device="cuda"):
 
     H, I, E, k = wl["H"], wl["I"], wl["E"], wl["k"]
     bias = synth.zipf_bias(E, wl["zipf"], seed=5) if wl.get("zipf") else None
+    if wl.get("layers", 1) > 1:
+        return oracle_chain_sample(wl, n_tokens, seed, budget_s, device)
     L = synth.packed_layer(synth.Shape(H=H, I=I, E=E, k=k), seed=seed, bias=bias, device=device)
     x = synth.tokens(n_tokens, H, seed=seed + 5, dtype=torch.bfloat16 if wl.get("bf16") else torch.float32).float()
     mode = 1 if wl.get("bf16") else 0
@@ -366,6 +426,35 @@ def oracle_sample(wl, n_tokens, seed=0, budget_s=20.0, device="cuda"):
             break
     dt = time.perf_counter() - t0
     return done / dt, done, dt
+
+
+def oracle_chain_sample(wl, n_tokens, seed, budget_s, device):
+    """Oracle tokens/s through the chain of layers (fp64 layers, binary32 between layers); only the time
+    of the oracle's router and layer calls counts (not the host copies of the selected experts' blocks)."""
+    import oracle
+    from bit_quantized_moe_softmax_b200 import synth
+
+    H, I, E, k, C = wl["H"], wl["I"], wl["E"], wl["k"], wl["layers"]
+    Ls = [synth.packed_layer(synth.Shape(H=H, I=I, E=E, k=k), seed=seed + l, router_std=wl.get("router_std", 0.02),
+                             device=device, d_range=synth.CHAIN_D_RANGE, shared_std=synth.CHAIN_SHARED_STD)
+          for l in range(C)]
+    x = synth.tokens(n_tokens, H, seed=seed + 5).numpy()
+    spent, done = 0.0, 0
+    for t in range(n_tokens):
+        cur = x[t:t + 1].astype(np.float32)
+        for L in Ls:
+            t0 = time.perf_counter()
+            rid, _ = oracle.topk_softmax(oracle.router_logits(cur, L["W_r"].cpu().numpy()), k)
+            spent += time.perf_counter() - t0
+            lay = oracle.layer_from_torch(L, experts=rid.ravel())
+            t0 = time.perf_counter()
+            y, _, _ = oracle.moe_forward(lay, cur, mode=0)
+            spent += time.perf_counter() - t0
+            cur = (cur.astype(np.float64) + y).astype(np.float32)
+        done += 1
+        if spent > budget_s:
+            break
+    return done / spent, done, spent
 
 
 def run_reference(args, wl, rank, world):

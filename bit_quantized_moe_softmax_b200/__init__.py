@@ -31,7 +31,8 @@ EXPORTS = ("ds4moe_create", "ds4moe_destroy", "ds4moe_weight_bytes", "ds4moe_wor
            "ds4moe_pack_q2k", "ds4moe_pack_iq2xxs", "ds4moe_set_grid", "ds4moe_set_router", "ds4moe_set_expert",
            "ds4moe_set_shared", "ds4moe_forward", "ds4moe_forward_host", "ds4moe_route", "ds4moe_dequant",
            "ds4moe_get_device_error", "ds4moe_last_error", "ds4moe_plan_launches", "ds4moe_plan_kernel",
-           "ds4moe_forward_profiled", "ds4moe_route_noalloc")
+           "ds4moe_forward_profiled", "ds4moe_route_noalloc", "ds4moe_forward_residual",
+           "ds4moe_forward_residual_profiled")
 
 
 class ds4moe_shape(ctypes.Structure):
@@ -76,6 +77,8 @@ def lib() -> ctypes.CDLL:
             "ds4moe_plan_kernel": ([vp, i32, i32], ctypes.c_char_p),
             "ds4moe_forward_profiled": ([vp, vp, i32, vp, ctypes.POINTER(vp), vp], i32),
             "ds4moe_route_noalloc": ([vp, vp, i32, vp, vp, vp], i32),
+            "ds4moe_forward_residual": ([vp, vp, i32, vp, vp], i32),
+            "ds4moe_forward_residual_profiled": ([vp, vp, i32, vp, ctypes.POINTER(vp), vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -157,6 +160,16 @@ def ds4moe_set_shared(h: int, gate: torch.Tensor, up: torch.Tensor, down: torch.
 
 def ds4moe_forward(h: int, x: torch.Tensor, out: torch.Tensor, stream=None):
     _ok(lib().ds4moe_forward(h, _ptr(x), x.shape[0], _ptr(out), _stream(stream)), "ds4moe_forward")
+
+
+def ds4moe_forward_residual(h: int, x: torch.Tensor, out: torch.Tensor, stream=None):
+    _ok(lib().ds4moe_forward_residual(h, _ptr(x), x.shape[0], _ptr(out), _stream(stream)), "ds4moe_forward_residual")
+
+
+def ds4moe_forward_residual_profiled(h: int, x: torch.Tensor, out: torch.Tensor, events, stream=None):
+    arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+    _ok(lib().ds4moe_forward_residual_profiled(h, _ptr(x), x.shape[0], _ptr(out), arr, _stream(stream)),
+        "ds4moe_forward_residual_profiled")
 
 
 def ds4moe_plan_launches(h: int, n_tokens: int) -> int:
@@ -271,10 +284,11 @@ class MoELayer:
         torch.cuda.current_stream(dev).synchronize()
         return layer
 
-    def forward(self, x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, out: torch.Tensor | None = None, residual: bool = False) -> torch.Tensor:
+        """The layer on x; with residual=True, x + the layer (x and out must not overlap)."""
         if out is None:
             out = torch.empty(x.shape[0], self.H, dtype=torch.float32, device=x.device)
-        ds4moe_forward(self.h, x, out)
+        (ds4moe_forward_residual if residual else ds4moe_forward)(self.h, x, out)
         return out
 
     def route(self, x: torch.Tensor):

@@ -810,7 +810,8 @@ __global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------- combine
-// out[t][r] = y_shared[t][r] + sum_j w[t][j] y[t*k + j][r], j in rank order.
+// out[t][r] = y_shared[t][r] + sum_j w[t][j] y[t*k + j][r], j in rank order
+// (then x[t][r] + that, when the call asks for the residual).
 __global__ void __launch_bounds__(256) k_combine_decode(Dims D, DecodeWs ws, float* out, int n) {
     griddep_wait();   // y of the down grid
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -829,7 +830,7 @@ __global__ void __launch_bounds__(256) k_combine_decode(Dims D, DecodeWs ws, flo
 #pragma unroll
     for (int j = 0; j < 16; ++j)
         if (j < k) acc = fmaf(w[j], y[j], acc);
-    out[i] = acc;
+    out[i] = ws.xres ? act_at(ws.xres, i, D.act_bf16) + acc : acc;
 }
 
 // ---------------------------------------------------------------- launchers

@@ -433,23 +433,43 @@ static ds4moe_status check_forward(ds4moe_t* h, const void* x, int32_t n, const 
 }
 
 static ds4moe_status forward_impl(ds4moe_t* h, const void* d_x, int32_t n, float* d_out, void* const* events,
-                                  void* stream, const char* who) {
+                                  void* stream, const char* who, bool residual = false) {
     ds4moe_status s = check_forward(h, d_x, n, d_out, who);
     if (s != DS4MOE_OK) return s;
     if (n == 0) return DS4MOE_OK;
     if (!aligned16(d_x) || !aligned16(d_out)) return fail(DS4MOE_ERR_ALIGN, "%s: x and out must be 16-byte aligned", who);
+    if (residual) {   // out is written while x is still read: the ranges may not overlap
+        const uintptr_t xa = reinterpret_cast<uintptr_t>(d_x), oa = reinterpret_cast<uintptr_t>(d_out);
+        const size_t xbytes = (size_t)n * h->D.H * (h->D.act_bf16 ? 2 : 4), obytes = (size_t)n * h->D.H * 4;
+        if (xa < oa + obytes && oa < xa + xbytes) return fail(DS4MOE_ERR_ARG, "%s: x and out overlap", who);
+    }
     cudaStream_t st = (cudaStream_t)stream;
     cudaEvent_t const* ev = reinterpret_cast<cudaEvent_t const*>(events);
     cudaError_t ce;
-    if (n <= h->decode_max)
-        ce = launch_decode(h->weights_view(), h->D, h->decode_ws(), d_x, n, d_out, h->n_sm, st, ev);
-    else
-        ce = launch_prefill(h->weights_view(), h->D, h->prefill_ws(), d_x, n, d_out, h->n_sm, st, ev);
+    if (n <= h->decode_max) {
+        DecodeWs ws = h->decode_ws();
+        ws.xres = residual ? d_x : nullptr;
+        ce = launch_decode(h->weights_view(), h->D, ws, d_x, n, d_out, h->n_sm, st, ev);
+    } else {
+        PrefillWs ws = h->prefill_ws();
+        ws.xres = residual ? d_x : nullptr;
+        ce = launch_prefill(h->weights_view(), h->D, ws, d_x, n, d_out, h->n_sm, st, ev);
+    }
     return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "forward launch");
 }
 
 ds4moe_status ds4moe_forward(ds4moe_t* h, const void* d_x, int32_t n, float* d_out, void* stream) {
     return forward_impl(h, d_x, n, d_out, nullptr, stream, "forward");
+}
+
+ds4moe_status ds4moe_forward_residual(ds4moe_t* h, const void* d_x, int32_t n, float* d_out, void* stream) {
+    return forward_impl(h, d_x, n, d_out, nullptr, stream, "forward_residual", true);
+}
+
+ds4moe_status ds4moe_forward_residual_profiled(ds4moe_t* h, const void* d_x, int32_t n, float* d_out,
+                                               void* const* events, void* stream) {
+    if (!events) return fail(DS4MOE_ERR_ARG, "forward_residual_profiled: NULL events");
+    return forward_impl(h, d_x, n, d_out, events, stream, "forward_residual_profiled", true);
 }
 
 ds4moe_status ds4moe_forward_profiled(ds4moe_t* h, const void* d_x, int32_t n, float* d_out, void* const* events,

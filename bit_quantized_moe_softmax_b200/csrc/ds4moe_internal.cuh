@@ -74,6 +74,7 @@ struct DecodeWs {
     float* h_sh;            // [n][I]
     float* y_rt;            // [n*k][H]
     float* y_sh;            // [n][H]
+    const void* xres;       // x again when the call adds the residual (out = x + layer(x)), else nullptr
 };
 
 // Workspace pointers (prefill plan).
@@ -95,9 +96,16 @@ struct PrefillWs {
     float* Y;               // [n k][H] routed outputs (unweighted)
     float* Ys;              // [n][H] shared output
     uint32_t* err;
+    const void* xres;       // x again when the call adds the residual (out = x + layer(x)), else nullptr
 };
 
 // ---------------------------------------------------------------- helpers
+// Element i of an activation array (binary32, or bf16 widened exactly).
+__device__ __forceinline__ float act_at(const void* x, int64_t i, int act_bf16) {
+    return act_bf16 ? __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(x) + i) << 16)
+                    : __ldg(reinterpret_cast<const float*>(x) + i);
+}
+
 __device__ __forceinline__ float half_bits(uint32_t b) { return __half2float(__ushort_as_half((unsigned short)b)); }
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {

@@ -731,7 +731,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
 
 // ---------------------------------------------------------------- combine
 __global__ void k_combine_prefill(Dims D, const float* ys, const float* y, const float* wts, const int32_t* pos_of_slot,
-                                  int n, float* out) {
+                                  int n, const void* xres, float* out) {
     const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // float4 index
     const int H = D.H, k = D.k;
     if (g >= (int64_t)n * H / 4) return;
@@ -746,6 +746,11 @@ __global__ void k_combine_prefill(Dims D, const float* ys, const float* y, const
         acc.y = fmaf(w, v.y, acc.y);
         acc.z = fmaf(w, v.z, acc.z);
         acc.w = fmaf(w, v.w, acc.w);
+    }
+    if (xres) {   // out = x + layer(x)
+        const int64_t e0 = (int64_t)t * H + 4 * r4;
+        acc = make_float4(act_at(xres, e0, D.act_bf16) + acc.x, act_at(xres, e0 + 1, D.act_bf16) + acc.y,
+                          act_at(xres, e0 + 2, D.act_bf16) + acc.z, act_at(xres, e0 + 3, D.act_bf16) + acc.w);
     }
     reinterpret_cast<float4*>(out + (int64_t)t * H)[r4] = acc;
 }
@@ -940,7 +945,7 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
     }
     const int64_t n4 = (int64_t)n * H / 4;
     mk.before();
-    k_combine_prefill<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(D, ws.Ys, ws.Y, ws.wts, ws.pos_of_slot, n, out);
+    k_combine_prefill<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(D, ws.Ys, ws.Y, ws.wts, ws.pos_of_slot, n, ws.xres, out);
     mk.after();
     return cudaGetLastError();
 }

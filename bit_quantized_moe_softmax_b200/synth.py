@@ -29,6 +29,14 @@ IQ2_BYTES = 66
 QK = 256
 
 
+# Scales of the chained-layer workload: superblock scales 8x below the
+# single-layer interval and a shared expert of std 0.01, so that the routed and
+# the shared part each add about 0.1 (std) to x ~ N(0, 1) per layer and 8
+# residual steps stay O(1).
+CHAIN_D_RANGE = (1e-3 / 8, 4e-3 / 8)
+CHAIN_SHARED_STD = 0.01
+
+
 def gen(seed: int, device="cpu") -> torch.Generator:
     g = torch.Generator(device=device)
     g.manual_seed(int(seed))
@@ -126,11 +134,12 @@ def float_layer(shape: Shape, seed: int, router_std=0.02, expert_std=0.02, share
 
 
 def packed_layer(shape: Shape, seed: int, router_std=0.02, shared_std=0.02,
-                 bias: torch.Tensor | None = None, device="cpu") -> dict:
+                 bias: torch.Tensor | None = None, device="cpu", d_range=(1e-3, 4e-3)) -> dict:
     """A layer whose quantized experts are drawn directly as packed blocks.
 
     Keys: W_r, b_r, grid as in float_layer; gate/up [E, I*H/256, 66] u8,
-    down [E, H*I/256, 84] u8; sh_gate/sh_up/sh_down bf16.
+    down [E, H*I/256, 84] u8; sh_gate/sh_up/sh_down bf16.  d_range: the
+    interval of the binary16 superblock scales d (and dmin).
     """
     g = gen(seed, device)
     H, I, E = shape.H, shape.I, shape.E
@@ -139,9 +148,10 @@ def packed_layer(shape: Shape, seed: int, router_std=0.02, shared_std=0.02,
     layer["W_r"] = normal((E, H), router_std, g, device)
     layer["b_r"] = bias
     layer["grid"] = grid_table(seed)
-    layer["gate"] = random_iq2_blocks(E * nb, g, device).view(E, nb, IQ2_BYTES)
-    layer["up"] = random_iq2_blocks(E * nb, g, device).view(E, nb, IQ2_BYTES)
-    layer["down"] = random_q2k_blocks(E * nb, g, device).view(E, nb, Q2_BYTES)
+    lo, hi = d_range
+    layer["gate"] = random_iq2_blocks(E * nb, g, device, lo, hi).view(E, nb, IQ2_BYTES)
+    layer["up"] = random_iq2_blocks(E * nb, g, device, lo, hi).view(E, nb, IQ2_BYTES)
+    layer["down"] = random_q2k_blocks(E * nb, g, device, lo, hi).view(E, nb, Q2_BYTES)
     if shape.shared:
         layer["sh_gate"] = bf16_normal((I, H), shared_std, g, device)
         layer["sh_up"] = bf16_normal((I, H), shared_std, g, device)

@@ -152,6 +152,14 @@ ds4moe_status ds4moe_set_shared(ds4moe_t* h, const void* d_gate, const void* d_u
  * n_tokens == 0 is a no-op.  Launches only; safe to capture in a CUDA graph. */
 ds4moe_status ds4moe_forward(ds4moe_t* h, const void* d_x, int32_t n_tokens, float* d_out, void* stream);
 
+/* out = x + layer(x): the residual step of a chain of layers (one layer's
+ * output is the next layer's input, x_{l+1} = x_l + MoE_l(x_l), with no norm
+ * in between: the pages' multi-token-prediction verify runs such chains).  The
+ * combine kernel adds x (bf16 widened exactly) after the gate-weighted sum, one
+ * binary32 add per element.  x and out must not overlap (DS4MOE_ERR_ARG);
+ * otherwise as ds4moe_forward. */
+ds4moe_status ds4moe_forward_residual(ds4moe_t* h, const void* d_x, int32_t n_tokens, float* d_out, void* stream);
+
 /* The same computation with HOST buffers: copies x_host to the device (into
  * the workspace), runs ds4moe_forward, copies the result to out_host and
  * synchronizes `stream`.  Pinned host memory gives the fastest copies. */
@@ -174,6 +182,10 @@ const char* ds4moe_plan_kernel(const ds4moe_t* h, int32_t n_tokens, int32_t i);
  * on the stream.  Same results as ds4moe_forward. */
 ds4moe_status ds4moe_forward_profiled(ds4moe_t* h, const void* d_x, int32_t n_tokens, float* d_out,
                                       void* const* events, void* stream);
+
+/* ds4moe_forward_residual with the same per-launch events. */
+ds4moe_status ds4moe_forward_residual_profiled(ds4moe_t* h, const void* d_x, int32_t n_tokens, float* d_out,
+                                               void* const* events, void* stream);
 
 /* ---- inspection hooks (same device code as the hot path) ----------------- */
 

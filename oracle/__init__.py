@@ -214,6 +214,26 @@ def moe_forward(layer: dict, x: np.ndarray, mode: int = 0):
     return out, ids, w
 
 
+def chain_forward(layers, x: np.ndarray, mode: int = 0):
+    """A chain of layers with the residual step x_{l+1} = x_l + MoE_l(x_l).
+
+    Follows the multi-token-prediction verify of the pages (ds4-server --help
+    text: MTP draft tokens verified through the model's layers) as read for a
+    stack of MoE layers with no norm in between.  Each layer's input is binary32
+    (the decode plan's activation type): the fp64 sum is rounded to binary32
+    before the next layer.  Returns (x_L as float32 [n,H], per-layer ids,
+    per-layer inputs as float32).
+    """
+    cur = np.asarray(x, dtype=np.float32).reshape(-1, int(layers[0]["H"]))
+    ids_all, inputs = [], []
+    for lay in layers:
+        inputs.append(cur.copy())
+        out, ids, _ = moe_forward(lay, cur, mode)
+        ids_all.append(ids)
+        cur = (cur.astype(np.float64) + out).astype(np.float32)
+    return cur, ids_all, inputs
+
+
 def layer_from_torch(layer: dict, experts=None) -> dict:
     """numpy view of a synthetic layer (torch tensors, any device) for moe_forward.
 

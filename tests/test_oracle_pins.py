@@ -354,6 +354,35 @@ def test_identical_experts_collapse_to_dense_ffn(orc):
     assert np.allclose(w.sum(1), 1.0, atol=1e-12)
 
 
+def test_chain_of_dense_layers(orc):
+    # two layers whose routed experts are identical: each layer is x + two dense
+    # FFNs (routed weights sum to 1, plus the shared expert), computed with torch
+    lays = [_packed_tiny(orc, identical=True, seed=s) for s in (0, 5)]
+    x = synth.tokens(3, 256, seed=6).numpy()
+    got, ids, inputs = orc.chain_forward([lay for lay, _ in lays], x)
+    cur = x.astype(np.float32)
+    for lay, L in lays:
+        grid = lay["grid"]
+        Wg = orc.dequant_iq2xxs(lay["gate"][0], grid).reshape(128, 256)
+        Wu = orc.dequant_iq2xxs(lay["up"][0], grid).reshape(128, 256)
+        Wd = orc.dequant_q2k(lay["down"][0]).reshape(256, 128)
+        xd = cur.astype(np.float64)
+        y = _dense_ffn(Wg, Wu, Wd, xd) + _dense_ffn(_bf16_f64(L["sh_gate"]), _bf16_f64(L["sh_up"]),
+                                                    _bf16_f64(L["sh_down"]), xd)
+        cur = (xd + y).astype(np.float32)
+    assert len(ids) == 2 and np.array_equal(inputs[0], x.astype(np.float32))
+    assert np.abs(got.astype(np.float64) - cur).max() <= 2 ** -20 * np.abs(cur).max()
+
+
+def test_chain_of_zero_layers_is_identity(orc):
+    lay, _ = _packed_tiny(orc, zero_routed=True)
+    for n in ("sh_gate", "sh_up", "sh_down"):
+        lay[n] = None
+    x = synth.tokens(2, 256, seed=7).numpy()
+    got, _, _ = orc.chain_forward([lay, lay, lay], x)
+    assert np.array_equal(got, x.astype(np.float32))
+
+
 def test_zero_routed_leaves_shared(orc):
     lay, L = _packed_tiny(orc, zero_routed=True)
     x = synth.tokens(3, 256, seed=2).numpy()
