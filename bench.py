@@ -187,6 +187,9 @@ def run_ours(args, wl, rank, local, world):
                                shared_std=synth.CHAIN_SHARED_STD if wl.get("chain_scales") else 0.02)
         lay = m.MoELayer(H, I, E, k, max_tokens=max(n, 8), act_dtype=act, has_bias=bias is not None, device=dev)
         lay.load(L)
+        if args.steer:
+            v = synth.normal((H,), 1.0, synth.gen(500 + r, dev), dev)
+            lay.set_steering((v / v.double().norm().float()).contiguous(), args.steer)
         layers.append(lay)
         del L
     P = 2 if prefill else 64
@@ -389,7 +392,8 @@ def run_ours(args, wl, rank, local, world):
                           "than L2" % (R, R * layers[0].weights.numel() / 1e9, P)) if not prefill else
                          "one layer (%.1f GB of weights) and %d token batches per step: inputs larger than L2"
                          % (layers[0].weights.numel() / 1e9, n),
-                   "parallelism": "dp%d replicas (no collective on the data path)" % world},
+                   "parallelism": "dp%d replicas (no collective on the data path)" % world,
+                   "steering_F": args.steer},
         "expert_weight_gbs": round(C * ab["routed"] / (ms_per_step * 1e-3) / 1e9, 1) if U else None,
         "layer_hbm_gbs": round(C * ab["layer"] / (ms_per_step * 1e-3) / 1e9, 1) if U else None,
         "layer_frac_of_hbm_peak": round(C * ab["layer"] / (ms_per_step * 1e-3) / 1e9 / peak, 4) if U else None,
@@ -483,6 +487,8 @@ def main():
     ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
     ap.add_argument("--instances", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--steer", type=float, default=0.0,
+                    help="directional steering strength F of every layer (unit direction, seeded); 0: off")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
     from bit_quantized_moe_softmax_b200 import dist as D

@@ -32,7 +32,7 @@ EXPORTS = ("ds4moe_create", "ds4moe_destroy", "ds4moe_weight_bytes", "ds4moe_wor
            "ds4moe_set_shared", "ds4moe_forward", "ds4moe_forward_host", "ds4moe_route", "ds4moe_dequant",
            "ds4moe_get_device_error", "ds4moe_last_error", "ds4moe_plan_launches", "ds4moe_plan_kernel",
            "ds4moe_forward_profiled", "ds4moe_route_noalloc", "ds4moe_forward_residual",
-           "ds4moe_forward_residual_profiled")
+           "ds4moe_forward_residual_profiled", "ds4moe_set_steering")
 
 
 class ds4moe_shape(ctypes.Structure):
@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
             "ds4moe_forward_profiled": ([vp, vp, i32, vp, ctypes.POINTER(vp), vp], i32),
             "ds4moe_route_noalloc": ([vp, vp, i32, vp, vp, vp], i32),
             "ds4moe_forward_residual": ([vp, vp, i32, vp, vp], i32),
+            "ds4moe_set_steering": ([vp, vp, ctypes.c_float, vp], i32),
             "ds4moe_forward_residual_profiled": ([vp, vp, i32, vp, ctypes.POINTER(vp), vp], i32),
         }
         for name, (args, res) in sig.items():
@@ -160,6 +161,11 @@ def ds4moe_set_shared(h: int, gate: torch.Tensor, up: torch.Tensor, down: torch.
 
 def ds4moe_forward(h: int, x: torch.Tensor, out: torch.Tensor, stream=None):
     _ok(lib().ds4moe_forward(h, _ptr(x), x.shape[0], _ptr(out), _stream(stream)), "ds4moe_forward")
+
+
+def ds4moe_set_steering(h: int, v: torch.Tensor | None, F: float, stream=None):
+    _ok(lib().ds4moe_set_steering(h, None if v is None else _ptr(v), ctypes.c_float(F), _stream(stream)),
+        "ds4moe_set_steering")
 
 
 def ds4moe_forward_residual(h: int, x: torch.Tensor, out: torch.Tensor, stream=None):
@@ -290,6 +296,10 @@ class MoELayer:
             out = torch.empty(x.shape[0], self.H, dtype=torch.float32, device=x.device)
         (ds4moe_forward_residual if residual else ds4moe_forward)(self.h, x, out)
         return out
+
+    def set_steering(self, v: torch.Tensor | None, F: float = 1.0):
+        """Steer the layer output: y -= F v (v . y) (v: [H] binary32 on the device; None turns it off)."""
+        ds4moe_set_steering(self.h, v, F)
 
     def route(self, x: torch.Tensor):
         ids = torch.empty(x.shape[0], self.k, dtype=torch.int32, device=x.device)

@@ -833,6 +833,40 @@ __global__ void __launch_bounds__(256) k_combine_decode(Dims D, DecodeWs ws, flo
     out[i] = ws.xres ? act_at(ws.xres, i, D.act_bf16) + acc : acc;
 }
 
+// The combine with directional steering of the layer output: one CTA per
+// token; y = y_shared + sum_j w_j y_j as above, then y - F v (v . y) with
+// v . y summed in a fixed order (per thread over its columns, then the CTA),
+// one FMA per element, then x + that when the call asks for the residual.
+constexpr int kSteerThreads = 256;
+
+__global__ void __launch_bounds__(kSteerThreads) k_combine_steer_decode(Dims D, DecodeWs ws, float* out, int n) {
+    griddep_wait();   // y of the down grid
+    __shared__ float red[kSteerThreads / 32];
+    const int t = blockIdx.x, H = D.H, k = D.k;
+    float acc[16];   // H <= 4096 = 16 columns per thread
+    float dot = 0.f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+        const int r = threadIdx.x + q * kSteerThreads;
+        if (r < H) {
+            float a = D.has_shared ? __ldcg(ws.y_sh + (int64_t)t * H + r) : 0.f;
+            for (int j = 0; j < k; ++j)
+                a = fmaf(__ldcg(ws.wts + t * k + j), __ldcg(ws.y_rt + (int64_t)(t * k + j) * H + r), a);
+            acc[q] = a;
+            dot = fmaf(ws.steer_v[r], a, dot);
+        }
+    }
+    const float sF = ws.steer_F * cta_sum_fixed<kSteerThreads>(dot, red);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+        const int r = threadIdx.x + q * kSteerThreads;
+        if (r < H) {
+            const float y = fmaf(-sF, ws.steer_v[r], acc[q]);
+            out[(int64_t)t * H + r] = ws.xres ? act_at(ws.xres, (int64_t)t * H + r, D.act_bf16) + y : y;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- launchers
 template <int NT>
 size_t gateup_smem_bytes(const Dims& D, int n) {
@@ -936,7 +970,10 @@ cudaError_t launch_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws,
     if (err != cudaSuccess) return err;
     const int64_t nel = (int64_t)n * D.H;
     mk.before();
-    err = launch_pdl(k_combine_decode, dim3((unsigned)((nel + 255) / 256)), dim3(256), 0, st, pdl, D, ws, out, n);
+    if (ws.steer_v)
+        err = launch_pdl(k_combine_steer_decode, dim3((unsigned)n), dim3(kSteerThreads), 0, st, pdl, D, ws, out, n);
+    else
+        err = launch_pdl(k_combine_decode, dim3((unsigned)((nel + 255) / 256)), dim3(256), 0, st, pdl, D, ws, out, n);
     mk.after();
     if (err != cudaSuccess) return err;
     return cudaGetLastError();

@@ -88,7 +88,7 @@ struct ds4moe {
     int decode_max;
     int n_sm;
     // weight buffer layout
-    size_t off_grid, off_Wr, off_Wr2, off_br, off_gate_qs, off_gate_d, off_up_qs, off_up_d, off_down_q, off_down_sc,
+    size_t off_grid, off_Wr, off_Wr2, off_br, off_steer, off_gate_qs, off_gate_d, off_up_qs, off_up_d, off_down_q, off_down_sc,
         off_down_dd, off_sh_gate, off_sh_up, off_sh_down, weight_bytes;
     size_t iq2_qs_stride, iq2_d_stride, q2_q_stride, q2_sc_stride, q2_dd_stride;
     uint8_t* weights = nullptr;
@@ -97,6 +97,8 @@ struct ds4moe {
     WsLayout L{};
     std::vector<uint8_t> loaded;
     bool grid_set = false, router_set = false, shared_set = false;
+    bool steer_on = false;   // directional steering of the layer output (ds4moe_set_steering)
+    float steer_F = 0.f;
 
     WsLayout layout(int cap) const {
         WsLayout w{};
@@ -276,6 +278,7 @@ ds4moe_status ds4moe_create(const ds4moe_shape* s, ds4moe_t** out) {
     h->off_Wr = o; o += align256(E * H * 4);
     h->off_Wr2 = o; o += align256(s->max_tokens > h->decode_max ? (E + 1) / 2 * 2 * H * 4 : 0);
     h->off_br = o; o += align256(E * 4);
+    h->off_steer = o; o += align256(H * 4);
     h->off_gate_qs = o; o += align256(E * h->iq2_qs_stride);
     h->off_gate_d = o; o += align256(E * h->iq2_d_stride * 2);
     h->off_up_qs = o; o += align256(E * h->iq2_qs_stride);
@@ -379,6 +382,24 @@ ds4moe_status ds4moe_set_router(ds4moe_t* h, const float* d_W, const float* d_bi
     return DS4MOE_OK;
 }
 
+ds4moe_status ds4moe_set_steering(ds4moe_t* h, const float* d_v, float F, void* stream) {
+    if (!h) return fail(DS4MOE_ERR_ARG, "set_steering: NULL handle");
+    if (!h->weights) return fail(DS4MOE_ERR_NOT_READY, "set_steering: buffers not bound");
+    if (!d_v || F == 0.f) {   // off
+        h->steer_on = false;
+        h->steer_F = 0.f;
+        return DS4MOE_OK;
+    }
+    if (h->D.H > 4096) return fail(DS4MOE_ERR_SHAPE, "set_steering: hidden %d above 4096", h->D.H);
+    if (!(F == F) || F - F != 0.f) return fail(DS4MOE_ERR_ARG, "set_steering: F not finite");
+    cudaError_t ce = cudaMemcpyAsync(h->weights + h->off_steer, d_v, (size_t)h->D.H * 4, cudaMemcpyDeviceToDevice,
+                                     (cudaStream_t)stream);
+    if (ce != cudaSuccess) return cuda_fail(ce, "set_steering copy");
+    h->steer_on = true;
+    h->steer_F = F;
+    return DS4MOE_OK;
+}
+
 ds4moe_status ds4moe_set_expert(ds4moe_t* h, int32_t e, const void* d_gate, const void* d_up, const void* d_down,
                                 void* stream) {
     if (!h || !d_gate || !d_up || !d_down) return fail(DS4MOE_ERR_ARG, "set_expert: NULL argument");
@@ -449,10 +470,14 @@ static ds4moe_status forward_impl(ds4moe_t* h, const void* d_x, int32_t n, float
     if (n <= h->decode_max) {
         DecodeWs ws = h->decode_ws();
         ws.xres = residual ? d_x : nullptr;
+        ws.steer_v = h->steer_on ? reinterpret_cast<const float*>(h->weights + h->off_steer) : nullptr;
+        ws.steer_F = h->steer_F;
         ce = launch_decode(h->weights_view(), h->D, ws, d_x, n, d_out, h->n_sm, st, ev);
     } else {
         PrefillWs ws = h->prefill_ws();
         ws.xres = residual ? d_x : nullptr;
+        ws.steer_v = h->steer_on ? reinterpret_cast<const float*>(h->weights + h->off_steer) : nullptr;
+        ws.steer_F = h->steer_F;
         ce = launch_prefill(h->weights_view(), h->D, ws, d_x, n, d_out, h->n_sm, st, ev);
     }
     return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "forward launch");
@@ -485,7 +510,9 @@ int32_t ds4moe_plan_launches(const ds4moe_t* h, int32_t n) {
 }
 
 const char* ds4moe_plan_kernel(const ds4moe_t* h, int32_t n, int32_t i) {
-    if (i < 0 || i >= ds4moe_plan_launches(h, n)) return nullptr;
+    const int nl = ds4moe_plan_launches(h, n);
+    if (i < 0 || i >= nl) return nullptr;
+    if (h->steer_on && i == nl - 1) return n <= h->decode_max ? "k_combine_steer_decode" : "k_combine_steer_prefill";
     if (n <= h->decode_max) return decode_kernel_name(i);
     return prefill_kernel_name(h->D, i);
 }

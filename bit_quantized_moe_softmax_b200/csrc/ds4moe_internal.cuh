@@ -75,6 +75,8 @@ struct DecodeWs {
     float* y_rt;            // [n*k][H]
     float* y_sh;            // [n][H]
     const void* xres;       // x again when the call adds the residual (out = x + layer(x)), else nullptr
+    const float* steer_v;   // [H] steering direction, or nullptr (no steering)
+    float steer_F;          // steering strength: y -= F v (v . y)
 };
 
 // Workspace pointers (prefill plan).
@@ -97,9 +99,28 @@ struct PrefillWs {
     float* Ys;              // [n][H] shared output
     uint32_t* err;
     const void* xres;       // x again when the call adds the residual (out = x + layer(x)), else nullptr
+    const float* steer_v;   // [H] steering direction, or nullptr (no steering)
+    float steer_F;          // steering strength: y -= F v (v . y)
 };
 
 // ---------------------------------------------------------------- helpers
+// Sum of one float per thread over a CTA of NT threads in a fixed order
+// (butterfly in each warp, then the warp sums in warp order); every thread
+// gets the result.  red: NT / 32 floats of shared memory.
+template <int NT>
+__device__ __forceinline__ float cta_sum_fixed(float v, float* red) {
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+    const int warp = threadIdx.x >> 5;
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[warp] = v;
+    __syncthreads();
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) s += red[w];
+    return s;
+}
+
 // Element i of an activation array (binary32, or bf16 widened exactly).
 __device__ __forceinline__ float act_at(const void* x, int64_t i, int act_bf16) {
     return act_bf16 ? __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(x) + i) << 16)

@@ -755,6 +755,43 @@ __global__ void k_combine_prefill(Dims D, const float* ys, const float* y, const
     reinterpret_cast<float4*>(out + (int64_t)t * H)[r4] = acc;
 }
 
+// The combine with directional steering of the layer output (one CTA per
+// token): y as above, then y - F v (v . y) with v . y summed in a fixed order,
+// then x + that when the call asks for the residual.
+constexpr int kSteerThreadsP = 256;
+
+__global__ void __launch_bounds__(kSteerThreadsP) k_combine_steer_prefill(Dims D, const float* ys, const float* y,
+                                                                          const float* wts, const int32_t* pos_of_slot,
+                                                                          const float* v, float F, const void* xres,
+                                                                          float* out) {
+    __shared__ float red[kSteerThreadsP / 32];
+    const int t = blockIdx.x, H = D.H, k = D.k;
+    float acc[16];   // H <= 4096
+    float dot = 0.f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+        const int r = threadIdx.x + q * kSteerThreadsP;
+        if (r < H) {
+            float a = D.has_shared ? __ldg(ys + (int64_t)t * H + r) : 0.f;
+            for (int j = 0; j < k; ++j) {
+                const int pos = __ldg(pos_of_slot + (int64_t)t * k + j);
+                a = fmaf(__ldg(wts + (int64_t)t * k + j), __ldg(y + (int64_t)pos * H + r), a);
+            }
+            acc[q] = a;
+            dot = fmaf(v[r], a, dot);
+        }
+    }
+    const float sF = F * cta_sum_fixed<kSteerThreadsP>(dot, red);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+        const int r = threadIdx.x + q * kSteerThreadsP;
+        if (r < H) {
+            const float o = fmaf(-sF, v[r], acc[q]);
+            out[(int64_t)t * H + r] = xres ? act_at(xres, (int64_t)t * H + r, D.act_bf16) + o : o;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- host side
 size_t gemm_smem_bytes() { return 1024 + (size_t)kGStages * (kGAStage + kGBStage) + kGSelBytes; }
 // Static shared memory of the GEMM kernels (the largest of the four modes).
@@ -945,7 +982,12 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
     }
     const int64_t n4 = (int64_t)n * H / 4;
     mk.before();
-    k_combine_prefill<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(D, ws.Ys, ws.Y, ws.wts, ws.pos_of_slot, n, ws.xres, out);
+    if (ws.steer_v)
+        k_combine_steer_prefill<<<(unsigned)n, kSteerThreadsP, 0, st>>>(D, ws.Ys, ws.Y, ws.wts, ws.pos_of_slot,
+                                                                      ws.steer_v, ws.steer_F, ws.xres, out);
+    else
+        k_combine_prefill<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(D, ws.Ys, ws.Y, ws.wts, ws.pos_of_slot, n,
+                                                                        ws.xres, out);
     mk.after();
     return cudaGetLastError();
 }

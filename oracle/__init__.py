@@ -214,6 +214,18 @@ def moe_forward(layer: dict, x: np.ndarray, mode: int = 0):
     return out, ids, w
 
 
+def steer(y: np.ndarray, v: np.ndarray, F: float) -> np.ndarray:
+    """Directional steering of a layer output, per token: y - F v (v . y), in fp64.
+
+    Follows the pages' server option that applies steering after FFN outputs
+    (ds4-server --help, "--dir-steering-ffn F": y -= F*v*dot(v,y), one f32
+    direction vector per layer).
+    """
+    y = np.asarray(y, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float32).astype(np.float64)
+    return y - float(F) * np.outer(y @ v, v)
+
+
 def chain_forward(layers, x: np.ndarray, mode: int = 0):
     """A chain of layers with the residual step x_{l+1} = x_l + MoE_l(x_l).
 

@@ -383,6 +383,22 @@ def test_chain_of_zero_layers_is_identity(orc):
     assert np.array_equal(got, x.astype(np.float32))
 
 
+def test_steer_closed_forms(orc):
+    rng = np.random.default_rng(0)
+    y = rng.standard_normal((5, 64))
+    v = rng.standard_normal(64).astype(np.float32)
+    v = (v / np.linalg.norm(v.astype(np.float64))).astype(np.float32)
+    vd = v.astype(np.float64)
+    for F in (0.0, 0.3, 1.0, 2.5):
+        ys = orc.steer(y, v, F)
+        nv = vd @ vd   # 1 up to the binary32 rounding of v
+        # the component along v scales by 1 - F |v|^2; the orthogonal part is unchanged
+        assert np.allclose(ys @ vd, (1 - F * nv) * (y @ vd), rtol=0, atol=1e-12)
+        perp = lambda a: a - np.outer(a @ vd, vd) / nv
+        assert np.allclose(perp(ys), perp(y), rtol=0, atol=1e-12)
+    assert np.array_equal(orc.steer(y, v, 0.0), y)
+
+
 def test_zero_routed_leaves_shared(orc):
     lay, L = _packed_tiny(orc, zero_routed=True)
     x = synth.tokens(3, 256, seed=2).numpy()
