@@ -91,7 +91,11 @@ def algorithmic_bytes(w: dict, U: int) -> dict:
 
 
 def traffic_from_profile(kernel: str, workload: str):
-    """dram bytes per launch recorded under profiles/, if the kernel source is unchanged since."""
+    """dram bytes per launch recorded under profiles/, if the kernel's sources are unchanged since.
+
+    The summary names its sources ("source_files: a.cu b.cuh", under the
+    package's csrc/) and the sha256 of their bytes concatenated in that order.
+    """
     name = kernel.replace("<", "_").replace(">", "")
     p = os.path.join(ROOT, "profiles", "%s_%s.md" % (name, workload))
     if not os.path.exists(p):
@@ -99,13 +103,16 @@ def traffic_from_profile(kernel: str, workload: str):
     txt = open(p).read()
     m1 = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
     m2 = re.search(r"source_sha256:\s*([0-9a-f]+)", txt)
-    m3 = re.search(r"source_file:\s*([A-Za-z0-9_.]+)", txt)
-    if not (m1 and m2):
+    m3 = re.search(r"source_files:\s*([A-Za-z0-9_. ]+)", txt)
+    if not (m1 and m2 and m3):
         return None
-    src = os.path.join(ROOT, "bit_quantized_moe_softmax_b200", "csrc", m3.group(1) if m3 else "decode.cu")
-    if not os.path.exists(src):
-        return None
-    if hashlib.sha256(open(src, "rb").read()).hexdigest() != m2.group(1):
+    h = hashlib.sha256()
+    for f in m3.group(1).split():
+        src = os.path.join(ROOT, "bit_quantized_moe_softmax_b200", "csrc", f)
+        if not os.path.exists(src):
+            return None
+        h.update(open(src, "rb").read())
+    if h.hexdigest() != m2.group(1):
         return None
     return float(m1.group(1))
 

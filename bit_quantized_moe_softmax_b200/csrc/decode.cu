@@ -837,16 +837,17 @@ __global__ void __launch_bounds__(256) k_combine_decode(Dims D, DecodeWs ws, flo
 // token; y = y_shared + sum_j w_j y_j as above, then y - F v (v . y) with
 // v . y summed in a fixed order (per thread over its columns, then the CTA),
 // one FMA per element, then x + that when the call asks for the residual.
-constexpr int kSteerThreads = 256;
+constexpr int kSteerThreads = 1024;   // few tokens: one wide CTA per token
+constexpr int kSteerCols = 4;          // columns per thread (H <= 4096)
 
 __global__ void __launch_bounds__(kSteerThreads) k_combine_steer_decode(Dims D, DecodeWs ws, float* out, int n) {
     griddep_wait();   // y of the down grid
     __shared__ float red[kSteerThreads / 32];
     const int t = blockIdx.x, H = D.H, k = D.k;
-    float acc[16];   // H <= 4096 = 16 columns per thread
+    float acc[kSteerCols];
     float dot = 0.f;
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
+    for (int q = 0; q < kSteerCols; ++q) {
         const int r = threadIdx.x + q * kSteerThreads;
         if (r < H) {
             float a = D.has_shared ? __ldcg(ws.y_sh + (int64_t)t * H + r) : 0.f;
@@ -858,7 +859,7 @@ __global__ void __launch_bounds__(kSteerThreads) k_combine_steer_decode(Dims D, 
     }
     const float sF = ws.steer_F * cta_sum_fixed<kSteerThreads>(dot, red);
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
+    for (int q = 0; q < kSteerCols; ++q) {
         const int r = threadIdx.x + q * kSteerThreads;
         if (r < H) {
             const float y = fmaf(-sF, ws.steer_v[r], acc[q]);

@@ -765,29 +765,52 @@ __global__ void __launch_bounds__(kSteerThreadsP) k_combine_steer_prefill(Dims D
                                                                           const float* v, float F, const void* xres,
                                                                           float* out) {
     __shared__ float red[kSteerThreadsP / 32];
+    __shared__ int s_pos[16];
+    __shared__ float s_w[16];
     const int t = blockIdx.x, H = D.H, k = D.k;
-    float acc[16];   // H <= 4096
+    if (threadIdx.x < k) {
+        s_pos[threadIdx.x] = __ldg(pos_of_slot + (int64_t)t * k + threadIdx.x);
+        s_w[threadIdx.x] = __ldg(wts + (int64_t)t * k + threadIdx.x);
+    }
+    __syncthreads();
+    float4 acc[4];   // H <= 4096: four float4 column groups per thread
     float dot = 0.f;
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-        const int r = threadIdx.x + q * kSteerThreadsP;
-        if (r < H) {
-            float a = D.has_shared ? __ldg(ys + (int64_t)t * H + r) : 0.f;
+    for (int q = 0; q < 4; ++q) {
+        const int c4 = threadIdx.x + q * kSteerThreadsP;   // float4 index in the row
+        if (4 * c4 < H) {
+            float4 a = D.has_shared ? __ldg(reinterpret_cast<const float4*>(ys + (int64_t)t * H) + c4)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
             for (int j = 0; j < k; ++j) {
-                const int pos = __ldg(pos_of_slot + (int64_t)t * k + j);
-                a = fmaf(__ldg(wts + (int64_t)t * k + j), __ldg(y + (int64_t)pos * H + r), a);
+                const float w = s_w[j];
+                const float4 yv = __ldg(reinterpret_cast<const float4*>(y + (int64_t)s_pos[j] * H) + c4);
+                a.x = fmaf(w, yv.x, a.x);
+                a.y = fmaf(w, yv.y, a.y);
+                a.z = fmaf(w, yv.z, a.z);
+                a.w = fmaf(w, yv.w, a.w);
             }
             acc[q] = a;
-            dot = fmaf(v[r], a, dot);
+            const float4 vv = __ldg(reinterpret_cast<const float4*>(v) + c4);
+            dot = fmaf(vv.x, a.x, dot);
+            dot = fmaf(vv.y, a.y, dot);
+            dot = fmaf(vv.z, a.z, dot);
+            dot = fmaf(vv.w, a.w, dot);
         }
     }
     const float sF = F * cta_sum_fixed<kSteerThreadsP>(dot, red);
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-        const int r = threadIdx.x + q * kSteerThreadsP;
-        if (r < H) {
-            const float o = fmaf(-sF, v[r], acc[q]);
-            out[(int64_t)t * H + r] = xres ? act_at(xres, (int64_t)t * H + r, D.act_bf16) + o : o;
+    for (int q = 0; q < 4; ++q) {
+        const int c4 = threadIdx.x + q * kSteerThreadsP;
+        if (4 * c4 < H) {
+            const float4 vv = __ldg(reinterpret_cast<const float4*>(v) + c4);
+            float4 o = make_float4(fmaf(-sF, vv.x, acc[q].x), fmaf(-sF, vv.y, acc[q].y), fmaf(-sF, vv.z, acc[q].z),
+                                   fmaf(-sF, vv.w, acc[q].w));
+            if (xres) {
+                const int64_t e0 = (int64_t)t * H + 4 * c4;
+                o = make_float4(act_at(xres, e0, D.act_bf16) + o.x, act_at(xres, e0 + 1, D.act_bf16) + o.y,
+                                act_at(xres, e0 + 2, D.act_bf16) + o.z, act_at(xres, e0 + 3, D.act_bf16) + o.w);
+            }
+            reinterpret_cast<float4*>(out + (int64_t)t * H)[c4] = o;
         }
     }
 }
