@@ -26,15 +26,16 @@
 namespace ds4 {
 
 // ---------------------------------------------------------------- router
-// CTA: 16 warps as 4 token groups x 4 expert groups, warp tile 8 tokens x 8
-// experts (4 expert pairs) -> CTA tile 32 tokens x 32 experts.  The 32 x 128
+// CTA: 8 warps as 4 token groups x 2 expert groups, warp tile 8 tokens x 8
+// experts (4 expert pairs) -> CTA tile 32 tokens x 16 experts.  The 32 x 128
 // slices of x and of the pair-interleaved router rows (W_r2: for each column the
 // weights of experts 2p and 2p+1 side by side) for each 128-column step stream
 // into a kRP_S-stage shared-memory ring with 16-byte asynchronous copies (rows
 // past n or E are zero-filled).  Lane L multiplies columns 4L .. 4L+3 of the
 // slice into its chain, fma in column order; one packed FMA advances the
 // chains of an expert pair, whose weights arrive as adjacent words.
-constexpr int kRP_T = 32, kRP_E = 32, kRP_S = 4;
+constexpr int kRP_T = 32, kRP_E = 16, kRP_S = 4;
+constexpr int kRP_Threads = 256;   // 8 warps; two CTAs per SM overlap each other's step barriers
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(valid ? 16 : 0)
@@ -45,7 +46,7 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <bool BF16X>
-__global__ void __launch_bounds__(512, 1) k_router_prefill(Weights W, Dims D, const void* x, int n, float* logits) {
+__global__ void __launch_bounds__(kRP_Threads, 2) k_router_prefill(Weights W, Dims D, const void* x, int n, float* logits) {
     constexpr int XB = BF16X ? 2 : 4;                       // bytes per x element
     constexpr int XSTAGE = kRP_T * 128 * XB, WSTAGE = kRP_E * 128 * 4;
     extern __shared__ __align__(16) unsigned char rp_smem[];
@@ -61,14 +62,14 @@ __global__ void __launch_bounds__(512, 1) k_router_prefill(Weights W, Dims D, co
         unsigned char* xs = rp_smem + (i % kRP_S) * (XSTAGE + WSTAGE);
         unsigned char* ws = xs + XSTAGE;
         // x: 32 rows x (128 * XB) bytes
-        for (int q = tid; q < kRP_T * 8 * XB; q += 512) {
+        for (int q = tid; q < kRP_T * 8 * XB; q += kRP_Threads) {
             const int row = q / (8 * XB), c = q % (8 * XB);
             const int t = t0 + row;
             const bool ok = t < n;
             cp_async16(xs + row * 128 * XB + 16 * c, xb + ((int64_t)(ok ? t : 0) * H + 128 * i) * XB + 16 * c, ok);
         }
-        // W_r2: 16 expert pairs x 1024 bytes
-        for (int q = tid; q < (kRP_E / 2) * 64; q += 512) {
+        // W_r2: kRP_E / 2 expert pairs x 1024 bytes
+        for (int q = tid; q < (kRP_E / 2) * 64; q += kRP_Threads) {
             const int pr = q >> 6, c = q & 63;
             const int p = p0 + pr;
             const bool ok = p < npairs;
@@ -159,7 +160,7 @@ static cudaError_t launch_router_prefill(const Weights& W, const Dims& D, const 
             if (e != cudaSuccess) return e;
             configured[dev] = true;
         }
-        k_router_prefill<true><<<grid, 512, smem, st>>>(W, D, x, n, logits);
+        k_router_prefill<true><<<grid, kRP_Threads, smem, st>>>(W, D, x, n, logits);
     } else {
         const int smem = kRP_S * (kRP_T * 128 * 4 + kRP_E * 128 * 4);
         static bool configured[64] = {};
@@ -170,7 +171,7 @@ static cudaError_t launch_router_prefill(const Weights& W, const Dims& D, const 
             if (e != cudaSuccess) return e;
             configured[dev] = true;
         }
-        k_router_prefill<false><<<grid, 512, smem, st>>>(W, D, x, n, logits);
+        k_router_prefill<false><<<grid, kRP_Threads, smem, st>>>(W, D, x, n, logits);
     }
     return cudaGetLastError();
 }
