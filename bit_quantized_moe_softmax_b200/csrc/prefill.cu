@@ -270,23 +270,26 @@ __global__ void __launch_bounds__(kSortBlock) k_scatter(const int32_t* ids, int 
     }
 }
 
-// Xp[pos][:] = bf16(x[slot / k][:]), 8 elements per thread.
-__global__ void k_gather(const void* x, int act_bf16, const int32_t* slot_of_pos, int nslots, int k, int H,
-                         __nv_bfloat16* Xp) {
-    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+// Xp[pos][:] = bf16(x[slot / k][:]): 64 threads per row (4 rows per 256-thread
+// block), 16-byte pieces, the row's source looked up once.
+__global__ void __launch_bounds__(256) k_gather(const void* x, int act_bf16, const int32_t* slot_of_pos, int nslots,
+                                                int k, int H, __nv_bfloat16* Xp) {
+    const int pos = blockIdx.x * 4 + (threadIdx.x >> 6), l = threadIdx.x & 63;
+    if (pos >= nslots) return;
     const int per = H / 8;
-    if (g >= (int64_t)nslots * per) return;
-    const int pos = (int)(g / per), c8 = (int)(g % per);
-    const int t = slot_of_pos[pos] / k;
-    uint4 v;
+    const int64_t t = __ldg(slot_of_pos + pos) / k;
+    uint4* dst = reinterpret_cast<uint4*>(Xp + (int64_t)pos * H);
     if (act_bf16) {
-        v = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(x) + (int64_t)t * H) + c8);
+        const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(x) + t * H);
+        for (int c8 = l; c8 < per; c8 += 64) dst[c8] = __ldg(src + c8);
     } else {
-        const float4* xr = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + (int64_t)t * H) + 2 * c8;
-        const float4 a = __ldg(xr), b = __ldg(xr + 1);
-        v = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+        const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + t * H);
+        for (int c8 = l; c8 < per; c8 += 64) {
+            const float4 a = __ldg(src + 2 * c8), b = __ldg(src + 2 * c8 + 1);
+            dst[c8] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                                 pack_bf16x2(b.z, b.w));
+        }
     }
-    reinterpret_cast<uint4*>(Xp + (int64_t)pos * H)[c8] = v;
 }
 
 // x (binary32) -> bf16, for the shared expert's A operand.
@@ -961,9 +964,8 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
     k_scatter<<<nblk, kSortBlock, 32 * E * sizeof(int), st>>>(ws.ids, nslots, E, ws.blk_off, ws.pos_of_slot,
                                                                ws.slot_of_pos);
     mk.after();
-    const int64_t ng = (int64_t)nslots * H / 8;
     mk.before();
-    k_gather<<<(unsigned)((ng + 255) / 256), 256, 0, st>>>(x, D.act_bf16, ws.slot_of_pos, nslots, k, H, ws.Xp);
+    k_gather<<<(unsigned)((nslots + 3) / 4), 256, 0, st>>>(x, D.act_bf16, ws.slot_of_pos, nslots, k, H, ws.Xp);
     mk.after();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 

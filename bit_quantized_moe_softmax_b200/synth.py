@@ -165,10 +165,6 @@ def tokens(n: int, H: int, seed: int, dtype=torch.float32, device="cpu") -> torc
     return normal((n, H), 1.0, g, device).to(dtype)
 
 
-def zipf_s(default: float = 1.1) -> float:
-    return default
-
-
 def router_std_unit_logits(H: int) -> float:
     """Router row std that makes x . w ~ N(0, 1) for x ~ N(0, 1)."""
     return 1.0 / math.sqrt(H)

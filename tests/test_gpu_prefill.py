@@ -101,3 +101,25 @@ def test_prefill_full_shape_short_prompt(orc):
     need = rid[sample].ravel()
     ref, _, _ = orc.moe_forward(oracle_layer(L, experts=need), x[sample].float().numpy(), mode=1)
     assert rel_err(out[sample], ref) < TOL
+
+
+def test_prefill_full_shape_long_prompt(orc):
+    """The long-prompt workload at full size (11,709 bf16 tokens, Zipf(1.1)), in the launch configuration the
+    bench times: routing ids exact for every token, outputs checked on sampled tokens."""
+    bias = synth.zipf_bias(256, 1.1, seed=5)
+    L = synth.packed_layer(synth.FULL, 7, bias=bias, device="cuda")
+    n = 11709
+    lay = _gpu(L, max_tokens=n)
+    x = synth.tokens(n, 4096, seed=12, dtype=torch.bfloat16)
+    out = lay.forward(x.cuda()).cpu().numpy()
+    ids, _ = lay.route(x.cuda())
+    lg = orc.router_logits(x.float().numpy(), L["W_r"].cpu().numpy(), bias.numpy())
+    rid, _ = orc.topk_softmax(lg, 8)
+    assert np.array_equal(ids.cpu().numpy(), rid)
+    counts = np.bincount(rid.ravel(), minlength=256)
+    assert counts.max() > 1000 and (counts < 128).sum() > 100   # the skew the workload is about
+    sample = [0, 1, 4096, 8191, n - 2, n - 1]
+    need = rid[sample].ravel()
+    ref, _, _ = orc.moe_forward(oracle_layer(L, experts=need), x[sample].float().numpy(), mode=1)
+    assert rel_err(out[sample], ref) < TOL
+    assert np.isfinite(out).all()
