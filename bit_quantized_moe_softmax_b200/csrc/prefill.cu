@@ -318,7 +318,7 @@ struct GemmArgs {
 
 struct GemmSmem {
     uint64_t fullA[kGStages], fullB[kGStages], empty[kGStages];
-    uint64_t accF, accE, done;
+    uint64_t accF[2], accE[2], done;   // per accumulator buffer (TMEM columns 0..255, 256..511)
     uint32_t tmem_base;
     int abort;
     int nval;          // distinct grid magnitudes (gate/up mode)
@@ -440,8 +440,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
             mbar_init(&S.fullB[s], kGDqWarps);
             mbar_init(&S.empty[s], 1);
         }
-        mbar_init(&S.accF, 1);
-        mbar_init(&S.accE, kGEpiWarps);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&S.accF[b], 1);
+            mbar_init(&S.accE[b], kGEpiWarps / 2);
+        }
         mbar_init(&S.done, 1);
         S.abort = 0;
         fence_barrier_init();
@@ -527,12 +529,20 @@ __global__ void __launch_bounds__(kGThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issue: two 128 x 256 x 16 MMAs per k16 share B
         const uint32_t idesc = umma_idesc_bf16(kGHalf, kGBN);
-        uint32_t it = 0, lt = 0;
-        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(S); tile += gridDim.x, ++lt) {
+        // A 256-row tile uses both accumulator buffers (its two row halves); a tile of at most 128
+        // rows uses one, alternating, so that its epilogue overlaps the next such tile's MMAs.
+        uint32_t it = 0, use0 = 0, use1 = 0, hc = 0;   // completed uses of each buffer
+        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(S); tile += gridDim.x) {
             const TileInfo ti = tile_info<MODE>(a, tile, NB);
             const bool two = ti.mvalid > kGHalf;
-            if (!mbar_wait(&S.accE, (lt & 1) ^ 1, a.err)) { g_set_abort(S); break; }
+            const int b1 = two ? 0 : (int)(hc++ & 1u);   // buffer of the tile's first row half
+            if (!mbar_wait(&S.accE[b1], ((b1 ? use1 : use0) & 1) ^ 1, a.err) ||
+                (two && !mbar_wait(&S.accE[1], (use1 & 1) ^ 1, a.err))) {
+                g_set_abort(S);
+                break;
+            }
             tc_fence_after();
+            const uint32_t dt0 = tmem + (uint32_t)b1 * kGBN;
             for (int ks = 0; ks < KS; ++ks, ++it) {
                 const int s = it % kGStages;
                 const uint32_t ph = (it / kGStages) & 1;
@@ -550,7 +560,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     constexpr uint32_t bstep = 16u;
 #pragma unroll
                     for (int kk = 0; kk < kGBK / 16; ++kk) {
-                        umma_bf16(tmem, da0 + 2 * kk, db + bstep * kk, idesc, (ks | kk) != 0);
+                        umma_bf16(dt0, da0 + 2 * kk, db + bstep * kk, idesc, (ks | kk) != 0);
                         if (two) umma_bf16(tmem + kGBN, da1 + 2 * kk, db + bstep * kk, idesc, (ks | kk) != 0);
                     }
                     umma_commit(&S.empty[s]);
@@ -558,8 +568,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 __syncwarp();
             }
             if (g_aborted(S)) break;
-            if (lane == 0) umma_commit(&S.accF);
+            if (lane == 0) {
+                umma_commit(&S.accF[b1]);
+                if (two) umma_commit(&S.accF[1]);
+            }
             __syncwarp();
+            if (two || b1 == 0) ++use0;
+            if (two || b1 == 1) ++use1;
         }
         // every issued MMA has finished before TMEM is released
         if (lane == 0) umma_commit(&S.done);
@@ -677,17 +692,23 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
     } else {
         // ------------------------------------------------ epilogue (TMEM -> registers -> global)
+        // warps 10..13 drain buffer 0 and warps 14..17 buffer 1, following the MMA warp's assignment
         const int qd = warp & 3;                          // TMEM lanes 32 qd .. 32 qd + 31
-        const int half = (warp - 2 - kGDqWarps) >> 2;     // accumulator (row half) of this warp
-        const int m = kGHalf * half + 32 * qd + lane;     // tile row of this thread
-        uint32_t lt = 0;
-        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(S); tile += gridDim.x, ++lt) {
+        const int bg = (warp - 2 - kGDqWarps) >> 2;       // accumulator buffer of this warp
+        uint32_t use = 0, hc = 0;
+        for (int tile = blockIdx.x; tile < ntiles && !g_aborted(S); tile += gridDim.x) {
             const TileInfo ti = tile_info<MODE>(a, tile, NB);
-            if (!mbar_wait(&S.accF, lt & 1, a.err)) { g_set_abort(S); break; }
+            const bool two = ti.mvalid > kGHalf;
+            const int b1 = two ? 0 : (int)(hc++ & 1u);
+            if (!two && b1 != bg) continue;               // the other buffer's warps drain this tile
+            const int half = two ? bg : 0;                // row half of the tile held in this buffer
+            const int m = kGHalf * half + 32 * qd + lane; // tile row of this thread
+            if (!mbar_wait(&S.accF[bg], use & 1, a.err)) { g_set_abort(S); break; }
+            ++use;
             tc_fence_after();
-            const uint32_t taddr = tmem + ((uint32_t)(32 * qd) << 16) + half * kGBN;
+            const uint32_t taddr = tmem + ((uint32_t)(32 * qd) << 16) + bg * kGBN;
             const bool live = m < ti.mvalid;
-            if (ti.mvalid > kGHalf * half) {   // this half was computed
+            {
                 // 16-column TMEM reads; each thread stores 32-byte pieces of its own row
                 if (kGateUp) {
                     __nv_bfloat16* dst = a.out_h + (size_t)(ti.row0 + m) * I + 128 * ti.nb;
@@ -722,7 +743,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&S.accE);
+            if (lane == 0) mbar_arrive(&S.accE[bg]);
         }
     }
     tc_fence_before();
