@@ -1,4 +1,4 @@
-// decode.cu -- the fp32 GEMV plan for 1..decode_max tokens (three launches).
+// decode.cu -- the fp32 GEMV plan for 1..decode_max tokens (four launches).
 //
 //   k_router_decode  warp per expert row, logits in the canonical binary32
 //                    order; the last CTA picks the top-k by (logit desc,
@@ -7,13 +7,16 @@
 //                    (read once, applied to all tokens that chose it) and for
 //                    the shared expert.
 //   k_down_decode    y = W_down h per selected expert and for the shared
-//                    expert; the last task to finish a 32-row block of the
-//                    output sums out = y_shared + sum_j w_j y_j in rank order.
+//                    expert.
+//   k_combine_decode out = y_shared + sum_j w_j y_j in rank order (then
+//                    x + that for the residual step; k_combine_steer_decode
+//                    also steers: y - F v (v . y)).
 //
 // The two GEMV kernels are persistent (one CTA per SM): a producer warp pulls
 // row tasks from an atomic queue and streams their weights into a ring of
-// shared-memory stages with bulk copies (cp.async.bulk + mbarrier), eight
-// consumer warps dequantize and multiply out of shared memory.  Each is
+// shared-memory stages with bulk copies (cp.async.bulk + mbarrier), 16 (for
+// up to 2 tokens; 8 otherwise) consumer warps dequantize and multiply out of
+// shared memory.  Each is
 // launched with programmatic dependent launch: the gate/up grid starts its
 // shared-expert tasks while the router still runs, and the down grid streams
 // its weights while gate/up finishes; both wait (griddepcontrol.wait) only

@@ -9,13 +9,15 @@
 //                      offs[e] + (number of earlier slots with the same expert)
 //   k_gather           Xp[pos] = bf16(x[slot(pos) / k])
 //   k_moe_gemm<mode>   persistent grouped GEMM on tcgen05: per (expert,
-//                      128-row tile, n tile) D[128 x 256] = A[128 x K] B[256 x K]^T
-//                      with A = permuted activations (TMA, 128-byte swizzle)
-//                      and B = the expert's weights dequantized to bf16 in
-//                      shared memory by eight warps, accumulators in TMEM
-//                      (two 256-column buffers), epilogue by four warps:
-//                      gate/up -> silu(g) * u as bf16, down -> binary32
+//                      256-row tile, n tile) D[256 x 256] = A[256 x K] B[256 x K]^T
+//                      as two 128-row MMA halves sharing B; A = permuted
+//                      activations (TMA, 128-byte swizzle), B = the expert's
+//                      weights dequantized to bf16 in shared memory by eight
+//                      warps (shared expert: copied by TMA), accumulators in
+//                      TMEM, epilogue by eight warps: gate/up -> silu(g) * u
+//                      as bf16, down -> binary32
 //   k_combine_prefill  out = y_shared + sum_j w_j y_{pos(t, j)}, rank order
+//                      (k_combine_steer_prefill: then y - F v (v . y))
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
