@@ -974,11 +974,12 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
     k_scan<<<1, 1024, 0, st>>>(ws.blk_cnt, nblk, E, ws.counts, ws.offs, ws.blk_off, ws.mt_prefix);
     mk.after();
     {
+        // opt in once per device for the largest expert count a handle may have (1024)
         static bool big[64] = {};
         int dev = 0;
         cudaGetDevice(&dev);
         if (32 * E * sizeof(int) > 48 * 1024 && dev < 64 && !big[dev]) {
-            e = cudaFuncSetAttribute(k_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * E * (int)sizeof(int));
+            e = cudaFuncSetAttribute(k_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 1024 * (int)sizeof(int));
             if (e != cudaSuccess) return e;
             big[dev] = true;
         }
