@@ -32,7 +32,8 @@ EXPORTS = ("ds4moe_create", "ds4moe_destroy", "ds4moe_weight_bytes", "ds4moe_wor
            "ds4moe_set_shared", "ds4moe_forward", "ds4moe_forward_host", "ds4moe_route", "ds4moe_dequant",
            "ds4moe_get_device_error", "ds4moe_last_error", "ds4moe_plan_launches", "ds4moe_plan_kernel",
            "ds4moe_forward_profiled", "ds4moe_route_noalloc", "ds4moe_forward_residual",
-           "ds4moe_forward_residual_profiled", "ds4moe_set_steering")
+           "ds4moe_forward_residual_profiled", "ds4moe_set_steering", "ds4moe_forward_host_async",
+           "ds4moe_host_sync")
 
 
 class ds4moe_shape(ctypes.Structure):
@@ -69,6 +70,8 @@ def lib() -> ctypes.CDLL:
             "ds4moe_set_shared": ([vp, vp, vp, vp, vp], i32),
             "ds4moe_forward": ([vp, vp, i32, vp, vp], i32),
             "ds4moe_forward_host": ([vp, vp, i32, vp, vp], i32),
+            "ds4moe_forward_host_async": ([vp, vp, i32, vp, vp], i32),
+            "ds4moe_host_sync": ([vp], i32),
             "ds4moe_route": ([vp, vp, i32, vp, vp, vp], i32),
             "ds4moe_dequant": ([vp, i32, i32, i32, vp, vp], i32),
             "ds4moe_get_device_error": ([vp, vp, ctypes.POINTER(i32)], i32),
@@ -197,6 +200,16 @@ def ds4moe_forward_profiled(h: int, x: torch.Tensor, out: torch.Tensor, events, 
 def ds4moe_forward_host(h: int, x_host: torch.Tensor, out_host: torch.Tensor, stream=None):
     _ok(lib().ds4moe_forward_host(h, _ptr(x_host), x_host.shape[0], _ptr(out_host), _stream(stream)),
         "ds4moe_forward_host")
+
+
+def ds4moe_forward_host_async(h: int, x_host: torch.Tensor, out_host: torch.Tensor, stream=None):
+    """Enqueue a host-buffer forward; out_host is valid after ds4moe_host_sync(h)."""
+    _ok(lib().ds4moe_forward_host_async(h, _ptr(x_host), x_host.shape[0], _ptr(out_host), _stream(stream)),
+        "ds4moe_forward_host_async")
+
+
+def ds4moe_host_sync(h: int):
+    _ok(lib().ds4moe_host_sync(h), "ds4moe_host_sync")
 
 
 def ds4moe_route(h: int, x: torch.Tensor, ids: torch.Tensor, w: torch.Tensor, stream=None):

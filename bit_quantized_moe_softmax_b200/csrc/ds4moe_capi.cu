@@ -74,6 +74,7 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
 struct WsLayout {
     size_t hdr, rbtick, logits, ids, wts, h_rt, hsum_rt, h_sh, y_rt, y_sh, x_stage, out_stage;
+    size_t x_slot, out_slot;   // bytes of one of the two staging slots of the host-buffer calls
     // prefill plan (capacity > decode_max only)
     size_t p_logits, p_ids, p_wts, p_blk_cnt, p_blk_off, p_counts, p_offs, p_mtp, p_pos, p_slot, p_xb, p_Xp, p_Hb,
         p_Hs, p_Y, p_Ys;
@@ -99,6 +100,38 @@ struct ds4moe {
     bool grid_set = false, router_set = false, shared_set = false;
     bool steer_on = false;   // directional steering of the layer output (ds4moe_set_steering)
     float steer_F = 0.f;
+    // host-buffer calls: upload / download streams (created on first use) and,
+    // per staging slot, the events of its upload, its forward and its download
+    cudaStream_t up = nullptr, down = nullptr;
+    cudaEvent_t ev_in[2] = {}, ev_done[2] = {}, ev_out[2] = {};
+    int slot = 0;
+
+    ~ds4moe() { release_host_streams(); }
+    void release_host_streams() {
+        if (up) cudaStreamSynchronize(up);
+        if (down) cudaStreamSynchronize(down);
+        for (int i = 0; i < 2; ++i) {
+            if (ev_in[i]) cudaEventDestroy(ev_in[i]);
+            if (ev_done[i]) cudaEventDestroy(ev_done[i]);
+            if (ev_out[i]) cudaEventDestroy(ev_out[i]);
+            ev_in[i] = ev_done[i] = ev_out[i] = nullptr;
+        }
+        if (up) cudaStreamDestroy(up);
+        if (down) cudaStreamDestroy(down);
+        up = down = nullptr;
+    }
+    cudaError_t host_streams() {
+        if (up) return cudaSuccess;
+        cudaError_t e = cudaStreamCreateWithFlags(&up, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&down, cudaStreamNonBlocking);
+        for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+            e = cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_done[i], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_out[i], cudaEventDisableTiming);
+        }
+        if (e != cudaSuccess) release_host_streams();
+        return e;
+    }
 
     WsLayout layout(int cap) const {
         WsLayout w{};
@@ -115,8 +148,10 @@ struct ds4moe {
         w.h_sh = o; o += align256(nd * I * 4);
         w.y_rt = o; o += align256(nd * k * H * 4);
         w.y_sh = o; o += align256(nd * H * 4);
-        w.x_stage = o; o += align256((size_t)cap * H * (D.act_bf16 ? 2 : 4));
-        w.out_stage = o; o += align256((size_t)cap * H * 4);
+        w.x_slot = align256((size_t)cap * H * (D.act_bf16 ? 2 : 4));
+        w.out_slot = align256((size_t)cap * H * 4);
+        w.x_stage = o; o += 2 * w.x_slot;
+        w.out_stage = o; o += 2 * w.out_slot;
         if (cap > decode_max) {
             const size_t N = cap, NK = N * k, nblk = (NK + 1023) / 1024;
             w.p_logits = o; o += align256(N * E * 4);
@@ -517,21 +552,51 @@ const char* ds4moe_plan_kernel(const ds4moe_t* h, int32_t n, int32_t i) {
     return prefill_kernel_name(h->D, i);
 }
 
-ds4moe_status ds4moe_forward_host(ds4moe_t* h, const void* x_host, int32_t n, float* out_host, void* stream) {
-    ds4moe_status s = check_forward(h, x_host, n, out_host, "forward_host");
+ds4moe_status ds4moe_forward_host_async(ds4moe_t* h, const void* x_host, int32_t n, float* out_host, void* stream) {
+    ds4moe_status s = check_forward(h, x_host, n, out_host, "forward_host_async");
     if (s != DS4MOE_OK) return s;
     if (n == 0) return DS4MOE_OK;
+    cudaError_t ce = h->host_streams();
+    if (ce != cudaSuccess) return cuda_fail(ce, "forward_host_async: streams");
     cudaStream_t st = (cudaStream_t)stream;
+    const int sl = h->slot;
+    h->slot ^= 1;
     const size_t xb = (size_t)n * h->D.H * (h->D.act_bf16 ? 2 : 4), ob = (size_t)n * h->D.H * 4;
-    void* dx = h->ws + h->L.x_stage;
-    float* dout = reinterpret_cast<float*>(h->ws + h->L.out_stage);
-    cudaError_t ce = cudaMemcpyAsync(dx, x_host, xb, cudaMemcpyHostToDevice, st);
-    if (ce != cudaSuccess) return cuda_fail(ce, "forward_host: copy in");
+    void* dx = h->ws + h->L.x_stage + sl * h->L.x_slot;
+    float* dout = reinterpret_cast<float*>(h->ws + h->L.out_stage + sl * h->L.out_slot);
+    // upload into the slot once the forward that last read it is done
+    ce = cudaStreamWaitEvent(h->up, h->ev_done[sl], 0);
+    if (ce == cudaSuccess) ce = cudaMemcpyAsync(dx, x_host, xb, cudaMemcpyHostToDevice, h->up);
+    if (ce == cudaSuccess) ce = cudaEventRecord(h->ev_in[sl], h->up);
+    // the forward once its input has landed and the slot's last result has left
+    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(st, h->ev_in[sl], 0);
+    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(st, h->ev_out[sl], 0);
+    if (ce != cudaSuccess) return cuda_fail(ce, "forward_host_async: copy in");
     s = ds4moe_forward(h, dx, n, dout, stream);
     if (s != DS4MOE_OK) return s;
-    ce = cudaMemcpyAsync(out_host, dout, ob, cudaMemcpyDeviceToHost, st);
-    if (ce != cudaSuccess) return cuda_fail(ce, "forward_host: copy out");
-    ce = cudaStreamSynchronize(st);
+    ce = cudaEventRecord(h->ev_done[sl], st);
+    // download once the forward is done
+    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(h->down, h->ev_done[sl], 0);
+    if (ce == cudaSuccess) ce = cudaMemcpyAsync(out_host, dout, ob, cudaMemcpyDeviceToHost, h->down);
+    if (ce == cudaSuccess) ce = cudaEventRecord(h->ev_out[sl], h->down);
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "forward_host_async: copy out");
+}
+
+ds4moe_status ds4moe_host_sync(ds4moe_t* h) {
+    if (!h) return fail(DS4MOE_ERR_ARG, "host_sync: NULL handle");
+    if (!h->up) return DS4MOE_OK;
+    cudaError_t ce = cudaStreamSynchronize(h->up);
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(h->down);   // its copies follow the forwards
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "host_sync");
+}
+
+ds4moe_status ds4moe_forward_host(ds4moe_t* h, const void* x_host, int32_t n, float* out_host, void* stream) {
+    ds4moe_status s = ds4moe_forward_host_async(h, x_host, n, out_host, stream);
+    if (s != DS4MOE_OK) return s;
+    if (n == 0) return DS4MOE_OK;
+    s = ds4moe_host_sync(h);
+    if (s != DS4MOE_OK) return s;
+    const cudaError_t ce = cudaStreamSynchronize((cudaStream_t)stream);
     return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "forward_host: synchronize");
 }
 

@@ -171,10 +171,33 @@ ds4moe_status ds4moe_forward(ds4moe_t* h, const void* d_x, int32_t n_tokens, flo
 ds4moe_status ds4moe_forward_residual(ds4moe_t* h, const void* d_x, int32_t n_tokens, float* d_out, void* stream);
 
 /* The same computation with HOST buffers: copies x_host to the device (into
- * the workspace), runs ds4moe_forward, copies the result to out_host and
- * synchronizes `stream`.  Pinned host memory gives the fastest copies. */
+ * the workspace), runs ds4moe_forward on `stream`, copies the result to
+ * out_host and waits for all of it (ds4moe_forward_host_async followed by
+ * ds4moe_host_sync and a synchronize of `stream`).  Pinned host memory gives
+ * the fastest copies. */
 ds4moe_status ds4moe_forward_host(ds4moe_t* h, const void* x_host, int32_t n_tokens, float* out_host,
                                   void* stream);
+
+/* Pipelined host-buffer forward; returns without waiting.  The workspace holds
+ * two staging slots that consecutive calls of a handle alternate between.  A
+ * call enqueues (1) the copy of x_host into its slot, on the handle's own
+ * upload stream, after the forward that last read that slot; (2) ds4moe_forward
+ * on `stream`, after that copy and after the slot's previous result has been
+ * copied out; (3) the copy of the result to out_host, on the handle's own
+ * download stream, after the forward.  So one call's copies overlap the
+ * kernels of its neighbours.  out_host holds the result after
+ * ds4moe_host_sync(h); until then x_host must stay unchanged and out_host
+ * untouched.  The streams and events are created on the first call (not
+ * allowed during stream capture) on the current device and released by
+ * ds4moe_destroy.  Errors: as ds4moe_forward; DS4MOE_ERR_CUDA if a copy or
+ * an event operation fails.  Not thread-safe per handle. */
+ds4moe_status ds4moe_forward_host_async(ds4moe_t* h, const void* x_host, int32_t n_tokens, float* out_host,
+                                        void* stream);
+
+/* Waits until every copy enqueued by ds4moe_forward_host_async on h has
+ * finished (and with them the forwards they follow).  DS4MOE_OK at once if
+ * the handle has made no such call. */
+ds4moe_status ds4moe_host_sync(ds4moe_t* h);
 
 /* ---- measurement ---------------------------------------------------------- */
 

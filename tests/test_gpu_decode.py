@@ -184,6 +184,26 @@ def test_forward_host_buffers(orc):
     assert torch.equal(out, ref)
 
 
+@pytest.mark.parametrize("n,max_tokens", [(3, 8), (40, 64)])
+def test_forward_host_async_pipeline(orc, n, max_tokens):
+    """Pipelined host-buffer calls: six calls in flight over the two staging
+    slots (decode and prefill plans), a blocking call in between; every
+    result equals the device-buffer forward of the same input bit for bit."""
+    L = _tiny(orc)
+    lay = _layer_on_gpu(L, max_tokens=max_tokens)
+    xs = [synth.tokens(n, 256, seed=100 + i).pin_memory() for i in range(6)]
+    outs = [torch.full((n, 256), float("nan"), dtype=torch.float32).pin_memory() for _ in range(6)]
+    for i in range(3):
+        m.ds4moe_forward_host_async(lay.h, xs[i], outs[i])
+    m.ds4moe_forward_host(lay.h, xs[3], outs[3])
+    for i in range(4, 6):
+        m.ds4moe_forward_host_async(lay.h, xs[i], outs[i])
+    m.ds4moe_host_sync(lay.h)
+    for i in range(6):
+        assert torch.equal(outs[i], lay.forward(xs[i].cuda()).cpu()), i
+    m.ds4moe_host_sync(lay.h)   # nothing pending: returns at once
+
+
 def test_forward_full_decode_shape(orc):
     """One token through a full-size layer (H 4096, I 2048, 256 experts top-8, bf16 shared)."""
     L = synth.packed_layer(synth.FULL, 0, device="cuda")
