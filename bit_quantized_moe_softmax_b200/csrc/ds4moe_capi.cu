@@ -353,6 +353,10 @@ ds4moe_status ds4moe_bind(ds4moe_t* h, void* d_weights, size_t weight_bytes, voi
         return fail(DS4MOE_ERR_ARG, "bind: weight buffer %zu bytes < %zu", weight_bytes, h->weight_bytes);
     WsLayout L = h->layout(h->shape.max_tokens);
     if (ws_bytes < L.total) return fail(DS4MOE_ERR_ARG, "bind: workspace %zu bytes < %zu", ws_bytes, L.total);
+    // pipelined host-buffer calls still in flight use the old staging slots
+    ds4moe_status hs = ds4moe_host_sync(h);
+    if (hs != DS4MOE_OK) return hs;
+    h->slot = 0;
     cudaError_t ce = cudaMemsetAsync(static_cast<uint8_t*>(d_workspace) + L.hdr, 0, L.logits - L.hdr,
                                      (cudaStream_t)stream);
     if (ce != cudaSuccess) return cuda_fail(ce, "bind: cudaMemsetAsync");
