@@ -21,6 +21,10 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "ds4moe_internal.cuh"
 #include "tcgen05.cuh"
 #include "topk.cuh"
@@ -148,31 +152,34 @@ __global__ void __launch_bounds__(kRP_Threads, 2) k_router_prefill(Weights W, Di
     }
 }
 
+// Raises a kernel's dynamic shared-memory limit to at least `bytes`, once per
+// (kernel, device) and thread-safe; the limit only ever grows.
+static cudaError_t smem_opt_in(const void* kernel, int bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, int> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    int& cur = done[std::make_pair(kernel, dev)];
+    if (cur >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) cur = bytes;
+    return e;
+}
+
 // Launch of the router for n tokens (stage ring in dynamic shared memory).
 static cudaError_t launch_router_prefill(const Weights& W, const Dims& D, const void* x, int n, float* logits,
                                          cudaStream_t st) {
     const dim3 grid((n + kRP_T - 1) / kRP_T, (D.E + kRP_E - 1) / kRP_E);
+    cudaError_t e;
     if (D.act_bf16) {
         const int smem = kRP_S * (kRP_T * 128 * 2 + kRP_E * 128 * 4);
-        static bool configured[64] = {};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (dev < 64 && !configured[dev]) {
-            cudaError_t e = cudaFuncSetAttribute(k_router_prefill<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e != cudaSuccess) return e;
-            configured[dev] = true;
-        }
+        if ((e = smem_opt_in(reinterpret_cast<const void*>(k_router_prefill<true>), smem)) != cudaSuccess) return e;
         k_router_prefill<true><<<grid, kRP_Threads, smem, st>>>(W, D, x, n, logits);
     } else {
         const int smem = kRP_S * (kRP_T * 128 * 4 + kRP_E * 128 * 4);
-        static bool configured[64] = {};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (dev < 64 && !configured[dev]) {
-            cudaError_t e = cudaFuncSetAttribute(k_router_prefill<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e != cudaSuccess) return e;
-            configured[dev] = true;
-        }
+        if ((e = smem_opt_in(reinterpret_cast<const void*>(k_router_prefill<false>), smem)) != cudaSuccess) return e;
         k_router_prefill<false><<<grid, kRP_Threads, smem, st>>>(W, D, x, n, logits);
     }
     return cudaGetLastError();
@@ -856,14 +863,13 @@ size_t gemm_static_smem_bytes() {
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
         cudaDriverEntryPointQueryResult q;
         void* p = nullptr;
         cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
         if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p) return nullptr;
-        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
     return fn;
 }
 
@@ -900,16 +906,9 @@ static cudaError_t encode_tmap_core(CUtensorMap* map, const void* base, uint64_t
 template <int MODE>
 static cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
                                const GemmArgs& args, int n_sm, cudaStream_t st) {
-    static bool configured[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
     const size_t smem = gemm_smem_bytes();
-    if (dev < 64 && !configured[dev]) {
-        e = cudaFuncSetAttribute(k_moe_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured[dev] = true;
-    }
+    cudaError_t e = smem_opt_in(reinterpret_cast<const void*>(k_moe_gemm<MODE>), (int)smem);
+    if (e != cudaSuccess) return e;
     k_moe_gemm<MODE><<<n_sm, kGThreads, smem, st>>>(mapA, mapB0, mapB1, args);
     return cudaGetLastError();
 }
@@ -973,17 +972,9 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
     mk.before();
     k_scan<<<1, 1024, 0, st>>>(ws.blk_cnt, nblk, E, ws.counts, ws.offs, ws.blk_off, ws.mt_prefix);
     mk.after();
-    {
-        // opt in once per device for the largest expert count a handle may have (1024)
-        static bool big[64] = {};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (32 * E * sizeof(int) > 48 * 1024 && dev < 64 && !big[dev]) {
-            e = cudaFuncSetAttribute(k_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 1024 * (int)sizeof(int));
-            if (e != cudaSuccess) return e;
-            big[dev] = true;
-        }
-    }
+    if (32 * E * sizeof(int) > 48 * 1024 &&
+        (e = smem_opt_in(reinterpret_cast<const void*>(k_scatter), 32 * E * (int)sizeof(int))) != cudaSuccess)
+        return e;
     mk.before();
     k_scatter<<<nblk, kSortBlock, 32 * E * sizeof(int), st>>>(ws.ids, nslots, E, ws.blk_off, ws.pos_of_slot,
                                                                ws.slot_of_pos);
