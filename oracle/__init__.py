@@ -24,6 +24,7 @@ _lib = None
 QK = 256
 Q2_BYTES = 84
 IQ2_BYTES = 66
+Q4_BYTES = 144
 
 
 def build(force: bool = False) -> str:
@@ -63,6 +64,9 @@ def lib():
         L.orc_dequant_iq2xxs.argtypes = [vp, i64, vp, vp]
         L.orc_pack_q2k.argtypes = [vp, i64, vp]
         L.orc_pack_q2k.restype = ctypes.c_int
+        L.orc_dequant_q4k.argtypes = [vp, i64, vp]
+        L.orc_pack_q4k.argtypes = [vp, i64, vp]
+        L.orc_pack_q4k.restype = ctypes.c_int
         L.orc_pack_iq2xxs.argtypes = [vp, i64, vp, vp]
         L.orc_pack_iq2xxs.restype = ctypes.c_int
         L.orc_router_logit.argtypes = [vp, vp, i32, vp]
@@ -121,6 +125,22 @@ def pack_q2k(w: np.ndarray) -> np.ndarray:
     out = np.zeros((x.size // QK, Q2_BYTES), dtype=np.uint8)
     if lib().orc_pack_q2k(_p(x), x.size, _p(out)) != 0:
         raise ValueError("pack_q2k: size must be a multiple of 256")
+    return out
+
+
+def dequant_q4k(blocks: np.ndarray) -> np.ndarray:
+    """Q4_K-style blocks (144 bytes / 256 weights, the 4-bit expert variant) -> binary32."""
+    b = _c(blocks, np.uint8).reshape(-1, Q4_BYTES)
+    out = np.empty(b.shape[0] * QK, dtype=np.float32)
+    lib().orc_dequant_q4k(_p(b), b.shape[0], _p(out))
+    return out
+
+
+def pack_q4k(w: np.ndarray) -> np.ndarray:
+    x = _c(w, np.float32).ravel()
+    out = np.zeros((x.size // QK, Q4_BYTES), dtype=np.uint8)
+    if lib().orc_pack_q4k(_p(x), x.size, _p(out)) != 0:
+        raise ValueError("pack_q4k: size must be a multiple of 256")
     return out
 
 

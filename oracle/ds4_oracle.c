@@ -38,6 +38,7 @@
 #define ORC_QK 256                 /* weights per superblock, both formats */
 #define ORC_Q2_BYTES 84            /* Q2_K-style block size */
 #define ORC_IQ2_BYTES 66           /* IQ2_XXS-style block size */
+#define ORC_Q4_BYTES 144           /* Q4_K-style block size (4-bit experts) */
 
 /* ------------------------------------------------------------------------ */
 /* IEEE binary16 and bfloat16, written from their definitions.               */
@@ -136,6 +137,47 @@ void orc_dequant_q2k(const uint8_t* blocks, int64_t n_blocks, float* out) {
 }
 
 /* ------------------------------------------------------------------------ */
+/* Q4_K-style superblock (144 bytes / 256 weights), the 4-bit routed-expert  */
+/* variant.  The pages name 4-bit models (q4, q4-imatrix) but describe no    */
+/* format; this reading carries the Q2_K-style structure over to 4-bit      */
+/* codes and 32-weight sub-blocks:                                           */
+/*   [0,2)    d    (binary16, little endian)                                 */
+/*   [2,4)    dmin (binary16, little endian)                                 */
+/*   [4,16)   sixteen 6-bit fields of the little-endian 96-bit integer of    */
+/*            these bytes: field f at bits 6f..6f+5; f = j is sc_j, f = 8+j  */
+/*            is m_j, sub-block j = weights 32j..32j+31                      */
+/*   [16,144) code q_i of weight i at byte 16 + i/2, low nibble for even i   */
+/* weight_i = (d*sc_j)*q_i - dmin*m_j, rounded once to binary32 (the double  */
+/* difference is exact while the lowest set bits of the two products are    */
+/* at most 32 binary places apart, as in every block a packer writes for    */
+/* weights of one magnitude).                                                */
+/* ------------------------------------------------------------------------ */
+static int orc_q4_field(const uint8_t* p, int f) {
+    /* bits 6f..6f+5 of bytes 4..15 read as one little-endian integer */
+    int v = 0;
+    for (int b = 0; b < 6; ++b) {
+        int bit = 6 * f + b;
+        v |= ((p[4 + bit / 8] >> (bit % 8)) & 1) << b;
+    }
+    return v;
+}
+
+void orc_dequant_q4k(const uint8_t* blocks, int64_t n_blocks, float* out) {
+    for (int64_t b = 0; b < n_blocks; ++b) {
+        const uint8_t* p = blocks + b * ORC_Q4_BYTES;
+        double d = orc_half_to_double(rd16(p + 0));
+        double dmin = orc_half_to_double(rd16(p + 2));
+        for (int i = 0; i < ORC_QK; ++i) {
+            int j = i / 32;
+            int sc = orc_q4_field(p, j), m = orc_q4_field(p, 8 + j);
+            int q = (p[16 + i / 2] >> (4 * (i % 2))) & 15;
+            double v = d * sc * q - dmin * m;
+            out[b * ORC_QK + i] = (float)v;     /* one rounding to binary32 */
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* IQ2_XXS-style superblock (66 bytes / 256 weights).                        */
 /*   [0,2)  d (binary16, little endian)                                      */
 /*   group g = 0..7 at offset 2 + 8g, covering weights 32g..32g+31:          */
@@ -221,6 +263,61 @@ int orc_pack_q2k(const float* w, int64_t n, uint8_t* out) {
         }
         p[80] = dh & 0xff; p[81] = dh >> 8;
         p[82] = mh & 0xff; p[83] = mh >> 8;
+    }
+    return 0;
+}
+
+/* Q4_K-style packer, per superblock (the Q2_K-style rule with 15 code steps
+ * and 6-bit fields):
+ *   per sub-block j (32 weights): lo = min(0, min w), hi = max(0, max w),
+ *                                 scale_j = (hi - lo)/15, min_j = -lo
+ *   d = half(max scale_j / 63), dmin = half(max min_j / 63)
+ *   sc_j = clamp(rne(scale_j/d), 0, 63), m_j = clamp(rne(min_j/dmin), 0, 63)
+ *   q_i  = clamp(rne((w_i + dmin*m_j)/(d*sc_j)), 0, 15)
+ * (a zero divisor gives a zero field).  n must be a multiple of 256. */
+static void orc_q4_set_field(uint8_t* p, int f, int v) {
+    for (int b = 0; b < 6; ++b) {
+        int bit = 6 * f + b;
+        if ((v >> b) & 1) p[4 + bit / 8] |= (uint8_t)(1 << (bit % 8));
+    }
+}
+
+int orc_pack_q4k(const float* w, int64_t n, uint8_t* out) {
+    if (n % ORC_QK) return -1;
+    for (int64_t b = 0; b < n / ORC_QK; ++b) {
+        const float* x = w + b * ORC_QK;
+        uint8_t* p = out + b * ORC_Q4_BYTES;
+        double scale[8], mn[8], max_scale = 0.0, max_min = 0.0;
+        for (int j = 0; j < 8; ++j) {
+            double lo = 0.0, hi = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double v = x[32 * j + i];
+                if (v < lo) lo = v;
+                if (v > hi) hi = v;
+            }
+            scale[j] = (hi - lo) / 15.0;
+            mn[j] = -lo;
+            if (scale[j] > max_scale) max_scale = scale[j];
+            if (mn[j] > max_min) max_min = mn[j];
+        }
+        uint16_t dh = orc_double_to_half(max_scale / 63.0);
+        uint16_t mh = orc_double_to_half(max_min / 63.0);
+        double d = orc_half_to_double(dh), dmin = orc_half_to_double(mh);
+        memset(p, 0, ORC_Q4_BYTES);
+        for (int j = 0; j < 8; ++j) {
+            int sc = d > 0.0 ? (int)clampd(nearbyint(scale[j] / d), 0, 63) : 0;
+            int m = dmin > 0.0 ? (int)clampd(nearbyint(mn[j] / dmin), 0, 63) : 0;
+            orc_q4_set_field(p, j, sc);
+            orc_q4_set_field(p, 8 + j, m);
+            double step = d * sc, off = dmin * m;
+            for (int i = 0; i < 32; ++i) {
+                int q = step > 0.0 ? (int)clampd(nearbyint((x[32 * j + i] + off) / step), 0, 15) : 0;
+                int k = 32 * j + i;
+                p[16 + k / 2] |= (uint8_t)(q << (4 * (k % 2)));
+            }
+        }
+        p[0] = dh & 0xff; p[1] = dh >> 8;
+        p[2] = mh & 0xff; p[3] = mh >> 8;
     }
     return 0;
 }

@@ -106,6 +106,94 @@ def test_q2k_dequant_rounds_once_to_binary32(orc):
     assert out[1] == np.float32(-15 * 2.0 ** -24)
 
 
+# ---------------------------------------------------------------- Q4_K-style (4-bit experts)
+def _q4_block(d, dmin, sc, m, q):
+    """144-byte block written from the layout: d, dmin binary16; sixteen 6-bit
+    fields (sc_0..7 then m_0..7) packed little-endian into bytes 4..15; codes
+    two per byte, low nibble first."""
+    b = np.zeros(144, dtype=np.uint8)
+    b[0:2] = np.frombuffer(np.array(d, np.float16).tobytes(), np.uint8)
+    b[2:4] = np.frombuffer(np.array(dmin, np.float16).tobytes(), np.uint8)
+    fields = 0
+    for f, v in enumerate(list(sc) + list(m)):
+        fields |= int(v) << (6 * f)
+    b[4:16] = np.frombuffer(fields.to_bytes(12, "little"), np.uint8)
+    for i in range(256):
+        b[16 + i // 2] |= int(q[i]) << (4 * (i % 2))
+    return b
+
+
+def test_q4k_dequant_closed_form(orc):
+    i = np.arange(256)
+    j = i // 32
+    sc, m = 8 * np.arange(8) + 7, 63 - 8 * np.arange(8)
+    out = orc.dequant_q4k(_q4_block(1.0, 0.5, sc, m, i % 16))
+    assert np.array_equal(out, (sc[j] * (i % 16) - 0.5 * m[j]).astype(np.float32))
+
+
+def test_q4k_field_bytes(orc):
+    # single fields set at the byte level: bit 6 of byte 4 is sc_1's lowest bit,
+    # bit 0 of byte 10 (bit 48) is m_0's, bits 2..7 of byte 15 (90..95) are m_7
+    b = np.zeros(144, dtype=np.uint8)
+    b[0:2] = [0x00, 0x40]            # d = 2
+    b[2:4] = [0x00, 0x34]            # dmin = 0.25
+    b[4] = 0x40                      # sc_1 = 1
+    b[10] = 0x01                     # m_0 = 1
+    b[15] = 0xFC                     # m_7 = 63
+    b[16:144] = 0x33                 # every code 3
+    b[16] = 0x21                     # q_0 = 1, q_1 = 2
+    out = orc.dequant_q4k(b)
+    exp = np.zeros(256, dtype=np.float32)
+    exp[0:32] = -0.25
+    exp[0], exp[1] = 2 * 0 * 1 - 0.25, 2 * 0 * 2 - 0.25
+    exp[32:64] = 2 * 1 * 3
+    exp[224:256] = -0.25 * 63
+    assert np.array_equal(out, exp)
+    # a second block after it keeps its own fields
+    two = orc.dequant_q4k(np.concatenate([_q4_block(1.0, 0.5, [1] * 8, [0] * 8, np.full(256, 15)), b]))
+    assert np.array_equal(two[:256], np.full(256, 15, np.float32)) and np.array_equal(two[256:], exp)
+
+
+def test_q4k_pack_exact_roundtrip(orc):
+    # codes 0..15 times step = 63 * 2^-6, no negatives: d = 2^-6, sc = 63, dmin = 0
+    rng = np.random.default_rng(7)
+    step = 63 * 2.0 ** -6
+    q = rng.integers(0, 16, (3, 256))
+    q[:, ::32] = 15
+    w = (q * step).astype(np.float32)
+    blocks = orc.pack_q4k(w)
+    assert blocks.shape == (3, 144)
+    assert np.array_equal(orc.dequant_q4k(blocks), w.ravel())
+    assert all(bytes(bl[0:2]) == np.array(2.0 ** -6, np.float16).tobytes() for bl in blocks)
+    assert np.all(blocks[:, 2:4] == 0)
+    assert np.array_equal(blocks[0], _q4_block(2.0 ** -6, 0.0, [63] * 8, [0] * 8, q[0]))
+
+
+def test_q4k_pack_zero_error_and_finer_than_q2k(orc):
+    assert not orc.pack_q4k(np.zeros(512, np.float32)).any()
+    with pytest.raises(ValueError):
+        orc.pack_q4k(np.zeros(300, np.float32))
+    rng = np.random.default_rng(8)
+    w = (rng.standard_normal(256 * 64) * 0.02).astype(np.float32)
+    r4 = orc.dequant_q4k(orc.pack_q4k(w))
+    r2 = orc.dequant_q2k(orc.pack_q2k(w))
+    e4 = np.sqrt(np.mean((r4 - w) ** 2)) / np.std(w)
+    e2 = np.sqrt(np.mean((r2 - w) ** 2)) / np.std(w)
+    assert e4 < 0.1 and e4 < e2 / 3, (e4, e2)   # 4.5 bits per weight against 2.6
+    # error of each weight: half a code step, plus what rounding the fields
+    # costs -- sc_j off by <= 1/2 (times 15 steps of d) and m_j by <= 1/2 (of dmin)
+    for blk, wb in zip(orc.pack_q4k(w), w.reshape(-1, 256)):
+        d = float(np.frombuffer(blk[0:2].tobytes(), np.float16)[0])
+        dmin = float(np.frombuffer(blk[2:4].tobytes(), np.float16)[0])
+        fields = int.from_bytes(blk[4:16].tobytes(), "little")
+        sc = [(fields >> (6 * j)) & 63 for j in range(8)]
+        dq = orc.dequant_q4k(blk).astype(np.float64)
+        for j in range(8):
+            s = slice(32 * j, 32 * j + 32)
+            bound = 0.5 * d * sc[j] + 7.5 * d + 0.5 * dmin
+            assert np.all(np.abs(dq[s] - wb[s]) <= bound * (1 + 1e-6))
+
+
 def _iq2_block(d_bits, groups):
     """groups: list of 8 tuples (indices[4], sigmas[4], s)."""
     b = np.zeros(66, dtype=np.uint8)
