@@ -44,6 +44,7 @@ class Layer(ctypes.Structure):
         ("gate", ctypes.POINTER(ctypes.c_void_p)), ("up", ctypes.POINTER(ctypes.c_void_p)),
         ("down", ctypes.POINTER(ctypes.c_void_p)),
         ("sh_gate", ctypes.c_void_p), ("sh_up", ctypes.c_void_p), ("sh_down", ctypes.c_void_p),
+        ("expert_bits", ctypes.c_int32),
     ]
 
 
@@ -192,7 +193,9 @@ def moe_forward(layer: dict, x: np.ndarray, mode: int = 0):
     ``layer`` holds: H, I, E, k, W_r [E,H] f32, b_r [E] f32 or None, grid
     [256,8] u8, gate/up/down: sequences of E canonical block arrays (an entry
     may be None for an expert no token selects), sh_gate/sh_up/sh_down: bf16
-    bit patterns as uint16 arrays or None.
+    bit patterns as uint16 arrays or None; expert_bits (default 2): 2 for
+    IQ2_XXS-style gate/up and Q2_K-style down blocks, 4 for Q4_K-style blocks
+    in all three.
     mode 0: fp64 decode reading; mode 1: bf16 tensor-core reading.
     Returns (out [n,H] f64, ids [n,k] i32, w [n,k] f64).
     """
@@ -224,7 +227,7 @@ def moe_forward(layer: dict, x: np.ndarray, mode: int = 0):
               ctypes.cast(gate, ctypes.POINTER(ctypes.c_void_p)),
               ctypes.cast(up, ctypes.POINTER(ctypes.c_void_p)),
               ctypes.cast(down, ctypes.POINTER(ctypes.c_void_p)),
-              _p(sg), _p(su), _p(sd))
+              _p(sg), _p(su), _p(sd), int(layer.get("expert_bits", 2)))
     out = np.zeros((n, H), dtype=np.float64)
     ids = np.zeros((n, k), dtype=np.int32)
     w = np.zeros((n, k), dtype=np.float64)
@@ -288,7 +291,8 @@ def layer_from_torch(layer: dict, experts=None) -> dict:
 
     out = dict(H=layer["H"], I=layer["I"], E=E, k=layer["k"], W_r=layer["W_r"].cpu().numpy(),
                b_r=None if b is None else b.cpu().numpy(), grid=layer["grid"].cpu().numpy(),
-               gate=gate, up=up, down=down, sh_gate=None, sh_up=None, sh_down=None)
+               gate=gate, up=up, down=down, sh_gate=None, sh_up=None, sh_down=None,
+               expert_bits=int(layer.get("expert_bits", 2)))
     if layer.get("sh_gate") is not None:
         out.update(sh_gate=bits(layer["sh_gate"]), sh_up=bits(layer["sh_up"]), sh_down=bits(layer["sh_down"]))
     return out

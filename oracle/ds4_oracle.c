@@ -481,6 +481,8 @@ typedef struct {
     const uint16_t* sh_gate;        /* bf16 bits [I][H] or NULL: no shared expert */
     const uint16_t* sh_up;          /* bf16 bits [I][H] */
     const uint16_t* sh_down;        /* bf16 bits [H][I] */
+    int32_t expert_bits;            /* 2: gate/up IQ2_XXS-style, down Q2_K-style;
+                                       4: all three Q4_K-style (the 4-bit variant) */
 } orc_layer;
 
 static double bf16_bits_to_double(uint16_t v) {
@@ -531,6 +533,7 @@ int orc_moe_forward(const orc_layer* L, const float* x, int64_t n, int32_t mode,
     const int64_t H = L->H, I = L->I;
     const int32_t E = L->E, k = L->k;
     if (H % 256 || k < 1 || k > E || n < 0) return -1;
+    if (L->expert_bits != 2 && L->expert_bits != 4) return -1;
     if (n == 0) return 0;
     float* logits = (float*)malloc(sizeof(float) * (size_t)(n * E));
     int32_t* ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n * k));
@@ -554,9 +557,15 @@ int orc_moe_forward(const orc_layer* L, const float* x, int64_t n, int32_t mode,
         for (int64_t s = 0; s < n * k; ++s) used |= ids[s] == e;
         if (!used) continue;
         if (!L->gate[e] || !L->up[e] || !L->down[e]) { rc = -1; break; }
-        orc_dequant_iq2xxs(L->gate[e], I * H / ORC_QK, L->grid, Wg);
-        orc_dequant_iq2xxs(L->up[e], I * H / ORC_QK, L->grid, Wu);
-        orc_dequant_q2k(L->down[e], H * I / ORC_QK, Wd);
+        if (L->expert_bits == 4) {
+            orc_dequant_q4k(L->gate[e], I * H / ORC_QK, Wg);
+            orc_dequant_q4k(L->up[e], I * H / ORC_QK, Wu);
+            orc_dequant_q4k(L->down[e], H * I / ORC_QK, Wd);
+        } else {
+            orc_dequant_iq2xxs(L->gate[e], I * H / ORC_QK, L->grid, Wg);
+            orc_dequant_iq2xxs(L->up[e], I * H / ORC_QK, L->grid, Wu);
+            orc_dequant_q2k(L->down[e], H * I / ORC_QK, Wd);
+        }
         if (mode == 1)
             for (int64_t i = 0; i < I * H; ++i) {
                 Wg[i] = orc_bf16_round(Wg[i]);

@@ -442,6 +442,32 @@ def test_identical_experts_collapse_to_dense_ffn(orc):
     assert np.allclose(w.sum(1), 1.0, atol=1e-12)
 
 
+def test_identical_q4_experts_collapse_to_dense_ffn(orc):
+    """The 4-bit variant: every expert the same Q4_K-style blocks (gate, up and
+    down), so the layer is one dense SwiGLU FFN of those weights plus the shared
+    expert, evaluated with torch; different experts' blocks change the output."""
+    L = synth.float_layer(synth.Shape(H=256, I=128, E=8, k=2), 3)
+    blocks = {n: orc.pack_q4k(L[n + "_f"][0].numpy()) for n in ("gate", "up", "down")}
+    lay = dict(H=256, I=128, E=8, k=2, W_r=L["W_r"].numpy(), b_r=None, grid=L["grid"].numpy(),
+               gate=[blocks["gate"]] * 8, up=[blocks["up"]] * 8, down=[blocks["down"]] * 8, expert_bits=4)
+    for n in ("sh_gate", "sh_up", "sh_down"):
+        lay[n] = L[n].view(torch.int16).numpy().view(np.uint16)
+    x = synth.tokens(6, 256, seed=2).numpy()
+    out, ids, w = orc.moe_forward(lay, x)
+    Wg = orc.dequant_q4k(blocks["gate"]).reshape(128, 256)
+    Wu = orc.dequant_q4k(blocks["up"]).reshape(128, 256)
+    Wd = orc.dequant_q4k(blocks["down"]).reshape(256, 128)
+    ref = _dense_ffn(Wg, Wu, Wd, x) + _dense_ffn(_bf16_f64(L["sh_gate"]), _bf16_f64(L["sh_up"]),
+                                                 _bf16_f64(L["sh_down"]), x)
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    # other down blocks give another output (the 4-bit blocks are what is read);
+    # a bit width other than 2 or 4 is refused
+    lay2 = dict(lay, down=[orc.pack_q4k(L["down_f"][1].numpy())] * 8)
+    assert not np.allclose(orc.moe_forward(lay2, x)[0], out)
+    with pytest.raises(ValueError):
+        orc.moe_forward(dict(lay, expert_bits=3), x)
+
+
 def test_chain_of_dense_layers(orc):
     # two layers whose routed experts are identical: each layer is x + two dense
     # FFNs (routed weights sum to 1, plus the shared expert), computed with torch
