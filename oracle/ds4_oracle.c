@@ -18,6 +18,9 @@
  *   - the layer as the project states it: a full-precision router, softmax
  *     over the top-k experts, SwiGLU experts, gate-weighted sum plus an
  *     unquantized shared expert.
+ *   - the 4-bit models the same pages name (q4, q4-imatrix), whose format
+ *     they leave open: a Q4_K-style block of this project's own definition
+ *     (see orc_dequant_q4k).
  *
  * Precision: floating point is fp64 except where a floating-point value
  * decides an integer (the router logits that pick the experts), which is
