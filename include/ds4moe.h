@@ -142,10 +142,11 @@ ds4moe_status ds4moe_set_expert(ds4moe_t* h, int32_t e, const void* d_gate, cons
 ds4moe_status ds4moe_set_shared(ds4moe_t* h, const void* d_gate, const void* d_up, const void* d_down,
                                 void* stream);
 
-/* Directional steering of the layer output, as the pages' server applies it
- * after FFN outputs ("--dir-steering-ffn F": y -= F*v*dot(v,y), one f32
- * direction vector per layer): every later forward replaces the layer output
- * y (per token, before any residual add) by y - F v (v . y).  d_v: device
+/* Directional steering of the layer output, as the pages' server offers it
+ * after the FFN outputs with one binary32 direction vector per layer (the
+ * server's option list in the modu-print.com article on ds4.c): every later
+ * forward replaces the layer output y (per token, before any residual add) by
+ * y - F v (v . y).  d_v: device
  * pointer to H binary32 values, copied on `stream` (the caller may free it
  * afterwards); v . y is summed in a fixed order, so results repeat bitwise.
  * d_v == NULL or F == 0 turns steering off.  Requires hidden <= 4096

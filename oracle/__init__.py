@@ -240,9 +240,9 @@ def moe_forward(layer: dict, x: np.ndarray, mode: int = 0):
 def steer(y: np.ndarray, v: np.ndarray, F: float) -> np.ndarray:
     """Directional steering of a layer output, per token: y - F v (v . y), in fp64.
 
-    Follows the pages' server option that applies steering after FFN outputs
-    (ds4-server --help, "--dir-steering-ffn F": y -= F*v*dot(v,y), one f32
-    direction vector per layer).
+    Follows the pages' server option for steering after the FFN outputs, one
+    binary32 direction vector per layer (the server's option list in the
+    modu-print.com article on ds4.c).
     """
     y = np.asarray(y, dtype=np.float64)
     v = np.asarray(v, dtype=np.float32).astype(np.float64)
@@ -252,9 +252,10 @@ def steer(y: np.ndarray, v: np.ndarray, F: float) -> np.ndarray:
 def chain_forward(layers, x: np.ndarray, mode: int = 0):
     """A chain of layers with the residual step x_{l+1} = x_l + MoE_l(x_l).
 
-    Follows the multi-token-prediction verify of the pages (ds4-server --help
-    text: MTP draft tokens verified through the model's layers) as read for a
-    stack of MoE layers with no norm in between.  Each layer's input is binary32
+    Follows the pages' multi-token-prediction draft-and-verify (the server's
+    option list in the modu-print.com article on ds4.c; the MTP note in the
+    amuse.peoplentools.com summary) as read for a stack of MoE layers with no
+    norm in between.  Each layer's input is binary32
     (the decode plan's activation type): the fp64 sum is rounded to binary32
     before the next layer.  Returns (x_L as float32 [n,H], per-layer ids,
     per-layer inputs as float32).
