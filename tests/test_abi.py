@@ -49,3 +49,33 @@ def test_last_error_without_gpu(libpath):
     import bit_quantized_moe_softmax_b200 as m
 
     assert isinstance(m.ds4moe_last_error(), str)
+
+
+def _declarations():
+    """{name: parameter count} for every function the header declares."""
+    src = open(os.path.join(ROOT, "include", "ds4moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    out = {}
+    for name, params in re.findall(r"\b(ds4moe_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", src):
+        p = " ".join(params.split())
+        out[name] = 0 if p in ("", "void") else p.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_header(libpath):
+    """Every ctypes signature has as many arguments as the C declaration, and
+    the shape struct's fields come in the header's order."""
+    import bit_quantized_moe_softmax_b200 as m
+
+    decl = _declarations()
+    assert set(decl) == set(_declared())
+    L = m.lib()
+    for name, count in decl.items():
+        assert len(getattr(L, name).argtypes) == count, (name, count)
+    src = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "ds4moe.h")).read(), flags=re.S)
+    body = re.search(r"typedef struct\s*\{(.*?)\}\s*ds4moe_shape\s*;", src, flags=re.S).group(1)
+    fields = re.findall(r"\b(\w+)\s*;", body)
+    assert fields == [f for f, _ in m.ds4moe_shape._fields_]
+    assert all(t is ctypes.c_int32 for _, t in m.ds4moe_shape._fields_)
+    assert "int32_t" in body and not re.search(r"\b(int64_t|size_t|float|double)\b", body)
