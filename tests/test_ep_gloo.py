@@ -1,5 +1,5 @@
-"""Expert parallelism's exchange steps on CPU: two gloo ranks, experts split
-between them (dispatch to the experts' owners, the owners' experts, combine
+"""Expert parallelism's exchange steps on CPU: two and three gloo ranks, experts
+split between them (dispatch to the experts' owners, the owners' experts, combine
 back in slot order).
 
 * plumbing: a stand-in expert (row times expert id + 1) makes every value
@@ -16,6 +16,7 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch
 import torch.multiprocessing as mp
 
@@ -102,7 +103,8 @@ def _worker(rank, world, port, q):
                       WORLD_SIZE=str(world))
     try:
         r, _, w = D.init("gloo", timeout_s=60)
-        res = {"plumbing": _plumbing(r, w, [5, 3]), "empty": _plumbing(r, w, [4, 0]), "layer": _layer(r, w)}
+        res = {"plumbing": _plumbing(r, w, [5, 3, 6][:w]), "empty": _plumbing(r, w, [4, 0, 2][:w]),
+               "layer": _layer(r, w)}
         D.barrier()
         q.put((r, res))
         D.finish()
@@ -112,21 +114,23 @@ def _worker(rank, world, port, q):
         q.put(("error", traceback.format_exc() + repr(e)))
 
 
-def test_expert_parallel_two_ranks_gloo():
+@pytest.mark.parametrize("world", [2, 3])
+def test_expert_parallel_gloo(world):
+    """Two ranks (4 experts each) and three (3, 3 and 2 experts: uneven splits)."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
-    got = [q.get(timeout=300) for _ in range(2)]
+    got = [q.get(timeout=300) for _ in range(world)]
     for p in procs:
         p.join(timeout=60)
     assert all(g[0] != "error" for g in got), got
     for r, res in got:
         assert res["plumbing"][:2] == (True, True), (r, res)
         assert res["empty"][:2] == (True, True), (r, res)
-        assert res["empty"][2][0] == (4 if r == 0 else 0)
+        assert res["empty"][2][0] == [4, 0, 2][r]
         ids_ok, rel = res["layer"]
         assert ids_ok and rel < 1e-12, (r, rel)
 
