@@ -616,3 +616,52 @@ def test_bf16_reading_exact_when_representable(orc):
     bound = 2.0 ** -8 * (np.abs(h) @ np.abs(Wdm).T) * 1.001
     assert np.all(np.abs(out1 - out0) <= bound + 1e-30)
     assert np.abs(out1 - out0).max() > 0
+
+
+def _bf16_reading_dense(Wg, Wu, Wd, x, round_w=True, round_x=True, round_h=True):
+    """The bf16 tensor-core reading written with torch library routines: the
+    dequantized weights, x and h rounded to bfloat16 by torch (h first to
+    binary32, as a kernel holding it in an fp32 register would), sums in fp64."""
+    def r(a, on):
+        t = torch.from_numpy(np.asarray(a, np.float32))
+        return (t.to(torch.bfloat16) if on else t).to(torch.float64)
+
+    X = r(x, round_x)
+    g = X @ r(Wg, round_w).T
+    u = X @ r(Wu, round_w).T
+    h = torch.nn.functional.silu(g) * u
+    if round_h:
+        h = h.to(torch.float32).to(torch.bfloat16).to(torch.float64)
+    return (h @ r(Wd, round_w).T).numpy()
+
+
+def test_bf16_reading_matches_torch_bf16_dense(orc):
+    """Pin of the oracle's bf16 reading (mode 1, the prefill plan's rounding
+    points: x, the dequantized routed weights and h rounded to bfloat16, sums in
+    fp64) on weights and activations that bf16 does NOT represent exactly:
+    one routed expert (E = k = 1, weight 1), no shared expert, against torch's
+    bfloat16 conversion and fp64 matmuls.  Dropping any one of the three
+    roundings moves the result far outside the 1e-12 tolerance, so a reading
+    that forgot one of them fails here."""
+    L = synth.float_layer(synth.Shape(H=256, I=128, E=1, k=1), 21)
+    grid = L["grid"].numpy()
+    gate = orc.pack_iq2xxs(L["gate_f"][0].numpy(), grid)
+    up = orc.pack_iq2xxs(L["up_f"][0].numpy(), grid)
+    down = orc.pack_q2k(L["down_f"][0].numpy())
+    lay = dict(H=256, I=128, E=1, k=1, W_r=L["W_r"].numpy(), b_r=None, grid=grid, gate=[gate], up=[up],
+               down=[down], sh_gate=None, sh_up=None, sh_down=None)
+    Wg = orc.dequant_iq2xxs(gate, grid).reshape(128, 256)
+    Wu = orc.dequant_iq2xxs(up, grid).reshape(128, 256)
+    Wd = orc.dequant_q2k(down).reshape(256, 128)
+    x = synth.tokens(3, 256, seed=22).numpy()          # binary32, not bf16-exact
+    # the inputs really need rounding: most weights and x values are not bf16 numbers
+    for a in (Wg, Wu, Wd, x):
+        assert np.mean(orc.bf16_round(a) != a) > 0.5
+    out, ids, w = orc.moe_forward(lay, x, mode=1)
+    assert np.all(ids == 0) and np.all(w == 1.0)
+    ref = _bf16_reading_dense(Wg, Wu, Wd, x)
+    scale = np.abs(ref).max()
+    assert np.abs(out - ref).max() <= 1e-12 * scale
+    for miss in (dict(round_w=False), dict(round_x=False), dict(round_h=False)):
+        alt = _bf16_reading_dense(Wg, Wu, Wd, x, **miss)
+        assert np.abs(alt - out).max() > 1e-6 * scale, miss
