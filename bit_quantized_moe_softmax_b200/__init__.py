@@ -132,9 +132,10 @@ def ds4moe_workspace_bytes(h: int, n_tokens: int) -> int:
     return lib().ds4moe_workspace_bytes(h, n_tokens)
 
 
-def ds4moe_bind(h: int, weights: torch.Tensor, workspace: torch.Tensor, stream=None):
-    _ok(lib().ds4moe_bind(h, _ptr(weights), weights.numel() * weights.element_size(), _ptr(workspace),
-                          workspace.numel() * workspace.element_size(), _stream(stream)), "ds4moe_bind")
+def ds4moe_bind(h: int, weights: torch.Tensor, workspace: torch.Tensor | None, stream=None):
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _ok(lib().ds4moe_bind(h, _ptr(weights), weights.numel() * weights.element_size(), _ptr(workspace), wsb,
+                          _stream(stream)), "ds4moe_bind")
 
 
 def ds4moe_pack_q2k(w: torch.Tensor, blocks: torch.Tensor, stream=None):
@@ -219,10 +220,11 @@ def ds4moe_route(h: int, x: torch.Tensor, ids: torch.Tensor, w: torch.Tensor, st
 def ds4moe_route_noalloc(h: int, x: torch.Tensor, ids: torch.Tensor, w: torch.Tensor, stream=None):
     """Routing with the library's static device scratch instead of the bound workspace.
 
-    For callers that cannot allocate device memory (for example while a CUDA
-    graph is being captured, or inside a host that owns all device buffers);
-    see include/ds4moe.h for the limit (n_tokens * n_experts <= 8192) and the
-    rule that overlapping calls race on the shared scratch.
+    For callers that cannot allocate device memory (a host that owns every
+    device buffer through its own pool, or code that must not stall the device
+    with a synchronizing allocation); the handle needs only its weight buffer
+    bound.  Limit: n_tokens * n_experts <= 8192; calls that overlap on the GPU
+    race on the shared scratch.
     """
     _ok(lib().ds4moe_route_noalloc(h, _ptr(x), x.shape[0], _ptr(ids), _ptr(w), _stream(stream)),
         "ds4moe_route_noalloc")

@@ -42,13 +42,20 @@ size_t gemm_static_smem_bytes();
 
 using namespace ds4;
 
-// Scratch of ds4moe_route_noalloc: a 64-word header (the router's ticket and
-// task counters; cleared before every call) followed by the logits of up to
-// kNoAllocLogits (token, expert) pairs.  One copy per device, for the life of
-// the process; its device address is looked up once per device.
+// Scratch of ds4moe_route_noalloc: a 64-word header (word 0: the device error
+// word, kept until ds4moe_get_device_error reads it; words 1.. : the router's
+// ticket and task counters, cleared before every call) followed by the logits
+// of up to kNoAllocLogits (token, expert) pairs.  kNoAllocLogits = 8192 is the
+// largest n_tokens * n_experts a handle can ask for (decode_max <= 8 tokens,
+// n_experts <= 1024), so the size check in the entry point is a defensive one.
+// One copy per device, for the life of the process; its device address is
+// looked up once per device (noalloc_scratch) and kept in g_noalloc_addr.
 constexpr int kNoAllocHeader = 64;
 constexpr int kNoAllocLogits = 8192;
+constexpr int kNoAllocDevices = 64;
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocHeader + kNoAllocLogits];
+static std::mutex g_noalloc_mu;
+static float* g_noalloc_addr[kNoAllocDevices] = {};
 
 namespace {
 
@@ -244,7 +251,8 @@ struct ds4moe {
     }
 
     bool ready(std::string* why) const {
-        if (!weights || !ws) { *why = "buffers not bound"; return false; }
+        if (!weights) { *why = "buffers not bound"; return false; }
+        if (!ws) { *why = "workspace not bound"; return false; }
         if (!grid_set) { *why = "grid not set"; return false; }
         if (!router_set) { *why = "router not set"; return false; }
         if (shape.has_shared && !shared_set) { *why = "shared expert not set"; return false; }
@@ -346,20 +354,24 @@ size_t ds4moe_workspace_bytes(const ds4moe_t* h, int32_t n_tokens) {
 
 ds4moe_status ds4moe_bind(ds4moe_t* h, void* d_weights, size_t weight_bytes, void* d_workspace, size_t ws_bytes,
                           void* stream) {
-    if (!h || !d_weights || !d_workspace) return fail(DS4MOE_ERR_ARG, "bind: NULL argument");
+    if (!h || !d_weights) return fail(DS4MOE_ERR_ARG, "bind: NULL argument");
+    if (!d_workspace && ws_bytes != 0) return fail(DS4MOE_ERR_ARG, "bind: NULL workspace with a nonzero size");
     if (((uintptr_t)d_weights & 255) || ((uintptr_t)d_workspace & 255))
         return fail(DS4MOE_ERR_ALIGN, "bind: buffers must be 256-byte aligned");
     if (weight_bytes < h->weight_bytes)
         return fail(DS4MOE_ERR_ARG, "bind: weight buffer %zu bytes < %zu", weight_bytes, h->weight_bytes);
     WsLayout L = h->layout(h->shape.max_tokens);
-    if (ws_bytes < L.total) return fail(DS4MOE_ERR_ARG, "bind: workspace %zu bytes < %zu", ws_bytes, L.total);
+    if (d_workspace && ws_bytes < L.total)
+        return fail(DS4MOE_ERR_ARG, "bind: workspace %zu bytes < %zu", ws_bytes, L.total);
     // pipelined host-buffer calls still in flight use the old staging slots
     ds4moe_status hs = ds4moe_host_sync(h);
     if (hs != DS4MOE_OK) return hs;
     h->slot = 0;
-    cudaError_t ce = cudaMemsetAsync(static_cast<uint8_t*>(d_workspace) + L.hdr, 0, L.logits - L.hdr,
-                                     (cudaStream_t)stream);
-    if (ce != cudaSuccess) return cuda_fail(ce, "bind: cudaMemsetAsync");
+    if (d_workspace) {
+        cudaError_t ce = cudaMemsetAsync(static_cast<uint8_t*>(d_workspace) + L.hdr, 0, L.logits - L.hdr,
+                                         (cudaStream_t)stream);
+        if (ce != cudaSuccess) return cuda_fail(ce, "bind: cudaMemsetAsync");
+    }
     h->weights = static_cast<uint8_t*>(d_weights);
     h->ws = static_cast<uint8_t*>(d_workspace);
     h->ws_bytes = ws_bytes;
@@ -670,14 +682,32 @@ ds4moe_status ds4moe_dequant(ds4moe_t* h, int32_t e, int32_t which, int32_t as_b
     return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "dequant launch");
 }
 
+// Device address of the no-allocation scratch on the current device: looked
+// up (cudaGetSymbolAddress, with this device current) on the first call per
+// device, then cached.  nullptr with *err set on failure.
+static float* noalloc_scratch(int dev, cudaError_t* err, bool lookup) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev] && lookup) {
+        void* p = nullptr;
+        *err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (*err != cudaSuccess) return nullptr;
+        g_noalloc_addr[dev] = static_cast<float*>(p);
+    }
+    return g_noalloc_addr[dev];
+}
+
 ds4moe_status ds4moe_route_noalloc(ds4moe_t* h, const void* d_x, int32_t n, int32_t* d_ids, float* d_w,
                                    void* stream) {
-    static std::mutex mu;
-    static float* scratch_of_device[64] = {};
-    ds4moe_status s = check_forward(h, d_x, n, d_ids, "route_noalloc");
-    if (s != DS4MOE_OK) return s;
+    // Needs the router and its inputs only: the bound workspace is not used,
+    // so a handle bound to a weight buffer (and any workspace) with grid and
+    // router loaded is enough.
+    if (!h) return fail(DS4MOE_ERR_ARG, "route_noalloc: NULL handle");
+    if (n < 0 || n > h->shape.max_tokens)
+        return fail(DS4MOE_ERR_ARG, "route_noalloc: n_tokens %d outside 0..%d", n, h->shape.max_tokens);
     if (n == 0) return DS4MOE_OK;
-    if (!d_w) return fail(DS4MOE_ERR_ARG, "route_noalloc: NULL weights");
+    if (!d_x || !d_ids || !d_w) return fail(DS4MOE_ERR_ARG, "route_noalloc: NULL buffer");
+    if (!h->weights) return fail(DS4MOE_ERR_NOT_READY, "route_noalloc: buffers not bound");
+    if (!h->grid_set || !h->router_set) return fail(DS4MOE_ERR_NOT_READY, "route_noalloc: router not loaded");
     if (!aligned16(d_x)) return fail(DS4MOE_ERR_ALIGN, "route_noalloc: x must be 16-byte aligned");
     if (n > h->decode_max) return fail(DS4MOE_ERR_ARG, "route_noalloc: n_tokens %d > decode_max %d", n, h->decode_max);
     if ((int64_t)n * h->D.E > kNoAllocLogits)
@@ -686,22 +716,15 @@ ds4moe_status ds4moe_route_noalloc(ds4moe_t* h, const void* d_x, int32_t n, int3
     int dev = 0;
     cudaError_t ce = cudaGetDevice(&dev);
     if (ce != cudaSuccess) return cuda_fail(ce, "route_noalloc: cudaGetDevice");
-    if (dev < 0 || dev >= 64) return fail(DS4MOE_ERR_ARG, "route_noalloc: device %d beyond 64", dev);
-    float* base = nullptr;
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        if (!scratch_of_device[dev]) {
-            void* p = nullptr;
-            ce = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-            if (ce != cudaSuccess) return cuda_fail(ce, "route_noalloc: cudaGetSymbolAddress");
-            scratch_of_device[dev] = static_cast<float*>(p);
-        }
-        base = scratch_of_device[dev];
-    }
+    if (dev < 0 || dev >= kNoAllocDevices)
+        return fail(DS4MOE_ERR_ARG, "route_noalloc: device %d beyond %d", dev, kNoAllocDevices);
+    float* base = noalloc_scratch(dev, &ce, true);
+    if (!base) return cuda_fail(ce, "route_noalloc: cudaGetSymbolAddress");
     cudaStream_t st = (cudaStream_t)stream;
-    // the counters must start at zero; the previous call's contents are stale
-    ce = cudaMemsetAsync(base, 0, kNoAllocHeader * sizeof(float), st);
-    if (ce != cudaSuccess) return cuda_fail(ce, "route_noalloc: clear header");
+    // the counters must start at zero (the previous call's are stale); the
+    // error word (word 0) stays until ds4moe_get_device_error reads it
+    ce = cudaMemsetAsync(base + 1, 0, (kNoAllocHeader - 1) * sizeof(float), st);
+    if (ce != cudaSuccess) return cuda_fail(ce, "route_noalloc: clear counters");
     uint32_t* hdr = reinterpret_cast<uint32_t*>(base);
     DecodeWs ws{};
     ws.err = hdr + 0;
@@ -717,13 +740,22 @@ ds4moe_status ds4moe_route_noalloc(ds4moe_t* h, const void* d_x, int32_t n, int3
 
 ds4moe_status ds4moe_get_device_error(ds4moe_t* h, void* stream, int32_t* code) {
     if (!h || !code) return fail(DS4MOE_ERR_ARG, "get_device_error: NULL argument");
-    if (!h->ws) return fail(DS4MOE_ERR_NOT_READY, "get_device_error: buffers not bound");
+    int dev = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce != cudaSuccess) return cuda_fail(ce, "get_device_error: cudaGetDevice");
+    // the no-allocation routing's error word on this device, if that entry point has run here
+    uint32_t* na = nullptr;
+    if (dev >= 0 && dev < kNoAllocDevices) na = reinterpret_cast<uint32_t*>(noalloc_scratch(dev, &ce, false));
+    if (!h->ws && !na) return fail(DS4MOE_ERR_NOT_READY, "get_device_error: buffers not bound");
     cudaStream_t st = (cudaStream_t)stream;
-    uint32_t v = 0;
-    cudaError_t ce = cudaStreamSynchronize(st);
-    if (ce == cudaSuccess) ce = cudaMemcpy(&v, h->ws + h->L.hdr, 4, cudaMemcpyDeviceToHost);
+    uint32_t v = 0, w = 0;
+    ce = cudaStreamSynchronize(st);
+    if (ce == cudaSuccess && h->ws) ce = cudaMemcpy(&v, h->ws + h->L.hdr, 4, cudaMemcpyDeviceToHost);
     if (ce == cudaSuccess && v) ce = cudaMemset(h->ws + h->L.hdr, 0, 4);
+    if (ce == cudaSuccess && na) ce = cudaMemcpy(&w, na, 4, cudaMemcpyDeviceToHost);
+    if (ce == cudaSuccess && w) ce = cudaMemset(na, 0, 4);
     if (ce != cudaSuccess) return cuda_fail(ce, "get_device_error");
+    v |= w;
     *code = (int32_t)v;
     if (v & kErrTimeout) return fail(DS4MOE_ERR_TIMEOUT, "a bounded device wait timed out (code %u)", v);
     if (v) return fail(DS4MOE_ERR_DEVICE, "device-side check failed (code %u)", v);

@@ -96,7 +96,10 @@ size_t ds4moe_workspace_bytes(const ds4moe_t* h, int32_t n_tokens);
 /* Bind caller-owned device buffers: d_weights (>= ds4moe_weight_bytes) and
  * d_workspace (>= ds4moe_workspace_bytes(h, max_tokens)), both 256-byte
  * aligned.  Clears the workspace's counters and error word on `stream`.
- * Rebinding marks every expert as not loaded. */
+ * d_workspace may be NULL (with workspace_bytes 0): the weights are bound
+ * alone, every call that needs the workspace returns DS4MOE_ERR_NOT_READY,
+ * and ds4moe_route_noalloc still works.  Rebinding marks every expert as not
+ * loaded. */
 ds4moe_status ds4moe_bind(ds4moe_t* h, void* d_weights, size_t weight_bytes, void* d_workspace,
                           size_t workspace_bytes, void* stream);
 
@@ -236,28 +239,36 @@ ds4moe_status ds4moe_dequant(ds4moe_t* h, int32_t e, int32_t which, int32_t as_b
 
 /* ---- routing without device allocation ------------------------------------ */
 
-/* ds4moe_route for callers that cannot allocate device memory: code that runs
- * while a CUDA graph is being captured (allocation is not allowed there and a
- * synchronizing allocator would break the capture), and hosts that own every
- * device buffer and hand this library only its inputs and outputs.  The
- * pages have no counterpart; this is an interface convenience.
+/* ds4moe_route for callers that cannot allocate device memory: hosts that own
+ * every device buffer through their own pool (a serving process, an embedded
+ * runtime) and hand this library only its inputs and outputs, and code that
+ * must not call the allocator because cudaMalloc synchronizes the device and
+ * would stall the work in flight.  The pages have no counterpart; this is an
+ * interface convenience.
  * The router's scratch (logits of up to 8192 token-expert pairs, i.e.
- * n_tokens * n_experts <= 8192, and a 256-byte counter header) lives in one
- * static device array inside the library, which every GPU that loads the
- * library holds until the process exits; the bound workspace is not used.
+ * n_tokens * n_experts <= 8192, and a 256-byte header of counters and an
+ * error word) lives in one static device array inside the library, which
+ * every GPU that loads the library holds until the process exits; the bound
+ * workspace is not used, and the handle needs only its weight buffer bound
+ * (ds4moe_bind accepts a NULL workspace) with the grid and the router loaded.
  * The caller passes x and the outputs ids[n][k] (int32) and weights[n][k]
  * (binary32), with the same results as ds4moe_route.  Larger n_tokens *
  * n_experts, or n_tokens > decode_max, is rejected with DS4MOE_ERR_ARG.
- * The first call on a device looks up the array's device address (make that
- * first call before any stream capture).  Every call shares the one array:
- * calls that overlap on the GPU (other streams, other threads) race, so
- * serialize them. */
+ * The first call on a device looks up the array's device address with that
+ * device current (make that first call before any stream capture).  Every
+ * call clears the array's counters and shares the one array: calls that
+ * overlap on the GPU (other streams, other threads) race, so serialize them.
+ * Device-side failures set the array's error word, which
+ * ds4moe_get_device_error reads and clears. */
 ds4moe_status ds4moe_route_noalloc(ds4moe_t* h, const void* d_x, int32_t n_tokens, int32_t* d_ids,
                                    float* d_weights, void* stream);
 
 /* Synchronize `stream`, then read and clear the workspace's device error word
- * into *code (0 = none; bit 0 = an index check failed, bit 1 = a bounded
- * wait timed out, bit 2 = the grid has more than four distinct magnitudes).  Returns DS4MOE_ERR_DEVICE / DS4MOE_ERR_TIMEOUT when set. */
+ * (and, when ds4moe_route_noalloc has run on the current device, the error
+ * word of its static scratch) into *code (0 = none; bit 0 = an index check
+ * failed, bit 1 = a bounded wait timed out, bit 2 = the grid has more than
+ * four distinct magnitudes).  Returns DS4MOE_ERR_DEVICE / DS4MOE_ERR_TIMEOUT
+ * when set; DS4MOE_ERR_NOT_READY when neither word exists. */
 ds4moe_status ds4moe_get_device_error(ds4moe_t* h, void* stream, int32_t* code);
 
 /* Message of the last error on the calling thread ("" if none). */
