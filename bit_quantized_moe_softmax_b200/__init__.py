@@ -33,7 +33,7 @@ EXPORTS = ("ds4moe_create", "ds4moe_destroy", "ds4moe_weight_bytes", "ds4moe_wor
            "ds4moe_get_device_error", "ds4moe_last_error", "ds4moe_plan_launches", "ds4moe_plan_kernel",
            "ds4moe_forward_profiled", "ds4moe_route_noalloc", "ds4moe_forward_residual",
            "ds4moe_forward_residual_profiled", "ds4moe_set_steering", "ds4moe_forward_host_async",
-           "ds4moe_host_sync")
+           "ds4moe_host_sync", "ds4moe_probe", "ds4moe_selftest_wait")
 
 
 class ds4moe_shape(ctypes.Structure):
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
             "ds4moe_host_sync": ([vp], i32),
             "ds4moe_route": ([vp, vp, i32, vp, vp, vp], i32),
             "ds4moe_dequant": ([vp, i32, i32, i32, vp, vp], i32),
+            "ds4moe_probe": ([vp, i32, i32, i32, vp, i32, vp, vp], i32),
+            "ds4moe_selftest_wait": ([vp, vp], i32),
             "ds4moe_get_device_error": ([vp, vp, ctypes.POINTER(i32)], i32),
             "ds4moe_last_error": ([], ctypes.c_char_p),
             "ds4moe_plan_launches": ([vp, i32], i32),
@@ -230,8 +232,18 @@ def ds4moe_route_noalloc(h: int, x: torch.Tensor, ids: torch.Tensor, w: torch.Te
         "ds4moe_route_noalloc")
 
 
+def ds4moe_probe(h: int, plan: int, which: int, e: int, inp: torch.Tensor, out: torch.Tensor, stream=None):
+    """Raw accumulators of one plan's projection kernels on caller rows, all routed to expert e (-1: shared)."""
+    _ok(lib().ds4moe_probe(h, plan, which, e, _ptr(inp), inp.shape[0], _ptr(out), _stream(stream)), "ds4moe_probe")
+
+
 def ds4moe_dequant(h: int, e: int, which: int, as_bf16: int, out: torch.Tensor, stream=None):
     _ok(lib().ds4moe_dequant(h, e, which, as_bf16, _ptr(out), _stream(stream)), "ds4moe_dequant")
+
+
+def ds4moe_selftest_wait(h: int, stream=None):
+    """A bounded wait on an mbarrier nothing arrives at: gives up after its limit and sets error bit 1."""
+    _ok(lib().ds4moe_selftest_wait(h, _stream(stream)), "ds4moe_selftest_wait")
 
 
 def ds4moe_get_device_error(h: int, stream=None) -> int:

@@ -871,6 +871,25 @@ __global__ void __launch_bounds__(kSteerThreads) k_combine_steer_decode(Dims D, 
     }
 }
 
+// ---------------------------------------------------------------- failure-path check
+// One warp waits, with the kernels' bounded wait routine, on an mbarrier that
+// no thread ever arrives at: the wait gives up after kWaitNs, records
+// kErrTimeout in the error word and the kernel returns.
+__global__ void k_wait_selftest(uint32_t* err) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    mbar_wait(&bar, 0, err);
+}
+
+cudaError_t launch_wait_selftest(uint32_t* err, cudaStream_t st) {
+    k_wait_selftest<<<1, 32, 0, st>>>(err);
+    return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- launchers
 template <int NT>
 size_t gateup_smem_bytes(const Dims& D, int n) {

@@ -34,6 +34,9 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
                            int n_sm, cudaStream_t st, cudaEvent_t const* ev);
 cudaError_t launch_route_prefill(const Weights& W, const Dims& D, const PrefillWs& ws, const void* x, int n,
                                  cudaStream_t st);
+cudaError_t launch_wait_selftest(uint32_t* err, cudaStream_t st);
+cudaError_t launch_probe_gemm(const Weights& W, const Dims& D, const PrefillWs& ws, int which, int e,
+                              const void* in, int n, float* out, int n_sm, cudaStream_t st);
 int prefill_launches(const Dims& D);
 const char* prefill_kernel_name(const Dims& D, int i);
 size_t gemm_smem_bytes();
@@ -247,6 +250,7 @@ struct ds4moe {
         w.Y = reinterpret_cast<float*>(ws + L.p_Y);
         w.Ys = reinterpret_cast<float*>(ws + L.p_Ys);
         w.err = reinterpret_cast<uint32_t*>(ws + L.hdr);
+        w.grid_refused = reinterpret_cast<uint32_t*>(ws + L.hdr) + 6;
         return w;
     }
 
@@ -644,6 +648,25 @@ ds4moe_status ds4moe_route(ds4moe_t* h, const void* d_x, int32_t n, int32_t* d_i
     return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "route");
 }
 
+ds4moe_status ds4moe_probe(ds4moe_t* h, int32_t plan, int32_t which, int32_t e, const void* d_in, int32_t n,
+                           float* d_out, void* stream) {
+    if (!h) return fail(DS4MOE_ERR_ARG, "probe: NULL handle");
+    if (plan != 1) return fail(DS4MOE_ERR_ARG, "probe: plan %d (1 = prefill)", plan);
+    if (which != 0 && which != 2) return fail(DS4MOE_ERR_ARG, "probe: which %d (0 gate/up, 2 down)", which);
+    if (n < 1 || n > (1 << 20)) return fail(DS4MOE_ERR_ARG, "probe: n_rows %d outside 1..2^20", n);
+    if (!d_in || !d_out) return fail(DS4MOE_ERR_ARG, "probe: NULL buffer");
+    if (!aligned16(d_in) || !aligned16(d_out)) return fail(DS4MOE_ERR_ALIGN, "probe: buffers must be 16-byte aligned");
+    std::string why;
+    if (!h->ready(&why)) return fail(DS4MOE_ERR_NOT_READY, "probe: %s", why.c_str());
+    if (e < -1 || e >= h->D.E) return fail(DS4MOE_ERR_ARG, "probe: expert %d out of range", e);
+    if (e == -1 && !h->shape.has_shared) return fail(DS4MOE_ERR_ARG, "probe: the layer has no shared expert");
+    if (h->shape.max_tokens <= h->decode_max)
+        return fail(DS4MOE_ERR_NOT_READY, "probe: the prefill plan needs max_tokens > decode_max");
+    cudaError_t ce = launch_probe_gemm(h->weights_view(), h->D, h->prefill_ws(), which, e, d_in, n, d_out, h->n_sm,
+                                       (cudaStream_t)stream);
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "probe launch");
+}
+
 ds4moe_status ds4moe_dequant(ds4moe_t* h, int32_t e, int32_t which, int32_t as_bf16, void* d_out, void* stream) {
     if (!h || !d_out) return fail(DS4MOE_ERR_ARG, "dequant: NULL argument");
     if (!h->weights) return fail(DS4MOE_ERR_NOT_READY, "dequant: buffers not bound");
@@ -736,6 +759,13 @@ ds4moe_status ds4moe_route_noalloc(ds4moe_t* h, const void* d_x, int32_t n, int3
     ws.wts = d_w;
     ce = launch_route(h->weights_view(), h->D, ws, d_x, n, st);
     return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "route_noalloc launch");
+}
+
+ds4moe_status ds4moe_selftest_wait(ds4moe_t* h, void* stream) {
+    if (!h) return fail(DS4MOE_ERR_ARG, "selftest_wait: NULL handle");
+    if (!h->ws) return fail(DS4MOE_ERR_NOT_READY, "selftest_wait: workspace not bound");
+    cudaError_t ce = launch_wait_selftest(reinterpret_cast<uint32_t*>(h->ws + h->L.hdr), (cudaStream_t)stream);
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "selftest_wait launch");
 }
 
 ds4moe_status ds4moe_get_device_error(ds4moe_t* h, void* stream, int32_t* code) {

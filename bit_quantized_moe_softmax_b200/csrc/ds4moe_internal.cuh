@@ -98,6 +98,7 @@ struct PrefillWs {
     float* Y;               // [n k][H] routed outputs (unweighted)
     float* Ys;              // [n][H] shared output
     uint32_t* err;
+    uint32_t* grid_refused; // this call's routed GEMMs refused the grid (more than four magnitudes): 1, else 0
     const void* xres;       // x again when the call adds the residual (out = x + layer(x)), else nullptr
     const float* steer_v;   // [H] steering direction, or nullptr (no steering)
     float steer_F;          // steering strength: y -= F v (v . y)

@@ -322,6 +322,9 @@ struct GemmArgs {
     int n_rows;                 // shared modes: tokens
     __nv_bfloat16* out_h;       // gate/up modes: [rows][I] bf16
     float* out_y;               // down modes: [rows][H] binary32
+    float* out_raw;             // gate/up modes, inspection only: when set, the binary32
+                                // accumulators [rows][2I] (gate columns, then up) instead of h
+    uint32_t* grid_refused;     // routed gate/up mode: set to 1 (grid has more than four magnitudes) or 0
     uint32_t* err;
 };
 
@@ -480,6 +483,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 set_err(a.err, kErrGrid);
                 S.abort = 1;
             }
+            if (blockIdx.x == 0 && a.grid_refused) *a.grid_refused = nv > 4 ? 1u : 0u;
         }
         __syncthreads();
         for (int row = tid; row < 256; row += kGThreads) {
@@ -719,7 +723,23 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const bool live = m < ti.mvalid;
             {
                 // 16-column TMEM reads; each thread stores 32-byte pieces of its own row
-                if (kGateUp) {
+                if (kGateUp && a.out_raw) {
+                    // inspection: the accumulators as they are (no SwiGLU)
+                    float* dg = a.out_raw + (size_t)(ti.row0 + m) * 2 * I + 128 * ti.nb;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < 128; c0 += 16) {
+                        uint32_t g[16], u[16];
+                        tmem_ld_32x16(taddr + c0, g);
+                        tmem_ld_32x16(taddr + 128 + c0, u);
+                        tmem_wait_ld();
+                        if (live) {
+                            st_global_v8(dg + c0, g[0], g[1], g[2], g[3], g[4], g[5], g[6], g[7]);
+                            st_global_v8(dg + c0 + 8, g[8], g[9], g[10], g[11], g[12], g[13], g[14], g[15]);
+                            st_global_v8(dg + I + c0, u[0], u[1], u[2], u[3], u[4], u[5], u[6], u[7]);
+                            st_global_v8(dg + I + c0 + 8, u[8], u[9], u[10], u[11], u[12], u[13], u[14], u[15]);
+                        }
+                    }
+                } else if (kGateUp) {
                     __nv_bfloat16* dst = a.out_h + (size_t)(ti.row0 + m) * I + 128 * ti.nb;
 #pragma unroll 1
                     for (int c0 = 0; c0 < 128; c0 += 16) {
@@ -765,10 +785,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
 
 // ---------------------------------------------------------------- combine
 __global__ void k_combine_prefill(Dims D, const float* ys, const float* y, const float* wts, const int32_t* pos_of_slot,
-                                  int n, const void* xres, float* out) {
+                                  int n, const void* xres, const uint32_t* grid_refused, float* out) {
     const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // float4 index
     const int H = D.H, k = D.k;
     if (g >= (int64_t)n * H / 4) return;
+    if (__ldcg(grid_refused)) return;   // this call's routed GEMMs refused the grid: out stays as it was
     const int t = (int)(g / (H / 4)), r4 = (int)(g % (H / 4));
     float4 acc = D.has_shared ? __ldg(reinterpret_cast<const float4*>(ys + (int64_t)t * H) + r4)
                               : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -797,8 +818,9 @@ constexpr int kSteerThreadsP = 256;
 __global__ void __launch_bounds__(kSteerThreadsP) k_combine_steer_prefill(Dims D, const float* ys, const float* y,
                                                                           const float* wts, const int32_t* pos_of_slot,
                                                                           const float* v, float F, const void* xres,
-                                                                          float* out) {
+                                                                          const uint32_t* grid_refused, float* out) {
     __shared__ float red[kSteerThreadsP / 32];
+    if (__ldcg(grid_refused)) return;   // this call's routed GEMMs refused the grid: out stays as it was
     __shared__ int s_pos[16];
     __shared__ float s_w[16];
     const int t = blockIdx.x, H = D.H, k = D.k;
@@ -991,6 +1013,7 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
     ga.offs = ws.offs;
     ga.mt_prefix = ws.mt_prefix;
     ga.err = ws.err;
+    ga.grid_refused = ws.grid_refused;
     CUtensorMap mA;
     // routed gate/up: A = Xp [n k][H] -> Hb [n k][I]
     if ((e = encode_tmap(&mA, ws.Xp, nslots, H)) != cudaSuccess) return e;
@@ -1025,12 +1048,61 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
     mk.before();
     if (ws.steer_v)
         k_combine_steer_prefill<<<(unsigned)n, kSteerThreadsP, 0, st>>>(D, ws.Ys, ws.Y, ws.wts, ws.pos_of_slot,
-                                                                      ws.steer_v, ws.steer_F, ws.xres, out);
+                                                                      ws.steer_v, ws.steer_F, ws.xres, ws.grid_refused, out);
     else
         k_combine_prefill<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(D, ws.Ys, ws.Y, ws.wts, ws.pos_of_slot, n,
-                                                                        ws.xres, out);
+                                                                        ws.xres, ws.grid_refused, out);
     mk.after();
     return cudaGetLastError();
+}
+
+// Plan of an inspection call: all n rows go to expert e (counts, offsets and
+// tile prefix of the grouped GEMM).
+__global__ void k_probe_plan(int E, int e, int n, int32_t* counts, int32_t* offs, int32_t* mt_prefix) {
+    for (int q = threadIdx.x; q <= E; q += blockDim.x) {
+        if (q < E) counts[q] = q == e ? n : 0;
+        offs[q] = q <= e ? 0 : n;
+        mt_prefix[q] = q <= e ? 0 : (n + kGBM - 1) / kGBM;
+    }
+}
+
+// Inspection: one grouped-GEMM launch of the prefill plan on caller rows, all
+// of them routed to expert e (e = -1: the shared expert).  which 0: gate/up,
+// in [n][H] bf16, out [n][2I] binary32 accumulators (no SwiGLU); which 2:
+// down, in [n][I] bf16, out [n][H] binary32.
+cudaError_t launch_probe_gemm(const Weights& W, const Dims& D, const PrefillWs& ws, int which, int e,
+                              const void* in, int n, float* out, int n_sm, cudaStream_t st) {
+    cudaError_t err;
+    GemmArgs ga{};
+    ga.W = W;
+    ga.D = D;
+    ga.counts = ws.counts;
+    ga.offs = ws.offs;
+    ga.mt_prefix = ws.mt_prefix;
+    ga.err = ws.err;
+    ga.n_rows = n;
+    CUtensorMap mA, mB0, mB1;
+    const int K = which == 0 ? D.H : D.I;
+    if ((err = encode_tmap(&mA, in, n, K)) != cudaSuccess) return err;
+    if (e >= 0) {
+        k_probe_plan<<<1, 256, 0, st>>>(D.E, e, n, ws.counts, ws.offs, ws.mt_prefix);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        if (which == 0) {
+            ga.out_raw = out;
+            return launch_gemm<kModeGateUp>(mA, mA, mA, ga, n_sm, st);
+        }
+        ga.out_y = out;
+        return launch_gemm<kModeDown>(mA, mA, mA, ga, n_sm, st);
+    }
+    if (which == 0) {
+        if ((err = encode_tmap_core(&mB0, W.sh_gate, D.I, D.H)) != cudaSuccess) return err;
+        if ((err = encode_tmap_core(&mB1, W.sh_up, D.I, D.H)) != cudaSuccess) return err;
+        ga.out_raw = out;
+        return launch_gemm<kModeShGateUp>(mA, mB0, mB1, ga, n_sm, st);
+    }
+    if ((err = encode_tmap_core(&mB0, W.sh_down, D.H, D.I)) != cudaSuccess) return err;
+    ga.out_y = out;
+    return launch_gemm<kModeShDown>(mA, mB0, mB0, ga, n_sm, st);
 }
 
 // Routing only (prefill sizes): logits and top-k.

@@ -128,8 +128,9 @@ ds4moe_status ds4moe_pack_iq2xxs(const float* d_w, int64_t n_weights, const uint
 
 /* Grid magnitudes [256][8] uint8.  The prefill plan (n_tokens > decode_max)
  * expects at most four distinct byte values in the grid (the format's grid
- * uses three); with more, a prefill forward writes no output and records
- * device error bit 2 (see ds4moe_get_device_error). */
+ * uses three); with more, a prefill forward leaves out as it was and records
+ * device error bit 2 (see ds4moe_get_device_error); the next forward with a
+ * valid grid writes out again. */
 ds4moe_status ds4moe_set_grid(ds4moe_t* h, const uint8_t* d_grid, void* stream);
 
 /* Router rows [E][H] binary32 and, when has_bias, bias [E] (else NULL). */
@@ -237,6 +238,20 @@ ds4moe_status ds4moe_route(ds4moe_t* h, const void* d_x, int32_t n_tokens, int32
 ds4moe_status ds4moe_dequant(ds4moe_t* h, int32_t e, int32_t which, int32_t as_bf16, void* d_out,
                              void* stream);
 
+/* The grouped-GEMM kernels of a plan run on caller rows, all of them routed to
+ * expert e (0..E-1; -1 = the shared expert), with the accumulators written
+ * out as they are: the inspection the bit-exactness of the weights the
+ * kernels multiply rests on (one-hot rows give back columns of the weight
+ * matrices exactly as the tensor cores consumed them).
+ *   plan 1 (the prefill plan; needs max_tokens > decode_max): the tcgen05
+ *     grouped GEMM.  which 0: d_in = activations [n][H] bfloat16, d_out =
+ *     [n][2I] binary32, gate accumulators then up accumulators (no SwiGLU);
+ *     which 2: d_in = h [n][I] bfloat16, d_out = [n][H] binary32.
+ * d_in and d_out are 16-byte aligned device buffers; n in 1..2^20.  Uses
+ * the prefill region of the workspace (its routing plan is overwritten). */
+ds4moe_status ds4moe_probe(ds4moe_t* h, int32_t plan, int32_t which, int32_t e, const void* d_in, int32_t n_rows,
+                           float* d_out, void* stream);
+
 /* ---- routing without device allocation ------------------------------------ */
 
 /* ds4moe_route for callers that cannot allocate device memory: hosts that own
@@ -262,6 +277,14 @@ ds4moe_status ds4moe_dequant(ds4moe_t* h, int32_t e, int32_t which, int32_t as_b
  * ds4moe_get_device_error reads and clears. */
 ds4moe_status ds4moe_route_noalloc(ds4moe_t* h, const void* d_x, int32_t n_tokens, int32_t* d_ids,
                                    float* d_weights, void* stream);
+
+/* Check of the failure path every bounded device-side wait takes: runs one
+ * warp whose wait (the routine all the kernels' waits use) is on an mbarrier
+ * that nothing arrives at.  The wait gives up after its limit (0.5 s), sets
+ * bit 1 of the workspace error word and the kernel returns, so the context
+ * stays usable; ds4moe_get_device_error then returns DS4MOE_ERR_TIMEOUT.
+ * Needs a bound workspace.  Nothing faults, traps or hangs. */
+ds4moe_status ds4moe_selftest_wait(ds4moe_t* h, void* stream);
 
 /* Synchronize `stream`, then read and clear the workspace's device error word
  * (and, when ds4moe_route_noalloc has run on the current device, the error
