@@ -33,7 +33,8 @@ EXPORTS = ("ds4moe_create", "ds4moe_destroy", "ds4moe_weight_bytes", "ds4moe_wor
            "ds4moe_get_device_error", "ds4moe_last_error", "ds4moe_plan_launches", "ds4moe_plan_kernel",
            "ds4moe_forward_profiled", "ds4moe_route_noalloc", "ds4moe_forward_residual",
            "ds4moe_forward_residual_profiled", "ds4moe_set_steering", "ds4moe_forward_host_async",
-           "ds4moe_host_sync", "ds4moe_probe", "ds4moe_selftest_wait")
+           "ds4moe_host_sync", "ds4moe_probe", "ds4moe_selftest_wait",
+           "ds4moe_permutation")
 
 
 class ds4moe_shape(ctypes.Structure):
@@ -76,6 +77,7 @@ def lib() -> ctypes.CDLL:
             "ds4moe_dequant": ([vp, i32, i32, i32, vp, vp], i32),
             "ds4moe_probe": ([vp, i32, i32, i32, vp, i32, vp, vp], i32),
             "ds4moe_selftest_wait": ([vp, vp], i32),
+            "ds4moe_permutation": ([vp, vp, i32, vp, vp, vp, vp], i32),
             "ds4moe_get_device_error": ([vp, vp, ctypes.POINTER(i32)], i32),
             "ds4moe_last_error": ([], ctypes.c_char_p),
             "ds4moe_plan_launches": ([vp, i32], i32),
@@ -239,6 +241,13 @@ def ds4moe_probe(h: int, plan: int, which: int, e: int, inp: torch.Tensor, out: 
 
 def ds4moe_dequant(h: int, e: int, which: int, as_bf16: int, out: torch.Tensor, stream=None):
     _ok(lib().ds4moe_dequant(h, e, which, as_bf16, _ptr(out), _stream(stream)), "ds4moe_dequant")
+
+
+def ds4moe_permutation(h: int, ids: torch.Tensor, counts: torch.Tensor, offsets: torch.Tensor,
+                       pos_of_slot: torch.Tensor, stream=None):
+    """The prefill plan's stable counting sort of the (token, slot) pairs of ids [n][k] by expert."""
+    _ok(lib().ds4moe_permutation(h, _ptr(ids), ids.shape[0], _ptr(counts), _ptr(offsets), _ptr(pos_of_slot),
+                                 _stream(stream)), "ds4moe_permutation")
 
 
 def ds4moe_selftest_wait(h: int, stream=None):

@@ -1,10 +1,10 @@
-// decode.cu -- the fp32 GEMV plan for 1..decode_max tokens (four launches).
+// decode.cu -- the decode plan for 1..decode_max tokens (four launches).
 //
-//   k_router_decode  warp per expert row, logits in the canonical binary32
+//   k_router_decode  one warp per expert row, logits in the canonical binary32
 //                    order; the last CTA picks the top-k by (logit desc,
 //                    index asc) and the softmax over the selected logits.
 //   k_gateup_decode  h = silu(W_gate x) * (W_up x) for every selected expert
-//                    (read once, applied to all tokens that chose it) and for
+//                    (read once, applied to every token that chose it) and for
 //                    the shared expert.
 //   k_down_decode    y = W_down h per selected expert and for the shared
 //                    expert.
@@ -12,19 +12,32 @@
 //                    x + that for the residual step; k_combine_steer_decode
 //                    also steers: y - F v (v . y)).
 //
-// The two GEMV kernels are persistent (one CTA per SM): a producer warp pulls
-// row tasks from an atomic queue and streams their weights into a ring of
-// shared-memory stages with bulk copies (cp.async.bulk + mbarrier), 16 (for
-// up to 2 tokens; 8 otherwise) consumer warps dequantize and multiply out of
-// shared memory.  Each is
-// launched with programmatic dependent launch: the gate/up grid starts its
-// shared-expert tasks while the router still runs, and the down grid streams
-// its weights while gate/up finishes; both wait (griddepcontrol.wait) only
-// where they read the previous grid's results.
-//
-// The IQ2 grid is expanded to binary32 in shared memory, in 8 interleaved
-// copies so that the per-lane random row lookups of a quarter warp never
-// share a bank.
+// The two projection kernels are persistent (one CTA per SM): a producer warp
+// pulls row tasks from an atomic queue and streams their weights into a ring
+// of shared-memory stages with bulk copies (cp.async.bulk + mbarrier); the
+// consumer warps turn the packed weights into exact small integers in
+// registers and multiply them on the tensor cores with warp-level MMAs, so the
+// per-weight work is the unpacking alone:
+//   IQ2 (gate, up): each 8-weight chunk becomes eight int8 values +-G by two
+//     byte permutes whose selectors come from two shared-memory tables (grid
+//     row -> magnitude classes, 7 sign bits -> sign flags with the parity of
+//     the eighth folded in); x enters as four int8 pieces of a per-token
+//     power-of-two scale (29 bits of precision), the int32 products of a
+//     32-weight group are scaled by its odd integer 2s+1 in int32, and every
+//     superblock's sum is converted once and scaled by d/8.
+//   Q2 (down): codes become the bfloat16 numbers 1 + q/4 by a rotate, a mask
+//     and two byte permutes; h enters as two bfloat16 pieces (hi, lo); each
+//     16-weight sub-block's result is 4 d sc (D - S) - dmin m S with D its
+//     MMA sum and S its sum of h.
+//   shared expert: the bf16 weights are the MMA operand as stored; x and h
+//     enter as two bfloat16 pieces.
+// The MMA's eight accumulator columns hold (token, piece) pairs or, when an
+// expert serves one token, different 32-weight groups (IQ2) or 16-weight
+// sub-blocks (Q2) of that token, so that their scales are applied once per
+// several MMAs.  Each kernel is launched with programmatic dependent launch:
+// the gate/up grid starts its shared-expert tasks while the router still runs,
+// and the down grid streams its weights while gate/up finishes; both wait
+// (griddepcontrol.wait) only where they read the previous grid's results.
 #include <map>
 #include <mutex>
 #include <utility>
@@ -34,66 +47,88 @@
 
 namespace ds4 {
 
-// Consumer warps per CTA of the GEMV kernels (plus one producer warp).
-template <int NT>
-struct Warps {
-    static constexpr int CW = NT <= 2 ? 16 : 8;
-    static constexpr int kThreads = (CW + 1) * 32;
-};
 constexpr int kMaxSlots = 128;                 // decode_max (<= 8) * top_k (<= 16)
 constexpr int kStageBytes = 34816;             // 32 KB of weights + 2 KB of scales
-constexpr int kRWarps = 4;                     // router warps per CTA
+constexpr int kRE = 2;                         // router rows (warps) per CTA
 
-// ---------------------------------------------------------------- router
-__device__ __forceinline__ float4 load_x4(const void* x, int act_bf16, int64_t idx) {
-    if (act_bf16) {
-        uint2 v = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(x) + idx));
-        return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
-                           __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
-    }
-    return __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + idx));
+// ---------------------------------------------------------------- warp MMAs
+// int8 A (16 x 32, row) times int8 B (32 x 8, col), int32 accumulators.
+__device__ __forceinline__ void imma_z(int (&d)[4], const uint32_t (&a)[4], uint2 b) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b.x), "r"(b.y), "r"(0));
+}
+__device__ __forceinline__ void imma(int (&d)[4], const uint32_t (&a)[4], uint2 b) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b.x), "r"(b.y));
+}
+// bf16 A (16 x 16, row) times bf16 B (16 x 8, col), binary32 accumulators.
+__device__ __forceinline__ void bmma(float (&d)[4], const uint32_t (&a)[4], uint2 b) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b.x), "r"(b.y));
 }
 
+__device__ __forceinline__ uint32_t bf16_bits(float v) {
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// ---------------------------------------------------------------- router
+// One CTA per kRE expert rows, one warp per row.  Thread 0 brings the CTA's
+// router rows and all n token vectors into shared memory with two bulk copies
+// on one mbarrier, so every CTA's rows are in flight at once (the 4 MB of
+// W_r arrive in about one memory latency).  Lane L then runs chain L of the
+// canonical order (columns 128 i + 4L + r, i ascending, r = 0..3, one fma
+// each), the chains meet in the fixed butterfly (xor 16, 8, 4, 2, 1) and
+// the bias is added once.  The last CTA to finish picks the top-k.
 template <int NT>
-__global__ void __launch_bounds__(kRWarps * 32) k_router_decode(Weights W, Dims D, DecodeWs ws, const void* x, int n) {
+__global__ void __launch_bounds__(kRE * 32) k_router_decode(Weights W, Dims D, DecodeWs ws, const void* x, int n) {
     griddep_launch();   // the gate/up grid may start its shared-expert work now
-    extern __shared__ __align__(16) float xs_r[];   // [n][H]
+    extern __shared__ __align__(128) unsigned char r_smem[];   // [kRE][H] f32 rows, then x as given [n][H]
+    __shared__ uint64_t bar;
+    __shared__ bool s_last;
+    __shared__ float s_logits[kRE][1024];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = blockIdx.x * kRWarps + warp;
     const int H = D.H, E = D.E;
-    constexpr int B = 16;
-    const float* wr = W.W_r + (int64_t)(e < E ? e : 0) * H + 4 * lane;
-    uint4 w4[B];
-#pragma unroll
-    for (int b = 0; b < B; ++b)   // first batch in flight while x is staged
-        if (b < H / 128) w4[b] = ld_stream_v4(wr + 128 * b);
-    for (int i = threadIdx.x * 4; i < n * H; i += kRWarps * 32 * 4)
-        *reinterpret_cast<float4*>(xs_r + i) = load_x4(x, D.act_bf16, i);
+    const int e0 = blockIdx.x * kRE;
+    const int nrows = E - e0 < kRE ? E - e0 : kRE;
+    const float* wrows = reinterpret_cast<const float*>(r_smem);
+    const unsigned char* xsm = r_smem + (size_t)kRE * H * 4;
+    if (threadIdx.x == 0) {
+        const uint32_t wbytes = (uint32_t)nrows * H * 4, xbytes = (uint32_t)n * H * (D.act_bf16 ? 2 : 4);
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+        mbar_arrive_expect_tx(&bar, wbytes + xbytes);
+        bulk_load_plain(r_smem, W.W_r + (size_t)e0 * H, wbytes, &bar);
+        bulk_load_plain(r_smem + (size_t)kRE * H * 4, x, xbytes, &bar);
+    }
     __syncthreads();
-    if (e < E) {
+    mbar_wait(&bar, 0, ws.err);
+    if (warp < nrows) {
+        const int e = e0 + warp;
+        const float* wr = wrows + (size_t)warp * H + 4 * lane;
         float acc[NT];
 #pragma unroll
         for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-        for (int i0 = 0; i0 < H / 128; i0 += B) {
-            if (i0 > 0) {
+#pragma unroll 4
+        for (int i = 0; i < H / 128; ++i) {
+            const float4 wv = *reinterpret_cast<const float4*>(wr + 128 * i);
 #pragma unroll
-                for (int b = 0; b < B; ++b)
-                    if (i0 + b < H / 128) w4[b] = ld_stream_v4(wr + 128 * (i0 + b));
-            }
-#pragma unroll
-            for (int b = 0; b < B; ++b) {
-                if (i0 + b >= H / 128) break;
-                const float4 wv = make_float4(__uint_as_float(w4[b].x), __uint_as_float(w4[b].y),
-                                              __uint_as_float(w4[b].z), __uint_as_float(w4[b].w));
-#pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    if (t < n) {
-                        const float4 x4 = *reinterpret_cast<const float4*>(xs_r + t * H + 128 * (i0 + b) + 4 * lane);
-                        acc[t] = fmaf(x4.x, wv.x, acc[t]);
-                        acc[t] = fmaf(x4.y, wv.y, acc[t]);
-                        acc[t] = fmaf(x4.z, wv.z, acc[t]);
-                        acc[t] = fmaf(x4.w, wv.w, acc[t]);
+            for (int t = 0; t < NT; ++t) {
+                if (t < n) {
+                    float4 x4;
+                    if (D.act_bf16) {
+                        const uint2 v = *reinterpret_cast<const uint2*>(xsm + ((size_t)t * H + 128 * i + 4 * lane) * 2);
+                        x4 = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                                         __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+                    } else {
+                        x4 = *reinterpret_cast<const float4*>(xsm + ((size_t)t * H + 128 * i + 4 * lane) * 4);
                     }
+                    acc[t] = fmaf(x4.x, wv.x, acc[t]);
+                    acc[t] = fmaf(x4.y, wv.y, acc[t]);
+                    acc[t] = fmaf(x4.z, wv.z, acc[t]);
+                    acc[t] = fmaf(x4.w, wv.w, acc[t]);
                 }
             }
         }
@@ -109,8 +144,6 @@ __global__ void __launch_bounds__(kRWarps * 32) k_router_decode(Weights W, Dims 
                 if (t < n) ws.logits[(int64_t)t * E + e] = W.b_r ? acc[t] + b : acc[t];
         }
     }
-    __shared__ bool s_last;
-    __shared__ float s_logits[kRWarps][1024];
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
@@ -121,13 +154,16 @@ __global__ void __launch_bounds__(kRWarps * 32) k_router_decode(Weights W, Dims 
     if (!s_last) return;
     __threadfence();
     if (threadIdx.x == 0) *ws.ticket = 0;
-    for (int t = warp; t < n; t += kRWarps)
+    for (int t = warp; t < n; t += kRE)
         topk_softmax_warp(ws.logits + (int64_t)t * E, s_logits[warp], E, D.k, ws.ids + t * D.k, ws.wts + t * D.k);
 }
 
 // ---------------------------------------------------------------- routing table
-// Unique selected experts in ascending order, and for each the slots
-// (t * k + j) that chose it, in increasing slot order.  Built by one warp.
+// Routed tasks' experts ("entries") in ascending expert order, each with the
+// slots (t * k + j) that chose it in increasing slot order, at most tpb slots
+// per entry (an expert chosen by more tokens gets several entries, each
+// reading its weights once).  Built by one warp.  Probe calls (probe 1) route
+// every token to expert probe_e through slot t * k; probe 2 has no entries.
 struct Routing {
     int nu;
     int uniq[kMaxSlots];
@@ -139,8 +175,22 @@ struct Routing {
     int pos[kMaxSlots];
 };
 
-__device__ void build_routing_warp(Routing& R, const int32_t* ids, int nk) {
-    const int lane = threadIdx.x & 31;
+__device__ void build_routing_warp(Routing& R, const int32_t* ids, int n, int k, int tpb, int probe, int probe_e) {
+    const int lane = threadIdx.x & 31, nk = n * k;
+    if (probe) {
+        if (lane == 0) {
+            const int nu = probe == 1 ? (n + tpb - 1) / tpb : 0;
+            for (int u = 0; u < nu; ++u) {
+                R.uniq[u] = probe_e;
+                R.ustart[u] = u * tpb;
+            }
+            R.ustart[nu] = n;
+            for (int t = 0; t < n; ++t) R.slot[t] = t * k;
+            R.nu = nu;
+        }
+        __syncwarp();
+        return;
+    }
     for (int s = lane; s < nk; s += 32) R.ids[s] = __ldcg(ids + s);
     __syncwarp();
     for (int s = lane; s < nk; s += 32) {
@@ -176,6 +226,21 @@ __device__ void build_routing_warp(Routing& R, const int32_t* ids, int nk) {
     __syncwarp();
     for (int s = lane; s < nk; s += 32) R.slot[R.ustart[R.rank[s]] + R.pos[s]] = s;
     __syncwarp();
+    if (lane == 0) {   // split the entries into runs of at most tpb slots (scratch: first = experts, rank = starts)
+        const int nu = R.nu;
+        for (int u = 0; u <= nu; ++u) R.rank[u] = R.ustart[u];
+        for (int u = 0; u < nu; ++u) R.first[u] = R.uniq[u];
+        int m = 0;
+        for (int u = 0; u < nu; ++u)
+            for (int s = R.rank[u]; s < R.rank[u + 1]; s += tpb) {
+                R.uniq[m] = R.first[u];
+                R.ustart[m] = s;
+                ++m;
+            }
+        R.ustart[m] = nk;
+        R.nu = m;
+    }
+    __syncwarp();
 }
 
 // ---------------------------------------------------------------- pipeline state
@@ -183,7 +248,7 @@ struct ChunkInfo {
     int task;      // -1: no more work
     int chunk;     // chunk index within the task
     int nchunk;    // chunks of the task
-    int lo, cnt;   // first k step of the chunk and how many
+    int lo, cnt;   // routed: first k step (64 columns) of the chunk and how many; shared: first column, columns
 };
 
 struct Pipe {
@@ -237,132 +302,164 @@ __device__ void producer_finish(Pipe& P, uint32_t it, int NS, uint32_t* err) {
     __syncwarp();
 }
 
-// ---------------------------------------------------------------- IQ2 groups
-// The eight signed grid magnitudes of one IQ2 chunk (grid row a, 7 sign bits
-// + parity taken from S), as binary32.  tabp: this lane's grid replica.
-template <int TR>
-__device__ __forceinline__ void iq2_chunk(uint32_t idx, uint32_t S, int c, const float* __restrict__ tabp,
-                                          float* w) {
-    const uint32_t a = (idx >> (8 * c)) & 255u;
-    uint32_t sg = (S >> (7 * c)) & 127u;
-    sg |= ((uint32_t)__popc(sg) & 1u) << 7;
-    const float* trow = tabp + a * (8 * TR);
-    const float4 g0 = *reinterpret_cast<const float4*>(trow);
-    const float4 g1 = *reinterpret_cast<const float4*>(trow + 4 * TR);
-    w[0] = g0.x; w[1] = g0.y; w[2] = g0.z; w[3] = g0.w;
-    w[4] = g1.x; w[5] = g1.y; w[6] = g1.z; w[7] = g1.w;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = __uint_as_float(__float_as_uint(w[i]) ^ ((sg << (31 - i)) & 0x80000000u));
+// Position of column c of h in the routed h layout ([I/64][2 pieces][64]
+// per slot): inside each 16-column block, column 4e + c4 sits at 4 c4 + e, the
+// order in which the down kernel's MMA fragments read the codes of a block.
+__device__ __forceinline__ int hrt_index(int c, int piece) {
+    const int w = c & 63;
+    return ((c >> 6) * 2 + piece) * 64 + (w & ~15) + 4 * (w & 3) + ((w >> 2) & 3);
 }
-
-// d * (2s + 1) / 8 for the group scale s in bits 28..31 of S (no int->float
-// conversion unit: 2s+1 < 2^23 is placed under exponent 2^23 and the bias
-// subtracted exactly).
-__device__ __forceinline__ float iq2_scale(uint32_t S, float d) {
-    const float odd = __uint_as_float(0x4b000001u | ((S >> 27) & 0x1eu)) - 8388608.0f;
-    return d * odd * 0.125f;
-}
-
-// A gate group and the up group at the same columns (32 weights each) against
-// NT token vectors; the token values are read once for both.
-template <int NT, int TR>
-__device__ __forceinline__ void iq2_group_pair(uint4 pg, uint4 pu, int half, float dg, float du,
-                                               const float* __restrict__ tabp, const float* __restrict__ xcol,
-                                               int H, const int* tok, int ns, float* ag, float* au) {
-    const uint32_t gi = half ? pg.z : pg.x, gS = half ? pg.w : pg.y;
-    const uint32_t ui = half ? pu.z : pu.x, uS = half ? pu.w : pu.y;
-    float2 gs[NT], us[NT];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) gs[t] = us[t] = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        float wg[8], wu[8];
-        iq2_chunk<TR>(gi, gS, c, tabp, wg);
-        iq2_chunk<TR>(ui, uS, c, tabp, wu);
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            if (t < ns) {
-                const float* xr = xcol + tok[t] * H + 8 * c;
-                const float4 x0 = *reinterpret_cast<const float4*>(xr);
-                const float4 x1 = *reinterpret_cast<const float4*>(xr + 4);
-                gs[t] = ffma2(make_float2(wg[0], wg[1]), make_float2(x0.x, x0.y), gs[t]);
-                us[t] = ffma2(make_float2(wu[0], wu[1]), make_float2(x0.x, x0.y), us[t]);
-                gs[t] = ffma2(make_float2(wg[2], wg[3]), make_float2(x0.z, x0.w), gs[t]);
-                us[t] = ffma2(make_float2(wu[2], wu[3]), make_float2(x0.z, x0.w), us[t]);
-                gs[t] = ffma2(make_float2(wg[4], wg[5]), make_float2(x1.x, x1.y), gs[t]);
-                us[t] = ffma2(make_float2(wu[4], wu[5]), make_float2(x1.x, x1.y), us[t]);
-                gs[t] = ffma2(make_float2(wg[6], wg[7]), make_float2(x1.z, x1.w), gs[t]);
-                us[t] = ffma2(make_float2(wu[6], wu[7]), make_float2(x1.z, x1.w), us[t]);
-            }
-        }
-    }
-    const float sgate = iq2_scale(gS, dg), sup = iq2_scale(uS, du);
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-        ag[t] = fmaf(sgate, gs[t].x + gs[t].y, ag[t]);
-        au[t] = fmaf(sup, us[t].x + us[t].y, au[t]);
-    }
-}
-
-// bf16x2 word -> two binary32 values, multiply-accumulated against x pairs.
-__device__ __forceinline__ float2 bf16x2_fma(uint32_t wbits, float2 x, float2 acc) {
-    return ffma2(make_float2(__uint_as_float(wbits << 16), __uint_as_float(wbits & 0xffff0000u)), x, acc);
-}
-
-__device__ __forceinline__ void bf16x8_dot(uint4 w, const float* xr, float2& acc) {
-    const float4 x0 = *reinterpret_cast<const float4*>(xr);
-    const float4 x1 = *reinterpret_cast<const float4*>(xr + 4);
-    acc = bf16x2_fma(w.x, make_float2(x0.x, x0.y), acc);
-    acc = bf16x2_fma(w.y, make_float2(x0.z, x0.w), acc);
-    acc = bf16x2_fma(w.z, make_float2(x1.x, x1.y), acc);
-    acc = bf16x2_fma(w.w, make_float2(x1.z, x1.w), acc);
-}
+__device__ __forceinline__ int hsh_index(int c, int piece) { return ((c >> 6) * 2 + piece) * 64 + (c & 63); }
 
 // ---------------------------------------------------------------- gate/up
 template <int NT>
 struct GateUpCfg {
-    static constexpr int TR = NT <= 2 ? 8 : 1;            // grid replicas
-    static constexpr int NS = NT <= 4 ? 3 : 2;            // stages
-    static constexpr int kTabFloats = 256 * 8 * TR;
-    static constexpr int CW = Warps<NT>::CW;
-    static constexpr int kRedFloats = CW * 2 * NT * 32;
+    static constexpr int CW = NT <= 2 ? 16 : 8;                   // consumer warps
+    static constexpr int NS = NT <= 4 ? 3 : 2;                    // stages
+    static constexpr int R = NT <= 2 ? 32 : (NT == 4 ? 16 : 8);   // copies of the selector tables
+    static constexpr int TPB = NT == 1 ? 1 : 2;                   // tokens of one routed entry
+    static constexpr int kThreads = (CW + 1) * 32;
+    static constexpr int kTabWords = (256 + 128) * R;
+    static constexpr int kRedFloats = CW * 4 * 64;                // [warp][4 tokens][64 rows]
+};
+
+// The IQ2 chunk of one thread (8 weights, grid row a from byte t of the
+// index word, sign field at bit 7t of S) as int8 +-G: weights 0..3 in lo,
+// 4..7 in hi.  The selector's nibble i is the magnitude class of weight i
+// plus 4 for a negative sign; (clo, chi) hold the four magnitudes and their
+// negatives.
+// tsel / tsgn point at this lane's copy of the tables (copies interleaved, R words per entry).
+template <int R>
+__device__ __forceinline__ void iq2_chunk_s8(uint32_t idx, uint32_t S, uint32_t selA, int t7, const uint32_t* tsel,
+                                             const uint32_t* tsgn, uint32_t clo, uint32_t chi, uint32_t& lo,
+                                             uint32_t& hi) {
+    const uint32_t a = __byte_perm(idx, 0u, selA);
+    const uint32_t sg = (S >> t7) & 127u;
+    const uint32_t sel = tsel[a * R] | tsgn[sg * R];
+    lo = __byte_perm(clo, chi, sel);
+    hi = __byte_perm(clo, chi, sel >> 16);
+}
+
+// Per consumer thread state of the gate/up kernel's tasks.
+template <int NT>
+struct GateUpAcc {
+    static constexpr int TG = (NT + 3) / 4;   // token groups of four (shared tasks)
+    float sh[TG][4][4];                       // shared task: [token group][tile][fragment]
+    float rt[GateUpCfg<NT>::TPB][4][2];       // routed task: [token][tile][row g, g + 8]
 };
 
 template <int NT>
-__global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
+__global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     k_gateup_decode(Weights W, Dims D, DecodeWs ws, const void* x, int n) {
     using C = GateUpCfg<NT>;
-    constexpr int NS = C::NS, TR = C::TR, CW = C::CW, kGThreads = Warps<NT>::kThreads;
+    constexpr int NS = C::NS, CW = C::CW, R = C::R, TPB = C::TPB, kThreads = C::kThreads;
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    unsigned char* stages = smem_raw;                                   // NS x kStageBytes
-    float* tab = reinterpret_cast<float*>(smem_raw + NS * kStageBytes);  // kTabFloats
-    float* red = tab + C::kTabFloats;                                   // kRedFloats
-    float* xs = red + C::kRedFloats;                                    // [n][H]
+    unsigned char* stages = smem_raw;                                            // NS x kStageBytes
+    uint32_t* tsel = reinterpret_cast<uint32_t*>(smem_raw + NS * kStageBytes);   // [256][R]
+    uint32_t* tsgn = tsel + 256 * R;                                             // [128][R]
+    float* red = reinterpret_cast<float*>(tsgn + 128 * R);                       // kRedFloats
+    unsigned char* xbuf = reinterpret_cast<unsigned char*>(red + C::kRedFloats);  // n x H x 4 bytes
+    unsigned char* zero = xbuf + (size_t)n * D.H * 4;                            // 64 bytes of zeros
     __shared__ Pipe P;
-    __shared__ Routing R;
-    __shared__ int s_last;
+    __shared__ Routing Rt;
+    __shared__ int s_last, s_refused;
+    __shared__ uint32_t s_cand[2];
+    __shared__ float s_tokmax[8];
+    __shared__ float s_cs[8][4];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
     const int H = D.H, I = D.I, k = D.k;
     const int nkt = H / 64, nsb = H / 256;
-    const int n_sh = D.has_shared ? I / 8 : 0;
+    const int n_sh = ws.probe == 1 ? 0 : (D.has_shared ? I / 32 : 0);
     const int rb_per_e = I / 32;
-    const int ck_rt = nkt < 32 ? nkt : 32;            // k steps (64 columns) per routed chunk
+    // k steps (64 columns) per routed chunk: the largest of 32, 16, 8, 4 that divides H / 64
+    const int ck_rt = nkt % 32 == 0 ? 32 : nkt % 16 == 0 ? 16 : nkt % 8 == 0 ? 8 : 4;
     const int nch_rt = nkt / ck_rt;
-    const int ck_sh = H / 8 < 128 ? H / 8 : 128;      // 8-column tiles per shared chunk
-    const int nch_sh = (H / 8) / ck_sh;
+    const int kcs = H < 256 ? H : 256;                // columns per shared chunk
+    const int nch_sh = H / kcs;
 
     pipe_init(P, NS, CW);
-    // grid: one 32-bit load per 4 magnitudes, expanded to TR interleaved copies
-    for (int q = tid; q < 512; q += kGThreads) {
-        const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(W.grid_u8) + q);
-        const int a = q >> 1, hf = q & 1;
-        const float4 f = make_float4((float)(v & 0xffu), (float)((v >> 8) & 0xffu), (float)((v >> 16) & 0xffu),
-                                     (float)(v >> 24));
+    // ---- grid: magnitude classes (at most four distinct values, each at most 127), selector tables
+    {
+        int* present = reinterpret_cast<int*>(red);
+        for (int v = tid; v < 256; v += kThreads) present[v] = 0;
+        if (tid < 4) reinterpret_cast<uint4*>(zero)[tid] = make_uint4(0, 0, 0, 0);
+        __syncthreads();
+        for (int q = tid; q < 2048; q += kThreads) present[W.grid_u8[q]] = 1;
+        __syncthreads();
+        if (tid == 0) {
+            int nv = 0;
+            uint32_t lo = 0, hi = 0;
+            bool big = false;
+            for (int v = 0; v < 256; ++v) {
+                if (!present[v]) continue;
+                if (nv < 4) {
+                    lo |= (uint32_t)v << (8 * nv);
+                    hi |= (uint32_t)((-v) & 0xff) << (8 * nv);
+                }
+                big |= v > 127;
+                present[v] = 1 + (nv < 4 ? nv : 3);   // class + 1
+                ++nv;
+            }
+            s_cand[0] = lo;
+            s_cand[1] = hi;
+            s_refused = (nv > 4 || big) ? 1 : 0;
+            if (s_refused) set_err(ws.err, kErrGrid);
+            if (blockIdx.x == 0) *ws.grid_refused = s_refused;
+        }
+        __syncthreads();
+        for (int a = tid; a < 256; a += kThreads) {
+            uint32_t w = 0;
 #pragma unroll
-        for (int p = 0; p < TR; ++p) *reinterpret_cast<float4*>(tab + a * (8 * TR) + hf * (4 * TR) + p * 4) = f;
+            for (int i = 0; i < 8; ++i) w |= (uint32_t)(present[W.grid_u8[a * 8 + i]] - 1) << (4 * i);
+#pragma unroll
+            for (int r = 0; r < R; ++r) tsel[a * R + r] = w;
+        }
+        for (int sg = tid; sg < 128; sg += kThreads) {
+            uint32_t w = ((uint32_t)__popc(sg) & 1u) << 30;
+#pragma unroll
+            for (int i = 0; i < 7; ++i) w |= ((uint32_t)(sg >> i) & 1u) << (4 * i + 2);
+#pragma unroll
+            for (int r = 0; r < R; ++r) tsgn[sg * R + r] = w;
+        }
     }
-    for (int i = tid * 4; i < n * H; i += kGThreads * 4) *reinterpret_cast<float4*>(xs + i) = load_x4(x, D.act_bf16, i);
-    __syncthreads();
+    // ---- token maxima (for the int8 pieces of the routed tasks) and the shared tasks' bf16 pieces
+    {
+        float mx[NT];
+#pragma unroll
+        for (int q = 0; q < NT; ++q) mx[q] = 0.f;
+        uint32_t* xb = reinterpret_cast<uint32_t*>(xbuf);   // [n][2][H] bf16 as pairs
+        for (int i = tid * 2; i < H; i += kThreads * 2) {
+#pragma unroll
+            for (int q = 0; q < NT; ++q) {
+                if (q < n) {
+                    const float v0 = act_at(x, (int64_t)q * H + i, D.act_bf16);
+                    const float v1 = act_at(x, (int64_t)q * H + i + 1, D.act_bf16);
+                    mx[q] = fmaxf(mx[q], fmaxf(fabsf(v0), fabsf(v1)));
+                    if (n_sh > 0) {
+                        const uint32_t h0 = bf16_bits(v0), h1 = bf16_bits(v1);
+                        const float r0 = v0 - __uint_as_float(h0 << 16), r1 = v1 - __uint_as_float(h1 << 16);
+                        xb[((size_t)q * 2 * H + i) / 2] = h0 | (h1 << 16);
+                        xb[((size_t)(q * 2 + 1) * H + i) / 2] = bf16_bits(r0) | (bf16_bits(r1) << 16);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < NT; ++q) {
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) mx[q] = fmaxf(mx[q], __shfl_xor_sync(0xffffffffu, mx[q], m));
+        }
+        if (tid < 8) s_tokmax[tid] = 0.f;
+        __syncthreads();
+        if (lane == 0) {
+#pragma unroll
+            for (int q = 0; q < NT; ++q)
+                if (q < n) atomicMax(reinterpret_cast<int*>(&s_tokmax[q]), __float_as_int(mx[q]));
+        }
+        __syncthreads();
+    }
+    const bool refused = s_refused != 0;
 
     if (warp == CW) {
         // ------------------------------------------------ producer warp
@@ -373,14 +470,14 @@ __global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
         int next = 0;
         if (lane == 0) next = (int)atomicAdd(ws.queue1, 1u);
         for (;;) {
-            if (aborted(P)) break;
+            if (aborted(P) || refused) break;
             int task = __shfl_sync(0xffffffffu, next, 0);
             if (lane == 0) next = (int)atomicAdd(ws.queue1, 1u);   // in flight while this task streams
             if (task >= n_sh && !routed) {
                 griddep_wait();                   // router results visible
-                build_routing_warp(R, ws.ids, n * k);
+                build_routing_warp(Rt, ws.ids, n, k, TPB, ws.probe == 1 ? 1 : (ws.probe == 2 ? 2 : 0), ws.probe_e);
                 routed = true;
-                total = n_sh + R.nu * rb_per_e;
+                total = n_sh + Rt.nu * rb_per_e;
                 griddep_launch();                 // the down grid may start streaming
             }
             if (task >= total) break;
@@ -393,16 +490,21 @@ __global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
                 if (lane == 0) {
                     unsigned char* st = stages + s * kStageBytes;
                     if (sh) {
-                        const int kc0 = c * ck_sh;
-                        const size_t off = ((size_t)task * (H / 8) + kc0) * 64;   // elements
-                        const uint32_t bytes = ck_sh * 128;
-                        P.info[s] = ChunkInfo{task, c, nch, kc0, ck_sh};
-                        mbar_arrive_expect_tx(&P.full[s], 2 * bytes);
-                        bulk_load(st, W.sh_gate + off, bytes, &P.full[s], pol);
-                        bulk_load(st + bytes, W.sh_up + off, bytes, &P.full[s], pol);
+                        // 32 rows of the gate and up matrices, columns c*kcs .. +kcs, as four 8-row
+                        // groups of core-matrix tiles per matrix
+                        const int kc0 = c * kcs;
+                        const uint32_t bytes = kcs * 16;
+                        P.info[s] = ChunkInfo{task, c, nch, kc0, kcs};
+                        mbar_arrive_expect_tx(&P.full[s], 8 * bytes);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const size_t off = ((size_t)(task * 4 + q) * (H / 8) + kc0 / 8) * 64;   // elements
+                            bulk_load(st + q * bytes, W.sh_gate + off, bytes, &P.full[s], pol);
+                            bulk_load(st + 4 * bytes + q * bytes, W.sh_up + off, bytes, &P.full[s], pol);
+                        }
                     } else {
                         const int tt = task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
-                        const int e = R.uniq[u];
+                        const int e = Rt.uniq[u];
                         const int kt0 = c * ck_rt;
                         const uint32_t pb = ck_rt * 512, db = ck_rt * 16;
                         const size_t qoff = (size_t)e * W.iq2_qs_stride + ((size_t)rb * nkt + kt0) * 512;
@@ -420,13 +522,20 @@ __global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
             }
         }
         producer_finish(P, it, NS, ws.err);
-    } else {
+    } else if (!refused) {
         // ------------------------------------------------ consumer warps
-        const float* tabp = tab + (lane & (TR - 1)) * 4;
+        const uint32_t selA = 0x4440u | (uint32_t)t;   // byte t of the index word
+        const uint32_t selS = (t >> 1) ? 0x4447u : 0x4443u;   // top byte of this lane's group's S word
+        const uint32_t* tselp = tsel + (lane % R);
+        const uint32_t* tsgnp = tsgn + (lane % R);
+        const uint32_t clo = s_cand[0], chi = s_cand[1];
+        // B operand lanes: column g of the MMA
+        const int jB = g >> 2, pB = g & 3;                // routed: 32-column group, int8 piece
         uint32_t it = 0, cph = 0;
-        float2 sg2[NT], su2[NT];     // shared-task partials (this lane's row, k quarter)
-        float ag[NT], au[NT];        // routed-task partials (this lane's row)
-        int tok[NT];
+        bool quantized = false;
+        GateUpAcc<NT> A;
+        int tokrow[TPB];
+        int tcount = 0;
         for (;;) {
             const int s = it % NS;
             if (!mbar_wait(&P.full[s], (it / NS) & 1, ws.err)) { set_abort(P); break; }
@@ -434,104 +543,236 @@ __global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
             if (inf.task < 0 || aborted(P)) break;
             const unsigned char* st = stages + s * kStageBytes;
             const bool sh = inf.task < n_sh;
+            if (!sh && !quantized) {
+                // first routed stage: every consumer warp is done with the shared tasks' bf16 pieces;
+                // x becomes four int8 pieces per token in the same buffer
+                if (!cons_sync(P, cph, ws.err)) break;
+                for (int q = tid; q < 8 * 4; q += CW * 32) {
+                    const int tk = q >> 2, p = q & 3;
+                    int e = 0;
+                    frexpf(s_tokmax[tk], &e);
+                    s_cs[tk][p] = s_tokmax[tk] > 0.f ? ldexpf(1.f, e - 7 - 7 * p) : 0.f;
+                }
+                for (int q = tid * 4; q < n * H; q += CW * 32 * 4) {
+                    const int tk = q / H, i = q % H;
+                    int e = 0;
+                    frexpf(s_tokmax[tk], &e);
+                    // v = x 2^(7-e), |v| < 128; the scaling is split so that no factor overflows
+                    const int sh1 = (7 - e) / 2, sh2 = 7 - e - sh1;
+                    const float f1 = ldexpf(1.f, sh1), f2 = ldexpf(1.f, sh2);
+                    uint32_t pw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float v = act_at(x, (int64_t)tk * H + i + j, D.act_bf16) * f1 * f2;
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) {
+                            const float tv = truncf(v);
+                            pw[p] |= ((uint32_t)(int)tv & 0xffu) << (8 * j);
+                            v = (v - tv) * 128.f;
+                        }
+                    }
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) *reinterpret_cast<uint32_t*>(xbuf + (size_t)(tk * 4 + p) * H + i) = pw[p];
+                }
+                quantized = true;
+                if (!cons_sync(P, cph, ws.err)) break;
+            }
             if (sh) {
-                const int rr = lane & 7, kq = lane >> 3;
                 if (inf.chunk == 0) {
 #pragma unroll
-                    for (int t = 0; t < NT; ++t) sg2[t] = su2[t] = make_float2(0.f, 0.f);
-                }
-                const uint4* gt = reinterpret_cast<const uint4*>(st);
-                const uint4* ut = reinterpret_cast<const uint4*>(st + inf.cnt * 128);
-                for (int kc = warp * 4 + kq; kc < inf.cnt; kc += 4 * CW) {
-                    const uint4 wg = gt[kc * 8 + rr], wu = ut[kc * 8 + rr];
-                    const int col = 8 * (inf.lo + kc);
+                    for (int tg = 0; tg < GateUpAcc<NT>::TG; ++tg)
 #pragma unroll
-                    for (int t = 0; t < NT; ++t) {
-                        if (t < n) {
-                            bf16x8_dot(wg, xs + t * H + col, sg2[t]);
-                            bf16x8_dot(wu, xs + t * H + col, su2[t]);
-                        }
+                        for (int T = 0; T < 4; ++T) A.sh[tg][T][0] = A.sh[tg][T][1] = A.sh[tg][T][2] = A.sh[tg][T][3] = 0.f;
+                }
+                const int kc = inf.cnt;                                 // columns of the chunk
+                const uint16_t* xb = reinterpret_cast<const uint16_t*>(xbuf);
+                for (int ks = warp; ks < kc / 16; ks += CW) {
+                    const int col = inf.lo + 16 * ks;
+                    uint2 B[GateUpAcc<NT>::TG];
+#pragma unroll
+                    for (int tg = 0; tg < GateUpAcc<NT>::TG; ++tg) {
+                        const int tk = 4 * tg + (g >> 1), p = g & 1;
+                        B[tg] = *reinterpret_cast<const uint2*>(
+                            tk < n ? reinterpret_cast<const unsigned char*>(xb + (size_t)(tk * 2 + p) * H + col + 4 * t)
+                                   : zero);
+                    }
+#pragma unroll
+                    for (int T = 0; T < 4; ++T) {
+                        const unsigned char* base = st + (T >> 1) * (kc * 64) + (2 * (T & 1)) * (kc * 16) +
+                                                    (2 * ks + (t >> 1)) * 128 + g * 16 + (t & 1) * 8;
+                        const uint2 r0 = *reinterpret_cast<const uint2*>(base);
+                        const uint2 r1 = *reinterpret_cast<const uint2*>(base + kc * 16);
+                        const uint32_t Af[4] = {r0.x, r1.x, r0.y, r1.y};
+#pragma unroll
+                        for (int tg = 0; tg < GateUpAcc<NT>::TG; ++tg) bmma(A.sh[tg][T], Af, B[tg]);
                     }
                 }
             } else {
                 const int tt = inf.task - n_sh, u = tt / rb_per_e;
-                const int s0 = R.ustart[u], ns = R.ustart[u + 1] - s0;
+                const int s0 = Rt.ustart[u], ns = Rt.ustart[u + 1] - s0;
                 if (inf.chunk == 0) {
+                    tcount = ns;
 #pragma unroll
-                    for (int t = 0; t < NT; ++t) {
-                        ag[t] = au[t] = 0.f;
-                        tok[t] = t < ns ? R.slot[s0 + t] / k : 0;
+                    for (int q = 0; q < TPB; ++q) {
+                        tokrow[q] = q < ns ? Rt.slot[s0 + q] / k : 0;
+#pragma unroll
+                        for (int T = 0; T < 4; ++T) A.rt[q][T][0] = A.rt[q][T][1] = 0.f;
                     }
                 }
-                const uint4* gp = reinterpret_cast<const uint4*>(st);
-                const uint4* up = reinterpret_cast<const uint4*>(st + inf.cnt * 512);
-                const uint16_t* gd = reinterpret_cast<const uint16_t*>(st + 2 * inf.cnt * 512);
-                const uint16_t* ud = gd + inf.cnt * 8;
-                for (int kt = warp; kt < inf.cnt; kt += CW) {
-                    const uint4 pg = gp[kt * 32 + lane], pu = up[kt * 32 + lane];
-                    const float dg = half_bits(gd[(kt >> 2) * 32 + lane]);
-                    const float du = half_bits(ud[(kt >> 2) * 32 + lane]);
-                    const float* xcol = xs + 64 * (inf.lo + kt);
-                    iq2_group_pair<NT, TR>(pg, pu, 0, dg, du, tabp, xcol, H, tok, ns, ag, au);
-                    iq2_group_pair<NT, TR>(pg, pu, 1, dg, du, tabp, xcol + 32, H, tok, ns, ag, au);
+                const int ck = inf.cnt;
+                const int kpw = ck >= CW ? ck / CW : 1;
+                const int kb = warp * kpw;
+                if (kb < ck) {
+                    int ai[TPB][4][4];
+#pragma unroll
+                    for (int q = 0; q < TPB; ++q)
+#pragma unroll
+                        for (int T = 0; T < 4; ++T) ai[q][T][0] = ai[q][T][1] = ai[q][T][2] = ai[q][T][3] = 0;
+                    for (int kq = 0; kq < kpw; ++kq) {
+                        const int kt = kb + kq;
+                        const int col = 64 * (inf.lo + kt);
+                        uint2 B[TPB][2];
+#pragma unroll
+                        for (int q = 0; q < TPB; ++q) {
+                            const unsigned char* live =
+                                xbuf + (size_t)(tokrow[q] * 4 + pB) * H + col + 32 * jB + 8 * t;
+                            B[q][0] = *reinterpret_cast<const uint2*>(q < tcount && jB == 0 ? live : zero);
+                            B[q][1] = *reinterpret_cast<const uint2*>(q < tcount && jB == 1 ? live : zero);
+                        }
+#pragma unroll
+                        for (int T = 0; T < 4; ++T) {
+                            const unsigned char* pay = st + (T >> 1) * (ck * 512) + kt * 512 + (16 * (T & 1) + g) * 16;
+                            const uint4 r0 = *reinterpret_cast<const uint4*>(pay);
+                            const uint4 r1 = *reinterpret_cast<const uint4*>(pay + 128);
+                            uint32_t A0[4], A1[4];
+                            iq2_chunk_s8<R>(r0.x, r0.y, selA, 7 * t, tselp, tsgnp, clo, chi, A0[0], A0[2]);
+                            iq2_chunk_s8<R>(r1.x, r1.y, selA, 7 * t, tselp, tsgnp, clo, chi, A0[1], A0[3]);
+                            iq2_chunk_s8<R>(r0.z, r0.w, selA, 7 * t, tselp, tsgnp, clo, chi, A1[0], A1[2]);
+                            iq2_chunk_s8<R>(r1.z, r1.w, selA, 7 * t, tselp, tsgnp, clo, chi, A1[1], A1[3]);
+                            const int o0 = (int)(((__byte_perm(r0.y, r0.w, selS) >> 3) & 0x1eu) | 1u);
+                            const int o1 = (int)(((__byte_perm(r1.y, r1.w, selS) >> 3) & 0x1eu) | 1u);
+#pragma unroll
+                            for (int q = 0; q < TPB; ++q) {
+                                if (q < tcount) {
+                                    int Dv[4];
+                                    imma_z(Dv, A0, B[q][0]);
+                                    imma(Dv, A1, B[q][1]);
+                                    ai[q][T][0] += Dv[0] * o0;
+                                    ai[q][T][1] += Dv[1] * o0;
+                                    ai[q][T][2] += Dv[2] * o1;
+                                    ai[q][T][3] += Dv[3] * o1;
+                                }
+                            }
+                        }
+                    }
+                    // one superblock: x d/8 and the columns' piece scales
+                    const uint16_t* dq = reinterpret_cast<const uint16_t*>(st + 2 * ck * 512);
+                    const int sbl = kb / 4;
+                    const int p0 = 2 * (t & 1);
+#pragma unroll
+                    for (int T = 0; T < 4; ++T) {
+                        const uint16_t* dm = dq + (T >> 1) * (ck / 4) * 32 + sbl * 32 + 16 * (T & 1) + g;
+                        const float d0 = half_bits(dm[0]) * 0.125f, d1 = half_bits(dm[8]) * 0.125f;
+#pragma unroll
+                        for (int q = 0; q < TPB; ++q) {
+                            if (q < tcount) {
+                                const float c0 = s_cs[tokrow[q]][p0], c1 = s_cs[tokrow[q]][p0 + 1];
+                                A.rt[q][T][0] = fmaf((float)ai[q][T][0], d0 * c0, A.rt[q][T][0]);
+                                A.rt[q][T][0] = fmaf((float)ai[q][T][1], d0 * c1, A.rt[q][T][0]);
+                                A.rt[q][T][1] = fmaf((float)ai[q][T][2], d1 * c0, A.rt[q][T][1]);
+                                A.rt[q][T][1] = fmaf((float)ai[q][T][3], d1 * c1, A.rt[q][T][1]);
+                            }
+                        }
+                    }
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&P.empty[s]);
             if (inf.chunk == inf.nchunk - 1) {
-                // task epilogue: reduce the eight warps' partials, SwiGLU, store h
+                // task epilogue: reduce the warps' partials, SwiGLU, store h (two bf16 pieces) and its block sums
+                bool ok = true;
                 if (sh) {
-                    const int rr = lane & 7, kq = lane >> 3;
 #pragma unroll
-                    for (int t = 0; t < NT; ++t) {
-                        float g = sg2[t].x + sg2[t].y, uu = su2[t].x + su2[t].y;
-                        g += __shfl_xor_sync(0xffffffffu, g, 8);
-                        g += __shfl_xor_sync(0xffffffffu, g, 16);
-                        uu += __shfl_xor_sync(0xffffffffu, uu, 8);
-                        uu += __shfl_xor_sync(0xffffffffu, uu, 16);
-                        if (kq == 0 && t < n) {
-                            red[((warp * 2 + 0) * NT + t) * 32 + rr] = g;
-                            red[((warp * 2 + 1) * NT + t) * 32 + rr] = uu;
+                    for (int tg = 0; tg < GateUpAcc<NT>::TG; ++tg) {
+                        // this lane's token is 4 tg + t: its columns 2t, 2t+1 are that token's two pieces
+#pragma unroll
+                        for (int T = 0; T < 4; ++T) {
+                            const int row = (T >> 1) * 32 + 16 * (T & 1) + g;
+                            red[(warp * 4 + t) * 64 + row] = A.sh[tg][T][0] + A.sh[tg][T][1];
+                            red[(warp * 4 + t) * 64 + row + 8] = A.sh[tg][T][2] + A.sh[tg][T][3];
                         }
-                    }
-                    if (!cons_sync(P, cph, ws.err)) break;
-                    if (tid < 8 * n) {
-                        const int r = tid & 7, t = tid >> 3;
-                        float g = 0.f, uu = 0.f;
-                        for (int w = 0; w < CW; ++w) {
-                            g += red[((w * 2 + 0) * NT + t) * 32 + r];
-                            uu += red[((w * 2 + 1) * NT + t) * 32 + r];
+                        if (!(ok = cons_sync(P, cph, ws.err))) break;
+                        if (tid < 128) {
+                            const int tl = tid >> 5, row = tid & 31, tok = 4 * tg + tl;
+                            float gv = 0.f, uv = 0.f;
+                            for (int w = 0; w < CW; ++w) {
+                                gv += red[(w * 4 + tl) * 64 + row];
+                                uv += red[(w * 4 + tl) * 64 + 32 + row];
+                            }
+                            const int c = 32 * inf.task + row;
+                            if (tok < n) {
+                                if (ws.probe) {
+                                    ws.probe_out[(size_t)tok * 2 * I + c] = gv;
+                                    ws.probe_out[(size_t)tok * 2 * I + I + c] = uv;
+                                } else {
+                                    const float h = silu(gv) * uv;
+                                    const uint32_t hi = bf16_bits(h);
+                                    const uint32_t lo = bf16_bits(h - __uint_as_float(hi << 16));
+                                    uint16_t* hb = ws.hb_sh + (size_t)tok * 2 * I;
+                                    hb[hsh_index(c, 0)] = (uint16_t)hi;
+                                    hb[hsh_index(c, 1)] = (uint16_t)lo;
+                                }
+                            }
                         }
-                        ws.h_sh[(int64_t)t * I + 8 * inf.task + r] = silu(g) * uu;
+                        if (!(ok = cons_sync(P, cph, ws.err))) break;
                     }
                 } else {
                     const int tt = inf.task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
-                    const int s0 = R.ustart[u], ns = R.ustart[u + 1] - s0;
+                    const int s0 = Rt.ustart[u];
 #pragma unroll
-                    for (int t = 0; t < NT; ++t) {
-                        if (t < ns) {
-                            red[((warp * 2 + 0) * NT + t) * 32 + lane] = ag[t];
-                            red[((warp * 2 + 1) * NT + t) * 32 + lane] = au[t];
+                    for (int q = 0; q < TPB; ++q) {
+#pragma unroll
+                        for (int T = 0; T < 4; ++T) {
+#pragma unroll
+                            for (int r = 0; r < 2; ++r) {
+                                float v = A.rt[q][T][r];
+                                v += __shfl_xor_sync(0xffffffffu, v, 1);
+                                v += __shfl_xor_sync(0xffffffffu, v, 2);
+                                if (t == 0) red[(warp * 4 + q) * 64 + (T >> 1) * 32 + 16 * (T & 1) + g + 8 * r] = v;
+                            }
                         }
                     }
-                    if (!cons_sync(P, cph, ws.err)) break;
-                    if (warp < ns) {
-                        const int t = warp;
-                        float g = 0.f, uu = 0.f;
-                        for (int w = 0; w < CW; ++w) {
-                            g += red[((w * 2 + 0) * NT + t) * 32 + lane];
-                            uu += red[((w * 2 + 1) * NT + t) * 32 + lane];
-                        }
-                        const float h = silu(g) * uu;
-                        const int slot = R.slot[s0 + t];
-                        ws.h_rt[(int64_t)slot * I + 32 * rb + lane] = h;
-                        float hs = h;
+                    if ((ok = cons_sync(P, cph, ws.err))) {
+                        if (warp < tcount) {
+                            const int q = warp, row = lane;
+                            float gv = 0.f, uv = 0.f;
+                            for (int w = 0; w < CW; ++w) {
+                                gv += red[(w * 4 + q) * 64 + row];
+                                uv += red[(w * 4 + q) * 64 + 32 + row];
+                            }
+                            const int slot = Rt.slot[s0 + q];
+                            const int c = 32 * rb + row;
+                            if (ws.probe) {
+                                ws.probe_out[(size_t)tokrow[q] * 2 * I + c] = gv;
+                                ws.probe_out[(size_t)tokrow[q] * 2 * I + I + c] = uv;
+                            } else {
+                                const float h = silu(gv) * uv;
+                                const uint32_t hi = bf16_bits(h);
+                                const float hf = __uint_as_float(hi << 16);
+                                const uint32_t lo = bf16_bits(h - hf);
+                                uint16_t* hb = ws.hb_rt + (size_t)slot * 2 * I;
+                                hb[hrt_index(c, 0)] = (uint16_t)hi;
+                                hb[hrt_index(c, 1)] = (uint16_t)lo;
+                                float hs = hf + __uint_as_float(lo << 16);
 #pragma unroll
-                        for (int m = 1; m <= 8; m <<= 1) hs += __shfl_xor_sync(0xffffffffu, hs, m);
-                        if ((lane & 15) == 0) ws.hsum_rt[(int64_t)slot * (I / 16) + 2 * rb + (lane >> 4)] = hs;
+                                for (int m = 1; m <= 8; m <<= 1) hs += __shfl_xor_sync(0xffffffffu, hs, m);
+                                if ((lane & 15) == 0) ws.hsum_rt[(size_t)slot * (I / 16) + 2 * rb + (lane >> 4)] = hs;
+                            }
+                        }
+                        ok = cons_sync(P, cph, ws.err);
                     }
                 }
-                if (!cons_sync(P, cph, ws.err)) break;
+                if (!ok) break;
             }
             ++it;
         }
@@ -550,52 +791,22 @@ __global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------- down
-// sum_i (1 + q_i/4) h_i over the 16 codes of one 32-bit word, against NT slots.
-template <int NT>
-__device__ __forceinline__ void q2_word(uint32_t word, const float* const* hp, int ns, float* A) {
-    const uint32_t t0 = ((word << 5) & 0x60606060u) | 0x80808080u;
-    const uint32_t t1 = ((word << 3) & 0x60606060u) | 0x80808080u;
-    const uint32_t t2 = ((word << 1) & 0x60606060u) | 0x80808080u;
-    const uint32_t t3 = ((word >> 1) & 0x60606060u) | 0x80808080u;
-    // byte j of t_k holds code 4j + k at bits 5..6 (over a set bit 7); a byte
-    // permute puts it under exponent 0x3f8: the binary32 value 1 + code/4
-    float f[16];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint32_t sel = 0x7044u | (uint32_t)(j << 8);
-        f[4 * j + 0] = __uint_as_float(__byte_perm(t0, 0x3f000000u, sel));
-        f[4 * j + 1] = __uint_as_float(__byte_perm(t1, 0x3f000000u, sel));
-        f[4 * j + 2] = __uint_as_float(__byte_perm(t2, 0x3f000000u, sel));
-        f[4 * j + 3] = __uint_as_float(__byte_perm(t3, 0x3f000000u, sel));
-    }
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-        if (t < ns) {
-            float2 a = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-                const float4 hv = *reinterpret_cast<const float4*>(hp[t] + i);
-                a = ffma2(make_float2(f[i], f[i + 1]), make_float2(hv.x, hv.y), a);
-                a = ffma2(make_float2(f[i + 2], f[i + 3]), make_float2(hv.z, hv.w), a);
-            }
-            A[t] = a.x + a.y;
-        }
-    }
-}
-
 template <int NT>
 struct DownCfg {
     static constexpr int NS = 4;
-    static constexpr int CW = Warps<NT>::CW;
-    static constexpr int kRedFloats = CW * NT * 32;
+    static constexpr int CW = NT <= 2 ? 16 : 8;
+    static constexpr int TPB = NT == 1 ? 1 : 2;
+    static constexpr int kThreads = (CW + 1) * 32;
+    static constexpr int kRedFloats = CW * 4 * 32;   // [warp][4 tokens][32 rows]
 };
 
-// k steps (64 columns) per routed down chunk for an expert chosen by ns
-// slots: codes, scales, (d, dmin) and the slots' h (and per-16 sums of h)
-// for those columns must fit one stage.
+// k steps (64 columns) per routed down chunk for an entry of ns slots: codes,
+// scales, (d, dmin) and the slots' h pieces (and per-16 sums) for those
+// columns must fit one stage.
 __device__ __forceinline__ int down_chunk_ksteps(int nkt, int nsb, int ns) {
-    int ck = nkt < 32 ? nkt : 32;
-    for (; ck > 1; ck >>= 1) {
+    // the largest of 32, 16, 8, 4 that divides the k steps (I / 64: a multiple of 4 for I >= 256)
+    int ck = nkt % 32 == 0 ? 32 : nkt % 16 == 0 ? 16 : nkt % 8 == 0 ? 8 : nkt % 4 == 0 ? 4 : nkt;
+    for (; ck > 1 && ck % 2 == 0; ck >>= 1) {
         const int nsbc = nsb > 1 ? (ck + 3) / 4 : 1;
         if (ck * 640 + nsbc * 128 + ns * ck * 272 <= kStageBytes) break;
     }
@@ -603,29 +814,39 @@ __device__ __forceinline__ int down_chunk_ksteps(int nkt, int nsb, int ns) {
 }
 
 template <int NT>
-__global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
+struct DownAcc {
+    static constexpr int TG = (NT + 3) / 4;
+    float sh[TG][2][4];                        // shared task: [token group][tile][fragment]
+    float rt[DownCfg<NT>::TPB][2][2];          // routed task: [token][tile][row g, g + 8]
+};
+
+template <int NT>
+__global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
     k_down_decode(Weights W, Dims D, DecodeWs ws, float* out, int n) {
     using C = DownCfg<NT>;
-    constexpr int NS = C::NS, CW = C::CW;
+    constexpr int NS = C::NS, CW = C::CW, TPB = C::TPB;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char* stages = smem_raw;
     float* red = reinterpret_cast<float*>(smem_raw + NS * kStageBytes);   // kRedFloats
-    float* hsh = red + C::kRedFloats;                                     // [n][I]
+    unsigned char* zero = reinterpret_cast<unsigned char*>(red + C::kRedFloats);
     __shared__ Pipe P;
-    __shared__ Routing R;
+    __shared__ Routing Rt;
     __shared__ int s_last;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
     const int H = D.H, I = D.I, k = D.k;
     const int nkt = I / 64, nsb = I >= 256 ? I / 256 : 1;
-    const int n_sh = D.has_shared ? H / 8 : 0;
+    const int n_sh = ws.probe == 1 ? 0 : (D.has_shared ? H / 32 : 0);
     const int rb_per_e = H / 32;
-    const int ck_sh = I / 8 < 256 ? I / 8 : 256;
-    const int nch_sh = (I / 8) / ck_sh;
+    const int kcs = I < 256 ? I : 256;        // columns per shared chunk
+    const int nch_sh = I / kcs;
 
     pipe_init(P, NS, CW);
-    if (warp == CW) build_routing_warp(R, ws.ids, n * k);   // ids final: the router grid is complete
+    if (tid < 16) reinterpret_cast<uint32_t*>(zero)[tid] = 0u;
+    if (warp == CW)   // ids final: the router grid is complete
+        build_routing_warp(Rt, ws.ids, n, k, TPB, ws.probe == 1 ? 1 : (ws.probe == 2 ? 2 : 0), ws.probe_e);
     __syncthreads();
-    const int total = n_sh + R.nu * rb_per_e;
+    const int total = n_sh + Rt.nu * rb_per_e;
 
     if (warp == CW) {
         // ------------------------------------------------ producer warp
@@ -644,7 +865,7 @@ __global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
             if (!sh) {
                 u = (task - n_sh) / rb_per_e;
                 rb = (task - n_sh) % rb_per_e;
-                ns = R.ustart[u + 1] - R.ustart[u];
+                ns = Rt.ustart[u + 1] - Rt.ustart[u];
                 ck = down_chunk_ksteps(nkt, nsb, ns);
             }
             const int nch = sh ? nch_sh : nkt / ck;
@@ -655,13 +876,21 @@ __global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
                 if (lane == 0) {
                     unsigned char* st = stages + s * kStageBytes;
                     if (sh) {
-                        const int kc0 = c * ck_sh;
-                        const uint32_t bytes = ck_sh * 128;
-                        P.info[s] = ChunkInfo{task, c, nch, kc0, ck_sh};
-                        mbar_arrive_expect_tx(&P.full[s], bytes);
-                        bulk_load(st, W.sh_down + ((size_t)task * (I / 8) + kc0) * 64, bytes, &P.full[s], pol);
+                        // 32 rows of the shared down matrix (four 8-row groups of core-matrix tiles),
+                        // columns c*kcs .. +kcs, then every token's h pieces for those columns
+                        const int kc0 = c * kcs;
+                        const uint32_t abytes = kcs * 16, hbytes = kcs * 4;
+                        P.info[s] = ChunkInfo{task, c, nch, kc0, kcs};
+                        mbar_arrive_expect_tx(&P.full[s], 4 * abytes + n * hbytes);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            bulk_load(st + q * abytes, W.sh_down + ((size_t)(task * 4 + q) * (I / 8) + kc0 / 8) * 64,
+                                      abytes, &P.full[s], pol);
+                        for (int q = 0; q < n; ++q)
+                            bulk_load_plain(st + 4 * abytes + q * hbytes, ws.hb_sh + ((size_t)q * (I / 64) + kc0 / 64) * 128,
+                                            hbytes, &P.full[s]);
                     } else {
-                        const int e = R.uniq[u], s0 = R.ustart[u];
+                        const int e = Rt.uniq[u], s0 = Rt.ustart[u];
                         const int kt0 = c * ck;
                         const int sb0 = nsb > 1 ? kt0 / 4 : 0, nsbc = nsb > 1 ? (ck + 3) / 4 : 1;
                         const uint32_t qb = ck * 512, sb = ck * 128, dbb = nsbc * 128;
@@ -676,10 +905,11 @@ __global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
                                   W.down_dd + (size_t)e * W.q2_dd_stride + ((size_t)rb * nsb + sb0) * 32, dbb,
                                   &P.full[s], pol);
                         unsigned char* hdst = st + qb + sb + dbb;
-                        for (int t = 0; t < ns; ++t) {
-                            const int slot = R.slot[s0 + t];
-                            bulk_load_plain(hdst + t * hb, ws.h_rt + (size_t)slot * I + 64 * kt0, hb, &P.full[s]);
-                            bulk_load_plain(hdst + ns * hb + t * hsb, ws.hsum_rt + (size_t)slot * (I / 16) + 4 * kt0,
+                        for (int q = 0; q < ns; ++q) {
+                            const int slot = Rt.slot[s0 + q];
+                            bulk_load_plain(hdst + q * hb, ws.hb_rt + ((size_t)slot * (I / 64) + kt0) * 128, hb,
+                                            &P.full[s]);
+                            bulk_load_plain(hdst + ns * hb + q * hsb, ws.hsum_rt + (size_t)slot * (I / 16) + 4 * kt0,
                                             hsb, &P.full[s]);
                         }
                     }
@@ -691,111 +921,167 @@ __global__ void __launch_bounds__(Warps<NT>::kThreads, 1)
         producer_finish(P, it, NS, ws.err);
     } else {
         // ------------------------------------------------ consumer warps
-        griddep_wait();   // h from the gate/up grid
-        if (D.has_shared)
-            for (int i = tid * 4; i < n * I; i += CW * 32 * 4)
-                *reinterpret_cast<float4*>(hsh + i) = __ldcg(reinterpret_cast<const float4*>(ws.h_sh + i));
+        const uint32_t rot = (5u - 2u * (uint32_t)t) & 31u;   // code t of each byte to bits 5..6
+        const int jB = g >> 1, pB = g & 1;                    // routed B lanes: sub-block, piece
         uint32_t it = 0, cph = 0;
-        const bool staged = cons_sync(P, cph, ws.err);
-        float2 ay2[NT];
-        float acc[NT];
-        for (; staged;) {
+        DownAcc<NT> A;
+        int tcount = 0;
+        for (;;) {
             const int s = it % NS;
             if (!mbar_wait(&P.full[s], (it / NS) & 1, ws.err)) { set_abort(P); break; }
             const ChunkInfo inf = P.info[s];
             if (inf.task < 0 || aborted(P)) break;
             const unsigned char* st = stages + s * kStageBytes;
             const bool sh = inf.task < n_sh;
-            int rb, ns = 0, s0 = 0;
             if (sh) {
-                const int rr = lane & 7, kq = lane >> 3;
                 if (inf.chunk == 0) {
 #pragma unroll
-                    for (int t = 0; t < NT; ++t) ay2[t] = make_float2(0.f, 0.f);
-                }
-                const uint4* dt = reinterpret_cast<const uint4*>(st);
-                for (int kc = warp * 4 + kq; kc < inf.cnt; kc += 4 * CW) {
-                    const uint4 wd = dt[kc * 8 + rr];
-                    const int col = 8 * (inf.lo + kc);
+                    for (int tg = 0; tg < DownAcc<NT>::TG; ++tg)
 #pragma unroll
-                    for (int t = 0; t < NT; ++t)
-                        if (t < n) bf16x8_dot(wd, hsh + t * I + col, ay2[t]);
+                        for (int T = 0; T < 2; ++T) A.sh[tg][T][0] = A.sh[tg][T][1] = A.sh[tg][T][2] = A.sh[tg][T][3] = 0.f;
+                }
+                const int kc = inf.cnt;
+                const unsigned char* hst = st + 4 * kc * 16;
+                for (int ks = warp; ks < kc / 16; ks += CW) {
+                    uint2 B[DownAcc<NT>::TG];
+#pragma unroll
+                    for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) {
+                        const int tk = 4 * tg + (g >> 1), p = g & 1;
+                        B[tg] = *reinterpret_cast<const uint2*>(
+                            tk < n ? hst + (size_t)tk * kc * 4 + ((ks >> 2) * 2 + p) * 128 + ((ks & 3) * 16 + 4 * t) * 2
+                                   : zero);
+                    }
+#pragma unroll
+                    for (int T = 0; T < 2; ++T) {
+                        const unsigned char* base = st + (2 * T) * (kc * 16) + (2 * ks + (t >> 1)) * 128 + g * 16 + (t & 1) * 8;
+                        const uint2 r0 = *reinterpret_cast<const uint2*>(base);
+                        const uint2 r1 = *reinterpret_cast<const uint2*>(base + kc * 16);
+                        const uint32_t Af[4] = {r0.x, r1.x, r0.y, r1.y};
+#pragma unroll
+                        for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) bmma(A.sh[tg][T], Af, B[tg]);
+                    }
                 }
             } else {
                 const int tt = inf.task - n_sh, u = tt / rb_per_e;
-                rb = tt % rb_per_e;
-                s0 = R.ustart[u];
-                ns = R.ustart[u + 1] - s0;
+                const int s0 = Rt.ustart[u], ns = Rt.ustart[u + 1] - s0;
                 if (inf.chunk == 0) {
+                    tcount = ns;
 #pragma unroll
-                    for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+                    for (int q = 0; q < TPB; ++q)
+#pragma unroll
+                        for (int T = 0; T < 2; ++T) A.rt[q][T][0] = A.rt[q][T][1] = 0.f;
                 }
-                const int nsbc = nsb > 1 ? (inf.cnt + 3) / 4 : 1;
-                const uint4* qv = reinterpret_cast<const uint4*>(st);
-                const uint32_t* scv = reinterpret_cast<const uint32_t*>(st + inf.cnt * 512);
-                const uint32_t* ddv = reinterpret_cast<const uint32_t*>(st + inf.cnt * 640);
-                const float* hst = reinterpret_cast<const float*>(st + inf.cnt * 640 + nsbc * 128);
-                const float* hsst = hst + ns * inf.cnt * 64;
-                for (int kt = warp; kt < inf.cnt; kt += CW) {
-                    const uint4 q = qv[kt * 32 + lane];
-                    const uint32_t scw = scv[kt * 32 + lane];
-                    const uint32_t dd = ddv[(nsb > 1 ? (kt >> 2) : 0) * 32 + lane];
-                    const float d = half_bits(dd & 0xffffu), dmin = half_bits(dd >> 16);
-                    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+                const int ck = inf.cnt;
+                const int nsbc = nsb > 1 ? (ck + 3) / 4 : 1;
+                const unsigned char* qv = st;
+                const uint32_t* scv = reinterpret_cast<const uint32_t*>(st + ck * 512);
+                const uint32_t* ddv = reinterpret_cast<const uint32_t*>(st + ck * 640);
+                const uint16_t* hst = reinterpret_cast<const uint16_t*>(st + ck * 640 + nsbc * 128);
+                const float* hss = reinterpret_cast<const float*>(st + ck * 640 + nsbc * 128 + ns * ck * 256);
+                for (int kt = warp; kt < ck; kt += CW) {
+                    const int sbi = nsb > 1 ? ((inf.lo + kt) >> 2) - (inf.lo >> 2) : 0;   // superblock in the stage
+                    uint2 Bl[TPB];
+                    float S[TPB];
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const float* hp[NT];
-                        float S[NT];
-#pragma unroll
-                        for (int t = 0; t < NT; ++t) {
-                            hp[t] = hst + (t * inf.cnt + kt) * 64 + 16 * jj;
-                            S[t] = t < ns ? hsst[(t * inf.cnt + kt) * 4 + jj] : 0.f;
+                    for (int q = 0; q < TPB; ++q) {
+                        Bl[q] = make_uint2(0u, 0u);
+                        S[q] = 0.f;
+                        if (q < tcount) {
+                            Bl[q] = *reinterpret_cast<const uint2*>(hst + (size_t)q * ck * 128 + (kt * 2 + pB) * 64 + 16 * jB + 4 * t);
+                            S[q] = hss[q * ck * 4 + kt * 4 + t];
                         }
-                        float A[NT];
-                        q2_word<NT>(words[jj], hp, ns, A);
-                        const uint32_t sb = (scw >> (8 * jj)) & 0xffu;
-                        const float scf = __uint_as_float(0x4b000000u | (sb & 15u)) - 8388608.0f;
-                        const float mf = __uint_as_float(0x4b000000u | (sb >> 4)) - 8388608.0f;
-                        const float a4 = 4.0f * d * scf;
-                        const float bb = fmaf(dmin, mf, a4);
+                    }
 #pragma unroll
-                        for (int t = 0; t < NT; ++t)
-                            if (t < ns) acc[t] = fmaf(a4, A[t], fmaf(-bb, S[t], acc[t]));
+                    for (int T = 0; T < 2; ++T) {
+                        const int rg = 16 * T + g;
+                        const uint4 q0 = *reinterpret_cast<const uint4*>(qv + kt * 512 + rg * 16);
+                        const uint4 q1 = *reinterpret_cast<const uint4*>(qv + kt * 512 + (rg + 8) * 16);
+                        const uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w}, w1[4] = {q1.x, q1.y, q1.z, q1.w};
+                        uint32_t Af[4][4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t y0 = (__funnelshift_l(w0[j], w0[j], rot) & 0x60606060u) | 0x80808080u;
+                            const uint32_t y1 = (__funnelshift_l(w1[j], w1[j], rot) & 0x60606060u) | 0x80808080u;
+                            Af[j][0] = __byte_perm(y0, 0x3f3f3f3fu, 0x5140);
+                            Af[j][1] = __byte_perm(y1, 0x3f3f3f3fu, 0x5140);
+                            Af[j][2] = __byte_perm(y0, 0x3f3f3f3fu, 0x7362);
+                            Af[j][3] = __byte_perm(y1, 0x3f3f3f3fu, 0x7362);
+                        }
+                        // this lane's sub-block t: a4 = 4 d sc, mm = dmin m, per row
+                        const uint32_t sw0 = scv[kt * 32 + rg], sw1 = scv[kt * 32 + rg + 8];
+                        const uint32_t dd0 = ddv[sbi * 32 + rg], dd1 = ddv[sbi * 32 + rg + 8];
+                        const float d0 = half_bits(dd0 & 0xffffu), m0 = half_bits(dd0 >> 16);
+                        const float d1 = half_bits(dd1 & 0xffffu), m1 = half_bits(dd1 >> 16);
+                        const uint32_t b0 = sw0 >> (8 * t), b1 = sw1 >> (8 * t);
+                        const float a40 = fmaf(__uint_as_float(0x4b000000u | (b0 & 15u)), 4.f * d0, -33554432.f * d0);
+                        const float a41 = fmaf(__uint_as_float(0x4b000000u | (b1 & 15u)), 4.f * d1, -33554432.f * d1);
+                        const float mm0 = fmaf(__uint_as_float(0x4b000000u | ((b0 >> 4) & 15u)), m0, -8388608.f * m0);
+                        const float mm1 = fmaf(__uint_as_float(0x4b000000u | ((b1 >> 4) & 15u)), m1, -8388608.f * m1);
+#pragma unroll
+                        for (int q = 0; q < TPB; ++q) {
+                            if (q < tcount) {
+                                float Dv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) bmma(Dv, Af[j], jB == j ? Bl[q] : make_uint2(0u, 0u));
+                                A.rt[q][T][0] = fmaf(a40, (Dv[0] + Dv[1]) - S[q], A.rt[q][T][0]);
+                                A.rt[q][T][0] = fmaf(-mm0, S[q], A.rt[q][T][0]);
+                                A.rt[q][T][1] = fmaf(a41, (Dv[2] + Dv[3]) - S[q], A.rt[q][T][1]);
+                                A.rt[q][T][1] = fmaf(-mm1, S[q], A.rt[q][T][1]);
+                            }
+                        }
                     }
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&P.empty[s]);
             if (inf.chunk == inf.nchunk - 1) {
-                // task epilogue: reduce, store y, count the task in its 32-row block
+                // task epilogue: reduce the warps' partials, store y
+                bool ok = true;
                 if (sh) {
-                    const int rr = lane & 7, kq = lane >> 3;
 #pragma unroll
-                    for (int t = 0; t < NT; ++t) {
-                        float y = ay2[t].x + ay2[t].y;
-                        y += __shfl_xor_sync(0xffffffffu, y, 8);
-                        y += __shfl_xor_sync(0xffffffffu, y, 16);
-                        if (kq == 0 && t < n) red[(warp * NT + t) * 32 + rr] = y;
-                    }
-                    if (!cons_sync(P, cph, ws.err)) break;
-                    if (tid < 8 * n) {
-                        const int r = tid & 7, t = tid >> 3;
-                        float y = 0.f;
-                        for (int w = 0; w < CW; ++w) y += red[(w * NT + t) * 32 + r];
-                        ws.y_sh[(int64_t)t * H + 8 * inf.task + r] = y;
+                    for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) {
+#pragma unroll
+                        for (int T = 0; T < 2; ++T) {
+                            red[(warp * 4 + t) * 32 + 16 * T + g] = A.sh[tg][T][0] + A.sh[tg][T][1];
+                            red[(warp * 4 + t) * 32 + 16 * T + g + 8] = A.sh[tg][T][2] + A.sh[tg][T][3];
+                        }
+                        if (!(ok = cons_sync(P, cph, ws.err))) break;
+                        if (tid < 128) {
+                            const int tl = tid >> 5, row = tid & 31, tok = 4 * tg + tl;
+                            float y = 0.f;
+                            for (int w = 0; w < CW; ++w) y += red[(w * 4 + tl) * 32 + row];
+                            if (tok < n) (ws.probe ? ws.probe_out : ws.y_sh)[(size_t)tok * H + 32 * inf.task + row] = y;
+                        }
+                        if (!(ok = cons_sync(P, cph, ws.err))) break;
                     }
                 } else {
+                    const int tt = inf.task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
+                    const int s0 = Rt.ustart[u];
 #pragma unroll
-                    for (int t = 0; t < NT; ++t)
-                        if (t < ns) red[(warp * NT + t) * 32 + lane] = acc[t];
-                    if (!cons_sync(P, cph, ws.err)) break;
-                    if (warp < ns) {
-                        float y = 0.f;
-                        for (int w = 0; w < CW; ++w) y += red[(w * NT + warp) * 32 + lane];
-                        ws.y_rt[(int64_t)R.slot[s0 + warp] * H + 32 * rb + lane] = y;
+                    for (int q = 0; q < TPB; ++q) {
+#pragma unroll
+                        for (int T = 0; T < 2; ++T) {
+#pragma unroll
+                            for (int r = 0; r < 2; ++r) {
+                                float v = A.rt[q][T][r];
+                                v += __shfl_xor_sync(0xffffffffu, v, 1);
+                                v += __shfl_xor_sync(0xffffffffu, v, 2);
+                                if (t == 0) red[(warp * 4 + q) * 32 + 16 * T + g + 8 * r] = v;
+                            }
+                        }
+                    }
+                    if ((ok = cons_sync(P, cph, ws.err))) {
+                        if (warp < tcount) {
+                            float y = 0.f;
+                            for (int w = 0; w < CW; ++w) y += red[(w * 4 + warp) * 32 + lane];
+                            const int slot = Rt.slot[s0 + warp];
+                            if (ws.probe) ws.probe_out[(size_t)(slot / k) * H + 32 * rb + lane] = y;
+                            else ws.y_rt[(size_t)slot * H + 32 * rb + lane] = y;
+                        }
+                        ok = cons_sync(P, cph, ws.err);
                     }
                 }
-                if (!cons_sync(P, cph, ws.err)) break;
+                if (!ok) break;
             }
             ++it;
         }
@@ -820,6 +1106,7 @@ __global__ void __launch_bounds__(256) k_combine_decode(Dims D, DecodeWs ws, flo
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int H = D.H, k = D.k;
     if (i >= (int64_t)n * H) return;
+    if (__ldcg(ws.grid_refused)) return;   // the gate/up grid refused the grid: out stays as it was
     const int t = (int)(i / H), r = (int)(i % H);
     float w[16], y[16];
 #pragma unroll
@@ -847,6 +1134,7 @@ __global__ void __launch_bounds__(kSteerThreads) k_combine_steer_decode(Dims D, 
     griddep_wait();   // y of the down grid
     __shared__ float red[kSteerThreads / 32];
     const int t = blockIdx.x, H = D.H, k = D.k;
+    if (__ldcg(ws.grid_refused)) return;   // the gate/up grid refused the grid: out stays as it was
     float acc[kSteerCols];
     float dot = 0.f;
 #pragma unroll
@@ -894,16 +1182,20 @@ cudaError_t launch_wait_selftest(uint32_t* err, cudaStream_t st) {
 template <int NT>
 size_t gateup_smem_bytes(const Dims& D, int n) {
     using C = GateUpCfg<NT>;
-    return (size_t)C::NS * kStageBytes + sizeof(float) * ((size_t)C::kTabFloats + C::kRedFloats + (size_t)n * D.H);
+    return (size_t)C::NS * kStageBytes + 4 * ((size_t)C::kTabWords + C::kRedFloats) + (size_t)n * D.H * 4 + 64;
 }
 
 template <int NT>
 size_t down_smem_bytes(const Dims& D, int n) {
     using C = DownCfg<NT>;
-    return (size_t)C::NS * kStageBytes + sizeof(float) * ((size_t)C::kRedFloats + (size_t)n * D.I);
+    (void)D;
+    (void)n;
+    return (size_t)C::NS * kStageBytes + 4 * (size_t)C::kRedFloats + 64;
 }
 
-size_t router_smem_bytes(const Dims& D, int n) { return sizeof(float) * (size_t)n * D.H; }
+size_t router_smem_bytes(const Dims& D, int n) {
+    return (size_t)kRE * D.H * 4 + (size_t)n * D.H * (D.act_bf16 ? 2 : 4);
+}
 
 // Events (optional): ev[2i] / ev[2i+1] recorded around launch i.  Under
 // stream capture they become external event-record nodes, so that replays
@@ -979,16 +1271,16 @@ cudaError_t launch_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws,
     if ((err = configure(k_router_decode<NT>)) != cudaSuccess) return err;
     Marks mk(ev, st);
     const bool pdl = ev == nullptr;   // profiled runs keep the kernels apart
-    const int rgrid = (D.E + kRWarps - 1) / kRWarps;
+    const int rgrid = (D.E + kRE - 1) / kRE;
     mk.before();
-    k_router_decode<NT><<<rgrid, kRWarps * 32, router_smem_bytes(D, n), st>>>(W, D, ws, x, n);
+    k_router_decode<NT><<<rgrid, kRE * 32, router_smem_bytes(D, n), st>>>(W, D, ws, x, n);
     mk.after();
     mk.before();
-    err = launch_pdl(k_gateup_decode<NT>, dim3(n_sm), dim3(Warps<NT>::kThreads), s1, st, pdl, W, D, ws, x, n);
+    err = launch_pdl(k_gateup_decode<NT>, dim3(n_sm), dim3(GateUpCfg<NT>::kThreads), s1, st, pdl, W, D, ws, x, n);
     mk.after();
     if (err != cudaSuccess) return err;
     mk.before();
-    err = launch_pdl(k_down_decode<NT>, dim3(n_sm), dim3(Warps<NT>::kThreads), s2, st, pdl, W, D, ws, out, n);
+    err = launch_pdl(k_down_decode<NT>, dim3(n_sm), dim3(DownCfg<NT>::kThreads), s2, st, pdl, W, D, ws, out, n);
     mk.after();
     if (err != cudaSuccess) return err;
     const int64_t nel = (int64_t)n * D.H;
@@ -1013,7 +1305,9 @@ size_t decode_smem_bytes(const Dims& D, int n) {
     else if (n <= 2) { a = gateup_smem_bytes<2>(D, n); b = down_smem_bytes<2>(D, n); }
     else if (n <= 4) { a = gateup_smem_bytes<4>(D, n); b = down_smem_bytes<4>(D, n); }
     else { a = gateup_smem_bytes<8>(D, n); b = down_smem_bytes<8>(D, n); }
-    return (a > b ? a : b) + sizeof(Pipe) + sizeof(Routing) + 64;
+    size_t need = (a > b ? a : b) + sizeof(Pipe) + sizeof(Routing) + 512;   // + the kernels' other static shared memory
+    const size_t r = router_smem_bytes(D, n) + sizeof(float) * kRE * 1024 + 64;
+    return r > need ? r : need;
 }
 
 cudaError_t launch_decode(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n, float* out,
@@ -1024,13 +1318,69 @@ cudaError_t launch_decode(const Weights& W, const Dims& D, const DecodeWs& ws, c
     return launch_decode_t<8>(W, D, ws, x, n, out, n_sm, st, ev);
 }
 
+// Probe of the down kernel: caller h [n][I] binary32 -> the workspace's h pieces (routed layout at slots
+// t * k, or the shared layout) and, for the routed layout, the per-16 sums of the pieces.
+__global__ void k_probe_h(const float* h, int n, int I, int k, int shared, uint16_t* hb_rt, float* hsum_rt,
+                          uint16_t* hb_sh) {
+    const int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // one 16-column block
+    if (q >= (int64_t)n * (I / 16)) return;
+    const int tk = (int)(q / (I / 16)), b = (int)(q % (I / 16));
+    float s = 0.f;
+    for (int j = 0; j < 16; ++j) {
+        const int c = 16 * b + j;
+        const float v = h[(int64_t)tk * I + c];
+        const uint32_t hi = bf16_bits(v);
+        const float hf = __uint_as_float(hi << 16);
+        const uint32_t lo = bf16_bits(v - hf);
+        if (shared) {
+            uint16_t* d = hb_sh + (size_t)tk * 2 * I;
+            d[hsh_index(c, 0)] = (uint16_t)hi;
+            d[hsh_index(c, 1)] = (uint16_t)lo;
+        } else {
+            uint16_t* d = hb_rt + (size_t)tk * k * 2 * I;
+            d[hrt_index(c, 0)] = (uint16_t)hi;
+            d[hrt_index(c, 1)] = (uint16_t)lo;
+            s += hf + __uint_as_float(lo << 16);
+        }
+    }
+    if (!shared) hsum_rt[(size_t)tk * k * (I / 16) + b] = s;
+}
+
+template <int NT>
+cudaError_t launch_probe_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws, int which, const void* in,
+                                  int n, int n_sm, cudaStream_t st) {
+    cudaError_t err;
+    if (which == 0) {
+        if ((err = configure(k_gateup_decode<NT>)) != cudaSuccess) return err;
+        k_gateup_decode<NT><<<n_sm, GateUpCfg<NT>::kThreads, gateup_smem_bytes<NT>(D, n), st>>>(W, D, ws, in, n);
+        return cudaGetLastError();
+    }
+    const int64_t nb = (int64_t)n * (D.I / 16);
+    k_probe_h<<<(unsigned)((nb + 127) / 128), 128, 0, st>>>(reinterpret_cast<const float*>(in), n, D.I, D.k,
+                                                            ws.probe == 2, ws.hb_rt, ws.hsum_rt, ws.hb_sh);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if ((err = configure(k_down_decode<NT>)) != cudaSuccess) return err;
+    k_down_decode<NT><<<n_sm, DownCfg<NT>::kThreads, down_smem_bytes<NT>(D, n), st>>>(W, D, ws, nullptr, n);
+    return cudaGetLastError();
+}
+
+// Inspection: the decode plan's projection kernels with every token routed to
+// one expert (ws.probe set by the caller), raw accumulators to ws.probe_out.
+cudaError_t launch_probe_decode(const Weights& W, const Dims& D, const DecodeWs& ws, int which, const void* in, int n,
+                                int n_sm, cudaStream_t st) {
+    if (n <= 1) return launch_probe_decode_t<1>(W, D, ws, which, in, n, n_sm, st);
+    if (n <= 2) return launch_probe_decode_t<2>(W, D, ws, which, in, n, n_sm, st);
+    if (n <= 4) return launch_probe_decode_t<4>(W, D, ws, which, in, n, n_sm, st);
+    return launch_probe_decode_t<8>(W, D, ws, which, in, n, n_sm, st);
+}
+
 template <int NT>
 cudaError_t launch_route_t(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n,
                            cudaStream_t st) {
     cudaError_t err;
     const size_t s0 = router_smem_bytes(D, n);
     if ((err = configure(k_router_decode<NT>)) != cudaSuccess) return err;
-    k_router_decode<NT><<<(D.E + kRWarps - 1) / kRWarps, kRWarps * 32, s0, st>>>(W, D, ws, x, n);
+    k_router_decode<NT><<<(D.E + kRE - 1) / kRE, kRE * 32, s0, st>>>(W, D, ws, x, n);
     return cudaGetLastError();
 }
 

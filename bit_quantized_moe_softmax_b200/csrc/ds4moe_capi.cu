@@ -35,6 +35,9 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
 cudaError_t launch_route_prefill(const Weights& W, const Dims& D, const PrefillWs& ws, const void* x, int n,
                                  cudaStream_t st);
 cudaError_t launch_wait_selftest(uint32_t* err, cudaStream_t st);
+cudaError_t launch_permutation(const Dims& D, const PrefillWs& ws, const int32_t* ids, int n, cudaStream_t st);
+cudaError_t launch_probe_decode(const Weights& W, const Dims& D, const DecodeWs& ws, int which, const void* in, int n,
+                                int n_sm, cudaStream_t st);
 cudaError_t launch_probe_gemm(const Weights& W, const Dims& D, const PrefillWs& ws, int which, int e,
                               const void* in, int n, float* out, int n_sm, cudaStream_t st);
 int prefill_launches(const Dims& D);
@@ -83,7 +86,7 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
 struct WsLayout {
-    size_t hdr, rbtick, logits, ids, wts, h_rt, hsum_rt, h_sh, y_rt, y_sh, x_stage, out_stage;
+    size_t hdr, logits, ids, wts, hb_rt, hsum_rt, hb_sh, y_rt, y_sh, x_stage, out_stage;
     size_t x_slot, out_slot;   // bytes of one of the two staging slots of the host-buffer calls
     // prefill plan (capacity > decode_max only)
     size_t p_logits, p_ids, p_wts, p_blk_cnt, p_blk_off, p_counts, p_offs, p_mtp, p_pos, p_slot, p_xb, p_Xp, p_Hb,
@@ -149,13 +152,12 @@ struct ds4moe {
         const size_t nd = (size_t)(cap < decode_max ? cap : decode_max);
         size_t o = 0;
         w.hdr = o; o += 256;
-        w.rbtick = o; o += align256(H / 32 * 4);
         w.logits = o; o += align256(nd * E * 4);
         w.ids = o; o += align256(nd * k * 4);
         w.wts = o; o += align256(nd * k * 4);
-        w.h_rt = o; o += align256(nd * k * I * 4);
+        w.hb_rt = o; o += align256(nd * k * I * 2 * 2);   // two bf16 pieces
         w.hsum_rt = o; o += align256(nd * k * (I / 16) * 4);
-        w.h_sh = o; o += align256(nd * I * 4);
+        w.hb_sh = o; o += align256(nd * I * 2 * 2);
         w.y_rt = o; o += align256(nd * k * H * 4);
         w.y_sh = o; o += align256(nd * H * 4);
         w.x_slot = align256((size_t)cap * H * (D.act_bf16 ? 2 : 4));
@@ -219,13 +221,13 @@ struct ds4moe {
         w.queue2 = hdr + 3;
         w.done1 = hdr + 4;
         w.done2 = hdr + 5;
-        w.rbtick = reinterpret_cast<uint32_t*>(ws + L.rbtick);
+        w.grid_refused = hdr + 6;
         w.logits = reinterpret_cast<float*>(ws + L.logits);
         w.ids = reinterpret_cast<int32_t*>(ws + L.ids);
         w.wts = reinterpret_cast<float*>(ws + L.wts);
-        w.h_rt = reinterpret_cast<float*>(ws + L.h_rt);
+        w.hb_rt = reinterpret_cast<uint16_t*>(ws + L.hb_rt);
         w.hsum_rt = reinterpret_cast<float*>(ws + L.hsum_rt);
-        w.h_sh = reinterpret_cast<float*>(ws + L.h_sh);
+        w.hb_sh = reinterpret_cast<uint16_t*>(ws + L.hb_sh);
         w.y_rt = reinterpret_cast<float*>(ws + L.y_rt);
         w.y_sh = reinterpret_cast<float*>(ws + L.y_sh);
         return w;
@@ -651,7 +653,7 @@ ds4moe_status ds4moe_route(ds4moe_t* h, const void* d_x, int32_t n, int32_t* d_i
 ds4moe_status ds4moe_probe(ds4moe_t* h, int32_t plan, int32_t which, int32_t e, const void* d_in, int32_t n,
                            float* d_out, void* stream) {
     if (!h) return fail(DS4MOE_ERR_ARG, "probe: NULL handle");
-    if (plan != 1) return fail(DS4MOE_ERR_ARG, "probe: plan %d (1 = prefill)", plan);
+    if (plan != 0 && plan != 1) return fail(DS4MOE_ERR_ARG, "probe: plan %d (0 decode, 1 prefill)", plan);
     if (which != 0 && which != 2) return fail(DS4MOE_ERR_ARG, "probe: which %d (0 gate/up, 2 down)", which);
     if (n < 1 || n > (1 << 20)) return fail(DS4MOE_ERR_ARG, "probe: n_rows %d outside 1..2^20", n);
     if (!d_in || !d_out) return fail(DS4MOE_ERR_ARG, "probe: NULL buffer");
@@ -660,6 +662,15 @@ ds4moe_status ds4moe_probe(ds4moe_t* h, int32_t plan, int32_t which, int32_t e, 
     if (!h->ready(&why)) return fail(DS4MOE_ERR_NOT_READY, "probe: %s", why.c_str());
     if (e < -1 || e >= h->D.E) return fail(DS4MOE_ERR_ARG, "probe: expert %d out of range", e);
     if (e == -1 && !h->shape.has_shared) return fail(DS4MOE_ERR_ARG, "probe: the layer has no shared expert");
+    if (plan == 0) {
+        if (n > h->decode_max) return fail(DS4MOE_ERR_ARG, "probe: n_rows %d > decode_max %d", n, h->decode_max);
+        DecodeWs ws = h->decode_ws();
+        ws.probe = e >= 0 ? 1 : 2;
+        ws.probe_e = e;
+        ws.probe_out = d_out;
+        cudaError_t ce = launch_probe_decode(h->weights_view(), h->D, ws, which, d_in, n, h->n_sm, (cudaStream_t)stream);
+        return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "probe launch");
+    }
     if (h->shape.max_tokens <= h->decode_max)
         return fail(DS4MOE_ERR_NOT_READY, "probe: the prefill plan needs max_tokens > decode_max");
     cudaError_t ce = launch_probe_gemm(h->weights_view(), h->D, h->prefill_ws(), which, e, d_in, n, d_out, h->n_sm,
@@ -759,6 +770,25 @@ ds4moe_status ds4moe_route_noalloc(ds4moe_t* h, const void* d_x, int32_t n, int3
     ws.wts = d_w;
     ce = launch_route(h->weights_view(), h->D, ws, d_x, n, st);
     return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "route_noalloc launch");
+}
+
+ds4moe_status ds4moe_permutation(ds4moe_t* h, const int32_t* d_ids, int32_t n, int32_t* d_counts,
+                                 int32_t* d_offsets, int32_t* d_pos_of_slot, void* stream) {
+    if (!h) return fail(DS4MOE_ERR_ARG, "permutation: NULL handle");
+    if (!d_ids || !d_counts || !d_offsets || !d_pos_of_slot) return fail(DS4MOE_ERR_ARG, "permutation: NULL buffer");
+    if (!h->ws) return fail(DS4MOE_ERR_NOT_READY, "permutation: workspace not bound");
+    if (h->shape.max_tokens <= h->decode_max)
+        return fail(DS4MOE_ERR_NOT_READY, "permutation: the prefill plan needs max_tokens > decode_max");
+    if (n < 1 || n > h->shape.max_tokens)
+        return fail(DS4MOE_ERR_ARG, "permutation: n_tokens %d outside 1..%d", n, h->shape.max_tokens);
+    cudaStream_t st = (cudaStream_t)stream;
+    PrefillWs ws = h->prefill_ws();
+    cudaError_t ce = launch_permutation(h->D, ws, d_ids, n, st);
+    const size_t E = h->D.E, nk = (size_t)n * h->D.k;
+    if (ce == cudaSuccess) ce = cudaMemcpyAsync(d_counts, ws.counts, E * 4, cudaMemcpyDeviceToDevice, st);
+    if (ce == cudaSuccess) ce = cudaMemcpyAsync(d_offsets, ws.offs, (E + 1) * 4, cudaMemcpyDeviceToDevice, st);
+    if (ce == cudaSuccess) ce = cudaMemcpyAsync(d_pos_of_slot, ws.pos_of_slot, nk * 4, cudaMemcpyDeviceToDevice, st);
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "permutation");
 }
 
 ds4moe_status ds4moe_selftest_wait(ds4moe_t* h, void* stream) {

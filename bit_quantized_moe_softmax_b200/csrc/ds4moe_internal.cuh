@@ -65,18 +65,22 @@ struct DecodeWs {
     uint32_t* queue2;       // down task counter
     uint32_t* done1;        // gate/up CTAs finished (the last one resets queue1)
     uint32_t* done2;        // down CTAs finished (the last one resets queue2)
-    uint32_t* rbtick;       // [H/32] tasks finished per 32-row block of the output
+    uint32_t* grid_refused; // this call's gate/up grid refused the grid (too many or too large magnitudes): 1, else 0
     float* logits;          // [n][E]
     int32_t* ids;           // [n][k]
     float* wts;             // [n][k]
-    float* h_rt;            // [n*k][I]
-    float* hsum_rt;         // [n*k][I/16]
-    float* h_sh;            // [n][I]
+    uint16_t* hb_rt;        // [n*k][I/64][2][64] bf16: h of each routed slot as two pieces (hi, lo = h - hi);
+                            //   inside each 16-column block position 4c + e holds column c + 4e
+    float* hsum_rt;         // [n*k][I/16]: per 16-column block, the sum of hi + lo
+    uint16_t* hb_sh;        // [n][I/64][2][64] bf16: h of the shared expert as two pieces, natural order
     float* y_rt;            // [n*k][H]
     float* y_sh;            // [n][H]
     const void* xres;       // x again when the call adds the residual (out = x + layer(x)), else nullptr
     const float* steer_v;   // [H] steering direction, or nullptr (no steering)
     float steer_F;          // steering strength: y -= F v (v . y)
+    int probe;              // 0: forward; 1: every token to routed expert probe_e; 2: the shared expert alone
+    int probe_e;
+    float* probe_out;       // probe: raw accumulators (gate/up: [n][2I]; down: [n][H])
 };
 
 // Workspace pointers (prefill plan).

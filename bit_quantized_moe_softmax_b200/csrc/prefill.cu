@@ -1105,6 +1105,22 @@ cudaError_t launch_probe_gemm(const Weights& W, const Dims& D, const PrefillWs& 
     return launch_gemm<kModeShDown>(mA, mB0, mB0, ga, n_sm, st);
 }
 
+// Inspection: the permutation of the prefill plan (histogram, scan, stable
+// scatter) on caller ids [n][k], results in the workspace.
+cudaError_t launch_permutation(const Dims& D, const PrefillWs& ws, const int32_t* ids, int n, cudaStream_t st) {
+    cudaError_t e;
+    const int E = D.E, nslots = n * D.k;
+    const int nblk = (nslots + kSortBlock - 1) / kSortBlock;
+    k_hist<<<nblk, kSortBlock, E * sizeof(int), st>>>(ids, nslots, E, ws.blk_cnt);
+    k_scan<<<1, 1024, 0, st>>>(ws.blk_cnt, nblk, E, ws.counts, ws.offs, ws.blk_off, ws.mt_prefix);
+    if (32 * E * sizeof(int) > 48 * 1024 &&
+        (e = smem_opt_in(reinterpret_cast<const void*>(k_scatter), 32 * E * (int)sizeof(int))) != cudaSuccess)
+        return e;
+    k_scatter<<<nblk, kSortBlock, 32 * E * sizeof(int), st>>>(ids, nslots, E, ws.blk_off, ws.pos_of_slot,
+                                                               ws.slot_of_pos);
+    return cudaGetLastError();
+}
+
 // Routing only (prefill sizes): logits and top-k.
 cudaError_t launch_route_prefill(const Weights& W, const Dims& D, const PrefillWs& ws, const void* x, int n,
                                  cudaStream_t st) {

@@ -243,14 +243,30 @@ ds4moe_status ds4moe_dequant(ds4moe_t* h, int32_t e, int32_t which, int32_t as_b
  * out as they are: the inspection the bit-exactness of the weights the
  * kernels multiply rests on (one-hot rows give back columns of the weight
  * matrices exactly as the tensor cores consumed them).
+ *   plan 0 (the decode plan; n <= decode_max): the persistent gate/up and
+ *     down kernels.  which 0: d_in = activations [n][H] binary32 (or bf16
+ *     when act_dtype is DS4MOE_ACT_BF16), d_out = [n][2I] binary32, gate
+ *     results then up results (no SwiGLU); which 2: d_in = h [n][I]
+ *     binary32 (entering as the kernel's two bf16 pieces), d_out = [n][H].
  *   plan 1 (the prefill plan; needs max_tokens > decode_max): the tcgen05
  *     grouped GEMM.  which 0: d_in = activations [n][H] bfloat16, d_out =
  *     [n][2I] binary32, gate accumulators then up accumulators (no SwiGLU);
  *     which 2: d_in = h [n][I] bfloat16, d_out = [n][H] binary32.
- * d_in and d_out are 16-byte aligned device buffers; n in 1..2^20.  Uses
- * the prefill region of the workspace (its routing plan is overwritten). */
+ * d_in and d_out are 16-byte aligned device buffers; n in 1..2^20 (plan 1).
+ * Uses the workspace of the plan (its routing and intermediates are
+ * overwritten). */
 ds4moe_status ds4moe_probe(ds4moe_t* h, int32_t plan, int32_t which, int32_t e, const void* d_in, int32_t n_rows,
                            float* d_out, void* stream);
+
+/* The prefill plan's permutation of (token, slot) pairs by expert, on caller
+ * ids [n][k] (int32, each in 0..E-1): d_counts [E] slots per expert,
+ * d_offsets [E+1] exclusive prefix of the counts, d_pos_of_slot [n*k] the
+ * position of slot t*k + j in the permuted order -- a stable counting sort
+ * (slots of one expert keep their slot order).  The same kernels the prefill
+ * forward runs; needs max_tokens > decode_max and 1 <= n <= max_tokens.
+ * Ids outside 0..E-1 are the caller's error (not checked on the device). */
+ds4moe_status ds4moe_permutation(ds4moe_t* h, const int32_t* d_ids, int32_t n_tokens, int32_t* d_counts,
+                                 int32_t* d_offsets, int32_t* d_pos_of_slot, void* stream);
 
 /* ---- routing without device allocation ------------------------------------ */
 

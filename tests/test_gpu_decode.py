@@ -204,16 +204,37 @@ def test_forward_host_async_pipeline(orc, n, max_tokens):
     m.ds4moe_host_sync(lay.h)   # nothing pending: returns at once
 
 
-def test_forward_full_decode_shape(orc):
-    """One token through a full-size layer (H 4096, I 2048, 256 experts top-8, bf16 shared)."""
+@pytest.mark.parametrize("n", [1, 2, 4, 8])
+def test_forward_full_decode_shape(orc, n):
+    """n tokens through a full-size layer (H 4096, I 2048, 256 experts top-8, bf16 shared), in the
+    launch configuration the bench times: n = 1 is the decode step, 2 / 4 / 8 the MTP-verify sizes
+    (8 tokens: about 57 distinct experts, some chosen by two tokens)."""
     L = synth.packed_layer(synth.FULL, 0, device="cuda")
     lay = _layer_on_gpu(L, max_tokens=8)
-    x = synth.tokens(2, 4096, seed=1)
+    x = synth.tokens(n, 4096, seed=1 + n)
     out = lay.forward(x.cuda()).cpu().numpy()
+    ids_gpu, _ = lay.route(x.cuda())
     lg = orc.router_logits(x.numpy(), L["W_r"].cpu().numpy())
     rid, _ = orc.topk_softmax(lg, 8)
+    assert np.array_equal(ids_gpu.cpu().numpy(), rid)
     ref, ids, _ = orc.moe_forward(oracle_layer(L, experts=rid.ravel()), x.numpy())
     assert np.array_equal(ids, rid)
+    assert rel_err(out, ref) < TOL
+
+
+def test_forward_full_shape_expert_of_every_token(orc):
+    """Eight tokens that all choose expert 17 (router bias): one expert serves more tokens than one
+    routed entry holds, so its weights are read by several entries; bf16 activations."""
+    bias = torch.zeros(256)
+    bias[17] = 30.0
+    L = synth.packed_layer(synth.FULL, 4, bias=bias, device="cuda")
+    lay = _layer_on_gpu(L, max_tokens=8, act=m.DS4MOE_ACT_BF16)
+    x = synth.tokens(8, 4096, seed=9, dtype=torch.bfloat16)
+    out = lay.forward(x.cuda()).cpu().numpy()
+    lg = orc.router_logits(x.float().numpy(), L["W_r"].cpu().numpy(), bias.numpy())
+    rid, _ = orc.topk_softmax(lg, 8)
+    assert np.all(rid[:, 0] == 17)
+    ref, ids, _ = orc.moe_forward(oracle_layer(L, experts=rid.ravel()), x.float().numpy())
     assert rel_err(out, ref) < TOL
 
 

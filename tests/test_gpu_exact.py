@@ -29,19 +29,25 @@ def _cuda():
     build.build()
 
 
-def _load(L, max_tokens):
-    lay = m.MoELayer(L["H"], L["I"], L["E"], L["k"], max_tokens, act_dtype=m.DS4MOE_ACT_BF16,
+def _load(L, max_tokens, act=m.DS4MOE_ACT_F32):
+    lay = m.MoELayer(L["H"], L["I"], L["E"], L["k"], max_tokens, act_dtype=act,
                      has_shared=L.get("sh_gate") is not None, has_bias=L.get("b_r") is not None)
     lay.load(L)
     return lay
 
 
 def _probe_columns(lay, plan, which, e):
-    """[K][rows]: column c of the probed matrices (gate rows then up rows for which 0)."""
+    """[K][rows]: column c of the probed matrices (gate rows then up rows for which 0).
+
+    The decode plan (plan 0) takes at most decode_max rows per call: the
+    one-hot rows go through it eight at a time."""
     K = lay.H if which == 0 else lay.I
-    eye = torch.eye(K, device="cuda", dtype=torch.bfloat16 if plan == 1 else torch.float32)
+    in_dtype = torch.bfloat16 if (plan == 1 or (which == 0 and lay.act_dtype == m.DS4MOE_ACT_BF16)) else torch.float32
+    eye = torch.eye(K, device="cuda", dtype=in_dtype)
     out = torch.empty(K, 2 * lay.I if which == 0 else lay.H, dtype=torch.float32, device="cuda")
-    m.ds4moe_probe(lay.h, plan, which, e, eye, out)
+    step = K if plan == 1 else 8
+    for r0 in range(0, K, step):
+        m.ds4moe_probe(lay.h, plan, which, e, eye[r0:r0 + step], out[r0:r0 + step])
     torch.cuda.synchronize()
     assert m.ds4moe_get_device_error(lay.h) == 0
     return out.cpu().numpy()
@@ -71,7 +77,7 @@ def _same_bits(a, b):
         bad.size, np.unravel_index(bad[0], a.shape), a.flat[bad[0]], b.flat[bad[0]])
 
 
-@pytest.mark.parametrize("plan", [1])
+@pytest.mark.parametrize("plan", [0, 1])
 def test_probe_tiny_bit_exact(orc, plan):
     L = synth.float_layer(synth.TINY, 0)
     L.update(pack_with_oracle(orc, L))
@@ -81,7 +87,7 @@ def test_probe_tiny_bit_exact(orc, plan):
             _same_bits(_probe_columns(lay, plan, which, e), _ref_columns(orc, L, which, e, bf16=plan == 1))
 
 
-@pytest.mark.parametrize("plan", [1])
+@pytest.mark.parametrize("plan", [0, 1])
 def test_probe_full_shape_bit_exact(orc, plan):
     """Full-size matrices (4096 x 2048) of three experts and the shared expert."""
     L = synth.packed_layer(synth.FULL, 31, device="cuda")
@@ -124,10 +130,10 @@ def _edge_layer():
     return L
 
 
-@pytest.mark.parametrize("plan", [1])
+@pytest.mark.parametrize("plan", [0, 1])
 def test_probe_edge_blocks_bit_exact(orc, plan):
     L = _edge_layer()
-    lay = m.MoELayer(L["H"], L["I"], 1, 1, 64, act_dtype=m.DS4MOE_ACT_BF16, has_shared=False)
+    lay = m.MoELayer(L["H"], L["I"], 1, 1, 64, has_shared=False)
     lay.load(L)
     for which in (0, 2):
         got = _probe_columns(lay, plan, which, 0)
