@@ -70,25 +70,47 @@ __device__ __forceinline__ void bmma(float (&d)[4], const uint32_t (&a)[4], uint
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b.x), "r"(b.y));
 }
 
+// Four consecutive activations (binary32, or bf16 widened exactly) from a 16-byte (8-byte) aligned index.
+__device__ __forceinline__ float4 load_act4(const void* x, int64_t idx, int act_bf16) {
+    if (act_bf16) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(x) + idx));
+        return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u), __uint_as_float(v.y << 16),
+                           __uint_as_float(v.y & 0xffff0000u));
+    }
+    return __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + idx));
+}
+
 __device__ __forceinline__ uint32_t bf16_bits(float v) {
     return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
 // ---------------------------------------------------------------- router
-// One CTA per kRE expert rows, one warp per row.  Thread 0 brings the CTA's
-// router rows and all n token vectors into shared memory with two bulk copies
-// on one mbarrier, so every CTA's rows are in flight at once (the 4 MB of
-// W_r arrive in about one memory latency).  Lane L then runs chain L of the
-// canonical order (columns 128 i + 4L + r, i ascending, r = 0..3, one fma
-// each), the chains meet in the fixed butterfly (xor 16, 8, 4, 2, 1) and
-// the bias is added once.  The last CTA to finish picks the top-k.
+// One CTA per kRE expert rows; each row's tokens are split over TW warps.
+// Thread 0 brings the CTA's router rows and all n token vectors into shared
+// memory with two bulk copies on one mbarrier, so every CTA's rows are in
+// flight at once (the 4 MB of W_r arrive in about one memory latency).  Lane
+// L then runs chain L of the canonical order (columns 128 i + 4L + r, i
+// ascending, r = 0..3, one fma each), the chains meet in the fixed butterfly
+// (xor 16, 8, 4, 2, 1) and the bias is added once.  The last CTA to finish
+// picks the top-k and, when `ready` is given, publishes it: every thread
+// fences its writes, then one store with release semantics sets *ready.
 template <int NT>
-__global__ void __launch_bounds__(kRE * 32) k_router_decode(Weights W, Dims D, DecodeWs ws, const void* x, int n) {
+struct RouterCfg {
+    static constexpr int TW = NT < 4 ? NT : 4;           // warps per row (token split)
+    static constexpr int TPW = (NT + TW - 1) / TW;       // tokens per warp
+    static constexpr int kWarps = kRE * TW;
+};
+
+template <int NT>
+__global__ void __launch_bounds__(RouterCfg<NT>::kWarps * 32)
+    k_router_decode(Weights W, Dims D, DecodeWs ws, const void* x, int n, uint32_t* ready) {
+    using C = RouterCfg<NT>;
+    constexpr int TW = C::TW, TPW = C::TPW, RW = C::kWarps;
     griddep_launch();   // the gate/up grid may start its shared-expert work now
     extern __shared__ __align__(128) unsigned char r_smem[];   // [kRE][H] f32 rows, then x as given [n][H]
     __shared__ uint64_t bar;
     __shared__ bool s_last;
-    __shared__ float s_logits[kRE][1024];
+    __shared__ float s_logits[RW][1024];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = D.H, E = D.E;
     const int e0 = blockIdx.x * kRE;
@@ -105,17 +127,19 @@ __global__ void __launch_bounds__(kRE * 32) k_router_decode(Weights W, Dims D, D
     }
     __syncthreads();
     mbar_wait(&bar, 0, ws.err);
-    if (warp < nrows) {
-        const int e = e0 + warp;
-        const float* wr = wrows + (size_t)warp * H + 4 * lane;
-        float acc[NT];
+    const int row = warp % kRE, tw = warp / kRE;
+    if (row < nrows) {
+        const int e = e0 + row;
+        const float* wr = wrows + (size_t)row * H + 4 * lane;
+        float acc[TPW];
 #pragma unroll
-        for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+        for (int j = 0; j < TPW; ++j) acc[j] = 0.f;
 #pragma unroll 4
         for (int i = 0; i < H / 128; ++i) {
             const float4 wv = *reinterpret_cast<const float4*>(wr + 128 * i);
 #pragma unroll
-            for (int t = 0; t < NT; ++t) {
+            for (int j = 0; j < TPW; ++j) {
+                const int t = tw + TW * j;
                 if (t < n) {
                     float4 x4;
                     if (D.act_bf16) {
@@ -125,23 +149,25 @@ __global__ void __launch_bounds__(kRE * 32) k_router_decode(Weights W, Dims D, D
                     } else {
                         x4 = *reinterpret_cast<const float4*>(xsm + ((size_t)t * H + 128 * i + 4 * lane) * 4);
                     }
-                    acc[t] = fmaf(x4.x, wv.x, acc[t]);
-                    acc[t] = fmaf(x4.y, wv.y, acc[t]);
-                    acc[t] = fmaf(x4.z, wv.z, acc[t]);
-                    acc[t] = fmaf(x4.w, wv.w, acc[t]);
+                    acc[j] = fmaf(x4.x, wv.x, acc[j]);
+                    acc[j] = fmaf(x4.y, wv.y, acc[j]);
+                    acc[j] = fmaf(x4.z, wv.z, acc[j]);
+                    acc[j] = fmaf(x4.w, wv.w, acc[j]);
                 }
             }
         }
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
+        for (int j = 0; j < TPW; ++j) {
 #pragma unroll
-            for (int m = 16; m >= 1; m >>= 1) acc[t] = acc[t] + __shfl_xor_sync(0xffffffffu, acc[t], m);
+            for (int m = 16; m >= 1; m >>= 1) acc[j] = acc[j] + __shfl_xor_sync(0xffffffffu, acc[j], m);
         }
         if (lane == 0) {
             const float b = W.b_r ? W.b_r[e] : 0.f;
 #pragma unroll
-            for (int t = 0; t < NT; ++t)
-                if (t < n) ws.logits[(int64_t)t * E + e] = W.b_r ? acc[t] + b : acc[t];
+            for (int j = 0; j < TPW; ++j) {
+                const int t = tw + TW * j;
+                if (t < n) ws.logits[(int64_t)t * E + e] = W.b_r ? acc[j] + b : acc[j];
+            }
         }
     }
     __syncthreads();
@@ -154,8 +180,30 @@ __global__ void __launch_bounds__(kRE * 32) k_router_decode(Weights W, Dims D, D
     if (!s_last) return;
     __threadfence();
     if (threadIdx.x == 0) *ws.ticket = 0;
-    for (int t = warp; t < n; t += kRE)
+    for (int t = warp; t < n; t += RW)
         topk_softmax_warp(ws.logits + (int64_t)t * E, s_logits[warp], E, D.k, ws.ids + t * D.k, ws.wts + t * D.k);
+    if (ready) {
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ready), "r"(1u) : "memory");
+    }
+}
+
+// Waits (bounded) until *flag is nonzero, reading it with acquire semantics.
+__device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t* err) {
+    uint64_t t0 = 0;
+    for (;;) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v) return true;
+        if (t0 == 0) {
+            t0 = global_ns();
+        } else if (global_ns() - t0 > kWaitNs) {
+            set_err(err, kErrTimeout);
+            return false;
+        }
+        __nanosleep(64);
+    }
 }
 
 // ---------------------------------------------------------------- routing table
@@ -320,7 +368,11 @@ struct GateUpCfg {
     static constexpr int TPB = NT == 1 ? 1 : 2;                   // tokens of one routed entry
     static constexpr int kThreads = (CW + 1) * 32;
     static constexpr int kTabWords = (256 + 128) * R;
-    static constexpr int kRedFloats = CW * 4 * 64;                // [warp][4 tokens][64 rows]
+    // task reductions: a ring of NB buffers of [warp][128] partial sums (routed: up to 2 tokens x 64
+    // rows; shared: up to 8 tokens x 16 rows); a warp can run at most NS stages (so NS tasks) ahead of
+    // the slowest, so NS + 1 buffers are never reused before their reduction is done
+    static constexpr int NB = NS + 1;
+    static constexpr int kRedFloats = NB * CW * 128;
 };
 
 // The IQ2 chunk of one thread (8 weights, grid row a from byte t of the
@@ -344,7 +396,7 @@ __device__ __forceinline__ void iq2_chunk_s8(uint32_t idx, uint32_t S, uint32_t 
 template <int NT>
 struct GateUpAcc {
     static constexpr int TG = (NT + 3) / 4;   // token groups of four (shared tasks)
-    float sh[TG][4][4];                       // shared task: [token group][tile][fragment]
+    float sh[TG][2][4];                       // shared task: [token group][gate, up][fragment] (rows g only)
     float rt[GateUpCfg<NT>::TPB][4][2];       // routed task: [token][tile][row g, g + 8]
 };
 
@@ -366,81 +418,52 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     __shared__ uint32_t s_cand[2];
     __shared__ float s_tokmax[8];
     __shared__ float s_cs[8][4];
+    __shared__ float s_f[8][2];
+    __shared__ int s_cnt[C::NB];      // warps done with the task that uses each reduction buffer
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     const int H = D.H, I = D.I, k = D.k;
     const int nkt = H / 64, nsb = H / 256;
-    const int n_sh = ws.probe == 1 ? 0 : (D.has_shared ? I / 32 : 0);
+    const int n_sh = ws.probe == 1 ? 0 : (D.has_shared ? I / 8 : 0);   // shared tasks: 8 rows of gate and up
     const int rb_per_e = I / 32;
     // k steps (64 columns) per routed chunk: the largest of 32, 16, 8, 4 that divides H / 64
     const int ck_rt = nkt % 32 == 0 ? 32 : nkt % 16 == 0 ? 16 : nkt % 8 == 0 ? 8 : 4;
     const int nch_rt = nkt / ck_rt;
-    const int kcs = H < 256 ? H : 256;                // columns per shared chunk
+    const int kcs = H < 1024 ? H : 1024;              // columns per shared chunk
     const int nch_sh = H / kcs;
 
     pipe_init(P, NS, CW);
-    // ---- grid: magnitude classes (at most four distinct values, each at most 127), selector tables
-    {
-        int* present = reinterpret_cast<int*>(red);
-        for (int v = tid; v < 256; v += kThreads) present[v] = 0;
-        if (tid < 4) reinterpret_cast<uint4*>(zero)[tid] = make_uint4(0, 0, 0, 0);
-        __syncthreads();
-        for (int q = tid; q < 2048; q += kThreads) present[W.grid_u8[q]] = 1;
-        __syncthreads();
-        if (tid == 0) {
-            int nv = 0;
-            uint32_t lo = 0, hi = 0;
-            bool big = false;
-            for (int v = 0; v < 256; ++v) {
-                if (!present[v]) continue;
-                if (nv < 4) {
-                    lo |= (uint32_t)v << (8 * nv);
-                    hi |= (uint32_t)((-v) & 0xff) << (8 * nv);
-                }
-                big |= v > 127;
-                present[v] = 1 + (nv < 4 ? nv : 3);   // class + 1
-                ++nv;
-            }
-            s_cand[0] = lo;
-            s_cand[1] = hi;
-            s_refused = (nv > 4 || big) ? 1 : 0;
-            if (s_refused) set_err(ws.err, kErrGrid);
-            if (blockIdx.x == 0) *ws.grid_refused = s_refused;
-        }
-        __syncthreads();
-        for (int a = tid; a < 256; a += kThreads) {
-            uint32_t w = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) w |= (uint32_t)(present[W.grid_u8[a * 8 + i]] - 1) << (4 * i);
-#pragma unroll
-            for (int r = 0; r < R; ++r) tsel[a * R + r] = w;
-        }
-        for (int sg = tid; sg < 128; sg += kThreads) {
-            uint32_t w = ((uint32_t)__popc(sg) & 1u) << 30;
-#pragma unroll
-            for (int i = 0; i < 7; ++i) w |= ((uint32_t)(sg >> i) & 1u) << (4 * i + 2);
-#pragma unroll
-            for (int r = 0; r < R; ++r) tsgn[sg * R + r] = w;
-        }
+    // ---- grid tables (made when the grid was loaded), one copy per lane position
+    for (int i = tid; i < 384 * R; i += kThreads) tsel[i] = __ldg(W.gtab + i / R);   // tsgn follows tsel
+    if (tid < 4) reinterpret_cast<uint4*>(zero)[tid] = make_uint4(0, 0, 0, 0);
+    if (tid < C::NB) s_cnt[tid] = 0;
+    if (tid == 0) {
+        s_cand[0] = __ldg(W.gtab + 384);
+        s_cand[1] = __ldg(W.gtab + 385);
+        s_refused = (int)__ldg(W.gtab + 386);
+        if (s_refused) set_err(ws.err, kErrGrid);
+        if (blockIdx.x == 0) *ws.grid_refused = (uint32_t)s_refused;
     }
-    // ---- token maxima (for the int8 pieces of the routed tasks) and the shared tasks' bf16 pieces
+    // ---- token maxima and int8-piece factors (routed tasks), bf16 pieces of x (shared tasks)
     {
         float mx[NT];
 #pragma unroll
         for (int q = 0; q < NT; ++q) mx[q] = 0.f;
-        uint32_t* xb = reinterpret_cast<uint32_t*>(xbuf);   // [n][2][H] bf16 as pairs
-        for (int i = tid * 2; i < H; i += kThreads * 2) {
+        for (int i = tid * 4; i < H; i += kThreads * 4) {
 #pragma unroll
             for (int q = 0; q < NT; ++q) {
                 if (q < n) {
-                    const float v0 = act_at(x, (int64_t)q * H + i, D.act_bf16);
-                    const float v1 = act_at(x, (int64_t)q * H + i + 1, D.act_bf16);
-                    mx[q] = fmaxf(mx[q], fmaxf(fabsf(v0), fabsf(v1)));
+                    const float4 v = load_act4(x, (int64_t)q * H + i, D.act_bf16);
+                    mx[q] = fmaxf(mx[q], fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
                     if (n_sh > 0) {
-                        const uint32_t h0 = bf16_bits(v0), h1 = bf16_bits(v1);
-                        const float r0 = v0 - __uint_as_float(h0 << 16), r1 = v1 - __uint_as_float(h1 << 16);
-                        xb[((size_t)q * 2 * H + i) / 2] = h0 | (h1 << 16);
-                        xb[((size_t)(q * 2 + 1) * H + i) / 2] = bf16_bits(r0) | (bf16_bits(r1) << 16);
+                        const uint32_t h0 = bf16_bits(v.x), h1 = bf16_bits(v.y), h2 = bf16_bits(v.z), h3 = bf16_bits(v.w);
+                        const uint32_t l0 = bf16_bits(v.x - __uint_as_float(h0 << 16));
+                        const uint32_t l1 = bf16_bits(v.y - __uint_as_float(h1 << 16));
+                        const uint32_t l2 = bf16_bits(v.z - __uint_as_float(h2 << 16));
+                        const uint32_t l3 = bf16_bits(v.w - __uint_as_float(h3 << 16));
+                        *reinterpret_cast<uint2*>(xbuf + ((size_t)q * 2 * H + i) * 2) = make_uint2(h0 | (h1 << 16), h2 | (h3 << 16));
+                        *reinterpret_cast<uint2*>(xbuf + ((size_t)(q * 2 + 1) * H + i) * 2) =
+                            make_uint2(l0 | (l1 << 16), l2 | (l3 << 16));
                     }
                 }
             }
@@ -456,6 +479,18 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
 #pragma unroll
             for (int q = 0; q < NT; ++q)
                 if (q < n) atomicMax(reinterpret_cast<int*>(&s_tokmax[q]), __float_as_int(mx[q]));
+        }
+        __syncthreads();
+        if (tid < n) {
+            // x 2^(7-e) has |v| < 128 (e: the exponent of the token's largest |x|); the scaling is split in
+            // two factors so that neither overflows; piece p weighs 2^(e - 7 - 7p)
+            int e = 0;
+            frexpf(s_tokmax[tid], &e);
+            const int sh1 = (7 - e) / 2, sh2 = 7 - e - sh1;
+            s_f[tid][0] = ldexpf(1.f, sh1);
+            s_f[tid][1] = ldexpf(1.f, sh2);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) s_cs[tid][p] = s_tokmax[tid] > 0.f ? ldexpf(1.f, e - 7 - 7 * p) : 0.f;
         }
         __syncthreads();
     }
@@ -474,7 +509,9 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             int task = __shfl_sync(0xffffffffu, next, 0);
             if (lane == 0) next = (int)atomicAdd(ws.queue1, 1u);   // in flight while this task streams
             if (task >= n_sh && !routed) {
-                griddep_wait();                   // router results visible
+                // the router's ids and weights: published by its last CTA through the ready flag (probe
+                // calls route by themselves)
+                if (!ws.probe && !wait_flag(ws.route_ready, ws.err)) { set_abort(P); break; }
                 build_routing_warp(Rt, ws.ids, n, k, TPB, ws.probe == 1 ? 1 : (ws.probe == 2 ? 2 : 0), ws.probe_e);
                 routed = true;
                 total = n_sh + Rt.nu * rb_per_e;
@@ -490,18 +527,15 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                 if (lane == 0) {
                     unsigned char* st = stages + s * kStageBytes;
                     if (sh) {
-                        // 32 rows of the gate and up matrices, columns c*kcs .. +kcs, as four 8-row
-                        // groups of core-matrix tiles per matrix
+                        // one 8-row group of the gate and of the up matrix (core-matrix tiles), columns
+                        // c*kcs .. +kcs
                         const int kc0 = c * kcs;
                         const uint32_t bytes = kcs * 16;
+                        const size_t off = ((size_t)task * (H / 8) + kc0 / 8) * 64;   // elements
                         P.info[s] = ChunkInfo{task, c, nch, kc0, kcs};
-                        mbar_arrive_expect_tx(&P.full[s], 8 * bytes);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const size_t off = ((size_t)(task * 4 + q) * (H / 8) + kc0 / 8) * 64;   // elements
-                            bulk_load(st + q * bytes, W.sh_gate + off, bytes, &P.full[s], pol);
-                            bulk_load(st + 4 * bytes + q * bytes, W.sh_up + off, bytes, &P.full[s], pol);
-                        }
+                        mbar_arrive_expect_tx(&P.full[s], 2 * bytes);
+                        bulk_load(st, W.sh_gate + off, bytes, &P.full[s], pol);
+                        bulk_load(st + bytes, W.sh_up + off, bytes, &P.full[s], pol);
                     } else {
                         const int tt = task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
                         const int e = Rt.uniq[u];
@@ -531,7 +565,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
         const uint32_t clo = s_cand[0], chi = s_cand[1];
         // B operand lanes: column g of the MMA
         const int jB = g >> 2, pB = g & 3;                // routed: 32-column group, int8 piece
-        uint32_t it = 0, cph = 0;
+        uint32_t it = 0, cph = 0, ntask = 0;
         bool quantized = false;
         GateUpAcc<NT> A;
         int tokrow[TPB];
@@ -547,23 +581,15 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                 // first routed stage: every consumer warp is done with the shared tasks' bf16 pieces;
                 // x becomes four int8 pieces per token in the same buffer
                 if (!cons_sync(P, cph, ws.err)) break;
-                for (int q = tid; q < 8 * 4; q += CW * 32) {
-                    const int tk = q >> 2, p = q & 3;
-                    int e = 0;
-                    frexpf(s_tokmax[tk], &e);
-                    s_cs[tk][p] = s_tokmax[tk] > 0.f ? ldexpf(1.f, e - 7 - 7 * p) : 0.f;
-                }
                 for (int q = tid * 4; q < n * H; q += CW * 32 * 4) {
-                    const int tk = q / H, i = q % H;
-                    int e = 0;
-                    frexpf(s_tokmax[tk], &e);
-                    // v = x 2^(7-e), |v| < 128; the scaling is split so that no factor overflows
-                    const int sh1 = (7 - e) / 2, sh2 = 7 - e - sh1;
-                    const float f1 = ldexpf(1.f, sh1), f2 = ldexpf(1.f, sh2);
+                    const int tk = q / H, i = q - tk * H;
+                    const float f1 = s_f[tk][0], f2 = s_f[tk][1];
+                    const float4 xv = load_act4(x, (int64_t)tk * H + i, D.act_bf16);
+                    const float vv[4] = {xv.x, xv.y, xv.z, xv.w};
                     uint32_t pw[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        float v = act_at(x, (int64_t)tk * H + i + j, D.act_bf16) * f1 * f2;
+                        float v = vv[j] * f1 * f2;
 #pragma unroll
                         for (int p = 0; p < 4; ++p) {
                             const float tv = truncf(v);
@@ -582,7 +608,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
 #pragma unroll
                     for (int tg = 0; tg < GateUpAcc<NT>::TG; ++tg)
 #pragma unroll
-                        for (int T = 0; T < 4; ++T) A.sh[tg][T][0] = A.sh[tg][T][1] = A.sh[tg][T][2] = A.sh[tg][T][3] = 0.f;
+                        for (int T = 0; T < 2; ++T) A.sh[tg][T][0] = A.sh[tg][T][1] = A.sh[tg][T][2] = A.sh[tg][T][3] = 0.f;
                 }
                 const int kc = inf.cnt;                                 // columns of the chunk
                 const uint16_t* xb = reinterpret_cast<const uint16_t*>(xbuf);
@@ -597,12 +623,10 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                                    : zero);
                     }
 #pragma unroll
-                    for (int T = 0; T < 4; ++T) {
-                        const unsigned char* base = st + (T >> 1) * (kc * 64) + (2 * (T & 1)) * (kc * 16) +
-                                                    (2 * ks + (t >> 1)) * 128 + g * 16 + (t & 1) * 8;
-                        const uint2 r0 = *reinterpret_cast<const uint2*>(base);
-                        const uint2 r1 = *reinterpret_cast<const uint2*>(base + kc * 16);
-                        const uint32_t Af[4] = {r0.x, r1.x, r0.y, r1.y};
+                    for (int T = 0; T < 2; ++T) {   // gate, up: 8 rows each (the MMA's rows g + 8 repeat rows g)
+                        const uint2 r0 = *reinterpret_cast<const uint2*>(st + T * (kc * 16) + (2 * ks + (t >> 1)) * 128 +
+                                                                         g * 16 + (t & 1) * 8);
+                        const uint32_t Af[4] = {r0.x, r0.x, r0.y, r0.y};
 #pragma unroll
                         for (int tg = 0; tg < GateUpAcc<NT>::TG; ++tg) bmma(A.sh[tg][T], Af, B[tg]);
                     }
@@ -689,46 +713,19 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&P.empty[s]);
             if (inf.chunk == inf.nchunk - 1) {
-                // task epilogue: reduce the warps' partials, SwiGLU, store h (two bf16 pieces) and its block sums
-                bool ok = true;
+                // task epilogue: this warp's partials into the task's reduction buffer; the last warp to
+                // arrive sums them in warp order, applies SwiGLU and stores h (two bf16 pieces, block sums)
+                const int b = (int)(ntask % C::NB);
+                ++ntask;
+                float* rbuf = red + (size_t)b * CW * 128;
                 if (sh) {
+                    // this lane's token is 4 tg + t: its columns 2t, 2t+1 are that token's two pieces
 #pragma unroll
-                    for (int tg = 0; tg < GateUpAcc<NT>::TG; ++tg) {
-                        // this lane's token is 4 tg + t: its columns 2t, 2t+1 are that token's two pieces
+                    for (int tg = 0; tg < GateUpAcc<NT>::TG; ++tg)
 #pragma unroll
-                        for (int T = 0; T < 4; ++T) {
-                            const int row = (T >> 1) * 32 + 16 * (T & 1) + g;
-                            red[(warp * 4 + t) * 64 + row] = A.sh[tg][T][0] + A.sh[tg][T][1];
-                            red[(warp * 4 + t) * 64 + row + 8] = A.sh[tg][T][2] + A.sh[tg][T][3];
-                        }
-                        if (!(ok = cons_sync(P, cph, ws.err))) break;
-                        if (tid < 128) {
-                            const int tl = tid >> 5, row = tid & 31, tok = 4 * tg + tl;
-                            float gv = 0.f, uv = 0.f;
-                            for (int w = 0; w < CW; ++w) {
-                                gv += red[(w * 4 + tl) * 64 + row];
-                                uv += red[(w * 4 + tl) * 64 + 32 + row];
-                            }
-                            const int c = 32 * inf.task + row;
-                            if (tok < n) {
-                                if (ws.probe) {
-                                    ws.probe_out[(size_t)tok * 2 * I + c] = gv;
-                                    ws.probe_out[(size_t)tok * 2 * I + I + c] = uv;
-                                } else {
-                                    const float h = silu(gv) * uv;
-                                    const uint32_t hi = bf16_bits(h);
-                                    const uint32_t lo = bf16_bits(h - __uint_as_float(hi << 16));
-                                    uint16_t* hb = ws.hb_sh + (size_t)tok * 2 * I;
-                                    hb[hsh_index(c, 0)] = (uint16_t)hi;
-                                    hb[hsh_index(c, 1)] = (uint16_t)lo;
-                                }
-                            }
-                        }
-                        if (!(ok = cons_sync(P, cph, ws.err))) break;
-                    }
+                        for (int T = 0; T < 2; ++T)
+                            rbuf[warp * 128 + (4 * tg + t) * 16 + T * 8 + g] = A.sh[tg][T][0] + A.sh[tg][T][1];
                 } else {
-                    const int tt = inf.task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
-                    const int s0 = Rt.ustart[u];
 #pragma unroll
                     for (int q = 0; q < TPB; ++q) {
 #pragma unroll
@@ -738,23 +735,55 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                                 float v = A.rt[q][T][r];
                                 v += __shfl_xor_sync(0xffffffffu, v, 1);
                                 v += __shfl_xor_sync(0xffffffffu, v, 2);
-                                if (t == 0) red[(warp * 4 + q) * 64 + (T >> 1) * 32 + 16 * (T & 1) + g + 8 * r] = v;
+                                if (t == 0) rbuf[warp * 128 + q * 64 + (T >> 1) * 32 + 16 * (T & 1) + g + 8 * r] = v;
                             }
                         }
                     }
-                    if ((ok = cons_sync(P, cph, ws.err))) {
-                        if (warp < tcount) {
-                            const int q = warp, row = lane;
+                }
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) {
+                    __threadfence_block();
+                    last = atomicAdd(&s_cnt[b], 1) == CW - 1;
+                }
+                if (__shfl_sync(0xffffffffu, last, 0)) {
+                    __threadfence_block();
+                    if (sh) {
+                        for (int q = lane; q < 8 * n; q += 32) {   // (token, row) pairs
+                            const int tok = q >> 3, row = q & 7;
                             float gv = 0.f, uv = 0.f;
                             for (int w = 0; w < CW; ++w) {
-                                gv += red[(w * 4 + q) * 64 + row];
-                                uv += red[(w * 4 + q) * 64 + 32 + row];
+                                gv += rbuf[w * 128 + tok * 16 + row];
+                                uv += rbuf[w * 128 + tok * 16 + 8 + row];
+                            }
+                            const int c = 8 * inf.task + row;
+                            if (ws.probe) {
+                                ws.probe_out[(size_t)tok * 2 * I + c] = gv;
+                                ws.probe_out[(size_t)tok * 2 * I + I + c] = uv;
+                            } else {
+                                const float h = silu(gv) * uv;
+                                const uint32_t hi = bf16_bits(h);
+                                const uint32_t lo = bf16_bits(h - __uint_as_float(hi << 16));
+                                uint16_t* hb = ws.hb_sh + (size_t)tok * 2 * I;
+                                hb[hsh_index(c, 0)] = (uint16_t)hi;
+                                hb[hsh_index(c, 1)] = (uint16_t)lo;
+                            }
+                        }
+                    } else {
+                        const int tt = inf.task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
+                        const int s0 = Rt.ustart[u];
+                        for (int q = 0; q < tcount; ++q) {
+                            const int row = lane;
+                            float gv = 0.f, uv = 0.f;
+                            for (int w = 0; w < CW; ++w) {
+                                gv += rbuf[w * 128 + q * 64 + row];
+                                uv += rbuf[w * 128 + q * 64 + 32 + row];
                             }
                             const int slot = Rt.slot[s0 + q];
                             const int c = 32 * rb + row;
                             if (ws.probe) {
-                                ws.probe_out[(size_t)tokrow[q] * 2 * I + c] = gv;
-                                ws.probe_out[(size_t)tokrow[q] * 2 * I + I + c] = uv;
+                                ws.probe_out[(size_t)(slot / k) * 2 * I + c] = gv;
+                                ws.probe_out[(size_t)(slot / k) * 2 * I + I + c] = uv;
                             } else {
                                 const float h = silu(gv) * uv;
                                 const uint32_t hi = bf16_bits(h);
@@ -769,10 +798,10 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                                 if ((lane & 15) == 0) ws.hsum_rt[(size_t)slot * (I / 16) + 2 * rb + (lane >> 4)] = hs;
                             }
                         }
-                        ok = cons_sync(P, cph, ws.err);
                     }
+                    __syncwarp();
+                    if (lane == 0) s_cnt[b] = 0;
                 }
-                if (!ok) break;
             }
             ++it;
         }
@@ -786,6 +815,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
         if (s_last) {
             *ws.queue1 = 0;
             *ws.done1 = 0;
+            *ws.route_ready = 0;
         }
     }
 }
@@ -797,7 +827,10 @@ struct DownCfg {
     static constexpr int CW = NT <= 2 ? 16 : 8;
     static constexpr int TPB = NT == 1 ? 1 : 2;
     static constexpr int kThreads = (CW + 1) * 32;
-    static constexpr int kRedFloats = CW * 4 * 32;   // [warp][4 tokens][32 rows]
+    // task reductions: a ring of NS + 1 buffers of [warp][128] partial sums (routed: up to 2 tokens
+    // x 32 rows; shared: up to 8 tokens x 16 rows), as in the gate/up kernel
+    static constexpr int NB = NS + 1;
+    static constexpr int kRedFloats = NB * CW * 128;
 };
 
 // k steps (64 columns) per routed down chunk for an entry of ns slots: codes,
@@ -816,7 +849,7 @@ __device__ __forceinline__ int down_chunk_ksteps(int nkt, int nsb, int ns) {
 template <int NT>
 struct DownAcc {
     static constexpr int TG = (NT + 3) / 4;
-    float sh[TG][2][4];                        // shared task: [token group][tile][fragment]
+    float sh[TG][4];                           // shared task: [token group][fragment]
     float rt[DownCfg<NT>::TPB][2][2];          // routed task: [token][tile][row g, g + 8]
 };
 
@@ -832,17 +865,19 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
     __shared__ Pipe P;
     __shared__ Routing Rt;
     __shared__ int s_last;
+    __shared__ int s_cnt[C::NB];      // warps done with the task that uses each reduction buffer
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     const int H = D.H, I = D.I, k = D.k;
     const int nkt = I / 64, nsb = I >= 256 ? I / 256 : 1;
-    const int n_sh = ws.probe == 1 ? 0 : (D.has_shared ? H / 32 : 0);
+    const int n_sh = ws.probe == 1 ? 0 : (D.has_shared ? H / 16 : 0);   // shared tasks: 16 rows
     const int rb_per_e = H / 32;
-    const int kcs = I < 256 ? I : 256;        // columns per shared chunk
+    const int kcs = I < 512 ? I : 512;        // columns per shared chunk
     const int nch_sh = I / kcs;
 
     pipe_init(P, NS, CW);
     if (tid < 16) reinterpret_cast<uint32_t*>(zero)[tid] = 0u;
+    if (tid < C::NB) s_cnt[tid] = 0;
     if (warp == CW)   // ids final: the router grid is complete
         build_routing_warp(Rt, ws.ids, n, k, TPB, ws.probe == 1 ? 1 : (ws.probe == 2 ? 2 : 0), ws.probe_e);
     __syncthreads();
@@ -876,18 +911,18 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
                 if (lane == 0) {
                     unsigned char* st = stages + s * kStageBytes;
                     if (sh) {
-                        // 32 rows of the shared down matrix (four 8-row groups of core-matrix tiles),
+                        // 16 rows of the shared down matrix (two 8-row groups of core-matrix tiles),
                         // columns c*kcs .. +kcs, then every token's h pieces for those columns
                         const int kc0 = c * kcs;
                         const uint32_t abytes = kcs * 16, hbytes = kcs * 4;
                         P.info[s] = ChunkInfo{task, c, nch, kc0, kcs};
-                        mbar_arrive_expect_tx(&P.full[s], 4 * abytes + n * hbytes);
+                        mbar_arrive_expect_tx(&P.full[s], 2 * abytes + n * hbytes);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            bulk_load(st + q * abytes, W.sh_down + ((size_t)(task * 4 + q) * (I / 8) + kc0 / 8) * 64,
+                        for (int q = 0; q < 2; ++q)
+                            bulk_load(st + q * abytes, W.sh_down + ((size_t)(task * 2 + q) * (I / 8) + kc0 / 8) * 64,
                                       abytes, &P.full[s], pol);
                         for (int q = 0; q < n; ++q)
-                            bulk_load_plain(st + 4 * abytes + q * hbytes, ws.hb_sh + ((size_t)q * (I / 64) + kc0 / 64) * 128,
+                            bulk_load_plain(st + 2 * abytes + q * hbytes, ws.hb_sh + ((size_t)q * (I / 64) + kc0 / 64) * 128,
                                             hbytes, &P.full[s]);
                     } else {
                         const int e = Rt.uniq[u], s0 = Rt.ustart[u];
@@ -923,7 +958,7 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
         // ------------------------------------------------ consumer warps
         const uint32_t rot = (5u - 2u * (uint32_t)t) & 31u;   // code t of each byte to bits 5..6
         const int jB = g >> 1, pB = g & 1;                    // routed B lanes: sub-block, piece
-        uint32_t it = 0, cph = 0;
+        uint32_t it = 0, ntask = 0;
         DownAcc<NT> A;
         int tcount = 0;
         for (;;) {
@@ -936,12 +971,10 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
             if (sh) {
                 if (inf.chunk == 0) {
 #pragma unroll
-                    for (int tg = 0; tg < DownAcc<NT>::TG; ++tg)
-#pragma unroll
-                        for (int T = 0; T < 2; ++T) A.sh[tg][T][0] = A.sh[tg][T][1] = A.sh[tg][T][2] = A.sh[tg][T][3] = 0.f;
+                    for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) A.sh[tg][0] = A.sh[tg][1] = A.sh[tg][2] = A.sh[tg][3] = 0.f;
                 }
                 const int kc = inf.cnt;
-                const unsigned char* hst = st + 4 * kc * 16;
+                const unsigned char* hst = st + 2 * kc * 16;
                 for (int ks = warp; ks < kc / 16; ks += CW) {
                     uint2 B[DownAcc<NT>::TG];
 #pragma unroll
@@ -951,14 +984,13 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
                             tk < n ? hst + (size_t)tk * kc * 4 + ((ks >> 2) * 2 + p) * 128 + ((ks & 3) * 16 + 4 * t) * 2
                                    : zero);
                     }
-#pragma unroll
-                    for (int T = 0; T < 2; ++T) {
-                        const unsigned char* base = st + (2 * T) * (kc * 16) + (2 * ks + (t >> 1)) * 128 + g * 16 + (t & 1) * 8;
+                    {
+                        const unsigned char* base = st + (2 * ks + (t >> 1)) * 128 + g * 16 + (t & 1) * 8;
                         const uint2 r0 = *reinterpret_cast<const uint2*>(base);
                         const uint2 r1 = *reinterpret_cast<const uint2*>(base + kc * 16);
                         const uint32_t Af[4] = {r0.x, r1.x, r0.y, r1.y};
 #pragma unroll
-                        for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) bmma(A.sh[tg][T], Af, B[tg]);
+                        for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) bmma(A.sh[tg], Af, B[tg]);
                     }
                 }
             } else {
@@ -1035,28 +1067,19 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&P.empty[s]);
             if (inf.chunk == inf.nchunk - 1) {
-                // task epilogue: reduce the warps' partials, store y
-                bool ok = true;
+                // task epilogue: this warp's partials into the task's reduction buffer; the last warp to
+                // arrive sums them in warp order and stores y
+                const int b = (int)(ntask % C::NB);
+                ++ntask;
+                float* rbuf = red + (size_t)b * CW * 128;
                 if (sh) {
+                    // this lane's token is 4 tg + t (its columns 2t, 2t+1 are that token's two pieces)
 #pragma unroll
                     for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) {
-#pragma unroll
-                        for (int T = 0; T < 2; ++T) {
-                            red[(warp * 4 + t) * 32 + 16 * T + g] = A.sh[tg][T][0] + A.sh[tg][T][1];
-                            red[(warp * 4 + t) * 32 + 16 * T + g + 8] = A.sh[tg][T][2] + A.sh[tg][T][3];
-                        }
-                        if (!(ok = cons_sync(P, cph, ws.err))) break;
-                        if (tid < 128) {
-                            const int tl = tid >> 5, row = tid & 31, tok = 4 * tg + tl;
-                            float y = 0.f;
-                            for (int w = 0; w < CW; ++w) y += red[(w * 4 + tl) * 32 + row];
-                            if (tok < n) (ws.probe ? ws.probe_out : ws.y_sh)[(size_t)tok * H + 32 * inf.task + row] = y;
-                        }
-                        if (!(ok = cons_sync(P, cph, ws.err))) break;
+                        rbuf[warp * 128 + (4 * tg + t) * 16 + g] = A.sh[tg][0] + A.sh[tg][1];
+                        rbuf[warp * 128 + (4 * tg + t) * 16 + g + 8] = A.sh[tg][2] + A.sh[tg][3];
                     }
                 } else {
-                    const int tt = inf.task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
-                    const int s0 = Rt.ustart[u];
 #pragma unroll
                     for (int q = 0; q < TPB; ++q) {
 #pragma unroll
@@ -1066,22 +1089,40 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
                                 float v = A.rt[q][T][r];
                                 v += __shfl_xor_sync(0xffffffffu, v, 1);
                                 v += __shfl_xor_sync(0xffffffffu, v, 2);
-                                if (t == 0) red[(warp * 4 + q) * 32 + 16 * T + g + 8 * r] = v;
+                                if (t == 0) rbuf[warp * 128 + q * 32 + 16 * T + g + 8 * r] = v;
                             }
                         }
                     }
-                    if ((ok = cons_sync(P, cph, ws.err))) {
-                        if (warp < tcount) {
+                }
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) {
+                    __threadfence_block();
+                    last = atomicAdd(&s_cnt[b], 1) == CW - 1;
+                }
+                if (__shfl_sync(0xffffffffu, last, 0)) {
+                    __threadfence_block();
+                    if (sh) {
+                        for (int q = lane; q < 16 * n; q += 32) {   // (token, row) pairs
+                            const int tok = q >> 4, row = q & 15;
                             float y = 0.f;
-                            for (int w = 0; w < CW; ++w) y += red[(w * 4 + warp) * 32 + lane];
-                            const int slot = Rt.slot[s0 + warp];
+                            for (int w = 0; w < CW; ++w) y += rbuf[w * 128 + tok * 16 + row];
+                            (ws.probe ? ws.probe_out : ws.y_sh)[(size_t)tok * H + 16 * inf.task + row] = y;
+                        }
+                    } else {
+                        const int tt = inf.task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
+                        const int s0 = Rt.ustart[u];
+                        for (int q = 0; q < tcount; ++q) {
+                            float y = 0.f;
+                            for (int w = 0; w < CW; ++w) y += rbuf[w * 128 + q * 32 + lane];
+                            const int slot = Rt.slot[s0 + q];
                             if (ws.probe) ws.probe_out[(size_t)(slot / k) * H + 32 * rb + lane] = y;
                             else ws.y_rt[(size_t)slot * H + 32 * rb + lane] = y;
                         }
-                        ok = cons_sync(P, cph, ws.err);
                     }
+                    __syncwarp();
+                    if (lane == 0) s_cnt[b] = 0;
                 }
-                if (!ok) break;
             }
             ++it;
         }
@@ -1157,6 +1198,56 @@ __global__ void __launch_bounds__(kSteerThreads) k_combine_steer_decode(Dims D, 
             out[(int64_t)t * H + r] = ws.xres ? act_at(ws.xres, (int64_t)t * H + r, D.act_bf16) + y : y;
         }
     }
+}
+
+// ---------------------------------------------------------------- grid tables
+// The decode plan's tables of a grid, made once when the grid is loaded (one
+// CTA of 256 threads): the distinct magnitudes in ascending order are classes
+// 0..3; gtab[a] holds the classes of row a's eight elements as nibbles,
+// gtab[256 + sg] the sign flags of the 7-bit sign field sg as bit 2 of each
+// nibble (element 7 negative for odd popcount), gtab[384..387] the magnitudes
+// as int8 bytes, their negatives, whether the grid is refused (more than four
+// distinct values, or a value above 127) and the number of distinct values.
+__global__ void __launch_bounds__(256) k_grid_tables(const uint8_t* grid, uint32_t* gtab) {
+    __shared__ int cls[256];
+    const int tid = threadIdx.x;
+    cls[tid] = 0;
+    __syncthreads();
+    for (int q = tid; q < 2048; q += 256) cls[grid[q]] = 1;
+    __syncthreads();
+    if (tid == 0) {
+        int nv = 0;
+        uint32_t lo = 0, hi = 0;
+        bool big = false;
+        for (int v = 0; v < 256; ++v) {
+            if (!cls[v]) continue;
+            if (nv < 4) {
+                lo |= (uint32_t)v << (8 * nv);
+                hi |= (uint32_t)((-v) & 0xff) << (8 * nv);
+            }
+            big |= v > 127;
+            cls[v] = 1 + (nv < 4 ? nv : 3);
+            ++nv;
+        }
+        gtab[384] = lo;
+        gtab[385] = hi;
+        gtab[386] = (nv > 4 || big) ? 1u : 0u;
+        gtab[387] = (uint32_t)nv;
+    }
+    __syncthreads();
+    uint32_t w = 0;
+    for (int i = 0; i < 8; ++i) w |= (uint32_t)(cls[grid[tid * 8 + i]] - 1) << (4 * i);
+    gtab[tid] = w;
+    if (tid < 128) {
+        uint32_t sgw = ((uint32_t)__popc(tid) & 1u) << 30;
+        for (int i = 0; i < 7; ++i) sgw |= ((uint32_t)(tid >> i) & 1u) << (4 * i + 2);
+        gtab[256 + tid] = sgw;
+    }
+}
+
+cudaError_t launch_grid_tables(const uint8_t* grid, uint32_t* gtab, cudaStream_t st) {
+    k_grid_tables<<<1, 256, 0, st>>>(grid, gtab);
+    return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- failure-path check
@@ -1273,7 +1364,8 @@ cudaError_t launch_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws,
     const bool pdl = ev == nullptr;   // profiled runs keep the kernels apart
     const int rgrid = (D.E + kRE - 1) / kRE;
     mk.before();
-    k_router_decode<NT><<<rgrid, kRE * 32, router_smem_bytes(D, n), st>>>(W, D, ws, x, n);
+    k_router_decode<NT><<<rgrid, RouterCfg<NT>::kWarps * 32, router_smem_bytes(D, n), st>>>(W, D, ws, x, n,
+                                                                                             ws.route_ready);
     mk.after();
     mk.before();
     err = launch_pdl(k_gateup_decode<NT>, dim3(n_sm), dim3(GateUpCfg<NT>::kThreads), s1, st, pdl, W, D, ws, x, n);
@@ -1306,7 +1398,7 @@ size_t decode_smem_bytes(const Dims& D, int n) {
     else if (n <= 4) { a = gateup_smem_bytes<4>(D, n); b = down_smem_bytes<4>(D, n); }
     else { a = gateup_smem_bytes<8>(D, n); b = down_smem_bytes<8>(D, n); }
     size_t need = (a > b ? a : b) + sizeof(Pipe) + sizeof(Routing) + 512;   // + the kernels' other static shared memory
-    const size_t r = router_smem_bytes(D, n) + sizeof(float) * kRE * 1024 + 64;
+    const size_t r = router_smem_bytes(D, n) + sizeof(float) * 8 * 1024 + 64;
     return r > need ? r : need;
 }
 
@@ -1380,7 +1472,7 @@ cudaError_t launch_route_t(const Weights& W, const Dims& D, const DecodeWs& ws, 
     cudaError_t err;
     const size_t s0 = router_smem_bytes(D, n);
     if ((err = configure(k_router_decode<NT>)) != cudaSuccess) return err;
-    k_router_decode<NT><<<(D.E + kRE - 1) / kRE, kRE * 32, s0, st>>>(W, D, ws, x, n);
+    k_router_decode<NT><<<(D.E + kRE - 1) / kRE, RouterCfg<NT>::kWarps * 32, s0, st>>>(W, D, ws, x, n, nullptr);
     return cudaGetLastError();
 }
 

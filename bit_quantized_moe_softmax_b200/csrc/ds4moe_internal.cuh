@@ -35,6 +35,10 @@ enum : uint32_t { kErrBounds = 1u, kErrTimeout = 2u, kErrGrid = 4u };
 // Pointers into the caller's weight buffer, in the layout above.
 struct Weights {
     const uint8_t* grid_u8;     // [256][8]
+    const uint32_t* gtab;       // decode tables of the grid, made by set_grid: [256] magnitude classes of each
+                                // row (nibble i = class of element i), [128] sign nibbles of each 7-bit sign
+                                // field (bit 2 of nibble i; element 7 from the parity), then the four
+                                // magnitudes as int8, their negatives, refused (0/1), distinct values
     const float* W_r;           // [E][H]
     const float* W_r2;          // [ceil(E/2)][H][2]: expert pairs interleaved per column (prefill plan), or nullptr
     const float* b_r;           // [E] or nullptr
@@ -66,6 +70,7 @@ struct DecodeWs {
     uint32_t* done1;        // gate/up CTAs finished (the last one resets queue1)
     uint32_t* done2;        // down CTAs finished (the last one resets queue2)
     uint32_t* grid_refused; // this call's gate/up grid refused the grid (too many or too large magnitudes): 1, else 0
+    uint32_t* route_ready;  // set by the router once ids / weights are written; reset by the gate/up grid
     float* logits;          // [n][E]
     int32_t* ids;           // [n][k]
     float* wts;             // [n][k]
