@@ -84,6 +84,25 @@ __device__ __forceinline__ uint32_t bf16_bits(float v) {
     return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
+// Byte permute in PTX form: a selector nibble with bit 3 set replicates the sign bit of its byte.
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+// 2s + 1 for the 4-bit IQ2 group scale s of an S word in device order (bit c of s in bit 7 of byte c):
+// selO (0xBA98 for the first word, 0xFEDC for the second) turns each byte into 0 or -1 by its top
+// bit; the dot product with bytes (-2, -4, -8, -16) plus 1 is 2s + 1.
+__device__ __forceinline__ int iq2_odd(uint32_t s0, uint32_t s1, uint32_t selO) {
+    return __dp4a((int)prmt_b32(s0, s1, selO), (int)0xF0F8FCFEu, 1);
+}
+
 // ---------------------------------------------------------------- router
 // One CTA per kRE expert rows; each row's tokens are split over TW warps.
 // Thread 0 brings the CTA's router rows and all n token vectors into shared
@@ -362,12 +381,17 @@ __device__ __forceinline__ int hsh_index(int c, int piece) { return ((c >> 6) * 
 // ---------------------------------------------------------------- gate/up
 template <int NT>
 struct GateUpCfg {
-    static constexpr int CW = NT <= 2 ? 16 : 8;                   // consumer warps
+    static constexpr int CW = NT == 1 ? 16 : 8;                   // consumer warps
     static constexpr int NS = NT <= 4 ? 3 : 2;                    // stages
-    static constexpr int R = NT <= 2 ? 32 : (NT == 4 ? 16 : 8);   // copies of the selector tables
+    // selector tables: ROWS form (one or two tokens): 256 rows of 256 B, bytes 0..127 of row r the
+    // class selectors of grid row r, bytes 128..255 the sign selectors of S byte r (signs r & 127),
+    // 32 copies each (one per lane), so that one byte-permute of a payload word and the lane's offset
+    // is the row's address; otherwise tsel [256][R] and tsgn [128][R] with R interleaved copies
+    static constexpr bool kRows = NT <= 2;
+    static constexpr int R = NT == 4 ? 16 : 8;
     static constexpr int TPB = NT == 1 ? 1 : 2;                   // tokens of one routed entry
     static constexpr int kThreads = (CW + 1) * 32;
-    static constexpr int kTabWords = (256 + 128) * R;
+    static constexpr int kTabWords = kRows ? 256 * 64 : (256 + 128) * R;
     // task reductions: a ring of NB buffers of [warp][128] partial sums (routed: up to 2 tokens x 64
     // rows; shared: up to 8 tokens x 16 rows); a warp can run at most NS stages (so NS tasks) ahead of
     // the slowest, so NS + 1 buffers are never reused before their reduction is done
@@ -376,17 +400,26 @@ struct GateUpCfg {
 };
 
 // The IQ2 chunk of one thread (8 weights, grid row a from byte t of the
-// index word, sign field at bit 7t of S) as int8 +-G: weights 0..3 in lo,
-// 4..7 in hi.  The selector's nibble i is the magnitude class of weight i
-// plus 4 for a negative sign; (clo, chi) hold the four magnitudes and their
-// negatives.
-// tsel / tsgn point at this lane's copy of the tables (copies interleaved, R words per entry).
+// index word, signs in byte t of S) as int8 +-G: weights 0..3 in lo, 4..7 in
+// hi.  The selector's nibble i is the magnitude class of weight i plus 4 for
+// a negative sign; (clo, chi) hold the four magnitudes and their negatives.
+// Rows form: tb = the table's shared address, lbA / lbB = this lane's byte
+// offset in the class / sign half of a row, selT puts byte t of the word in
+// byte 1 of the offset.
+__device__ __forceinline__ void iq2_chunk_rows(uint32_t idx, uint32_t S, uint32_t tb, uint32_t lbA, uint32_t lbB,
+                                               uint32_t selT, uint32_t clo, uint32_t chi, uint32_t& lo,
+                                               uint32_t& hi) {
+    const uint32_t sel = ld_shared_u32(tb + __byte_perm(idx, lbA, selT)) | ld_shared_u32(tb + __byte_perm(S, lbB, selT));
+    lo = __byte_perm(clo, chi, sel);
+    hi = __byte_perm(clo, chi, sel >> 16);
+}
+// Interleaved form: tsel / tsgn point at this lane's copy (R words per entry).
 template <int R>
-__device__ __forceinline__ void iq2_chunk_s8(uint32_t idx, uint32_t S, uint32_t selA, int t7, const uint32_t* tsel,
+__device__ __forceinline__ void iq2_chunk_s8(uint32_t idx, uint32_t S, uint32_t selA, int t8, const uint32_t* tsel,
                                              const uint32_t* tsgn, uint32_t clo, uint32_t chi, uint32_t& lo,
                                              uint32_t& hi) {
     const uint32_t a = __byte_perm(idx, 0u, selA);
-    const uint32_t sg = (S >> t7) & 127u;
+    const uint32_t sg = (S >> t8) & 127u;
     const uint32_t sel = tsel[a * R] | tsgn[sg * R];
     lo = __byte_perm(clo, chi, sel);
     hi = __byte_perm(clo, chi, sel >> 16);
@@ -406,10 +439,10 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     using C = GateUpCfg<NT>;
     constexpr int NS = C::NS, CW = C::CW, R = C::R, TPB = C::TPB, kThreads = C::kThreads;
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    unsigned char* stages = smem_raw;                                            // NS x kStageBytes
-    uint32_t* tsel = reinterpret_cast<uint32_t*>(smem_raw + NS * kStageBytes);   // [256][R]
-    uint32_t* tsgn = tsel + 256 * R;                                             // [128][R]
-    float* red = reinterpret_cast<float*>(tsgn + 128 * R);                       // kRedFloats
+    uint32_t* tsel = reinterpret_cast<uint32_t*>(smem_raw);                      // rows [256][64] or [256][R]
+    uint32_t* tsgn = tsel + 256 * R;                                             // [128][R] (interleaved form)
+    unsigned char* stages = smem_raw + 4 * C::kTabWords;                         // NS x kStageBytes
+    float* red = reinterpret_cast<float*>(stages + NS * kStageBytes);            // kRedFloats
     unsigned char* xbuf = reinterpret_cast<unsigned char*>(red + C::kRedFloats);  // n x H x 4 bytes
     unsigned char* zero = xbuf + (size_t)n * D.H * 4;                            // 64 bytes of zeros
     __shared__ Pipe P;
@@ -433,8 +466,15 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     const int nch_sh = H / kcs;
 
     pipe_init(P, NS, CW);
-    // ---- grid tables (made when the grid was loaded), one copy per lane position
-    for (int i = tid; i < 384 * R; i += kThreads) tsel[i] = __ldg(W.gtab + i / R);   // tsgn follows tsel
+    // ---- grid tables (made when the grid was loaded)
+    if (C::kRows) {
+        for (int i = tid; i < 256 * 64; i += kThreads) {
+            const int r = i >> 6;
+            tsel[i] = __ldg(W.gtab + ((i & 32) ? 256 + (r & 127) : r));
+        }
+    } else {
+        for (int i = tid; i < 384 * R; i += kThreads) tsel[i] = __ldg(W.gtab + i / R);   // tsgn follows tsel
+    }
     if (tid < 4) reinterpret_cast<uint4*>(zero)[tid] = make_uint4(0, 0, 0, 0);
     if (tid < C::NB) s_cnt[tid] = 0;
     if (tid == 0) {
@@ -559,9 +599,12 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     } else if (!refused) {
         // ------------------------------------------------ consumer warps
         const uint32_t selA = 0x4440u | (uint32_t)t;   // byte t of the index word
-        const uint32_t selS = (t >> 1) ? 0x4447u : 0x4443u;   // top byte of this lane's group's S word
+        const uint32_t selO = (t >> 1) ? 0xFEDCu : 0xBA98u;   // this lane's group's S word, top bits
         const uint32_t* tselp = tsel + (lane % R);
         const uint32_t* tsgnp = tsgn + (lane % R);
+        const uint32_t tb = smem_addr(tsel);
+        const uint32_t lbA = (uint32_t)lane << 2, lbB = 128u | ((uint32_t)lane << 2);
+        const uint32_t selT = 0x7604u | ((uint32_t)t << 4);
         const uint32_t clo = s_cand[0], chi = s_cand[1];
         // B operand lanes: column g of the MMA
         const int jB = g >> 2, pB = g & 3;                // routed: 32-column group, int8 piece
@@ -669,12 +712,19 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                             const uint4 r0 = *reinterpret_cast<const uint4*>(pay);
                             const uint4 r1 = *reinterpret_cast<const uint4*>(pay + 128);
                             uint32_t A0[4], A1[4];
-                            iq2_chunk_s8<R>(r0.x, r0.y, selA, 7 * t, tselp, tsgnp, clo, chi, A0[0], A0[2]);
-                            iq2_chunk_s8<R>(r1.x, r1.y, selA, 7 * t, tselp, tsgnp, clo, chi, A0[1], A0[3]);
-                            iq2_chunk_s8<R>(r0.z, r0.w, selA, 7 * t, tselp, tsgnp, clo, chi, A1[0], A1[2]);
-                            iq2_chunk_s8<R>(r1.z, r1.w, selA, 7 * t, tselp, tsgnp, clo, chi, A1[1], A1[3]);
-                            const int o0 = (int)(((__byte_perm(r0.y, r0.w, selS) >> 3) & 0x1eu) | 1u);
-                            const int o1 = (int)(((__byte_perm(r1.y, r1.w, selS) >> 3) & 0x1eu) | 1u);
+                            if (C::kRows) {
+                                iq2_chunk_rows(r0.x, r0.y, tb, lbA, lbB, selT, clo, chi, A0[0], A0[2]);
+                                iq2_chunk_rows(r1.x, r1.y, tb, lbA, lbB, selT, clo, chi, A0[1], A0[3]);
+                                iq2_chunk_rows(r0.z, r0.w, tb, lbA, lbB, selT, clo, chi, A1[0], A1[2]);
+                                iq2_chunk_rows(r1.z, r1.w, tb, lbA, lbB, selT, clo, chi, A1[1], A1[3]);
+                            } else {
+                                iq2_chunk_s8<R>(r0.x, r0.y, selA, 8 * t, tselp, tsgnp, clo, chi, A0[0], A0[2]);
+                                iq2_chunk_s8<R>(r1.x, r1.y, selA, 8 * t, tselp, tsgnp, clo, chi, A0[1], A0[3]);
+                                iq2_chunk_s8<R>(r0.z, r0.w, selA, 8 * t, tselp, tsgnp, clo, chi, A1[0], A1[2]);
+                                iq2_chunk_s8<R>(r1.z, r1.w, selA, 8 * t, tselp, tsgnp, clo, chi, A1[1], A1[3]);
+                            }
+                            const int o0 = iq2_odd(r0.y, r0.w, selO);
+                            const int o1 = iq2_odd(r1.y, r1.w, selO);
 #pragma unroll
                             for (int q = 0; q < TPB; ++q) {
                                 if (q < tcount) {
@@ -824,7 +874,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
 template <int NT>
 struct DownCfg {
     static constexpr int NS = 4;
-    static constexpr int CW = NT <= 2 ? 16 : 8;
+    static constexpr int CW = NT == 1 ? 16 : 8;
     static constexpr int TPB = NT == 1 ? 1 : 2;
     static constexpr int kThreads = (CW + 1) * 32;
     // task reductions: a ring of NS + 1 buffers of [warp][128] partial sums (routed: up to 2 tokens

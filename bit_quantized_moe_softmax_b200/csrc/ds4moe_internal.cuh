@@ -7,7 +7,8 @@
 // rows back to back, so one warp (lane = row) reads 512 contiguous bytes per
 // 64-column step.  Per matrix:
 //   IQ2 payload  [R/32][C/64][32][16 B]   the two 8-byte groups of columns
-//                                        64kt..64kt+63 (grid indices + S word)
+//                                        64kt..64kt+63 (grid indices + S word,
+//                                        S in the device order below)
 //   IQ2 d        [R/32][C/256][32] binary16
 //   Q2 codes     [R/32][C/64][32][16 B]  64 two-bit codes, canonical bit order
 //   Q2 scales    [R/32][C/64][32][4 B]   the 4 scale/min bytes of those codes
@@ -17,6 +18,10 @@
 // weights) except that a C < 256 matrix stores its (d, dmin) once per row.
 // Shared (bf16) matrices are stored in 8x8 core-matrix tiles:
 //   [R/8][C/8][8 rows][8 cols], 128 contiguous bytes per tile.
+// IQ2 S word, device order: byte c (c = 0..3) holds the seven stored signs of
+// chunk c in bits 0..6 and bit c of the 4-bit group scale in bit 7 (the block
+// keeps the signs at bits 7c..7c+6 and the scale at bits 28..31).  One byte
+// per chunk lets a byte-permute place a chunk's signs in a table address.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -27,6 +32,17 @@
 namespace ds4 {
 
 constexpr int kQK = 256;
+
+// IQ2 S word: block order -> device order, and the fields of the device order.
+__host__ __device__ __forceinline__ uint32_t iq2_s_to_device(uint32_t S) {
+    uint32_t o = 0;
+    for (int c = 0; c < 4; ++c) o |= (((S >> (7 * c)) & 127u) | (((S >> (28 + c)) & 1u) << 7)) << (8 * c);
+    return o;
+}
+__host__ __device__ __forceinline__ uint32_t iq2_dev_scale(uint32_t Sd) {
+    return ((Sd >> 7) & 1u) | ((Sd >> 14) & 2u) | ((Sd >> 21) & 4u) | ((Sd >> 28) & 8u);
+}
+__host__ __device__ __forceinline__ uint32_t iq2_dev_signs(uint32_t Sd, int c) { return (Sd >> (8 * c)) & 127u; }
 constexpr int kQ2Bytes = 84;
 constexpr int kIQ2Bytes = 66;
 

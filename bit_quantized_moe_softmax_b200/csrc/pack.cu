@@ -126,7 +126,7 @@ __global__ void k_pack_iq2(const float* __restrict__ w, int64_t n_blocks, const 
 
 // ---------------------------------------------------------------- repack
 // IQ2 canonical blocks of an [R][C] matrix -> payload [R/32][C/64][32][16 B]
-// and d [R/32][C/256][32].  One thread per (block, group).
+// (S words in the device order) and d [R/32][C/256][32].  One thread per (block, group).
 __global__ void k_repack_iq2(const uint8_t* __restrict__ src, int R, int C, uint8_t* __restrict__ qs,
                              uint16_t* __restrict__ dd) {
     int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -139,7 +139,11 @@ __global__ void k_repack_iq2(const uint8_t* __restrict__ src, int R, int C, uint
     const uint8_t* blk = src + b * kIQ2Bytes;
     int kt = 4 * sb + (g >> 1), half = g & 1;
     uint8_t* dst = qs + (((int64_t)(r >> 5) * (C / 64) + kt) * 32 + (r & 31)) * 16 + half * 8;
-    for (int i = 0; i < 8; ++i) dst[i] = blk[2 + 8 * g + i];
+    for (int i = 0; i < 4; ++i) dst[i] = blk[2 + 8 * g + i];
+    const uint8_t* sp = blk + 2 + 8 * g + 4;
+    const uint32_t S = iq2_s_to_device((uint32_t)sp[0] | ((uint32_t)sp[1] << 8) | ((uint32_t)sp[2] << 16) |
+                                       ((uint32_t)sp[3] << 24));
+    for (int i = 0; i < 4; ++i) dst[4 + i] = (uint8_t)(S >> (8 * i));
     if (g == 0) dd[((int64_t)(r >> 5) * nsb + sb) * 32 + (r & 31)] = (uint16_t)(blk[0] | (blk[1] << 8));
 }
 
@@ -200,8 +204,8 @@ __global__ void k_dequant_iq2(const uint8_t* __restrict__ qs, const uint16_t* __
     const uint8_t* p = qs + (((int64_t)(r >> 5) * (C / 64) + kt) * 32 + (r & 31)) * 16 + half * 8;
     uint32_t S = (uint32_t)p[4] | ((uint32_t)p[5] << 8) | ((uint32_t)p[6] << 16) | ((uint32_t)p[7] << 24);
     float d = half_bits(dd[((int64_t)(r >> 5) * (C / kQK) + col / kQK) * 32 + (r & 31)]);
-    float db = d * (float)(2 * (S >> 28) + 1) * 0.125f;
-    uint32_t sigma = (S >> (7 * c)) & 127u;
+    float db = d * (float)(2 * iq2_dev_scale(S) + 1) * 0.125f;
+    uint32_t sigma = iq2_dev_signs(S, c);
     uint32_t neg = i < 7 ? (sigma >> i) & 1u : (uint32_t)(__popc(sigma) & 1);
     float v = db * (float)grid[p[c] * 8 + i];
     v = neg ? -v : v;

@@ -389,7 +389,7 @@ __device__ __forceinline__ uint32_t b_row_off(int r) { return (uint32_t)((r >> 3
 // bit 15 and bit 2j+1 at bit 31 (the two shifted copies of the 8-bit sign byte
 // do not overlap, so the multiply has no carries).
 __device__ __forceinline__ uint4 iq2_chunk_bf16(uint2 sl, uint32_t S, int c, uint32_t cand01, uint32_t cand23) {
-    const uint32_t sg = (S >> (7 * c)) & 127u;
+    const uint32_t sg = iq2_dev_signs(S, c);
     // sign of element 7 = parity of the seven stored bits, added at bit 31 of the last mask
     const uint32_t m3 = sg * 0x01000200u + ((uint32_t)__popc(sg) << 31);
     return make_uint4(__byte_perm(cand01, cand23, sl.x) ^ ((sg * 0x40008000u) & 0x80008000u),
@@ -674,7 +674,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                                 sl[c] = *reinterpret_cast<const uint2*>(selp + __byte_perm(idx, 0u, 0x4440u | c) *
                                                                                    (kGSelRep * 8));
                             const float db =
-                                d * (__uint_as_float(0x4b000001u | ((Sw >> 27) & 0x1eu)) - 8388608.0f) * 0.125f;
+                                d * (__uint_as_float(0x4b000001u | (iq2_dev_scale(Sw) << 1)) - 8388608.0f) * 0.125f;
                             const float2 db2 = make_float2(db, db);
                             const float2 c01 = fmul2(db2, gv01), c23 = fmul2(db2, gv23);
                             const uint32_t cand01 = pack_bf16x2(c01.x, c01.y), cand23 = pack_bf16x2(c23.x, c23.y);
