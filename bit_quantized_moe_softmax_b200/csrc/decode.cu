@@ -225,6 +225,26 @@ __device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t* err) {
     }
 }
 
+// Waits (bounded) until *counter >= target, reading it with acquire semantics, then orders the
+// generic-proxy writes it published before this thread's later bulk copies (async proxy).
+__device__ __forceinline__ bool wait_count(const uint32_t* counter, uint32_t target, uint32_t* err) {
+    uint64_t t0 = 0;
+    for (;;) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+        if (v >= target) break;
+        if (t0 == 0) {
+            t0 = global_ns();
+        } else if (global_ns() - t0 > kWaitNs) {
+            set_err(err, kErrTimeout);
+            return false;
+        }
+        __nanosleep(32);
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    return true;
+}
+
 // ---------------------------------------------------------------- routing table
 // Routed tasks' experts ("entries") in ascending expert order, each with the
 // slots (t * k + j) that chose it in increasing slot order, at most tpb slots
@@ -378,10 +398,129 @@ __device__ __forceinline__ int hrt_index(int c, int piece) {
 }
 __device__ __forceinline__ int hsh_index(int c, int piece) { return ((c >> 6) * 2 + piece) * 64 + (c & 63); }
 
+// ---------------------------------------------------------------- task order
+// Queue position -> task.  The first `lead` positions are shared-expert tasks 0..lead-1 (they need no
+// routing); the remaining n_sh - lead shared tasks are spread evenly among the n_rt routed tasks
+// (numbered n_sh + i), so that each SM alternates between bandwidth-bound shared-expert stages and
+// dequantization-bound routed stages.  Positions past the end map to n_sh + n_rt (no task).
+__device__ __forceinline__ int task_at(int pos, int lead, int n_sh, int n_rt) {
+    if (pos < lead) return pos;
+    const int S = n_sh - lead, r = pos - lead;
+    if (r >= S + n_rt) return n_sh + n_rt;
+    const int a = (int)((int64_t)(r + 1) * S / (S + n_rt)), b = (int)((int64_t)r * S / (S + n_rt));
+    return a > b ? lead + b : n_sh + (r - a);
+}
+
+// ---------------------------------------------------------------- task reductions
+// The consumer warps of a projection kernel split every task's columns, so a task ends with a sum over
+// the warps.  Each consumer warp writes its partial sums into reduction buffer b = (its task count) % NB
+// and counts itself in; a separate epilogue warp takes the buffers in order, sums the partials in warp
+// order (deterministic), finishes the task (activation, stores, completion count) and frees the buffer
+// for its next use.  The consumers thus never wait on a task's final reduction, only (rarely) on a
+// buffer that the epilogue warp has not freed yet.
+constexpr int kMaxRedBufs = 8;
+struct RedRing {
+    int cnt[kMaxRedBufs];     // consumer warps that wrote their partials into buffer b
+    int task[kMaxRedBufs];    // the task whose partials buffer b holds
+    int freed[kMaxRedBufs];   // uses of buffer b that the epilogue warp has finished
+    int exits;                // consumer warps that left their loop
+    int ntasks;               // tasks the consumer warps finished (read once exits == consumer warps)
+};
+
+__device__ __forceinline__ int ld_shared_volatile(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
+
+// Consumer side: waits (bounded) until buffer b is free for its use number `use`.
+__device__ __forceinline__ bool ring_acquire(RedRing& R, int b, int use, uint32_t* err) {
+    if (ld_shared_volatile(&R.freed[b]) >= use) return true;
+    const uint64_t t0 = global_ns();
+    while (ld_shared_volatile(&R.freed[b]) < use) {
+        if (global_ns() - t0 > kWaitNs) {
+            set_err(err, kErrTimeout);
+            return false;
+        }
+        __nanosleep(32);
+    }
+    return true;
+}
+
+// Consumer side, lane 0 after the warp's partials are written: buffer b holds task `task`.
+__device__ __forceinline__ void ring_publish(RedRing& R, int b, int task) {
+    R.task[b] = task;
+    __threadfence_block();
+    atomicAdd(&R.cnt[b], 1);
+}
+
+// Consumer side, lane 0 when the warp leaves its loop after finishing `ntask` tasks.
+__device__ __forceinline__ void ring_exit(RedRing& R, int ntask) {
+    atomicMax(&R.ntasks, ntask);
+    __threadfence_block();
+    atomicAdd(&R.exits, 1);
+}
+
+// Epilogue side (whole warp): waits (bounded) until buffer j % nb holds the partials of every consumer
+// warp; false once the consumers have left and buffer j will not be filled.
+__device__ __forceinline__ bool ring_take(RedRing& R, uint32_t j, int nb, int cw, uint32_t* err) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) {
+        const int b = (int)(j % nb);
+        uint64_t t0 = 0;
+        for (;;) {
+            if (ld_shared_volatile(&R.cnt[b]) == cw) { ok = 1; break; }
+            if (ld_shared_volatile(&R.exits) == cw && (int)j >= ld_shared_volatile(&R.ntasks)) break;
+            if (t0 == 0) {
+                t0 = global_ns();
+            } else if (global_ns() - t0 > kWaitNs) {
+                set_err(err, kErrTimeout);
+                break;
+            }
+            __nanosleep(32);
+        }
+        __threadfence_block();
+    }
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Epilogue side (whole warp) after finishing buffer j: free it for its next use.
+__device__ __forceinline__ void ring_free(RedRing& R, uint32_t j, int nb) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+        const int b = (int)(j % nb);
+        R.cnt[b] = 0;
+        __threadfence_block();
+        R.freed[b] = (int)(j / nb) + 1;
+    }
+    __syncwarp();
+}
+
+// x (n tokens of H) as four int8 pieces per value, [n][4][H] bytes: v = x f1 f2 (|v| < 128), piece p
+// = trunc of the remaining fraction times 128^p.  Threads tid of nthreads, four values each.
+__device__ __forceinline__ void quantize_x(const void* x, int act_bf16, int n, int H, const float (*s_f)[2],
+                                           unsigned char* xq, int tid, int nthreads) {
+    for (int q = tid * 4; q < n * H; q += nthreads * 4) {
+        const int tk = q / H, i = q - tk * H;
+        const float f1 = s_f[tk][0], f2 = s_f[tk][1];
+        const float4 xv = load_act4(x, (int64_t)tk * H + i, act_bf16);
+        const float vv[4] = {xv.x, xv.y, xv.z, xv.w};
+        uint32_t pw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float v = vv[j] * f1 * f2;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const float tv = truncf(v);
+                pw[p] |= ((uint32_t)(int)tv & 0xffu) << (8 * j);
+                v = (v - tv) * 128.f;
+            }
+        }
+#pragma unroll
+        for (int p = 0; p < 4; ++p) *reinterpret_cast<uint32_t*>(xq + (size_t)(tk * 4 + p) * H + i) = pw[p];
+    }
+}
+
 // ---------------------------------------------------------------- gate/up
 template <int NT>
 struct GateUpCfg {
-    static constexpr int CW = NT == 1 ? 16 : 8;                   // consumer warps
+    static constexpr int CW = 8;                                  // consumer warps
     static constexpr int NS = NT <= 4 ? 3 : 2;                    // stages
     // selector tables: ROWS form (one or two tokens): 256 rows of 256 B, bytes 0..127 of row r the
     // class selectors of grid row r, bytes 128..255 the sign selectors of S byte r (signs r & 127),
@@ -390,13 +529,16 @@ struct GateUpCfg {
     static constexpr bool kRows = NT <= 2;
     static constexpr int R = NT == 4 ? 16 : 8;
     static constexpr int TPB = NT == 1 ? 1 : 2;                   // tokens of one routed entry
-    static constexpr int kThreads = (CW + 1) * 32;
+    static constexpr int kThreads = (CW + 2) * 32;                // + producer warp + epilogue warp
     static constexpr int kTabWords = kRows ? 256 * 64 : (256 + 128) * R;
-    // task reductions: a ring of NB buffers of [warp][128] partial sums (routed: up to 2 tokens x 64
-    // rows; shared: up to 8 tokens x 16 rows); a warp can run at most NS stages (so NS tasks) ahead of
-    // the slowest, so NS + 1 buffers are never reused before their reduction is done
-    static constexpr int NB = NS + 1;
-    static constexpr int kRedFloats = NB * CW * 128;
+    // task reductions: a ring of NB buffers of [warp][kRedPer] partial sums (routed: TPB tokens x 64
+    // rows; shared: up to 8 tokens x 16 rows)
+    static constexpr int NB = NT == 8 ? NS + 1 : NS + 2;
+    static constexpr int kRedPer = NT == 1 ? 64 : 128;
+    static constexpr int kRedFloats = NB * CW * kRedPer;
+    // one token: x's int8 pieces get their own buffer, made in the prologue; otherwise they replace the
+    // bf16 pieces once the shared-expert tasks are done
+    static constexpr bool kSplitX = NT == 1;
 };
 
 // The IQ2 chunk of one thread (8 weights, grid row a from byte t of the
@@ -443,8 +585,9 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     uint32_t* tsgn = tsel + 256 * R;                                             // [128][R] (interleaved form)
     unsigned char* stages = smem_raw + 4 * C::kTabWords;                         // NS x kStageBytes
     float* red = reinterpret_cast<float*>(stages + NS * kStageBytes);            // kRedFloats
-    unsigned char* xbuf = reinterpret_cast<unsigned char*>(red + C::kRedFloats);  // n x H x 4 bytes
-    unsigned char* zero = xbuf + (size_t)n * D.H * 4;                            // 64 bytes of zeros
+    unsigned char* xbuf = reinterpret_cast<unsigned char*>(red + C::kRedFloats);  // n x H x 4 bytes: bf16 pieces
+    unsigned char* xq = C::kSplitX ? xbuf + (size_t)n * D.H * 4 : xbuf;          // int8 pieces
+    unsigned char* zero = xq + (size_t)n * D.H * 4;                              // 64 bytes of zeros
     __shared__ Pipe P;
     __shared__ Routing Rt;
     __shared__ int s_last, s_refused;
@@ -452,7 +595,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     __shared__ float s_tokmax[8];
     __shared__ float s_cs[8][4];
     __shared__ float s_f[8][2];
-    __shared__ int s_cnt[C::NB];      // warps done with the task that uses each reduction buffer
+    __shared__ RedRing RR;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     const int H = D.H, I = D.I, k = D.k;
@@ -476,7 +619,8 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
         for (int i = tid; i < 384 * R; i += kThreads) tsel[i] = __ldg(W.gtab + i / R);   // tsgn follows tsel
     }
     if (tid < 4) reinterpret_cast<uint4*>(zero)[tid] = make_uint4(0, 0, 0, 0);
-    if (tid < C::NB) s_cnt[tid] = 0;
+    if (tid < kMaxRedBufs) RR.cnt[tid] = RR.task[tid] = RR.freed[tid] = 0;
+    if (tid == 0) RR.exits = RR.ntasks = 0;
     if (tid == 0) {
         s_cand[0] = __ldg(W.gtab + 384);
         s_cand[1] = __ldg(W.gtab + 385);
@@ -533,6 +677,10 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             for (int p = 0; p < 4; ++p) s_cs[tid][p] = s_tokmax[tid] > 0.f ? ldexpf(1.f, e - 7 - 7 * p) : 0.f;
         }
         __syncthreads();
+        if (C::kSplitX) {
+            quantize_x(x, D.act_bf16, n, H, s_f, xq, tid, kThreads);
+            __syncthreads();
+        }
     }
     const bool refused = s_refused != 0;
 
@@ -542,21 +690,36 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
         uint32_t it = 0;
         bool routed = false;
         int total = 0x7fffffff;
-        int next = 0;
-        if (lane == 0) next = (int)atomicAdd(ws.queue1, 1u);
+        // task queue, two ahead (the atomic for the one after next is in flight while this task streams).
+        // One shared-expert task per CTA leads (while the router finishes); the rest interleave with
+        // routed tasks, except when x's int8 pieces replace its bf16 pieces (all shared-expert tasks come
+        // first then).
+        const int lead = !C::kSplitX ? n_sh : (n_sh < (int)gridDim.x ? n_sh : (int)gridDim.x);
+        int nxt = 0, nxt2 = 0;
+        auto route = [&]() {
+            build_routing_warp(Rt, ws.ids, n, k, TPB, ws.probe == 1 ? 1 : (ws.probe == 2 ? 2 : 0), ws.probe_e);
+            routed = true;
+            total = n_sh + Rt.nu * rb_per_e;
+            griddep_launch();                 // the down grid may start streaming
+        };
+        if (lane == 0) {
+            nxt = (int)atomicAdd(ws.queue1, 1u);
+            nxt2 = (int)atomicAdd(ws.queue1, 1u);
+        }
         for (;;) {
             if (aborted(P) || refused) break;
-            int task = __shfl_sync(0xffffffffu, next, 0);
-            if (lane == 0) next = (int)atomicAdd(ws.queue1, 1u);   // in flight while this task streams
-            if (task >= n_sh && !routed) {
+            const int pos = __shfl_sync(0xffffffffu, nxt, 0);
+            if (lane == 0) {
+                nxt = nxt2;
+                nxt2 = (int)atomicAdd(ws.queue1, 1u);   // in flight while this task streams
+            }
+            if (pos >= lead && !routed) {
                 // the router's ids and weights: published by its last CTA through the ready flag (probe
                 // calls route by themselves)
                 if (!ws.probe && !wait_flag(ws.route_ready, ws.err)) { set_abort(P); break; }
-                build_routing_warp(Rt, ws.ids, n, k, TPB, ws.probe == 1 ? 1 : (ws.probe == 2 ? 2 : 0), ws.probe_e);
-                routed = true;
-                total = n_sh + Rt.nu * rb_per_e;
-                griddep_launch();                 // the down grid may start streaming
+                route();
             }
+            const int task = pos < lead ? pos : task_at(pos, lead, n_sh, total - n_sh);
             if (task >= total) break;
             const bool sh = task < n_sh;
             const int nch = sh ? nch_sh : nch_rt;
@@ -596,7 +759,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             }
         }
         producer_finish(P, it, NS, ws.err);
-    } else if (!refused) {
+    } else if (warp < CW && !refused) {
         // ------------------------------------------------ consumer warps
         const uint32_t selA = 0x4440u | (uint32_t)t;   // byte t of the index word
         const uint32_t selO = (t >> 1) ? 0xFEDCu : 0xBA98u;   // this lane's group's S word, top bits
@@ -620,29 +783,11 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             if (inf.task < 0 || aborted(P)) break;
             const unsigned char* st = stages + s * kStageBytes;
             const bool sh = inf.task < n_sh;
-            if (!sh && !quantized) {
+            if (!C::kSplitX && !sh && !quantized) {
                 // first routed stage: every consumer warp is done with the shared tasks' bf16 pieces;
                 // x becomes four int8 pieces per token in the same buffer
                 if (!cons_sync(P, cph, ws.err)) break;
-                for (int q = tid * 4; q < n * H; q += CW * 32 * 4) {
-                    const int tk = q / H, i = q - tk * H;
-                    const float f1 = s_f[tk][0], f2 = s_f[tk][1];
-                    const float4 xv = load_act4(x, (int64_t)tk * H + i, D.act_bf16);
-                    const float vv[4] = {xv.x, xv.y, xv.z, xv.w};
-                    uint32_t pw[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        float v = vv[j] * f1 * f2;
-#pragma unroll
-                        for (int p = 0; p < 4; ++p) {
-                            const float tv = truncf(v);
-                            pw[p] |= ((uint32_t)(int)tv & 0xffu) << (8 * j);
-                            v = (v - tv) * 128.f;
-                        }
-                    }
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) *reinterpret_cast<uint32_t*>(xbuf + (size_t)(tk * 4 + p) * H + i) = pw[p];
-                }
+                quantize_x(x, D.act_bf16, n, H, s_f, xq, tid, CW * 32);
                 quantized = true;
                 if (!cons_sync(P, cph, ws.err)) break;
             }
@@ -702,7 +847,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
 #pragma unroll
                         for (int q = 0; q < TPB; ++q) {
                             const unsigned char* live =
-                                xbuf + (size_t)(tokrow[q] * 4 + pB) * H + col + 32 * jB + 8 * t;
+                                xq + (size_t)(tokrow[q] * 4 + pB) * H + col + 32 * jB + 8 * t;
                             B[q][0] = *reinterpret_cast<const uint2*>(q < tcount && jB == 0 ? live : zero);
                             B[q][1] = *reinterpret_cast<const uint2*>(q < tcount && jB == 1 ? live : zero);
                         }
@@ -725,17 +870,16 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                             }
                             const int o0 = iq2_odd(r0.y, r0.w, selO);
                             const int o1 = iq2_odd(r1.y, r1.w, selO);
+                            // no branch on the entry's token count: an absent token's B is zero
 #pragma unroll
                             for (int q = 0; q < TPB; ++q) {
-                                if (q < tcount) {
-                                    int Dv[4];
-                                    imma_z(Dv, A0, B[q][0]);
-                                    imma(Dv, A1, B[q][1]);
-                                    ai[q][T][0] += Dv[0] * o0;
-                                    ai[q][T][1] += Dv[1] * o0;
-                                    ai[q][T][2] += Dv[2] * o1;
-                                    ai[q][T][3] += Dv[3] * o1;
-                                }
+                                int Dv[4];
+                                imma_z(Dv, A0, B[q][0]);
+                                imma(Dv, A1, B[q][1]);
+                                ai[q][T][0] += Dv[0] * o0;
+                                ai[q][T][1] += Dv[1] * o0;
+                                ai[q][T][2] += Dv[2] * o1;
+                                ai[q][T][3] += Dv[3] * o1;
                             }
                         }
                     }
@@ -748,14 +892,12 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                         const uint16_t* dm = dq + (T >> 1) * (ck / 4) * 32 + sbl * 32 + 16 * (T & 1) + g;
                         const float d0 = half_bits(dm[0]) * 0.125f, d1 = half_bits(dm[8]) * 0.125f;
 #pragma unroll
-                        for (int q = 0; q < TPB; ++q) {
-                            if (q < tcount) {
-                                const float c0 = s_cs[tokrow[q]][p0], c1 = s_cs[tokrow[q]][p0 + 1];
-                                A.rt[q][T][0] = fmaf((float)ai[q][T][0], d0 * c0, A.rt[q][T][0]);
-                                A.rt[q][T][0] = fmaf((float)ai[q][T][1], d0 * c1, A.rt[q][T][0]);
-                                A.rt[q][T][1] = fmaf((float)ai[q][T][2], d1 * c0, A.rt[q][T][1]);
-                                A.rt[q][T][1] = fmaf((float)ai[q][T][3], d1 * c1, A.rt[q][T][1]);
-                            }
+                        for (int q = 0; q < TPB; ++q) {   // absent tokens: ai = 0
+                            const float c0 = s_cs[tokrow[q]][p0], c1 = s_cs[tokrow[q]][p0 + 1];
+                            A.rt[q][T][0] = fmaf((float)ai[q][T][0], d0 * c0, A.rt[q][T][0]);
+                            A.rt[q][T][0] = fmaf((float)ai[q][T][1], d0 * c1, A.rt[q][T][0]);
+                            A.rt[q][T][1] = fmaf((float)ai[q][T][2], d1 * c0, A.rt[q][T][1]);
+                            A.rt[q][T][1] = fmaf((float)ai[q][T][3], d1 * c1, A.rt[q][T][1]);
                         }
                     }
                 }
@@ -763,18 +905,18 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&P.empty[s]);
             if (inf.chunk == inf.nchunk - 1) {
-                // task epilogue: this warp's partials into the task's reduction buffer; the last warp to
-                // arrive sums them in warp order, applies SwiGLU and stores h (two bf16 pieces, block sums)
+                // task end: this warp's partials into the task's reduction buffer (the epilogue warp
+                // finishes the task)
                 const int b = (int)(ntask % C::NB);
-                ++ntask;
-                float* rbuf = red + (size_t)b * CW * 128;
+                if (!ring_acquire(RR, b, (int)(ntask / C::NB), ws.err)) { set_abort(P); break; }
+                float* rbuf = red + (size_t)b * CW * C::kRedPer + warp * C::kRedPer;
                 if (sh) {
                     // this lane's token is 4 tg + t: its columns 2t, 2t+1 are that token's two pieces
 #pragma unroll
                     for (int tg = 0; tg < GateUpAcc<NT>::TG; ++tg)
 #pragma unroll
                         for (int T = 0; T < 2; ++T)
-                            rbuf[warp * 128 + (4 * tg + t) * 16 + T * 8 + g] = A.sh[tg][T][0] + A.sh[tg][T][1];
+                            if (4 * tg + t < n) rbuf[(4 * tg + t) * 16 + T * 8 + g] = A.sh[tg][T][0] + A.sh[tg][T][1];
                 } else {
 #pragma unroll
                     for (int q = 0; q < TPB; ++q) {
@@ -785,75 +927,86 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                                 float v = A.rt[q][T][r];
                                 v += __shfl_xor_sync(0xffffffffu, v, 1);
                                 v += __shfl_xor_sync(0xffffffffu, v, 2);
-                                if (t == 0) rbuf[warp * 128 + q * 64 + (T >> 1) * 32 + 16 * (T & 1) + g + 8 * r] = v;
+                                if (t == 0) rbuf[q * 64 + (T >> 1) * 32 + 16 * (T & 1) + g + 8 * r] = v;
                             }
                         }
                     }
                 }
                 __syncwarp();
-                int last = 0;
-                if (lane == 0) {
-                    __threadfence_block();
-                    last = atomicAdd(&s_cnt[b], 1) == CW - 1;
-                }
-                if (__shfl_sync(0xffffffffu, last, 0)) {
-                    __threadfence_block();
-                    if (sh) {
-                        for (int q = lane; q < 8 * n; q += 32) {   // (token, row) pairs
-                            const int tok = q >> 3, row = q & 7;
-                            float gv = 0.f, uv = 0.f;
-                            for (int w = 0; w < CW; ++w) {
-                                gv += rbuf[w * 128 + tok * 16 + row];
-                                uv += rbuf[w * 128 + tok * 16 + 8 + row];
-                            }
-                            const int c = 8 * inf.task + row;
-                            if (ws.probe) {
-                                ws.probe_out[(size_t)tok * 2 * I + c] = gv;
-                                ws.probe_out[(size_t)tok * 2 * I + I + c] = uv;
-                            } else {
-                                const float h = silu(gv) * uv;
-                                const uint32_t hi = bf16_bits(h);
-                                const uint32_t lo = bf16_bits(h - __uint_as_float(hi << 16));
-                                uint16_t* hb = ws.hb_sh + (size_t)tok * 2 * I;
-                                hb[hsh_index(c, 0)] = (uint16_t)hi;
-                                hb[hsh_index(c, 1)] = (uint16_t)lo;
-                            }
-                        }
-                    } else {
-                        const int tt = inf.task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
-                        const int s0 = Rt.ustart[u];
-                        for (int q = 0; q < tcount; ++q) {
-                            const int row = lane;
-                            float gv = 0.f, uv = 0.f;
-                            for (int w = 0; w < CW; ++w) {
-                                gv += rbuf[w * 128 + q * 64 + row];
-                                uv += rbuf[w * 128 + q * 64 + 32 + row];
-                            }
-                            const int slot = Rt.slot[s0 + q];
-                            const int c = 32 * rb + row;
-                            if (ws.probe) {
-                                ws.probe_out[(size_t)(slot / k) * 2 * I + c] = gv;
-                                ws.probe_out[(size_t)(slot / k) * 2 * I + I + c] = uv;
-                            } else {
-                                const float h = silu(gv) * uv;
-                                const uint32_t hi = bf16_bits(h);
-                                const float hf = __uint_as_float(hi << 16);
-                                const uint32_t lo = bf16_bits(h - hf);
-                                uint16_t* hb = ws.hb_rt + (size_t)slot * 2 * I;
-                                hb[hrt_index(c, 0)] = (uint16_t)hi;
-                                hb[hrt_index(c, 1)] = (uint16_t)lo;
-                                float hs = hf + __uint_as_float(lo << 16);
-#pragma unroll
-                                for (int m = 1; m <= 8; m <<= 1) hs += __shfl_xor_sync(0xffffffffu, hs, m);
-                                if ((lane & 15) == 0) ws.hsum_rt[(size_t)slot * (I / 16) + 2 * rb + (lane >> 4)] = hs;
-                            }
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) s_cnt[b] = 0;
-                }
+                if (lane == 0) ring_publish(RR, b, inf.task);
+                ++ntask;
             }
             ++it;
+        }
+        if (lane == 0) ring_exit(RR, (int)ntask);
+    } else if (warp == CW + 1 && !refused) {
+        // ------------------------------------------------ epilogue warp
+        for (uint32_t j = 0; ring_take(RR, j, C::NB, CW, ws.err); ++j) {
+            const int b = (int)(j % C::NB);
+            const float* rbuf = red + (size_t)b * CW * C::kRedPer;
+            const int task = RR.task[b];
+            const bool sh = task < n_sh;
+            if (sh) {
+                for (int q = lane; q < 8 * n; q += 32) {   // (token, row) pairs
+                    const int tok = q >> 3, row = q & 7;
+                    float gv = 0.f, uv = 0.f;
+                    for (int w = 0; w < CW; ++w) {
+                        gv += rbuf[w * C::kRedPer + tok * 16 + row];
+                        uv += rbuf[w * C::kRedPer + tok * 16 + 8 + row];
+                    }
+                    const int c = 8 * task + row;
+                    if (ws.probe) {
+                        ws.probe_out[(size_t)tok * 2 * I + c] = gv;
+                        ws.probe_out[(size_t)tok * 2 * I + I + c] = uv;
+                    } else {
+                        const float h = silu(gv) * uv;
+                        const uint32_t hi = bf16_bits(h);
+                        const uint32_t lo = bf16_bits(h - __uint_as_float(hi << 16));
+                        uint16_t* hb = ws.hb_sh + (size_t)tok * 2 * I;
+                        hb[hsh_index(c, 0)] = (uint16_t)hi;
+                        hb[hsh_index(c, 1)] = (uint16_t)lo;
+                    }
+                }
+            } else {
+                const int tt = task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
+                const int s0 = Rt.ustart[u], ns = Rt.ustart[u + 1] - s0;
+                for (int q = 0; q < ns; ++q) {
+                    const int row = lane;
+                    float gv = 0.f, uv = 0.f;
+                    for (int w = 0; w < CW; ++w) {
+                        gv += rbuf[w * C::kRedPer + q * 64 + row];
+                        uv += rbuf[w * C::kRedPer + q * 64 + 32 + row];
+                    }
+                    const int slot = Rt.slot[s0 + q];
+                    const int c = 32 * rb + row;
+                    if (ws.probe) {
+                        ws.probe_out[(size_t)(slot / k) * 2 * I + c] = gv;
+                        ws.probe_out[(size_t)(slot / k) * 2 * I + I + c] = uv;
+                    } else {
+                        const float h = silu(gv) * uv;
+                        const uint32_t hi = bf16_bits(h);
+                        const float hf = __uint_as_float(hi << 16);
+                        const uint32_t lo = bf16_bits(h - hf);
+                        uint16_t* hb = ws.hb_rt + (size_t)slot * 2 * I;
+                        hb[hrt_index(c, 0)] = (uint16_t)hi;
+                        hb[hrt_index(c, 1)] = (uint16_t)lo;
+                        float hs = hf + __uint_as_float(lo << 16);
+#pragma unroll
+                        for (int m = 1; m <= 8; m <<= 1) hs += __shfl_xor_sync(0xffffffffu, hs, m);
+                        if ((lane & 15) == 0) ws.hsum_rt[(size_t)slot * (I / 16) + 2 * rb + (lane >> 4)] = hs;
+                    }
+                }
+            }
+            if (!ws.probe) {
+                // h of this task is complete: publish it to the down grid (the warp barrier orders every
+                // lane's stores before lane 0's fence, which is cumulative)
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence();
+                    atomicAdd(ws.gu_done + (sh ? 0 : 1 + (task - n_sh) / rb_per_e), 1u);
+                }
+            }
+            ring_free(RR, j, C::NB);
         }
     }
     griddep_launch();
@@ -865,7 +1018,6 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
         if (s_last) {
             *ws.queue1 = 0;
             *ws.done1 = 0;
-            *ws.route_ready = 0;
         }
     }
 }
@@ -874,13 +1026,14 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
 template <int NT>
 struct DownCfg {
     static constexpr int NS = 4;
-    static constexpr int CW = NT == 1 ? 16 : 8;
+    static constexpr int CW = 8;
     static constexpr int TPB = NT == 1 ? 1 : 2;
-    static constexpr int kThreads = (CW + 1) * 32;
-    // task reductions: a ring of NS + 1 buffers of [warp][128] partial sums (routed: up to 2 tokens
-    // x 32 rows; shared: up to 8 tokens x 16 rows), as in the gate/up kernel
-    static constexpr int NB = NS + 1;
-    static constexpr int kRedFloats = NB * CW * 128;
+    static constexpr int kThreads = (CW + 2) * 32;                // + producer warp + epilogue warp
+    // task reductions: a ring of NB buffers of [warp][kRedPer] partial sums (routed: TPB tokens x 32
+    // rows; shared: up to 8 tokens x 16 rows), as in the gate/up kernel
+    static constexpr int NB = NS + 2;
+    static constexpr int kRedPer = NT == 1 ? 64 : 128;
+    static constexpr int kRedFloats = NB * CW * kRedPer;
 };
 
 // k steps (64 columns) per routed down chunk for an entry of ns slots: codes,
@@ -915,7 +1068,7 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
     __shared__ Pipe P;
     __shared__ Routing Rt;
     __shared__ int s_last;
-    __shared__ int s_cnt[C::NB];      // warps done with the task that uses each reduction buffer
+    __shared__ RedRing RR;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     const int H = D.H, I = D.I, k = D.k;
@@ -927,15 +1080,22 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
 
     pipe_init(P, NS, CW);
     if (tid < 16) reinterpret_cast<uint32_t*>(zero)[tid] = 0u;
-    if (tid < C::NB) s_cnt[tid] = 0;
-    if (warp == CW)   // ids final: the router grid is complete
-        build_routing_warp(Rt, ws.ids, n, k, TPB, ws.probe == 1 ? 1 : (ws.probe == 2 ? 2 : 0), ws.probe_e);
+    if (tid < kMaxRedBufs) RR.cnt[tid] = RR.task[tid] = RR.freed[tid] = 0;
+    if (tid == 0) RR.exits = RR.ntasks = 0;
+    if (warp == CW) {   // ids published by the router (probe calls route by themselves)
+        if (ws.probe || wait_flag(ws.route_ready, ws.err)) {
+            build_routing_warp(Rt, ws.ids, n, k, TPB, ws.probe == 1 ? 1 : (ws.probe == 2 ? 2 : 0), ws.probe_e);
+        } else if (lane == 0) {
+            Rt.nu = 0;
+        }
+    }
     __syncthreads();
     const int total = n_sh + Rt.nu * rb_per_e;
 
     if (warp == CW) {
         // ------------------------------------------------ producer warp
-        griddep_wait();   // h of the gate/up grid is copied along with the weights
+        // h comes from the gate/up grid, still running on other SMs: each task first waits until the
+        // gate/up tasks producing its h have published it (counters in gu_done)
         const uint64_t pol = policy_evict_first();
         uint32_t it = 0;
         int next = 0;
@@ -954,6 +1114,11 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
                 ck = down_chunk_ksteps(nkt, nsb, ns);
             }
             const int nch = sh ? nch_sh : nkt / ck;
+            if (!ws.probe) {
+                const bool ok = sh ? wait_count(ws.gu_done, (uint32_t)(I / 8), ws.err)
+                                   : wait_count(ws.gu_done + 1 + u, (uint32_t)(I / 32), ws.err);
+                if (!ok) { set_abort(P); break; }
+            }
             for (int c = 0; c < nch; ++c) {
                 const int s = it % NS;
                 const uint32_t ph = (it / NS) & 1;
@@ -1004,7 +1169,7 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
             }
         }
         producer_finish(P, it, NS, ws.err);
-    } else {
+    } else if (warp < CW) {
         // ------------------------------------------------ consumer warps
         const uint32_t rot = (5u - 2u * (uint32_t)t) & 31u;   // code t of each byte to bits 5..6
         const int jB = g >> 1, pB = g & 1;                    // routed B lanes: sub-block, piece
@@ -1099,17 +1264,16 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
                         const float a41 = fmaf(__uint_as_float(0x4b000000u | (b1 & 15u)), 4.f * d1, -33554432.f * d1);
                         const float mm0 = fmaf(__uint_as_float(0x4b000000u | ((b0 >> 4) & 15u)), m0, -8388608.f * m0);
                         const float mm1 = fmaf(__uint_as_float(0x4b000000u | ((b1 >> 4) & 15u)), m1, -8388608.f * m1);
+                        // no branch on the entry's slot count: an absent slot's h and S are zero
 #pragma unroll
                         for (int q = 0; q < TPB; ++q) {
-                            if (q < tcount) {
-                                float Dv[4] = {0.f, 0.f, 0.f, 0.f};
+                            float Dv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                                for (int j = 0; j < 4; ++j) bmma(Dv, Af[j], jB == j ? Bl[q] : make_uint2(0u, 0u));
-                                A.rt[q][T][0] = fmaf(a40, (Dv[0] + Dv[1]) - S[q], A.rt[q][T][0]);
-                                A.rt[q][T][0] = fmaf(-mm0, S[q], A.rt[q][T][0]);
-                                A.rt[q][T][1] = fmaf(a41, (Dv[2] + Dv[3]) - S[q], A.rt[q][T][1]);
-                                A.rt[q][T][1] = fmaf(-mm1, S[q], A.rt[q][T][1]);
-                            }
+                            for (int j = 0; j < 4; ++j) bmma(Dv, Af[j], jB == j ? Bl[q] : make_uint2(0u, 0u));
+                            A.rt[q][T][0] = fmaf(a40, (Dv[0] + Dv[1]) - S[q], A.rt[q][T][0]);
+                            A.rt[q][T][0] = fmaf(-mm0, S[q], A.rt[q][T][0]);
+                            A.rt[q][T][1] = fmaf(a41, (Dv[2] + Dv[3]) - S[q], A.rt[q][T][1]);
+                            A.rt[q][T][1] = fmaf(-mm1, S[q], A.rt[q][T][1]);
                         }
                     }
                 }
@@ -1117,17 +1281,19 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&P.empty[s]);
             if (inf.chunk == inf.nchunk - 1) {
-                // task epilogue: this warp's partials into the task's reduction buffer; the last warp to
-                // arrive sums them in warp order and stores y
+                // task end: this warp's partials into the task's reduction buffer (the epilogue warp
+                // finishes the task)
                 const int b = (int)(ntask % C::NB);
-                ++ntask;
-                float* rbuf = red + (size_t)b * CW * 128;
+                if (!ring_acquire(RR, b, (int)(ntask / C::NB), ws.err)) { set_abort(P); break; }
+                float* rbuf = red + (size_t)b * CW * C::kRedPer + warp * C::kRedPer;
                 if (sh) {
                     // this lane's token is 4 tg + t (its columns 2t, 2t+1 are that token's two pieces)
 #pragma unroll
                     for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) {
-                        rbuf[warp * 128 + (4 * tg + t) * 16 + g] = A.sh[tg][0] + A.sh[tg][1];
-                        rbuf[warp * 128 + (4 * tg + t) * 16 + g + 8] = A.sh[tg][2] + A.sh[tg][3];
+                        if (4 * tg + t < n) {
+                            rbuf[(4 * tg + t) * 16 + g] = A.sh[tg][0] + A.sh[tg][1];
+                            rbuf[(4 * tg + t) * 16 + g + 8] = A.sh[tg][2] + A.sh[tg][3];
+                        }
                     }
                 } else {
 #pragma unroll
@@ -1139,42 +1305,43 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
                                 float v = A.rt[q][T][r];
                                 v += __shfl_xor_sync(0xffffffffu, v, 1);
                                 v += __shfl_xor_sync(0xffffffffu, v, 2);
-                                if (t == 0) rbuf[warp * 128 + q * 32 + 16 * T + g + 8 * r] = v;
+                                if (t == 0) rbuf[q * 32 + 16 * T + g + 8 * r] = v;
                             }
                         }
                     }
                 }
                 __syncwarp();
-                int last = 0;
-                if (lane == 0) {
-                    __threadfence_block();
-                    last = atomicAdd(&s_cnt[b], 1) == CW - 1;
-                }
-                if (__shfl_sync(0xffffffffu, last, 0)) {
-                    __threadfence_block();
-                    if (sh) {
-                        for (int q = lane; q < 16 * n; q += 32) {   // (token, row) pairs
-                            const int tok = q >> 4, row = q & 15;
-                            float y = 0.f;
-                            for (int w = 0; w < CW; ++w) y += rbuf[w * 128 + tok * 16 + row];
-                            (ws.probe ? ws.probe_out : ws.y_sh)[(size_t)tok * H + 16 * inf.task + row] = y;
-                        }
-                    } else {
-                        const int tt = inf.task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
-                        const int s0 = Rt.ustart[u];
-                        for (int q = 0; q < tcount; ++q) {
-                            float y = 0.f;
-                            for (int w = 0; w < CW; ++w) y += rbuf[w * 128 + q * 32 + lane];
-                            const int slot = Rt.slot[s0 + q];
-                            if (ws.probe) ws.probe_out[(size_t)(slot / k) * H + 32 * rb + lane] = y;
-                            else ws.y_rt[(size_t)slot * H + 32 * rb + lane] = y;
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) s_cnt[b] = 0;
-                }
+                if (lane == 0) ring_publish(RR, b, inf.task);
+                ++ntask;
             }
             ++it;
+        }
+        if (lane == 0) ring_exit(RR, (int)ntask);
+    } else {
+        // ------------------------------------------------ epilogue warp
+        for (uint32_t j = 0; ring_take(RR, j, C::NB, CW, ws.err); ++j) {
+            const int b = (int)(j % C::NB);
+            const float* rbuf = red + (size_t)b * CW * C::kRedPer;
+            const int task = RR.task[b];
+            if (task < n_sh) {
+                for (int q = lane; q < 16 * n; q += 32) {   // (token, row) pairs
+                    const int tok = q >> 4, row = q & 15;
+                    float y = 0.f;
+                    for (int w = 0; w < CW; ++w) y += rbuf[w * C::kRedPer + tok * 16 + row];
+                    (ws.probe ? ws.probe_out : ws.y_sh)[(size_t)tok * H + 16 * task + row] = y;
+                }
+            } else {
+                const int tt = task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
+                const int s0 = Rt.ustart[u], ns = Rt.ustart[u + 1] - s0;
+                for (int q = 0; q < ns; ++q) {
+                    float y = 0.f;
+                    for (int w = 0; w < CW; ++w) y += rbuf[w * C::kRedPer + q * 32 + lane];
+                    const int slot = Rt.slot[s0 + q];
+                    if (ws.probe) ws.probe_out[(size_t)(slot / k) * H + 32 * rb + lane] = y;
+                    else ws.y_rt[(size_t)slot * H + 32 * rb + lane] = y;
+                }
+            }
+            ring_free(RR, j, C::NB);
         }
     }
     griddep_launch();
@@ -1185,7 +1352,13 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
         if (s_last) {
             *ws.queue2 = 0;
             *ws.done2 = 0;
+            *ws.route_ready = 0;
         }
+    }
+    // the last CTA also clears the gate/up completion counters for the next forward
+    __syncthreads();
+    if (s_last && !ws.probe) {
+        for (int i = tid; i < 1 + kMaxSlots; i += blockDim.x) ws.gu_done[i] = 0;
     }
 }
 
@@ -1323,7 +1496,8 @@ cudaError_t launch_wait_selftest(uint32_t* err, cudaStream_t st) {
 template <int NT>
 size_t gateup_smem_bytes(const Dims& D, int n) {
     using C = GateUpCfg<NT>;
-    return (size_t)C::NS * kStageBytes + 4 * ((size_t)C::kTabWords + C::kRedFloats) + (size_t)n * D.H * 4 + 64;
+    return (size_t)C::NS * kStageBytes + 4 * ((size_t)C::kTabWords + C::kRedFloats) +
+           (size_t)(C::kSplitX ? 2 : 1) * n * D.H * 4 + 64;
 }
 
 template <int NT>

@@ -152,7 +152,7 @@ struct ds4moe {
         const size_t H = D.H, I = D.I, E = D.E, k = D.k;
         const size_t nd = (size_t)(cap < decode_max ? cap : decode_max);
         size_t o = 0;
-        w.hdr = o; o += 256;
+        w.hdr = o; o += 1024;   // 256 words: control words 0..7, gate/up completion counters from word 16
         w.logits = o; o += align256(nd * E * 4);
         w.ids = o; o += align256(nd * k * 4);
         w.wts = o; o += align256(nd * k * 4);
@@ -225,6 +225,7 @@ struct ds4moe {
         w.done2 = hdr + 5;
         w.grid_refused = hdr + 6;
         w.route_ready = hdr + 7;
+        w.gu_done = hdr + 16;
         w.logits = reinterpret_cast<float*>(ws + L.logits);
         w.ids = reinterpret_cast<int32_t*>(ws + L.ids);
         w.wts = reinterpret_cast<float*>(ws + L.wts);

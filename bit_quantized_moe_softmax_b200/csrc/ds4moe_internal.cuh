@@ -86,7 +86,9 @@ struct DecodeWs {
     uint32_t* done1;        // gate/up CTAs finished (the last one resets queue1)
     uint32_t* done2;        // down CTAs finished (the last one resets queue2)
     uint32_t* grid_refused; // this call's gate/up grid refused the grid (too many or too large magnitudes): 1, else 0
-    uint32_t* route_ready;  // set by the router once ids / weights are written; reset by the gate/up grid
+    uint32_t* route_ready;  // set by the router once ids / weights are written; reset by the down grid
+    uint32_t* gu_done;      // gate/up tasks finished, h stored: [0] shared (of I/8), [1 + u] routed entry u
+                            //   (of I/32); the down grid waits on them; its last CTA resets them
     float* logits;          // [n][E]
     int32_t* ids;           // [n][k]
     float* wts;             // [n][k]
@@ -291,6 +293,22 @@ __device__ __forceinline__ void bulk_load_plain(void* dst, const void* src, uint
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
                  : "memory");
+}
+
+// L2 prefetch of bytes at p (16-byte aligned, a multiple of 16 bytes); no completion to wait for.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Part `part` of `nparts` of a region (16-byte aligned start) prefetched into L2 in pieces of at most
+// 64 KB; the parts are 256-byte aligned and the region's last partial 16 bytes are left out.
+__device__ inline void prefetch_share(const void* base, size_t bytes, int part, int nparts) {
+    const size_t per = ((bytes + nparts - 1) / nparts + 255) & ~(size_t)255;
+    const size_t lo = (size_t)part * per;
+    if (lo >= bytes) return;
+    const size_t hi = (lo + per < bytes ? lo + per : bytes) & ~(size_t)15;
+    for (size_t o = lo; o < hi; o += 65536)
+        prefetch_l2(static_cast<const unsigned char*>(base) + o, (uint32_t)(hi - o < 65536 ? hi - o : 65536));
 }
 
 __device__ __forceinline__ uint64_t policy_evict_first() {
