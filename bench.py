@@ -85,8 +85,9 @@ def algorithmic_bytes(w: dict, U: int) -> dict:
     sh_gu, sh_d = 2 * I * H * 2, H * I * 2
     return {
         "k_router_decode": E * H * 4 + n * H * 4 + n * E * 4,
-        "k_gateup_decode": U * 2 * iq2 + sh_gu + n * H * 4 + (n * k + n) * I * 4,
-        "k_down_decode": U * q2 + sh_d + (n * k + n) * I * 4 + (n * k + n) * H * 4,
+        # gate/up and down in one kernel: every selected expert and the shared expert once, x in, h out and
+        # back in (two bf16 pieces per value), y out
+        "k_moe_decode": U * (2 * iq2 + q2) + sh_gu + sh_d + n * H * 4 + 2 * (n * k + n) * I * 4 + (n * k + n) * H * 4,
         "k_combine_decode": (n * k + n) * H * 4 + n * H * 4,
         "routed": U * (2 * iq2 + q2),
         # prefill GEMMs (U = experts touched): weights once, permuted activations in, results out

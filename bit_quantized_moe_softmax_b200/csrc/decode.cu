@@ -1,30 +1,34 @@
-// decode.cu -- the decode plan for 1..decode_max tokens (four launches).
+// decode.cu -- the decode plan for 1..decode_max tokens (three launches).
 //
 //   k_router_decode  one warp per expert row, logits in the canonical binary32
 //                    order; the last CTA picks the top-k by (logit desc,
 //                    index asc) and the softmax over the selected logits.
-//   k_gateup_decode  h = silu(W_gate x) * (W_up x) for every selected expert
-//                    (read once, applied to every token that chose it) and for
-//                    the shared expert.
-//   k_down_decode    y = W_down h per selected expert and for the shared
-//                    expert.
+//   k_moe_decode     h = silu(W_gate x) * (W_up x), then y = W_down h, for
+//                    every selected expert (read once, applied to every token
+//                    that chose it) and for the shared expert.
 //   k_combine_decode out = y_shared + sum_j w_j y_j in rank order (then
 //                    x + that for the residual step; k_combine_steer_decode
 //                    also steers: y - F v (v . y)).
 //
-// The two projection kernels are persistent (one CTA per SM): a producer warp
-// pulls row tasks from an atomic queue and streams their weights into a ring
-// of shared-memory stages with bulk copies (cp.async.bulk + mbarrier); the
-// consumer warps turn the packed weights into exact small integers in
-// registers and multiply them on the tensor cores with warp-level MMAs, so the
-// per-weight work is the unpacking alone:
+// k_moe_decode is persistent (one CTA per SM).  A producer warp pulls tasks
+// from an atomic queue -- gate/up tasks (shared-expert 8-row groups, then
+// (expert, 32-row block) pieces), then down tasks (shared-expert 16-row
+// groups, then (expert, 32-row block) pieces) -- and streams their weights
+// into a ring of shared-memory stages with bulk copies (cp.async.bulk +
+// mbarrier).  A down task first waits (bounded) until the gate/up tasks that
+// produce its h have published it through completion counters.  The consumer
+// warps turn the packed weights into exact small integers in registers and
+// multiply them on the tensor cores with warp-level MMAs, so that the
+// per-weight work is the unpacking alone; an epilogue warp sums the consumer
+// warps' partial results of each task in a fixed order and finishes it:
 //   IQ2 (gate, up): each 8-weight chunk becomes eight int8 values +-G by two
 //     byte permutes whose selectors come from two shared-memory tables (grid
-//     row -> magnitude classes, 7 sign bits -> sign flags with the parity of
-//     the eighth folded in); x enters as four int8 pieces of a per-token
-//     power-of-two scale (29 bits of precision), the int32 products of a
-//     32-weight group are scaled by its odd integer 2s+1 in int32, and every
-//     superblock's sum is converted once and scaled by d/8.
+//     row -> magnitude classes, sign byte -> sign flags with the parity of
+//     the eighth folded in), addressed by one byte permute each; x enters as
+//     four int8 pieces of a per-token power-of-two scale (29 bits of
+//     precision), the int32 products of a 32-weight group are scaled by its
+//     odd integer 2s+1 in int32, and every superblock's sum is converted once
+//     and scaled by d/8.
 //   Q2 (down): codes become the bfloat16 numbers 1 + q/4 by a rotate, a mask
 //     and two byte permutes; h enters as two bfloat16 pieces (hi, lo); each
 //     16-weight sub-block's result is 4 d sc (D - S) - dmin m S with D its
@@ -34,10 +38,10 @@
 // The MMA's eight accumulator columns hold (token, piece) pairs or, when an
 // expert serves one token, different 32-weight groups (IQ2) or 16-weight
 // sub-blocks (Q2) of that token, so that their scales are applied once per
-// several MMAs.  Each kernel is launched with programmatic dependent launch:
-// the gate/up grid starts its shared-expert tasks while the router still runs,
-// and the down grid streams its weights while gate/up finishes; both wait
-// (griddepcontrol.wait) only where they read the previous grid's results.
+// several MMAs.  k_moe_decode is launched with programmatic dependent launch:
+// it starts its shared-expert tasks while the router still runs and takes the
+// routing from the router's ready flag; the combine waits for it
+// (griddepcontrol.wait).
 #include <map>
 #include <mutex>
 #include <utility>
@@ -125,7 +129,7 @@ __global__ void __launch_bounds__(RouterCfg<NT>::kWarps * 32)
     k_router_decode(Weights W, Dims D, DecodeWs ws, const void* x, int n, uint32_t* ready) {
     using C = RouterCfg<NT>;
     constexpr int TW = C::TW, TPW = C::TPW, RW = C::kWarps;
-    griddep_launch();   // the gate/up grid may start its shared-expert work now
+    griddep_launch();   // the projection grid may start its shared-expert work now
     extern __shared__ __align__(128) unsigned char r_smem[];   // [kRE][H] f32 rows, then x as given [n][H]
     __shared__ uint64_t bar;
     __shared__ bool s_last;
@@ -575,9 +579,31 @@ struct GateUpAcc {
     float rt[GateUpCfg<NT>::TPB][4][2];       // routed task: [token][tile][row g, g + 8]
 };
 
+// ---------------------------------------------------------------- down projection pieces
+// k steps (64 columns) per routed down chunk for an entry of ns slots: codes,
+// scales, (d, dmin) and the slots' h pieces (and per-16 sums) for those
+// columns must fit one stage.
+__device__ __forceinline__ int down_chunk_ksteps(int nkt, int nsb, int ns) {
+    // the largest of 32, 16, 8, 4 that divides the k steps (I / 64: a multiple of 4 for I >= 256)
+    int ck = nkt % 32 == 0 ? 32 : nkt % 16 == 0 ? 16 : nkt % 8 == 0 ? 8 : nkt % 4 == 0 ? 4 : nkt;
+    for (; ck > 1 && ck % 2 == 0; ck >>= 1) {
+        const int nsbc = nsb > 1 ? (ck + 3) / 4 : 1;
+        if (ck * 640 + nsbc * 128 + ns * ck * 272 <= kStageBytes) break;
+    }
+    return ck;
+}
+
+template <int NT>
+struct DownAcc {
+    static constexpr int TG = (NT + 3) / 4;
+    float sh[TG][4];                           // shared task: [token group][fragment]
+    float rt[GateUpCfg<NT>::TPB][2][2];          // routed task: [token][tile][row g, g + 8]
+};
+
+
 template <int NT>
 __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
-    k_gateup_decode(Weights W, Dims D, DecodeWs ws, const void* x, int n) {
+    k_moe_decode(Weights W, Dims D, DecodeWs ws, const void* x, int n) {
     using C = GateUpCfg<NT>;
     constexpr int NS = C::NS, CW = C::CW, R = C::R, TPB = C::TPB, kThreads = C::kThreads;
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -600,13 +626,22 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     const int g = lane >> 2, t = lane & 3;
     const int H = D.H, I = D.I, k = D.k;
     const int nkt = H / 64, nsb = H / 256;
-    const int n_sh = ws.probe == 1 ? 0 : (D.has_shared ? I / 8 : 0);   // shared tasks: 8 rows of gate and up
+    // which projections this call runs: the forward runs both; the inspection probes run one
+    const bool do_gu = (ws.stages & 1) != 0, do_dn = (ws.stages & 2) != 0;
+    const int n_sh = !do_gu || ws.probe == 1 ? 0 : (D.has_shared ? I / 8 : 0);   // shared tasks: 8 rows of gate and up
     const int rb_per_e = I / 32;
     // k steps (64 columns) per routed chunk: the largest of 32, 16, 8, 4 that divides H / 64
     const int ck_rt = nkt % 32 == 0 ? 32 : nkt % 16 == 0 ? 16 : nkt % 8 == 0 ? 8 : 4;
     const int nch_rt = nkt / ck_rt;
     const int kcs = H < 1024 ? H : 1024;              // columns per shared chunk
     const int nch_sh = H / kcs;
+    // down projection: tasks of 16 shared-expert rows, then (entry, 32-row block), numbered after the
+    // gate/up tasks; a task first waits until the gate/up tasks producing its h are done
+    const int dnkt = I / 64, dnsb = I >= 256 ? I / 256 : 1;
+    const int dn_sh = !do_dn || ws.probe == 1 ? 0 : (D.has_shared ? H / 16 : 0);
+    const int drb = H / 32;
+    const int dkcs = I < 512 ? I : 512;   // columns per shared-expert chunk
+    const int dnch_sh = I / dkcs;
 
     pipe_init(P, NS, CW);
     // ---- grid tables (made when the grid was loaded)
@@ -633,7 +668,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
         float mx[NT];
 #pragma unroll
         for (int q = 0; q < NT; ++q) mx[q] = 0.f;
-        for (int i = tid * 4; i < H; i += kThreads * 4) {
+        for (int i = tid * 4; do_gu && i < H; i += kThreads * 4) {
 #pragma unroll
             for (int q = 0; q < NT; ++q) {
                 if (q < n) {
@@ -677,7 +712,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             for (int p = 0; p < 4; ++p) s_cs[tid][p] = s_tokmax[tid] > 0.f ? ldexpf(1.f, e - 7 - 7 * p) : 0.f;
         }
         __syncthreads();
-        if (C::kSplitX) {
+        if (C::kSplitX && do_gu) {
             quantize_x(x, D.act_bf16, n, H, s_f, xq, tid, kThreads);
             __syncthreads();
         }
@@ -696,22 +731,23 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
         // first then).
         const int lead = !C::kSplitX ? n_sh : (n_sh < (int)gridDim.x ? n_sh : (int)gridDim.x);
         int nxt = 0, nxt2 = 0;
+        int d_total = 0;
         auto route = [&]() {
             build_routing_warp(Rt, ws.ids, n, k, TPB, ws.probe == 1 ? 1 : (ws.probe == 2 ? 2 : 0), ws.probe_e);
             routed = true;
-            total = n_sh + Rt.nu * rb_per_e;
-            griddep_launch();                 // the down grid may start streaming
+            total = n_sh + (do_gu ? Rt.nu * rb_per_e : 0);
+            d_total = dn_sh + (do_dn ? Rt.nu * drb : 0);
         };
         if (lane == 0) {
-            nxt = (int)atomicAdd(ws.queue1, 1u);
-            nxt2 = (int)atomicAdd(ws.queue1, 1u);
+            nxt = (int)atomicAdd(ws.queue, 1u);
+            nxt2 = (int)atomicAdd(ws.queue, 1u);
         }
         for (;;) {
             if (aborted(P) || refused) break;
             const int pos = __shfl_sync(0xffffffffu, nxt, 0);
             if (lane == 0) {
                 nxt = nxt2;
-                nxt2 = (int)atomicAdd(ws.queue1, 1u);   // in flight while this task streams
+                nxt2 = (int)atomicAdd(ws.queue, 1u);   // in flight while this task streams
             }
             if (pos >= lead && !routed) {
                 // the router's ids and weights: published by its last CTA through the ready flag (probe
@@ -719,8 +755,75 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                 if (!ws.probe && !wait_flag(ws.route_ready, ws.err)) { set_abort(P); break; }
                 route();
             }
+            if (pos >= total) {
+                // down-projection task pos - total
+                const int dt = pos - total;
+                if (dt >= d_total) break;
+            const bool dsh = dt < dn_sh;
+            int u = 0, rb = 0, ns = 0, ck = 0;
+            if (!dsh) {
+                u = (dt - dn_sh) / drb;
+                rb = (dt - dn_sh) % drb;
+                ns = Rt.ustart[u + 1] - Rt.ustart[u];
+                ck = down_chunk_ksteps(dnkt, dnsb, ns);
+            }
+            const int nch = dsh ? dnch_sh : dnkt / ck;
+            if (!ws.probe) {
+                const bool ok = dsh ? wait_count(ws.gu_done, (uint32_t)(I / 8), ws.err)
+                                   : wait_count(ws.gu_done + 1 + u, (uint32_t)(I / 32), ws.err);
+                if (!ok) { set_abort(P); break; }
+            }
+            for (int c = 0; c < nch; ++c) {
+                const int s = it % NS;
+                const uint32_t ph = (it / NS) & 1;
+                if (!mbar_wait(&P.empty[s], ph ^ 1, ws.err)) { set_abort(P); break; }
+                if (lane == 0) {
+                    unsigned char* st = stages + s * kStageBytes;
+                    if (dsh) {
+                        // 16 rows of the shared down matrix (two 8-row groups of core-matrix tiles),
+                        // columns c*dkcs .. +dkcs, then every token's h pieces for those columns
+                        const int kc0 = c * dkcs;
+                        const uint32_t abytes = dkcs * 16, hbytes = dkcs * 4;
+                        P.info[s] = ChunkInfo{total + dt, c, nch, kc0, dkcs};
+                        mbar_arrive_expect_tx(&P.full[s], 2 * abytes + n * hbytes);
+#pragma unroll
+                        for (int q = 0; q < 2; ++q)
+                            bulk_load(st + q * abytes, W.sh_down + ((size_t)(dt * 2 + q) * (I / 8) + kc0 / 8) * 64,
+                                      abytes, &P.full[s], pol);
+                        for (int q = 0; q < n; ++q)
+                            bulk_load_plain(st + 2 * abytes + q * hbytes, ws.hb_sh + ((size_t)q * (I / 64) + kc0 / 64) * 128,
+                                            hbytes, &P.full[s]);
+                    } else {
+                        const int e = Rt.uniq[u], s0 = Rt.ustart[u];
+                        const int kt0 = c * ck;
+                        const int sb0 = dnsb > 1 ? kt0 / 4 : 0, nsbc = dnsb > 1 ? (ck + 3) / 4 : 1;
+                        const uint32_t qb = ck * 512, sb = ck * 128, dbb = nsbc * 128;
+                        const uint32_t hb = ck * 256, hsb = ck * 16;
+                        P.info[s] = ChunkInfo{total + dt, c, nch, kt0, ck};
+                        mbar_arrive_expect_tx(&P.full[s], qb + sb + dbb + ns * (hb + hsb));
+                        bulk_load(st, W.down_q + (size_t)e * W.q2_q_stride + ((size_t)rb * dnkt + kt0) * 512, qb,
+                                  &P.full[s], pol);
+                        bulk_load(st + qb, W.down_sc + (size_t)e * W.q2_sc_stride + ((size_t)rb * dnkt + kt0) * 32,
+                                  sb, &P.full[s], pol);
+                        bulk_load(st + qb + sb,
+                                  W.down_dd + (size_t)e * W.q2_dd_stride + ((size_t)rb * dnsb + sb0) * 32, dbb,
+                                  &P.full[s], pol);
+                        unsigned char* hdst = st + qb + sb + dbb;
+                        for (int q = 0; q < ns; ++q) {
+                            const int slot = Rt.slot[s0 + q];
+                            bulk_load_plain(hdst + q * hb, ws.hb_rt + ((size_t)slot * (I / 64) + kt0) * 128, hb,
+                                            &P.full[s]);
+                            bulk_load_plain(hdst + ns * hb + q * hsb, ws.hsum_rt + (size_t)slot * (I / 16) + 4 * kt0,
+                                            hsb, &P.full[s]);
+                        }
+                    }
+                }
+                __syncwarp();
+                ++it;
+            }
+                continue;
+            }
             const int task = pos < lead ? pos : task_at(pos, lead, n_sh, total - n_sh);
-            if (task >= total) break;
             const bool sh = task < n_sh;
             const int nch = sh ? nch_sh : nch_rt;
             for (int c = 0; c < nch; ++c) {
@@ -771,9 +874,13 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
         const uint32_t clo = s_cand[0], chi = s_cand[1];
         // B operand lanes: column g of the MMA
         const int jB = g >> 2, pB = g & 3;                // routed: 32-column group, int8 piece
+        const uint32_t rot = (5u - 2u * (uint32_t)t) & 31u;   // down: code t of each byte to bits 5..6
+        const int jD = g >> 1, pD = g & 1;                    // down, routed B lanes: sub-block, piece
         uint32_t it = 0, cph = 0, ntask = 0;
         bool quantized = false;
         GateUpAcc<NT> A;
+        DownAcc<NT> A2;
+        int dtcount = 0;
         int tokrow[TPB];
         int tcount = 0;
         for (;;) {
@@ -782,6 +889,146 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             const ChunkInfo inf = P.info[s];
             if (inf.task < 0 || aborted(P)) break;
             const unsigned char* st = stages + s * kStageBytes;
+            const int T_gu = inf.task < n_sh ? n_sh : n_sh + (do_gu ? Rt.nu * rb_per_e : 0);
+            if (inf.task >= T_gu) {
+                // ---- down projection
+            const int dt = inf.task - T_gu;
+            const bool dsh = dt < dn_sh;
+            if (dsh) {
+                if (inf.chunk == 0) {
+#pragma unroll
+                    for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) A2.sh[tg][0] = A2.sh[tg][1] = A2.sh[tg][2] = A2.sh[tg][3] = 0.f;
+                }
+                const int kc = inf.cnt;
+                const unsigned char* hst = st + 2 * kc * 16;
+                for (int ks = warp; ks < kc / 16; ks += CW) {
+                    uint2 B[DownAcc<NT>::TG];
+#pragma unroll
+                    for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) {
+                        const int tk = 4 * tg + (g >> 1), p = g & 1;
+                        B[tg] = *reinterpret_cast<const uint2*>(
+                            tk < n ? hst + (size_t)tk * kc * 4 + ((ks >> 2) * 2 + p) * 128 + ((ks & 3) * 16 + 4 * t) * 2
+                                   : zero);
+                    }
+                    {
+                        const unsigned char* base = st + (2 * ks + (t >> 1)) * 128 + g * 16 + (t & 1) * 8;
+                        const uint2 r0 = *reinterpret_cast<const uint2*>(base);
+                        const uint2 r1 = *reinterpret_cast<const uint2*>(base + kc * 16);
+                        const uint32_t Af[4] = {r0.x, r1.x, r0.y, r1.y};
+#pragma unroll
+                        for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) bmma(A2.sh[tg], Af, B[tg]);
+                    }
+                }
+            } else {
+                const int tt = dt - dn_sh, u = tt / drb;
+                const int s0 = Rt.ustart[u], ns = Rt.ustart[u + 1] - s0;
+                if (inf.chunk == 0) {
+                    dtcount = ns;
+#pragma unroll
+                    for (int q = 0; q < TPB; ++q)
+#pragma unroll
+                        for (int T = 0; T < 2; ++T) A2.rt[q][T][0] = A2.rt[q][T][1] = 0.f;
+                }
+                const int ck = inf.cnt;
+                const int nsbc = dnsb > 1 ? (ck + 3) / 4 : 1;
+                const unsigned char* qv = st;
+                const uint32_t* scv = reinterpret_cast<const uint32_t*>(st + ck * 512);
+                const uint32_t* ddv = reinterpret_cast<const uint32_t*>(st + ck * 640);
+                const uint16_t* hst = reinterpret_cast<const uint16_t*>(st + ck * 640 + nsbc * 128);
+                const float* hss = reinterpret_cast<const float*>(st + ck * 640 + nsbc * 128 + ns * ck * 256);
+                for (int kt = warp; kt < ck; kt += CW) {
+                    const int sbi = dnsb > 1 ? ((inf.lo + kt) >> 2) - (inf.lo >> 2) : 0;   // superblock in the stage
+                    uint2 Bl[TPB];
+                    float S[TPB];
+#pragma unroll
+                    for (int q = 0; q < TPB; ++q) {
+                        Bl[q] = make_uint2(0u, 0u);
+                        S[q] = 0.f;
+                        if (q < dtcount) {
+                            Bl[q] = *reinterpret_cast<const uint2*>(hst + (size_t)q * ck * 128 + (kt * 2 + pD) * 64 + 16 * jD + 4 * t);
+                            S[q] = hss[q * ck * 4 + kt * 4 + t];
+                        }
+                    }
+#pragma unroll
+                    for (int T = 0; T < 2; ++T) {
+                        const int rg = 16 * T + g;
+                        const uint4 q0 = *reinterpret_cast<const uint4*>(qv + kt * 512 + rg * 16);
+                        const uint4 q1 = *reinterpret_cast<const uint4*>(qv + kt * 512 + (rg + 8) * 16);
+                        const uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w}, w1[4] = {q1.x, q1.y, q1.z, q1.w};
+                        uint32_t Af[4][4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t y0 = (__funnelshift_l(w0[j], w0[j], rot) & 0x60606060u) | 0x80808080u;
+                            const uint32_t y1 = (__funnelshift_l(w1[j], w1[j], rot) & 0x60606060u) | 0x80808080u;
+                            Af[j][0] = __byte_perm(y0, 0x3f3f3f3fu, 0x5140);
+                            Af[j][1] = __byte_perm(y1, 0x3f3f3f3fu, 0x5140);
+                            Af[j][2] = __byte_perm(y0, 0x3f3f3f3fu, 0x7362);
+                            Af[j][3] = __byte_perm(y1, 0x3f3f3f3fu, 0x7362);
+                        }
+                        // this lane's sub-block t: a4 = 4 d sc, mm = dmin m, per row
+                        const uint32_t sw0 = scv[kt * 32 + rg], sw1 = scv[kt * 32 + rg + 8];
+                        const uint32_t dd0 = ddv[sbi * 32 + rg], dd1 = ddv[sbi * 32 + rg + 8];
+                        const float d0 = half_bits(dd0 & 0xffffu), m0 = half_bits(dd0 >> 16);
+                        const float d1 = half_bits(dd1 & 0xffffu), m1 = half_bits(dd1 >> 16);
+                        const uint32_t b0 = sw0 >> (8 * t), b1 = sw1 >> (8 * t);
+                        const float a40 = fmaf(__uint_as_float(0x4b000000u | (b0 & 15u)), 4.f * d0, -33554432.f * d0);
+                        const float a41 = fmaf(__uint_as_float(0x4b000000u | (b1 & 15u)), 4.f * d1, -33554432.f * d1);
+                        const float mm0 = fmaf(__uint_as_float(0x4b000000u | ((b0 >> 4) & 15u)), m0, -8388608.f * m0);
+                        const float mm1 = fmaf(__uint_as_float(0x4b000000u | ((b1 >> 4) & 15u)), m1, -8388608.f * m1);
+                        // no branch on the entry's slot count: an absent slot's h and S are zero
+#pragma unroll
+                        for (int q = 0; q < TPB; ++q) {
+                            float Dv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) bmma(Dv, Af[j], jD == j ? Bl[q] : make_uint2(0u, 0u));
+                            A2.rt[q][T][0] = fmaf(a40, (Dv[0] + Dv[1]) - S[q], A2.rt[q][T][0]);
+                            A2.rt[q][T][0] = fmaf(-mm0, S[q], A2.rt[q][T][0]);
+                            A2.rt[q][T][1] = fmaf(a41, (Dv[2] + Dv[3]) - S[q], A2.rt[q][T][1]);
+                            A2.rt[q][T][1] = fmaf(-mm1, S[q], A2.rt[q][T][1]);
+                        }
+                    }
+                }
+            }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&P.empty[s]);
+            if (inf.chunk == inf.nchunk - 1) {
+                // task end: this warp's partials into the task's reduction buffer (the epilogue warp
+                // finishes the task)
+                const int b = (int)(ntask % C::NB);
+                if (!ring_acquire(RR, b, (int)(ntask / C::NB), ws.err)) { set_abort(P); break; }
+                float* rbuf = red + (size_t)b * CW * C::kRedPer + warp * C::kRedPer;
+                if (dsh) {
+                    // this lane's token is 4 tg + t (its columns 2t, 2t+1 are that token's two pieces)
+#pragma unroll
+                    for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) {
+                        if (4 * tg + t < n) {
+                            rbuf[(4 * tg + t) * 16 + g] = A2.sh[tg][0] + A2.sh[tg][1];
+                            rbuf[(4 * tg + t) * 16 + g + 8] = A2.sh[tg][2] + A2.sh[tg][3];
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < TPB; ++q) {
+#pragma unroll
+                        for (int T = 0; T < 2; ++T) {
+#pragma unroll
+                            for (int r = 0; r < 2; ++r) {
+                                float v = A2.rt[q][T][r];
+                                v += __shfl_xor_sync(0xffffffffu, v, 1);
+                                v += __shfl_xor_sync(0xffffffffu, v, 2);
+                                if (t == 0) rbuf[q * 32 + 16 * T + g + 8 * r] = v;
+                            }
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) ring_publish(RR, b, inf.task);
+                ++ntask;
+            }
+                ++it;
+                continue;
+            }
+            // ---- gate and up projections
             const bool sh = inf.task < n_sh;
             if (!C::kSplitX && !sh && !quantized) {
                 // first routed stage: every consumer warp is done with the shared tasks' bf16 pieces;
@@ -945,6 +1192,31 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             const int b = (int)(j % C::NB);
             const float* rbuf = red + (size_t)b * CW * C::kRedPer;
             const int task = RR.task[b];
+            const int T_gu = task < n_sh ? n_sh : n_sh + (do_gu ? Rt.nu * rb_per_e : 0);
+            if (task >= T_gu) {
+                // ---- down projection: y of the task's rows
+                const int dt = task - T_gu;
+            if (dt < dn_sh) {
+                for (int q = lane; q < 16 * n; q += 32) {   // (token, row) pairs
+                    const int tok = q >> 4, row = q & 15;
+                    float y = 0.f;
+                    for (int w = 0; w < CW; ++w) y += rbuf[w * C::kRedPer + tok * 16 + row];
+                    (ws.probe ? ws.probe_out : ws.y_sh)[(size_t)tok * H + 16 * dt + row] = y;
+                }
+            } else {
+                const int tt = dt - dn_sh, u = tt / drb, rb = tt % drb;
+                const int s0 = Rt.ustart[u], ns = Rt.ustart[u + 1] - s0;
+                for (int q = 0; q < ns; ++q) {
+                    float y = 0.f;
+                    for (int w = 0; w < CW; ++w) y += rbuf[w * C::kRedPer + q * 32 + lane];
+                    const int slot = Rt.slot[s0 + q];
+                    if (ws.probe) ws.probe_out[(size_t)(slot / k) * H + 32 * rb + lane] = y;
+                    else ws.y_rt[(size_t)slot * H + 32 * rb + lane] = y;
+                }
+            }
+                ring_free(RR, j, C::NB);
+                continue;
+            }
             const bool sh = task < n_sh;
             if (sh) {
                 for (int q = lane; q < 8 * n; q += 32) {   // (token, row) pairs
@@ -998,7 +1270,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                 }
             }
             if (!ws.probe) {
-                // h of this task is complete: publish it to the down grid (the warp barrier orders every
+                // h of this task is complete: publish it to the down tasks (the warp barrier orders every
                 // lane's stores before lane 0's fence, which is cumulative)
                 __syncwarp();
                 if (lane == 0) {
@@ -1014,344 +1286,10 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     __syncthreads();
     if (tid == 0) {
         __threadfence();
-        s_last = atomicAdd(ws.done1, 1u) == gridDim.x - 1;
+        s_last = atomicAdd(ws.done, 1u) == gridDim.x - 1;
         if (s_last) {
-            *ws.queue1 = 0;
-            *ws.done1 = 0;
-        }
-    }
-}
-
-// ---------------------------------------------------------------- down
-template <int NT>
-struct DownCfg {
-    static constexpr int NS = 4;
-    static constexpr int CW = 8;
-    static constexpr int TPB = NT == 1 ? 1 : 2;
-    static constexpr int kThreads = (CW + 2) * 32;                // + producer warp + epilogue warp
-    // task reductions: a ring of NB buffers of [warp][kRedPer] partial sums (routed: TPB tokens x 32
-    // rows; shared: up to 8 tokens x 16 rows), as in the gate/up kernel
-    static constexpr int NB = NS + 2;
-    static constexpr int kRedPer = NT == 1 ? 64 : 128;
-    static constexpr int kRedFloats = NB * CW * kRedPer;
-};
-
-// k steps (64 columns) per routed down chunk for an entry of ns slots: codes,
-// scales, (d, dmin) and the slots' h pieces (and per-16 sums) for those
-// columns must fit one stage.
-__device__ __forceinline__ int down_chunk_ksteps(int nkt, int nsb, int ns) {
-    // the largest of 32, 16, 8, 4 that divides the k steps (I / 64: a multiple of 4 for I >= 256)
-    int ck = nkt % 32 == 0 ? 32 : nkt % 16 == 0 ? 16 : nkt % 8 == 0 ? 8 : nkt % 4 == 0 ? 4 : nkt;
-    for (; ck > 1 && ck % 2 == 0; ck >>= 1) {
-        const int nsbc = nsb > 1 ? (ck + 3) / 4 : 1;
-        if (ck * 640 + nsbc * 128 + ns * ck * 272 <= kStageBytes) break;
-    }
-    return ck;
-}
-
-template <int NT>
-struct DownAcc {
-    static constexpr int TG = (NT + 3) / 4;
-    float sh[TG][4];                           // shared task: [token group][fragment]
-    float rt[DownCfg<NT>::TPB][2][2];          // routed task: [token][tile][row g, g + 8]
-};
-
-template <int NT>
-__global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
-    k_down_decode(Weights W, Dims D, DecodeWs ws, float* out, int n) {
-    using C = DownCfg<NT>;
-    constexpr int NS = C::NS, CW = C::CW, TPB = C::TPB;
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    unsigned char* stages = smem_raw;
-    float* red = reinterpret_cast<float*>(smem_raw + NS * kStageBytes);   // kRedFloats
-    unsigned char* zero = reinterpret_cast<unsigned char*>(red + C::kRedFloats);
-    __shared__ Pipe P;
-    __shared__ Routing Rt;
-    __shared__ int s_last;
-    __shared__ RedRing RR;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int H = D.H, I = D.I, k = D.k;
-    const int nkt = I / 64, nsb = I >= 256 ? I / 256 : 1;
-    const int n_sh = ws.probe == 1 ? 0 : (D.has_shared ? H / 16 : 0);   // shared tasks: 16 rows
-    const int rb_per_e = H / 32;
-    const int kcs = I < 512 ? I : 512;        // columns per shared chunk
-    const int nch_sh = I / kcs;
-
-    pipe_init(P, NS, CW);
-    if (tid < 16) reinterpret_cast<uint32_t*>(zero)[tid] = 0u;
-    if (tid < kMaxRedBufs) RR.cnt[tid] = RR.task[tid] = RR.freed[tid] = 0;
-    if (tid == 0) RR.exits = RR.ntasks = 0;
-    if (warp == CW) {   // ids published by the router (probe calls route by themselves)
-        if (ws.probe || wait_flag(ws.route_ready, ws.err)) {
-            build_routing_warp(Rt, ws.ids, n, k, TPB, ws.probe == 1 ? 1 : (ws.probe == 2 ? 2 : 0), ws.probe_e);
-        } else if (lane == 0) {
-            Rt.nu = 0;
-        }
-    }
-    __syncthreads();
-    const int total = n_sh + Rt.nu * rb_per_e;
-
-    if (warp == CW) {
-        // ------------------------------------------------ producer warp
-        // h comes from the gate/up grid, still running on other SMs: each task first waits until the
-        // gate/up tasks producing its h have published it (counters in gu_done)
-        const uint64_t pol = policy_evict_first();
-        uint32_t it = 0;
-        int next = 0;
-        if (lane == 0) next = (int)atomicAdd(ws.queue2, 1u);
-        for (;;) {
-            if (aborted(P)) break;
-            const int task = __shfl_sync(0xffffffffu, next, 0);
-            if (lane == 0) next = (int)atomicAdd(ws.queue2, 1u);   // in flight while this task streams
-            if (task >= total) break;
-            const bool sh = task < n_sh;
-            int u = 0, rb = 0, ns = 0, ck = 0;
-            if (!sh) {
-                u = (task - n_sh) / rb_per_e;
-                rb = (task - n_sh) % rb_per_e;
-                ns = Rt.ustart[u + 1] - Rt.ustart[u];
-                ck = down_chunk_ksteps(nkt, nsb, ns);
-            }
-            const int nch = sh ? nch_sh : nkt / ck;
-            if (!ws.probe) {
-                const bool ok = sh ? wait_count(ws.gu_done, (uint32_t)(I / 8), ws.err)
-                                   : wait_count(ws.gu_done + 1 + u, (uint32_t)(I / 32), ws.err);
-                if (!ok) { set_abort(P); break; }
-            }
-            for (int c = 0; c < nch; ++c) {
-                const int s = it % NS;
-                const uint32_t ph = (it / NS) & 1;
-                if (!mbar_wait(&P.empty[s], ph ^ 1, ws.err)) { set_abort(P); break; }
-                if (lane == 0) {
-                    unsigned char* st = stages + s * kStageBytes;
-                    if (sh) {
-                        // 16 rows of the shared down matrix (two 8-row groups of core-matrix tiles),
-                        // columns c*kcs .. +kcs, then every token's h pieces for those columns
-                        const int kc0 = c * kcs;
-                        const uint32_t abytes = kcs * 16, hbytes = kcs * 4;
-                        P.info[s] = ChunkInfo{task, c, nch, kc0, kcs};
-                        mbar_arrive_expect_tx(&P.full[s], 2 * abytes + n * hbytes);
-#pragma unroll
-                        for (int q = 0; q < 2; ++q)
-                            bulk_load(st + q * abytes, W.sh_down + ((size_t)(task * 2 + q) * (I / 8) + kc0 / 8) * 64,
-                                      abytes, &P.full[s], pol);
-                        for (int q = 0; q < n; ++q)
-                            bulk_load_plain(st + 2 * abytes + q * hbytes, ws.hb_sh + ((size_t)q * (I / 64) + kc0 / 64) * 128,
-                                            hbytes, &P.full[s]);
-                    } else {
-                        const int e = Rt.uniq[u], s0 = Rt.ustart[u];
-                        const int kt0 = c * ck;
-                        const int sb0 = nsb > 1 ? kt0 / 4 : 0, nsbc = nsb > 1 ? (ck + 3) / 4 : 1;
-                        const uint32_t qb = ck * 512, sb = ck * 128, dbb = nsbc * 128;
-                        const uint32_t hb = ck * 256, hsb = ck * 16;
-                        P.info[s] = ChunkInfo{task, c, nch, kt0, ck};
-                        mbar_arrive_expect_tx(&P.full[s], qb + sb + dbb + ns * (hb + hsb));
-                        bulk_load(st, W.down_q + (size_t)e * W.q2_q_stride + ((size_t)rb * nkt + kt0) * 512, qb,
-                                  &P.full[s], pol);
-                        bulk_load(st + qb, W.down_sc + (size_t)e * W.q2_sc_stride + ((size_t)rb * nkt + kt0) * 32,
-                                  sb, &P.full[s], pol);
-                        bulk_load(st + qb + sb,
-                                  W.down_dd + (size_t)e * W.q2_dd_stride + ((size_t)rb * nsb + sb0) * 32, dbb,
-                                  &P.full[s], pol);
-                        unsigned char* hdst = st + qb + sb + dbb;
-                        for (int q = 0; q < ns; ++q) {
-                            const int slot = Rt.slot[s0 + q];
-                            bulk_load_plain(hdst + q * hb, ws.hb_rt + ((size_t)slot * (I / 64) + kt0) * 128, hb,
-                                            &P.full[s]);
-                            bulk_load_plain(hdst + ns * hb + q * hsb, ws.hsum_rt + (size_t)slot * (I / 16) + 4 * kt0,
-                                            hsb, &P.full[s]);
-                        }
-                    }
-                }
-                __syncwarp();
-                ++it;
-            }
-        }
-        producer_finish(P, it, NS, ws.err);
-    } else if (warp < CW) {
-        // ------------------------------------------------ consumer warps
-        const uint32_t rot = (5u - 2u * (uint32_t)t) & 31u;   // code t of each byte to bits 5..6
-        const int jB = g >> 1, pB = g & 1;                    // routed B lanes: sub-block, piece
-        uint32_t it = 0, ntask = 0;
-        DownAcc<NT> A;
-        int tcount = 0;
-        for (;;) {
-            const int s = it % NS;
-            if (!mbar_wait(&P.full[s], (it / NS) & 1, ws.err)) { set_abort(P); break; }
-            const ChunkInfo inf = P.info[s];
-            if (inf.task < 0 || aborted(P)) break;
-            const unsigned char* st = stages + s * kStageBytes;
-            const bool sh = inf.task < n_sh;
-            if (sh) {
-                if (inf.chunk == 0) {
-#pragma unroll
-                    for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) A.sh[tg][0] = A.sh[tg][1] = A.sh[tg][2] = A.sh[tg][3] = 0.f;
-                }
-                const int kc = inf.cnt;
-                const unsigned char* hst = st + 2 * kc * 16;
-                for (int ks = warp; ks < kc / 16; ks += CW) {
-                    uint2 B[DownAcc<NT>::TG];
-#pragma unroll
-                    for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) {
-                        const int tk = 4 * tg + (g >> 1), p = g & 1;
-                        B[tg] = *reinterpret_cast<const uint2*>(
-                            tk < n ? hst + (size_t)tk * kc * 4 + ((ks >> 2) * 2 + p) * 128 + ((ks & 3) * 16 + 4 * t) * 2
-                                   : zero);
-                    }
-                    {
-                        const unsigned char* base = st + (2 * ks + (t >> 1)) * 128 + g * 16 + (t & 1) * 8;
-                        const uint2 r0 = *reinterpret_cast<const uint2*>(base);
-                        const uint2 r1 = *reinterpret_cast<const uint2*>(base + kc * 16);
-                        const uint32_t Af[4] = {r0.x, r1.x, r0.y, r1.y};
-#pragma unroll
-                        for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) bmma(A.sh[tg], Af, B[tg]);
-                    }
-                }
-            } else {
-                const int tt = inf.task - n_sh, u = tt / rb_per_e;
-                const int s0 = Rt.ustart[u], ns = Rt.ustart[u + 1] - s0;
-                if (inf.chunk == 0) {
-                    tcount = ns;
-#pragma unroll
-                    for (int q = 0; q < TPB; ++q)
-#pragma unroll
-                        for (int T = 0; T < 2; ++T) A.rt[q][T][0] = A.rt[q][T][1] = 0.f;
-                }
-                const int ck = inf.cnt;
-                const int nsbc = nsb > 1 ? (ck + 3) / 4 : 1;
-                const unsigned char* qv = st;
-                const uint32_t* scv = reinterpret_cast<const uint32_t*>(st + ck * 512);
-                const uint32_t* ddv = reinterpret_cast<const uint32_t*>(st + ck * 640);
-                const uint16_t* hst = reinterpret_cast<const uint16_t*>(st + ck * 640 + nsbc * 128);
-                const float* hss = reinterpret_cast<const float*>(st + ck * 640 + nsbc * 128 + ns * ck * 256);
-                for (int kt = warp; kt < ck; kt += CW) {
-                    const int sbi = nsb > 1 ? ((inf.lo + kt) >> 2) - (inf.lo >> 2) : 0;   // superblock in the stage
-                    uint2 Bl[TPB];
-                    float S[TPB];
-#pragma unroll
-                    for (int q = 0; q < TPB; ++q) {
-                        Bl[q] = make_uint2(0u, 0u);
-                        S[q] = 0.f;
-                        if (q < tcount) {
-                            Bl[q] = *reinterpret_cast<const uint2*>(hst + (size_t)q * ck * 128 + (kt * 2 + pB) * 64 + 16 * jB + 4 * t);
-                            S[q] = hss[q * ck * 4 + kt * 4 + t];
-                        }
-                    }
-#pragma unroll
-                    for (int T = 0; T < 2; ++T) {
-                        const int rg = 16 * T + g;
-                        const uint4 q0 = *reinterpret_cast<const uint4*>(qv + kt * 512 + rg * 16);
-                        const uint4 q1 = *reinterpret_cast<const uint4*>(qv + kt * 512 + (rg + 8) * 16);
-                        const uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w}, w1[4] = {q1.x, q1.y, q1.z, q1.w};
-                        uint32_t Af[4][4];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint32_t y0 = (__funnelshift_l(w0[j], w0[j], rot) & 0x60606060u) | 0x80808080u;
-                            const uint32_t y1 = (__funnelshift_l(w1[j], w1[j], rot) & 0x60606060u) | 0x80808080u;
-                            Af[j][0] = __byte_perm(y0, 0x3f3f3f3fu, 0x5140);
-                            Af[j][1] = __byte_perm(y1, 0x3f3f3f3fu, 0x5140);
-                            Af[j][2] = __byte_perm(y0, 0x3f3f3f3fu, 0x7362);
-                            Af[j][3] = __byte_perm(y1, 0x3f3f3f3fu, 0x7362);
-                        }
-                        // this lane's sub-block t: a4 = 4 d sc, mm = dmin m, per row
-                        const uint32_t sw0 = scv[kt * 32 + rg], sw1 = scv[kt * 32 + rg + 8];
-                        const uint32_t dd0 = ddv[sbi * 32 + rg], dd1 = ddv[sbi * 32 + rg + 8];
-                        const float d0 = half_bits(dd0 & 0xffffu), m0 = half_bits(dd0 >> 16);
-                        const float d1 = half_bits(dd1 & 0xffffu), m1 = half_bits(dd1 >> 16);
-                        const uint32_t b0 = sw0 >> (8 * t), b1 = sw1 >> (8 * t);
-                        const float a40 = fmaf(__uint_as_float(0x4b000000u | (b0 & 15u)), 4.f * d0, -33554432.f * d0);
-                        const float a41 = fmaf(__uint_as_float(0x4b000000u | (b1 & 15u)), 4.f * d1, -33554432.f * d1);
-                        const float mm0 = fmaf(__uint_as_float(0x4b000000u | ((b0 >> 4) & 15u)), m0, -8388608.f * m0);
-                        const float mm1 = fmaf(__uint_as_float(0x4b000000u | ((b1 >> 4) & 15u)), m1, -8388608.f * m1);
-                        // no branch on the entry's slot count: an absent slot's h and S are zero
-#pragma unroll
-                        for (int q = 0; q < TPB; ++q) {
-                            float Dv[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) bmma(Dv, Af[j], jB == j ? Bl[q] : make_uint2(0u, 0u));
-                            A.rt[q][T][0] = fmaf(a40, (Dv[0] + Dv[1]) - S[q], A.rt[q][T][0]);
-                            A.rt[q][T][0] = fmaf(-mm0, S[q], A.rt[q][T][0]);
-                            A.rt[q][T][1] = fmaf(a41, (Dv[2] + Dv[3]) - S[q], A.rt[q][T][1]);
-                            A.rt[q][T][1] = fmaf(-mm1, S[q], A.rt[q][T][1]);
-                        }
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&P.empty[s]);
-            if (inf.chunk == inf.nchunk - 1) {
-                // task end: this warp's partials into the task's reduction buffer (the epilogue warp
-                // finishes the task)
-                const int b = (int)(ntask % C::NB);
-                if (!ring_acquire(RR, b, (int)(ntask / C::NB), ws.err)) { set_abort(P); break; }
-                float* rbuf = red + (size_t)b * CW * C::kRedPer + warp * C::kRedPer;
-                if (sh) {
-                    // this lane's token is 4 tg + t (its columns 2t, 2t+1 are that token's two pieces)
-#pragma unroll
-                    for (int tg = 0; tg < DownAcc<NT>::TG; ++tg) {
-                        if (4 * tg + t < n) {
-                            rbuf[(4 * tg + t) * 16 + g] = A.sh[tg][0] + A.sh[tg][1];
-                            rbuf[(4 * tg + t) * 16 + g + 8] = A.sh[tg][2] + A.sh[tg][3];
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < TPB; ++q) {
-#pragma unroll
-                        for (int T = 0; T < 2; ++T) {
-#pragma unroll
-                            for (int r = 0; r < 2; ++r) {
-                                float v = A.rt[q][T][r];
-                                v += __shfl_xor_sync(0xffffffffu, v, 1);
-                                v += __shfl_xor_sync(0xffffffffu, v, 2);
-                                if (t == 0) rbuf[q * 32 + 16 * T + g + 8 * r] = v;
-                            }
-                        }
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) ring_publish(RR, b, inf.task);
-                ++ntask;
-            }
-            ++it;
-        }
-        if (lane == 0) ring_exit(RR, (int)ntask);
-    } else {
-        // ------------------------------------------------ epilogue warp
-        for (uint32_t j = 0; ring_take(RR, j, C::NB, CW, ws.err); ++j) {
-            const int b = (int)(j % C::NB);
-            const float* rbuf = red + (size_t)b * CW * C::kRedPer;
-            const int task = RR.task[b];
-            if (task < n_sh) {
-                for (int q = lane; q < 16 * n; q += 32) {   // (token, row) pairs
-                    const int tok = q >> 4, row = q & 15;
-                    float y = 0.f;
-                    for (int w = 0; w < CW; ++w) y += rbuf[w * C::kRedPer + tok * 16 + row];
-                    (ws.probe ? ws.probe_out : ws.y_sh)[(size_t)tok * H + 16 * task + row] = y;
-                }
-            } else {
-                const int tt = task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
-                const int s0 = Rt.ustart[u], ns = Rt.ustart[u + 1] - s0;
-                for (int q = 0; q < ns; ++q) {
-                    float y = 0.f;
-                    for (int w = 0; w < CW; ++w) y += rbuf[w * C::kRedPer + q * 32 + lane];
-                    const int slot = Rt.slot[s0 + q];
-                    if (ws.probe) ws.probe_out[(size_t)(slot / k) * H + 32 * rb + lane] = y;
-                    else ws.y_rt[(size_t)slot * H + 32 * rb + lane] = y;
-                }
-            }
-            ring_free(RR, j, C::NB);
-        }
-    }
-    griddep_launch();
-    __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        s_last = atomicAdd(ws.done2, 1u) == gridDim.x - 1;
-        if (s_last) {
-            *ws.queue2 = 0;
-            *ws.done2 = 0;
+            *ws.queue = 0;
+            *ws.done = 0;
             *ws.route_ready = 0;
         }
     }
@@ -1366,11 +1304,11 @@ __global__ void __launch_bounds__(DownCfg<NT>::kThreads, 1)
 // out[t][r] = y_shared[t][r] + sum_j w[t][j] y[t*k + j][r], j in rank order
 // (then x[t][r] + that, when the call asks for the residual).
 __global__ void __launch_bounds__(256) k_combine_decode(Dims D, DecodeWs ws, float* out, int n) {
-    griddep_wait();   // y of the down grid
+    griddep_wait();   // y of the projection grid
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int H = D.H, k = D.k;
     if (i >= (int64_t)n * H) return;
-    if (__ldcg(ws.grid_refused)) return;   // the gate/up grid refused the grid: out stays as it was
+    if (__ldcg(ws.grid_refused)) return;   // the projection grid refused the grid: out stays as it was
     const int t = (int)(i / H), r = (int)(i % H);
     float w[16], y[16];
 #pragma unroll
@@ -1395,10 +1333,10 @@ constexpr int kSteerThreads = 1024;   // few tokens: one wide CTA per token
 constexpr int kSteerCols = 4;          // columns per thread (H <= 4096)
 
 __global__ void __launch_bounds__(kSteerThreads) k_combine_steer_decode(Dims D, DecodeWs ws, float* out, int n) {
-    griddep_wait();   // y of the down grid
+    griddep_wait();   // y of the projection grid
     __shared__ float red[kSteerThreads / 32];
     const int t = blockIdx.x, H = D.H, k = D.k;
-    if (__ldcg(ws.grid_refused)) return;   // the gate/up grid refused the grid: out stays as it was
+    if (__ldcg(ws.grid_refused)) return;   // the projection grid refused the grid: out stays as it was
     float acc[kSteerCols];
     float dot = 0.f;
 #pragma unroll
@@ -1500,14 +1438,6 @@ size_t gateup_smem_bytes(const Dims& D, int n) {
            (size_t)(C::kSplitX ? 2 : 1) * n * D.H * 4 + 64;
 }
 
-template <int NT>
-size_t down_smem_bytes(const Dims& D, int n) {
-    using C = DownCfg<NT>;
-    (void)D;
-    (void)n;
-    return (size_t)C::NS * kStageBytes + 4 * (size_t)C::kRedFloats + 64;
-}
-
 size_t router_smem_bytes(const Dims& D, int n) {
     return (size_t)kRE * D.H * 4 + (size_t)n * D.H * (D.act_bf16 ? 2 : 4);
 }
@@ -1532,7 +1462,7 @@ struct Marks {
     }
 };
 
-const char* const kDecodeKernels[4] = {"k_router_decode", "k_gateup_decode", "k_down_decode", "k_combine_decode"};
+const char* const kDecodeKernels[3] = {"k_router_decode", "k_moe_decode", "k_combine_decode"};
 
 
 // Dynamic shared memory opt-in: raised once per (kernel, device) to the
@@ -1580,9 +1510,8 @@ template <int NT>
 cudaError_t launch_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n, float* out,
                             int n_sm, cudaStream_t st, cudaEvent_t const* ev) {
     cudaError_t err;
-    const size_t s1 = gateup_smem_bytes<NT>(D, n), s2 = down_smem_bytes<NT>(D, n);
-    if ((err = configure(k_gateup_decode<NT>)) != cudaSuccess) return err;
-    if ((err = configure(k_down_decode<NT>)) != cudaSuccess) return err;
+    const size_t s1 = gateup_smem_bytes<NT>(D, n);
+    if ((err = configure(k_moe_decode<NT>)) != cudaSuccess) return err;
     if ((err = configure(k_router_decode<NT>)) != cudaSuccess) return err;
     Marks mk(ev, st);
     const bool pdl = ev == nullptr;   // profiled runs keep the kernels apart
@@ -1592,11 +1521,7 @@ cudaError_t launch_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws,
                                                                                              ws.route_ready);
     mk.after();
     mk.before();
-    err = launch_pdl(k_gateup_decode<NT>, dim3(n_sm), dim3(GateUpCfg<NT>::kThreads), s1, st, pdl, W, D, ws, x, n);
-    mk.after();
-    if (err != cudaSuccess) return err;
-    mk.before();
-    err = launch_pdl(k_down_decode<NT>, dim3(n_sm), dim3(DownCfg<NT>::kThreads), s2, st, pdl, W, D, ws, out, n);
+    err = launch_pdl(k_moe_decode<NT>, dim3(n_sm), dim3(GateUpCfg<NT>::kThreads), s1, st, pdl, W, D, ws, x, n);
     mk.after();
     if (err != cudaSuccess) return err;
     const int64_t nel = (int64_t)n * D.H;
@@ -1610,18 +1535,18 @@ cudaError_t launch_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws,
     return cudaGetLastError();
 }
 
-int decode_launches() { return 4; }
-const char* decode_kernel_name(int i) { return (i >= 0 && i < 4) ? kDecodeKernels[i] : nullptr; }
+int decode_launches() { return 3; }
+const char* decode_kernel_name(int i) { return (i >= 0 && i < 3) ? kDecodeKernels[i] : nullptr; }
 
 // Dynamic shared memory of the larger decode kernel for n tokens, plus its
 // static shared memory (pipeline barriers, routing table).
 size_t decode_smem_bytes(const Dims& D, int n) {
-    size_t a, b;
-    if (n <= 1) { a = gateup_smem_bytes<1>(D, n); b = down_smem_bytes<1>(D, n); }
-    else if (n <= 2) { a = gateup_smem_bytes<2>(D, n); b = down_smem_bytes<2>(D, n); }
-    else if (n <= 4) { a = gateup_smem_bytes<4>(D, n); b = down_smem_bytes<4>(D, n); }
-    else { a = gateup_smem_bytes<8>(D, n); b = down_smem_bytes<8>(D, n); }
-    size_t need = (a > b ? a : b) + sizeof(Pipe) + sizeof(Routing) + 512;   // + the kernels' other static shared memory
+    size_t a;
+    if (n <= 1) a = gateup_smem_bytes<1>(D, n);
+    else if (n <= 2) a = gateup_smem_bytes<2>(D, n);
+    else if (n <= 4) a = gateup_smem_bytes<4>(D, n);
+    else a = gateup_smem_bytes<8>(D, n);
+    size_t need = a + sizeof(Pipe) + sizeof(Routing) + 512;   // + the kernel's other static shared memory
     const size_t r = router_smem_bytes(D, n) + sizeof(float) * 8 * 1024 + 64;
     return r > need ? r : need;
 }
@@ -1666,17 +1591,19 @@ template <int NT>
 cudaError_t launch_probe_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws, int which, const void* in,
                                   int n, int n_sm, cudaStream_t st) {
     cudaError_t err;
-    if (which == 0) {
-        if ((err = configure(k_gateup_decode<NT>)) != cudaSuccess) return err;
-        k_gateup_decode<NT><<<n_sm, GateUpCfg<NT>::kThreads, gateup_smem_bytes<NT>(D, n), st>>>(W, D, ws, in, n);
+    if ((err = configure(k_moe_decode<NT>)) != cudaSuccess) return err;
+    DecodeWs w = ws;
+    if (which == 0) {   // gate and up projections of x = in
+        w.stages = 1;
+        k_moe_decode<NT><<<n_sm, GateUpCfg<NT>::kThreads, gateup_smem_bytes<NT>(D, n), st>>>(W, D, w, in, n);
         return cudaGetLastError();
     }
     const int64_t nb = (int64_t)n * (D.I / 16);
     k_probe_h<<<(unsigned)((nb + 127) / 128), 128, 0, st>>>(reinterpret_cast<const float*>(in), n, D.I, D.k,
                                                             ws.probe == 2, ws.hb_rt, ws.hsum_rt, ws.hb_sh);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    if ((err = configure(k_down_decode<NT>)) != cudaSuccess) return err;
-    k_down_decode<NT><<<n_sm, DownCfg<NT>::kThreads, down_smem_bytes<NT>(D, n), st>>>(W, D, ws, nullptr, n);
+    w.stages = 2;   // down projection of h = in
+    k_moe_decode<NT><<<n_sm, GateUpCfg<NT>::kThreads, gateup_smem_bytes<NT>(D, n), st>>>(W, D, w, nullptr, n);
     return cudaGetLastError();
 }
 

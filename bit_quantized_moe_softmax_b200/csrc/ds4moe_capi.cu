@@ -219,13 +219,12 @@ struct ds4moe {
         uint32_t* hdr = reinterpret_cast<uint32_t*>(ws + L.hdr);
         w.err = hdr + 0;
         w.ticket = hdr + 1;
-        w.queue1 = hdr + 2;
-        w.queue2 = hdr + 3;
-        w.done1 = hdr + 4;
-        w.done2 = hdr + 5;
+        w.queue = hdr + 2;
+        w.done = hdr + 4;
         w.grid_refused = hdr + 6;
         w.route_ready = hdr + 7;
         w.gu_done = hdr + 16;
+        w.stages = 3;
         w.logits = reinterpret_cast<float*>(ws + L.logits);
         w.ids = reinterpret_cast<int32_t*>(ws + L.ids);
         w.wts = reinterpret_cast<float*>(ws + L.wts);
@@ -771,8 +770,7 @@ ds4moe_status ds4moe_route_noalloc(ds4moe_t* h, const void* d_x, int32_t n, int3
     DecodeWs ws{};
     ws.err = hdr + 0;
     ws.ticket = hdr + 1;
-    ws.queue1 = hdr + 2;
-    ws.queue2 = hdr + 3;
+    ws.queue = hdr + 2;
     ws.logits = base + kNoAllocHeader;
     ws.ids = d_ids;
     ws.wts = d_w;

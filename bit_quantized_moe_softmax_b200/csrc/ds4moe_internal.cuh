@@ -81,14 +81,12 @@ struct Dims {
 struct DecodeWs {
     uint32_t* err;          // device error word
     uint32_t* ticket;       // router last-CTA ticket
-    uint32_t* queue1;       // gate/up task counter
-    uint32_t* queue2;       // down task counter
-    uint32_t* done1;        // gate/up CTAs finished (the last one resets queue1)
-    uint32_t* done2;        // down CTAs finished (the last one resets queue2)
-    uint32_t* grid_refused; // this call's gate/up grid refused the grid (too many or too large magnitudes): 1, else 0
-    uint32_t* route_ready;  // set by the router once ids / weights are written; reset by the down grid
+    uint32_t* queue;        // projection task counter
+    uint32_t* done;         // projection CTAs finished (the last one resets the counters)
+    uint32_t* grid_refused; // this call's projection grid refused the grid (too many or too large magnitudes): 1, else 0
+    uint32_t* route_ready;  // set by the router once ids / weights are written; reset by the projection grid
     uint32_t* gu_done;      // gate/up tasks finished, h stored: [0] shared (of I/8), [1 + u] routed entry u
-                            //   (of I/32); the down grid waits on them; its last CTA resets them
+                            //   (of I/32); the down tasks wait on them; the last CTA resets them
     float* logits;          // [n][E]
     int32_t* ids;           // [n][k]
     float* wts;             // [n][k]
@@ -101,6 +99,7 @@ struct DecodeWs {
     const void* xres;       // x again when the call adds the residual (out = x + layer(x)), else nullptr
     const float* steer_v;   // [H] steering direction, or nullptr (no steering)
     float steer_F;          // steering strength: y -= F v (v . y)
+    int stages;             // projections run: 1 gate and up, 2 down, 3 both (the forward)
     int probe;              // 0: forward; 1: every token to routed expert probe_e; 2: the shared expert alone
     int probe_e;
     float* probe_out;       // probe: raw accumulators (gate/up: [n][2I]; down: [n][H])

@@ -26,19 +26,18 @@ def test_block_matrix_sizes():
 
 def test_decode_bytes_one_token():
     ab = bench.algorithmic_bytes(bench.WORKLOADS["decode"], 8)
-    # 8 experts' gate and up blocks + the bf16 shared gate and up + x + h (9 rows of I floats)
-    assert ab["k_gateup_decode"] == 8 * 2 * IQ2_MATRIX + 2 * I * H * 2 + H * 4 + 9 * I * 4 == 68_247_552
+    # 8 experts' blocks + the bf16 shared expert + x + h written and read (9 rows of I values, 4 bytes) + y
+    assert ab["k_moe_decode"] == 8 * 7_077_888 + 3 * I * H * 2 + H * 4 + 2 * 9 * I * 4 + 9 * H * 4 == 107_266_048
     # router rows + 8 routed experts + the whole shared expert
     assert ab["layer"] == E * H * 4 + 8 * 7_077_888 + 3 * I * H * 2 == 111_149_056
     assert ab["routed"] == 8 * 7_077_888
-    assert ab["k_down_decode"] == 8 * Q2_MATRIX + H * I * 2 + 9 * I * 4 + 9 * H * 4
 
 
 def test_decode_bytes_scale_with_distinct_experts():
     w = bench.WORKLOADS["decode2"]
     a, b = bench.algorithmic_bytes(w, 8), bench.algorithmic_bytes(w, 16)
     assert b["routed"] - a["routed"] == 8 * 7_077_888
-    assert b["k_gateup_decode"] - a["k_gateup_decode"] == 8 * 2 * IQ2_MATRIX
+    assert b["k_moe_decode"] - a["k_moe_decode"] == 8 * 7_077_888
 
 
 def test_prefill_flops_and_bytes():
