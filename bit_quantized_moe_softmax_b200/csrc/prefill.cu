@@ -611,9 +611,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const uint16_t* dq = nullptr;
             const uint32_t* scp = nullptr;
             const uint32_t* ddp = nullptr;
+            // an expert with more than one row tile has its weights read by each of them (its row tiles
+            // run on neighbouring CTAs at about the same time): keep those weights in L2
+            const uint64_t pol_keep = policy_evict_last();
+            bool keep = false;
             auto set_src = [&](int tile) {
                 const TileInfo ti = tile_info<MODE>(a, tile, NB);
                 const size_t e = (size_t)ti.e;
+                keep = __ldg(a.counts + e) > kGBM;
                 if (MODE == kModeGateUp) {
                     const int row = 128 * ti.nb + (r & 127);
                     qs = (r < 128 ? a.W.gate_qs : a.W.up_qs) + e * a.W.iq2_qs_stride +
@@ -629,7 +634,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 }
             };
             auto fetch = [&](BFrag& f) {
-                f.q = ld_stream_v4(qs + (size_t)cks * 512);
+                f.q = keep ? ld_stream_v4_hint(qs + (size_t)cks * 512, pol_keep) : ld_stream_v4(qs + (size_t)cks * 512);
                 if (MODE == kModeGateUp) {
                     f.a0 = ld_stream_u16(dq + (cks >> 2) * 32);
                 } else {
