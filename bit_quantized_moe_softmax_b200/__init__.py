@@ -34,13 +34,14 @@ EXPORTS = ("ds4moe_create", "ds4moe_destroy", "ds4moe_weight_bytes", "ds4moe_wor
            "ds4moe_forward_profiled", "ds4moe_route_noalloc", "ds4moe_forward_residual",
            "ds4moe_forward_residual_profiled", "ds4moe_set_steering", "ds4moe_forward_host_async",
            "ds4moe_host_sync", "ds4moe_probe", "ds4moe_selftest_wait",
-           "ds4moe_permutation")
+           "ds4moe_permutation", "ds4moe_pack_q4k")
 
 
 class ds4moe_shape(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int32), ("inter", ctypes.c_int32), ("n_experts", ctypes.c_int32),
                 ("top_k", ctypes.c_int32), ("max_tokens", ctypes.c_int32), ("act_dtype", ctypes.c_int32),
-                ("has_shared", ctypes.c_int32), ("has_bias", ctypes.c_int32), ("decode_max", ctypes.c_int32)]
+                ("has_shared", ctypes.c_int32), ("has_bias", ctypes.c_int32), ("decode_max", ctypes.c_int32),
+                ("expert_bits", ctypes.c_int32)]
 
 
 class Ds4MoeError(RuntimeError):
@@ -64,6 +65,7 @@ def lib() -> ctypes.CDLL:
             "ds4moe_workspace_bytes": ([vp, i32], sz),
             "ds4moe_bind": ([vp, vp, sz, vp, sz, vp], i32),
             "ds4moe_pack_q2k": ([vp, i64, vp, vp], i32),
+            "ds4moe_pack_q4k": ([vp, i64, vp, vp], i32),
             "ds4moe_pack_iq2xxs": ([vp, i64, vp, vp, vp], i32),
             "ds4moe_set_grid": ([vp, vp, vp], i32),
             "ds4moe_set_router": ([vp, vp, vp, vp], i32),
@@ -117,8 +119,9 @@ def _ptr(t) -> int | None:
 
 # ------------------------------------------------------------------ C ABI names
 def ds4moe_create(hidden, inter, n_experts, top_k, max_tokens, act_dtype=DS4MOE_ACT_F32, has_shared=1,
-                  has_bias=0, decode_max=0) -> int:
-    s = ds4moe_shape(hidden, inter, n_experts, top_k, max_tokens, act_dtype, has_shared, has_bias, decode_max)
+                  has_bias=0, decode_max=0, expert_bits=0) -> int:
+    s = ds4moe_shape(hidden, inter, n_experts, top_k, max_tokens, act_dtype, has_shared, has_bias, decode_max,
+                     expert_bits)
     h = ctypes.c_void_p()
     _ok(lib().ds4moe_create(ctypes.byref(s), ctypes.byref(h)), "ds4moe_create")
     return h.value
@@ -144,6 +147,10 @@ def ds4moe_bind(h: int, weights: torch.Tensor, workspace: torch.Tensor | None, s
 
 def ds4moe_pack_q2k(w: torch.Tensor, blocks: torch.Tensor, stream=None):
     _ok(lib().ds4moe_pack_q2k(_ptr(w), w.numel(), _ptr(blocks), _stream(stream)), "ds4moe_pack_q2k")
+
+
+def ds4moe_pack_q4k(w: torch.Tensor, blocks: torch.Tensor, stream=None):
+    _ok(lib().ds4moe_pack_q4k(_ptr(w), w.numel(), _ptr(blocks), _stream(stream)), "ds4moe_pack_q4k")
 
 
 def ds4moe_pack_iq2xxs(w: torch.Tensor, grid: torch.Tensor, blocks: torch.Tensor, stream=None):
@@ -270,16 +277,20 @@ class MoELayer:
     ``load`` takes a dict with H, I, E, k, W_r, b_r, grid and either packed
     blocks (gate, up: [E, I*H/256, 66] u8; down: [E, H*I/256, 84] u8) or float
     weights to pack on the device (gate_f, up_f: [E, I, H]; down_f: [E, H, I]),
-    plus sh_gate/sh_up/sh_down bf16 when has_shared.
+    plus sh_gate/sh_up/sh_down bf16 when has_shared.  With expert_bits=4 all
+    three expert matrices are Q4_K-style blocks ([E, n/256, 144] u8) and no
+    grid is needed.
     """
 
     def __init__(self, H, I, E, k, max_tokens, act_dtype=DS4MOE_ACT_F32, has_shared=True, has_bias=False,
-                 decode_max=0, device="cuda"):
+                 decode_max=0, device="cuda", expert_bits=0):
         self.H, self.I, self.E, self.k = H, I, E, k
+        self.expert_bits = expert_bits
         self.max_tokens = max_tokens
         self.act_dtype = act_dtype
         self.device = torch.device(device)
-        self.h = ds4moe_create(H, I, E, k, max_tokens, act_dtype, int(has_shared), int(has_bias), decode_max)
+        self.h = ds4moe_create(H, I, E, k, max_tokens, act_dtype, int(has_shared), int(has_bias), decode_max,
+                               expert_bits)
         wb = ds4moe_weight_bytes(self.h)
         sb = ds4moe_workspace_bytes(self.h, max_tokens)
         self.weights = torch.empty(wb, dtype=torch.uint8, device=self.device)
@@ -299,8 +310,16 @@ class MoELayer:
         """Pack float expert weights with the device quantizers; returns gate/up/down blocks."""
         H, I, E = self.H, self.I, self.E
         dev = self.device
-        grid = layer["grid"].to(dev).contiguous()
         nb = I * H // 256
+        if self.expert_bits == 4:
+            blocks = {}
+            for name in ("gate", "up", "down"):
+                t = torch.empty(E, nb, 144, dtype=torch.uint8, device=dev)
+                for e in range(E):
+                    ds4moe_pack_q4k(layer[name + "_f"][e].to(dev).contiguous(), t[e])
+                blocks[name] = t
+            return blocks
+        grid = layer["grid"].to(dev).contiguous()
         gate = torch.empty(E, nb, 66, dtype=torch.uint8, device=dev)
         up = torch.empty(E, nb, 66, dtype=torch.uint8, device=dev)
         down = torch.empty(E, nb, 84, dtype=torch.uint8, device=dev)
@@ -314,7 +333,8 @@ class MoELayer:
         dev = self.device
         if "gate" not in layer:
             layer = {**layer, **self.pack(layer)}
-        ds4moe_set_grid(self.h, layer["grid"].to(dev).contiguous())
+        if layer.get("grid") is not None:
+            ds4moe_set_grid(self.h, layer["grid"].to(dev).contiguous())
         b = layer.get("b_r")
         ds4moe_set_router(self.h, layer["W_r"].to(dev).contiguous(), None if b is None else b.to(dev).contiguous())
         for e in range(self.E):

@@ -571,6 +571,21 @@ __device__ __forceinline__ void iq2_chunk_s8(uint32_t idx, uint32_t S, uint32_t 
     hi = __byte_perm(clo, chi, sel >> 16);
 }
 
+// Q4 down codes (mode-1 order) of rows g (w0) and g + 8 (w1), one word = two
+// 16-column groups: the bf16 A fragments of those groups, each element
+// 1 + q/16 (exact: 0x3F80 | q << 3).
+__device__ __forceinline__ void q4_down_frags(uint32_t w0, uint32_t w1, uint32_t (&a)[4], uint32_t (&b)[4]) {
+    constexpr uint32_t M = 0x00780078u, ONE = 0x3F803F80u;
+    a[0] = ((w0 << 3) & M) | ONE;
+    a[1] = ((w1 << 3) & M) | ONE;
+    a[2] = ((w0 >> 1) & M) | ONE;
+    a[3] = ((w1 >> 1) & M) | ONE;
+    b[0] = ((w0 >> 5) & M) | ONE;
+    b[1] = ((w1 >> 5) & M) | ONE;
+    b[2] = ((w0 >> 9) & M) | ONE;
+    b[3] = ((w1 >> 9) & M) | ONE;
+}
+
 // Per consumer thread state of the gate/up kernel's tasks.
 template <int NT>
 struct GateUpAcc {
@@ -581,14 +596,14 @@ struct GateUpAcc {
 
 // ---------------------------------------------------------------- down projection pieces
 // k steps (64 columns) per routed down chunk for an entry of ns slots: codes,
-// scales, (d, dmin) and the slots' h pieces (and per-16 sums) for those
-// columns must fit one stage.
-__device__ __forceinline__ int down_chunk_ksteps(int nkt, int nsb, int ns) {
+// scales (step_bytes per step: 640 for Q2, 1152 for Q4), (d, dmin) and the
+// slots' h pieces (and per-16 sums) for those columns must fit one stage.
+__device__ __forceinline__ int down_chunk_ksteps(int nkt, int nsb, int ns, int step_bytes) {
     // the largest of 32, 16, 8, 4 that divides the k steps (I / 64: a multiple of 4 for I >= 256)
     int ck = nkt % 32 == 0 ? 32 : nkt % 16 == 0 ? 16 : nkt % 8 == 0 ? 8 : nkt % 4 == 0 ? 4 : nkt;
     for (; ck > 1 && ck % 2 == 0; ck >>= 1) {
         const int nsbc = nsb > 1 ? (ck + 3) / 4 : 1;
-        if (ck * 640 + nsbc * 128 + ns * ck * 272 <= kStageBytes) break;
+        if (ck * step_bytes + nsbc * 128 + ns * ck * 272 <= kStageBytes) break;
     }
     return ck;
 }
@@ -601,19 +616,23 @@ struct DownAcc {
 };
 
 
-template <int NT>
+// Q4: the routed experts' three matrices are Q4 blocks (no grid tables; x's
+// per-32-column sums for the min terms).
+template <int NT, bool Q4>
 __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     k_moe_decode(Weights W, Dims D, DecodeWs ws, const void* x, int n) {
     using C = GateUpCfg<NT>;
     constexpr int NS = C::NS, CW = C::CW, R = C::R, TPB = C::TPB, kThreads = C::kThreads;
+    constexpr int kTab = Q4 ? 0 : C::kTabWords;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     uint32_t* tsel = reinterpret_cast<uint32_t*>(smem_raw);                      // rows [256][64] or [256][R]
     uint32_t* tsgn = tsel + 256 * R;                                             // [128][R] (interleaved form)
-    unsigned char* stages = smem_raw + 4 * C::kTabWords;                         // NS x kStageBytes
+    unsigned char* stages = smem_raw + 4 * kTab;                                 // NS x kStageBytes
     float* red = reinterpret_cast<float*>(stages + NS * kStageBytes);            // kRedFloats
     unsigned char* xbuf = reinterpret_cast<unsigned char*>(red + C::kRedFloats);  // n x H x 4 bytes: bf16 pieces
     unsigned char* xq = C::kSplitX ? xbuf + (size_t)n * D.H * 4 : xbuf;          // int8 pieces
     unsigned char* zero = xq + (size_t)n * D.H * 4;                              // 64 bytes of zeros
+    float* xsum = reinterpret_cast<float*>(zero + 64);                           // Q4: [n][H / 32] sums of x
     __shared__ Pipe P;
     __shared__ Routing Rt;
     __shared__ int s_last, s_refused;
@@ -630,8 +649,8 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     const bool do_gu = (ws.stages & 1) != 0, do_dn = (ws.stages & 2) != 0;
     const int n_sh = !do_gu || ws.probe == 1 ? 0 : (D.has_shared ? I / 8 : 0);   // shared tasks: 8 rows of gate and up
     const int rb_per_e = I / 32;
-    // k steps (64 columns) per routed chunk: the largest of 32, 16, 8, 4 that divides H / 64
-    const int ck_rt = nkt % 32 == 0 ? 32 : nkt % 16 == 0 ? 16 : nkt % 8 == 0 ? 8 : 4;
+    // k steps (64 columns) per routed chunk: the largest of 32, 16, 8, 4 that divides H / 64 (Q4: of 8, 4)
+    const int ck_rt = (!Q4 && nkt % 32 == 0) ? 32 : (!Q4 && nkt % 16 == 0) ? 16 : nkt % 8 == 0 ? 8 : 4;
     const int nch_rt = nkt / ck_rt;
     const int kcs = H < 1024 ? H : 1024;              // columns per shared chunk
     const int nch_sh = H / kcs;
@@ -645,7 +664,8 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
 
     pipe_init(P, NS, CW);
     // ---- grid tables (made when the grid was loaded)
-    if (C::kRows) {
+    if (Q4) {
+    } else if (C::kRows) {
         for (int i = tid; i < 256 * 64; i += kThreads) {
             const int r = i >> 6;
             tsel[i] = __ldg(W.gtab + ((i & 32) ? 256 + (r & 127) : r));
@@ -657,9 +677,9 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     if (tid < kMaxRedBufs) RR.cnt[tid] = RR.task[tid] = RR.freed[tid] = 0;
     if (tid == 0) RR.exits = RR.ntasks = 0;
     if (tid == 0) {
-        s_cand[0] = __ldg(W.gtab + 384);
-        s_cand[1] = __ldg(W.gtab + 385);
-        s_refused = (int)__ldg(W.gtab + 386);
+        s_cand[0] = Q4 ? 0u : __ldg(W.gtab + 384);
+        s_cand[1] = Q4 ? 0u : __ldg(W.gtab + 385);
+        s_refused = Q4 ? 0 : (int)__ldg(W.gtab + 386);
         if (s_refused) set_err(ws.err, kErrGrid);
         if (blockIdx.x == 0) *ws.grid_refused = (uint32_t)s_refused;
     }
@@ -712,6 +732,20 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             for (int p = 0; p < 4; ++p) s_cs[tid][p] = s_tokmax[tid] > 0.f ? ldexpf(1.f, e - 7 - 7 * p) : 0.f;
         }
         __syncthreads();
+        if (Q4 && do_gu) {
+            // sums of x over each 32-column sub-block (the min terms)
+            for (int i = tid; i < n * (H / 32); i += kThreads) {
+                const int tk = i / (H / 32), j = i - tk * (H / 32);
+                float sx = 0.f;
+#pragma unroll
+                for (int c = 0; c < 32; c += 4) {
+                    const float4 v = load_act4(x, (int64_t)tk * H + 32 * j + c, D.act_bf16);
+                    sx += (v.x + v.y) + (v.z + v.w);
+                }
+                xsum[i] = sx;
+            }
+            if (!C::kSplitX) __syncthreads();
+        }
         if (C::kSplitX && do_gu) {
             quantize_x(x, D.act_bf16, n, H, s_f, xq, tid, kThreads);
             __syncthreads();
@@ -765,7 +799,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                 u = (dt - dn_sh) / drb;
                 rb = (dt - dn_sh) % drb;
                 ns = Rt.ustart[u + 1] - Rt.ustart[u];
-                ck = down_chunk_ksteps(dnkt, dnsb, ns);
+                ck = down_chunk_ksteps(dnkt, dnsb, ns, Q4 ? 1152 : 640);
             }
             const int nch = dsh ? dnch_sh : dnkt / ck;
             if (!ws.probe) {
@@ -797,17 +831,18 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                         const int e = Rt.uniq[u], s0 = Rt.ustart[u];
                         const int kt0 = c * ck;
                         const int sb0 = dnsb > 1 ? kt0 / 4 : 0, nsbc = dnsb > 1 ? (ck + 3) / 4 : 1;
-                        const uint32_t qb = ck * 512, sb = ck * 128, dbb = nsbc * 128;
+                        const uint32_t cpb = Q4 ? 1024 : 512;   // code bytes per 32-row step
+                        const uint32_t qb = ck * cpb, sb = ck * 128, dbb = nsbc * 128;
                         const uint32_t hb = ck * 256, hsb = ck * 16;
                         P.info[s] = ChunkInfo{total + dt, c, nch, kt0, ck};
                         mbar_arrive_expect_tx(&P.full[s], qb + sb + dbb + ns * (hb + hsb));
-                        bulk_load(st, W.down_q + (size_t)e * W.q2_q_stride + ((size_t)rb * dnkt + kt0) * 512, qb,
+                        const size_t qs_stride = Q4 ? W.q4_q_stride : W.q2_q_stride;
+                        const uint32_t* scp = Q4 ? W.down_sc4 + (size_t)e * W.q4_sc_stride : W.down_sc + (size_t)e * W.q2_sc_stride;
+                        const uint32_t* ddp = Q4 ? W.down_dd4 + (size_t)e * W.q4_dd_stride : W.down_dd + (size_t)e * W.q2_dd_stride;
+                        bulk_load(st, W.down_q + (size_t)e * qs_stride + ((size_t)rb * dnkt + kt0) * cpb, qb,
                                   &P.full[s], pol);
-                        bulk_load(st + qb, W.down_sc + (size_t)e * W.q2_sc_stride + ((size_t)rb * dnkt + kt0) * 32,
-                                  sb, &P.full[s], pol);
-                        bulk_load(st + qb + sb,
-                                  W.down_dd + (size_t)e * W.q2_dd_stride + ((size_t)rb * dnsb + sb0) * 32, dbb,
-                                  &P.full[s], pol);
+                        bulk_load(st + qb, scp + ((size_t)rb * dnkt + kt0) * 32, sb, &P.full[s], pol);
+                        bulk_load(st + qb + sb, ddp + ((size_t)rb * dnsb + sb0) * 32, dbb, &P.full[s], pol);
                         unsigned char* hdst = st + qb + sb + dbb;
                         for (int q = 0; q < ns; ++q) {
                             const int slot = Rt.slot[s0 + q];
@@ -846,15 +881,31 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                         const int tt = task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
                         const int e = Rt.uniq[u];
                         const int kt0 = c * ck_rt;
-                        const uint32_t pb = ck_rt * 512, db = ck_rt * 16;
-                        const size_t qoff = (size_t)e * W.iq2_qs_stride + ((size_t)rb * nkt + kt0) * 512;
-                        const size_t doff = (size_t)e * W.iq2_d_stride + ((size_t)rb * nsb + kt0 / 4) * 32;
                         P.info[s] = ChunkInfo{task, c, nch, kt0, ck_rt};
-                        mbar_arrive_expect_tx(&P.full[s], 2 * pb + 2 * db);
-                        bulk_load(st, W.gate_qs + qoff, pb, &P.full[s], pol);
-                        bulk_load(st + pb, W.up_qs + qoff, pb, &P.full[s], pol);
-                        bulk_load(st + 2 * pb, W.gate_d + doff, db, &P.full[s], pol);
-                        bulk_load(st + 2 * pb + db, W.up_d + doff, db, &P.full[s], pol);
+                        if (Q4) {
+                            // gate codes, up codes [ck][32][32 B], their scale words [ck][32], (d, dmin)
+                            // words [ck / 4][32]
+                            const uint32_t cb = ck_rt * 1024, sb = ck_rt * 128, db = (ck_rt / 4) * 128;
+                            const size_t qoff = (size_t)e * W.q4_q_stride + ((size_t)rb * nkt + kt0) * 1024;
+                            const size_t soff = (size_t)e * W.q4_sc_stride + ((size_t)rb * nkt + kt0) * 32;
+                            const size_t doff = (size_t)e * W.q4_dd_stride + ((size_t)rb * nsb + kt0 / 4) * 32;
+                            mbar_arrive_expect_tx(&P.full[s], 2 * (cb + sb + db));
+                            bulk_load(st, W.gate_qs + qoff, cb, &P.full[s], pol);
+                            bulk_load(st + cb, W.up_qs + qoff, cb, &P.full[s], pol);
+                            bulk_load(st + 2 * cb, W.gate_sc4 + soff, sb, &P.full[s], pol);
+                            bulk_load(st + 2 * cb + sb, W.up_sc4 + soff, sb, &P.full[s], pol);
+                            bulk_load(st + 2 * (cb + sb), W.gate_dd4 + doff, db, &P.full[s], pol);
+                            bulk_load(st + 2 * (cb + sb) + db, W.up_dd4 + doff, db, &P.full[s], pol);
+                        } else {
+                            const uint32_t pb = ck_rt * 512, db = ck_rt * 16;
+                            const size_t qoff = (size_t)e * W.iq2_qs_stride + ((size_t)rb * nkt + kt0) * 512;
+                            const size_t doff = (size_t)e * W.iq2_d_stride + ((size_t)rb * nsb + kt0 / 4) * 32;
+                            mbar_arrive_expect_tx(&P.full[s], 2 * pb + 2 * db);
+                            bulk_load(st, W.gate_qs + qoff, pb, &P.full[s], pol);
+                            bulk_load(st + pb, W.up_qs + qoff, pb, &P.full[s], pol);
+                            bulk_load(st + 2 * pb, W.gate_d + doff, db, &P.full[s], pol);
+                            bulk_load(st + 2 * pb + db, W.up_d + doff, db, &P.full[s], pol);
+                        }
                     }
                 }
                 __syncwarp();
@@ -931,6 +982,56 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                 }
                 const int ck = inf.cnt;
                 const int nsbc = dnsb > 1 ? (ck + 3) / 4 : 1;
+                if constexpr (Q4) {
+                // codes [ck][32][32 B], scale words [ck][32], (d, dmin) words [nsbc][32], then the slots' h
+                // pieces and per-16 sums
+                const unsigned char* qv = st;
+                const uint32_t* scv = reinterpret_cast<const uint32_t*>(st + ck * 1024);
+                const uint32_t* ddv = reinterpret_cast<const uint32_t*>(st + ck * 1152);
+                const uint16_t* hst = reinterpret_cast<const uint16_t*>(st + ck * 1152 + nsbc * 128);
+                const float* hss = reinterpret_cast<const float*>(st + ck * 1152 + nsbc * 128 + ns * ck * 256);
+                const int jj = t >> 1;   // this lane's 16-column group t lies in 32-column sub-block t / 2
+                for (int kt = warp; kt < ck; kt += CW) {
+                    const int sbi = dnsb > 1 ? ((inf.lo + kt) >> 2) - (inf.lo >> 2) : 0;
+                    uint2 Bl[TPB];
+                    float S[TPB];
+#pragma unroll
+                    for (int q = 0; q < TPB; ++q) {
+                        Bl[q] = make_uint2(0u, 0u);
+                        S[q] = 0.f;
+                        if (q < dtcount) {
+                            Bl[q] = *reinterpret_cast<const uint2*>(hst + (size_t)q * ck * 128 + (kt * 2 + pD) * 64 + 16 * jD + 4 * t);
+                            S[q] = hss[q * ck * 4 + kt * 4 + t];
+                        }
+                    }
+#pragma unroll
+                    for (int T = 0; T < 2; ++T) {
+                        const int rg = 16 * T + g;
+                        const uint2 c0 = *reinterpret_cast<const uint2*>(qv + kt * 1024 + rg * 32 + 8 * t);
+                        const uint2 c1 = *reinterpret_cast<const uint2*>(qv + kt * 1024 + (rg + 8) * 32 + 8 * t);
+                        uint32_t Af[4][4];
+                        q4_down_frags(c0.x, c1.x, Af[0], Af[1]);
+                        q4_down_frags(c0.y, c1.y, Af[2], Af[3]);
+                        // sum q h = 16 (D - S) over the lane's group; a16 = 16 d sc, mm = dmin m, per row
+                        const uint32_t sw0 = scv[kt * 32 + rg], sw1 = scv[kt * 32 + rg + 8];
+                        const uint32_t dd0 = ddv[sbi * 32 + rg], dd1 = ddv[sbi * 32 + rg + 8];
+                        const float a160 = 16.f * half_bits(dd0 & 0xffffu) * (float)((sw0 >> (8 * jj)) & 0xffu);
+                        const float a161 = 16.f * half_bits(dd1 & 0xffffu) * (float)((sw1 >> (8 * jj)) & 0xffu);
+                        const float mm0 = half_bits(dd0 >> 16) * (float)((sw0 >> (16 + 8 * jj)) & 0xffu);
+                        const float mm1 = half_bits(dd1 >> 16) * (float)((sw1 >> (16 + 8 * jj)) & 0xffu);
+#pragma unroll
+                        for (int q = 0; q < TPB; ++q) {
+                            float Dv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) bmma(Dv, Af[j], jD == j ? Bl[q] : make_uint2(0u, 0u));
+                            A2.rt[q][T][0] = fmaf(a160, (Dv[0] + Dv[1]) - S[q], A2.rt[q][T][0]);
+                            A2.rt[q][T][0] = fmaf(-mm0, S[q], A2.rt[q][T][0]);
+                            A2.rt[q][T][1] = fmaf(a161, (Dv[2] + Dv[3]) - S[q], A2.rt[q][T][1]);
+                            A2.rt[q][T][1] = fmaf(-mm1, S[q], A2.rt[q][T][1]);
+                        }
+                    }
+                }
+                } else {
                 const unsigned char* qv = st;
                 const uint32_t* scv = reinterpret_cast<const uint32_t*>(st + ck * 512);
                 const uint32_t* ddv = reinterpret_cast<const uint32_t*>(st + ck * 640);
@@ -987,6 +1088,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                             A2.rt[q][T][1] = fmaf(-mm1, S[q], A2.rt[q][T][1]);
                         }
                     }
+                }
                 }
             }
                 __syncwarp();
@@ -1079,6 +1181,55 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                     }
                 }
                 const int ck = inf.cnt;
+                if constexpr (Q4) {
+                    // gate codes, up codes [ck][32][32 B], scale words [2][ck][32], (d, dmin) words [2][ck/4][32]
+                    const uint32_t* scw = reinterpret_cast<const uint32_t*>(st + 2 * ck * 1024);
+                    const uint32_t* ddw = scw + 2 * ck * 32;
+                    const int jj = t >> 1;            // this lane's 32-column half of a step
+                    const int p0 = 2 * (t & 1);       // and its two int8 pieces
+                    for (int kt = warp; kt < ck; kt += CW) {
+                        const int col = 64 * (inf.lo + kt);
+                        uint2 B[TPB][2];
+                        float xs[TPB];
+#pragma unroll
+                        for (int q = 0; q < TPB; ++q) {
+                            const unsigned char* live =
+                                xq + (size_t)(tokrow[q] * 4 + pB) * H + col + 32 * jB + 8 * t;
+                            B[q][0] = *reinterpret_cast<const uint2*>(q < tcount && jB == 0 ? live : zero);
+                            B[q][1] = *reinterpret_cast<const uint2*>(q < tcount && jB == 1 ? live : zero);
+                            // the min term of the lane's half, once per half (even t)
+                            xs[q] = q < tcount && (t & 1) == 0 ? xsum[tokrow[q] * (H / 32) + (col >> 5) + jj] : 0.f;
+                        }
+#pragma unroll
+                        for (int T = 0; T < 4; ++T) {
+                            const int mt = T >> 1, rg = 16 * (T & 1) + g;
+                            const unsigned char* pay = st + (mt * ck + kt) * 1024 + rg * 32 + 8 * t;
+                            const uint2 c0 = *reinterpret_cast<const uint2*>(pay);
+                            const uint2 c1 = *reinterpret_cast<const uint2*>(pay + 256);   // row rg + 8
+                            constexpr uint32_t M = 0x0F0F0F0Fu;
+                            const uint32_t A0[4] = {c0.x & M, c1.x & M, (c0.x >> 4) & M, (c1.x >> 4) & M};
+                            const uint32_t A1[4] = {c0.y & M, c1.y & M, (c0.y >> 4) & M, (c1.y >> 4) & M};
+                            const uint32_t sw0 = scw[(mt * ck + kt) * 32 + rg], sw1 = scw[(mt * ck + kt) * 32 + rg + 8];
+                            const uint32_t dw0 = ddw[(mt * (ck / 4) + kt / 4) * 32 + rg];
+                            const uint32_t dw1 = ddw[(mt * (ck / 4) + kt / 4) * 32 + rg + 8];
+                            const float a0 = half_bits(dw0 & 0xffffu) * (float)((sw0 >> (8 * jj)) & 0xffu);
+                            const float a1 = half_bits(dw1 & 0xffffu) * (float)((sw1 >> (8 * jj)) & 0xffu);
+                            const float m0 = half_bits(dw0 >> 16) * (float)((sw0 >> (16 + 8 * jj)) & 0xffu);
+                            const float m1 = half_bits(dw1 >> 16) * (float)((sw1 >> (16 + 8 * jj)) & 0xffu);
+#pragma unroll
+                            for (int q = 0; q < TPB; ++q) {   // absent tokens: B = 0, xs = 0
+                                int Dv[4];
+                                imma_z(Dv, A0, B[q][0]);
+                                imma(Dv, A1, B[q][1]);
+                                const float c0f = s_cs[tokrow[q]][p0], c1f = s_cs[tokrow[q]][p0 + 1];
+                                A.rt[q][T][0] = fmaf(a0, fmaf((float)Dv[0], c0f, (float)Dv[1] * c1f), A.rt[q][T][0]);
+                                A.rt[q][T][0] = fmaf(-m0, xs[q], A.rt[q][T][0]);
+                                A.rt[q][T][1] = fmaf(a1, fmaf((float)Dv[2], c0f, (float)Dv[3] * c1f), A.rt[q][T][1]);
+                                A.rt[q][T][1] = fmaf(-m1, xs[q], A.rt[q][T][1]);
+                            }
+                        }
+                    }
+                } else {
                 const int kpw = ck >= CW ? ck / CW : 1;
                 const int kb = warp * kpw;
                 if (kb < ck) {
@@ -1147,6 +1298,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                             A.rt[q][T][1] = fmaf((float)ai[q][T][3], d1 * c1, A.rt[q][T][1]);
                         }
                     }
+                }
                 }
             }
             __syncwarp();
@@ -1434,8 +1586,8 @@ cudaError_t launch_wait_selftest(uint32_t* err, cudaStream_t st) {
 template <int NT>
 size_t gateup_smem_bytes(const Dims& D, int n) {
     using C = GateUpCfg<NT>;
-    return (size_t)C::NS * kStageBytes + 4 * ((size_t)C::kTabWords + C::kRedFloats) +
-           (size_t)(C::kSplitX ? 2 : 1) * n * D.H * 4 + 64;
+    return (size_t)C::NS * kStageBytes + 4 * ((size_t)(D.q4 ? 0 : C::kTabWords) + C::kRedFloats) +
+           (size_t)(C::kSplitX ? 2 : 1) * n * D.H * 4 + 64 + (D.q4 ? (size_t)n * (D.H / 32) * 4 : 0);
 }
 
 size_t router_smem_bytes(const Dims& D, int n) {
@@ -1506,12 +1658,12 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <int NT>
+template <int NT, bool Q4>
 cudaError_t launch_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n, float* out,
                             int n_sm, cudaStream_t st, cudaEvent_t const* ev) {
     cudaError_t err;
     const size_t s1 = gateup_smem_bytes<NT>(D, n);
-    if ((err = configure(k_moe_decode<NT>)) != cudaSuccess) return err;
+    if ((err = configure(k_moe_decode<NT, Q4>)) != cudaSuccess) return err;
     if ((err = configure(k_router_decode<NT>)) != cudaSuccess) return err;
     Marks mk(ev, st);
     const bool pdl = ev == nullptr;   // profiled runs keep the kernels apart
@@ -1521,7 +1673,7 @@ cudaError_t launch_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws,
                                                                                              ws.route_ready);
     mk.after();
     mk.before();
-    err = launch_pdl(k_moe_decode<NT>, dim3(n_sm), dim3(GateUpCfg<NT>::kThreads), s1, st, pdl, W, D, ws, x, n);
+    err = launch_pdl(k_moe_decode<NT, Q4>, dim3(n_sm), dim3(GateUpCfg<NT>::kThreads), s1, st, pdl, W, D, ws, x, n);
     mk.after();
     if (err != cudaSuccess) return err;
     const int64_t nel = (int64_t)n * D.H;
@@ -1553,10 +1705,16 @@ size_t decode_smem_bytes(const Dims& D, int n) {
 
 cudaError_t launch_decode(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n, float* out,
                           int n_sm, cudaStream_t st, cudaEvent_t const* ev) {
-    if (n <= 1) return launch_decode_t<1>(W, D, ws, x, n, out, n_sm, st, ev);
-    if (n <= 2) return launch_decode_t<2>(W, D, ws, x, n, out, n_sm, st, ev);
-    if (n <= 4) return launch_decode_t<4>(W, D, ws, x, n, out, n_sm, st, ev);
-    return launch_decode_t<8>(W, D, ws, x, n, out, n_sm, st, ev);
+    if (D.q4) {
+        if (n <= 1) return launch_decode_t<1, true>(W, D, ws, x, n, out, n_sm, st, ev);
+        if (n <= 2) return launch_decode_t<2, true>(W, D, ws, x, n, out, n_sm, st, ev);
+        if (n <= 4) return launch_decode_t<4, true>(W, D, ws, x, n, out, n_sm, st, ev);
+        return launch_decode_t<8, true>(W, D, ws, x, n, out, n_sm, st, ev);
+    }
+    if (n <= 1) return launch_decode_t<1, false>(W, D, ws, x, n, out, n_sm, st, ev);
+    if (n <= 2) return launch_decode_t<2, false>(W, D, ws, x, n, out, n_sm, st, ev);
+    if (n <= 4) return launch_decode_t<4, false>(W, D, ws, x, n, out, n_sm, st, ev);
+    return launch_decode_t<8, false>(W, D, ws, x, n, out, n_sm, st, ev);
 }
 
 // Probe of the down kernel: caller h [n][I] binary32 -> the workspace's h pieces (routed layout at slots
@@ -1587,15 +1745,15 @@ __global__ void k_probe_h(const float* h, int n, int I, int k, int shared, uint1
     if (!shared) hsum_rt[(size_t)tk * k * (I / 16) + b] = s;
 }
 
-template <int NT>
+template <int NT, bool Q4>
 cudaError_t launch_probe_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws, int which, const void* in,
                                   int n, int n_sm, cudaStream_t st) {
     cudaError_t err;
-    if ((err = configure(k_moe_decode<NT>)) != cudaSuccess) return err;
+    if ((err = configure(k_moe_decode<NT, Q4>)) != cudaSuccess) return err;
     DecodeWs w = ws;
     if (which == 0) {   // gate and up projections of x = in
         w.stages = 1;
-        k_moe_decode<NT><<<n_sm, GateUpCfg<NT>::kThreads, gateup_smem_bytes<NT>(D, n), st>>>(W, D, w, in, n);
+        k_moe_decode<NT, Q4><<<n_sm, GateUpCfg<NT>::kThreads, gateup_smem_bytes<NT>(D, n), st>>>(W, D, w, in, n);
         return cudaGetLastError();
     }
     const int64_t nb = (int64_t)n * (D.I / 16);
@@ -1603,7 +1761,7 @@ cudaError_t launch_probe_decode_t(const Weights& W, const Dims& D, const DecodeW
                                                             ws.probe == 2, ws.hb_rt, ws.hsum_rt, ws.hb_sh);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     w.stages = 2;   // down projection of h = in
-    k_moe_decode<NT><<<n_sm, GateUpCfg<NT>::kThreads, gateup_smem_bytes<NT>(D, n), st>>>(W, D, w, nullptr, n);
+    k_moe_decode<NT, Q4><<<n_sm, GateUpCfg<NT>::kThreads, gateup_smem_bytes<NT>(D, n), st>>>(W, D, w, nullptr, n);
     return cudaGetLastError();
 }
 
@@ -1611,10 +1769,16 @@ cudaError_t launch_probe_decode_t(const Weights& W, const Dims& D, const DecodeW
 // one expert (ws.probe set by the caller), raw accumulators to ws.probe_out.
 cudaError_t launch_probe_decode(const Weights& W, const Dims& D, const DecodeWs& ws, int which, const void* in, int n,
                                 int n_sm, cudaStream_t st) {
-    if (n <= 1) return launch_probe_decode_t<1>(W, D, ws, which, in, n, n_sm, st);
-    if (n <= 2) return launch_probe_decode_t<2>(W, D, ws, which, in, n, n_sm, st);
-    if (n <= 4) return launch_probe_decode_t<4>(W, D, ws, which, in, n, n_sm, st);
-    return launch_probe_decode_t<8>(W, D, ws, which, in, n, n_sm, st);
+    if (D.q4) {
+        if (n <= 1) return launch_probe_decode_t<1, true>(W, D, ws, which, in, n, n_sm, st);
+        if (n <= 2) return launch_probe_decode_t<2, true>(W, D, ws, which, in, n, n_sm, st);
+        if (n <= 4) return launch_probe_decode_t<4, true>(W, D, ws, which, in, n, n_sm, st);
+        return launch_probe_decode_t<8, true>(W, D, ws, which, in, n, n_sm, st);
+    }
+    if (n <= 1) return launch_probe_decode_t<1, false>(W, D, ws, which, in, n, n_sm, st);
+    if (n <= 2) return launch_probe_decode_t<2, false>(W, D, ws, which, in, n, n_sm, st);
+    if (n <= 4) return launch_probe_decode_t<4, false>(W, D, ws, which, in, n, n_sm, st);
+    return launch_probe_decode_t<8, false>(W, D, ws, which, in, n, n_sm, st);
 }
 
 template <int NT>

@@ -17,6 +17,10 @@ __global__ void k_pack_iq2(const float* w, int64_t n_blocks, const uint8_t* grid
 __global__ void k_repack_iq2(const uint8_t* src, int R, int C, uint8_t* qs, uint16_t* dd);
 __global__ void k_repack_q2(const uint8_t* src, int R, int C, uint8_t* q, uint32_t* sc, uint32_t* dd);
 __global__ void k_repack_bf16(const uint4* src, int R, int C, uint4* dst);
+__global__ void k_pack_q4k(const float* w, int64_t n_blocks, uint8_t* out);
+__global__ void k_repack_q4(const uint8_t* src, int R, int C, int mode, uint8_t* q, uint32_t* sc, uint32_t* dd);
+__global__ void k_dequant_q4(const uint8_t* q, const uint32_t* sc, const uint32_t* dd, int R, int C, int mode,
+                             float* out_f, __nv_bfloat16* out_b);
 __global__ void k_interleave_router(const float* W, int E, int H, float* W2);
 __global__ void k_dequant_iq2(const uint8_t* qs, const uint16_t* dd, const uint8_t* grid, int R, int C, float* out_f,
                               __nv_bfloat16* out_b);
@@ -106,6 +110,9 @@ struct ds4moe {
     size_t off_grid, off_gtab, off_Wr, off_Wr2, off_br, off_steer, off_gate_qs, off_gate_d, off_up_qs, off_up_d, off_down_q, off_down_sc,
         off_down_dd, off_sh_gate, off_sh_up, off_sh_down, weight_bytes;
     size_t iq2_qs_stride, iq2_d_stride, q2_q_stride, q2_sc_stride, q2_dd_stride;
+    // 4-bit layers: codes at off_gate_qs / off_up_qs / off_down_q, scale and (d, dmin) words here
+    size_t off_gate_sc4 = 0, off_up_sc4 = 0, off_down_sc4 = 0, off_gate_dd4 = 0, off_up_dd4 = 0, off_down_dd4 = 0;
+    size_t q4_q_stride = 0, q4_sc_stride = 0, q4_dd_stride = 0;
     uint8_t* weights = nullptr;
     uint8_t* ws = nullptr;
     size_t ws_bytes = 0;
@@ -211,6 +218,17 @@ struct ds4moe {
         W.q2_q_stride = q2_q_stride;
         W.q2_sc_stride = q2_sc_stride;
         W.q2_dd_stride = q2_dd_stride;
+        if (D.q4) {
+            W.gate_sc4 = reinterpret_cast<const uint32_t*>(b + off_gate_sc4);
+            W.up_sc4 = reinterpret_cast<const uint32_t*>(b + off_up_sc4);
+            W.down_sc4 = reinterpret_cast<const uint32_t*>(b + off_down_sc4);
+            W.gate_dd4 = reinterpret_cast<const uint32_t*>(b + off_gate_dd4);
+            W.up_dd4 = reinterpret_cast<const uint32_t*>(b + off_up_dd4);
+            W.down_dd4 = reinterpret_cast<const uint32_t*>(b + off_down_dd4);
+            W.q4_q_stride = q4_q_stride;
+            W.q4_sc_stride = q4_sc_stride;
+            W.q4_dd_stride = q4_dd_stride;
+        }
         return W;
     }
 
@@ -262,7 +280,7 @@ struct ds4moe {
     bool ready(std::string* why) const {
         if (!weights) { *why = "buffers not bound"; return false; }
         if (!ws) { *why = "workspace not bound"; return false; }
-        if (!grid_set) { *why = "grid not set"; return false; }
+        if (!grid_set && !D.q4) { *why = "grid not set"; return false; }
         if (!router_set) { *why = "router not set"; return false; }
         if (shape.has_shared && !shared_set) { *why = "shared expert not set"; return false; }
         for (size_t e = 0; e < loaded.size(); ++e)
@@ -288,6 +306,15 @@ ds4moe_status ds4moe_create(const ds4moe_shape* s, ds4moe_t** out) {
     if (s->act_dtype != DS4MOE_ACT_F32 && s->act_dtype != DS4MOE_ACT_BF16)
         return fail(DS4MOE_ERR_SHAPE, "act_dtype %d unknown", s->act_dtype);
     if (s->decode_max < 0 || s->decode_max > 8) return fail(DS4MOE_ERR_SHAPE, "decode_max %d: need 0..8", s->decode_max);
+    if (s->expert_bits != 0 && s->expert_bits != 2 && s->expert_bits != 4)
+        return fail(DS4MOE_ERR_SHAPE, "expert_bits %d: need 0, 2 or 4", s->expert_bits);
+    if (s->expert_bits == 4) {
+        const int dm = s->decode_max ? s->decode_max : 8;
+        if (s->inter % 256) return fail(DS4MOE_ERR_SHAPE, "expert_bits 4: inter %d not a multiple of 256", s->inter);
+        if (s->max_tokens > dm)
+            return fail(DS4MOE_ERR_SHAPE, "expert_bits 4: max_tokens %d above decode_max %d (4-bit layers run the "
+                        "decode plan only)", s->max_tokens, dm);
+    }
     int dev = 0;
     cudaError_t ce = cudaGetDevice(&dev);
     if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
@@ -303,6 +330,7 @@ ds4moe_status ds4moe_create(const ds4moe_shape* s, ds4moe_t** out) {
     h->D.k = s->top_k;
     h->D.has_shared = s->has_shared ? 1 : 0;
     h->D.act_bf16 = s->act_dtype == DS4MOE_ACT_BF16;
+    h->D.q4 = s->expert_bits == 4;
     h->decode_max = s->decode_max ? s->decode_max : 8;
     h->n_sm = n_sm;
     {
@@ -332,13 +360,30 @@ ds4moe_status ds4moe_create(const ds4moe_shape* s, ds4moe_t** out) {
     h->off_Wr2 = o; o += align256(s->max_tokens > h->decode_max ? (E + 1) / 2 * 2 * H * 4 : 0);
     h->off_br = o; o += align256(E * 4);
     h->off_steer = o; o += align256(H * 4);
-    h->off_gate_qs = o; o += align256(E * h->iq2_qs_stride);
-    h->off_gate_d = o; o += align256(E * h->iq2_d_stride * 2);
-    h->off_up_qs = o; o += align256(E * h->iq2_qs_stride);
-    h->off_up_d = o; o += align256(E * h->iq2_d_stride * 2);
-    h->off_down_q = o; o += align256(E * h->q2_q_stride);
-    h->off_down_sc = o; o += align256(E * h->q2_sc_stride * 4);
-    h->off_down_dd = o; o += align256(E * h->q2_dd_stride * 4);
+    if (h->D.q4) {
+        // codes 32 bytes, one scale word per (row, 64 columns), one (d, dmin) word per (row, 256 columns)
+        h->q4_q_stride = I * H / 2;
+        h->q4_sc_stride = I * H / 64;
+        h->q4_dd_stride = I * H / 256;
+        h->off_gate_qs = o; o += align256(E * h->q4_q_stride);
+        h->off_up_qs = o; o += align256(E * h->q4_q_stride);
+        h->off_down_q = o; o += align256(E * h->q4_q_stride);
+        h->off_gate_sc4 = o; o += align256(E * h->q4_sc_stride * 4);
+        h->off_up_sc4 = o; o += align256(E * h->q4_sc_stride * 4);
+        h->off_down_sc4 = o; o += align256(E * h->q4_sc_stride * 4);
+        h->off_gate_dd4 = o; o += align256(E * h->q4_dd_stride * 4);
+        h->off_up_dd4 = o; o += align256(E * h->q4_dd_stride * 4);
+        h->off_down_dd4 = o; o += align256(E * h->q4_dd_stride * 4);
+        h->off_gate_d = h->off_up_d = h->off_down_sc = h->off_down_dd = 0;
+    } else {
+        h->off_gate_qs = o; o += align256(E * h->iq2_qs_stride);
+        h->off_gate_d = o; o += align256(E * h->iq2_d_stride * 2);
+        h->off_up_qs = o; o += align256(E * h->iq2_qs_stride);
+        h->off_up_d = o; o += align256(E * h->iq2_d_stride * 2);
+        h->off_down_q = o; o += align256(E * h->q2_q_stride);
+        h->off_down_sc = o; o += align256(E * h->q2_sc_stride * 4);
+        h->off_down_dd = o; o += align256(E * h->q2_dd_stride * 4);
+    }
     h->off_sh_gate = o; o += align256(s->has_shared ? I * H * 2 : 0);
     h->off_sh_up = o; o += align256(s->has_shared ? I * H * 2 : 0);
     h->off_sh_down = o; o += align256(s->has_shared ? H * I * 2 : 0);
@@ -399,6 +444,16 @@ ds4moe_status ds4moe_pack_q2k(const float* d_w, int64_t n, void* d_blocks, void*
     k_pack_q2k<<<(unsigned)((nb + 127) / 128), 128, 0, (cudaStream_t)stream>>>(d_w, nb, (uint8_t*)d_blocks);
     cudaError_t ce = cudaGetLastError();
     return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "pack_q2k launch");
+}
+
+ds4moe_status ds4moe_pack_q4k(const float* d_w, int64_t n, void* d_blocks, void* stream) {
+    if (!d_w || !d_blocks) return fail(DS4MOE_ERR_ARG, "pack_q4k: NULL argument");
+    if (n <= 0 || n % kQK) return fail(DS4MOE_ERR_ARG, "pack_q4k: n_weights %lld not a positive multiple of 256", (long long)n);
+    if (!aligned16(d_w)) return fail(DS4MOE_ERR_ALIGN, "pack_q4k: weights not 16-byte aligned");
+    const int64_t nb = n / kQK;
+    k_pack_q4k<<<(unsigned)((nb + 127) / 128), 128, 0, (cudaStream_t)stream>>>(d_w, nb, (uint8_t*)d_blocks);
+    cudaError_t ce = cudaGetLastError();
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "pack_q4k launch");
 }
 
 ds4moe_status ds4moe_pack_iq2xxs(const float* d_w, int64_t n, const uint8_t* d_grid, void* d_blocks, void* stream) {
@@ -471,6 +526,25 @@ ds4moe_status ds4moe_set_expert(ds4moe_t* h, int32_t e, const void* d_gate, cons
     if (e < 0 || e >= h->D.E) return fail(DS4MOE_ERR_ARG, "set_expert: expert %d out of range", e);
     cudaStream_t st = (cudaStream_t)stream;
     const int H = h->D.H, I = h->D.I;
+    if (h->D.q4) {
+        const int64_t nsteps = (int64_t)I * H / 64;   // (row, 64-column step) pieces of each matrix
+        const unsigned g = (unsigned)((nsteps + 255) / 256);
+        uint8_t* b = h->weights;
+        const size_t qo = e * h->q4_q_stride, so = e * h->q4_sc_stride, dof = e * h->q4_dd_stride;
+        k_repack_q4<<<g, 256, 0, st>>>((const uint8_t*)d_gate, I, H, 0, b + h->off_gate_qs + qo,
+                                       reinterpret_cast<uint32_t*>(b + h->off_gate_sc4) + so,
+                                       reinterpret_cast<uint32_t*>(b + h->off_gate_dd4) + dof);
+        k_repack_q4<<<g, 256, 0, st>>>((const uint8_t*)d_up, I, H, 0, b + h->off_up_qs + qo,
+                                       reinterpret_cast<uint32_t*>(b + h->off_up_sc4) + so,
+                                       reinterpret_cast<uint32_t*>(b + h->off_up_dd4) + dof);
+        k_repack_q4<<<g, 256, 0, st>>>((const uint8_t*)d_down, H, I, 1, b + h->off_down_q + qo,
+                                       reinterpret_cast<uint32_t*>(b + h->off_down_sc4) + so,
+                                       reinterpret_cast<uint32_t*>(b + h->off_down_dd4) + dof);
+        cudaError_t ce = cudaGetLastError();
+        if (ce != cudaSuccess) return cuda_fail(ce, "set_expert launch");
+        h->loaded[e] = 1;
+        return DS4MOE_OK;
+    }
     const int64_t nb = (int64_t)I * H / kQK;
     const unsigned g1 = (unsigned)((nb * 8 + 255) / 256);
     k_repack_iq2<<<g1, 256, 0, st>>>((const uint8_t*)d_gate, I, H, h->weights + h->off_gate_qs + e * h->iq2_qs_stride,
@@ -703,7 +777,18 @@ ds4moe_status ds4moe_dequant(ds4moe_t* h, int32_t e, int32_t which, int32_t as_b
     } else {
         if (e < 0 || e >= h->D.E) return fail(DS4MOE_ERR_ARG, "dequant: expert %d out of range", e);
         if (!h->loaded[e]) return fail(DS4MOE_ERR_NOT_READY, "dequant: expert %d not loaded", e);
-        if (which == 0 || which == 1) {
+        if (h->D.q4) {
+            if (which < 0 || which > 2) return fail(DS4MOE_ERR_ARG, "dequant: which %d", which);
+            const size_t oq = which == 0 ? h->off_gate_qs : which == 1 ? h->off_up_qs : h->off_down_q;
+            const size_t os = which == 0 ? h->off_gate_sc4 : which == 1 ? h->off_up_sc4 : h->off_down_sc4;
+            const size_t od = which == 0 ? h->off_gate_dd4 : which == 1 ? h->off_up_dd4 : h->off_down_dd4;
+            const int R = which == 2 ? H : I, C = which == 2 ? I : H;
+            const unsigned g4 = (unsigned)(((int64_t)R * (C / 64) + 255) / 256);
+            k_dequant_q4<<<g4, 256, 0, st>>>(h->weights + oq + e * h->q4_q_stride,
+                                             reinterpret_cast<const uint32_t*>(h->weights + os) + e * h->q4_sc_stride,
+                                             reinterpret_cast<const uint32_t*>(h->weights + od) + e * h->q4_dd_stride,
+                                             R, C, which == 2 ? 1 : 0, of, ob);
+        } else if (which == 0 || which == 1) {
             if (!h->grid_set) return fail(DS4MOE_ERR_NOT_READY, "dequant: grid not set");
             const size_t oq = which == 0 ? h->off_gate_qs : h->off_up_qs;
             const size_t od = which == 0 ? h->off_gate_d : h->off_up_d;

@@ -16,6 +16,26 @@
 //                of the superblock holding column 256*sb of the row
 // The algorithmic bytes equal the canonical blocks' bytes (66 and 84 per 256
 // weights) except that a C < 256 matrix stores its (d, dmin) once per row.
+// Q4 layout (layers with 4-bit experts), per matrix:
+//   Q4 codes     [R/32][C/64][32][32 B]  64 four-bit codes in the code order
+//                                        below
+//   Q4 scales    [R/32][C/64][32][4 B]   sc of the 32-weight sub-blocks 2j, 2j+1
+//                                        of the 64 columns, then their m
+//   Q4 d,dmin    [R/32][C/256][32][2 x binary16]
+// (148 bytes per 256 weights against the block's 144: the 6-bit fields are
+// kept as bytes).
+// Q4 code order: nibble i of word h of lane t (byte 8t + 4h + i/2 of a row's
+// 64-column step) holds the code of column q4_dev_col(mode, t, h, i).
+//   mode 0 (gate, up; int8 m16n8k32 fragments): word h is the 32-column half
+//     h; its low nibbles (i even) are columns 8t + i/2, the high nibbles
+//     columns 8t + 4 + i/2 -- one mask gives the A register of columns
+//     8t..8t+3, a shift and the mask that of 8t+4..8t+7.
+//   mode 1 (down; bf16 m16n8k16 fragments over the routed h layout, where
+//     lane t's four values of a 16-column group are its columns t, 4+t, 8+t,
+//     12+t): word h covers the 16-column groups 2h, 2h+1; nibbles (p, p+4)
+//     are columns 16 (2h + p/2) + 8 (p & 1) + t + {0, 4}, so that one shift
+//     and mask of the word lands both codes in a bf16 pair's mantissas.
+//   (q4_dev_col below.)
 // Shared (bf16) matrices are stored in 8x8 core-matrix tiles:
 //   [R/8][C/8][8 rows][8 cols], 128 contiguous bytes per tile.
 // IQ2 S word, device order: byte c (c = 0..3) holds the seven stored signs of
@@ -44,6 +64,16 @@ __host__ __device__ __forceinline__ uint32_t iq2_dev_scale(uint32_t Sd) {
 }
 __host__ __device__ __forceinline__ uint32_t iq2_dev_signs(uint32_t Sd, int c) { return (Sd >> (8 * c)) & 127u; }
 constexpr int kQ2Bytes = 84;
+constexpr int kQ4Bytes = 144;
+
+// Column (0..63, within a 64-column step) of the Q4 code at nibble i of word
+// h of lane t, for the gate/up (mode 0) and down (mode 1) code orders.
+__host__ __device__ __forceinline__ int q4_dev_col(int mode, int t, int h, int i) {
+    if (mode == 0) return 32 * h + 8 * t + 4 * (i & 1) + (i >> 1);
+    const int p = i & 3, e = i >> 2;
+    return 32 * h + 16 * (p >> 1) + 8 * (p & 1) + 4 * e + t;
+}
+
 constexpr int kIQ2Bytes = 66;
 
 enum : uint32_t { kErrBounds = 1u, kErrTimeout = 2u, kErrGrid = 4u };
@@ -69,12 +99,23 @@ struct Weights {
     const __nv_bfloat16* sh_up;
     const __nv_bfloat16* sh_down;   // [H/8][I/8][8][8]
     size_t iq2_qs_stride, iq2_d_stride, q2_q_stride, q2_sc_stride, q2_dd_stride;
+    // Q4 layout (expert_bits 4): codes in gate_qs / up_qs / down_q, expert stride q4_q_stride bytes; scale
+    // words and (d, dmin) words below, expert strides q4_sc_stride / q4_dd_stride words (gate and up share
+    // the strides; down's shape is the transpose, same sizes)
+    const uint32_t* gate_sc4;
+    const uint32_t* up_sc4;
+    const uint32_t* down_sc4;
+    const uint32_t* gate_dd4;
+    const uint32_t* up_dd4;
+    const uint32_t* down_dd4;
+    size_t q4_q_stride, q4_sc_stride, q4_dd_stride;
 };
 
 struct Dims {
     int H, I, E, k;
     int has_shared;
     int act_bf16;
+    int q4;                     // routed experts in the Q4 layout (all three matrices)
 };
 
 // Workspace pointers (decode plan).

@@ -54,6 +54,67 @@ __global__ void k_pack_q2k(const float* __restrict__ w, int64_t n_blocks, uint8_
     for (int i = 0; i < kQ2Bytes; ++i) o[i] = blk[i];
 }
 
+// ---------------------------------------------------------------- Q4_K-style
+// 6-bit field f of the little-endian 96-bit integer held in bytes 4..15 of a
+// block.
+__device__ __forceinline__ void q4_set_field(uint8_t* blk, int f, int v) {
+    for (int b = 0; b < 6; ++b) {
+        const int bit = 6 * f + b;
+        blk[4 + bit / 8] |= (uint8_t)(((v >> b) & 1) << (bit % 8));
+    }
+}
+__device__ __forceinline__ int q4_field(const uint8_t* blk, int f) {
+    int v = 0;
+    for (int b = 0; b < 6; ++b) {
+        const int bit = 6 * f + b;
+        v |= ((blk[4 + bit / 8] >> (bit % 8)) & 1) << b;
+    }
+    return v;
+}
+
+// One thread per 256-weight block: eight 32-weight sub-blocks, the Q2_K-style
+// rule with 4-bit codes and 6-bit scales and mins.
+__global__ void k_pack_q4k(const float* __restrict__ w, int64_t n_blocks, uint8_t* __restrict__ out) {
+    int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= n_blocks) return;
+    const float* x = w + b * kQK;
+    uint8_t blk[kQ4Bytes];
+    double scale[8], mn[8], max_scale = 0.0, max_min = 0.0;
+    for (int j = 0; j < 8; ++j) {
+        double lo = 0.0, hi = 0.0;
+        for (int i = 0; i < 32; ++i) {
+            const double v = (double)x[32 * j + i];
+            lo = v < lo ? v : lo;
+            hi = v > hi ? v : hi;
+        }
+        scale[j] = __ddiv_rn(__dsub_rn(hi, lo), 15.0);
+        mn[j] = -lo;
+        max_scale = scale[j] > max_scale ? scale[j] : max_scale;
+        max_min = mn[j] > max_min ? mn[j] : max_min;
+    }
+    const uint16_t dh = to_half_bits(__ddiv_rn(max_scale, 63.0));
+    const uint16_t mh = to_half_bits(__ddiv_rn(max_min, 63.0));
+    const double d = from_half_bits(dh), dmin = from_half_bits(mh);
+    for (int i = 0; i < kQ4Bytes; ++i) blk[i] = 0;
+    for (int j = 0; j < 8; ++j) {
+        const int sc = d > 0.0 ? (int)clamp_rne(__ddiv_rn(scale[j], d), 63.0) : 0;
+        const int m = dmin > 0.0 ? (int)clamp_rne(__ddiv_rn(mn[j], dmin), 63.0) : 0;
+        q4_set_field(blk, j, sc);
+        q4_set_field(blk, 8 + j, m);
+        const double step = __dmul_rn(d, (double)sc), off = __dmul_rn(dmin, (double)m);
+        for (int i = 0; i < 32; ++i) {
+            int q = 0;
+            if (step > 0.0) q = (int)clamp_rne(__ddiv_rn(__dadd_rn((double)x[32 * j + i], off), step), 15.0);
+            const int kk = 32 * j + i;
+            blk[16 + kk / 2] |= (uint8_t)(q << (4 * (kk % 2)));
+        }
+    }
+    blk[0] = dh & 0xff; blk[1] = dh >> 8;
+    blk[2] = mh & 0xff; blk[3] = mh >> 8;
+    uint8_t* o = out + b * kQ4Bytes;
+    for (int i = 0; i < kQ4Bytes; ++i) o[i] = blk[i];
+}
+
 // ---------------------------------------------------------------- IQ2_XXS-style
 // One warp per 256-weight block; lane = 8-weight chunk (group = lane / 4).
 __global__ void k_pack_iq2(const float* __restrict__ w, int64_t n_blocks, const uint8_t* __restrict__ grid,
@@ -172,6 +233,39 @@ __global__ void k_repack_q2(const uint8_t* __restrict__ src, int R, int C, uint8
     }
 }
 
+// Q4 canonical blocks of an [R][C] matrix (C a multiple of 256) -> codes
+// [R/32][C/64][32][32 B], scale words [R/32][C/64][32] and (d, dmin) words
+// [R/32][C/256][32].  Code byte 8t + 4h + i/2 (nibble i & 1) of a row's
+// 64-column step holds the code of column q4_dev_col(mode, t, h, i).  One
+// thread per (row, 64-column step).
+__global__ void k_repack_q4(const uint8_t* __restrict__ src, int R, int C, int mode, uint8_t* __restrict__ q,
+                            uint32_t* __restrict__ sc, uint32_t* __restrict__ dd) {
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int nkt = C / 64;
+    if (gid >= (int64_t)R * nkt) return;
+    const int r = (int)(gid / nkt), kt = (int)(gid % nkt);
+    const uint8_t* blk = src + ((int64_t)r * (C / kQK) + kt / 4) * kQ4Bytes;
+    const int o = 64 * (kt % 4);   // first weight of the step in the block
+    const int64_t piece = ((int64_t)(r >> 5) * nkt + kt) * 32 + (r & 31);
+    uint8_t bytes[32];
+    for (int i = 0; i < 32; ++i) bytes[i] = 0;
+    for (int t = 0; t < 4; ++t)
+        for (int h = 0; h < 2; ++h)
+            for (int i = 0; i < 8; ++i) {
+                const int c = o + q4_dev_col(mode, t, h, i);
+                const uint32_t code = (blk[16 + c / 2] >> (4 * (c % 2))) & 15u;
+                bytes[8 * t + 4 * h + i / 2] |= (uint8_t)(code << (4 * (i & 1)));
+            }
+    uint8_t* qd = q + piece * 32;
+    for (int i = 0; i < 32; ++i) qd[i] = bytes[i];
+    const int j0 = 2 * (kt % 4);   // the step's two 32-weight sub-blocks
+    sc[piece] = (uint32_t)q4_field(blk, j0) | ((uint32_t)q4_field(blk, j0 + 1) << 8) |
+                ((uint32_t)q4_field(blk, 8 + j0) << 16) | ((uint32_t)q4_field(blk, 9 + j0) << 24);
+    if (kt % 4 == 0)
+        dd[((int64_t)(r >> 5) * (C / kQK) + kt / 4) * 32 + (r & 31)] =
+            (uint32_t)blk[0] | ((uint32_t)blk[1] << 8) | ((uint32_t)blk[2] << 16) | ((uint32_t)blk[3] << 24);
+}
+
 // bf16 row-major [R][C] -> core-matrix tiles [R/8][C/8][8][8].
 __global__ void k_repack_bf16(const uint4* __restrict__ src, int R, int C, uint4* __restrict__ dst) {
     int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -228,6 +322,32 @@ __global__ void k_dequant_q2(const uint8_t* __restrict__ q, const uint32_t* __re
     float v = (d * (float)(sb & 15u)) * (float)code - dmin * (float)(sb >> 4);
     if (out_f) out_f[gid] = v;
     else out_b[gid] = __float2bfloat16_rn(v);
+}
+
+// One thread per (row, 64-column step): the step's 64 values.
+__global__ void k_dequant_q4(const uint8_t* __restrict__ q, const uint32_t* __restrict__ sc,
+                             const uint32_t* __restrict__ dd, int R, int C, int mode, float* out_f,
+                             __nv_bfloat16* out_b) {
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int nkt = C / 64;
+    if (gid >= (int64_t)R * nkt) return;
+    const int r = (int)(gid / nkt), kt = (int)(gid % nkt);
+    const int64_t piece = ((int64_t)(r >> 5) * nkt + kt) * 32 + (r & 31);
+    const uint32_t sw = sc[piece];
+    const uint32_t p = dd[((int64_t)(r >> 5) * (C / kQK) + kt / 4) * 32 + (r & 31)];
+    const float d = half_bits(p & 0xffffu), dmin = half_bits(p >> 16);
+    for (int t = 0; t < 4; ++t)
+        for (int h = 0; h < 2; ++h)
+            for (int i = 0; i < 8; ++i) {
+                const int c = q4_dev_col(mode, t, h, i);
+                const uint32_t code = (q[piece * 32 + 8 * t + 4 * h + i / 2] >> (4 * (i & 1))) & 15u;
+                const int j = c / 32;
+                const float v = (d * (float)((sw >> (8 * j)) & 0xffu)) * (float)code -
+                                dmin * (float)((sw >> (16 + 8 * j)) & 0xffu);
+                const int64_t at = (int64_t)r * C + 64 * kt + c;
+                if (out_f) out_f[at] = v;
+                else out_b[at] = __float2bfloat16_rn(v);
+            }
 }
 
 __global__ void k_dequant_bf16_tiles(const __nv_bfloat16* __restrict__ t, int R, int C, float* out_f,

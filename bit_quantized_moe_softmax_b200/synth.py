@@ -12,7 +12,8 @@ Recipes (the pages publish no weights or prompts; these stand in for them):
     packs with its own packer.
   * quantized experts, full shapes: the packed fields drawn directly -- every
     byte uniform, except the binary16 scales d (and dmin) which are uniform in
-    [1e-3, 4e-3].
+    [1e-3, 4e-3] (4-bit blocks: [1e-4, 4e-4], the range a packer gives
+    N(0, 0.02) weights, since their codes and 6-bit scales reach 15 and 63).
   * grid: 256 distinct rows of 8 magnitudes drawn from {8, 25, 43}.
   * Zipf(s) expert popularity: router bias b_e = ln p_{pi(e)}, p_r ~ r^-s over
     ranks r = 1..E, pi a seeded permutation.
@@ -26,6 +27,7 @@ import torch
 
 Q2_BYTES = 84
 IQ2_BYTES = 66
+Q4_BYTES = 144
 QK = 256
 
 
@@ -76,6 +78,14 @@ def random_q2k_blocks(n_blocks: int, g, device="cpu", lo=1e-3, hi=4e-3) -> torch
     b = torch.randint(0, 256, (n_blocks, Q2_BYTES), generator=g, device=device, dtype=torch.uint8)
     dd = _fp16_uniform(2 * n_blocks, lo, hi, g, device).view(torch.uint8).view(n_blocks, 4)
     b[:, 80:84] = dd
+    return b
+
+
+def random_q4k_blocks(n_blocks: int, g, device="cpu", lo=1e-4, hi=4e-4) -> torch.Tensor:
+    """[n_blocks, 144] uint8 Q4_K-style blocks with uniform bytes and d, dmin ~ U[lo, hi] (binary16)."""
+    b = torch.randint(0, 256, (n_blocks, Q4_BYTES), generator=g, device=device, dtype=torch.uint8)
+    dd = _fp16_uniform(2 * n_blocks, lo, hi, g, device).view(torch.uint8).view(n_blocks, 4)
+    b[:, 0:4] = dd
     return b
 
 
@@ -134,12 +144,14 @@ def float_layer(shape: Shape, seed: int, router_std=0.02, expert_std=0.02, share
 
 
 def packed_layer(shape: Shape, seed: int, router_std=0.02, shared_std=0.02,
-                 bias: torch.Tensor | None = None, device="cpu", d_range=(1e-3, 4e-3)) -> dict:
+                 bias: torch.Tensor | None = None, device="cpu", d_range=None, expert_bits=2) -> dict:
     """A layer whose quantized experts are drawn directly as packed blocks.
 
     Keys: W_r, b_r, grid as in float_layer; gate/up [E, I*H/256, 66] u8,
-    down [E, H*I/256, 84] u8; sh_gate/sh_up/sh_down bf16.  d_range: the
-    interval of the binary16 superblock scales d (and dmin).
+    down [E, H*I/256, 84] u8 (expert_bits 4: all three [E, n/256, 144] u8,
+    and expert_bits = 4); sh_gate/sh_up/sh_down bf16.  d_range: the interval
+    of the binary16 superblock scales d (and dmin); default [1e-3, 4e-3]
+    ([1e-4, 4e-4] for 4-bit blocks).
     """
     g = gen(seed, device)
     H, I, E = shape.H, shape.I, shape.E
@@ -148,10 +160,16 @@ def packed_layer(shape: Shape, seed: int, router_std=0.02, shared_std=0.02,
     layer["W_r"] = normal((E, H), router_std, g, device)
     layer["b_r"] = bias
     layer["grid"] = grid_table(seed)
-    lo, hi = d_range
-    layer["gate"] = random_iq2_blocks(E * nb, g, device, lo, hi).view(E, nb, IQ2_BYTES)
-    layer["up"] = random_iq2_blocks(E * nb, g, device, lo, hi).view(E, nb, IQ2_BYTES)
-    layer["down"] = random_q2k_blocks(E * nb, g, device, lo, hi).view(E, nb, Q2_BYTES)
+    if expert_bits == 4:
+        lo, hi = d_range or (1e-4, 4e-4)
+        for name in ("gate", "up", "down"):
+            layer[name] = random_q4k_blocks(E * nb, g, device, lo, hi).view(E, nb, Q4_BYTES)
+        layer["expert_bits"] = 4
+    else:
+        lo, hi = d_range or (1e-3, 4e-3)
+        layer["gate"] = random_iq2_blocks(E * nb, g, device, lo, hi).view(E, nb, IQ2_BYTES)
+        layer["up"] = random_iq2_blocks(E * nb, g, device, lo, hi).view(E, nb, IQ2_BYTES)
+        layer["down"] = random_q2k_blocks(E * nb, g, device, lo, hi).view(E, nb, Q2_BYTES)
     if shape.shared:
         layer["sh_gate"] = bf16_normal((I, H), shared_std, g, device)
         layer["sh_up"] = bf16_normal((I, H), shared_std, g, device)

@@ -72,9 +72,19 @@ typedef struct {
     int32_t act_dtype;     /* DS4MOE_ACT_F32 or DS4MOE_ACT_BF16: element type of x */
     int32_t has_shared;    /* 1: add the bf16 shared expert; 0: routed experts only */
     int32_t has_bias;      /* 1: the router adds a bias b[E] */
-    int32_t decode_max;    /* n_tokens <= decode_max uses the fp32 GEMV plan
+    int32_t decode_max;    /* n_tokens <= decode_max uses the decode plan
                               (0 selects the default, 8); larger n uses the
                               bf16 tensor-core plan */
+    int32_t expert_bits;   /* routed-expert format: 0 or 2 = gate, up IQ2_XXS-
+                              style and down Q2_K-style blocks; 4 = all three
+                              Q4_K-style blocks (144 bytes per 256 weights:
+                              d, dmin binary16; sixteen 6-bit fields (eight
+                              scales, eight mins of 32-weight sub-blocks) in
+                              the little-endian 96-bit integer of bytes 4..15;
+                              the 4-bit code of weight i at byte 16 + i/2, low
+                              nibble for even i; weight = d sc q - dmin m).
+                              4-bit layers run the decode plan only:
+                              max_tokens <= decode_max, inter % 256 == 0. */
 } ds4moe_shape;
 
 typedef struct ds4moe ds4moe_t;   /* opaque handle; host memory owned by the library */
@@ -124,6 +134,14 @@ ds4moe_status ds4moe_pack_q2k(const float* d_w, int64_t n_weights, void* d_block
 ds4moe_status ds4moe_pack_iq2xxs(const float* d_w, int64_t n_weights, const uint8_t* d_grid, void* d_blocks,
                                  void* stream);
 
+/* Quantize into Q4_K-style blocks (n_weights/256 * 144 bytes).  Decisions in
+ * fp64, the Q2_K-style rule with 32-weight sub-blocks: per sub-block
+ * lo = min(0, min w), hi = max(0, max w), scale = (hi-lo)/15, min = -lo;
+ * d = half(max scale/63), dmin = half(max min/63);
+ * sc = clamp(rne(scale/d), 0, 63), m = clamp(rne(min/dmin), 0, 63);
+ * q = clamp(rne((w + dmin m)/(d sc)), 0, 15); zero divisors give zero fields. */
+ds4moe_status ds4moe_pack_q4k(const float* d_w, int64_t n_weights, void* d_blocks, void* stream);
+
 /* ---- loading (device pointers in; repacked into the bound weight buffer) - */
 
 /* Grid magnitudes [256][8] uint8.  The prefill plan (n_tokens > decode_max)
@@ -137,7 +155,9 @@ ds4moe_status ds4moe_set_grid(ds4moe_t* h, const uint8_t* d_grid, void* stream);
 ds4moe_status ds4moe_set_router(ds4moe_t* h, const float* d_W, const float* d_bias, void* stream);
 
 /* Expert e's three matrices as canonical blocks: gate, up IQ2_XXS-style
- * ([I][H] -> I*H/256 blocks), down Q2_K-style ([H][I] -> H*I/256 blocks). */
+ * ([I][H] -> I*H/256 blocks), down Q2_K-style ([H][I] -> H*I/256 blocks); for
+ * a layer created with expert_bits = 4 all three Q4_K-style (same block
+ * counts, 144 bytes each). */
 ds4moe_status ds4moe_set_expert(ds4moe_t* h, int32_t e, const void* d_gate, const void* d_up,
                                 const void* d_down, void* stream);
 

@@ -27,3 +27,12 @@ def pack_with_oracle(orc, layer: dict) -> dict:
     up = np.stack([orc.pack_iq2xxs(layer["up_f"][e].numpy(), grid) for e in range(E)])
     down = np.stack([orc.pack_q2k(layer["down_f"][e].numpy()) for e in range(E)])
     return dict(gate=torch.from_numpy(gate), up=torch.from_numpy(up), down=torch.from_numpy(down))
+
+
+def pack_q4_with_oracle(orc, layer: dict) -> dict:
+    """Q4_K-style blocks of a float layer's three expert matrices, packed by the oracle."""
+    E = layer["E"]
+    out = {n: torch.from_numpy(np.stack([orc.pack_q4k(layer[n + "_f"][e].numpy()) for e in range(E)]))
+           for n in ("gate", "up", "down")}
+    out["expert_bits"] = 4
+    return out

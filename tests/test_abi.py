@@ -79,3 +79,18 @@ def test_binding_signatures_match_header(libpath):
     assert fields == [f for f, _ in m.ds4moe_shape._fields_]
     assert all(t is ctypes.c_int32 for _, t in m.ds4moe_shape._fields_)
     assert "int32_t" in body and not re.search(r"\b(int64_t|size_t|float|double)\b", body)
+
+
+def test_q4_shape_rules_without_gpu(libpath):
+    """Shape checks come before any CUDA call: 4-bit layers need inter a
+    multiple of 256 and max_tokens <= decode_max; other bit widths are refused."""
+    import bit_quantized_moe_softmax_b200 as m
+
+    for kw, why in ((dict(inter=128), "inter"), (dict(max_tokens=9), "max_tokens"),
+                    (dict(max_tokens=5, decode_max=4), "decode_max"), (dict(expert_bits=3), "bits")):
+        args = dict(inter=256, max_tokens=8, decode_max=0, expert_bits=4)
+        args.update(kw)
+        with pytest.raises(m.Ds4MoeError) as ei:
+            m.ds4moe_create(256, args["inter"], 8, 2, args["max_tokens"], decode_max=args["decode_max"],
+                            expert_bits=args["expert_bits"])
+        assert ei.value.status == -3, why
