@@ -44,6 +44,9 @@ WORKLOADS = {
     "decode": dict(n=1, H=4096, I=2048, E=256, k=8,
                    desc="decode step: 1 token, one MoE layer (hidden 4096, expert intermediate 2048, "
                         "256 routed experts top-8 in IQ2_XXS/Q2_K-style 2-bit blocks, 1 bf16 shared expert)"),
+    "decode_q4": dict(n=1, H=4096, I=2048, E=256, k=8, expert_bits=4,
+                      desc="decode step, 4-bit experts: 1 token, one MoE layer (hidden 4096, expert intermediate "
+                           "2048, 256 routed experts top-8 in Q4_K-style blocks, 1 bf16 shared expert)"),
     "decode8": dict(n=8, H=4096, I=2048, E=256, k=8,
                     desc="MTP-verify style decode: 8 tokens, one MoE layer of the decode shape"),
     "decode2": dict(n=2, H=4096, I=2048, E=256, k=8,
@@ -82,6 +85,8 @@ def algorithmic_bytes(w: dict, U: int) -> dict:
     H, I, E, k, n = w["H"], w["I"], w["E"], w["k"], w["n"]
     iq2 = I * H // 256 * 66          # one gate or up matrix
     q2 = H * I // 256 * 84           # one down matrix
+    if w.get("expert_bits") == 4:    # all three matrices in 144-byte Q4_K-style blocks
+        iq2 = q2 = I * H // 256 * 144
     sh_gu, sh_d = 2 * I * H * 2, H * I * 2
     return {
         "k_router_decode": E * H * 4 + n * H * 4 + n * E * 4,
@@ -257,9 +262,11 @@ def run_ours(args, wl, rank, local, world):
     layers = []
     for r in range(R):
         L = synth.packed_layer(shape, seed=1000 * rank + r, router_std=wl.get("router_std", 0.02), bias=bias,
-                               device=dev, d_range=synth.CHAIN_D_RANGE if wl.get("chain_scales") else (1e-3, 4e-3),
-                               shared_std=synth.CHAIN_SHARED_STD if wl.get("chain_scales") else 0.02)
-        lay = m.MoELayer(H, I, E, k, max_tokens=max(n, 8), act_dtype=act, has_bias=bias is not None, device=dev)
+                               device=dev, d_range=synth.CHAIN_D_RANGE if wl.get("chain_scales") else None,
+                               shared_std=synth.CHAIN_SHARED_STD if wl.get("chain_scales") else 0.02,
+                               expert_bits=wl.get("expert_bits", 2))
+        lay = m.MoELayer(H, I, E, k, max_tokens=max(n, 8), act_dtype=act, has_bias=bias is not None, device=dev,
+                         expert_bits=wl.get("expert_bits", 0))
         lay.load(L)
         if args.steer:
             v = synth.normal((H,), 1.0, synth.gen(500 + r, dev), dev)
@@ -454,6 +461,7 @@ def _timed_run(args, wl, rank, local, world, dev, layers, xs, outs, stream, nl, 
                    else "ds4moe_forward_host_async per step (two staging slots per layer), ds4moe_host_sync at the end")}
 
     # roofline of the dominant kernel
+    wname = next(key for key, v in WORKLOADS.items() if v is wl)
     peaks, peak_kind = load_peaks()
     mean = {nm: (statistics.mean(v) if v else 0.0) for nm, v in durs.items()}
     dom = max(mean, key=lambda nm: mean[nm])
@@ -467,7 +475,7 @@ def _timed_run(args, wl, rank, local, world, dev, layers, xs, outs, stream, nl, 
         peak = peaks["bf16_tflops"]
         sustained_s = ms_per_step * args.steps / 1e3
         roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
-                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic_from_profile(dom, args.workload),
+                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic_from_profile(dom, wname),
                     "algorithmic_flops_per_launch": fl[dom], "mean_launch_us": round(mean[dom] * 1e3, 2),
                     # the same launch against HBM: weights of the touched experts, activations in and out
                     "hbm_view": ({"achieved": round(ab[dom] / (mean[dom] * 1e-3) / 1e9, 1), "peak": peaks["hbm_gbs"],
@@ -484,7 +492,7 @@ def _timed_run(args, wl, rank, local, world, dev, layers, xs, outs, stream, nl, 
         achieved = ab[dom] / (mean[dom] * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                    "frac": round(achieved / peak, 4), "traffic": traffic_from_profile(dom, args.workload),
+                    "frac": round(achieved / peak, 4), "traffic": traffic_from_profile(dom, wname),
                     "algorithmic_bytes_per_launch": int(round(ab[dom])), "mean_launch_us": round(mean[dom] * 1e3, 2),
                     "nominal": {"peak": NOMINAL["hbm_gbs"], "frac": round(achieved / NOMINAL["hbm_gbs"], 4),
                                 "source": NOMINAL["source"]},
@@ -546,7 +554,8 @@ def oracle_sample(wl, n_tokens, seed=0, budget_s=20.0, device="cuda"):
     bias = synth.zipf_bias(E, wl["zipf"], seed=5) if wl.get("zipf") else None
     if wl.get("layers", 1) > 1:
         return oracle_chain_sample(wl, n_tokens, seed, budget_s, device)
-    L = synth.packed_layer(synth.Shape(H=H, I=I, E=E, k=k), seed=seed, bias=bias, device=device)
+    L = synth.packed_layer(synth.Shape(H=H, I=I, E=E, k=k), seed=seed, bias=bias, device=device,
+                           expert_bits=wl.get("expert_bits", 2))
     x = synth.tokens(n_tokens, H, seed=seed + 5, dtype=torch.bfloat16 if wl.get("bf16") else torch.float32).float()
     mode = 1 if wl.get("bf16") else 0
     lg = oracle.router_logits(x.numpy(), L["W_r"].cpu().numpy(), None if bias is None else bias.numpy())
@@ -612,7 +621,7 @@ def run_reference(args, wl, rank, world):
             "e2e": {"value": round(rate, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-SUB_WORKLOADS = ("prefill512", "prefill11709")
+SUB_WORKLOADS = ("decode_q4", "prefill512", "prefill11709")
 
 
 def sub_record(line: dict) -> dict:
@@ -632,7 +641,7 @@ def main():
     ap.add_argument("--instances", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
-                    help="with the default decode workload: skip the prefill sub-records")
+                    help="with the default decode workload: skip the sub-records (4-bit decode, prefill)")
     ap.add_argument("--steer", type=float, default=0.0,
                     help="directional steering strength F of every layer (unit direction, seeded); 0: off")
     args = ap.parse_args()
@@ -656,7 +665,8 @@ def main():
     line = run_ours(args, wl, rank, local, world)
     if baseline:
         line["cpu_baseline"] = cpu_baseline_record(wl, n_tokens=4 * cores, budget_s=15.0, device=dev)
-    # the metric covers decode and prefill: the default run adds both prefill workloads as sub-records
+    # the metric covers decode and prefill: the default run adds the 4-bit decode step and both prefill
+    # workloads as sub-records
     if args.workload == "decode" and not args.no_prefill:
         subs = {}
         for name in SUB_WORKLOADS:

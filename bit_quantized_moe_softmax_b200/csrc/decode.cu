@@ -229,24 +229,38 @@ __device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t* err) {
     }
 }
 
-// Waits (bounded) until *counter >= target, reading it with acquire semantics, then orders the
-// generic-proxy writes it published before this thread's later bulk copies (async proxy).
-__device__ __forceinline__ bool wait_count(const uint32_t* counter, uint32_t target, uint32_t* err) {
+// Producer warp: waits (bounded) until gate/up completion counter c (0: the shared expert, 1 + u: entry u)
+// has reached its target (t_sh for counter 0, t_rt for the others).  `known` caches what earlier polls saw
+// (per lane, bit j: counter lane + 32 j complete), so a complete counter is not read again; a poll reads
+// every unfinished counter at once, one per lane and word, instead of one load latency per task.  Orders
+// the generic-proxy writes it observed before the warp's later bulk copies.
+__device__ __forceinline__ bool wait_deps_warp(const uint32_t* ctr, int c, int ncnt, uint32_t t_sh, uint32_t t_rt,
+                                               uint32_t& known, uint32_t* err) {
+    const int lane = threadIdx.x & 31;
     uint64_t t0 = 0;
     for (;;) {
-        uint32_t v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
-        if (v >= target) break;
+        const uint32_t kb = __shfl_sync(0xffffffffu, known, c & 31);
+        if ((kb >> (c >> 5)) & 1u) return true;
+        if (t0 != 0) __nanosleep(32);
+#pragma unroll
+        for (int j = 0; j < 5; ++j) {
+            const int idx = lane + 32 * j;
+            if (idx < ncnt && !((known >> j) & 1u)) {
+                uint32_t v;
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr + idx) : "memory");
+                if (v >= (idx == 0 ? t_sh : t_rt)) known |= 1u << j;
+            }
+        }
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncwarp();
+        const uint64_t now = __shfl_sync(0xffffffffu, (unsigned long long)global_ns(), 0);
         if (t0 == 0) {
-            t0 = global_ns();
-        } else if (global_ns() - t0 > kWaitNs) {
-            set_err(err, kErrTimeout);
+            t0 = now;
+        } else if (now - t0 > kWaitNs) {
+            if (lane == 0) set_err(err, kErrTimeout);
             return false;
         }
-        __nanosleep(32);
     }
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-    return true;
 }
 
 // ---------------------------------------------------------------- routing table
@@ -497,28 +511,35 @@ __device__ __forceinline__ void ring_free(RedRing& R, uint32_t j, int nb) {
 }
 
 // x (n tokens of H) as four int8 pieces per value, [n][4][H] bytes: v = x f1 f2 (|v| < 128), piece p
-// = trunc of the remaining fraction times 128^p.  Threads tid of nthreads, four values each.
+// = trunc of the remaining fraction times 128^p.  quantize4 writes values i..i+3 of token tk.
+__device__ __forceinline__ void quantize4(float4 xv, float f1, float f2, unsigned char* xq, int H, int tk, int i) {
+    const float vv[4] = {xv.x, xv.y, xv.z, xv.w};
+    uint32_t pw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float v = vv[j] * f1 * f2;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float tv = truncf(v);
+            pw[p] |= ((uint32_t)(int)tv & 0xffu) << (8 * j);
+            v = (v - tv) * 128.f;
+        }
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) *reinterpret_cast<uint32_t*>(xq + (size_t)(tk * 4 + p) * H + i) = pw[p];
+}
+// Every token's values, threads tid of nthreads, four values each.
 __device__ __forceinline__ void quantize_x(const void* x, int act_bf16, int n, int H, const float (*s_f)[2],
                                            unsigned char* xq, int tid, int nthreads) {
     for (int q = tid * 4; q < n * H; q += nthreads * 4) {
         const int tk = q / H, i = q - tk * H;
-        const float f1 = s_f[tk][0], f2 = s_f[tk][1];
-        const float4 xv = load_act4(x, (int64_t)tk * H + i, act_bf16);
-        const float vv[4] = {xv.x, xv.y, xv.z, xv.w};
-        uint32_t pw[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float v = vv[j] * f1 * f2;
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const float tv = truncf(v);
-                pw[p] |= ((uint32_t)(int)tv & 0xffu) << (8 * j);
-                v = (v - tv) * 128.f;
-            }
-        }
-#pragma unroll
-        for (int p = 0; p < 4; ++p) *reinterpret_cast<uint32_t*>(xq + (size_t)(tk * 4 + p) * H + i) = pw[p];
+        quantize4(load_act4(x, (int64_t)tk * H + i, act_bf16), s_f[tk][0], s_f[tk][1], xq, H, tk, i);
     }
+}
+
+// Barrier 1 of the threads that run the projection kernel's prologue.
+__device__ __forceinline__ void prologue_sync(int nthreads) {
+    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
 // ---------------------------------------------------------------- gate/up
@@ -654,24 +675,35 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     const int nch_rt = nkt / ck_rt;
     const int kcs = H < 1024 ? H : 1024;              // columns per shared chunk
     const int nch_sh = H / kcs;
-    // down projection: tasks of 16 shared-expert rows, then (entry, 32-row block), numbered after the
-    // gate/up tasks; a task first waits until the gate/up tasks producing its h are done
+    // down projection: tasks (entry, 32-row block) in entry order, then tasks of 16 shared-expert rows,
+    // numbered after the gate/up tasks; a task first waits until the gate/up tasks producing its h are
+    // done (the first entries' h is the first ready; the shared expert's h needs every shared gate/up
+    // task, some of which come last)
     const int dnkt = I / 64, dnsb = I >= 256 ? I / 256 : 1;
     const int dn_sh = !do_dn || ws.probe == 1 ? 0 : (D.has_shared ? H / 16 : 0);
     const int drb = H / 32;
     const int dkcs = I < 512 ? I : 512;   // columns per shared-expert chunk
     const int dnch_sh = I / dkcs;
 
+    __shared__ uint64_t tab_bar;
     pipe_init(P, NS, CW);
+    if (!Q4 && C::kRows && tid == 0) {
+        // the selector table: one bulk copy, waited for at the end of the prologue
+        mbar_init(&tab_bar, 1);
+        fence_barrier_init();
+        mbar_arrive_expect_tx(&tab_bar, 256 * 64 * 4);
+        bulk_load_plain(tsel, W.gtab_rows, 256 * 64 * 4, &tab_bar);
+    }
+    __syncthreads();   // the pipeline's barriers are initialized
+    // ---- prologue, on every warp but the producer's (which starts streaming at once): ptid / kPro
+    // number its threads
+    constexpr int kPro = kThreads - 32;
+    const int ptid = tid < CW * 32 ? tid : tid - 32;
+    if (warp != CW) {
     // ---- grid tables (made when the grid was loaded)
-    if (Q4) {
-    } else if (C::kRows) {
-        for (int i = tid; i < 256 * 64; i += kThreads) {
-            const int r = i >> 6;
-            tsel[i] = __ldg(W.gtab + ((i & 32) ? 256 + (r & 127) : r));
-        }
+    if (Q4 || C::kRows) {
     } else {
-        for (int i = tid; i < 384 * R; i += kThreads) tsel[i] = __ldg(W.gtab + i / R);   // tsgn follows tsel
+        for (int i = ptid; i < 384 * R; i += kPro) tsel[i] = __ldg(W.gtab + i / R);   // tsgn follows tsel
     }
     if (tid < 4) reinterpret_cast<uint4*>(zero)[tid] = make_uint4(0, 0, 0, 0);
     if (tid < kMaxRedBufs) RR.cnt[tid] = RR.task[tid] = RR.freed[tid] = 0;
@@ -688,7 +720,43 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
         float mx[NT];
 #pragma unroll
         for (int q = 0; q < NT; ++q) mx[q] = 0.f;
-        for (int i = tid * 4; do_gu && i < H; i += kThreads * 4) {
+        // one token, H <= 16 kPro: this thread's values stay in registers for the int8 pieces
+        constexpr int kXr = 4;
+        static_assert(kPro % 8 == 0, "32-column blocks of x per eight threads");
+        const bool xreg = C::kSplitX && H <= kXr * 4 * kPro;
+        float4 xr[kXr];
+#pragma unroll
+        for (int j = 0; j < kXr; ++j) xr[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (xreg && do_gu) {
+#pragma unroll
+            for (int j = 0; j < kXr; ++j) {
+                const int i = (ptid + j * kPro) * 4;
+                if (i < H) {
+                    xr[j] = load_act4(x, i, D.act_bf16);
+                    const float4 v = xr[j];
+                    mx[0] = fmaxf(mx[0], fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+                    if (n_sh > 0) {
+                        const uint32_t h0 = bf16_bits(v.x), h1 = bf16_bits(v.y), h2 = bf16_bits(v.z), h3 = bf16_bits(v.w);
+                        const uint32_t l0 = bf16_bits(v.x - __uint_as_float(h0 << 16));
+                        const uint32_t l1 = bf16_bits(v.y - __uint_as_float(h1 << 16));
+                        const uint32_t l2 = bf16_bits(v.z - __uint_as_float(h2 << 16));
+                        const uint32_t l3 = bf16_bits(v.w - __uint_as_float(h3 << 16));
+                        *reinterpret_cast<uint2*>(xbuf + (size_t)i * 2) = make_uint2(h0 | (h1 << 16), h2 | (h3 << 16));
+                        *reinterpret_cast<uint2*>(xbuf + ((size_t)H + i) * 2) = make_uint2(l0 | (l1 << 16), l2 | (l3 << 16));
+                    }
+                }
+                if (Q4) {
+                    // the 32-column sums: eight consecutive threads hold one 32-column block
+                    // (kPro is a multiple of 8)
+                    float sx = i < H ? (xr[j].x + xr[j].y) + (xr[j].z + xr[j].w) : 0.f;
+                    sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+                    sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+                    sx += __shfl_xor_sync(0xffffffffu, sx, 4);
+                    if (i < H && (lane & 7) == 0) xsum[i >> 5] = sx;
+                }
+            }
+        }
+        for (int i = ptid * 4; !xreg && do_gu && i < H; i += kPro * 4) {
 #pragma unroll
             for (int q = 0; q < NT; ++q) {
                 if (q < n) {
@@ -713,13 +781,13 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             for (int m = 16; m >= 1; m >>= 1) mx[q] = fmaxf(mx[q], __shfl_xor_sync(0xffffffffu, mx[q], m));
         }
         if (tid < 8) s_tokmax[tid] = 0.f;
-        __syncthreads();
+        prologue_sync(kPro);
         if (lane == 0) {
 #pragma unroll
             for (int q = 0; q < NT; ++q)
                 if (q < n) atomicMax(reinterpret_cast<int*>(&s_tokmax[q]), __float_as_int(mx[q]));
         }
-        __syncthreads();
+        prologue_sync(kPro);
         if (tid < n) {
             // x 2^(7-e) has |v| < 128 (e: the exponent of the token's largest |x|); the scaling is split in
             // two factors so that neither overflows; piece p weighs 2^(e - 7 - 7p)
@@ -731,10 +799,10 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
 #pragma unroll
             for (int p = 0; p < 4; ++p) s_cs[tid][p] = s_tokmax[tid] > 0.f ? ldexpf(1.f, e - 7 - 7 * p) : 0.f;
         }
-        __syncthreads();
-        if (Q4 && do_gu) {
+        prologue_sync(kPro);
+        if (Q4 && do_gu && !xreg) {
             // sums of x over each 32-column sub-block (the min terms)
-            for (int i = tid; i < n * (H / 32); i += kThreads) {
+            for (int i = ptid; i < n * (H / 32); i += kPro) {
                 const int tk = i / (H / 32), j = i - tk * (H / 32);
                 float sx = 0.f;
 #pragma unroll
@@ -744,14 +812,25 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                 }
                 xsum[i] = sx;
             }
-            if (!C::kSplitX) __syncthreads();
+            if (!C::kSplitX) prologue_sync(kPro);
         }
         if (C::kSplitX && do_gu) {
-            quantize_x(x, D.act_bf16, n, H, s_f, xq, tid, kThreads);
-            __syncthreads();
+            if (xreg) {
+#pragma unroll
+                for (int j = 0; j < kXr; ++j) {
+                    const int i = (ptid + j * kPro) * 4;
+                    if (i < H) quantize4(xr[j], s_f[0][0], s_f[0][1], xq, H, 0, i);
+                }
+            } else {
+                quantize_x(x, D.act_bf16, n, H, s_f, xq, ptid, kPro);
+            }
+            prologue_sync(kPro);
         }
     }
-    const bool refused = s_refused != 0;
+    if (!Q4 && C::kRows && !mbar_wait(&tab_bar, 0, ws.err)) set_abort(P);
+    }
+    // the producer reads the grid's verdict itself (the prologue's copy is not yet written)
+    const bool refused = warp == CW ? (!Q4 && __ldg(W.gtab + 386) != 0) : s_refused != 0;
 
     if (warp == CW) {
         // ------------------------------------------------ producer warp
@@ -766,6 +845,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
         const int lead = !C::kSplitX ? n_sh : (n_sh < (int)gridDim.x ? n_sh : (int)gridDim.x);
         int nxt = 0, nxt2 = 0;
         int d_total = 0;
+        uint32_t dknown = 0;   // gate/up completion counters seen complete (wait_deps_warp)
         auto route = [&]() {
             build_routing_warp(Rt, ws.ids, n, k, TPB, ws.probe == 1 ? 1 : (ws.probe == 2 ? 2 : 0), ws.probe_e);
             routed = true;
@@ -793,19 +873,22 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                 // down-projection task pos - total
                 const int dt = pos - total;
                 if (dt >= d_total) break;
-            const bool dsh = dt < dn_sh;
+            const int nd_rt = do_dn ? Rt.nu * drb : 0;
+            const bool dsh = dt >= nd_rt;
+            const int dts = dt - nd_rt;   // shared-expert down task
             int u = 0, rb = 0, ns = 0, ck = 0;
             if (!dsh) {
-                u = (dt - dn_sh) / drb;
-                rb = (dt - dn_sh) % drb;
+                u = dt / drb;
+                rb = dt % drb;
                 ns = Rt.ustart[u + 1] - Rt.ustart[u];
                 ck = down_chunk_ksteps(dnkt, dnsb, ns, Q4 ? 1152 : 640);
             }
             const int nch = dsh ? dnch_sh : dnkt / ck;
-            if (!ws.probe) {
-                const bool ok = dsh ? wait_count(ws.gu_done, (uint32_t)(I / 8), ws.err)
-                                   : wait_count(ws.gu_done + 1 + u, (uint32_t)(I / 32), ws.err);
-                if (!ok) { set_abort(P); break; }
+            if (!ws.probe &&
+                !wait_deps_warp(ws.gu_done, dsh ? 0 : 1 + u, 1 + Rt.nu, (uint32_t)(I / 8), (uint32_t)(I / 32), dknown,
+                                ws.err)) {
+                set_abort(P);
+                break;
             }
             for (int c = 0; c < nch; ++c) {
                 const int s = it % NS;
@@ -822,7 +905,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                         mbar_arrive_expect_tx(&P.full[s], 2 * abytes + n * hbytes);
 #pragma unroll
                         for (int q = 0; q < 2; ++q)
-                            bulk_load(st + q * abytes, W.sh_down + ((size_t)(dt * 2 + q) * (I / 8) + kc0 / 8) * 64,
+                            bulk_load(st + q * abytes, W.sh_down + ((size_t)(dts * 2 + q) * (I / 8) + kc0 / 8) * 64,
                                       abytes, &P.full[s], pol);
                         for (int q = 0; q < n; ++q)
                             bulk_load_plain(st + 2 * abytes + q * hbytes, ws.hb_sh + ((size_t)q * (I / 64) + kc0 / 64) * 128,
@@ -944,7 +1027,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             if (inf.task >= T_gu) {
                 // ---- down projection
             const int dt = inf.task - T_gu;
-            const bool dsh = dt < dn_sh;
+            const bool dsh = dt >= (do_dn ? Rt.nu * drb : 0);
             if (dsh) {
                 if (inf.chunk == 0) {
 #pragma unroll
@@ -971,7 +1054,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                     }
                 }
             } else {
-                const int tt = dt - dn_sh, u = tt / drb;
+                const int tt = dt, u = tt / drb;
                 const int s0 = Rt.ustart[u], ns = Rt.ustart[u + 1] - s0;
                 if (inf.chunk == 0) {
                     dtcount = ns;
@@ -1348,15 +1431,16 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             if (task >= T_gu) {
                 // ---- down projection: y of the task's rows
                 const int dt = task - T_gu;
-            if (dt < dn_sh) {
+            const int nd_rt = do_dn ? Rt.nu * drb : 0;
+            if (dt >= nd_rt) {
                 for (int q = lane; q < 16 * n; q += 32) {   // (token, row) pairs
                     const int tok = q >> 4, row = q & 15;
                     float y = 0.f;
                     for (int w = 0; w < CW; ++w) y += rbuf[w * C::kRedPer + tok * 16 + row];
-                    (ws.probe ? ws.probe_out : ws.y_sh)[(size_t)tok * H + 16 * dt + row] = y;
+                    (ws.probe ? ws.probe_out : ws.y_sh)[(size_t)tok * H + 16 * (dt - nd_rt) + row] = y;
                 }
             } else {
-                const int tt = dt - dn_sh, u = tt / drb, rb = tt % drb;
+                const int tt = dt, u = tt / drb, rb = tt % drb;
                 const int s0 = Rt.ustart[u], ns = Rt.ustart[u + 1] - s0;
                 for (int q = 0; q < ns; ++q) {
                     float y = 0.f;
@@ -1521,8 +1605,9 @@ __global__ void __launch_bounds__(kSteerThreads) k_combine_steer_decode(Dims D, 
 // nibble (element 7 negative for odd popcount), gtab[384..387] the magnitudes
 // as int8 bytes, their negatives, whether the grid is refused (more than four
 // distinct values, or a value above 127) and the number of distinct values.
-__global__ void __launch_bounds__(256) k_grid_tables(const uint8_t* grid, uint32_t* gtab) {
+__global__ void __launch_bounds__(256) k_grid_tables(const uint8_t* grid, uint32_t* gtab, uint32_t* rows) {
     __shared__ int cls[256];
+    __shared__ uint32_t words[384];
     const int tid = threadIdx.x;
     cls[tid] = 0;
     __syncthreads();
@@ -1551,15 +1636,23 @@ __global__ void __launch_bounds__(256) k_grid_tables(const uint8_t* grid, uint32
     uint32_t w = 0;
     for (int i = 0; i < 8; ++i) w |= (uint32_t)(cls[grid[tid * 8 + i]] - 1) << (4 * i);
     gtab[tid] = w;
+    words[tid] = w;
     if (tid < 128) {
         uint32_t sgw = ((uint32_t)__popc(tid) & 1u) << 30;
         for (int i = 0; i < 7; ++i) sgw |= ((uint32_t)(tid >> i) & 1u) << (4 * i + 2);
         gtab[256 + tid] = sgw;
+        words[256 + tid] = sgw;
+    }
+    __syncthreads();
+    // rows form: one copy of the row's class word per lane, then one of its sign word
+    for (int i = tid; i < 256 * 64; i += 256) {
+        const int r = i >> 6;
+        rows[i] = words[(i & 32) ? 256 + (r & 127) : r];
     }
 }
 
-cudaError_t launch_grid_tables(const uint8_t* grid, uint32_t* gtab, cudaStream_t st) {
-    k_grid_tables<<<1, 256, 0, st>>>(grid, gtab);
+cudaError_t launch_grid_tables(const uint8_t* grid, uint32_t* gtab, uint32_t* rows, cudaStream_t st) {
+    k_grid_tables<<<1, 256, 0, st>>>(grid, gtab, rows);
     return cudaGetLastError();
 }
 

@@ -39,7 +39,7 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
 cudaError_t launch_route_prefill(const Weights& W, const Dims& D, const PrefillWs& ws, const void* x, int n,
                                  cudaStream_t st);
 cudaError_t launch_wait_selftest(uint32_t* err, cudaStream_t st);
-cudaError_t launch_grid_tables(const uint8_t* grid, uint32_t* gtab, cudaStream_t st);
+cudaError_t launch_grid_tables(const uint8_t* grid, uint32_t* gtab, uint32_t* rows, cudaStream_t st);
 cudaError_t launch_permutation(const Dims& D, const PrefillWs& ws, const int32_t* ids, int n, cudaStream_t st);
 cudaError_t launch_probe_decode(const Weights& W, const Dims& D, const DecodeWs& ws, int which, const void* in, int n,
                                 int n_sm, cudaStream_t st);
@@ -107,7 +107,7 @@ struct ds4moe {
     int decode_max;
     int n_sm;
     // weight buffer layout
-    size_t off_grid, off_gtab, off_Wr, off_Wr2, off_br, off_steer, off_gate_qs, off_gate_d, off_up_qs, off_up_d, off_down_q, off_down_sc,
+    size_t off_grid, off_gtab, off_gtab_rows, off_Wr, off_Wr2, off_br, off_steer, off_gate_qs, off_gate_d, off_up_qs, off_up_d, off_down_q, off_down_sc,
         off_down_dd, off_sh_gate, off_sh_up, off_sh_down, weight_bytes;
     size_t iq2_qs_stride, iq2_d_stride, q2_q_stride, q2_sc_stride, q2_dd_stride;
     // 4-bit layers: codes at off_gate_qs / off_up_qs / off_down_q, scale and (d, dmin) words here
@@ -200,6 +200,7 @@ struct ds4moe {
         const uint8_t* b = weights;
         W.grid_u8 = b + off_grid;
         W.gtab = reinterpret_cast<const uint32_t*>(b + off_gtab);
+        W.gtab_rows = reinterpret_cast<const uint32_t*>(b + off_gtab_rows);
         W.W_r = reinterpret_cast<const float*>(b + off_Wr);
         W.W_r2 = shape.max_tokens > decode_max ? reinterpret_cast<const float*>(b + off_Wr2) : nullptr;
         W.b_r = shape.has_bias ? reinterpret_cast<const float*>(b + off_br) : nullptr;
@@ -356,6 +357,7 @@ ds4moe_status ds4moe_create(const ds4moe_shape* s, ds4moe_t** out) {
     size_t o = 0;
     h->off_grid = o; o += align256(256 * 8);
     h->off_gtab = o; o += align256((256 + 128 + 4) * 4);
+    h->off_gtab_rows = o; o += align256(256 * 64 * 4);
     h->off_Wr = o; o += align256(E * H * 4);
     h->off_Wr2 = o; o += align256(s->max_tokens > h->decode_max ? (E + 1) / 2 * 2 * H * 4 : 0);
     h->off_br = o; o += align256(E * 4);
@@ -473,6 +475,7 @@ ds4moe_status ds4moe_set_grid(ds4moe_t* h, const uint8_t* d_grid, void* stream) 
                                      (cudaStream_t)stream);
     if (ce == cudaSuccess)
         ce = launch_grid_tables(h->weights + h->off_grid, reinterpret_cast<uint32_t*>(h->weights + h->off_gtab),
+                                reinterpret_cast<uint32_t*>(h->weights + h->off_gtab_rows),
                                 (cudaStream_t)stream);
     if (ce != cudaSuccess) return cuda_fail(ce, "set_grid copy");
     h->grid_set = true;

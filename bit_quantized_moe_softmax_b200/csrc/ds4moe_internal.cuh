@@ -85,6 +85,9 @@ struct Weights {
                                 // row (nibble i = class of element i), [128] sign nibbles of each 7-bit sign
                                 // field (bit 2 of nibble i; element 7 from the parity), then the four
                                 // magnitudes as int8, their negatives, refused (0/1), distinct values
+    const uint32_t* gtab_rows;  // the decode kernel's shared-memory selector table for one or two tokens
+                                // ([256][64] words: row r holds class word r in lanes 0..31 and sign word
+                                // r & 127 in lanes 32..63), made by set_grid, copied in with one bulk copy
     const float* W_r;           // [E][H]
     const float* W_r2;          // [ceil(E/2)][H][2]: expert pairs interleaved per column (prefill plan), or nullptr
     const float* b_r;           // [E] or nullptr
