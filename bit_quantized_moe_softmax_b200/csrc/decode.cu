@@ -543,10 +543,13 @@ __device__ __forceinline__ void prologue_sync(int nthreads) {
 }
 
 // ---------------------------------------------------------------- gate/up
-template <int NT>
+template <int NT, bool Q4 = false>
 struct GateUpCfg {
     static constexpr int CW = 8;                                  // consumer warps
-    static constexpr int NS = NT <= 4 ? 3 : 2;                    // stages
+    // stages: 4-bit layers have no selector table, and one or two tokens take four stages of 37 KB
+    // (16 k steps of gate and up codes with their scales) to keep more bytes in flight
+    static constexpr int NS = NT <= 2 && Q4 ? 4 : NT <= 4 ? 3 : 2;
+    static constexpr int kStage = Q4 && NT <= 4 ? 37888 : kStageBytes;
     // selector tables: ROWS form (one or two tokens): 256 rows of 256 B, bytes 0..127 of row r the
     // class selectors of grid row r, bytes 128..255 the sign selectors of S byte r (signs r & 127),
     // 32 copies each (one per lane), so that one byte-permute of a payload word and the lane's offset
@@ -618,13 +621,14 @@ struct GateUpAcc {
 // ---------------------------------------------------------------- down projection pieces
 // k steps (64 columns) per routed down chunk for an entry of ns slots: codes,
 // scales (step_bytes per step: 640 for Q2, 1152 for Q4), (d, dmin) and the
-// slots' h pieces (and per-16 sums) for those columns must fit one stage.
-__device__ __forceinline__ int down_chunk_ksteps(int nkt, int nsb, int ns, int step_bytes) {
+// slots' h pieces (and per-16 sums) for those columns must fit one stage of
+// stage_bytes.
+__device__ __forceinline__ int down_chunk_ksteps(int nkt, int nsb, int ns, int step_bytes, int stage_bytes) {
     // the largest of 32, 16, 8, 4 that divides the k steps (I / 64: a multiple of 4 for I >= 256)
     int ck = nkt % 32 == 0 ? 32 : nkt % 16 == 0 ? 16 : nkt % 8 == 0 ? 8 : nkt % 4 == 0 ? 4 : nkt;
     for (; ck > 1 && ck % 2 == 0; ck >>= 1) {
         const int nsbc = nsb > 1 ? (ck + 3) / 4 : 1;
-        if (ck * step_bytes + nsbc * 128 + ns * ck * 272 <= kStageBytes) break;
+        if (ck * step_bytes + nsbc * 128 + ns * ck * 272 <= stage_bytes) break;
     }
     return ck;
 }
@@ -642,14 +646,15 @@ struct DownAcc {
 template <int NT, bool Q4>
 __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     k_moe_decode(Weights W, Dims D, DecodeWs ws, const void* x, int n) {
-    using C = GateUpCfg<NT>;
+    using C = GateUpCfg<NT, Q4>;
     constexpr int NS = C::NS, CW = C::CW, R = C::R, TPB = C::TPB, kThreads = C::kThreads;
     constexpr int kTab = Q4 ? 0 : C::kTabWords;
+    constexpr int kStage = C::kStage;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     uint32_t* tsel = reinterpret_cast<uint32_t*>(smem_raw);                      // rows [256][64] or [256][R]
     uint32_t* tsgn = tsel + 256 * R;                                             // [128][R] (interleaved form)
-    unsigned char* stages = smem_raw + 4 * kTab;                                 // NS x kStageBytes
-    float* red = reinterpret_cast<float*>(stages + NS * kStageBytes);            // kRedFloats
+    unsigned char* stages = smem_raw + 4 * kTab;                                 // NS x kStage
+    float* red = reinterpret_cast<float*>(stages + NS * kStage);                 // kRedFloats
     unsigned char* xbuf = reinterpret_cast<unsigned char*>(red + C::kRedFloats);  // n x H x 4 bytes: bf16 pieces
     unsigned char* xq = C::kSplitX ? xbuf + (size_t)n * D.H * 4 : xbuf;          // int8 pieces
     unsigned char* zero = xq + (size_t)n * D.H * 4;                              // 64 bytes of zeros
@@ -670,8 +675,11 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     const bool do_gu = (ws.stages & 1) != 0, do_dn = (ws.stages & 2) != 0;
     const int n_sh = !do_gu || ws.probe == 1 ? 0 : (D.has_shared ? I / 8 : 0);   // shared tasks: 8 rows of gate and up
     const int rb_per_e = I / 32;
-    // k steps (64 columns) per routed chunk: the largest of 32, 16, 8, 4 that divides H / 64 (Q4: of 8, 4)
-    const int ck_rt = (!Q4 && nkt % 32 == 0) ? 32 : (!Q4 && nkt % 16 == 0) ? 16 : nkt % 8 == 0 ? 8 : 4;
+    // k steps (64 columns) per routed chunk: the largest of 32, 16, 8, 4 that divides H / 64 and fits a
+    // stage (Q4: 16 with the 37 KB stage, else 8)
+    const int ck_rt = (!Q4 && nkt % 32 == 0) ? 32
+                      : ((!Q4 || kStage >= 37888) && nkt % 16 == 0) ? 16
+                      : nkt % 8 == 0 ? 8 : 4;
     const int nch_rt = nkt / ck_rt;
     const int kcs = H < 1024 ? H : 1024;              // columns per shared chunk
     const int nch_sh = H / kcs;
@@ -881,7 +889,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                 u = dt / drb;
                 rb = dt % drb;
                 ns = Rt.ustart[u + 1] - Rt.ustart[u];
-                ck = down_chunk_ksteps(dnkt, dnsb, ns, Q4 ? 1152 : 640);
+                ck = down_chunk_ksteps(dnkt, dnsb, ns, Q4 ? 1152 : 640, kStage);
             }
             const int nch = dsh ? dnch_sh : dnkt / ck;
             if (!ws.probe &&
@@ -895,7 +903,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                 const uint32_t ph = (it / NS) & 1;
                 if (!mbar_wait(&P.empty[s], ph ^ 1, ws.err)) { set_abort(P); break; }
                 if (lane == 0) {
-                    unsigned char* st = stages + s * kStageBytes;
+                    unsigned char* st = stages + s * kStage;
                     if (dsh) {
                         // 16 rows of the shared down matrix (two 8-row groups of core-matrix tiles),
                         // columns c*dkcs .. +dkcs, then every token's h pieces for those columns
@@ -949,7 +957,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                 const uint32_t ph = (it / NS) & 1;
                 if (!mbar_wait(&P.empty[s], ph ^ 1, ws.err)) { set_abort(P); break; }
                 if (lane == 0) {
-                    unsigned char* st = stages + s * kStageBytes;
+                    unsigned char* st = stages + s * kStage;
                     if (sh) {
                         // one 8-row group of the gate and of the up matrix (core-matrix tiles), columns
                         // c*kcs .. +kcs
@@ -1022,7 +1030,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             if (!mbar_wait(&P.full[s], (it / NS) & 1, ws.err)) { set_abort(P); break; }
             const ChunkInfo inf = P.info[s];
             if (inf.task < 0 || aborted(P)) break;
-            const unsigned char* st = stages + s * kStageBytes;
+            const unsigned char* st = stages + s * kStage;
             const int T_gu = inf.task < n_sh ? n_sh : n_sh + (do_gu ? Rt.nu * rb_per_e : 0);
             if (inf.task >= T_gu) {
                 // ---- down projection
@@ -1676,11 +1684,15 @@ cudaError_t launch_wait_selftest(uint32_t* err, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------- launchers
+template <int NT, bool Q4>
+size_t gateup_smem_bytes_t(const Dims& D, int n) {
+    using C = GateUpCfg<NT, Q4>;
+    return (size_t)C::NS * C::kStage + 4 * ((size_t)(Q4 ? 0 : C::kTabWords) + C::kRedFloats) +
+           (size_t)(C::kSplitX ? 2 : 1) * n * D.H * 4 + 64 + (Q4 ? (size_t)n * (D.H / 32) * 4 : 0);
+}
 template <int NT>
 size_t gateup_smem_bytes(const Dims& D, int n) {
-    using C = GateUpCfg<NT>;
-    return (size_t)C::NS * kStageBytes + 4 * ((size_t)(D.q4 ? 0 : C::kTabWords) + C::kRedFloats) +
-           (size_t)(C::kSplitX ? 2 : 1) * n * D.H * 4 + 64 + (D.q4 ? (size_t)n * (D.H / 32) * 4 : 0);
+    return D.q4 ? gateup_smem_bytes_t<NT, true>(D, n) : gateup_smem_bytes_t<NT, false>(D, n);
 }
 
 size_t router_smem_bytes(const Dims& D, int n) {
