@@ -282,8 +282,13 @@ def run_ours(args, wl, rank, local, world):
     names = [m.ds4moe_plan_kernel(layers[0].h, n, i) for i in range(nl)]
 
     cbufs = [torch.empty(n, H, dtype=torch.float32, device=dev) for _ in range(C)] if chain else []
+    cwork = torch.empty(2, n, H, dtype=torch.float32, device=dev) if chain else None
+    handles = [lay.h for lay in layers]
 
     def step(i, events=None):
+        if chain and events is None:   # the whole chain in one call (layers as programmatic dependents)
+            m.ds4moe_forward_chain(handles, xs[i % P], cbufs[-1], cwork, stream)
+            return
         if chain:   # every layer of the chain, the residual added by each layer's combine kernel
             cur = xs[i % P]
             for l in range(C):
@@ -457,7 +462,7 @@ def _timed_run(args, wl, rank, local, world, dev, layers, xs, outs, stream, nl, 
     e2e_s = D.max_over_ranks(t1 - t0, dev)
     e2e = {"value": n * K2 * world / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": n * H * xh.element_size(),
            "d2h_bytes_per_step": n * H * 4, "steps": K2,
-           "api": ("torch copies around the chained ds4moe_forward_residual calls, synchronized per step" if chain
+           "api": ("torch copies around one ds4moe_forward_chain call, synchronized per step" if chain
                    else "ds4moe_forward_host_async per step (two staging slots per layer), ds4moe_host_sync at the end")}
 
     # roofline of the dominant kernel
@@ -621,7 +626,7 @@ def run_reference(args, wl, rank, world):
             "e2e": {"value": round(rate, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-SUB_WORKLOADS = ("decode_q4", "prefill512", "prefill11709")
+SUB_WORKLOADS = ("decode_q4", "mtp8", "prefill512", "prefill11709")
 
 
 def sub_record(line: dict) -> dict:
@@ -641,7 +646,7 @@ def main():
     ap.add_argument("--instances", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
-                    help="with the default decode workload: skip the sub-records (4-bit decode, prefill)")
+                    help="with the default decode workload: skip the sub-records (4-bit decode, chain, prefill)")
     ap.add_argument("--steer", type=float, default=0.0,
                     help="directional steering strength F of every layer (unit direction, seeded); 0: off")
     args = ap.parse_args()
@@ -665,8 +670,8 @@ def main():
     line = run_ours(args, wl, rank, local, world)
     if baseline:
         line["cpu_baseline"] = cpu_baseline_record(wl, n_tokens=4 * cores, budget_s=15.0, device=dev)
-    # the metric covers decode and prefill: the default run adds the 4-bit decode step and both prefill
-    # workloads as sub-records
+    # the metric covers decode and prefill: the default run adds the 4-bit decode step, the chained
+    # verify step and both prefill workloads as sub-records
     if args.workload == "decode" and not args.no_prefill:
         subs = {}
         for name in SUB_WORKLOADS:

@@ -34,7 +34,7 @@ EXPORTS = ("ds4moe_create", "ds4moe_destroy", "ds4moe_weight_bytes", "ds4moe_wor
            "ds4moe_forward_profiled", "ds4moe_route_noalloc", "ds4moe_forward_residual",
            "ds4moe_forward_residual_profiled", "ds4moe_set_steering", "ds4moe_forward_host_async",
            "ds4moe_host_sync", "ds4moe_probe", "ds4moe_selftest_wait",
-           "ds4moe_permutation", "ds4moe_pack_q4k")
+           "ds4moe_permutation", "ds4moe_pack_q4k", "ds4moe_forward_chain")
 
 
 class ds4moe_shape(ctypes.Structure):
@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
             "ds4moe_forward_profiled": ([vp, vp, i32, vp, ctypes.POINTER(vp), vp], i32),
             "ds4moe_route_noalloc": ([vp, vp, i32, vp, vp, vp], i32),
             "ds4moe_forward_residual": ([vp, vp, i32, vp, vp], i32),
+            "ds4moe_forward_chain": ([ctypes.POINTER(vp), i32, vp, i32, vp, vp, vp], i32),
             "ds4moe_set_steering": ([vp, vp, ctypes.c_float, vp], i32),
             "ds4moe_forward_residual_profiled": ([vp, vp, i32, vp, ctypes.POINTER(vp), vp], i32),
         }
@@ -181,6 +182,12 @@ def ds4moe_forward(h: int, x: torch.Tensor, out: torch.Tensor, stream=None):
 def ds4moe_set_steering(h: int, v: torch.Tensor | None, F: float, stream=None):
     _ok(lib().ds4moe_set_steering(h, None if v is None else _ptr(v), ctypes.c_float(F), _stream(stream)),
         "ds4moe_set_steering")
+
+
+def ds4moe_forward_chain(handles, x: torch.Tensor, out: torch.Tensor, work: torch.Tensor, stream=None):
+    arr = (ctypes.c_void_p * len(handles))(*handles)
+    _ok(lib().ds4moe_forward_chain(arr, len(handles), _ptr(x), x.shape[0], _ptr(out), _ptr(work), _stream(stream)),
+        "ds4moe_forward_chain")
 
 
 def ds4moe_forward_residual(h: int, x: torch.Tensor, out: torch.Tensor, stream=None):

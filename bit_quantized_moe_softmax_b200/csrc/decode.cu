@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(RouterCfg<NT>::kWarps * 32)
         fence_barrier_init();
         mbar_arrive_expect_tx(&bar, wbytes + xbytes);
         bulk_load_plain(r_smem, W.W_r + (size_t)e0 * H, wbytes, &bar);
+        griddep_wait();   // chained layers: x is the previous layer's output (no-op otherwise)
         bulk_load_plain(r_smem + (size_t)kRE * H * 4, x, xbytes, &bar);
     }
     __syncthreads();
@@ -219,6 +220,23 @@ __device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t* err) {
         uint32_t v;
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
         if (v) return true;
+        if (t0 == 0) {
+            t0 = global_ns();
+        } else if (global_ns() - t0 > kWaitNs) {
+            set_err(err, kErrTimeout);
+            return false;
+        }
+        __nanosleep(64);
+    }
+}
+
+// Waits (bounded) until *counter >= target, reading it with acquire semantics.
+__device__ __forceinline__ bool wait_ge(const uint32_t* counter, uint32_t target, uint32_t* err) {
+    uint64_t t0 = 0;
+    for (;;) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+        if (v >= target) return true;
         if (t0 == 0) {
             t0 = global_ns();
         } else if (global_ns() - t0 > kWaitNs) {
@@ -708,6 +726,11 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     constexpr int kPro = kThreads - 32;
     const int ptid = tid < CW * 32 ? tid : tid - 32;
     if (warp != CW) {
+    if (ws.chain_wait) {
+        // chained layers: x is the previous layer's output, complete once its combine CTAs have counted
+        if (tid == 0 && !wait_ge(ws.chain_wait, ws.chain_target, ws.err)) set_abort(P);
+        prologue_sync(kPro);
+    }
     // ---- grid tables (made when the grid was loaded)
     if (Q4 || C::kRows) {
     } else {
@@ -1541,18 +1564,27 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     __syncthreads();
     if (s_last && !ws.probe) {
         for (int i = tid; i < 1 + kMaxSlots; i += blockDim.x) ws.gu_done[i] = 0;
+        if (tid == 0 && ws.chain_wait) *ws.chain_wait = 0;
     }
 }
 
 // ---------------------------------------------------------------- combine
 // out[t][r] = y_shared[t][r] + sum_j w[t][j] y[t*k + j][r], j in rank order
 // (then x[t][r] + that, when the call asks for the residual).
-__global__ void __launch_bounds__(256) k_combine_decode(Dims D, DecodeWs ws, float* out, int n) {
-    griddep_wait();   // y of the projection grid
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+// Chained layers: once every thread of the CTA has written its part of out,
+// one thread publishes it (fence, then count) to the next layer.
+__device__ __forceinline__ void chain_count(uint32_t* chain_done) {
+    if (!chain_done) return;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(chain_done, 1u);
+    }
+}
+
+// out[i] (token t = i / H, row r = i % H).
+__device__ __forceinline__ void combine_one(const Dims& D, const DecodeWs& ws, float* out, int64_t i) {
     const int H = D.H, k = D.k;
-    if (i >= (int64_t)n * H) return;
-    if (__ldcg(ws.grid_refused)) return;   // the projection grid refused the grid: out stays as it was
     const int t = (int)(i / H), r = (int)(i % H);
     float w[16], y[16];
 #pragma unroll
@@ -1569,6 +1601,15 @@ __global__ void __launch_bounds__(256) k_combine_decode(Dims D, DecodeWs ws, flo
     out[i] = ws.xres ? act_at(ws.xres, i, D.act_bf16) + acc : acc;
 }
 
+__global__ void __launch_bounds__(256) k_combine_decode(Dims D, DecodeWs ws, float* out, int n) {
+    griddep_launch();   // chained layers: the next layer's router may load its rows now
+    griddep_wait();     // y of the projection grid
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    // the projection grid refused the grid: out stays as it was
+    if (i < (int64_t)n * D.H && !__ldcg(ws.grid_refused)) combine_one(D, ws, out, i);
+    chain_count(ws.chain_done);
+}
+
 // The combine with directional steering of the layer output: one CTA per
 // token; y = y_shared + sum_j w_j y_j as above, then y - F v (v . y) with
 // v . y summed in a fixed order (per thread over its columns, then the CTA),
@@ -1576,11 +1617,10 @@ __global__ void __launch_bounds__(256) k_combine_decode(Dims D, DecodeWs ws, flo
 constexpr int kSteerThreads = 1024;   // few tokens: one wide CTA per token
 constexpr int kSteerCols = 4;          // columns per thread (H <= 4096)
 
-__global__ void __launch_bounds__(kSteerThreads) k_combine_steer_decode(Dims D, DecodeWs ws, float* out, int n) {
-    griddep_wait();   // y of the projection grid
+// One token (the CTA's) of the steered combine.
+__device__ __forceinline__ void steer_one(const Dims& D, const DecodeWs& ws, float* out) {
     __shared__ float red[kSteerThreads / 32];
     const int t = blockIdx.x, H = D.H, k = D.k;
-    if (__ldcg(ws.grid_refused)) return;   // the projection grid refused the grid: out stays as it was
     float acc[kSteerCols];
     float dot = 0.f;
 #pragma unroll
@@ -1603,6 +1643,14 @@ __global__ void __launch_bounds__(kSteerThreads) k_combine_steer_decode(Dims D, 
             out[(int64_t)t * H + r] = ws.xres ? act_at(ws.xres, (int64_t)t * H + r, D.act_bf16) + y : y;
         }
     }
+}
+
+__global__ void __launch_bounds__(kSteerThreads) k_combine_steer_decode(Dims D, DecodeWs ws, float* out, int n) {
+    griddep_launch();   // chained layers: the next layer's router may load its rows now
+    griddep_wait();     // y of the projection grid
+    // the projection grid refused the grid: out stays as it was (a CTA-uniform test)
+    if (!__ldcg(ws.grid_refused)) steer_one(D, ws, out);
+    chain_count(ws.chain_done);
 }
 
 // ---------------------------------------------------------------- grid tables
@@ -1774,9 +1822,11 @@ cudaError_t launch_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws,
     const bool pdl = ev == nullptr;   // profiled runs keep the kernels apart
     const int rgrid = (D.E + kRE - 1) / kRE;
     mk.before();
-    k_router_decode<NT><<<rgrid, RouterCfg<NT>::kWarps * 32, router_smem_bytes(D, n), st>>>(W, D, ws, x, n,
-                                                                                             ws.route_ready);
+    // chained layers: a programmatic dependent of the previous layer's combine (it loads its rows, then waits)
+    err = launch_pdl(k_router_decode<NT>, dim3(rgrid), dim3(RouterCfg<NT>::kWarps * 32), router_smem_bytes(D, n), st,
+                     pdl && ws.chain_wait != nullptr, W, D, ws, x, n, ws.route_ready);
     mk.after();
+    if (err != cudaSuccess) return err;
     mk.before();
     err = launch_pdl(k_moe_decode<NT, Q4>, dim3(n_sm), dim3(GateUpCfg<NT>::kThreads), s1, st, pdl, W, D, ws, x, n);
     mk.after();
@@ -1793,6 +1843,10 @@ cudaError_t launch_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws,
 }
 
 int decode_launches() { return 3; }
+// CTAs of the decode plan's combine launch for n tokens (what a chained layer counts).
+unsigned decode_combine_ctas(const Dims& D, int n, bool steer) {
+    return steer ? (unsigned)n : (unsigned)(((int64_t)n * D.H + 255) / 256);
+}
 const char* decode_kernel_name(int i) { return (i >= 0 && i < 3) ? kDecodeKernels[i] : nullptr; }
 
 // Dynamic shared memory of the larger decode kernel for n tokens, plus its

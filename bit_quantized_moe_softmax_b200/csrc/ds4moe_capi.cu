@@ -39,6 +39,7 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
 cudaError_t launch_route_prefill(const Weights& W, const Dims& D, const PrefillWs& ws, const void* x, int n,
                                  cudaStream_t st);
 cudaError_t launch_wait_selftest(uint32_t* err, cudaStream_t st);
+unsigned decode_combine_ctas(const Dims& D, int n, bool steer);
 cudaError_t launch_grid_tables(const uint8_t* grid, uint32_t* gtab, uint32_t* rows, cudaStream_t st);
 cudaError_t launch_permutation(const Dims& D, const PrefillWs& ws, const int32_t* ids, int n, cudaStream_t st);
 cudaError_t launch_probe_decode(const Weights& W, const Dims& D, const DecodeWs& ws, int which, const void* in, int n,
@@ -242,7 +243,7 @@ struct ds4moe {
         w.done = hdr + 4;
         w.grid_refused = hdr + 6;
         w.route_ready = hdr + 7;
-        w.gu_done = hdr + 16;
+        w.gu_done = hdr + 16;   // word 10: this layer's count of combine CTAs in a chained forward
         w.stages = 3;
         w.logits = reinterpret_cast<float*>(ws + L.logits);
         w.ids = reinterpret_cast<int32_t*>(ws + L.ids);
@@ -636,6 +637,53 @@ ds4moe_status ds4moe_forward_residual_profiled(ds4moe_t* h, const void* d_x, int
                                                void* const* events, void* stream) {
     if (!events) return fail(DS4MOE_ERR_ARG, "forward_residual_profiled: NULL events");
     return forward_impl(h, d_x, n, d_out, events, stream, "forward_residual_profiled", true);
+}
+
+ds4moe_status ds4moe_forward_chain(ds4moe_t* const* layers, int32_t L, const void* d_x, int32_t n, float* d_out,
+                                   float* d_work, void* stream) {
+    if (!layers || L < 1) return fail(DS4MOE_ERR_ARG, "forward_chain: no layers");
+    if (n == 0) return DS4MOE_OK;
+    if (!d_x || !d_out || !d_work) return fail(DS4MOE_ERR_ARG, "forward_chain: NULL buffer");
+    if (!aligned16(d_x) || !aligned16(d_out) || !aligned16(d_work))
+        return fail(DS4MOE_ERR_ALIGN, "forward_chain: x, out and work must be 16-byte aligned");
+    for (int l = 0; l < L; ++l) {
+        ds4moe_t* h = layers[l];
+        ds4moe_status s = check_forward(h, d_x, n, d_out, "forward_chain");
+        if (s != DS4MOE_OK) return s;
+        if (n > h->decode_max) return fail(DS4MOE_ERR_ARG, "forward_chain: n_tokens %d above layer %d's decode_max %d", n, l,
+                                           h->decode_max);
+        if (h->D.H != layers[0]->D.H) return fail(DS4MOE_ERR_SHAPE, "forward_chain: layer %d hidden differs", l);
+        if (l > 0 && h->D.act_bf16) return fail(DS4MOE_ERR_SHAPE, "forward_chain: layer %d takes bf16 x", l);
+        for (int j = 0; j < l; ++j)
+            if (layers[j] == h) return fail(DS4MOE_ERR_ARG, "forward_chain: layer %d repeats layer %d's handle", l, j);
+    }
+    const size_t H = layers[0]->D.H;
+    const size_t xb = (size_t)n * H * (layers[0]->D.act_bf16 ? 2 : 4), ob = (size_t)n * H * 4;
+    auto overlap = [](const void* a, size_t na, const void* b, size_t nb) {
+        const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+        return x < y + nb && y < x + na;
+    };
+    if (overlap(d_work, 2 * ob, d_x, xb) || overlap(d_work, 2 * ob, d_out, ob) || overlap(d_x, xb, d_out, ob))
+        return fail(DS4MOE_ERR_ARG, "forward_chain: x, out and work overlap");
+    cudaStream_t st = (cudaStream_t)stream;
+    for (int l = 0; l < L; ++l) {
+        ds4moe_t* h = layers[l];
+        const void* in = l == 0 ? d_x : d_work + (size_t)((l - 1) % 2) * n * H;
+        float* o = l == L - 1 ? d_out : d_work + (size_t)(l % 2) * n * H;
+        DecodeWs ws = h->decode_ws();
+        ws.xres = in;
+        ws.steer_v = h->steer_on ? reinterpret_cast<const float*>(h->weights + h->off_steer) : nullptr;
+        ws.steer_F = h->steer_F;
+        if (l < L - 1) ws.chain_done = reinterpret_cast<uint32_t*>(h->ws + h->L.hdr) + 10;
+        if (l > 0) {
+            ds4moe_t* p = layers[l - 1];
+            ws.chain_wait = reinterpret_cast<uint32_t*>(p->ws + p->L.hdr) + 10;
+            ws.chain_target = decode_combine_ctas(p->D, n, p->steer_on);
+        }
+        const cudaError_t ce = launch_decode(h->weights_view(), h->D, ws, in, n, o, h->n_sm, st, nullptr);
+        if (ce != cudaSuccess) return cuda_fail(ce, "forward_chain launch");
+    }
+    return DS4MOE_OK;
 }
 
 ds4moe_status ds4moe_forward_profiled(ds4moe_t* h, const void* d_x, int32_t n, float* d_out, void* const* events,

@@ -147,6 +147,12 @@ struct DecodeWs {
     int probe;              // 0: forward; 1: every token to routed expert probe_e; 2: the shared expert alone
     int probe_e;
     float* probe_out;       // probe: raw accumulators (gate/up: [n][2I]; down: [n][H])
+    // chained forward (ds4moe_forward_chain): the combine CTAs add 1 to chain_done once out is written;
+    // the next layer's projection prologue waits until chain_wait (the previous layer's chain_done)
+    // reaches chain_target, and its last CTA resets that counter
+    uint32_t* chain_done;
+    uint32_t* chain_wait;
+    uint32_t chain_target;
 };
 
 // Workspace pointers (prefill plan).

@@ -195,6 +195,25 @@ ds4moe_status ds4moe_forward(ds4moe_t* h, const void* d_x, int32_t n_tokens, flo
  * otherwise as ds4moe_forward. */
 ds4moe_status ds4moe_forward_residual(ds4moe_t* h, const void* d_x, int32_t n_tokens, float* d_out, void* stream);
 
+/* A chain of layers on the decode plan: x_{l+1} = x_l + layer_l(x_l) for
+ * l = 0 .. n_layers-1 (layers[l] applied to the previous layer's output),
+ * x_0 = d_x, the last output to d_out ([n_tokens][hidden] binary32).  The
+ * multi-token-prediction verify step of a model whose layers are these
+ * handles.  Every handle: bound, loaded, the same hidden size, n_tokens <=
+ * its decode_max and max_tokens; layers after the first take binary32 x
+ * (act_dtype F32).  d_work: caller device scratch of 2 * n_tokens * hidden
+ * binary32 (the intermediate outputs, ping-pong), 16-byte aligned, not
+ * overlapping d_x or d_out.  Layer l+1's kernels are launched as programmatic
+ * dependents of layer l's: its router loads its rows while layer l's combine
+ * runs, and its projection kernel streams the first shared-expert weights
+ * before x_{l+1} is ready (its prologue waits, bounded, on a counter that
+ * layer l's combine CTAs raise).  Results equal ds4moe_forward_residual layer
+ * by layer bit for bit.  Layer handles must be distinct (each keeps its own
+ * counters).  Errors as ds4moe_forward; a wait that runs out records
+ * DS4MOE_ERR_TIMEOUT in the device error word of the waiting layer. */
+ds4moe_status ds4moe_forward_chain(ds4moe_t* const* layers, int32_t n_layers, const void* d_x, int32_t n_tokens,
+                                   float* d_out, float* d_work, void* stream);
+
 /* The same computation with HOST buffers: copies x_host to the device (into
  * the workspace), runs ds4moe_forward on `stream`, copies the result to
  * out_host and waits for all of it (ds4moe_forward_host_async followed by

@@ -126,3 +126,91 @@ def test_chain_full_shape_two_tokens(orc):
         y, _, _ = orc.moe_forward(oracle_layer(L, experts=rid.ravel()), cur)
         cur = (cur.astype(np.float64) + y).astype(np.float32)
     assert rel_err(out.cpu().numpy(), cur) < 1e-4
+
+
+# ------------------------------------------------------------------ one call for the whole chain
+def _chain_call(lays, x, n):
+    out = torch.empty(n, lays[0].H, device="cuda")
+    work = torch.empty(2, n, lays[0].H, device="cuda")
+    m.ds4moe_forward_chain([lay.h for lay in lays], x, out, work)
+    torch.cuda.synchronize()
+    for lay in lays:
+        assert m.ds4moe_get_device_error(lay.h) == 0
+    return out
+
+
+@pytest.mark.parametrize("n", [1, 2, 8])
+def test_forward_chain_equals_layer_by_layer(orc, n):
+    """ds4moe_forward_chain (layers launched as programmatic dependents of one another, each prologue
+    waiting on the previous combine's count) gives the layer-by-layer residual chain bit for bit,
+    and so the oracle's chain within 1e-4; repeated calls reuse the counters."""
+    Ls, lays = _tiny_chain(orc)
+    x = synth.tokens(n, 256, seed=40 + n).cuda()
+    _, seq = _run_chain(lays, x)
+    for _ in range(3):
+        out = _chain_call(lays, x, n)
+        assert torch.equal(out, seq)
+    ref, _, _ = orc.chain_forward([oracle_layer(L) for L in Ls], x.cpu().numpy())
+    assert rel_err(out.cpu().numpy(), ref) < 1e-4
+
+
+def test_forward_chain_mixed_bits_and_steering(orc):
+    """A chain whose layers alternate 2-bit and 4-bit experts, one layer steered (its combine is the
+    one-CTA-per-token kernel, which the next layer counts), a bf16 first layer."""
+    from tests._util import pack_q4_with_oracle
+
+    H = 256
+    lays, Ls = [], []
+    for l in range(4):
+        L = synth.float_layer(synth.Shape(H=H, I=256, E=8, k=2), 500 + l, router_std=1.0 / math.sqrt(H))
+        bits = 4 if l % 2 else 0
+        L.update(pack_q4_with_oracle(orc, L) if bits == 4 else pack_with_oracle(orc, L))
+        lay = m.MoELayer(H, 256, 8, 2, 8, act_dtype=m.DS4MOE_ACT_BF16 if l == 0 else m.DS4MOE_ACT_F32,
+                         expert_bits=bits)
+        lay.load(L if bits != 4 else {**L, "grid": None})
+        lays.append(lay)
+        Ls.append(L)
+    v = synth.normal((H,), 1.0, synth.gen(7))
+    lays[2].set_steering((v / v.double().norm().float()).cuda().contiguous(), 0.5)
+    x = synth.tokens(3, H, seed=8, dtype=torch.bfloat16).cuda()
+    cur = x
+    for lay in lays:
+        cur = lay.forward(cur, residual=True)
+    out = _chain_call(lays, x, 3)
+    assert torch.equal(out, cur)
+
+
+def test_forward_chain_full_shape_two_tokens():
+    """8 full-shape layers, 2 tokens: the one-call chain equals the layer-by-layer chain bit for bit."""
+    H = 4096
+    shape = synth.Shape(H=H, I=2048, E=256, k=8)
+    lays = []
+    for l in range(LAYERS):
+        L = synth.packed_layer(shape, 300 + l, router_std=1.0 / math.sqrt(H), device="cuda",
+                               d_range=synth.CHAIN_D_RANGE, shared_std=synth.CHAIN_SHARED_STD)
+        lay = m.MoELayer(H, 2048, 256, 8, 8)
+        lay.load(L)
+        lays.append(lay)
+        del L
+    x = synth.tokens(2, H, seed=11).cuda()
+    _, seq = _run_chain(lays, x)
+    for _ in range(2):
+        assert torch.equal(_chain_call(lays, x, 2), seq)
+
+
+def test_forward_chain_argument_errors(orc):
+    Ls, lays = _tiny_chain(orc)
+    x = synth.tokens(2, 256, seed=1).cuda()
+    out = torch.empty(2, 256, device="cuda")
+    work = torch.empty(2, 2, 256, device="cuda")
+    with pytest.raises(m.Ds4MoeError) as ei:   # one handle twice
+        m.ds4moe_forward_chain([lays[0].h, lays[0].h], x, out, work)
+    assert ei.value.status == -1
+    with pytest.raises(m.Ds4MoeError) as ei:   # work overlaps out
+        m.ds4moe_forward_chain([lay.h for lay in lays], x, work[0], work)
+    assert ei.value.status == -1
+    bf = m.MoELayer(256, 128, 8, 2, 8, act_dtype=m.DS4MOE_ACT_BF16)
+    bf.load(Ls[1])
+    with pytest.raises(m.Ds4MoeError) as ei:   # a bf16 layer after the first
+        m.ds4moe_forward_chain([lays[0].h, bf.h], x, out, work)
+    assert ei.value.status == -3
