@@ -34,7 +34,8 @@ EXPORTS = ("ds4moe_create", "ds4moe_destroy", "ds4moe_weight_bytes", "ds4moe_wor
            "ds4moe_forward_profiled", "ds4moe_route_noalloc", "ds4moe_forward_residual",
            "ds4moe_forward_residual_profiled", "ds4moe_set_steering", "ds4moe_forward_host_async",
            "ds4moe_host_sync", "ds4moe_probe", "ds4moe_selftest_wait",
-           "ds4moe_permutation", "ds4moe_pack_q4k", "ds4moe_forward_chain")
+           "ds4moe_permutation", "ds4moe_pack_q4k", "ds4moe_forward_chain", "ds4moe_forward_routed",
+           "ds4moe_combine_slots")
 
 
 class ds4moe_shape(ctypes.Structure):
@@ -88,6 +89,8 @@ def lib() -> ctypes.CDLL:
             "ds4moe_route_noalloc": ([vp, vp, i32, vp, vp, vp], i32),
             "ds4moe_forward_residual": ([vp, vp, i32, vp, vp], i32),
             "ds4moe_forward_chain": ([ctypes.POINTER(vp), i32, vp, i32, vp, vp, vp], i32),
+            "ds4moe_forward_routed": ([vp, vp, i32, vp, vp, vp, vp], i32),
+            "ds4moe_combine_slots": ([vp, vp, vp, i32, i32, i32, vp, vp], i32),
             "ds4moe_set_steering": ([vp, vp, ctypes.c_float, vp], i32),
             "ds4moe_forward_residual_profiled": ([vp, vp, i32, vp, ctypes.POINTER(vp), vp], i32),
         }
@@ -182,6 +185,19 @@ def ds4moe_forward(h: int, x: torch.Tensor, out: torch.Tensor, stream=None):
 def ds4moe_set_steering(h: int, v: torch.Tensor | None, F: float, stream=None):
     _ok(lib().ds4moe_set_steering(h, None if v is None else _ptr(v), ctypes.c_float(F), _stream(stream)),
         "ds4moe_set_steering")
+
+
+def ds4moe_forward_routed(h: int, x: torch.Tensor, ids: torch.Tensor, w: torch.Tensor, out: torch.Tensor,
+                          stream=None):
+    _ok(lib().ds4moe_forward_routed(h, _ptr(x), x.shape[0], _ptr(ids), _ptr(w), _ptr(out), _stream(stream)),
+        "ds4moe_forward_routed")
+
+
+def ds4moe_combine_slots(y: torch.Tensor, w: torch.Tensor, base: torch.Tensor | None, out: torch.Tensor,
+                         stream=None):
+    n, k = w.shape
+    _ok(lib().ds4moe_combine_slots(_ptr(y), _ptr(w), _ptr(base), n, k, out.shape[1], _ptr(out), _stream(stream)),
+        "ds4moe_combine_slots")
 
 
 def ds4moe_forward_chain(handles, x: torch.Tensor, out: torch.Tensor, work: torch.Tensor, stream=None):

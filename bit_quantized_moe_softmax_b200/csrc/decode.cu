@@ -1653,6 +1653,44 @@ __global__ void __launch_bounds__(kSteerThreads) k_combine_steer_decode(Dims D, 
     chain_count(ws.chain_done);
 }
 
+// ---------------------------------------------------------------- caller routing
+__global__ void k_routing_in(const int32_t* ids_in, const float* wts_in, int nslots, int E, int32_t* ids, float* wts,
+                             uint32_t* ready, uint32_t* err) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nslots; i += gridDim.x * blockDim.x) {
+        const int e = ids_in[i];
+        const bool ok = e >= 0 && e < E;
+        if (!ok) set_err(err, kErrBounds);
+        ids[i] = ok ? e : 0;
+        wts[i] = ok ? wts_in[i] : 0.f;
+    }
+    if (ready) {
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ready), "r"(1u) : "memory");
+        }
+    }
+}
+
+// Expert-parallel combine: out[t][r] = base[t][r] + sum_j w[t][j] y[t k + j][r], j ascending, one FMA
+// per slot (the order of the layer's own combine); base may be absent (zero).
+__global__ void __launch_bounds__(256) k_combine_slots(const float* y, const float* w, const float* base, int n, int k,
+                                                       int H, float* out) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (int64_t)n * H) return;
+    const int t = (int)(i / H), r = (int)(i % H);
+    float acc = base ? base[i] : 0.f;
+    for (int j = 0; j < k; ++j) acc = fmaf(w[t * k + j], y[(int64_t)(t * k + j) * H + r], acc);
+    out[i] = acc;
+}
+
+cudaError_t launch_combine_slots(const float* y, const float* w, const float* base, int n, int k, int H, float* out,
+                                 cudaStream_t st) {
+    const int64_t nel = (int64_t)n * H;
+    k_combine_slots<<<(unsigned)((nel + 255) / 256), 256, 0, st>>>(y, w, base, n, k, H, out);
+    return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- grid tables
 // The decode plan's tables of a grid, made once when the grid is loaded (one
 // CTA of 256 threads): the distinct magnitudes in ascending order are classes
@@ -1813,7 +1851,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 template <int NT, bool Q4>
 cudaError_t launch_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n, float* out,
-                            int n_sm, cudaStream_t st, cudaEvent_t const* ev) {
+                            int n_sm, cudaStream_t st, cudaEvent_t const* ev, const int32_t* ids_in,
+                            const float* wts_in) {
     cudaError_t err;
     const size_t s1 = gateup_smem_bytes<NT>(D, n);
     if ((err = configure(k_moe_decode<NT, Q4>)) != cudaSuccess) return err;
@@ -1822,9 +1861,14 @@ cudaError_t launch_decode_t(const Weights& W, const Dims& D, const DecodeWs& ws,
     const bool pdl = ev == nullptr;   // profiled runs keep the kernels apart
     const int rgrid = (D.E + kRE - 1) / kRE;
     mk.before();
-    // chained layers: a programmatic dependent of the previous layer's combine (it loads its rows, then waits)
-    err = launch_pdl(k_router_decode<NT>, dim3(rgrid), dim3(RouterCfg<NT>::kWarps * 32), router_smem_bytes(D, n), st,
-                     pdl && ws.chain_wait != nullptr, W, D, ws, x, n, ws.route_ready);
+    if (ids_in) {   // caller routing: copied (and checked) in place of the router's, then published
+        k_routing_in<<<1, 128, 0, st>>>(ids_in, wts_in, n * D.k, D.E, ws.ids, ws.wts, ws.route_ready, ws.err);
+        err = cudaGetLastError();
+    } else {
+        // chained layers: a programmatic dependent of the previous layer's combine (it loads its rows, then waits)
+        err = launch_pdl(k_router_decode<NT>, dim3(rgrid), dim3(RouterCfg<NT>::kWarps * 32), router_smem_bytes(D, n),
+                         st, pdl && ws.chain_wait != nullptr, W, D, ws, x, n, ws.route_ready);
+    }
     mk.after();
     if (err != cudaSuccess) return err;
     mk.before();
@@ -1863,17 +1907,18 @@ size_t decode_smem_bytes(const Dims& D, int n) {
 }
 
 cudaError_t launch_decode(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n, float* out,
-                          int n_sm, cudaStream_t st, cudaEvent_t const* ev) {
+                          int n_sm, cudaStream_t st, cudaEvent_t const* ev, const int32_t* ids_in,
+                          const float* wts_in) {
     if (D.q4) {
-        if (n <= 1) return launch_decode_t<1, true>(W, D, ws, x, n, out, n_sm, st, ev);
-        if (n <= 2) return launch_decode_t<2, true>(W, D, ws, x, n, out, n_sm, st, ev);
-        if (n <= 4) return launch_decode_t<4, true>(W, D, ws, x, n, out, n_sm, st, ev);
-        return launch_decode_t<8, true>(W, D, ws, x, n, out, n_sm, st, ev);
+        if (n <= 1) return launch_decode_t<1, true>(W, D, ws, x, n, out, n_sm, st, ev, ids_in, wts_in);
+        if (n <= 2) return launch_decode_t<2, true>(W, D, ws, x, n, out, n_sm, st, ev, ids_in, wts_in);
+        if (n <= 4) return launch_decode_t<4, true>(W, D, ws, x, n, out, n_sm, st, ev, ids_in, wts_in);
+        return launch_decode_t<8, true>(W, D, ws, x, n, out, n_sm, st, ev, ids_in, wts_in);
     }
-    if (n <= 1) return launch_decode_t<1, false>(W, D, ws, x, n, out, n_sm, st, ev);
-    if (n <= 2) return launch_decode_t<2, false>(W, D, ws, x, n, out, n_sm, st, ev);
-    if (n <= 4) return launch_decode_t<4, false>(W, D, ws, x, n, out, n_sm, st, ev);
-    return launch_decode_t<8, false>(W, D, ws, x, n, out, n_sm, st, ev);
+    if (n <= 1) return launch_decode_t<1, false>(W, D, ws, x, n, out, n_sm, st, ev, ids_in, wts_in);
+    if (n <= 2) return launch_decode_t<2, false>(W, D, ws, x, n, out, n_sm, st, ev, ids_in, wts_in);
+    if (n <= 4) return launch_decode_t<4, false>(W, D, ws, x, n, out, n_sm, st, ev, ids_in, wts_in);
+    return launch_decode_t<8, false>(W, D, ws, x, n, out, n_sm, st, ev, ids_in, wts_in);
 }
 
 // Probe of the down kernel: caller h [n][I] binary32 -> the workspace's h pieces (routed layout at slots

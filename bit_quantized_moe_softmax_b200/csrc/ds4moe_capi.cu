@@ -28,14 +28,18 @@ __global__ void k_dequant_q2(const uint8_t* q, const uint32_t* sc, const uint32_
                              __nv_bfloat16* out_b);
 __global__ void k_dequant_bf16_tiles(const __nv_bfloat16* t, int R, int C, float* out_f, __nv_bfloat16* out_b);
 cudaError_t launch_decode(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n, float* out,
-                          int n_sm, cudaStream_t st, cudaEvent_t const* ev);
+                          int n_sm, cudaStream_t st, cudaEvent_t const* ev, const int32_t* ids_in = nullptr,
+                          const float* wts_in = nullptr);
+cudaError_t launch_combine_slots(const float* y, const float* w, const float* base, int n, int k, int H, float* out,
+                                 cudaStream_t st);
 int decode_launches();
 const char* decode_kernel_name(int i);
 size_t decode_smem_bytes(const Dims& D, int n);
 cudaError_t launch_route(const Weights& W, const Dims& D, const DecodeWs& ws, const void* x, int n,
                          cudaStream_t st);
 cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws, const void* x, int n, float* out,
-                           int n_sm, cudaStream_t st, cudaEvent_t const* ev);
+                           int n_sm, cudaStream_t st, cudaEvent_t const* ev, const int32_t* ids_in = nullptr,
+                           const float* wts_in = nullptr);
 cudaError_t launch_route_prefill(const Weights& W, const Dims& D, const PrefillWs& ws, const void* x, int n,
                                  cudaStream_t st);
 cudaError_t launch_wait_selftest(uint32_t* err, cudaStream_t st);
@@ -596,7 +600,8 @@ static ds4moe_status check_forward(ds4moe_t* h, const void* x, int32_t n, const 
 }
 
 static ds4moe_status forward_impl(ds4moe_t* h, const void* d_x, int32_t n, float* d_out, void* const* events,
-                                  void* stream, const char* who, bool residual = false) {
+                                  void* stream, const char* who, bool residual = false,
+                                  const int32_t* ids_in = nullptr, const float* wts_in = nullptr) {
     ds4moe_status s = check_forward(h, d_x, n, d_out, who);
     if (s != DS4MOE_OK) return s;
     if (n == 0) return DS4MOE_OK;
@@ -614,19 +619,36 @@ static ds4moe_status forward_impl(ds4moe_t* h, const void* d_x, int32_t n, float
         ws.xres = residual ? d_x : nullptr;
         ws.steer_v = h->steer_on ? reinterpret_cast<const float*>(h->weights + h->off_steer) : nullptr;
         ws.steer_F = h->steer_F;
-        ce = launch_decode(h->weights_view(), h->D, ws, d_x, n, d_out, h->n_sm, st, ev);
+        ce = launch_decode(h->weights_view(), h->D, ws, d_x, n, d_out, h->n_sm, st, ev, ids_in, wts_in);
     } else {
         PrefillWs ws = h->prefill_ws();
         ws.xres = residual ? d_x : nullptr;
         ws.steer_v = h->steer_on ? reinterpret_cast<const float*>(h->weights + h->off_steer) : nullptr;
         ws.steer_F = h->steer_F;
-        ce = launch_prefill(h->weights_view(), h->D, ws, d_x, n, d_out, h->n_sm, st, ev);
+        ce = launch_prefill(h->weights_view(), h->D, ws, d_x, n, d_out, h->n_sm, st, ev, ids_in, wts_in);
     }
     return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "forward launch");
 }
 
 ds4moe_status ds4moe_forward(ds4moe_t* h, const void* d_x, int32_t n, float* d_out, void* stream) {
     return forward_impl(h, d_x, n, d_out, nullptr, stream, "forward");
+}
+
+ds4moe_status ds4moe_forward_routed(ds4moe_t* h, const void* d_x, int32_t n, const int32_t* d_ids, const float* d_w,
+                                    float* d_out, void* stream) {
+    if (n > 0 && (!d_ids || !d_w)) return fail(DS4MOE_ERR_ARG, "forward_routed: NULL routing");
+    if ((reinterpret_cast<uintptr_t>(d_ids) | reinterpret_cast<uintptr_t>(d_w)) & 3)
+        return fail(DS4MOE_ERR_ALIGN, "forward_routed: ids and weights must be 4-byte aligned");
+    return forward_impl(h, d_x, n, d_out, nullptr, stream, "forward_routed", false, d_ids, d_w);
+}
+
+ds4moe_status ds4moe_combine_slots(const float* d_y, const float* d_w, const float* d_base, int32_t n, int32_t k,
+                                   int32_t H, float* d_out, void* stream) {
+    if (n < 0 || k < 1 || H < 1) return fail(DS4MOE_ERR_ARG, "combine_slots: n %d, k %d, hidden %d", n, k, H);
+    if (n == 0) return DS4MOE_OK;
+    if (!d_y || !d_w || !d_out) return fail(DS4MOE_ERR_ARG, "combine_slots: NULL buffer");
+    const cudaError_t ce = launch_combine_slots(d_y, d_w, d_base, n, k, H, d_out, (cudaStream_t)stream);
+    return ce == cudaSuccess ? DS4MOE_OK : cuda_fail(ce, "combine_slots launch");
 }
 
 ds4moe_status ds4moe_forward_residual(ds4moe_t* h, const void* d_x, int32_t n, float* d_out, void* stream) {

@@ -155,6 +155,13 @@ struct DecodeWs {
     uint32_t chain_target;
 };
 
+// Caller routing (ds4moe_forward_routed): ids_in / wts_in [nslots] copied to
+// ids / wts; an id outside [0, E) becomes expert 0 with weight 0 and sets
+// kErrBounds.  With `ready`, one CTA, which publishes the routing through it
+// (release) once every slot is written.
+__global__ void k_routing_in(const int32_t* ids_in, const float* wts_in, int nslots, int E, int32_t* ids, float* wts,
+                             uint32_t* ready, uint32_t* err);
+
 // Workspace pointers (prefill plan).
 struct PrefillWs {
     float* logits;          // [n][E]

@@ -974,7 +974,8 @@ struct Marks2 {
 };
 
 cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws, const void* x, int n, float* out,
-                           int n_sm, cudaStream_t st, cudaEvent_t const* ev) {
+                           int n_sm, cudaStream_t st, cudaEvent_t const* ev, const int32_t* ids_in,
+                           const float* wts_in) {
     cudaError_t e;
     Marks2 mk(ev, st);
     const int H = D.H, E = D.E, k = D.k, nslots = n * k;
@@ -987,12 +988,21 @@ cudaError_t launch_prefill(const Weights& W, const Dims& D, const PrefillWs& ws,
         mk.after();
         xb = ws.xb;
     }
-    mk.before();
-    if ((e = launch_router_prefill(W, D, x, n, ws.logits, st)) != cudaSuccess) return e;
-    mk.after();
-    mk.before();
-    k_topk_prefill<<<(n + 7) / 8, 256, 0, st>>>(D, ws.logits, n, ws.ids, ws.wts);
-    mk.after();
+    if (ids_in) {   // caller routing, copied (and checked) in place of the router's
+        mk.before();
+        k_routing_in<<<(unsigned)((nslots + 255) / 256), 256, 0, st>>>(ids_in, wts_in, nslots, E, ws.ids, ws.wts,
+                                                                      nullptr, ws.err);
+        mk.after();
+        mk.before();
+        mk.after();
+    } else {
+        mk.before();
+        if ((e = launch_router_prefill(W, D, x, n, ws.logits, st)) != cudaSuccess) return e;
+        mk.after();
+        mk.before();
+        k_topk_prefill<<<(n + 7) / 8, 256, 0, st>>>(D, ws.logits, n, ws.ids, ws.wts);
+        mk.after();
+    }
     mk.before();
     k_hist<<<nblk, kSortBlock, E * sizeof(int), st>>>(ws.ids, nslots, E, ws.blk_cnt);
     mk.after();

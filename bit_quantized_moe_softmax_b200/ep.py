@@ -122,3 +122,60 @@ def moe_forward_ep(x: torch.Tensor, ids: torch.Tensor, w: torch.Tensor, E: int, 
     rows, eid = dispatch(x, ids, p, group)
     y = local_fn(rows, eid) if rows.shape[0] else rows.new_zeros((0,) + tuple(base.shape[1:]))
     return combine(y, w, p, base, group)
+
+
+# ------------------------------------------------------------------ GPU halves (one rank's device work)
+class GpuExpertShard:
+    """This rank's experts on its GPU, as ``local_fn`` of ``moe_forward_ep``.
+
+    A ds4moe handle over the contiguous expert range the rank owns, with top_k
+    1 and no shared expert; every received row is one token routed to its
+    local expert with weight 1 (ds4moe_forward_routed), so each output row is
+    that expert's output for the row, computed by the same kernels as the
+    one-GPU layer.  ``layer``: canonical blocks of every expert (gate, up,
+    down indexed by global expert id), grid, H, I; rows beyond ``max_rows``
+    are processed in chunks (decode plan up to decode_max rows, the tensor-core
+    plan above)."""
+
+    def __init__(self, layer: dict, E: int, rank: int, world: int, max_rows: int, device="cuda", expert_bits=0):
+        from . import MoELayer
+
+        rng = local_experts(E, rank, world)
+        self.first, self.count = rng.start, len(rng)
+        self.max_rows = max_rows
+        self.H = layer["H"]
+        self.lay = MoELayer(layer["H"], layer["I"], self.count, 1, max_rows, has_shared=False, device=device,
+                            expert_bits=expert_bits) if self.count else None
+        if self.lay is not None:
+            sl = slice(self.first, self.first + self.count)
+            self.lay.load(dict(H=layer["H"], I=layer["I"], E=self.count, k=1,
+                               grid=layer.get("grid") if expert_bits != 4 else None,
+                               W_r=torch.zeros(self.count, layer["H"]), b_r=None,
+                               gate=layer["gate"][sl], up=layer["up"][sl], down=layer["down"][sl]))
+
+    def __call__(self, rows: torch.Tensor, row_expert: torch.Tensor) -> torch.Tensor:
+        from . import ds4moe_forward_routed
+
+        R = rows.shape[0]
+        out = torch.empty(R, self.H, dtype=torch.float32, device=rows.device)
+        ids = (row_expert - self.first).to(torch.int32).reshape(R, 1).contiguous()
+        ones = torch.ones(R, 1, dtype=torch.float32, device=rows.device)
+        for a in range(0, R, self.max_rows):
+            b = min(R, a + self.max_rows)
+            ds4moe_forward_routed(self.lay.h, rows[a:b].contiguous(), ids[a:b], ones[a:b], out[a:b])
+        return out
+
+
+def combine_gpu(y_rows: torch.Tensor, w: torch.Tensor, p: DispatchPlan, base: torch.Tensor, group=None):
+    """``combine`` with the sum on the device: the rows travel back and are put
+    in slot order as there, then ds4moe_combine_slots adds base + sum_j w_j
+    y_j, j ascending, one fused multiply-add per slot (the one-GPU layer's
+    combine order, so a layer split over ranks gives the same bits)."""
+    from . import ds4moe_combine_slots
+
+    back = _exchange(y_rows, p.n * p.k, p.recv_counts, p.send_counts, group)
+    ys = torch.empty_like(back)
+    ys[p.order] = back
+    out = torch.empty_like(base)
+    ds4moe_combine_slots(ys.contiguous(), w.to(torch.float32).contiguous(), base.contiguous(), out)
+    return out

@@ -195,6 +195,25 @@ ds4moe_status ds4moe_forward(ds4moe_t* h, const void* d_x, int32_t n_tokens, flo
  * otherwise as ds4moe_forward. */
 ds4moe_status ds4moe_forward_residual(ds4moe_t* h, const void* d_x, int32_t n_tokens, float* d_out, void* stream);
 
+/* The layer with the caller's routing instead of the router's: d_ids
+ * [n_tokens][top_k] int32 expert ids and d_w [n_tokens][top_k] binary32
+ * weights (device, 4-byte aligned), out[t] = shared(x_t) + sum_j w[t][j]
+ * expert_{ids[t][j]}(x_t), j in order, on the plan n_tokens selects.  An id
+ * outside [0, n_experts) counts as expert 0 with weight 0 and sets bit 0 of
+ * the device error word (ds4moe_get_device_error).  An id may repeat within a
+ * token.  The expert step of expert parallelism: a handle over one rank's
+ * experts with top_k 1, no shared expert, every received row a token, its
+ * local expert id and weight 1, gives each row's expert output. */
+ds4moe_status ds4moe_forward_routed(ds4moe_t* h, const void* d_x, int32_t n_tokens, const int32_t* d_ids,
+                                    const float* d_w, float* d_out, void* stream);
+
+/* Expert-parallel combine (no handle): out[t][r] = base[t][r] + sum_j
+ * w[t][j] y[t k + j][r], j = 0..k-1 in order, one fused multiply-add per slot
+ * (the layer's own combine order).  d_y [n k][H], d_w [n][k], d_base [n][H]
+ * or NULL (zero), d_out [n][H]: device binary32; d_out may alias d_base. */
+ds4moe_status ds4moe_combine_slots(const float* d_y, const float* d_w, const float* d_base, int32_t n, int32_t k,
+                                   int32_t hidden, float* d_out, void* stream);
+
 /* A chain of layers on the decode plan: x_{l+1} = x_l + layer_l(x_l) for
  * l = 0 .. n_layers-1 (layers[l] applied to the previous layer's output),
  * x_0 = d_x, the last output to d_out ([n_tokens][hidden] binary32).  The
