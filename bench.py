@@ -57,6 +57,9 @@ WORKLOADS = {
     "prefill512": dict(n=512, H=4096, I=2048, E=256, k=8, zipf=1.1, bf16=True,
                        desc="short-prompt prefill: 512 bf16 tokens, one MoE layer of the decode shape, "
                             "Zipf(1.1) expert popularity"),
+    "prefill512_q4": dict(n=512, H=4096, I=2048, E=256, k=8, zipf=1.1, bf16=True, expert_bits=4,
+                          desc="short-prompt prefill, 4-bit experts: 512 bf16 tokens, one MoE layer of the decode "
+                               "shape with Q4_K-style routed experts, Zipf(1.1) expert popularity"),
     "prefill11709": dict(n=11709, H=4096, I=2048, E=256, k=8, zipf=1.1, bf16=True,
                          desc="long-prompt prefill: 11,709 bf16 tokens, one MoE layer (hidden 4096, expert "
                               "intermediate 2048, 256 experts top-8 + shared), Zipf(1.1) expert popularity"),

@@ -314,13 +314,8 @@ ds4moe_status ds4moe_create(const ds4moe_shape* s, ds4moe_t** out) {
     if (s->decode_max < 0 || s->decode_max > 8) return fail(DS4MOE_ERR_SHAPE, "decode_max %d: need 0..8", s->decode_max);
     if (s->expert_bits != 0 && s->expert_bits != 2 && s->expert_bits != 4)
         return fail(DS4MOE_ERR_SHAPE, "expert_bits %d: need 0, 2 or 4", s->expert_bits);
-    if (s->expert_bits == 4) {
-        const int dm = s->decode_max ? s->decode_max : 8;
-        if (s->inter % 256) return fail(DS4MOE_ERR_SHAPE, "expert_bits 4: inter %d not a multiple of 256", s->inter);
-        if (s->max_tokens > dm)
-            return fail(DS4MOE_ERR_SHAPE, "expert_bits 4: max_tokens %d above decode_max %d (4-bit layers run the "
-                        "decode plan only)", s->max_tokens, dm);
-    }
+    if (s->expert_bits == 4 && s->inter % 256)
+        return fail(DS4MOE_ERR_SHAPE, "expert_bits 4: inter %d not a multiple of 256", s->inter);
     int dev = 0;
     cudaError_t ce = cudaGetDevice(&dev);
     if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
@@ -906,7 +901,8 @@ ds4moe_status ds4moe_route_noalloc(ds4moe_t* h, const void* d_x, int32_t n, int3
     if (n == 0) return DS4MOE_OK;
     if (!d_x || !d_ids || !d_w) return fail(DS4MOE_ERR_ARG, "route_noalloc: NULL buffer");
     if (!h->weights) return fail(DS4MOE_ERR_NOT_READY, "route_noalloc: buffers not bound");
-    if (!h->grid_set || !h->router_set) return fail(DS4MOE_ERR_NOT_READY, "route_noalloc: router not loaded");
+    if ((!h->grid_set && !h->D.q4) || !h->router_set)
+        return fail(DS4MOE_ERR_NOT_READY, "route_noalloc: router not loaded");
     if (!aligned16(d_x)) return fail(DS4MOE_ERR_ALIGN, "route_noalloc: x must be 16-byte aligned");
     if (n > h->decode_max) return fail(DS4MOE_ERR_ARG, "route_noalloc: n_tokens %d > decode_max %d", n, h->decode_max);
     if ((int64_t)n * h->D.E > kNoAllocLogits)

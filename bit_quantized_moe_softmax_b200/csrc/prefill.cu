@@ -417,15 +417,57 @@ __device__ __forceinline__ uint4 q2_unit_bf16(uint32_t x, float2 sc2, float2 nmn
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// Eight 4-bit codes (byte j: column j in the low nibble, column 4 + j in the
+// high nibble) -> 8 bf16 of (d sc) q - dmin m, columns 0..7.  With the two
+// bytes of a pair in the low half of v, the nibble at bits b..b+3 (b <= 12,
+// inside the mantissa) becomes the binary32 2^(23-b) + q with one AND-OR
+// (biased exponent 150 - b), as in q2_unit_bf16; one FMA then rounds the
+// weight once.
+__device__ __forceinline__ uint4 q4_word_bf16(uint32_t x, float2 sc2, float2 nmn2) {
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        // columns 2j, 2j+1: bytes 0, 1 (j even) or 2, 3 (j odd) of x; low nibbles for j < 2, high after
+        const uint32_t v = (j & 1) ? (x >> 16) : (x & 0xffffu);
+        const int b0 = (j & 2) ? 4 : 0, b1 = b0 + 8;
+        const float f0 = __uint_as_float(((150u - b0) << 23) | (v & (15u << b0)));
+        const float f1 = __uint_as_float(((150u - b1) << 23) | (v & (15u << b1)));
+        const float2 q = fadd2(make_float2(f0, f1), make_float2(-__uint_as_float((150u - b0) << 23),
+                                                                -__uint_as_float((150u - b1) << 23)));
+        const float2 w = ffma2(sc2, q, nmn2);
+        o[j] = pack_bf16x2(w.x, w.y);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// The eight codes of 16-byte unit 4h + p (columns 8(4h + p) .. +7 of a
+// 64-column step) of a down row in the 4-bit code order (q4_dev_col mode 1:
+// column 32h + 16 (p >> 1) + 8 (p & 1) + 4e + t sits at nibble p + 4e of word
+// (t, h); wh[t] = word (t, h)), gathered into q4_word_bf16's byte order.
+__device__ __forceinline__ uint32_t q4_down_unit(const uint32_t (&wh)[4], int p) {
+    const uint32_t a0 = wh[0] >> (4 * p), a1 = wh[1] >> (4 * p), a2 = wh[2] >> (4 * p), a3 = wh[3] >> (4 * p);
+    // nibble p of word t (e = 0) in the low nibble of byte t, nibble p + 4 (e = 1) in its high nibble
+    const uint32_t lo = __byte_perm(__byte_perm(a0, a1, 0x0040u), __byte_perm(a2, a3, 0x0040u), 0x5410u);
+    const uint32_t hi = __byte_perm(__byte_perm(a0, a1, 0x0062u), __byte_perm(a2, a3, 0x0062u), 0x5410u);
+    return (lo & 0x0F0F0F0Fu) | ((hi & 0x0F0F0F0Fu) << 4);
+}
+
 // One dequantizing thread's packed weights for one k step (64 weights of one B row).
+template <bool Q4>
 struct BFrag {
-    uint4 q;        // IQ2: two (grid indices, signs+scale) pairs; Q2: 64 codes
-    uint32_t a0;    // IQ2: d (binary16 bits); Q2: four scale bytes
-    uint32_t a1;    // Q2: d | dmin << 16
+    uint4 q;        // IQ2: two (grid indices, signs+scale) pairs; Q2: 64 codes; Q4: codes of columns 0..31
+    uint32_t a0;    // IQ2: d (binary16 bits); Q2: four scale bytes; Q4: sc, sc, m, m of the two sub-blocks
+    uint32_t a1;    // Q2, Q4: d | dmin << 16
+};
+template <>
+struct BFrag<true> {
+    uint4 q, q2;    // Q4: the row's 32 code bytes of the step
+    uint32_t a0, a1;
 };
 
-// Warp roles: 0 TMA, 1 MMA, 2..9 dequantize B, 10..17 epilogue.
-template <int MODE>
+// Warp roles: 0 TMA, 1 MMA, 2..9 dequantize B, 10..17 epilogue.  Q4: the routed
+// experts are 4-bit blocks (no grid).
+template <int MODE, bool Q4>
 __global__ void __launch_bounds__(kGThreads, 1)
     k_moe_gemm(const __grid_constant__ CUtensorMap tmapA, const __grid_constant__ CUtensorMap tmapB0,
                const __grid_constant__ CUtensorMap tmapB1, GemmArgs a) {
@@ -460,7 +502,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
         S.abort = 0;
         fence_barrier_init();
     }
-    if (MODE == kModeGateUp) {
+    if (MODE == kModeGateUp && Q4 && tid == 0 && blockIdx.x == 0 && a.grid_refused) *a.grid_refused = 0u;
+    if (MODE == kModeGateUp && !Q4) {
         // magnitude classes of the grid bytes (stage A is free until the pipeline starts)
         int* present = reinterpret_cast<int*>(stA);
         int* cls = present + 256;
@@ -599,7 +642,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int r = tid - 64;   // B-tile row 0..255
             const unsigned char* selp = seltab + (lane & 15) * 8;
             float2 gv01 = make_float2(0.f, 0.f), gv23 = make_float2(0.f, 0.f);
-            if (MODE == kModeGateUp) {
+            if (MODE == kModeGateUp && !Q4) {
                 gv01 = make_float2(S.gval[0], S.gval[1]);
                 gv23 = make_float2(S.gval[2], S.gval[3]);
             }
@@ -619,7 +662,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 const TileInfo ti = tile_info<MODE>(a, tile, NB);
                 const size_t e = (size_t)ti.e;
                 keep = __ldg(a.counts + e) > kGBM;
-                if (MODE == kModeGateUp) {
+                if (Q4) {
+                    // codes [R/32][C/64][32][32 B], scale words [R/32][C/64][32], (d, dmin) [R/32][C/256][32]
+                    const bool gu = MODE == kModeGateUp;
+                    const int row = gu ? 128 * ti.nb + (r & 127) : kGBN * ti.nb + r;
+                    const int nkt = (gu ? H : I) / 64, nsb = (gu ? H : I) / 256;
+                    const uint8_t* qb = gu ? (r < 128 ? a.W.gate_qs : a.W.up_qs) : a.W.down_q;
+                    const uint32_t* sb = gu ? (r < 128 ? a.W.gate_sc4 : a.W.up_sc4) : a.W.down_sc4;
+                    const uint32_t* db = gu ? (r < 128 ? a.W.gate_dd4 : a.W.up_dd4) : a.W.down_dd4;
+                    qs = qb + e * a.W.q4_q_stride + ((size_t)(row >> 5) * nkt * 32 + (row & 31)) * 32;
+                    scp = sb + e * a.W.q4_sc_stride + (size_t)(row >> 5) * nkt * 32 + (row & 31);
+                    ddp = db + e * a.W.q4_dd_stride + (size_t)(row >> 5) * nsb * 32 + (row & 31);
+                } else if (MODE == kModeGateUp) {
                     const int row = 128 * ti.nb + (r & 127);
                     qs = (r < 128 ? a.W.gate_qs : a.W.up_qs) + e * a.W.iq2_qs_stride +
                          (size_t)(row >> 5) * (H / 64) * 512 + (row & 31) * 16;
@@ -633,7 +687,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     ddp = a.W.down_dd + e * a.W.q2_dd_stride + (size_t)(row >> 5) * nsb * 32 + (row & 31);
                 }
             };
-            auto fetch = [&](BFrag& f) {
+            auto fetch = [&](BFrag<Q4>& f) {
+                if constexpr (Q4) {
+                    const uint8_t* src = qs + (size_t)cks * 1024;
+                    f.q = keep ? ld_stream_v4_hint(src, pol_keep) : ld_stream_v4(src);
+                    f.q2 = keep ? ld_stream_v4_hint(src + 16, pol_keep) : ld_stream_v4(src + 16);
+                    f.a0 = ld_stream_u32(scp + cks * 32);
+                    f.a1 = ld_stream_u32(ddp + (cks >> 2) * 32);
+                } else {
                 f.q = keep ? ld_stream_v4_hint(qs + (size_t)cks * 512, pol_keep) : ld_stream_v4(qs + (size_t)cks * 512);
                 if (MODE == kModeGateUp) {
                     f.a0 = ld_stream_u16(dq + (cks >> 2) * 32);
@@ -641,14 +702,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     f.a0 = ld_stream_u32(scp + cks * 32);
                     f.a1 = ld_stream_u32(ddp + (I >= 256 ? (cks >> 2) : 0) * 32);
                 }
+                }
                 if (++cks == KS) {
                     cks = 0;
                     ctile += gridDim.x;
                     if (ctile < ntiles) set_src(ctile);
                 }
             };
-            constexpr int PD = 4;   // k steps of packed weights in flight
-            BFrag ring[PD];
+            constexpr int PD = Q4 ? 2 : 4;   // k steps of packed weights in flight (4-bit steps are 32 bytes)
+            BFrag<Q4> ring[PD];
             if (total > 0) set_src(ctile);
 #pragma unroll
             for (int p = 0; p < PD; ++p)
@@ -658,7 +720,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
                 for (int p = 0; p < PD; ++p) {
                     if (j0 + p >= total) break;
-                    const BFrag cur = ring[p];
+                    const BFrag<Q4> cur = ring[p];
                     if (j0 + p + PD < total) fetch(ring[p]);
                     const int s = it % kGStages;
                     if (!mbar_wait(&S.empty[s], ((it / kGStages) & 1) ^ 1, a.err)) {
@@ -666,7 +728,26 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         break;
                     }
                     unsigned char* bt = stB + s * kGBStage + b_row_off(r);
-                    if (MODE == kModeGateUp) {
+                    if constexpr (Q4) {
+                        // 16-byte unit c = columns 8c .. 8c+7, in the 32-column sub-block c >> 2
+                        const float d = half_bits(cur.a1 & 0xffffu), dmin = half_bits(cur.a1 >> 16);
+                        // one 32-column half at a time (both unrolled spill at the 96-register budget); word
+                        // (t, h) of the step is code bytes 8t + 4h .. +3
+#pragma unroll 1
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t wh[4] = {h ? cur.q.y : cur.q.x, h ? cur.q.w : cur.q.z,
+                                                    h ? cur.q2.y : cur.q2.x, h ? cur.q2.w : cur.q2.z};
+                            const float sc = d * (float)((cur.a0 >> (8 * h)) & 0xffu);
+                            const float mn = dmin * (float)((cur.a0 >> (16 + 8 * h)) & 0xffu);
+                            const float2 sc2 = make_float2(sc, sc), nmn2 = make_float2(-mn, -mn);
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                // gate/up (code order mode 0): unit 4h + t is word (t, h) as it stands
+                                const uint32_t x = MODE == kModeGateUp ? wh[t] : q4_down_unit(wh, t);
+                                *reinterpret_cast<uint4*>(bt + (4 * h + t) * 128) = q4_word_bf16(x, sc2, nmn2);
+                            }
+                        }
+                    } else if (MODE == kModeGateUp) {
                         const float d = half_bits(cur.a0);
 #pragma unroll
                         for (int hf = 0; hf < 2; ++hf) {
@@ -882,10 +963,12 @@ size_t gemm_smem_bytes() { return 1024 + (size_t)kGStages * (kGAStage + kGBStage
 size_t gemm_static_smem_bytes() {
     size_t m = 0;
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeGateUp>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
-    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeDown>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
-    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeShGateUp>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
-    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeShDown>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeGateUp, false>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeDown, false>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeGateUp, true>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeDown, true>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeShGateUp, false>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, k_moe_gemm<kModeShDown, false>) == cudaSuccess && fa.sharedSizeBytes > m) m = fa.sharedSizeBytes;
     return m > sizeof(GemmSmem) ? m : sizeof(GemmSmem);
 }
 
@@ -930,14 +1013,23 @@ static cudaError_t encode_tmap_core(CUtensorMap* map, const void* base, uint64_t
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+template <int MODE, bool Q4>
+static cudaError_t launch_gemm_t(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
+                                 const GemmArgs& args, int n_sm, cudaStream_t st) {
+    const size_t smem = gemm_smem_bytes();
+    cudaError_t e = smem_opt_in(reinterpret_cast<const void*>(k_moe_gemm<MODE, Q4>), (int)smem);
+    if (e != cudaSuccess) return e;
+    k_moe_gemm<MODE, Q4><<<n_sm, kGThreads, smem, st>>>(mapA, mapB0, mapB1, args);
+    return cudaGetLastError();
+}
+// The routed modes take the layer's expert format; the shared-expert modes have one.
 template <int MODE>
 static cudaError_t launch_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB0, const CUtensorMap& mapB1,
                                const GemmArgs& args, int n_sm, cudaStream_t st) {
-    const size_t smem = gemm_smem_bytes();
-    cudaError_t e = smem_opt_in(reinterpret_cast<const void*>(k_moe_gemm<MODE>), (int)smem);
-    if (e != cudaSuccess) return e;
-    k_moe_gemm<MODE><<<n_sm, kGThreads, smem, st>>>(mapA, mapB0, mapB1, args);
-    return cudaGetLastError();
+    if constexpr (MODE == kModeGateUp || MODE == kModeDown) {
+        if (args.D.q4) return launch_gemm_t<MODE, true>(mapA, mapB0, mapB1, args, n_sm, st);
+    }
+    return launch_gemm_t<MODE, false>(mapA, mapB0, mapB1, args, n_sm, st);
 }
 
 const char* const kPrefillKernels[] = {"k_router_prefill", "k_topk_prefill", "k_hist", "k_scan", "k_scatter",

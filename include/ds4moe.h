@@ -83,8 +83,8 @@ typedef struct {
                               the little-endian 96-bit integer of bytes 4..15;
                               the 4-bit code of weight i at byte 16 + i/2, low
                               nibble for even i; weight = d sc q - dmin m).
-                              4-bit layers run the decode plan only:
-                              max_tokens <= decode_max, inter % 256 == 0. */
+                              4-bit layers need inter % 256 == 0 and no
+                              grid. */
 } ds4moe_shape;
 
 typedef struct ds4moe ds4moe_t;   /* opaque handle; host memory owned by the library */

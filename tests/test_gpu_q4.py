@@ -206,3 +206,75 @@ def test_forward_q4_repeatable(orc):
     for o in outs[1:]:
         assert np.array_equal(o, outs[0])
 
+
+
+# ------------------------------------------------------------------ tensor-core plan (more than decode_max tokens)
+PTOL = 2e-3   # the bf16 reading's bar (x, dequantized weights and h rounded to bf16, fp32 accumulation)
+
+
+@pytest.mark.parametrize("n", [24, 200])
+def test_forward_q4_prefill_tiny_matches_oracle(orc, n):
+    L = _tiny(orc)
+    lay = _load(L, max_tokens=256, act=m.DS4MOE_ACT_BF16)
+    x = synth.tokens(n, 256, seed=80 + n, dtype=torch.bfloat16)
+    out = lay.forward(x.cuda()).cpu().numpy()
+    ref, _, _ = orc.moe_forward(oracle_layer(L), x.float().numpy(), mode=1)
+    assert rel_err(out, ref) < PTOL
+
+
+@pytest.mark.parametrize("variant", ["f32_act", "no_shared", "bias", "two_row_tiles", "wide_hidden"])
+def test_forward_q4_prefill_variants(orc, variant):
+    kw = dict(bias=variant == "bias", shared=variant != "no_shared")
+    n = 64
+    if variant == "two_row_tiles":   # about 300 rows per expert: a full 256-row tile and a ragged one
+        kw.update(E=4, k=2)
+        n = 600
+    if variant == "wide_hidden":
+        kw.update(H=1024, I=512)
+    L = _tiny(orc, **kw)
+    act = m.DS4MOE_ACT_F32 if variant == "f32_act" else m.DS4MOE_ACT_BF16
+    lay = _load(L, max_tokens=n, act=act)
+    x = synth.tokens(n, L["H"], seed=90, dtype=torch.float32 if act == m.DS4MOE_ACT_F32 else torch.bfloat16)
+    out = lay.forward(x.cuda()).cpu().numpy()
+    ref, _, _ = orc.moe_forward(oracle_layer(L), x.float().numpy(), mode=1)
+    assert rel_err(out, ref) < PTOL
+
+
+@pytest.mark.parametrize("which", [0, 2])
+def test_probe_q4_prefill_bit_exact(orc, which):
+    """One-hot bf16 rows through the tensor-core plan's GEMM: column c of each matrix is the oracle's
+    dequantized weight rounded to bf16, bit for bit (edge blocks included)."""
+    from tests.test_gpu_exact import _probe_columns, _same_bits
+
+    H, I, E = 256, 512, 4
+    L = _tiny(orc, E=E, k=1, H=H, I=I)
+    nb = H * I // 256
+    L["gate"][1] = _edge_blocks(nb, 4)
+    L["up"][1] = _edge_blocks(nb, 5)
+    L["down"][1] = _edge_blocks(nb, 6)
+    lay = _load(L, max_tokens=64)
+    for e in (1, 2):
+        got = _probe_columns(lay, 1, which, e)
+        if which == 0:
+            ref = np.concatenate([orc.dequant_q4k(L[n][e].numpy()).reshape(I, H) for n in ("gate", "up")]).T
+        else:
+            ref = orc.dequant_q4k(L["down"][e].numpy()).reshape(H, I).T
+        _same_bits(got, orc.bf16_round(ref))
+
+
+def test_forward_q4_prefill_full_shape_short_prompt(orc):
+    """512 bf16 tokens through a full-size 4-bit layer with Zipf(1.1) expert popularity (sampled outputs)."""
+    bias = synth.zipf_bias(256, 1.1, seed=5)
+    L = synth.packed_layer(synth.FULL, 6, bias=bias, device="cuda", expert_bits=4)
+    n = 512
+    lay = _load(L, max_tokens=n, act=m.DS4MOE_ACT_BF16)
+    x = synth.tokens(n, 4096, seed=9, dtype=torch.bfloat16)
+    out = lay.forward(x.cuda()).cpu().numpy()
+    lg = orc.router_logits(x.float().numpy(), L["W_r"].cpu().numpy(), bias.numpy())
+    rid, _ = orc.topk_softmax(lg, 8)
+    ids, _ = lay.route(x.cuda())
+    assert np.array_equal(ids.cpu().numpy(), rid)
+    sample = [0, 1, 255, 511]
+    ref, _, _ = orc.moe_forward(oracle_layer(L, experts=rid[sample].ravel()), x[sample].float().numpy(), mode=1)
+    assert rel_err(out[sample], ref) < PTOL
+    assert np.isfinite(out).all()
