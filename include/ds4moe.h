@@ -291,8 +291,11 @@ ds4moe_status ds4moe_route(ds4moe_t* h, const void* d_x, int32_t n_tokens, int32
 
 /* Dequantize expert e's matrix `which` (0 gate, 1 up, 2 down) from the
  * loaded device layout into d_out, row-major, as binary32 (as_bf16 = 0) or
- * bfloat16 rounded to nearest even (as_bf16 = 1): exactly the values the
- * kernels multiply. */
+ * bfloat16 rounded to nearest even (as_bf16 = 1): the weights the block
+ * format defines, read back from the device layout by a plain per-element
+ * kernel (a check of the layout and the repack; the hot-path kernels keep
+ * their own operand forms, e.g. 1 + q/4 with an affine correction, and
+ * ds4moe_probe shows that what they multiply equals these values). */
 ds4moe_status ds4moe_dequant(ds4moe_t* h, int32_t e, int32_t which, int32_t as_bf16, void* d_out,
                              void* stream);
 
@@ -301,8 +304,8 @@ ds4moe_status ds4moe_dequant(ds4moe_t* h, int32_t e, int32_t which, int32_t as_b
  * out as they are: the inspection the bit-exactness of the weights the
  * kernels multiply rests on (one-hot rows give back columns of the weight
  * matrices exactly as the tensor cores consumed them).
- *   plan 0 (the decode plan; n <= decode_max): the persistent gate/up and
- *     down kernels.  which 0: d_in = activations [n][H] binary32 (or bf16
+ *   plan 0 (the decode plan; n <= decode_max): the persistent projection
+ *     kernel (gate/up or down tasks only).  which 0: d_in = activations [n][H] binary32 (or bf16
  *     when act_dtype is DS4MOE_ACT_BF16), d_out = [n][2I] binary32, gate
  *     results then up results (no SwiGLU); which 2: d_in = h [n][I]
  *     binary32 (entering as the kernel's two bf16 pieces), d_out = [n][H].
