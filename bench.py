@@ -522,7 +522,7 @@ def _timed_run(args, wl, rank, local, world, dev, layers, xs, outs, stream, nl, 
                    "steering_F": args.steer},
         "expert_weight_gbs": round(C * ab["routed"] / (ms_per_step * 1e-3) / 1e9, 1) if U else None,
         "layer_hbm_gbs": round(C * ab["layer"] / (ms_per_step * 1e-3) / 1e9, 1) if U else None,
-        "layer_frac_of_hbm_peak": round(C * ab["layer"] / (ms_per_step * 1e-3) / 1e9 / peak, 4) if U else None,
+        "layer_frac_of_hbm_peak": round(C * ab["layer"] / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4) if U else None,
         "kernel_us": {nm: round(mean[nm] * 1e3, 2) for nm in names},
         "ms_per_step_profiled": round(ms_prof / args.steps, 5),
         "roofline": roofline, "e2e": e2e, "gpu_launches": nl * C * args.steps, "clocks": clocks,
