@@ -53,6 +53,7 @@ namespace ds4 {
 
 constexpr int kMaxSlots = 128;                 // decode_max (<= 8) * top_k (<= 16)
 constexpr int kStageBytes = 34816;             // 32 KB of weights + 2 KB of scales
+constexpr uint32_t kTabAddr = 0x20000;          // shared address of the one- and two-token selector table
 constexpr int kRE = 2;                         // router rows (warps) per CTA
 
 // ---------------------------------------------------------------- warp MMAs
@@ -669,11 +670,18 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     constexpr int kTab = Q4 ? 0 : C::kTabWords;
     constexpr int kStage = C::kStage;
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    uint32_t* tsel = reinterpret_cast<uint32_t*>(smem_raw);                      // rows [256][64] or [256][R]
+    // one or two tokens (rows table): the table sits at shared address kTabAddr, after the stages and the
+    // reduction ring, so that one byte permute (grid row, lane offset, the address's upper bytes) is a
+    // row's address with no add; x's buffers follow it
+    constexpr bool kAbs = !Q4 && C::kRows;
+    const uint32_t base = smem_addr(smem_raw);
+    uint32_t* tsel = kAbs ? reinterpret_cast<uint32_t*>(smem_raw + (kTabAddr - base))
+                          : reinterpret_cast<uint32_t*>(smem_raw);                // rows [256][64] or [256][R]
     uint32_t* tsgn = tsel + 256 * R;                                             // [128][R] (interleaved form)
-    unsigned char* stages = smem_raw + 4 * kTab;                                 // NS x kStage
+    unsigned char* stages = kAbs ? smem_raw : smem_raw + 4 * kTab;               // NS x kStage
     float* red = reinterpret_cast<float*>(stages + NS * kStage);                 // kRedFloats
-    unsigned char* xbuf = reinterpret_cast<unsigned char*>(red + C::kRedFloats);  // n x H x 4 bytes: bf16 pieces
+    unsigned char* xbuf = kAbs ? reinterpret_cast<unsigned char*>(tsel + 256 * 64)
+                               : reinterpret_cast<unsigned char*>(red + C::kRedFloats);  // n x H x 4 bytes: bf16 pieces
     unsigned char* xq = C::kSplitX ? xbuf + (size_t)n * D.H * 4 : xbuf;          // int8 pieces
     unsigned char* zero = xq + (size_t)n * D.H * 4;                              // 64 bytes of zeros
     float* xsum = reinterpret_cast<float*>(zero + 64);                           // Q4: [n][H / 32] sums of x
@@ -712,6 +720,18 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
     const int dnch_sh = I / dkcs;
 
     __shared__ uint64_t tab_bar;
+    if (kAbs) {
+        // the layout needs the dynamic shared memory to reach past the table (the launch asks for it, counting
+        // at least 4 KB of static shared memory before it): refuse the call instead of running out of it
+        uint32_t dyn;
+        asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+        const uint32_t need_end = kTabAddr + 256 * 64 * 4 + (C::kSplitX ? 2u : 1u) * n * D.H * 4 + 64;
+        const uint32_t low_end = base + NS * kStage + 4 * C::kRedFloats;
+        if (low_end > kTabAddr || need_end > base + dyn) {
+            if (tid == 0) set_err(ws.err, kErrBounds);
+            return;
+        }
+    }
     pipe_init(P, NS, CW);
     if (!Q4 && C::kRows && tid == 0) {
         // the selector table: one bulk copy, waited for at the end of the prologue
@@ -1033,8 +1053,9 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
         const uint32_t selO = (t >> 1) ? 0xFEDCu : 0xBA98u;   // this lane's group's S word, top bits
         const uint32_t* tselp = tsel + (lane % R);
         const uint32_t* tsgnp = tsgn + (lane % R);
-        const uint32_t tb = smem_addr(tsel);
-        const uint32_t lbA = (uint32_t)lane << 2, lbB = 128u | ((uint32_t)lane << 2);
+        const uint32_t tb = kAbs ? 0u : smem_addr(tsel);
+        const uint32_t hiA = kAbs ? (kTabAddr >> 16) << 16 : 0u;   // bytes 2, 3 of a row's address
+        const uint32_t lbA = hiA | ((uint32_t)lane << 2), lbB = hiA | 128u | ((uint32_t)lane << 2);
         const uint32_t selT = 0x7604u | ((uint32_t)t << 4);
         const uint32_t clo = s_cand[0], chi = s_cand[1];
         // B operand lanes: column g of the MMA
@@ -1773,6 +1794,8 @@ cudaError_t launch_wait_selftest(uint32_t* err, cudaStream_t st) {
 template <int NT, bool Q4>
 size_t gateup_smem_bytes_t(const Dims& D, int n) {
     using C = GateUpCfg<NT, Q4>;
+    if (!Q4 && C::kRows)   // up to the table's end, less the static shared memory (at least 4 KB) before it
+        return (size_t)kTabAddr + 256 * 64 * 4 + (size_t)(C::kSplitX ? 2 : 1) * n * D.H * 4 + 64 - 4096;
     return (size_t)C::NS * C::kStage + 4 * ((size_t)(Q4 ? 0 : C::kTabWords) + C::kRedFloats) +
            (size_t)(C::kSplitX ? 2 : 1) * n * D.H * 4 + 64 + (Q4 ? (size_t)n * (D.H / 32) * 4 : 0);
 }
