@@ -552,16 +552,16 @@ def _pool_map(fn, items, budget_s):
     return done, time.perf_counter() - t0
 
 
-def oracle_sample(wl, n_tokens, seed=0, budget_s=20.0, device="cuda"):
+def oracle_sample(wl, n_tokens, seed=0, budget_s=20.0, device="cuda", warmup=0):
     """Oracle tokens/s on a bounded sample of the workload (router + top-k + experts + shared), one token per
-    task, on all host cores.  Returns (tokens/s, tokens done, seconds, cores)."""
+    task, on all host cores, after `warmup` untimed tokens.  Returns (tokens/s, tokens done, seconds, cores)."""
     import oracle
     from bit_quantized_moe_softmax_b200 import synth
 
     H, I, E, k = wl["H"], wl["I"], wl["E"], wl["k"]
     bias = synth.zipf_bias(E, wl["zipf"], seed=5) if wl.get("zipf") else None
     if wl.get("layers", 1) > 1:
-        return oracle_chain_sample(wl, n_tokens, seed, budget_s, device)
+        return oracle_chain_sample(wl, n_tokens, seed, budget_s, device, warmup)
     L = synth.packed_layer(synth.Shape(H=H, I=I, E=E, k=k), seed=seed, bias=bias, device=device,
                            expert_bits=wl.get("expert_bits", 2))
     x = synth.tokens(n_tokens, H, seed=seed + 5, dtype=torch.bfloat16 if wl.get("bf16") else torch.float32).float()
@@ -571,11 +571,13 @@ def oracle_sample(wl, n_tokens, seed=0, budget_s=20.0, device="cuda"):
     lay = oracle.layer_from_torch(L, experts=rid.ravel())
     del L
     xs = x.numpy()
+    if warmup:
+        _pool_map(lambda t: oracle.moe_forward(lay, xs[t:t + 1], mode=mode), range(min(warmup, n_tokens)), budget_s)
     done, dt = _pool_map(lambda t: oracle.moe_forward(lay, xs[t:t + 1], mode=mode), range(n_tokens), budget_s)
     return len(done) / dt, len(done), dt, os.cpu_count() or 1
 
 
-def oracle_chain_sample(wl, n_tokens, seed, budget_s, device):
+def oracle_chain_sample(wl, n_tokens, seed, budget_s, device, warmup=0):
     """Oracle tokens/s through the chain of layers (fp64 layers, binary32 between layers), one token per task
     on all host cores; each task routes its token layer by layer and runs the layer on the experts it picks."""
     import oracle
@@ -596,6 +598,8 @@ def oracle_chain_sample(wl, n_tokens, seed, budget_s, device):
             cur = (cur.astype(np.float64) + y).astype(np.float32)
         return cur
 
+    if warmup:
+        _pool_map(one, range(min(warmup, n_tokens)), budget_s)
     done, dt = _pool_map(one, range(n_tokens), budget_s)
     return len(done) / dt, len(done), dt, os.cpu_count() or 1
 
@@ -615,15 +619,23 @@ def run_reference(args, wl, rank, world):
         return None
     budget = 120.0
     cores = os.cpu_count() or 1
-    rate, done, dt, cores = oracle_sample(wl, n_tokens=max(cores, args.steps), budget_s=budget)
+    # the seeded layer is drawn on the GPU when there is one (the same bytes as our arm's); without one,
+    # torch's CPU generator draws a layer of the same shape and distribution
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    warm = max(3, min(args.warmup, cores))   # untimed tokens first (one per host thread at most)
+    rate, done, dt, cores = oracle_sample(wl, n_tokens=max(cores, args.steps), budget_s=budget, device=device,
+                                          warmup=warm)
     cpu = host_cpu()
     sample = ("%d tokens (one per task; %d requested steps, n=%d per step in our arm) through the CPU oracle "
-              "(canonical binary32 router, fp64 dequantized experts and shared expert) on %d host threads, "
-              "no new task after a %.0f s budget" % (done, args.steps, wl["n"], cores, budget))
+              "(canonical binary32 router, fp64 dequantized experts and shared expert) on %d host threads after %d "
+              "untimed tokens, no new task after a %.0f s budget" % (done, args.steps, wl["n"], cores, warm, budget))
     return {"impl": "reference", "metric": METRIC, "value": round(rate, 4), "unit": "tokens/s", "n_gpus": world,
-            "steps": done, "steps_requested": args.steps, "warmup": 0, "ms_per_step": round(dt / done * 1e3, 2),
+            "steps": done, "steps_requested": args.steps, "warmup": warm, "ms_per_step": round(dt / done * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl["desc"], "n_tokens_per_step": 1},
+            "config": {"workload": wl["desc"], "n_tokens_per_step": wl["n"], "hidden": wl["H"],
+                       "expert_inter": wl["I"], "experts": wl["E"], "top_k": wl["k"],
+                       "chained_layers": wl.get("layers", 1), "parallelism": "oracle on the host cores of rank 0",
+                       "steering_F": args.steer},
             "cpu_baseline": {"value": round(rate, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "cpu_model": cpu["model"], "sample": sample},
             "e2e": {"value": round(rate, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
