@@ -11,11 +11,11 @@
 //                    also steers: y - F v (v . y)).
 //
 // k_moe_decode is persistent (one CTA per SM).  A producer warp pulls tasks
-// from an atomic queue -- gate/up tasks (shared-expert 8-row groups, then
-// (expert, 32-row block) pieces), then down tasks (shared-expert 16-row
-// groups, then (expert, 32-row block) pieces) -- and streams their weights
-// into a ring of shared-memory stages with bulk copies (cp.async.bulk +
-// mbarrier).  A down task first waits (bounded) until the gate/up tasks that
+// from atomic queues -- gate/up tasks (shared-expert 8-row groups and
+// (expert, 32-row block) pieces; for one token from two queues, their chunks
+// taken in turn), then down tasks ((expert, 32-row block) pieces, then
+// shared-expert 16-row groups) -- and streams their weights into a ring of
+// shared-memory stages with bulk copies (cp.async.bulk + mbarrier).  A down task first waits (bounded) until the gate/up tasks that
 // produce its h have published it through completion counters.  The consumer
 // warps turn the packed weights into exact small integers in registers and
 // multiply them on the tensor cores with warp-level MMAs, so that the
@@ -434,19 +434,6 @@ __device__ __forceinline__ int hrt_index(int c, int piece) {
     return ((c >> 6) * 2 + piece) * 64 + (w & ~15) + 4 * (w & 3) + ((w >> 2) & 3);
 }
 __device__ __forceinline__ int hsh_index(int c, int piece) { return ((c >> 6) * 2 + piece) * 64 + (c & 63); }
-
-// ---------------------------------------------------------------- task order
-// Queue position -> task.  The first `lead` positions are shared-expert tasks 0..lead-1 (they need no
-// routing); the remaining n_sh - lead shared tasks are spread evenly among the n_rt routed tasks
-// (numbered n_sh + i), so that each SM alternates between bandwidth-bound shared-expert stages and
-// dequantization-bound routed stages.  Positions past the end map to n_sh + n_rt (no task).
-__device__ __forceinline__ int task_at(int pos, int lead, int n_sh, int n_rt) {
-    if (pos < lead) return pos;
-    const int S = n_sh - lead, r = pos - lead;
-    if (r >= S + n_rt) return n_sh + n_rt;
-    const int a = (int)((int64_t)(r + 1) * S / (S + n_rt)), b = (int)((int64_t)r * S / (S + n_rt));
-    return a > b ? lead + b : n_sh + (r - a);
-}
 
 // ---------------------------------------------------------------- task reductions
 // The consumer warps of a projection kernel split every task's columns, so a task ends with a sum over
@@ -889,12 +876,6 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
         uint32_t it = 0;
         bool routed = false;
         int total = 0x7fffffff;
-        // task queue, two ahead (the atomic for the one after next is in flight while this task streams).
-        // One shared-expert task per CTA leads (while the router finishes); the rest interleave with
-        // routed tasks, except when x's int8 pieces replace its bf16 pieces (all shared-expert tasks come
-        // first then).
-        const int lead = !C::kSplitX ? n_sh : (n_sh < (int)gridDim.x ? n_sh : (int)gridDim.x);
-        int nxt = 0, nxt2 = 0;
         int d_total = 0;
         uint32_t dknown = 0;   // gate/up completion counters seen complete (wait_deps_warp)
         auto route = [&]() {
@@ -903,27 +884,62 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
             total = n_sh + (do_gu ? Rt.nu * rb_per_e : 0);
             d_total = dn_sh + (do_dn ? Rt.nu * drb : 0);
         };
-        if (lane == 0) {
-            nxt = (int)atomicAdd(ws.queue, 1u);
-            nxt2 = (int)atomicAdd(ws.queue, 1u);
-        }
-        for (;;) {
-            if (aborted(P) || refused) break;
-            const int pos = __shfl_sync(0xffffffffu, nxt, 0);
+        // one chunk c of gate/up task `task` (shared expert below n_sh, routed above) into the next stage
+        auto issue_gu = [&](int task, int c) -> bool {
+            const bool sh = task < n_sh;
+            const int nch = sh ? nch_sh : nch_rt;
+            const int s = it % NS;
+            const uint32_t ph = (it / NS) & 1;
+            if (!mbar_wait(&P.empty[s], ph ^ 1, ws.err)) { set_abort(P); return false; }
             if (lane == 0) {
-                nxt = nxt2;
-                nxt2 = (int)atomicAdd(ws.queue, 1u);   // in flight while this task streams
+                unsigned char* st = stages + s * kStage;
+                if (sh) {
+                    // one 8-row group of the gate and of the up matrix (core-matrix tiles), columns
+                    // c*kcs .. +kcs
+                    const int kc0 = c * kcs;
+                    const uint32_t bytes = kcs * 16;
+                    const size_t off = ((size_t)task * (H / 8) + kc0 / 8) * 64;   // elements
+                    P.info[s] = ChunkInfo{task, c, nch, kc0, kcs};
+                    mbar_arrive_expect_tx(&P.full[s], 2 * bytes);
+                    bulk_load(st, W.sh_gate + off, bytes, &P.full[s], pol);
+                    bulk_load(st + bytes, W.sh_up + off, bytes, &P.full[s], pol);
+                } else {
+                    const int tt = task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
+                    const int e = Rt.uniq[u];
+                    const int kt0 = c * ck_rt;
+                    P.info[s] = ChunkInfo{task, c, nch, kt0, ck_rt};
+                    if (Q4) {
+                        // gate codes, up codes [ck][32][32 B], their scale words [ck][32], (d, dmin)
+                        // words [ck / 4][32]
+                        const uint32_t cb = ck_rt * 1024, sb = ck_rt * 128, db = (ck_rt / 4) * 128;
+                        const size_t qoff = (size_t)e * W.q4_q_stride + ((size_t)rb * nkt + kt0) * 1024;
+                        const size_t soff = (size_t)e * W.q4_sc_stride + ((size_t)rb * nkt + kt0) * 32;
+                        const size_t doff = (size_t)e * W.q4_dd_stride + ((size_t)rb * nsb + kt0 / 4) * 32;
+                        mbar_arrive_expect_tx(&P.full[s], 2 * (cb + sb + db));
+                        bulk_load(st, W.gate_qs + qoff, cb, &P.full[s], pol);
+                        bulk_load(st + cb, W.up_qs + qoff, cb, &P.full[s], pol);
+                        bulk_load(st + 2 * cb, W.gate_sc4 + soff, sb, &P.full[s], pol);
+                        bulk_load(st + 2 * cb + sb, W.up_sc4 + soff, sb, &P.full[s], pol);
+                        bulk_load(st + 2 * (cb + sb), W.gate_dd4 + doff, db, &P.full[s], pol);
+                        bulk_load(st + 2 * (cb + sb) + db, W.up_dd4 + doff, db, &P.full[s], pol);
+                    } else {
+                        const uint32_t pb = ck_rt * 512, db = ck_rt * 16;
+                        const size_t qoff = (size_t)e * W.iq2_qs_stride + ((size_t)rb * nkt + kt0) * 512;
+                        const size_t doff = (size_t)e * W.iq2_d_stride + ((size_t)rb * nsb + kt0 / 4) * 32;
+                        mbar_arrive_expect_tx(&P.full[s], 2 * pb + 2 * db);
+                        bulk_load(st, W.gate_qs + qoff, pb, &P.full[s], pol);
+                        bulk_load(st + pb, W.up_qs + qoff, pb, &P.full[s], pol);
+                        bulk_load(st + 2 * pb, W.gate_d + doff, db, &P.full[s], pol);
+                        bulk_load(st + 2 * pb + db, W.up_d + doff, db, &P.full[s], pol);
+                    }
+                }
             }
-            if (pos >= lead && !routed) {
-                // the router's ids and weights: published by its last CTA through the ready flag (probe
-                // calls route by themselves)
-                if (!ws.probe && !wait_flag(ws.route_ready, ws.err)) { set_abort(P); break; }
-                route();
-            }
-            if (pos >= total) {
-                // down-projection task pos - total
-                const int dt = pos - total;
-                if (dt >= d_total) break;
+            __syncwarp();
+            ++it;
+            return true;
+        };
+        // down task dt: waits (bounded) for the gate/up tasks that produce its h, then streams its chunks
+        auto run_down = [&](int dt) -> bool {
             const int nd_rt = do_dn ? Rt.nu * drb : 0;
             const bool dsh = dt >= nd_rt;
             const int dts = dt - nd_rt;   // shared-expert down task
@@ -939,7 +955,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                 !wait_deps_warp(ws.gu_done, dsh ? 0 : 1 + u, 1 + Rt.nu, (uint32_t)(I / 8), (uint32_t)(I / 32), dknown,
                                 ws.err)) {
                 set_abort(P);
-                break;
+                return false;
             }
             for (int c = 0; c < nch; ++c) {
                 const int s = it % NS;
@@ -990,61 +1006,112 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
                 __syncwarp();
                 ++it;
             }
-                continue;
-            }
-            const int task = pos < lead ? pos : task_at(pos, lead, n_sh, total - n_sh);
-            const bool sh = task < n_sh;
-            const int nch = sh ? nch_sh : nch_rt;
-            for (int c = 0; c < nch; ++c) {
-                const int s = it % NS;
-                const uint32_t ph = (it / NS) & 1;
-                if (!mbar_wait(&P.empty[s], ph ^ 1, ws.err)) { set_abort(P); break; }
-                if (lane == 0) {
-                    unsigned char* st = stages + s * kStage;
-                    if (sh) {
-                        // one 8-row group of the gate and of the up matrix (core-matrix tiles), columns
-                        // c*kcs .. +kcs
-                        const int kc0 = c * kcs;
-                        const uint32_t bytes = kcs * 16;
-                        const size_t off = ((size_t)task * (H / 8) + kc0 / 8) * 64;   // elements
-                        P.info[s] = ChunkInfo{task, c, nch, kc0, kcs};
-                        mbar_arrive_expect_tx(&P.full[s], 2 * bytes);
-                        bulk_load(st, W.sh_gate + off, bytes, &P.full[s], pol);
-                        bulk_load(st + bytes, W.sh_up + off, bytes, &P.full[s], pol);
+            return !aborted(P);
+        };
+        if constexpr (C::kSplitX) {
+            // One token: two streams of gate/up tasks, shared-expert tasks (queue: their numbers, then the
+            // down tasks) and routed tasks (queue_rt), taken chunk by chunk in turn, so that a
+            // dequantization-bound routed stage and a bandwidth-bound shared-expert stage alternate and every
+            // stage's copy is issued two stages ahead of its use.  One shared-expert task leads while the
+            // router finishes.  The down tasks follow once both streams are exhausted and this producer's
+            // gate/up chunks are all issued (a down task waits only for gate/up tasks that other producers
+            // have issued in full or will issue without waiting).  Each queue's next position is in flight
+            // while the current task streams.
+            int qs = 0, qr = 0;
+            int sh_task = -1, sh_c = 0, sh_taken = 0, rt_task = -1, rt_c = 0, dn_pos = 0;
+            bool sh_out = false, rt_out = false, pref_rt = false;
+            if (lane == 0) qs = (int)atomicAdd(ws.queue, 1u);
+            for (;;) {
+                if (aborted(P) || refused) break;
+                if (!routed && sh_task < 0 && (sh_taken > 0 || sh_out)) {
+                    // the router's ids and weights: published by its last CTA through the ready flag (probe
+                    // calls route by themselves)
+                    if (!ws.probe && !wait_flag(ws.route_ready, ws.err)) { set_abort(P); break; }
+                    route();
+                    if (lane == 0) qr = (int)atomicAdd(ws.queue_rt, 1u);
+                }
+                if (sh_task < 0 && !sh_out) {
+                    const int q = __shfl_sync(0xffffffffu, qs, 0);
+                    if (q < n_sh) {
+                        sh_task = q;
+                        sh_c = 0;
+                        ++sh_taken;
+                        if (lane == 0) qs = (int)atomicAdd(ws.queue, 1u);
                     } else {
-                        const int tt = task - n_sh, u = tt / rb_per_e, rb = tt % rb_per_e;
-                        const int e = Rt.uniq[u];
-                        const int kt0 = c * ck_rt;
-                        P.info[s] = ChunkInfo{task, c, nch, kt0, ck_rt};
-                        if (Q4) {
-                            // gate codes, up codes [ck][32][32 B], their scale words [ck][32], (d, dmin)
-                            // words [ck / 4][32]
-                            const uint32_t cb = ck_rt * 1024, sb = ck_rt * 128, db = (ck_rt / 4) * 128;
-                            const size_t qoff = (size_t)e * W.q4_q_stride + ((size_t)rb * nkt + kt0) * 1024;
-                            const size_t soff = (size_t)e * W.q4_sc_stride + ((size_t)rb * nkt + kt0) * 32;
-                            const size_t doff = (size_t)e * W.q4_dd_stride + ((size_t)rb * nsb + kt0 / 4) * 32;
-                            mbar_arrive_expect_tx(&P.full[s], 2 * (cb + sb + db));
-                            bulk_load(st, W.gate_qs + qoff, cb, &P.full[s], pol);
-                            bulk_load(st + cb, W.up_qs + qoff, cb, &P.full[s], pol);
-                            bulk_load(st + 2 * cb, W.gate_sc4 + soff, sb, &P.full[s], pol);
-                            bulk_load(st + 2 * cb + sb, W.up_sc4 + soff, sb, &P.full[s], pol);
-                            bulk_load(st + 2 * (cb + sb), W.gate_dd4 + doff, db, &P.full[s], pol);
-                            bulk_load(st + 2 * (cb + sb) + db, W.up_dd4 + doff, db, &P.full[s], pol);
-                        } else {
-                            const uint32_t pb = ck_rt * 512, db = ck_rt * 16;
-                            const size_t qoff = (size_t)e * W.iq2_qs_stride + ((size_t)rb * nkt + kt0) * 512;
-                            const size_t doff = (size_t)e * W.iq2_d_stride + ((size_t)rb * nsb + kt0 / 4) * 32;
-                            mbar_arrive_expect_tx(&P.full[s], 2 * pb + 2 * db);
-                            bulk_load(st, W.gate_qs + qoff, pb, &P.full[s], pol);
-                            bulk_load(st + pb, W.up_qs + qoff, pb, &P.full[s], pol);
-                            bulk_load(st + 2 * pb, W.gate_d + doff, db, &P.full[s], pol);
-                            bulk_load(st + 2 * pb + db, W.up_d + doff, db, &P.full[s], pol);
-                        }
+                        sh_out = true;
+                        dn_pos = q;
                     }
                 }
-                __syncwarp();
-                ++it;
+                if (routed && rt_task < 0 && !rt_out) {
+                    const int q = __shfl_sync(0xffffffffu, qr, 0);
+                    if (q < total - n_sh) {
+                        rt_task = n_sh + q;
+                        rt_c = 0;
+                        if (lane == 0) qr = (int)atomicAdd(ws.queue_rt, 1u);
+                    } else {
+                        rt_out = true;
+                    }
+                }
+                if (sh_task < 0 && rt_task < 0) {
+                    if (routed) break;   // both streams exhausted
+                    continue;            // the shared stream ran out first: route, then take routed tasks
+                }
+                const bool use_rt = rt_task >= 0 && (pref_rt || sh_task < 0);
+                if (use_rt) {
+                    if (!issue_gu(rt_task, rt_c)) break;
+                    if (++rt_c == nch_rt) rt_task = -1;
+                } else {
+                    if (!issue_gu(sh_task, sh_c)) break;
+                    if (++sh_c == nch_sh) sh_task = -1;
+                }
+                pref_rt = !use_rt;
             }
+            if (!aborted(P) && !refused && routed) {
+                int pos = dn_pos, nxt = 0;
+                if (lane == 0) nxt = (int)atomicAdd(ws.queue, 1u);
+                for (;;) {
+                    const int dt = pos - n_sh;
+                    if (dt >= d_total || aborted(P)) break;
+                    if (!run_down(dt)) break;
+                    pos = __shfl_sync(0xffffffffu, nxt, 0);
+                    if (lane == 0) nxt = (int)atomicAdd(ws.queue, 1u);
+                }
+                asm volatile("" ::"r"(nxt));
+            }
+            // the prefetched positions are read, so every queue atomic of this CTA has completed before the
+            // last CTA resets the queues
+            asm volatile("" ::"r"(qs), "r"(qr));
+        } else {
+            // Two or more tokens: one queue, two ahead (the atomic for the one after next is in flight while
+            // this task streams): every shared-expert task (x's int8 pieces replace its bf16 pieces once
+            // they are done), then the routed gate/up tasks, then the down tasks.
+            int nxt = 0, nxt2 = 0;
+            if (lane == 0) {
+                nxt = (int)atomicAdd(ws.queue, 1u);
+                nxt2 = (int)atomicAdd(ws.queue, 1u);
+            }
+            for (;;) {
+                if (aborted(P) || refused) break;
+                const int pos = __shfl_sync(0xffffffffu, nxt, 0);
+                if (lane == 0) {
+                    nxt = nxt2;
+                    nxt2 = (int)atomicAdd(ws.queue, 1u);   // in flight while this task streams
+                }
+                if (pos >= n_sh && !routed) {
+                    if (!ws.probe && !wait_flag(ws.route_ready, ws.err)) { set_abort(P); break; }
+                    route();
+                }
+                if (pos >= total) {
+                    const int dt = pos - total;
+                    if (dt >= d_total || !run_down(dt)) break;
+                    continue;
+                }
+                const int nch = pos < n_sh ? nch_sh : nch_rt;
+                bool ok = true;
+                for (int c = 0; c < nch && ok; ++c) ok = issue_gu(pos, c);
+                if (!ok) break;
+            }
+            asm volatile("" ::"r"(nxt), "r"(nxt2));
         }
         producer_finish(P, it, NS, ws.err);
     } else if (warp < CW && !refused) {
@@ -1577,6 +1644,7 @@ __global__ void __launch_bounds__(GateUpCfg<NT>::kThreads, 1)
         s_last = atomicAdd(ws.done, 1u) == gridDim.x - 1;
         if (s_last) {
             *ws.queue = 0;
+            *ws.queue_rt = 0;
             *ws.done = 0;
             *ws.route_ready = 0;
         }

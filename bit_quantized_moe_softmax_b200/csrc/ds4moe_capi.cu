@@ -244,6 +244,7 @@ struct ds4moe {
         w.err = hdr + 0;
         w.ticket = hdr + 1;
         w.queue = hdr + 2;
+        w.queue_rt = hdr + 3;
         w.done = hdr + 4;
         w.grid_refused = hdr + 6;
         w.route_ready = hdr + 7;
@@ -925,6 +926,7 @@ ds4moe_status ds4moe_route_noalloc(ds4moe_t* h, const void* d_x, int32_t n, int3
     ws.err = hdr + 0;
     ws.ticket = hdr + 1;
     ws.queue = hdr + 2;
+    ws.queue_rt = hdr + 3;
     ws.logits = base + kNoAllocHeader;
     ws.ids = d_ids;
     ws.wts = d_w;

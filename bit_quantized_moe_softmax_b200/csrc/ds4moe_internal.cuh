@@ -125,7 +125,8 @@ struct Dims {
 struct DecodeWs {
     uint32_t* err;          // device error word
     uint32_t* ticket;       // router last-CTA ticket
-    uint32_t* queue;        // projection task counter
+    uint32_t* queue;        // projection task counter (one token: shared-expert gate/up tasks, then down tasks)
+    uint32_t* queue_rt;     // one token: the routed gate/up task counter
     uint32_t* done;         // projection CTAs finished (the last one resets the counters)
     uint32_t* grid_refused; // this call's projection grid refused the grid (too many or too large magnitudes): 1, else 0
     uint32_t* route_ready;  // set by the router once ids / weights are written; reset by the projection grid
