@@ -133,8 +133,11 @@ def test_forward_tiny_matches_oracle(orc, n):
     assert rel_err(out, ref) < TOL
 
 
+# n = 1 takes the one-token producer (shared-expert and routed gate/up tasks from two queues, in turn),
+# n = 3 the single-queue one
+@pytest.mark.parametrize("n", [1, 3])
 @pytest.mark.parametrize("variant", ["bias", "no_shared", "one_expert", "k_equals_E", "bf16_act", "unit_logits"])
-def test_forward_tiny_variants(orc, variant):
+def test_forward_tiny_variants(orc, variant, n):
     kw = dict(bias=variant == "bias", shared=variant != "no_shared")
     if variant == "one_expert":
         kw.update(E=1, k=1)
@@ -145,7 +148,6 @@ def test_forward_tiny_variants(orc, variant):
     L = _tiny(orc, **kw)
     act = m.DS4MOE_ACT_BF16 if variant == "bf16_act" else m.DS4MOE_ACT_F32
     lay = _layer_on_gpu(L, act=act)
-    n = 3
     x = synth.tokens(n, 256, seed=21, dtype=torch.bfloat16 if act else torch.float32)
     out = lay.forward(x.cuda()).cpu().numpy()
     ref, _, _ = orc.moe_forward(oracle_layer(L), x.float().numpy())
